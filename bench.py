@@ -1,0 +1,477 @@
+"""Benchmark of the quantized KV-cache hot path: one step = append one new bf16
+K/V token per sequence (quantize, residual window, flush when a key group
+fills) + decode attention for every sequence over the packed paged cache.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 3] [--impl kvq|reference]
+
+Prints ONE JSON line (rank 0).  `value` is decode-attention KV GB/s: the
+algorithmic bytes of the decode call (codes, scales, zero-points, BF16 window
+rows, q, out, block-table entries) over its device time, summed over ranks and
+divided by the max over ranks.  Inputs live in HBM before the timed region; L2
+is flushed (256 MB write, untimed) before every timed step.  `e2e` is the same
+metric through the C ABI with host buffers: pinned H2D of the step's new K/V
+and q and D2H of the attention output inside the timed region.  With N > 1 every
+rank runs its own replica (sequences shard across GPUs; no collective is on the
+data path; the only collectives are the barrier and the max-over-ranks timing).
+`--impl reference` times the CPU oracle (test infrastructure) on a bounded
+sample of the same workload.
+"""
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from quantized_kv_cache_14_b200.workloads import Draws, workload  # noqa: E402
+
+D = 128
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes
+# ---------------------------------------------------------------------------
+
+def decode_bytes(w, lengths):
+    """Bytes a decode call must move: codes + scales (+ zero-points) of the
+    quantized tokens, BF16 rows of the residual window, q, out and one
+    block-table entry per page read."""
+    f = w.fmt
+    es = 4 if f.scale_fp32 else 2
+    meta = es * (1 + f.asym)
+    per_tok_q = w.h_kv * (2 * D * f.bits // 8 + D * meta // f.g_k + D * meta // f.g_v)
+    per_tok_r = w.h_kv * 2 * D * 2
+    total = 0
+    for L in lengths:
+        Lq = (L // f.residual) * f.residual if f.residual else L
+        total += Lq * per_tok_q + (L - Lq) * per_tok_r + ((Lq + f.page - 1) // f.page) * 4
+    total += len(lengths) * w.h_q * D * (2 + 4)
+    return total
+
+
+def append_bytes(w, lengths_before, n_new_per_seq=1):
+    """Bytes an append of one token per sequence must move: the new bf16 K/V
+    rows read, residual slots written, and for every key group that fills, its
+    residual rows re-read plus the codes and scales written."""
+    f = w.fmt
+    es = 4 if f.scale_fp32 else 2
+    meta = es * (1 + f.asym)
+    row = w.h_kv * D * 2
+    total = 0
+    for L in lengths_before:
+        total += 2 * row                                # new K and V rows read
+        if f.residual == 0:
+            total += w.h_kv * (2 * D * f.bits // 8 + D * meta // f.g_k + D * meta // f.g_v)
+        elif (L + 1) % f.residual == 0:
+            R = f.residual
+            total += 2 * row * (R - 1)                  # window rows re-read
+            total += R * w.h_kv * (2 * D * f.bits // 8 + D * meta // f.g_v) + w.h_kv * D * meta
+        else:
+            total += 2 * row                            # written to the window
+    return total
+
+
+def pool_blocks(lengths, growth, page):
+    return int(sum((L + growth + page - 1) // page for L in lengths)) + 64
+
+
+# ---------------------------------------------------------------------------
+# environment: ranks, clocks, peaks
+# ---------------------------------------------------------------------------
+
+def dist_setup(n_gpus):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws == 1:
+        return 0, 1, None
+    import datetime
+    import torch
+    import torch.distributed as dist
+    backend = os.environ.get("KVQ_BENCH_BACKEND", "nccl" if torch.cuda.is_available() else "gloo")
+    rank = int(os.environ["RANK"])
+    if backend == "nccl":
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", rank)))
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, ws, dist
+
+
+def barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
+def max_over_ranks(dist, values):
+    """Elementwise max of a list of floats over ranks."""
+    if dist is None:
+        return list(values)
+    import torch
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor(values, dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.cpu().tolist()
+
+
+def sum_over_ranks(dist, values):
+    if dist is None:
+        return list(values)
+    import torch
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor(values, dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return t.cpu().tolist()
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons while timing."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index, enabled=True, period_ms=50):
+        self.proc = None
+        self.device_index = device_index
+        if not enabled:
+            return
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={device_index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", f"-lms={period_ms}"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(smax)),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for f in ("kvq_decode.cu", "kvq_device.cuh", "kvq_internal.h"):
+        with open(os.path.join(ROOT, "quantized_kv_cache_14_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(workload_name):
+    """Per-launch DRAM bytes of the attention kernel from the committed ncu
+    summary, if it was taken from the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    if rec.get("kernel_source_sha") != kernel_source_sha():
+        return None
+    return rec.get("traffic_bytes_per_launch", {}).get(workload_name)
+
+
+# ---------------------------------------------------------------------------
+# the CUDA arm
+# ---------------------------------------------------------------------------
+
+def run_gpu(args, rank, ws, dist):
+    import torch
+    from quantized_kv_cache_14_b200 import kvq
+
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", rank)) if ws > 1 else 0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = workload(args.workload)
+    w.seed = w.seed + 1000 * rank        # each replica draws its own inputs
+    total_steps = args.warmup + args.steps
+    dr = Draws(w, steps=2 * total_steps)
+    f = w.fmt
+    nb = pool_blocks(dr.lengths, 2 * total_steps + 2, f.page)
+    mbps = max((L + 2 * total_steps + 2) // f.page + 2 for L in dr.lengths)
+    cache = kvq.KVCache(kvq.Format(f.bits, f.asym, f.k_axis, f.g_k, f.g_v, f.scale_fp32,
+                                   f.residual, f.page), w.h_q, w.h_kv, max_seqs=w.batch,
+                        num_blocks=nb, max_blocks_per_seq=mbps, seed=w.seed,
+                        device=torch.cuda.current_device())
+
+    def bf16_dev(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    # prefill (bulk append), untimed
+    cache.append(bf16_dev(dr.k), bf16_dev(dr.v), dr.seq_ids)
+    lens = list(dr.lengths)
+    B = w.batch
+    ids = np.arange(B, dtype=np.int32)
+    steps_in = [dr.step() for _ in range(2 * total_steps)]
+    dev_in = [(bf16_dev(k), bf16_dev(v), bf16_dev(q)) for k, v, q in steps_in]
+    host_in = [tuple(torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
+                     for a in s) for s in steps_in]
+    del dr
+    seq_lens = torch.tensor(lens, dtype=torch.int32, device=dev)
+    out = torch.empty((B, w.h_q, D), dtype=torch.float32, device=dev)
+    out_host = torch.empty_like(out, device="cpu").pin_memory()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    ev_mid = torch.cuda.Event(enable_timing=True)
+    cache.set_decode_event(ev_mid)
+    torch.cuda.synchronize()
+    assert cache.sync_status() == 0
+
+    def one_step(s, e2e, evs):
+        nonlocal lens
+        ev0, ev1, ev2 = evs
+        flush.zero_()                                   # untimed: evicts L2
+        ev0.record()
+        if e2e:
+            kh, vh, qh = host_in[s]
+            k = kh.to(dev, non_blocking=True)
+            v = vh.to(dev, non_blocking=True)
+            q = qh.to(dev, non_blocking=True)
+        else:
+            k, v, q = dev_in[s]
+        cache.append(k, v, ids)
+        lens = [L + 1 for L in lens]
+        seq_lens.add_(1)
+        ev1.record()
+        cache.decode(q, seq_lens, out)
+        if e2e:
+            out_host.copy_(out, non_blocking=True)
+        ev2.record()
+
+    # warm-up
+    for s in range(args.warmup):
+        one_step(s, False, [torch.cuda.Event(enable_timing=True) for _ in range(3)])
+    torch.cuda.synchronize()
+    assert cache.sync_status() == 0
+
+    # timed: device-resident inputs
+    st0 = cache.stats()["kernel_launches"]
+    sampler = ClockSampler(torch.cuda.current_device(), enabled=not args.no_clocks)
+    time.sleep(0.15 if sampler.proc else 0)
+    barrier(dist)
+    torch.cuda.synchronize()
+    recs = []
+    kv_bytes, app_bytes, seq_tokens = 0, 0, 0
+    for s in range(args.warmup, total_steps):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        before = list(lens)
+        one_step(s, False, evs)
+        evs[2].synchronize()
+        # ev_mid was recorded by the library between the attention kernel and the merge
+        recs.append((evs[0].elapsed_time(evs[1]), evs[1].elapsed_time(ev_mid),
+                     evs[1].elapsed_time(evs[2])))
+        kv_bytes += decode_bytes(w, lens)
+        app_bytes += append_bytes(w, before)
+        seq_tokens += sum(lens)
+    torch.cuda.synchronize()
+    barrier(dist)
+    launches = cache.stats()["kernel_launches"] - st0
+    clocks = sampler.stop()
+    assert cache.sync_status() == 0
+
+    # timed: end to end through the C ABI with host buffers
+    barrier(dist)
+    torch.cuda.synchronize()
+    e2e_ms, e2e_bytes = 0.0, 0
+    for s in range(total_steps, total_steps + args.steps):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        one_step(s, True, evs)
+        evs[2].synchronize()
+        e2e_ms += evs[0].elapsed_time(evs[2])
+        e2e_bytes += decode_bytes(w, lens)
+    torch.cuda.synchronize()
+    barrier(dist)
+    assert cache.sync_status() == 0
+    cache.close()
+
+    t_app = sum(r[0] for r in recs)
+    t_attn = sum(r[1] for r in recs)
+    t_dec = sum(r[2] for r in recs)
+    step_ms = t_app + t_dec
+    mx = max_over_ranks(dist, [t_app, t_attn, t_dec, step_ms, e2e_ms])
+    tot = sum_over_ranks(dist, [kv_bytes, app_bytes, seq_tokens, e2e_bytes])
+    K = args.steps
+    res = {
+        "w": w, "K": K, "ws": ws, "launches": launches, "clocks": clocks,
+        "kv_gbs": tot[0] / (mx[2] * 1e-3) / 1e9,
+        "attn_gbs": (kv_bytes / K) / (t_attn / K * 1e-3) / 1e9,
+        "attn_us": t_attn / K * 1e3,
+        "decode_us": t_dec / K * 1e3,
+        "append_us": t_app / K * 1e3,
+        "append_gbs": tot[1] / (mx[0] * 1e-3) / 1e9,
+        "seq_tok_s": tot[2] / (mx[3] * 1e-3),
+        "ms_per_step": mx[3] / K,
+        "e2e_gbs": tot[3] / (mx[4] * 1e-3) / 1e9,
+        "kv_bytes_per_step": kv_bytes / K,
+        "lens_final": lens,
+        "h2d": B * w.h_kv * D * 2 * 2 + B * w.h_q * D * 2,
+        "d2h": B * w.h_q * D * 4,
+    }
+    return res
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle (baseline / reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_cache_for(w, dr, growth):
+    from oracle import oracle as O
+    f = w.fmt
+    nb = pool_blocks(dr.lengths, growth, f.page)
+    mbps = max((L + growth) // f.page + 2 for L in dr.lengths)
+    oc = O.OracleCache(bits=f.bits, asym=f.asym, k_axis=f.k_axis, g_k=f.g_k, g_v=f.g_v,
+                       scale_fp32=f.scale_fp32, residual=f.residual, page=f.page, h_q=w.h_q,
+                       h_kv=w.h_kv, d_h=D, max_seqs=w.batch, num_blocks=nb,
+                       max_blocks_per_seq=mbps, seed=w.seed, fail_alloc_after=-1)
+    assert oc.append(dr.k, dr.v, dr.seq_ids) == 0
+    return oc
+
+
+def run_oracle_sample(w, steps, warmup, rows, threads):
+    """Oracle steps (append one token per sequence + decode of `rows`
+    sequences); returns (decode GB/s, seconds timed, bytes)."""
+    dr = Draws(w, steps=steps + warmup)
+    oc = oracle_cache_for(w, dr, steps + warmup + 2)
+    lens = list(dr.lengths)
+    ids = np.arange(w.batch, dtype=np.int32)
+    t_dec, nbytes = 0.0, 0
+    for s in range(warmup + steps):
+        k, v, q = dr.step()
+        assert oc.append(k, v, ids) == 0
+        lens = [L + 1 for L in lens]
+        sub = np.arange(rows, dtype=np.int32)
+        t0 = time.perf_counter()
+        oc.decode(q[:rows], [lens[i] for i in sub], seq_ids=sub, nthreads=threads)
+        dt = time.perf_counter() - t0
+        if s >= warmup:
+            t_dec += dt
+            nbytes += decode_bytes(w, [lens[i] for i in sub])
+    oc.close()
+    return nbytes / t_dec / 1e9, t_dec, nbytes, lens
+
+
+def workload_config(w, lens):
+    f = w.fmt
+    kind = {(8, 0): "INT8 sym", (4, 0): "INT4 sym", (2, 1): "INT2 asym", (2, 0): "INT2 sym",
+            (4, 1): "INT4 asym", (8, 1): "INT8 asym"}[(f.bits, f.asym)]
+    axis = "per-channel" if f.k_axis else "per-token"
+    return {
+        "workload": f"{w.name}: {w.note}",
+        "format": f"{kind}, keys {axis} G={f.g_k}, values per-token G={f.g_v}, "
+                  f"{'fp32' if f.scale_fp32 else 'fp16'} scales, page {f.page}, BF16 window {f.residual}",
+        "batch": w.batch, "h_q": w.h_q, "h_kv": w.h_kv, "d_h": D,
+        "seq_len_start": int(min(lens)), "seq_len_max": int(max(lens)),
+        "l2": "flushed before every timed step (256 MB write, untimed)",
+        "step": "append 1 token per sequence (quantize/window/flush) + decode attention",
+        "parallelism": "replicas",
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", type=int, default=3, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=0, help="rows of the CPU oracle sample")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank, ws, dist = dist_setup(args.gpus)
+    w = workload(args.workload)
+    threads = os.cpu_count() or 1
+    rows = args.cpu_rows or min(w.batch, 16)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        steps = min(args.steps, 5)
+        gbs, secs, nbytes, lens = run_oracle_sample(w, steps, min(args.warmup, 1), rows, threads)
+        line = {
+            "metric": "decode-attn KV GB/s", "value": gbs, "unit": "GB/s", "impl": "reference",
+            "n_gpus": 0, "steps": steps, "warmup": min(args.warmup, 1),
+            "ms_per_step": secs / steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w, lens),
+            "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                             "sample": f"{steps} steps: append 1 token to each of {w.batch} sequences, "
+                                       f"decode {rows} of them, fp64 C++ oracle"},
+            "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line))
+        return
+
+    res = run_gpu(args, rank, ws, dist)
+    if rank != 0:
+        return
+    peak, peak_kind = measured_peak()
+    cpu = None
+    if ws == 1 and not args.no_cpu_baseline:
+        gbs, secs, _, _ = run_oracle_sample(w, 2, 0, rows, threads)
+        cpu = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": f"2 steps of {rows}/{w.batch} sequences (append + fp64 decode), "
+                         f"{secs:.1f} s timed"}
+    traffic = committed_traffic(w.name)
+    line = {
+        "metric": "decode-attn KV GB/s", "value": res["kv_gbs"], "unit": "GB/s",
+        "n_gpus": ws, "steps": res["K"], "warmup": args.warmup,
+        "ms_per_step": res["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(w, res["lens_final"]),
+        "roofline": {"bound": "hbm", "achieved": res["attn_gbs"], "peak": peak, "unit": "GB/s",
+                     "frac": res["attn_gbs"] / peak, "traffic": traffic,
+                     "peak_kind": peak_kind, "kernel": "decode_kernel (attention, without the merge)"},
+        "cpu_baseline": cpu,
+        "e2e": {"value": res["e2e_gbs"], "unit": "GB/s", "h2d_bytes_per_step": res["h2d"],
+                "d2h_bytes_per_step": res["d2h"]},
+        "gpu_launches": res["launches"],
+        "clocks": res["clocks"],
+        "seq_tokens_per_s": res["seq_tok_s"],
+        "append_gbs": res["append_gbs"],
+        "attn_us": res["attn_us"], "decode_us": res["decode_us"], "append_us": res["append_us"],
+        "kv_bytes_per_step": res["kv_bytes_per_step"],
+        "frac_of_8TBps": res["kv_gbs"] / 8000.0,
+        "frac_of_peak": res["kv_gbs"] / peak,
+    }
+    print(json.dumps(line))
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,258 @@
+/*
+ * kvq.h -- C ABI of libkvq.so: a quantized, paged KV cache with decode
+ * attention over the packed low-bit cache, for NVIDIA B200 (sm_100a).
+ *
+ * The method follows the pages on KV-cache quantization:
+ *  - llmdaily.org "KV-cache quantization -- making long-context inference fit
+ *    in memory" (day 65): the attention equation and the memory formula
+ *    (section "Why the KV cache grows so quickly"), the symmetric quantizer
+ *    s = max|x| / (2^(b-1) - 1), q = clip(round(x/s), -Q, Q), x_hat = s q and
+ *    the asymmetric zero-point variant (section "From BF16 to INT8, INT4, or
+ *    even fewer bits"), one scale per group and different grouping directions
+ *    for keys and values (section "Why scales and groups matter"), the BF16
+ *    residual window (section "Why some systems keep a full-precision
+ *    window"), blocks addressed through block tables (section "How this
+ *    connects to paging and prefix caching"), and fused dequantization
+ *    (section "Why compression may also improve speed");
+ *  - oh-bug.com "KV Cache Quantization in Practice": keys per channel, values
+ *    per token (the KIVI paragraph), asymmetric 2-bit (the list under
+ *    "4-bit / 3-bit / 2-bit").
+ *
+ * Conventions for every call:
+ *  - Plain pointers and sizes only.  "device" pointers are CUDA global memory
+ *    of the handle's device; "host" pointers are ordinary CPU memory.
+ *    `stream` is a cudaStream_t passed as void* (NULL = legacy default).
+ *  - Status codes are returned; nothing is thrown and nothing aborts.  The
+ *    text of the last failure on the calling thread is kvq_last_error().
+ *  - Work is enqueued asynchronously on `stream`; host-side bookkeeping
+ *    (lengths, block tables, free list) is updated before the call returns.
+ *    A failing kvq_append leaves all state unchanged.
+ *  - Device pointers passed in must be 16-byte aligned (KVQ_ERR_INVALID_ARG).
+ *  - Kernels check block ids, lengths and grid coverage themselves and record
+ *    failures in a device error word instead of faulting; kvq_sync_status()
+ *    reports and clears it.
+ *  - A handle may be used from one host thread at a time.
+ */
+#ifndef KVQ_H_
+#define KVQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct kvq_handle_s* kvq_handle;
+
+typedef enum kvq_status {
+  KVQ_OK = 0,
+  KVQ_ERR_INVALID_ARG = 1,   /* bad pointer, size, alignment or config field   */
+  KVQ_ERR_OOM = 2,           /* no free block, block-table row full, or the
+                                fail_alloc_after test hook fired               */
+  KVQ_ERR_BAD_SEQ = 3,       /* sequence id outside [0, max_seqs)              */
+  KVQ_ERR_CUDA = 4,          /* a CUDA runtime call failed                     */
+  KVQ_ERR_DEVICE_CHECK = 5,  /* a kernel's own check fired (see kvq_sync_status)*/
+  KVQ_ERR_UNSUPPORTED = 6    /* valid but unsupported combination             */
+} kvq_status;
+
+/* Bits of the device error word (kvq_sync_status). */
+#define KVQ_DEVERR_BLOCK_ID 0x1u   /* block-table entry outside [0, num_blocks)  */
+#define KVQ_DEVERR_SEQ_LEN  0x2u   /* seq_lens[i] < 0 or > the stored length      */
+#define KVQ_DEVERR_TIMEOUT  0x4u   /* a bounded wait on a copy gave up            */
+#define KVQ_DEVERR_SEQ_ID   0x8u   /* decode row names an invalid sequence        */
+
+enum { KVQ_AXIS_TOKEN = 0, KVQ_AXIS_CHANNEL = 1 };
+
+/* Storage format and capacity of one layer's cache.
+ *   bits        8, 4 or 2 bits per stored element.
+ *   asym        0: symmetric codes in [-Q, Q], Q = 2^(bits-1) - 1;
+ *               1: unsigned codes in [0, 2^bits - 1] with a zero-point.
+ *   k_axis      KVQ_AXIS_TOKEN: key groups are g_k consecutive channels of
+ *               one token (residual must be 0);
+ *               KVQ_AXIS_CHANNEL: key groups are g_k consecutive tokens of one
+ *               channel (residual must equal g_k; page divides g_k).
+ *   g_k, g_v    group sizes: 16, 32, 64 or 128 (g_k is tokens on the channel
+ *               axis).  Values are always grouped per token over g_v channels.
+ *   scale_fp32  0: scales and zero-points stored as fp16 (round to nearest
+ *               even, saturating at 65504); 1: stored as fp32.
+ *   residual    R, the BF16 window length (0 or g_k).
+ *   page        P tokens per block: a multiple of 16.
+ *   h_q, h_kv   query and key/value heads; h_q / h_kv must be 1, 2 or 4.
+ *   d_h         head dimension: 128.
+ *   max_seqs, num_blocks, max_blocks_per_seq   capacity.
+ *   seed        seeds the free list: a Fisher-Yates shuffle of
+ *               [0, num_blocks) driven by splitmix64(seed); blocks are taken
+ *               from its front and freed blocks return to its back.
+ *   fail_alloc_after  test hook: allocation number k (0-based, cumulative)
+ *               fails when k >= fail_alloc_after; -1 disables it.
+ *   host_only   1: no device memory and no kernels (host bookkeeping only;
+ *               for tests on machines without a GPU).
+ *   device      CUDA device ordinal (ignored when host_only). */
+typedef struct kvq_config {
+  int32_t bits;
+  int32_t asym;
+  int32_t k_axis;
+  int32_t g_k;
+  int32_t g_v;
+  int32_t scale_fp32;
+  int32_t residual;
+  int32_t page;
+  int32_t h_q;
+  int32_t h_kv;
+  int32_t d_h;
+  int32_t max_seqs;
+  int32_t num_blocks;
+  int32_t max_blocks_per_seq;
+  uint64_t seed;
+  int32_t fail_alloc_after;
+  int32_t host_only;
+  int32_t device;
+} kvq_config;
+
+/* Byte geometry of the paged format.  A block holds `page` token slots of all
+ * h_kv heads; block b, head h starts at b * block_bytes + h * chunk_bytes.  A
+ * chunk holds, in order: key codes (page/16 sub-tiles of 16 tokens), value
+ * codes (same), value scales [page][d_h/g_v] then zero-points, key metadata
+ * (token axis: [page][d_h/g_k] scales then zero-points; channel axis: a slice
+ * of kslice entries of the group's scales, then zero-points).  The bit-level
+ * placement of codes is given in the project's format notes; the CUDA kernels
+ * and the CPU oracle implement it independently. */
+typedef struct kvq_layout_info {
+  uint64_t row_bytes;    /* key row: d_h * bits / 8                         */
+  uint64_t sub_bytes;    /* one 16-token sub-tile of codes                  */
+  uint64_t off_v;        /* value codes, from the chunk start               */
+  uint64_t off_vmeta;    /* value scales (+ zero-points)                    */
+  uint64_t off_kmeta;    /* key scales (+ zero-points)                      */
+  uint64_t chunk_bytes;  /* one (block, head): 32-byte multiple             */
+  uint64_t block_bytes;  /* h_kv * chunk_bytes                              */
+  uint64_t kslice;       /* channel axis: key-scale entries per block       */
+} kvq_layout_info;
+
+typedef struct kvq_stats_t {
+  uint64_t blocks_used;
+  uint64_t blocks_free;
+  uint64_t tokens_stored;     /* sum of stored lengths                      */
+  uint64_t bytes_pool;        /* device bytes of the block pool             */
+  uint64_t bytes_residual;    /* device bytes of the BF16 windows (K + V)   */
+  uint64_t bytes_workspace;   /* plans, split partials, prefix, error word  */
+  uint64_t bytes_formula;     /* tokens_stored by the memory formula (one
+                                 layer), kvq_cache_bytes()                  */
+  uint64_t kernel_launches;   /* kernels this handle has launched so far    */
+} kvq_stats_t;
+
+/* Validates `cfg`, allocates the pool, residual windows, block table and
+ * workspace on cfg->device, zero-fills them, and builds the free list.
+ * Ownership: the handle owns every allocation until kvq_destroy().
+ * Errors: KVQ_ERR_INVALID_ARG / KVQ_ERR_UNSUPPORTED (config), KVQ_ERR_CUDA. */
+kvq_status kvq_create(const kvq_config* cfg, kvq_handle* out);
+
+/* Frees everything the handle owns (synchronizes the device first). */
+void kvq_destroy(kvq_handle h);
+
+/* Appends n tokens.  k_bf16, v_bf16: device, bf16 [n][h_kv][d_h] (row-major),
+ * caller-owned, read before the enqueued work finishes (keep them alive until
+ * the stream reaches that point).  seq_ids_host: host int32 [n]; tokens of one
+ * sequence are appended in array order, exactly as if appended one at a time.
+ * Token-axis formats quantize each token into its page row at once
+ * (chipfoundryservices.com "KV Cache Quantization", per-token quantization).
+ * Channel-axis formats keep the newest tokens as BF16 in the residual window
+ * and, when it holds R = g_k tokens, quantize keys per channel and values per
+ * token into the group's pages (day-65 page, "Why some systems keep a
+ * full-precision window"; oh-bug.com, KIVI paragraph).
+ * Errors (state unchanged): KVQ_ERR_INVALID_ARG, KVQ_ERR_BAD_SEQ, KVQ_ERR_OOM,
+ * KVQ_ERR_CUDA. */
+kvq_status kvq_append(kvq_handle h, const void* k_bf16, const void* v_bf16,
+                      const int32_t* seq_ids_host, int32_t n, void* stream);
+
+/* Decode attention over the packed cache (day-65 page, "Why the KV cache
+ * grows so quickly"): for each batch row i and query head hq,
+ *   out[i][hq] = softmax(q[i][hq] K^T / sqrt(d_h)) V
+ * over positions [0, seq_lens[i]) of the row's sequence, reading kv head
+ * hq / (h_q / h_kv), dequantizing codes inside the kernel.
+ *   q_bf16      device bf16 [batch][h_q][d_h].
+ *   block_table device int32 [batch][bt_stride] (row i = batch row i), or NULL
+ *               to use the handle's own table (row = sequence id).
+ *   seq_lens    device int32 [batch]: positions to attend, 0 <= seq_lens[i]
+ *               <= the stored length (quantized + residual tokens).
+ *   seq_ids_host host int32 [batch] mapping rows to sequence ids, or NULL for
+ *               row i = sequence i.
+ *   out         device fp32 [batch][h_q][d_h]; empty rows give zeros.
+ * The library's split-K partials live in its workspace; one call at a time per
+ * handle may be in flight on the GPU.
+ * Errors: KVQ_ERR_INVALID_ARG, KVQ_ERR_BAD_SEQ, KVQ_ERR_CUDA. */
+kvq_status kvq_decode_attn(kvq_handle h, const void* q_bf16,
+                           const int32_t* block_table, int32_t bt_stride,
+                           const int32_t* seq_lens, const int32_t* seq_ids_host,
+                           int32_t batch, float* out, void* stream);
+
+/* Library-owned device block table: int32 [max_seqs][*stride], entry
+ * [s][j] = physical block of logical block j of sequence s, -1 if none.
+ * Valid until kvq_destroy; updated by appends in stream order. */
+kvq_status kvq_block_table(kvq_handle h, const int32_t** dev_ptr, int32_t* stride);
+
+/* Host copy of one sequence's block-table row: writes up to max_entries ids
+ * to dst (host) and the row's length to *n_entries. */
+kvq_status kvq_block_table_host(kvq_handle h, int32_t seq, int32_t* dst,
+                                int32_t max_entries, int32_t* n_entries);
+
+/* Stored length of a sequence (quantized + residual tokens). */
+kvq_status kvq_seq_len(kvq_handle h, int32_t seq, int32_t* len);
+
+/* Library-owned device array int32 [max_seqs] of stored lengths, updated by
+ * appends in stream order (usable as seq_lens when rows are sequences). */
+kvq_status kvq_seq_lens_device(kvq_handle h, const int32_t** dev_ptr);
+
+/* Returns a sequence's blocks to the back of the free list, in logical order,
+ * and resets its length to 0.  `stream` orders the device-side reset. */
+kvq_status kvq_free_seq(kvq_handle h, int32_t seq, void* stream);
+
+/* Capacity and usage counters (day-65 page's memory formula for bytes_formula;
+ * oh-bug.com checklist item on monitoring KV-cache usage). */
+kvq_status kvq_stats(kvq_handle h, kvq_stats_t* out);
+
+/* The day-65 memory formula M = 2 L T H_kv d_h b with b the bytes per element
+ * of the format including its group metadata: keys bits/8 + meta/g_k, values
+ * bits/8 + meta/g_v, meta = scale bytes (+ zero-point bytes).  For L=32,
+ * T=8192, H_kv=8, d_h=128, 4 bits, fp16 scale per 64: 285,212,672 bytes
+ * (272 MiB).  Returns 0 for an invalid config. */
+uint64_t kvq_cache_bytes(int32_t layers, int64_t tokens, int32_t h_kv, int32_t d_h,
+                         const kvq_config* cfg);
+
+/* Byte geometry of a format (no handle needed). */
+kvq_status kvq_layout(const kvq_config* cfg, kvq_layout_info* out);
+
+/* Copies the whole block pool (device) to host_dst: num_blocks * block_bytes
+ * bytes; synchronizes `stream`.  For parity checks and debugging. */
+kvq_status kvq_read_pool(kvq_handle h, void* host_dst, uint64_t bytes, void* stream);
+
+/* Copies the residual windows (device, bf16 [max_seqs][h_kv][R][d_h]) of keys
+ * and values to host; each buffer takes `bytes`; synchronizes `stream`. */
+kvq_status kvq_read_residual(kvq_handle h, void* k_host, void* v_host, uint64_t bytes,
+                             void* stream);
+
+/* Synchronizes `stream`, reads and clears the device error word.  Returns
+ * KVQ_ERR_DEVICE_CHECK (and the word in *bits_out if not NULL) when a kernel's
+ * check fired, KVQ_ERR_CUDA on a CUDA error, else KVQ_OK. */
+kvq_status kvq_sync_status(kvq_handle h, void* stream, uint32_t* bits_out);
+
+/* Overrides the decode kernel's grid (number of CTAs); 0 restores the default
+ * (one resident wave on every SM).  Changes how the key range is split across
+ * CTAs, never the result beyond rounding. */
+kvq_status kvq_set_decode_grid(kvq_handle h, int32_t ctas);
+
+/* Profiling hook: when `event` (a cudaEvent_t) is not NULL, every later
+ * kvq_decode_attn records it on its stream between the attention kernel and
+ * the kernel that merges split partials, so a caller can time the attention
+ * kernel alone with CUDA events.  NULL turns it off.  The event stays owned by
+ * the caller and must outlive its use. */
+kvq_status kvq_set_decode_event(kvq_handle h, void* event);
+
+/* Text of the last failure on the calling thread ("" if none). */
+const char* kvq_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H_ */

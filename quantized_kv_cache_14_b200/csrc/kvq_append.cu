@@ -1,0 +1,398 @@
+// kvq_append.cu -- kernels of kvq_append: quantize new K/V tokens into the
+// paged cache.
+//
+//  * apply: zero newly allocated blocks that this call does not fill, and
+//    write block-table / length updates of the host planner.
+//  * quant_token (token-axis keys, no residual window): one warp per (token,
+//    head) quantizes the key row per g_k channels and the value row per g_v
+//    channels (chipfoundryservices.com "KV Cache Quantization", per-token
+//    quantization; llmdaily.org day-65, "From BF16 to INT8, INT4, or even
+//    fewer bits", symmetric quantizer and asymmetric zero-points).
+//  * flush (channel-axis keys): once a sequence's BF16 residual window holds a
+//    whole key group of R = g_k tokens, one CTA per (group, head) quantizes
+//    keys per channel over the g_k tokens and values per token over g_v
+//    channels and writes the group's pages (day-65, "Why some systems keep a
+//    full-precision window"; oh-bug.com "KV Cache Quantization in Practice",
+//    KIVI: keys per channel, values per token).  Tokens of the group appended
+//    in this call are read straight from the input, earlier ones from the
+//    window; the bytes equal those of appending one token at a time.
+//  * residual: copy the tokens that stay in the window to their slots.
+#include <algorithm>
+#include <cstdint>
+#include <type_traits>
+
+#include "kvq_device.cuh"
+
+namespace kvq {
+namespace {
+
+// ---------------------------------------------------------------------------
+__global__ void apply_kernel(const Geo g, const DevState d, const PlanView p) {
+  const int64_t tid = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t nthr = int64_t(gridDim.x) * blockDim.x;
+  // zero whole blocks (16-byte stores)
+  const int64_t per_block = g.block_bytes / 16;
+  const int64_t zero_items = int64_t(p.n_zero) * per_block;
+  for (int64_t i = tid; i < zero_items; i += nthr) {
+    const int32_t blk = p.plan[p.off_zero + i / per_block];
+    reinterpret_cast<uint4*>(d.pool + int64_t(blk) * g.block_bytes)[i % per_block] =
+        make_uint4(0, 0, 0, 0);
+  }
+  for (int64_t i = tid; i < p.n_tab; i += nthr)
+    d.table[p.plan[p.off_tab + 2 * i]] = p.plan[p.off_tab + 2 * i + 1];
+  for (int64_t i = tid; i < p.n_len; i += nthr)
+    d.len[p.plan[p.off_len + 2 * i]] = p.plan[p.off_len + 2 * i + 1];
+}
+
+// ---------------------------------------------------------------------------
+// Per-token quantization: one warp per (token, head); lane l holds channels
+// 4l .. 4l+3.
+template <int BITS, int ASYM>
+__global__ void __launch_bounds__(256) quant_token_kernel(const Geo g, const DevState d,
+                                                          const PlanView p, const uint16_t* kin,
+                                                          const uint16_t* vin) {
+  constexpr int D = kD;
+  constexpr int N = 32 / BITS;                 // codes per word
+  constexpr int Q = ASYM ? (1 << BITS) - 1 : (1 << (BITS - 1)) - 1;
+  __shared__ int8_t s_codes[8][D];             // per warp: codes by channel
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int64_t item = int64_t(blockIdx.x) * 8 + wib;
+  if (item >= int64_t(p.n_tok) * g.h_kv) return;
+  const int e = int(item / g.h_kv), h = int(item % g.h_kv);
+  const int32_t src = p.plan[p.off_tok + 3 * e];
+  const int32_t blk = p.plan[p.off_tok + 3 * e + 1];
+  const int32_t tok = p.plan[p.off_tok + 3 * e + 2];
+  uint8_t* chunk = d.pool + int64_t(blk) * g.block_bytes + int64_t(h) * g.chunk_bytes;
+  const int sub = tok >> 4, r = tok & 15;
+
+  for (int which = 0; which < 2; ++which) {      // 0: key row, 1: value row
+    const uint16_t* row = (which ? vin : kin) + (int64_t(src) * g.h_kv + h) * D;
+    const uint2 raw = *reinterpret_cast<const uint2*>(row + 4 * lane);
+    float x[4] = {bf16_bits_to_float(raw.x & 0xFFFF), bf16_bits_to_float(raw.x >> 16),
+                  bf16_bits_to_float(raw.y & 0xFFFF), bf16_bits_to_float(raw.y >> 16)};
+    const int gsz = which ? g.g_v : g.g_k;
+    const int ng = which ? g.nvg : g.nkg;
+    const int lanes_per_group = gsz / 4;
+    float a = 0.0f, mn = x[0], mx = x[0];
+    for (int i = 0; i < 4; ++i) {
+      a = fmaxf(a, fabsf(x[i]));
+      mn = fminf(mn, x[i]);
+      mx = fmaxf(mx, x[i]);
+    }
+    for (int off = 1; off < lanes_per_group; off <<= 1) {
+      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    }
+    float sh, zh = 0.0f;
+    if (ASYM) {
+      zh = stored_value(mn, g.scale_fp32);
+      sh = stored_value(__fdiv_rn(__fsub_rn(mx, mn), float(Q)), g.scale_fp32);
+    } else {
+      sh = stored_value(__fdiv_rn(a, float(Q)), g.scale_fp32);
+    }
+    for (int i = 0; i < 4; ++i)
+      s_codes[wib][4 * lane + i] =
+          int8_t(ASYM ? quant_asym(x[i], sh, zh, Q) : quant_sym(x[i], sh, Q));
+    const int gi = (4 * lane) / gsz;
+    if ((4 * lane) % gsz == 0) {
+      const int off_meta = which ? g.off_Vm : g.off_Km;
+      uint8_t* m = chunk + off_meta + (int64_t(tok) * ng + gi) * g.es;
+      store_meta(m, sh, g.scale_fp32);
+      if (ASYM) store_meta(m + int64_t(g.P) * ng * g.es, zh, g.scale_fp32);
+    }
+    __syncwarp();
+    if (which == 0) {
+      // key row: D*BITS/32 words, element l of word w is list position w*N + l
+      if (lane < D * BITS / 32) {
+        uint32_t word = 0;
+        for (int l = 0; l < N; ++l) {
+          const int c = key_channel(lane * N + l);
+          word |= (uint32_t(s_codes[wib][c]) & ((1u << BITS) - 1)) << (BITS * word_field(l, N));
+        }
+        *reinterpret_cast<uint32_t*>(chunk + sub * g.sub_bytes + r * g.row_bytes + 4 * lane) = word;
+      }
+    } else {
+      // value codes: this token owns whole bytes of its sub-tile
+      const int tau = r, tq = (tau & 7) >> 1, hi = tau & 1, second = tau >> 3;
+      uint8_t* vsub = chunk + g.off_V + sub * g.sub_bytes;
+      constexpr int bytes_per_token = D * BITS / 8;
+      for (int bi = lane; bi < bytes_per_token; bi += 32) {
+        uint32_t byte = 0;
+        int gq, word, bsel;
+        if (BITS == 4) {
+          gq = bi >> 3;
+          const int i = bi & 7;
+          word = i;
+          bsel = 2 * hi + second;
+          byte = (uint32_t(s_codes[wib][16 * i + gq]) & 15u) |
+                 ((uint32_t(s_codes[wib][16 * i + gq + 8]) & 15u) << 4);
+        } else if (BITS == 2) {
+          gq = bi >> 2;
+          const int i2 = bi & 3;
+          word = i2;
+          bsel = 2 * hi + second;
+          const int cs[4] = {32 * i2 + gq, 32 * i2 + gq + 8, 32 * i2 + 16 + gq, 32 * i2 + 24 + gq};
+          for (int m = 0; m < 4; ++m) byte |= (uint32_t(s_codes[wib][cs[m]]) & 3u) << (2 * m);
+        } else {
+          gq = bi >> 4;
+          const int rest = bi & 15, i = rest >> 1, half = rest & 1;
+          word = 2 * i + second;
+          bsel = 2 * hi + half;
+          byte = uint32_t(s_codes[wib][16 * i + gq + 8 * half]) & 255u;
+        }
+        const int lam = 4 * gq + tq;
+        vsub[lam * (8 * BITS) + 4 * word + bsel] = uint8_t(byte);
+      }
+    }
+    __syncwarp();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Per-channel key flush: one CTA per (flushed group, head).
+template <int BITS, int ASYM>
+__global__ void __launch_bounds__(kFlushThreads) flush_kernel(const Geo g, const DevState d,
+                                                              const PlanView p,
+                                                              const uint16_t* kin,
+                                                              const uint16_t* vin) {
+  constexpr int D = kD;
+  constexpr int N = 32 / BITS;
+  constexpr int Q = ASYM ? (1 << BITS) - 1 : (1 << (BITS - 1)) - 1;
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int R = g.R;
+  uint16_t* kt = reinterpret_cast<uint16_t*>(smem);                  // [R][D] bf16
+  uint16_t* vt = kt + R * D;                                         // [R][D]
+  float* ksc = reinterpret_cast<float*>(vt + R * D);                 // [D]
+  float* kzp = ksc + D;                                              // [D]
+  float* vsc = kzp + D;                                              // [R][nvg]
+  float* vzp = vsc + R * g.nvg;                                      // [R][nvg]
+
+  const int e = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+  const int32_t* ent = p.plan + p.off_flush + e * kFlushEntryInts;
+  const int seq = ent[0];
+  const int npg = ent[2];
+  const int32_t* srcs = p.plan + p.off_src + int64_t(e) * R;
+
+  // 1. gather the group's K and V rows (bf16) into shared memory
+  for (int idx = tid; idx < R * (D / 8) * 2; idx += blockDim.x) {
+    const int which = idx / (R * (D / 8));
+    const int rem = idx % (R * (D / 8));
+    const int r = rem / (D / 8), c8 = rem % (D / 8);
+    const int32_t s = srcs[r];
+    const uint16_t* src;
+    if (s >= 0) src = (which ? vin : kin) + (int64_t(s) * g.h_kv + h) * D;
+    else src = (which ? d.vres : d.kres) + ((int64_t(seq) * g.h_kv + h) * R + (-1 - s)) * D;
+    reinterpret_cast<uint4*>((which ? vt : kt) + r * D)[c8] = reinterpret_cast<const uint4*>(src)[c8];
+  }
+  __syncthreads();
+
+  // 2. statistics: key channels (threads 0..127), value (token, group) rows
+  if (tid < D) {
+    const int c = tid;
+    float a = 0.0f, mn = bf16_bits_to_float(kt[c]), mx = mn;
+    for (int r = 0; r < R; ++r) {
+      const float x = bf16_bits_to_float(kt[r * D + c]);
+      a = fmaxf(a, fabsf(x));
+      mn = fminf(mn, x);
+      mx = fmaxf(mx, x);
+    }
+    if (ASYM) {
+      kzp[c] = stored_value(mn, g.scale_fp32);
+      ksc[c] = stored_value(__fdiv_rn(__fsub_rn(mx, mn), float(Q)), g.scale_fp32);
+    } else {
+      ksc[c] = stored_value(__fdiv_rn(a, float(Q)), g.scale_fp32);
+      kzp[c] = 0.0f;
+    }
+  } else {
+    const int w = (tid - D) >> 5, lane = tid & 31;
+    const int lanes_per_group = g.g_v / 4;
+    for (int r = w; r < R; r += (blockDim.x - D) / 32) {
+      float x[4];
+      for (int i = 0; i < 4; ++i) x[i] = bf16_bits_to_float(vt[r * D + 4 * lane + i]);
+      float a = 0.0f, mn = x[0], mx = x[0];
+      for (int i = 0; i < 4; ++i) {
+        a = fmaxf(a, fabsf(x[i]));
+        mn = fminf(mn, x[i]);
+        mx = fmaxf(mx, x[i]);
+      }
+      for (int off = 1; off < lanes_per_group; off <<= 1) {
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      }
+      if ((4 * lane) % g.g_v == 0) {
+        const int gi = (4 * lane) / g.g_v;
+        if (ASYM) {
+          vzp[r * g.nvg + gi] = stored_value(mn, g.scale_fp32);
+          vsc[r * g.nvg + gi] = stored_value(__fdiv_rn(__fsub_rn(mx, mn), float(Q)), g.scale_fp32);
+        } else {
+          vsc[r * g.nvg + gi] = stored_value(__fdiv_rn(a, float(Q)), g.scale_fp32);
+          vzp[r * g.nvg + gi] = 0.0f;
+        }
+      }
+    }
+  }
+  __syncthreads();
+
+  auto chunk_of = [&](int page) -> uint8_t* {
+    return d.pool + int64_t(ent[3 + page]) * g.block_bytes + int64_t(h) * g.chunk_bytes;
+  };
+  auto kcode = [&](int r, int c) -> uint32_t {
+    const float x = bf16_bits_to_float(kt[r * D + c]);
+    const int q = ASYM ? quant_asym(x, ksc[c], kzp[c], Q) : quant_sym(x, ksc[c], Q);
+    return uint32_t(q) & ((1u << BITS) - 1);
+  };
+  auto vcode = [&](int r, int c) -> uint32_t {
+    const float x = bf16_bits_to_float(vt[r * D + c]);
+    const int gi = c / g.g_v;
+    const int q = ASYM ? quant_asym(x, vsc[r * g.nvg + gi], vzp[r * g.nvg + gi], Q)
+                       : quant_sym(x, vsc[r * g.nvg + gi], Q);
+    return uint32_t(q) & ((1u << BITS) - 1);
+  };
+  const int subs_per_page = g.P / 16;
+
+  // 3. key codes: word W of the group -> (sub-tile, row, word in row)
+  const int row_words = D * BITS / 32;
+  const int k_words = R * row_words;
+  for (int W = tid; W < k_words; W += blockDim.x) {
+    const int rowi = W / row_words, w = W % row_words;       // rowi = token in group
+    uint32_t word = 0;
+    for (int l = 0; l < N; ++l) word |= kcode(rowi, key_channel(w * N + l)) << (BITS * word_field(l, N));
+    const int sub = rowi >> 4, rr = rowi & 15;
+    uint8_t* dst = chunk_of(sub / subs_per_page) + (sub % subs_per_page) * g.sub_bytes +
+                   rr * g.row_bytes + 4 * w;
+    *reinterpret_cast<uint32_t*>(dst) = word;
+  }
+
+  // 4. value codes: word W -> (sub-tile, lane record, word in record); the
+  //    record of lane (4 gq + tq) packs mma operand registers a0..a3 of each
+  //    16-channel tile i: a0 = (ch 16i+gq, tok 2tq | 2tq+1), a1 = ch + 8,
+  //    a2 = tokens + 8, a3 = both.
+  const int rec_words = 2 * BITS;
+  const int v_words = (R / 16) * 32 * rec_words;
+  for (int W = tid; W < v_words; W += blockDim.x) {
+    const int sub = W / (32 * rec_words), rem = W % (32 * rec_words);
+    const int lam = rem / rec_words, w = rem % rec_words;
+    const int gq = lam >> 2, tq = lam & 3;
+    uint32_t word = 0;
+    for (int x = 0; x < N / 2; ++x) {
+      int i, reg;
+      if (BITS == 8) { i = w >> 1; reg = 2 * (w & 1) + x; }
+      else if (BITS == 4) { i = w; reg = x; }
+      else { i = 2 * w + ((x >> 1) & 1); reg = 2 * (x >> 2) + (x & 1); }
+      const int c = 16 * i + gq + 8 * (reg & 1);
+      const int t0 = 16 * sub + 2 * tq + 8 * (reg >> 1);
+      word |= vcode(t0, c) << (BITS * x);
+      word |= vcode(t0 + 1, c) << (BITS * (x + N / 2));
+    }
+    uint8_t* dst = chunk_of(sub / subs_per_page) + g.off_V + (sub % subs_per_page) * g.sub_bytes +
+                   lam * (8 * BITS) + 4 * w;
+    *reinterpret_cast<uint32_t*>(dst) = word;
+  }
+
+  // 5. metadata: key scales in list order, striped over the group's pages;
+  //    value scales per token row
+  for (int f = tid; f < D; f += blockDim.x) {
+    const int c = key_channel(f);
+    const int page = f / g.kslice, off = f % g.kslice;
+    uint8_t* km = chunk_of(page) + g.off_Km;
+    store_meta(km + off * g.es, ksc[c], g.scale_fp32);
+    if (ASYM) store_meta(km + (g.kslice + off) * g.es, kzp[c], g.scale_fp32);
+  }
+  for (int idx = tid; idx < R * g.nvg; idx += blockDim.x) {
+    const int r = idx / g.nvg, gi = idx % g.nvg;
+    const int page = r / g.P, rp = r % g.P;
+    uint8_t* vm = chunk_of(page) + g.off_Vm;
+    store_meta(vm + (rp * g.nvg + gi) * g.es, vsc[idx], g.scale_fp32);
+    if (ASYM) store_meta(vm + (g.P * g.nvg + rp * g.nvg + gi) * g.es, vzp[idx], g.scale_fp32);
+  }
+  (void)npg;
+}
+
+// ---------------------------------------------------------------------------
+__global__ void residual_kernel(const Geo g, const DevState d, const PlanView p,
+                                const uint16_t* kin, const uint16_t* vin) {
+  constexpr int D = kD;
+  const int64_t total = int64_t(p.n_res) * g.h_kv * 2 * (D / 8);
+  for (int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += int64_t(gridDim.x) * blockDim.x) {
+    const int c8 = int(idx % (D / 8));
+    int64_t rest = idx / (D / 8);
+    const int which = int(rest % 2);
+    rest /= 2;
+    const int h = int(rest % g.h_kv);
+    const int e = int(rest / g.h_kv);
+    const int32_t src = p.plan[p.off_res + 3 * e];
+    const int32_t seq = p.plan[p.off_res + 3 * e + 1];
+    const int32_t slot = p.plan[p.off_res + 3 * e + 2];
+    const uint16_t* s = (which ? vin : kin) + (int64_t(src) * g.h_kv + h) * D;
+    uint16_t* dst = (which ? d.vres : d.kres) + ((int64_t(seq) * g.h_kv + h) * g.R + slot) * D;
+    reinterpret_cast<uint4*>(dst)[c8] = reinterpret_cast<const uint4*>(s)[c8];
+  }
+}
+
+template <typename F>
+cudaError_t by_format(const Geo& g, F&& f) {
+  if (g.bits == 8) return g.asym ? f(std::integral_constant<int, 8>(), std::integral_constant<int, 1>())
+                                 : f(std::integral_constant<int, 8>(), std::integral_constant<int, 0>());
+  if (g.bits == 4) return g.asym ? f(std::integral_constant<int, 4>(), std::integral_constant<int, 1>())
+                                 : f(std::integral_constant<int, 4>(), std::integral_constant<int, 0>());
+  return g.asym ? f(std::integral_constant<int, 2>(), std::integral_constant<int, 1>())
+                : f(std::integral_constant<int, 2>(), std::integral_constant<int, 0>());
+}
+
+size_t flush_smem_bytes(const Geo& g) {
+  return size_t(2) * g.R * kD * 2 + size_t(2) * kD * 4 + size_t(2) * g.R * g.nvg * 4;
+}
+
+}  // namespace
+
+cudaError_t launch_apply(const Geo& g, const DevState& d, const PlanView& p, cudaStream_t s,
+                         int* launches) {
+  const int64_t work = std::max<int64_t>(int64_t(p.n_zero) * (g.block_bytes / 16),
+                                         std::max(p.n_tab, p.n_len));
+  if (work == 0) return cudaSuccess;
+  const int blocks = int(std::min<int64_t>((work + 255) / 256, 4096));
+  apply_kernel<<<blocks, 256, 0, s>>>(g, d, p);
+  ++*launches;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_token(const Geo& g, const DevState& d, const PlanView& p,
+                               const uint16_t* k, const uint16_t* v, cudaStream_t s, int* launches) {
+  if (p.n_tok == 0) return cudaSuccess;
+  const int64_t items = int64_t(p.n_tok) * g.h_kv;
+  const int blocks = int((items + 7) / 8);
+  return by_format(g, [&](auto B, auto A) {
+    quant_token_kernel<decltype(B)::value, decltype(A)::value><<<blocks, 256, 0, s>>>(g, d, p, k, v);
+    ++*launches;
+    return cudaGetLastError();
+  });
+}
+
+cudaError_t launch_flush(const Geo& g, const DevState& d, const PlanView& p, const uint16_t* k,
+                         const uint16_t* v, cudaStream_t s, int* launches) {
+  if (p.n_flush == 0) return cudaSuccess;
+  const size_t smem = flush_smem_bytes(g);
+  return by_format(g, [&](auto B, auto A) {
+    auto kern = flush_kernel<decltype(B)::value, decltype(A)::value>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    kern<<<dim3(p.n_flush, g.h_kv), kFlushThreads, smem, s>>>(g, d, p, k, v);
+    ++*launches;
+    return cudaGetLastError();
+  });
+}
+
+cudaError_t launch_residual(const Geo& g, const DevState& d, const PlanView& p, const uint16_t* k,
+                            const uint16_t* v, cudaStream_t s, int* launches) {
+  if (p.n_res == 0) return cudaSuccess;
+  const int64_t total = int64_t(p.n_res) * g.h_kv * 2 * (kD / 8);
+  const int blocks = int(std::min<int64_t>((total + 255) / 256, 8192));
+  residual_kernel<<<blocks, 256, 0, s>>>(g, d, p, k, v);
+  ++*launches;
+  return cudaGetLastError();
+}
+
+}  // namespace kvq

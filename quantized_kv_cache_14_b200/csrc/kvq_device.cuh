@@ -1,0 +1,236 @@
+// kvq_device.cuh -- device helpers of the kvq kernels: the storage format's
+// word packing, code unpacking to bf16 operand pairs, the quantizer, and thin
+// wrappers over PTX (mma.sync, ldmatrix, mbarrier, bulk async copies).
+#pragma once
+
+#include <cstdint>
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "kvq_internal.h"
+
+namespace kvq {
+
+// ---------------------------------------------------------------------------
+// Format rules (the storage contract; see the format notes).
+// ---------------------------------------------------------------------------
+
+// Key rows list channels in mma-operand order: position f = 32 t + 4 j + e
+// holds channel 16 j + 2 t + (e & 1) + 8 (e >> 1).
+__host__ __device__ constexpr int key_channel(int f) {
+  return 16 * ((f >> 2) & 7) + 2 * (f >> 5) + (f & 1) + 8 * ((f >> 1) & 1);
+}
+
+// Element l of a word of n elements occupies field (l >> 1) + (n / 2)(l & 1):
+// even elements take the low half-word, odd elements the high half-word.
+__host__ __device__ constexpr int word_field(int l, int n) { return (l >> 1) + (n >> 1) * (l & 1); }
+
+// bf16 bit pattern of an exactly representable float (compile time).
+__host__ __device__ constexpr uint32_t bf16x2_of(float x) {
+  return (__builtin_bit_cast(uint32_t, x) >> 16) * 0x10001u;
+}
+
+// ---------------------------------------------------------------------------
+// PTX wrappers.
+// ---------------------------------------------------------------------------
+
+// r = (a & mask) ^ k  (one LOP3).
+__device__ __forceinline__ uint32_t and_xor(uint32_t a, uint32_t mask, uint32_t k) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(r) : "r"(a), "r"(mask), "r"(k));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t bf2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t r;
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+
+// D += A * B, m16n8k16, bf16 operands, fp32 accumulation.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_init_fence() {
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bulk (TMA, non-tensor) copy global -> shared, completing on an mbarrier.
+// dst/src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                         uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// Orders this thread's earlier generic-proxy shared-memory accesses before
+// later async-proxy (bulk copy) writes to the same buffer.
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+
+// Bounded wait on an mbarrier phase: true when complete, false after
+// `limit` polls (the caller records a timeout and stops issuing work).
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint32_t limit) {
+  for (uint32_t it = 0; it < limit; ++it)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
+// ---------------------------------------------------------------------------
+// Unpacking codes into bf16x2 operand registers.
+//
+// A bf16 with exponent field 0x86 holds 128 + m for a 7-bit integer m in its
+// mantissa bits, so OR-ing a small field into the mantissa of 0x4300 gives
+// 128 + field exactly; one bf16x2 FMA then removes the 128 (and a signed code's
+// offset) and undoes any left shift of the field.  Two's complement fields are
+// turned into offset binary by flipping their top bit in the same LOP3.
+// ---------------------------------------------------------------------------
+
+// 4-bit fields at bit 4x (low half) and 16 + 4x (high half) -> bf16x2.
+template <bool SIGNED>
+__device__ __forceinline__ uint32_t nib_pair(uint32_t w, int x) {
+  const uint32_t v = x ? (w >> (4 * x)) : w;
+  const uint32_t r = and_xor(v, 0x000F000Fu, SIGNED ? 0x43084308u : 0x43004300u);
+  return bf2_fma(r, bf16x2_of(1.0f), SIGNED ? bf16x2_of(-136.0f) : bf16x2_of(-128.0f));
+}
+
+// 2-bit fields at bit 2x and 16 + 2x, x in [0, 8).
+template <bool SIGNED>
+__device__ __forceinline__ uint32_t crumb_pair(uint32_t w, int x) {
+  // fields 0..2 read from w, 3..5 from w >> 6, 6..7 from w >> 12, at local
+  // position y (bits 2y..2y+1 of each half, all inside the 7 mantissa bits)
+  const int shift = x < 3 ? 0 : (x < 6 ? 6 : 12);
+  const int y = x - (x < 3 ? 0 : (x < 6 ? 3 : 6));
+  const uint32_t v = shift ? (w >> shift) : w;
+  const uint32_t m = 0x00030003u << (2 * y);
+  const uint32_t k = 0x43004300u | (SIGNED ? (0x00020002u << (2 * y)) : 0u);
+  const uint32_t r = and_xor(v, m, k);
+  // r = 128 + 4^y c  ->  c - offset = r / 4^y - 128 / 4^y - offset
+  const float off = SIGNED ? 2.0f : 0.0f;
+  const uint32_t mul = y == 0 ? bf16x2_of(1.0f) : (y == 1 ? bf16x2_of(0.25f) : bf16x2_of(0.0625f));
+  const uint32_t add = y == 0 ? bf16x2_of(-128.0f - off)
+                              : (y == 1 ? bf16x2_of(-32.0f - off) : bf16x2_of(-8.0f - off));
+  return bf2_fma(r, mul, add);
+}
+
+// 8-bit fields at byte x and byte x + 2 (x in {0, 1}) -> bf16x2, built from
+// the two nibble planes: code = low nibble (unsigned) + 16 * high nibble.
+template <bool SIGNED>
+__device__ __forceinline__ uint32_t byte_pair(uint32_t w, int x) {
+  const uint32_t vlo = x ? (w >> 8) : w;
+  const uint32_t vhi = x ? (w >> 12) : (w >> 4);
+  const uint32_t lo = bf2_fma(and_xor(vlo, 0x000F000Fu, 0x43004300u), bf16x2_of(1.0f),
+                              bf16x2_of(-128.0f));
+  const uint32_t hr = and_xor(vhi, 0x000F000Fu, SIGNED ? 0x43084308u : 0x43004300u);
+  const uint32_t hi16 = bf2_fma(hr, bf16x2_of(16.0f), SIGNED ? bf16x2_of(-2176.0f) : bf16x2_of(-2048.0f));
+  return bf2_fma(lo, bf16x2_of(1.0f), hi16);
+}
+
+// ---------------------------------------------------------------------------
+// hi/lo bf16 split of fp32 values for a two-column tensor-core product:
+// hi = bf16_rn(x), lo = bf16_rn(x - hi); hi + lo carries x with relative error
+// <= 2^-16.  Returns the pair (x0, x1) as packed hi parts, or as packed lo
+// parts when `lo` is set.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t split_pack(float x0, float x1, bool lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);   // .x = x0 (low half)
+  const uint32_t hb = *reinterpret_cast<const uint32_t*>(&h);
+  const float h0 = __uint_as_float(hb << 16);
+  const float h1 = __uint_as_float(hb & 0xFFFF0000u);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - h0, x1 - h1);
+  const uint32_t lb = *reinterpret_cast<const uint32_t*>(&l);
+  return lo ? lb : hb;
+}
+
+// ---------------------------------------------------------------------------
+// The quantizer (IEEE fp32 division, round half to even, stored scale).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float stored_value(float s, int scale_fp32) {
+  if (scale_fp32) return s;
+  float r = __half2float(__float2half_rn(s));
+  if (isinf(r)) r = r > 0.0f ? 65504.0f : -65504.0f;
+  return r;
+}
+
+__device__ __forceinline__ int quant_sym(float x, float sh, int Q) {
+  if (sh == 0.0f) return 0;
+  int q = __float2int_rn(__fdiv_rn(x, sh));
+  return q < -Q ? -Q : (q > Q ? Q : q);
+}
+
+__device__ __forceinline__ int quant_asym(float x, float sh, float zh, int Qa) {
+  if (sh == 0.0f) return 0;
+  int q = __float2int_rn(__fdiv_rn(__fsub_rn(x, zh), sh));
+  return q < 0 ? 0 : (q > Qa ? Qa : q);
+}
+
+__device__ __forceinline__ void store_meta(uint8_t* p, float v, int scale_fp32) {
+  if (scale_fp32) *reinterpret_cast<float*>(p) = v;
+  else *reinterpret_cast<uint16_t*>(p) = __half_as_ushort(__float2half_rn(v));
+}
+
+__device__ __forceinline__ float load_meta(const uint8_t* p, int scale_fp32) {
+  if (scale_fp32) return *reinterpret_cast<const float*>(p);
+  return __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t*>(p)));
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+  return __uint_as_float(uint32_t(b) << 16);
+}
+
+}  // namespace kvq

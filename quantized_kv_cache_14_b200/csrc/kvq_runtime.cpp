@@ -1,0 +1,691 @@
+// kvq_runtime.cpp -- host runtime of libkvq.so: the C ABI of include/kvq.h.
+//
+// Owns the device pool, the BF16 residual windows, the block table and the
+// workspace; keeps the authoritative host bookkeeping (lengths, block tables,
+// the free list) and turns each kvq_append into a compact plan that one H2D
+// copy and a few kernels execute (llmdaily.org day-65, "How this connects to
+// paging and prefix caching": blocks allocated on demand and addressed
+// through a block table).
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <deque>
+#include <string>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "kvq.h"
+#include "kvq_internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+kvq_status fail(kvq_status s, const std::string& msg) {
+  g_last_error = msg;
+  return s;
+}
+
+#define KVQ_CUDA(call)                                                                     \
+  do {                                                                                     \
+    cudaError_t e_ = (call);                                                               \
+    if (e_ != cudaSuccess)                                                                 \
+      return fail(KVQ_ERR_CUDA, std::string(#call) + ": " + cudaGetErrorString(e_));       \
+  } while (0)
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// splitmix64 (Steele, Lea, Flood 2014).
+uint64_t splitmix64(uint64_t& state) {
+  state += 0x9E3779B97F4A7C15ull;
+  uint64_t z = state;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+bool is_group_size(int g) { return g == 16 || g == 32 || g == 64 || g == 128; }
+
+kvq_status validate(const kvq_config* c) {
+  if (!c) return fail(KVQ_ERR_INVALID_ARG, "config is null");
+  if (c->bits != 2 && c->bits != 4 && c->bits != 8) return fail(KVQ_ERR_INVALID_ARG, "bits must be 2, 4 or 8");
+  if (c->asym != 0 && c->asym != 1) return fail(KVQ_ERR_INVALID_ARG, "asym must be 0 or 1");
+  if (c->scale_fp32 != 0 && c->scale_fp32 != 1) return fail(KVQ_ERR_INVALID_ARG, "scale_fp32 must be 0 or 1");
+  if (c->d_h != kvq::kD) return fail(KVQ_ERR_UNSUPPORTED, "d_h must be 128");
+  if (c->h_kv < 1 || c->h_q < 1 || c->h_q % c->h_kv != 0)
+    return fail(KVQ_ERR_INVALID_ARG, "h_q must be a positive multiple of h_kv");
+  const int G = c->h_q / c->h_kv;
+  if (G != 1 && G != 2 && G != 4) return fail(KVQ_ERR_UNSUPPORTED, "h_q / h_kv must be 1, 2 or 4");
+  if (c->g_v != 32 && c->g_v != 64 && c->g_v != 128) return fail(KVQ_ERR_UNSUPPORTED, "g_v must be 32, 64 or 128");
+  if (c->page < 16 || c->page % 16 != 0) return fail(KVQ_ERR_INVALID_ARG, "page must be a positive multiple of 16");
+  if (c->k_axis == KVQ_AXIS_TOKEN) {
+    if (c->g_k != 32 && c->g_k != 64 && c->g_k != 128)
+      return fail(KVQ_ERR_UNSUPPORTED, "token-axis g_k must be 32, 64 or 128");
+    if (c->residual != 0) return fail(KVQ_ERR_INVALID_ARG, "token-axis keys take no residual window");
+    if (c->page > 4096) return fail(KVQ_ERR_UNSUPPORTED, "page must be <= 4096");
+  } else if (c->k_axis == KVQ_AXIS_CHANNEL) {
+    if (!is_group_size(c->g_k)) return fail(KVQ_ERR_UNSUPPORTED, "channel-axis g_k must be 16, 32, 64 or 128");
+    if (c->residual != c->g_k) return fail(KVQ_ERR_INVALID_ARG, "channel-axis keys need residual == g_k");
+    if (c->page > c->g_k || c->g_k % c->page != 0)
+      return fail(KVQ_ERR_UNSUPPORTED, "channel-axis keys need page to divide g_k");
+  } else {
+    return fail(KVQ_ERR_INVALID_ARG, "k_axis must be 0 (token) or 1 (channel)");
+  }
+  if (c->max_seqs < 1 || c->num_blocks < 1 || c->max_blocks_per_seq < 1)
+    return fail(KVQ_ERR_INVALID_ARG, "capacity fields must be positive");
+  if (c->fail_alloc_after < -1) return fail(KVQ_ERR_INVALID_ARG, "fail_alloc_after must be >= -1");
+  return KVQ_OK;
+}
+
+kvq::Geo make_geo(const kvq_config& c) {
+  kvq::Geo g{};
+  const int D = kvq::kD, A = 1 + c.asym;
+  g.bits = c.bits; g.asym = c.asym; g.k_axis = c.k_axis; g.g_k = c.g_k; g.g_v = c.g_v;
+  g.scale_fp32 = c.scale_fp32; g.R = c.residual; g.P = c.page; g.h_q = c.h_q; g.h_kv = c.h_kv;
+  g.G = c.h_q / c.h_kv;
+  g.n = 32 / c.bits;
+  g.row_bytes = D * c.bits / 8;
+  g.sub_bytes = 16 * g.row_bytes;
+  g.es = c.scale_fp32 ? 4 : 2;
+  g.nvg = D / c.g_v;
+  g.secK = (c.page / 16) * g.sub_bytes;
+  g.secV = g.secK;
+  g.secVm = int(align_up(size_t(c.page) * g.nvg * g.es * A, 16));
+  if (c.k_axis == KVQ_AXIS_TOKEN) {
+    g.nkg = D / c.g_k;
+    g.kslice = 0;
+    g.secKm = int(align_up(size_t(c.page) * g.nkg * g.es * A, 16));
+  } else {
+    g.nkg = 1;
+    g.kslice = D / (c.g_k / c.page);
+    g.secKm = int(align_up(size_t(g.kslice) * g.es * A, 16));
+  }
+  g.off_V = g.secK;
+  g.off_Vm = g.off_V + g.secV;
+  g.off_Km = g.off_Vm + g.secVm;
+  g.chunk_used = g.off_Km + g.secKm;
+  g.chunk_bytes = int64_t(align_up(size_t(g.chunk_used), 32));
+  g.block_bytes = int64_t(c.h_kv) * g.chunk_bytes;
+  g.num_blocks = c.num_blocks;
+  g.max_seqs = c.max_seqs;
+  g.mbps = c.max_blocks_per_seq;
+  g.tileT = c.k_axis == KVQ_AXIS_CHANNEL ? c.g_k : 16;
+  g.vm16 = int(align_up(size_t(16) * g.nvg * g.es * A, 16));
+  g.km16 = int(align_up(size_t(16) * g.nkg * g.es * A, 16));
+  g.qtile_bytes = c.k_axis == KVQ_AXIS_CHANNEL ? (c.g_k / c.page) * g.chunk_used
+                                               : 2 * g.sub_bytes + g.vm16 + g.km16;
+  return g;
+}
+
+int64_t blocks_for_len(const kvq_config& c, int64_t len) {
+  if (c.residual == 0) return (len + c.page - 1) / c.page;
+  return (len / c.residual) * (c.residual / c.page);
+}
+
+struct PinnedSlot {
+  int32_t* host = nullptr;
+  size_t cap = 0;   // int32 entries
+  cudaEvent_t ev = nullptr;
+  bool pending = false;
+};
+
+}  // namespace
+
+struct kvq_handle_s {
+  kvq_config cfg{};
+  kvq::Geo geo{};
+  std::vector<int32_t> len;     // stored length per sequence
+  std::vector<int32_t> table;   // [max_seqs][mbps], -1 = none
+  std::vector<int32_t> nblk;    // blocks per sequence
+  std::deque<int32_t> freelist;
+  int64_t alloc_count = 0;
+  // device
+  int device = 0;
+  uint8_t* d_pool = nullptr;
+  uint16_t* d_kres = nullptr;
+  uint16_t* d_vres = nullptr;
+  int32_t* d_table = nullptr;
+  int32_t* d_len = nullptr;
+  uint32_t* d_err = nullptr;
+  int32_t* d_plan = nullptr;
+  size_t plan_cap = 0;          // int32 entries
+  float* d_part = nullptr;
+  size_t part_bytes = 0;
+  int32_t* d_prefix = nullptr;
+  int32_t* d_seqmap = nullptr;
+  PinnedSlot slots[4];
+  int slot_next = 0;
+  int sm_count = 0;
+  int decode_ctas = 0;
+  int decode_override = 0;
+  int nstages = 0;
+  int stage_bytes = 0;
+  size_t decode_smem = 0;
+  size_t bytes_workspace = 0;
+  cudaEvent_t decode_event = nullptr;
+  int launches = 0;
+};
+
+namespace {
+
+kvq_status device_guard(kvq_handle h) {
+  if (h->cfg.host_only) return fail(KVQ_ERR_INVALID_ARG, "handle is host-only");
+  KVQ_CUDA(cudaSetDevice(h->device));
+  return KVQ_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Copies `ints` int32 values from `src` into a pinned slot and then to the
+// device buffer `dst` on `stream`.
+kvq_status stage_upload(kvq_handle h, const int32_t* src, size_t ints, int32_t* dst, cudaStream_t stream) {
+  PinnedSlot& s = h->slots[h->slot_next];
+  h->slot_next = (h->slot_next + 1) % 4;
+  if (s.pending) {
+    KVQ_CUDA(cudaEventSynchronize(s.ev));
+    s.pending = false;
+  }
+  if (s.cap < ints) {
+    if (s.host) KVQ_CUDA(cudaFreeHost(s.host));
+    s.host = nullptr;
+    s.cap = std::max(ints, size_t(1) << 16);
+    KVQ_CUDA(cudaMallocHost(&s.host, s.cap * sizeof(int32_t)));
+  }
+  std::memcpy(s.host, src, ints * sizeof(int32_t));
+  KVQ_CUDA(cudaMemcpyAsync(dst, s.host, ints * sizeof(int32_t), cudaMemcpyHostToDevice, stream));
+  KVQ_CUDA(cudaEventRecord(s.ev, stream));
+  s.pending = true;
+  return KVQ_OK;
+}
+
+kvq_status ensure_plan_capacity(kvq_handle h, size_t ints) {
+  if (ints <= h->plan_cap) return KVQ_OK;
+  // earlier launches may still read the old plan: wait for the device
+  KVQ_CUDA(cudaDeviceSynchronize());
+  if (h->d_plan) KVQ_CUDA(cudaFree(h->d_plan));
+  h->d_plan = nullptr;
+  size_t cap = std::max(ints, h->plan_cap * 2);
+  KVQ_CUDA(cudaMalloc(&h->d_plan, cap * sizeof(int32_t)));
+  h->bytes_workspace += (cap - h->plan_cap) * sizeof(int32_t);
+  h->plan_cap = cap;
+  return KVQ_OK;
+}
+
+// A plan: sections of int32 entries, uploaded as one array.
+struct Plan {
+  std::vector<int32_t> tok, flush, src, res, tab, lens, zero;
+};
+
+kvq_status run_plan(kvq_handle h, const Plan& pl, const uint16_t* k, const uint16_t* v,
+                    cudaStream_t stream) {
+  constexpr int kHeader = 0;
+  kvq::PlanView pv{};
+  pv.n_tok = int(pl.tok.size() / 3);
+  pv.n_flush = int(pl.flush.size() / kvq::kFlushEntryInts);
+  pv.n_res = int(pl.res.size() / 3);
+  pv.n_tab = int(pl.tab.size() / 2);
+  pv.n_len = int(pl.lens.size() / 2);
+  pv.n_zero = int(pl.zero.size());
+  size_t off = kHeader;
+  pv.off_tok = int(off); off += pl.tok.size();
+  pv.off_flush = int(off); off += pl.flush.size();
+  pv.off_src = int(off); off += pl.src.size();
+  pv.off_res = int(off); off += pl.res.size();
+  pv.off_tab = int(off); off += pl.tab.size();
+  pv.off_len = int(off); off += pl.lens.size();
+  pv.off_zero = int(off); off += pl.zero.size();
+  if (off == 0) return KVQ_OK;
+  std::vector<int32_t> flat;
+  flat.reserve(off);
+  for (const auto* sec : {&pl.tok, &pl.flush, &pl.src, &pl.res, &pl.tab, &pl.lens, &pl.zero})
+    flat.insert(flat.end(), sec->begin(), sec->end());
+  kvq_status st = ensure_plan_capacity(h, off);
+  if (st != KVQ_OK) return st;
+  st = stage_upload(h, flat.data(), off, h->d_plan, stream);
+  if (st != KVQ_OK) return st;
+  pv.plan = h->d_plan;
+  kvq::DevState d{h->d_pool, h->d_kres, h->d_vres, h->d_table, h->d_len, h->d_err};
+  KVQ_CUDA(kvq::launch_apply(h->geo, d, pv, stream, &h->launches));
+  KVQ_CUDA(kvq::launch_quant_token(h->geo, d, pv, k, v, stream, &h->launches));
+  KVQ_CUDA(kvq::launch_flush(h->geo, d, pv, k, v, stream, &h->launches));
+  KVQ_CUDA(kvq::launch_residual(h->geo, d, pv, k, v, stream, &h->launches));
+  return KVQ_OK;
+}
+
+void destroy_device(kvq_handle h) {
+  if (h->cfg.host_only) return;
+  cudaSetDevice(h->device);
+  cudaDeviceSynchronize();
+  cudaFree(h->d_pool);
+  cudaFree(h->d_kres);
+  cudaFree(h->d_vres);
+  cudaFree(h->d_table);
+  cudaFree(h->d_len);
+  cudaFree(h->d_err);
+  cudaFree(h->d_plan);
+  cudaFree(h->d_part);
+  cudaFree(h->d_prefix);
+  cudaFree(h->d_seqmap);
+  for (auto& s : h->slots) {
+    if (s.host) cudaFreeHost(s.host);
+    if (s.ev) cudaEventDestroy(s.ev);
+  }
+}
+
+kvq_status create_device(kvq_handle h) {
+  const kvq_config& c = h->cfg;
+  const kvq::Geo& g = h->geo;
+  h->device = c.device;
+  KVQ_CUDA(cudaSetDevice(h->device));
+  KVQ_CUDA(cudaDeviceGetAttribute(&h->sm_count, cudaDevAttrMultiProcessorCount, h->device));
+  const size_t pool = size_t(c.num_blocks) * size_t(g.block_bytes);
+  KVQ_CUDA(cudaMalloc(&h->d_pool, pool));
+  KVQ_CUDA(cudaMemset(h->d_pool, 0, pool));
+  const size_t res = std::max<size_t>(1, size_t(c.max_seqs) * c.h_kv * c.residual * c.d_h) * 2;
+  KVQ_CUDA(cudaMalloc(&h->d_kres, res));
+  KVQ_CUDA(cudaMalloc(&h->d_vres, res));
+  KVQ_CUDA(cudaMemset(h->d_kres, 0, res));
+  KVQ_CUDA(cudaMemset(h->d_vres, 0, res));
+  const size_t tab = size_t(c.max_seqs) * c.max_blocks_per_seq * sizeof(int32_t);
+  KVQ_CUDA(cudaMalloc(&h->d_table, tab));
+  KVQ_CUDA(cudaMemset(h->d_table, 0xFF, tab));
+  KVQ_CUDA(cudaMalloc(&h->d_len, size_t(c.max_seqs) * sizeof(int32_t)));
+  KVQ_CUDA(cudaMemset(h->d_len, 0, size_t(c.max_seqs) * sizeof(int32_t)));
+  KVQ_CUDA(cudaMalloc(&h->d_err, sizeof(uint32_t)));
+  KVQ_CUDA(cudaMemset(h->d_err, 0, sizeof(uint32_t)));
+  for (auto& s : h->slots) KVQ_CUDA(cudaEventCreateWithFlags(&s.ev, cudaEventDisableTiming));
+
+  // decode pipeline: per-warp ring of stages, two resident CTAs per SM if possible
+  const int res_tile = c.residual ? 2 * 16 * kvq::kD * 2 : 0;
+  h->stage_bytes = int(align_up(size_t(std::max(g.qtile_bytes, res_tile)), 128));
+  const size_t budget = 113 * 1024;
+  const size_t fixed = size_t(kvq::decode_prefix_bytes(c.max_seqs));
+  int ns = int((budget > fixed ? budget - fixed : 0) / (size_t(kvq::kDecodeWarps) * (h->stage_bytes + 8)));
+  ns = std::max(1, std::min(ns, 8));
+  size_t smem = kvq::decode_smem_bytes(c.max_seqs, ns, h->stage_bytes);
+  int max_optin = 0;
+  KVQ_CUDA(cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, h->device));
+  while (smem > size_t(max_optin) && ns > 1) smem = kvq::decode_smem_bytes(c.max_seqs, --ns, h->stage_bytes);
+  if (smem > size_t(max_optin)) return fail(KVQ_ERR_UNSUPPORTED, "decode tile does not fit in shared memory");
+  h->nstages = ns;
+  h->decode_smem = smem;
+  const void* kern = kvq::decode_kernel_ptr(g);
+  KVQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
+  int per_sm = 0;
+  KVQ_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kvq::kDecodeWarps * 32, smem));
+  if (per_sm < 1) return fail(KVQ_ERR_UNSUPPORTED, "decode kernel cannot be resident");
+  h->decode_ctas = h->sm_count * per_sm;
+
+  // workspace: split partials for up to max_seqs rows and any grid we launch
+  const int max_grid = std::max(h->decode_ctas, 4096);
+  const size_t recs = (size_t(c.max_seqs) * c.h_kv + size_t(max_grid) * kvq::kDecodeWarps) * g.G;
+  h->part_bytes = recs * (kvq::kD + 2) * sizeof(float);
+  KVQ_CUDA(cudaMalloc(&h->d_part, h->part_bytes));
+  KVQ_CUDA(cudaMalloc(&h->d_prefix, size_t(c.max_seqs + 1) * sizeof(int32_t)));
+  KVQ_CUDA(cudaMalloc(&h->d_seqmap, size_t(c.max_seqs) * sizeof(int32_t)));
+  h->bytes_workspace = h->part_bytes + size_t(c.max_seqs + 1) * 4 + size_t(c.max_seqs) * 4 + 4;
+  return ensure_plan_capacity(h, size_t(1) << 16);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* kvq_last_error(void) { return g_last_error.c_str(); }
+
+kvq_status kvq_layout(const kvq_config* cfg, kvq_layout_info* out) {
+  kvq_status st = validate(cfg);
+  if (st != KVQ_OK) return st;
+  if (!out) return fail(KVQ_ERR_INVALID_ARG, "out is null");
+  const kvq::Geo g = make_geo(*cfg);
+  out->row_bytes = uint64_t(g.row_bytes);
+  out->sub_bytes = uint64_t(g.sub_bytes);
+  out->off_v = uint64_t(g.off_V);
+  out->off_vmeta = uint64_t(g.off_Vm);
+  out->off_kmeta = uint64_t(g.off_Km);
+  out->chunk_bytes = uint64_t(g.chunk_bytes);
+  out->block_bytes = uint64_t(g.block_bytes);
+  out->kslice = uint64_t(g.kslice);
+  return KVQ_OK;
+}
+
+uint64_t kvq_cache_bytes(int32_t layers, int64_t tokens, int32_t h_kv, int32_t d_h, const kvq_config* cfg) {
+  if (!cfg || layers < 0 || tokens < 0 || h_kv < 0 || d_h < 0) return 0;
+  if (cfg->bits != 2 && cfg->bits != 4 && cfg->bits != 8) return 0;
+  if (cfg->g_k <= 0 || cfg->g_v <= 0) return 0;
+  // M = 2 L T H_kv d_h b: codes for K and V, plus per-group metadata
+  const uint64_t elems = uint64_t(layers) * uint64_t(tokens) * uint64_t(h_kv) * uint64_t(d_h);
+  const uint64_t meta = uint64_t(cfg->scale_fp32 ? 4 : 2) * uint64_t(1 + cfg->asym);
+  const uint64_t codes = 2 * elems * uint64_t(cfg->bits) / 8;
+  const uint64_t kmeta = (elems * meta + uint64_t(cfg->g_k) - 1) / uint64_t(cfg->g_k);
+  const uint64_t vmeta = (elems * meta + uint64_t(cfg->g_v) - 1) / uint64_t(cfg->g_v);
+  return codes + kmeta + vmeta;
+}
+
+kvq_status kvq_create(const kvq_config* cfg, kvq_handle* out) {
+  if (!out) return fail(KVQ_ERR_INVALID_ARG, "out is null");
+  *out = nullptr;
+  kvq_status st = validate(cfg);
+  if (st != KVQ_OK) return st;
+  kvq_handle h = new kvq_handle_s();
+  h->cfg = *cfg;
+  h->geo = make_geo(*cfg);
+  h->len.assign(size_t(cfg->max_seqs), 0);
+  h->nblk.assign(size_t(cfg->max_seqs), 0);
+  h->table.assign(size_t(cfg->max_seqs) * cfg->max_blocks_per_seq, -1);
+  // free list: Fisher-Yates over [0, num_blocks) driven by splitmix64(seed)
+  std::vector<int32_t> perm(size_t(cfg->num_blocks));
+  for (int32_t i = 0; i < cfg->num_blocks; ++i) perm[size_t(i)] = i;
+  uint64_t sm = cfg->seed;
+  for (int32_t i = cfg->num_blocks - 1; i >= 1; --i) {
+    const uint64_t j = splitmix64(sm) % uint64_t(i + 1);
+    std::swap(perm[size_t(i)], perm[size_t(j)]);
+  }
+  h->freelist.assign(perm.begin(), perm.end());
+  if (!cfg->host_only) {
+    st = create_device(h);
+    if (st != KVQ_OK) {
+      const std::string msg = g_last_error;
+      destroy_device(h);
+      delete h;
+      return fail(st, msg);
+    }
+  }
+  *out = h;
+  return KVQ_OK;
+}
+
+void kvq_destroy(kvq_handle h) {
+  if (!h) return;
+  destroy_device(h);
+  delete h;
+}
+
+kvq_status kvq_append(kvq_handle h, const void* k_bf16, const void* v_bf16, const int32_t* seq_ids_host,
+                      int32_t n, void* stream_) {
+  if (!h) return fail(KVQ_ERR_INVALID_ARG, "handle is null");
+  if (n < 0) return fail(KVQ_ERR_INVALID_ARG, "n must be >= 0");
+  if (n == 0) return KVQ_OK;
+  if (!seq_ids_host) return fail(KVQ_ERR_INVALID_ARG, "seq_ids_host is null");
+  if (!h->cfg.host_only) {
+    if (!k_bf16 || !v_bf16) return fail(KVQ_ERR_INVALID_ARG, "k/v pointer is null");
+    if (!aligned16(k_bf16) || !aligned16(v_bf16)) return fail(KVQ_ERR_INVALID_ARG, "k/v must be 16-byte aligned");
+  }
+  const kvq_config& c = h->cfg;
+  const int S = c.max_seqs, R = c.residual, P = c.page, MB = c.max_blocks_per_seq;
+
+  // ---- admission (no state change on failure) ----------------------------
+  std::vector<int64_t> newlen(h->len.begin(), h->len.end());
+  for (int32_t i = 0; i < n; ++i) {
+    const int32_t s = seq_ids_host[i];
+    if (s < 0 || s >= S) return fail(KVQ_ERR_BAD_SEQ, "sequence id " + std::to_string(s) + " out of range");
+    ++newlen[size_t(s)];
+  }
+  int64_t need = 0;
+  for (int s = 0; s < S; ++s) {
+    if (newlen[size_t(s)] == h->len[size_t(s)]) continue;
+    if (newlen[size_t(s)] > INT32_MAX / 2) return fail(KVQ_ERR_INVALID_ARG, "sequence too long");
+    const int64_t nb = blocks_for_len(c, newlen[size_t(s)]);
+    if (nb > MB) return fail(KVQ_ERR_OOM, "block-table row of sequence " + std::to_string(s) + " is full");
+    need += nb - h->nblk[size_t(s)];
+  }
+  if (need > int64_t(h->freelist.size())) return fail(KVQ_ERR_OOM, "out of free blocks");
+  if (c.fail_alloc_after >= 0 && h->alloc_count + need > c.fail_alloc_after)
+    return fail(KVQ_ERR_OOM, "allocation refused by fail_alloc_after");
+
+  // ---- plan (state is committed below, after the plan is complete) --------
+  Plan pl;
+  std::vector<int32_t> first(h->len.begin(), h->len.end());   // length before the call
+  std::vector<int32_t> cur(first);
+  std::vector<int32_t> nblk(h->nblk);
+  std::vector<int32_t> tbl(h->table);                           // table after the call
+  std::vector<std::pair<int32_t, int32_t>> tab_changes;        // (index, block)
+  std::vector<std::vector<int32_t>> arrivals(static_cast<size_t>(S));  // input rows per sequence
+  int64_t allocs = 0;
+  auto take = [&]() { return h->freelist[size_t(allocs++)]; };  // front of the free list, in order
+  for (int32_t i = 0; i < n; ++i) {
+    const int32_t s = seq_ids_host[i];
+    const int32_t pos = cur[size_t(s)]++;
+    if (R == 0) {
+      const int32_t lb = pos / P;
+      if (lb == nblk[size_t(s)]) {
+        const int32_t b = take();
+        tab_changes.push_back({s * MB + lb, b});
+        tbl[size_t(s) * MB + lb] = b;
+        ++nblk[size_t(s)];
+        if (newlen[size_t(s)] < int64_t(lb + 1) * P) pl.zero.push_back(b);
+      }
+      pl.tok.insert(pl.tok.end(), {i, tbl[size_t(s) * MB + lb], pos % P});
+    } else {
+      arrivals[size_t(s)].push_back(i);
+      if (pos % R == R - 1) {
+        const int32_t grp = pos / R, npg = R / P;
+        std::vector<int32_t> ent = {s, grp, npg};
+        for (int j = 0; j < npg; ++j) {
+          const int32_t b = take();
+          tab_changes.push_back({s * MB + nblk[size_t(s)], b});
+          tbl[size_t(s) * MB + nblk[size_t(s)]] = b;
+          ++nblk[size_t(s)];
+          ent.push_back(b);
+        }
+        ent.resize(kvq::kFlushEntryInts, -1);
+        pl.flush.insert(pl.flush.end(), ent.begin(), ent.end());
+        for (int r = 0; r < R; ++r) {
+          const int32_t p = grp * R + r;
+          pl.src.push_back(p < first[size_t(s)] ? -1 - (p % R)
+                                                : arrivals[size_t(s)][size_t(p - first[size_t(s)])]);
+        }
+      }
+    }
+  }
+  if (R > 0) {
+    for (int s = 0; s < S; ++s) {
+      const int32_t L = cur[size_t(s)];
+      if (L == first[size_t(s)]) continue;
+      const int32_t lo = std::max(first[size_t(s)], (L / R) * R);
+      for (int32_t p = lo; p < L; ++p)
+        pl.res.insert(pl.res.end(), {arrivals[size_t(s)][size_t(p - first[size_t(s)])], s, p % R});
+    }
+  }
+  for (const auto& tc : tab_changes) pl.tab.insert(pl.tab.end(), {tc.first, tc.second});
+  for (int s = 0; s < S; ++s)
+    if (cur[size_t(s)] != first[size_t(s)]) pl.lens.insert(pl.lens.end(), {s, cur[size_t(s)]});
+
+  if (!c.host_only) {
+    kvq_status st = device_guard(h);
+    if (st != KVQ_OK) return st;
+    st = run_plan(h, pl, static_cast<const uint16_t*>(k_bf16), static_cast<const uint16_t*>(v_bf16),
+                  static_cast<cudaStream_t>(stream_));
+    if (st != KVQ_OK) return st;
+  }
+  // ---- commit host state -----------------------------------------------------
+  h->table.swap(tbl);
+  h->nblk = nblk;
+  h->freelist.erase(h->freelist.begin(), h->freelist.begin() + allocs);
+  h->alloc_count += allocs;
+  for (int s = 0; s < S; ++s) h->len[size_t(s)] = cur[size_t(s)];
+  return KVQ_OK;
+}
+
+kvq_status kvq_decode_attn(kvq_handle h, const void* q_bf16, const int32_t* block_table, int32_t bt_stride,
+                           const int32_t* seq_lens, const int32_t* seq_ids_host, int32_t batch, float* out,
+                           void* stream_) {
+  if (!h) return fail(KVQ_ERR_INVALID_ARG, "handle is null");
+  if (batch < 0) return fail(KVQ_ERR_INVALID_ARG, "batch must be >= 0");
+  if (batch == 0) return KVQ_OK;
+  if (batch > h->cfg.max_seqs) return fail(KVQ_ERR_INVALID_ARG, "batch exceeds max_seqs");
+  kvq_status st = device_guard(h);
+  if (st != KVQ_OK) return st;
+  if (!q_bf16 || !seq_lens || !out) return fail(KVQ_ERR_INVALID_ARG, "q, seq_lens and out are required");
+  if (!aligned16(q_bf16) || !aligned16(out)) return fail(KVQ_ERR_INVALID_ARG, "q/out must be 16-byte aligned");
+  if (block_table && bt_stride < 1) return fail(KVQ_ERR_INVALID_ARG, "bt_stride must be >= 1");
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  const int32_t* seqmap = nullptr;
+  if (seq_ids_host) {
+    for (int32_t i = 0; i < batch; ++i)
+      if (seq_ids_host[i] < 0 || seq_ids_host[i] >= h->cfg.max_seqs)
+        return fail(KVQ_ERR_BAD_SEQ, "sequence id " + std::to_string(seq_ids_host[i]) + " out of range");
+    st = stage_upload(h, seq_ids_host, size_t(batch), h->d_seqmap, stream);
+    if (st != KVQ_OK) return st;
+    seqmap = h->d_seqmap;
+  }
+  kvq::DecodeArgs a{};
+  a.pool = h->d_pool;
+  a.kres = h->d_kres;
+  a.vres = h->d_vres;
+  a.table = block_table ? block_table : h->d_table;
+  a.table_stride = block_table ? bt_stride : h->cfg.max_blocks_per_seq;
+  a.table_by_seq = block_table ? 0 : 1;
+  a.seq_lens = seq_lens;
+  a.seqmap = seqmap;
+  a.stored_len = h->d_len;
+  a.q = static_cast<const uint16_t*>(q_bf16);
+  a.out = out;
+  a.partials = h->d_part;
+  a.prefix = h->d_prefix;
+  a.err = h->d_err;
+  a.B = batch;
+  a.nstages = h->nstages;
+  a.stage_bytes = h->stage_bytes;
+  a.pre_bytes = kvq::decode_prefix_bytes(batch);
+  const int grid = h->decode_override > 0 ? h->decode_override : h->decode_ctas;
+  a.nw = grid * kvq::kDecodeWarps;
+  a.qk_scale = float(1.4426950408889634 / std::sqrt(double(kvq::kD)));
+  a.g = h->geo;
+  const size_t smem = kvq::decode_smem_bytes(batch, h->nstages, h->stage_bytes);
+  KVQ_CUDA(kvq::launch_decode(a, grid, smem, stream, h->decode_event, &h->launches));
+  return KVQ_OK;
+}
+
+kvq_status kvq_block_table(kvq_handle h, const int32_t** dev_ptr, int32_t* stride) {
+  if (!h || !dev_ptr || !stride) return fail(KVQ_ERR_INVALID_ARG, "null argument");
+  *dev_ptr = h->d_table;
+  *stride = h->cfg.max_blocks_per_seq;
+  return KVQ_OK;
+}
+
+kvq_status kvq_block_table_host(kvq_handle h, int32_t seq, int32_t* dst, int32_t max_entries,
+                                int32_t* n_entries) {
+  if (!h || !n_entries) return fail(KVQ_ERR_INVALID_ARG, "null argument");
+  if (seq < 0 || seq >= h->cfg.max_seqs) return fail(KVQ_ERR_BAD_SEQ, "sequence id out of range");
+  const int32_t nb = h->nblk[size_t(seq)];
+  *n_entries = nb;
+  for (int32_t j = 0; dst && j < std::min(nb, max_entries); ++j)
+    dst[j] = h->table[size_t(seq) * h->cfg.max_blocks_per_seq + j];
+  return KVQ_OK;
+}
+
+kvq_status kvq_seq_len(kvq_handle h, int32_t seq, int32_t* len) {
+  if (!h || !len) return fail(KVQ_ERR_INVALID_ARG, "null argument");
+  if (seq < 0 || seq >= h->cfg.max_seqs) return fail(KVQ_ERR_BAD_SEQ, "sequence id out of range");
+  *len = h->len[size_t(seq)];
+  return KVQ_OK;
+}
+
+kvq_status kvq_seq_lens_device(kvq_handle h, const int32_t** dev_ptr) {
+  if (!h || !dev_ptr) return fail(KVQ_ERR_INVALID_ARG, "null argument");
+  *dev_ptr = h->d_len;
+  return KVQ_OK;
+}
+
+kvq_status kvq_free_seq(kvq_handle h, int32_t seq, void* stream_) {
+  if (!h) return fail(KVQ_ERR_INVALID_ARG, "handle is null");
+  if (seq < 0 || seq >= h->cfg.max_seqs) return fail(KVQ_ERR_BAD_SEQ, "sequence id out of range");
+  const int MB = h->cfg.max_blocks_per_seq;
+  Plan pl;
+  for (int32_t j = 0; j < h->nblk[size_t(seq)]; ++j) pl.tab.insert(pl.tab.end(), {seq * MB + j, -1});
+  pl.lens.insert(pl.lens.end(), {seq, 0});
+  if (!h->cfg.host_only) {
+    kvq_status st = device_guard(h);
+    if (st != KVQ_OK) return st;
+    st = run_plan(h, pl, nullptr, nullptr, static_cast<cudaStream_t>(stream_));
+    if (st != KVQ_OK) return st;
+  }
+  for (int32_t j = 0; j < h->nblk[size_t(seq)]; ++j) {
+    int32_t& e = h->table[size_t(seq) * MB + j];
+    h->freelist.push_back(e);
+    e = -1;
+  }
+  h->nblk[size_t(seq)] = 0;
+  h->len[size_t(seq)] = 0;
+  return KVQ_OK;
+}
+
+kvq_status kvq_stats(kvq_handle h, kvq_stats_t* out) {
+  if (!h || !out) return fail(KVQ_ERR_INVALID_ARG, "null argument");
+  const kvq_config& c = h->cfg;
+  uint64_t tokens = 0;
+  for (int32_t L : h->len) tokens += uint64_t(L);
+  out->blocks_free = h->freelist.size();
+  out->blocks_used = uint64_t(c.num_blocks) - out->blocks_free;
+  out->tokens_stored = tokens;
+  out->bytes_pool = c.host_only ? 0 : uint64_t(c.num_blocks) * uint64_t(h->geo.block_bytes);
+  out->bytes_residual = c.host_only ? 0 : 2ull * c.max_seqs * c.h_kv * c.residual * c.d_h * 2;
+  out->bytes_workspace = c.host_only ? 0 : h->bytes_workspace;
+  out->bytes_formula = kvq_cache_bytes(1, int64_t(tokens), c.h_kv, c.d_h, &c);
+  out->kernel_launches = uint64_t(h->launches);
+  return KVQ_OK;
+}
+
+kvq_status kvq_read_pool(kvq_handle h, void* host_dst, uint64_t bytes, void* stream_) {
+  if (!h || !host_dst) return fail(KVQ_ERR_INVALID_ARG, "null argument");
+  kvq_status st = device_guard(h);
+  if (st != KVQ_OK) return st;
+  const uint64_t total = uint64_t(h->cfg.num_blocks) * uint64_t(h->geo.block_bytes);
+  if (bytes != total) return fail(KVQ_ERR_INVALID_ARG, "bytes must equal num_blocks * block_bytes");
+  cudaStream_t s = static_cast<cudaStream_t>(stream_);
+  KVQ_CUDA(cudaMemcpyAsync(host_dst, h->d_pool, total, cudaMemcpyDeviceToHost, s));
+  KVQ_CUDA(cudaStreamSynchronize(s));
+  return KVQ_OK;
+}
+
+kvq_status kvq_read_residual(kvq_handle h, void* k_host, void* v_host, uint64_t bytes, void* stream_) {
+  if (!h || !k_host || !v_host) return fail(KVQ_ERR_INVALID_ARG, "null argument");
+  kvq_status st = device_guard(h);
+  if (st != KVQ_OK) return st;
+  const kvq_config& c = h->cfg;
+  const uint64_t total = uint64_t(c.max_seqs) * c.h_kv * c.residual * c.d_h * 2;
+  if (bytes != total) return fail(KVQ_ERR_INVALID_ARG, "bytes must equal max_seqs * h_kv * residual * d_h * 2");
+  if (total == 0) return KVQ_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream_);
+  KVQ_CUDA(cudaMemcpyAsync(k_host, h->d_kres, total, cudaMemcpyDeviceToHost, s));
+  KVQ_CUDA(cudaMemcpyAsync(v_host, h->d_vres, total, cudaMemcpyDeviceToHost, s));
+  KVQ_CUDA(cudaStreamSynchronize(s));
+  return KVQ_OK;
+}
+
+kvq_status kvq_sync_status(kvq_handle h, void* stream_, uint32_t* bits_out) {
+  if (!h) return fail(KVQ_ERR_INVALID_ARG, "handle is null");
+  kvq_status st = device_guard(h);
+  if (st != KVQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream_);
+  KVQ_CUDA(cudaStreamSynchronize(s));
+  KVQ_CUDA(cudaGetLastError());
+  uint32_t bits = 0;
+  KVQ_CUDA(cudaMemcpy(&bits, h->d_err, sizeof(bits), cudaMemcpyDeviceToHost));
+  KVQ_CUDA(cudaMemset(h->d_err, 0, sizeof(uint32_t)));
+  if (bits_out) *bits_out = bits;
+  if (bits) {
+    char buf[96];
+    std::snprintf(buf, sizeof(buf), "device check fired: error bits 0x%x", bits);
+    return fail(KVQ_ERR_DEVICE_CHECK, buf);
+  }
+  return KVQ_OK;
+}
+
+kvq_status kvq_set_decode_event(kvq_handle h, void* event) {
+  if (!h) return fail(KVQ_ERR_INVALID_ARG, "handle is null");
+  h->decode_event = static_cast<cudaEvent_t>(event);
+  return KVQ_OK;
+}
+
+kvq_status kvq_set_decode_grid(kvq_handle h, int32_t ctas) {
+  if (!h) return fail(KVQ_ERR_INVALID_ARG, "handle is null");
+  if (ctas < 0 || ctas > 4096) return fail(KVQ_ERR_INVALID_ARG, "ctas must be in [0, 4096]");
+  h->decode_override = ctas;
+  return KVQ_OK;
+}
+
+}  // extern "C"

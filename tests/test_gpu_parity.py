@@ -1,0 +1,242 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle on the
+same seeded inputs.  Codes, scales, zero-points, packing and block placement
+must match bit for bit (the whole pool, the live residual slots and the block
+tables); attention output must be within 2e-3 (max abs) of the oracle's fp64
+attention over the same dequantized cache."""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from quantized_kv_cache_14_b200 import build as kbuild
+from quantized_kv_cache_14_b200.workloads import Draws, random_bf16, workload
+from tests.gpu_util import ATOL, Pair, bits_to_cuda_bf16
+
+pytestmark = pytest.mark.gpu
+
+D = 128
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    kbuild.build()
+
+
+FMTS = {
+    "int8_tok_p16": dict(bits=8, asym=0, k_axis=0, g_k=128, g_v=128, scale_fp32=0, residual=0, page=16),
+    "int8_tok_p512_fp32": dict(bits=8, asym=0, k_axis=0, g_k=128, g_v=128, scale_fp32=1, residual=0, page=512),
+    "int4_chan64": dict(bits=4, asym=0, k_axis=1, g_k=64, g_v=64, scale_fp32=0, residual=64, page=16),
+    "int2_asym_chan32": dict(bits=2, asym=1, k_axis=1, g_k=32, g_v=32, scale_fp32=0, residual=32, page=16),
+    "int4_chan64_p32_gv32": dict(bits=4, asym=0, k_axis=1, g_k=64, g_v=32, scale_fp32=0, residual=64, page=32),
+    "int4_asym_tok32": dict(bits=4, asym=1, k_axis=0, g_k=32, g_v=32, scale_fp32=0, residual=0, page=32),
+    "int8_asym_chan128_p64": dict(bits=8, asym=1, k_axis=1, g_k=128, g_v=128, scale_fp32=0, residual=128, page=64),
+    "int2_sym_tok64_fp32": dict(bits=2, asym=0, k_axis=0, g_k=64, g_v=64, scale_fp32=1, residual=0, page=16),
+    "int4_chan16": dict(bits=4, asym=0, k_axis=1, g_k=16, g_v=128, scale_fp32=0, residual=16, page=16),
+}
+
+
+def outlier_keys(rng, n, h_kv, gain=20.0):
+    k = rng.standard_normal((n, h_kv, D), dtype=np.float32)
+    k[:, :, 3] *= gain
+    k[:, :, 77] *= gain
+    from quantized_kv_cache_14_b200.workloads import to_bf16_bits
+    return to_bf16_bits(k)
+
+
+@pytest.mark.parametrize("name", list(FMTS))
+@pytest.mark.parametrize("lens", [[1], [15, 16, 17], [63, 64, 65], [200, 1, 129], [0, 31, 33]])
+def test_small_bulk_append_and_decode(name, lens):
+    rng = np.random.default_rng(sum(lens) + len(name))
+    h_q, h_kv = 8, 2
+    p = Pair(FMTS[name], h_q, h_kv, max_seqs=3, num_blocks=120, mbps=64, seed=5)
+    ids = np.repeat(np.arange(len(lens), dtype=np.int32), lens)
+    n = int(ids.size)
+    if n:
+        p.append(outlier_keys(rng, n, h_kv), random_bf16(rng, (n, h_kv, D)), ids)
+    p.check_state()
+    q = random_bf16(rng, (len(lens), h_q, D))
+    p.check_decode(q, lens)
+    p.close()
+
+
+@pytest.mark.parametrize("name", list(FMTS))
+def test_incremental_appends_interleaved(name):
+    """Appends of random sizes to interleaved sequences equal the oracle's
+    one-token-at-a-time definition, with decode checked along the way."""
+    rng = np.random.default_rng(7)
+    h_q, h_kv = 4, 1
+    p = Pair(FMTS[name], h_q, h_kv, max_seqs=3, num_blocks=300, mbps=128, seed=9)
+    lens = [0, 0, 0]
+    for step in range(14):
+        n = int(rng.integers(1, 70))
+        ids = rng.integers(0, 3, size=n).astype(np.int32)
+        p.append(outlier_keys(rng, n, h_kv), random_bf16(rng, (n, h_kv, D)), ids)
+        for s in ids:
+            lens[int(s)] += 1
+        if step % 4 == 3:
+            p.check_state()
+            p.check_decode(random_bf16(rng, (3, h_q, D)), lens)
+    p.check_state()
+    p.close()
+
+
+@pytest.mark.parametrize("name", ["int4_chan64", "int8_tok_p16", "int2_asym_chan32"])
+def test_split_k_merge_is_invariant_to_grid(name):
+    rng = np.random.default_rng(3)
+    h_q, h_kv = 16, 4
+    p = Pair(FMTS[name], h_q, h_kv, max_seqs=4, num_blocks=900, mbps=256, seed=1)
+    lens = [1500, 3, 640, 999]
+    ids = np.repeat(np.arange(4, dtype=np.int32), lens)
+    n = int(ids.size)
+    p.append(outlier_keys(rng, n, h_kv), random_bf16(rng, (n, h_kv, D)), ids)
+    q = random_bf16(rng, (4, h_q, D))
+    outs = []
+    for grid in (0, 1, 2, 7, 64, 1000):
+        p.gpu.set_decode_grid(grid)
+        got, want = p.decode(q, lens)
+        assert np.max(np.abs(got - want)) <= ATOL, grid
+        outs.append(got)
+    for o in outs[1:]:
+        assert np.max(np.abs(o - outs[0])) <= 1e-4
+    p.close()
+
+
+def test_prefix_lengths_empty_rows_and_seq_map():
+    rng = np.random.default_rng(4)
+    fmt = FMTS["int4_chan64"]
+    h_q, h_kv = 8, 2
+    p = Pair(fmt, h_q, h_kv, max_seqs=4, num_blocks=200, mbps=64, seed=2)
+    lens = [300, 64, 129, 0]
+    ids = np.repeat(np.arange(4, dtype=np.int32), lens)
+    n = int(ids.size)
+    p.append(outlier_keys(rng, n, h_kv), random_bf16(rng, (n, h_kv, D)), ids)
+    q = random_bf16(rng, (4, h_q, D))
+    # attend to prefixes (inside quantized groups and inside the window)
+    p.check_decode(q, [250, 64, 100, 0])
+    p.check_decode(q, [1, 0, 129, 0])
+    # rows mapped to other sequences, repeated
+    seq_ids = np.array([2, 2, 0, 1], np.int32)
+    p.check_decode(q, [129, 65, 300, 64], seq_ids=seq_ids)
+    p.close()
+
+
+def test_caller_block_table():
+    rng = np.random.default_rng(5)
+    fmt = FMTS["int8_tok_p16"]
+    h_q, h_kv = 4, 1
+    p = Pair(fmt, h_q, h_kv, max_seqs=3, num_blocks=100, mbps=40, seed=2)
+    lens = [100, 37, 250]
+    ids = np.repeat(np.arange(3, dtype=np.int32), lens)
+    n = int(ids.size)
+    p.append(outlier_keys(rng, n, h_kv), random_bf16(rng, (n, h_kv, D)), ids)
+    # batch rows (2, 0): a caller-built table of those rows, stride 20
+    rows = [2, 0]
+    bt = np.full((2, 20), -1, np.int32)
+    for r, s in enumerate(rows):
+        t = p.orc.block_table(s)
+        bt[r, :len(t)] = t
+    q = random_bf16(rng, (2, h_q, D))
+    got, want = p.decode(q, [lens[2], lens[0]], seq_ids=np.array(rows, np.int32),
+                         block_table=torch.tensor(bt, device="cuda"), bt_stride=20)
+    assert np.max(np.abs(got - want)) <= ATOL
+    p.close()
+
+
+def test_free_and_reuse_blocks():
+    rng = np.random.default_rng(6)
+    fmt = FMTS["int4_chan64"]
+    p = Pair(fmt, 4, 1, max_seqs=3, num_blocks=40, mbps=40, seed=8)
+    for s, L in ((0, 130), (1, 70)):
+        p.append(outlier_keys(rng, L, 1), random_bf16(rng, (L, 1, D)), np.full(L, s, np.int32))
+    p.check_state()
+    p.gpu.free_seq(0)
+    assert p.orc.free_seq(0) == 0
+    p.append(outlier_keys(rng, 200, 1), random_bf16(rng, (200, 1, D)), np.full(200, 2, np.int32))
+    p.check_state()
+    p.check_decode(random_bf16(rng, (3, 4, D)), [0, 70, 200])
+    p.close()
+
+
+def test_device_check_flags_bad_lengths():
+    rng = np.random.default_rng(2)
+    fmt = FMTS["int4_chan64"]
+    p = Pair(fmt, 4, 1, max_seqs=2, num_blocks=20, mbps=20, seed=1)
+    p.append(outlier_keys(rng, 80, 1), random_bf16(rng, (80, 1, D)), np.zeros(80, np.int32))
+    q = bits_to_cuda_bf16(random_bf16(rng, (2, 4, D)))
+    sl = torch.tensor([500, -3], dtype=torch.int32, device="cuda")   # beyond the stored length
+    out = torch.zeros((2, 4, D), dtype=torch.float32, device="cuda")
+    p.gpu.decode(q, sl, out)
+    from quantized_kv_cache_14_b200 import kvq
+    bits = p.gpu.sync_status()
+    assert bits & kvq.KVQ_DEVERR_SEQ_LEN
+    assert p.gpu.sync_status() == 0        # cleared
+    p.close()
+
+
+# ----------------------------------------------------------- full workloads
+
+def pool_blocks(lengths, growth, page, residual):
+    return int(sum((L + growth + page - 1) // page for L in lengths)) + 64
+
+
+def run_full(idx, steps_checked=(), max_steps=0, check_every_pool=False):
+    w = workload(idx)
+    dr = Draws(w, steps=max_steps)
+    f = w.fmt
+    fmt = dict(bits=f.bits, asym=f.asym, k_axis=f.k_axis, g_k=f.g_k, g_v=f.g_v,
+               scale_fp32=f.scale_fp32, residual=f.residual, page=f.page)
+    nb = pool_blocks(dr.lengths, max_steps, f.page, f.residual)
+    mbps = max((L + max_steps) // f.page + 2 for L in dr.lengths)
+    p = Pair(fmt, w.h_q, w.h_kv, max_seqs=w.batch, num_blocks=nb, mbps=mbps, seed=w.seed)
+    p.append(dr.k, dr.v, dr.seq_ids)
+    p.check_state()
+    lens = list(dr.lengths)
+    errs = [p.check_decode(dr.q, lens, nthreads=os.cpu_count() or 8)]
+    for step in range(max_steps):
+        k, v, q = dr.step()
+        p.append(k, v, np.arange(w.batch, dtype=np.int32))
+        lens = [L + 1 for L in lens]
+        if step in steps_checked:
+            p.check_state(pool=check_every_pool or step in (0, max_steps - 1))
+            errs.append(p.check_decode(q, lens, nthreads=os.cpu_count() or 8))
+    p.close()
+    return errs
+
+
+def test_workload_1_tiny_int8():
+    run_full(1)
+
+
+def test_workload_2_int8_paged_gqa():
+    run_full(2)
+
+
+def test_workload_3_int4_kivi():
+    run_full(3)
+
+
+def test_workload_4_int2_asym_long_context():
+    run_full(4)
+
+
+def test_workload_4_without_residual_tail():
+    w = workload(4)
+    dr = Draws(w, length_override=[131072])
+    f = w.fmt
+    fmt = dict(bits=f.bits, asym=f.asym, k_axis=f.k_axis, g_k=f.g_k, g_v=f.g_v,
+               scale_fp32=f.scale_fp32, residual=f.residual, page=f.page)
+    p = Pair(fmt, w.h_q, w.h_kv, max_seqs=1, num_blocks=131072 // 16 + 64, mbps=131072 // 16 + 4,
+             seed=w.seed)
+    p.append(dr.k, dr.v, dr.seq_ids)
+    p.check_state(pool=False)
+    p.check_decode(dr.q, [131072], nthreads=os.cpu_count() or 8)
+    p.close()
+
+
+def test_workload_5_continuous_batching():
+    steps = int(os.environ.get("KVQ_CB_STEPS", "100"))
+    checked = set(range(steps)) if os.environ.get("KVQ_CB_FULL") else {0, 1, 2, 49, 98, 99}
+    run_full(5, steps_checked={s for s in checked if s < steps}, max_steps=steps)
