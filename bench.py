@@ -245,6 +245,9 @@ def run_gpu(args, rank, ws, dist):
     out_host = torch.empty_like(out, device="cpu").pin_memory()
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     ev_mid = torch.cuda.Event(enable_timing=True)
+    ev_mid.record()               # torch creates the CUDA event on its first record
+    torch.cuda.synchronize()
+    assert ev_mid.cuda_event != 0
     cache.set_decode_event(ev_mid)
     torch.cuda.synchronize()
     assert cache.sync_status() == 0
@@ -392,7 +395,7 @@ def workload_config(w, lens):
         "format": f"{kind}, keys {axis} G={f.g_k}, values per-token G={f.g_v}, "
                   f"{'fp32' if f.scale_fp32 else 'fp16'} scales, page {f.page}, BF16 window {f.residual}",
         "batch": w.batch, "h_q": w.h_q, "h_kv": w.h_kv, "d_h": D,
-        "seq_len_start": int(min(lens)), "seq_len_max": int(max(lens)),
+        "seq_len_min": int(min(lens)), "seq_len_max": int(max(lens)),
         "l2": "flushed before every timed step (256 MB write, untimed)",
         "step": "append 1 token per sequence (quantize/window/flush) + decode attention",
         "parallelism": "replicas",

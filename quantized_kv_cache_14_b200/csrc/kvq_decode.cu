@@ -446,8 +446,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const __grid_
     }
   };
 
+  bool bq_holds_q = false;    // bq currently carries q itself (token axis, BF16 window)
   auto setup_pair = [&](int row, int h) {
     state_reset(st);
+    bq_holds_q = !KAXIS;
     float qv[32];
     load_q(row, h, qv);
     if (KAXIS) {
@@ -508,6 +510,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const __grid_
           }
         }
         make_bq(xq);
+        bq_holds_q = false;
         if (ASYM) {
           zdot += __shfl_xor_sync(0xffffffffu, zdot, 1);
           zdot += __shfl_xor_sync(0xffffffffu, zdot, 2);
@@ -593,11 +596,12 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const __grid_
       }
     } else {
       // ------------------------- BF16 residual tile -------------------------
-      if (cit.k == cri.nq) {
+      if (!bq_holds_q) {
         // B operand of q itself (exact in bf16: lo columns are zero)
         float qv[32];
         load_q(cit.i, cit.h, qv);
         make_bq(qv);
+        bq_holds_q = true;
       }
       const uint32_t kaddr = smem_addr(stg), vaddr = kaddr + 16 * D * 2;
       float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
@@ -673,16 +677,27 @@ __global__ void __launch_bounds__(128) reduce_kernel(const __grid_constant__ Dec
       *out = 0.0f;
       continue;
     }
+    // warps whose ranges hold this pair's tiles: start at the owner of its
+    // first tile and jump from range end to range end (warps with empty
+    // ranges in between own nothing and wrote nothing)
     const int64_t ua = int64_t(pre[i]) * g.h_kv + int64_t(h) * n, ub = ua + n - 1;
     const int64_t w0 = ((ua + 1) * a.nw - 1) / U, w1 = ((ub + 1) * a.nw - 1) / U;
+    auto next_warp = [&](int64_t w) {
+      const int64_t end = ((w + 1) * U) / a.nw;     // first tile after warp w's range
+      return ((end + 1) * a.nw - 1) / U;
+    };
     float M = -INFINITY;
-    for (int64_t w = w0; w <= w1; ++w) M = fmaxf(M, a.partials[((p + w) * g.G + hd) * (D + 2)]);
+    for (int64_t w = w0;; w = next_warp(w)) {
+      M = fmaxf(M, a.partials[((p + w) * g.G + hd) * (D + 2)]);
+      if (w >= w1) break;
+    }
     float num = 0.0f, den = 0.0f;
-    for (int64_t w = w0; w <= w1; ++w) {
+    for (int64_t w = w0;; w = next_warp(w)) {
       const float* rec = a.partials + ((p + w) * g.G + hd) * (D + 2);
       const float sc = fast_exp2(rec[0] - M);
       den = fmaf(sc, rec[1], den);
       num = fmaf(sc, rec[2 + c], num);
+      if (w >= w1) break;
     }
     *out = num / den;
   }

@@ -323,6 +323,8 @@ kvq_status create_device(kvq_handle h) {
   const size_t recs = (size_t(c.max_seqs) * c.h_kv + size_t(max_grid) * kvq::kDecodeWarps) * g.G;
   h->part_bytes = recs * (kvq::kD + 2) * sizeof(float);
   KVQ_CUDA(cudaMalloc(&h->d_part, h->part_bytes));
+  // NaN-fill: a merge that ever read a slot no warp wrote shows up as NaN
+  KVQ_CUDA(cudaMemset(h->d_part, 0xFF, h->part_bytes));
   KVQ_CUDA(cudaMalloc(&h->d_prefix, size_t(c.max_seqs + 1) * sizeof(int32_t)));
   KVQ_CUDA(cudaMalloc(&h->d_seqmap, size_t(c.max_seqs) * sizeof(int32_t)));
   h->bytes_workspace = h->part_bytes + size_t(c.max_seqs + 1) * 4 + size_t(c.max_seqs) * 4 + 4;
