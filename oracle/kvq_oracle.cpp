@@ -28,7 +28,7 @@
 //  * "KV Cache Quantization" (chipfoundryservices.com): per-token
 //    scale/zero-point quantization.
 //
-// Readings where the pages are silent (each listed in the design doc):
+// Readings where the pages are silent:
 //  * round() is round-half-to-even; the division is one IEEE fp32 division.
 //  * the codes are computed with the STORED scale (fp16-rounded, saturating at
 //    65504), so reconstruction uses the same number that divided.

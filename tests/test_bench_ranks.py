@@ -1,0 +1,57 @@
+"""The N>1 path of bench.py on CPU: two gloo ranks, each a replica, combine their
+timings by max and their work by sum (the only collectives), and the
+algorithmic byte counts match the format arithmetic."""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE="2",
+                      RANK=str(rank), LOCAL_RANK=str(rank), KVQ_BENCH_BACKEND="gloo")
+    import bench
+    r, ws, dist = bench.dist_setup(2)
+    assert (r, ws) == (rank, 2)
+    bench.barrier(dist)
+    mx = bench.max_over_ranks(dist, [1.0 + rank, 10.0 - rank])
+    sm = bench.sum_over_ranks(dist, [3.0, float(rank)])
+    q.put((rank, mx, sm))
+    dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_max_and_sum():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    got = sorted(q.get(timeout=10) for _ in range(2))
+    for rank, mx, sm in got:
+        assert mx == [2.0, 10.0]
+        assert sm == [6.0, 1.0]
+
+
+def test_algorithmic_bytes_of_the_int4_workload():
+    import bench
+    from quantized_kv_cache_14_b200.workloads import workload
+    w = workload(3)
+    # 8192 quantized tokens: 8 heads x (64 + 64 codes + 2 + 2 scale bytes) per token,
+    # no window tokens, plus q (32 x 128 bf16) and out (fp32), plus 512 table entries
+    b = bench.decode_bytes(w, [8192])
+    assert b == 8192 * 8 * 136 + 32 * 128 * 6 + 512 * 4
+    # the first config's 16 x 8192 quantized tokens are the survey's 142,606,336 bytes
+    assert 16 * 8192 * 8 * 136 == 142_606_336
+    # 63 window tokens are bf16 rows of K and V
+    assert bench.decode_bytes(w, [8192 + 63]) - b == 63 * 8 * 2 * 128 * 2
