@@ -248,6 +248,41 @@ kvq_status kvq_set_decode_grid(kvq_handle h, int32_t ctas);
  * the caller and must outlive its use. */
 kvq_status kvq_set_decode_event(kvq_handle h, void* event);
 
+/* Decode attention (as kvq_decode_attn) over caller-owned cache buffers,
+ * allocating no device memory.  The pages have no counterpart to this call:
+ * it serves callers that cannot allocate when they decode -- a runtime that
+ * hands the library a pre-sized arena, a process that must allocate everything
+ * at start-up, or a serving path where allocation is forbidden.  Its scratch
+ * (split-K partials, tile prefix, error word) is a fixed 4 MiB array in the
+ * library's device image, held by every GPU that loads the library until the
+ * process exits; calls size-check against it and never call cudaMalloc,
+ * cudaFree or an allocating library routine.
+ *   cfg          format and capacity; max_seqs bounds batch.  Not a handle.
+ *   pool         device, num_blocks * block_bytes in the kvq_layout format.
+ *   k_window, v_window  device bf16 [batch][h_kv][residual][d_h] BF16 windows
+ *                (may be NULL when residual == 0).
+ *   block_table  device int32 [batch][bt_stride], row i = batch row i.
+ *   stored_lens  device int32 [batch]: tokens stored for row i (quantized +
+ *                window), which fixes where the window starts.
+ *   seq_lens     device int32 [batch]: positions to attend, <= stored_lens[i].
+ *   q_bf16, out  as in kvq_decode_attn (row i uses window row i).
+ *   error_bits_dev  optional device uint32: receives this call's device
+ *                check bits (KVQ_DEVERR_*), 0 if none fired.
+ * Runs on the current CUDA device.  The first call on a device looks up the
+ * scratch array's device address (cudaGetSymbolAddress) and sets the decode
+ * kernel's shared-memory limit; make that first call before any stream
+ * capture.  All calls share the one array and it keeps the last call's
+ * contents: calls whose work can overlap on the GPU (different streams
+ * without ordering) race on it.  Returns KVQ_ERR_INVALID_ARG with a message
+ * giving both sizes when batch * h_kv needs more scratch than the array holds
+ * (with 4 query heads per kv head and one resident wave of 296 CTAs, up to
+ * about 800 (row, kv head) pairs). */
+kvq_status kvq_decode_attn_noalloc(const kvq_config* cfg, const void* pool, const void* k_window,
+                                   const void* v_window, const int32_t* block_table,
+                                   int32_t bt_stride, const int32_t* stored_lens,
+                                   const int32_t* seq_lens, const void* q_bf16, int32_t batch,
+                                   float* out, uint32_t* error_bits_dev, void* stream);
+
 /* Text of the last failure on the calling thread ("" if none). */
 const char* kvq_last_error(void);
 

@@ -18,7 +18,7 @@ constexpr int kMaxPagesPerGroup = 8;
 // flush plan entry: seq, group, n_pages, blocks[kMaxPagesPerGroup]
 constexpr int kFlushEntryInts = 3 + kMaxPagesPerGroup;
 
-// Byte geometry of a format (see the format notes in kvq.h / the design doc).
+// Byte geometry of a format (the layout described in kvq.h).
 struct Geo {
   int bits, asym, k_axis, g_k, g_v, scale_fp32, R, P, h_q, h_kv, G;
   int n;                    // codes per 32-bit word
@@ -94,5 +94,9 @@ cudaError_t launch_decode(const DecodeArgs& a, int grid, size_t smem, cudaStream
                           cudaEvent_t between, int* launches);
 size_t decode_smem_bytes(int B, int nstages, int stage_bytes);
 int decode_prefix_bytes(int B);
+
+// Fixed decode scratch of kvq_decode_attn_noalloc (kvq_noalloc.cu).
+size_t noalloc_scratch_bytes();
+cudaError_t noalloc_scratch(void** out);
 
 }  // namespace kvq

@@ -690,4 +690,90 @@ kvq_status kvq_set_decode_grid(kvq_handle h, int32_t ctas) {
   return KVQ_OK;
 }
 
+// Decode over caller-owned buffers with the library's fixed scratch array:
+// allocates nothing (see include/kvq.h).
+kvq_status kvq_decode_attn_noalloc(const kvq_config* cfg, const void* pool, const void* k_window,
+                                   const void* v_window, const int32_t* block_table, int32_t bt_stride,
+                                   const int32_t* stored_lens, const int32_t* seq_lens, const void* q_bf16,
+                                   int32_t batch, float* out, uint32_t* error_bits_dev, void* stream_) {
+  kvq_status st = validate(cfg);
+  if (st != KVQ_OK) return st;
+  if (batch < 0 || batch > cfg->max_seqs) return fail(KVQ_ERR_INVALID_ARG, "batch must be in [0, max_seqs]");
+  if (batch == 0) return KVQ_OK;
+  if (!pool || !block_table || !stored_lens || !seq_lens || !q_bf16 || !out)
+    return fail(KVQ_ERR_INVALID_ARG, "pool, block_table, stored_lens, seq_lens, q and out are required");
+  if (cfg->residual > 0 && (!k_window || !v_window))
+    return fail(KVQ_ERR_INVALID_ARG, "a format with a BF16 window needs k_window and v_window");
+  if (bt_stride < 1) return fail(KVQ_ERR_INVALID_ARG, "bt_stride must be >= 1");
+  for (const void* p : {pool, q_bf16, static_cast<const void*>(out), k_window, v_window})
+    if (p && !aligned16(p)) return fail(KVQ_ERR_INVALID_ARG, "device buffers must be 16-byte aligned");
+  const kvq::Geo g = make_geo(*cfg);
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+
+  int dev = 0, sms = 0, max_optin = 0;
+  KVQ_CUDA(cudaGetDevice(&dev));
+  KVQ_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  KVQ_CUDA(cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
+  // the same stage sizing as a handle's decode
+  const int res_tile = cfg->residual ? 2 * 16 * kvq::kD * 2 : 0;
+  const int stage_bytes = int(align_up(size_t(std::max(g.qtile_bytes, res_tile)), 128));
+  const size_t budget = 113 * 1024;
+  const size_t fixed = size_t(kvq::decode_prefix_bytes(cfg->max_seqs));
+  int ns = int((budget > fixed ? budget - fixed : 0) / (size_t(kvq::kDecodeWarps) * (stage_bytes + 8)));
+  ns = std::max(1, std::min(ns, 8));
+  size_t smem_max = kvq::decode_smem_bytes(cfg->max_seqs, ns, stage_bytes);
+  while (smem_max > size_t(max_optin) && ns > 1) smem_max = kvq::decode_smem_bytes(cfg->max_seqs, --ns, stage_bytes);
+  if (smem_max > size_t(max_optin)) return fail(KVQ_ERR_UNSUPPORTED, "decode tile does not fit in shared memory");
+  const void* kern = kvq::decode_kernel_ptr(g);
+  KVQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_max)));
+  int per_sm = 0;
+  KVQ_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kvq::kDecodeWarps * 32, smem_max));
+  if (per_sm < 1) return fail(KVQ_ERR_UNSUPPORTED, "decode kernel cannot be resident");
+  const int grid = sms * per_sm;
+  const int nw = grid * kvq::kDecodeWarps;
+
+  // scratch layout: [error word | pad to 256][prefix (batch + 1) | pad to 256][partials]
+  const size_t off_prefix = 256;
+  const size_t off_part = off_prefix + align_up(size_t(batch + 1) * 4, 256);
+  const size_t part_bytes = (size_t(batch) * g.h_kv + size_t(nw)) * g.G * (kvq::kD + 2) * sizeof(float);
+  if (off_part + part_bytes > kvq::noalloc_scratch_bytes())
+    return fail(KVQ_ERR_INVALID_ARG,
+                "batch * h_kv too large for the fixed decode scratch of " +
+                    std::to_string(kvq::noalloc_scratch_bytes()) + " bytes (needs " +
+                    std::to_string(off_part + part_bytes) + ")");
+  void* scratch = nullptr;
+  KVQ_CUDA(kvq::noalloc_scratch(&scratch));
+  uint8_t* base = static_cast<uint8_t*>(scratch);
+  KVQ_CUDA(cudaMemsetAsync(base, 0, sizeof(uint32_t), stream));   // error word starts clear
+
+  kvq::DecodeArgs a{};
+  a.pool = static_cast<const uint8_t*>(pool);
+  a.kres = static_cast<const uint16_t*>(k_window);
+  a.vres = static_cast<const uint16_t*>(v_window);
+  a.table = block_table;
+  a.table_stride = bt_stride;
+  a.table_by_seq = 0;
+  a.seq_lens = seq_lens;
+  a.seqmap = nullptr;            // row i is sequence i of the caller's buffers
+  a.stored_len = stored_lens;
+  a.q = static_cast<const uint16_t*>(q_bf16);
+  a.out = out;
+  a.partials = reinterpret_cast<float*>(base + off_part);
+  a.prefix = reinterpret_cast<int32_t*>(base + off_prefix);
+  a.err = reinterpret_cast<uint32_t*>(base);
+  a.B = batch;
+  a.nstages = ns;
+  a.stage_bytes = stage_bytes;
+  a.pre_bytes = kvq::decode_prefix_bytes(batch);
+  a.nw = nw;
+  a.qk_scale = float(1.4426950408889634 / std::sqrt(double(kvq::kD)));
+  a.g = g;
+  int launches = 0;
+  KVQ_CUDA(kvq::launch_decode(a, grid, kvq::decode_smem_bytes(batch, ns, stage_bytes), stream, nullptr,
+                              &launches));
+  if (error_bits_dev)
+    KVQ_CUDA(cudaMemcpyAsync(error_bits_dev, base, sizeof(uint32_t), cudaMemcpyDeviceToDevice, stream));
+  return KVQ_OK;
+}
+
 }  // extern "C"

@@ -39,7 +39,8 @@ EXPORTS = (
     "kvq_create", "kvq_destroy", "kvq_append", "kvq_decode_attn", "kvq_block_table",
     "kvq_block_table_host", "kvq_seq_len", "kvq_seq_lens_device", "kvq_free_seq",
     "kvq_stats", "kvq_cache_bytes", "kvq_layout", "kvq_read_pool", "kvq_read_residual",
-    "kvq_sync_status", "kvq_set_decode_grid", "kvq_set_decode_event", "kvq_last_error",
+    "kvq_sync_status", "kvq_set_decode_grid", "kvq_set_decode_event", "kvq_decode_attn_noalloc",
+    "kvq_last_error",
 )
 
 
@@ -104,6 +105,8 @@ def lib():
             "kvq_sync_status": (st, [P, P, ctypes.POINTER(ctypes.c_uint32)]),
             "kvq_set_decode_grid": (st, [P, I32]),
             "kvq_set_decode_event": (st, [P, P]),
+            "kvq_decode_attn_noalloc": (st, [ctypes.POINTER(KvqConfig), P, P, P, P, I32, P, P, P, I32,
+                                             P, P, P]),
             "kvq_last_error": (ctypes.c_char_p, []),
         }
         for name, (res, args) in sig.items():
@@ -236,6 +239,19 @@ def kvq_set_decode_grid(h, ctas: int):
 
 def kvq_set_decode_event(h, event: int):
     _check(lib().kvq_set_decode_event(h, ctypes.c_void_p(event or None)))
+
+
+def kvq_decode_attn_noalloc(cfg: KvqConfig, pool_ptr: int, k_window_ptr: int, v_window_ptr: int,
+                            block_table_ptr: int, bt_stride: int, stored_lens_ptr: int,
+                            seq_lens_ptr: int, q_ptr: int, batch: int, out_ptr: int,
+                            error_bits_ptr: int = 0, stream: int = 0):
+    """Decode over caller-owned device buffers; the library allocates nothing
+    (its scratch is a fixed device array).  Pointers are device addresses."""
+    V = ctypes.c_void_p
+    _check(lib().kvq_decode_attn_noalloc(ctypes.byref(cfg), V(pool_ptr), V(k_window_ptr or None),
+                                         V(v_window_ptr or None), V(block_table_ptr), int(bt_stride),
+                                         V(stored_lens_ptr), V(seq_lens_ptr), V(q_ptr), int(batch),
+                                         V(out_ptr), V(error_bits_ptr or None), V(stream)))
 
 
 def kvq_last_error() -> str:
