@@ -77,7 +77,7 @@ enum { KVQ_AXIS_TOKEN = 0, KVQ_AXIS_CHANNEL = 1 };
  *   scale_fp32  0: scales and zero-points stored as fp16 (round to nearest
  *               even, saturating at 65504); 1: stored as fp32.
  *   residual    R, the BF16 window length (0 or g_k).
- *   page        P tokens per block: a multiple of 16.
+ *   page        P tokens per block: a power of two, at least 16.
  *   h_q, h_kv   query and key/value heads; h_q / h_kv must be 1, 2 or 4.
  *   d_h         head dimension: 128.
  *   max_seqs, num_blocks, max_blocks_per_seq   capacity.
@@ -253,7 +253,7 @@ kvq_status kvq_set_decode_event(kvq_handle h, void* event);
  * it serves callers that cannot allocate when they decode -- a runtime that
  * hands the library a pre-sized arena, a process that must allocate everything
  * at start-up, or a serving path where allocation is forbidden.  Its scratch
- * (split-K partials, tile prefix, error word) is a fixed 4 MiB array in the
+ * (split-K partials, tile prefix, error word) is a fixed 16 MiB array in the
  * library's device image, held by every GPU that loads the library until the
  * process exits; calls size-check against it and never call cudaMalloc,
  * cudaFree or an allocating library routine.
@@ -274,9 +274,10 @@ kvq_status kvq_set_decode_event(kvq_handle h, void* event);
  * capture.  All calls share the one array and it keeps the last call's
  * contents: calls whose work can overlap on the GPU (different streams
  * without ordering) race on it.  Returns KVQ_ERR_INVALID_ARG with a message
- * giving both sizes when batch * h_kv needs more scratch than the array holds
- * (with 4 query heads per kv head and one resident wave of 296 CTAs, up to
- * about 800 (row, kv head) pairs). */
+ * giving both sizes when batch * h_kv needs more scratch than the array holds.
+ * The partials take (batch * h_kv + grid) * 4 * G * 520 bytes, G = h_q / h_kv
+ * and grid = resident decode CTAs (3 per SM, 444 on 148 SMs): with G = 4 that
+ * allows about 1,500 (row, kv head) pairs. */
 kvq_status kvq_decode_attn_noalloc(const kvq_config* cfg, const void* pool, const void* k_window,
                                    const void* v_window, const int32_t* block_table,
                                    int32_t bt_stride, const int32_t* stored_lens,

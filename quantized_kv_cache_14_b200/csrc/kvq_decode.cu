@@ -4,34 +4,34 @@
 // Computes out = softmax(q K^T / sqrt(d_h)) V for one query token per
 // sequence (llmdaily.org day-65, "Why the KV cache grows so quickly"), where K
 // and V are the dequantized cache x_hat = s q (+ z) ("From BF16 to INT8, INT4,
-// or even fewer bits") plus the BF16 residual window ("Why some systems keep a
+// or even fewer bits") plus the BF16 window ("Why some systems keep a
 // full-precision window"), read through the block table ("How this connects
 // to paging and prefix caching").  The pages' trade-off -- memory traffic
 // saved versus dequantization work ("Why compression may also improve speed";
-// oh-bug.com, misconception 1) -- decides the design:
+// oh-bug.com, misconception 1) -- shapes the design:
 //
-//  * Work is a list of tiles: per (row, kv head), one tile per key group
-//    (channel-axis keys) or per 16 tokens (token-axis keys), then the residual
-//    window in 16-token tiles.  Every warp of a persistent grid takes a
-//    contiguous, equal share of that list (split-K without a fixed split
-//    size), so all SMs stay busy for any length mix.  A pair that spans
-//    several warps leaves one (m, l, o) partial per warp; the reduce kernel
-//    merges them by log-sum-exp.
-//  * Each warp streams its tiles through its own ring of shared-memory stages
-//    filled by bulk asynchronous copies (TMA, cp.async.bulk) completing on
-//    mbarriers, so many KB per SM are in flight while it computes.
+//  * Work is a list of units per (row, kv head): quantized units of 64 tokens
+//    (one key group when groups are longer), then the BF16 window in 16-token
+//    tiles.  A persistent grid gives every CTA a contiguous, equal share of
+//    the whole list (split-K whose split points come from balance), so all SMs
+//    stay busy for any length mix.
+//  * A CTA is one producer warp and four consumer warps around a ring of
+//    shared-memory stages.  The producer's lane 0 fills a stage with bulk
+//    asynchronous copies (TMA, cp.async.bulk) of whole page chunks completing
+//    on the stage's "full" mbarrier; the consumers release it on its "empty"
+//    mbarrier.  Each consumer warp takes one 16-token sub-tile of a unit.
 //  * The g = h_q / h_kv query heads sharing a kv head are processed together:
-//    every cached byte is read once.  Scores S = K_hat q'^T and the product
-//    P' V_hat run on mma.sync m16n8k16 with bf16 operands and fp32
-//    accumulation: the integer codes are exact in bf16, the scale is folded
-//    into the other operand (q' = q * s_channel for per-channel keys,
-//    p' = p * s_token for per-token values) and that operand is split into
-//    bf16 hi + lo columns (2 x 4 heads = the 8 columns of the mma), keeping 16
-//    significant bits.  Zero-points enter as a per-group bias (keys) and a
-//    p-weighted sum (values).  Codes are unpacked with one LOP3 + one bf16x2
-//    FMA per pair of elements.
+//    every cached byte is read once.  Scores K_hat q'^T and P' V_hat run on
+//    mma.sync m16n8k16 with bf16 operands and fp32 accumulation.  Codes are
+//    exact in bf16; the scale goes into the other operand (q' = q * s_channel
+//    per key group, computed once per unit by the four consumer warps into
+//    shared memory; p' = p * s_token per value group), split into bf16 hi + lo
+//    columns (4 heads x {hi, lo} = the 8 mma columns, 16 significant bits).
+//    Zero-points enter as a per-group key bias and a p-weighted value sum.
 //  * Online softmax in the log2 domain with warp-shuffle reductions; the
-//    running max is only moved when it grows by more than 8 (p <= 256).
+//    running max moves only when it grows by more than 8 (p <= 256).  Each
+//    consumer warp leaves one (m, l, o) partial per pair its CTA touched; the
+//    merge kernel combines them by log-sum-exp in a fixed order.
 #include <cstdint>
 
 #include "kvq_device.cuh"
@@ -39,14 +39,31 @@
 namespace kvq {
 namespace {
 
-constexpr uint32_t kWaitPolls = 1u << 20;
+constexpr uint64_t kWaitNs = 2000000000ull;   // give up on a copy after 2 s
+constexpr int kQbufBytes = 32 * 16 * 4;   // one key group's q' operand: 32 lanes x 16 words
+constexpr int kBiasBytes = 16;            // one key group's zero-point bias of 4 heads
+
+struct SmemLayout {
+  int stages, qbuf, bias, bars, flag, total;
+};
+
+__host__ __device__ inline SmemLayout smem_layout(int B, const DecodePipe& p) {
+  SmemLayout L;
+  L.stages = ((B + 1 + 32) * 4 + 127) / 128 * 128;      // prefix table + scan scratch
+  L.qbuf = L.stages + p.nstages * p.stage_bytes;
+  L.bias = L.qbuf + 2 * p.ngr * kQbufBytes;
+  L.bars = L.bias + 2 * p.ngr * kBiasBytes;
+  L.flag = L.bars + 2 * p.nstages * 8;
+  L.total = L.flag + 16;
+  return L;
+}
 
 struct RowInfo {
   int seq;
   int qa;   // quantized positions attended
-  int ra;   // residual positions attended
-  int nq;   // quantized tiles
-  int nr;   // residual tiles
+  int ra;   // window positions attended
+  int nq;   // quantized units
+  int nr;   // window tiles
   const int32_t* trow;
 };
 
@@ -67,16 +84,17 @@ __device__ __forceinline__ RowInfo row_info(const DecodeArgs& a, int i, bool fla
     if (flag) atomicOr(a.err, KVQ_DEVERR_SEQ_LEN);
     len = min(max(len, 0), stored);
   }
-  const int Lq = g.R ? (stored / g.R) * g.R : stored;
+  const int Lq = g.R ? (stored >> g.lg_gk) << g.lg_gk : stored;   // R == g_k
   r.qa = min(len, Lq);
   r.ra = max(0, len - Lq);
-  r.nq = (r.qa + g.tileT - 1) / g.tileT;
+  r.nq = (r.qa + a.pipe.sup - 1) >> a.pipe.lg_sup;
   r.nr = (r.ra + 15) / 16;
   r.trow = a.table + int64_t(a.table_by_seq ? seq : i) * a.table_stride;
   return r;
 }
 
-// Exclusive prefix over s[1..n] (counts) -> s[0..n]; all threads participate.
+// Exclusive prefix over s[1..n] (counts) -> s[0..n]; every thread of the CTA
+// takes part.
 __device__ void block_scan(int32_t* s, int n, int32_t* scratch) {
   const int T = blockDim.x, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int chunk = (n + T - 1) / T;
@@ -106,7 +124,7 @@ struct It {
 };
 
 __device__ __forceinline__ void it_seek(It& it, const int32_t* pre, int B, int hkv, int64_t u) {
-  int lo = 0, hi = B;   // first j in [0, B] with pre[j] * hkv > u, minus one
+  int lo = 0, hi = B;   // the row whose units hold u
   while (lo < hi) {
     const int mid = (lo + hi) >> 1;
     if (int64_t(pre[mid + 1]) * hkv > u) hi = mid;
@@ -129,66 +147,18 @@ __device__ __forceinline__ bool it_next(It& it, const int32_t* pre, int B, int h
   return true;   // row changed
 }
 
-// Issue the bulk copies of one tile into a stage (lane 0 only).
-template <int ASYM, int KAXIS>
-__device__ void issue_tile(const DecodeArgs& a, const It& it, const RowInfo& ri, uint32_t dst,
-                           uint32_t bar) {
-  const Geo& g = a.g;
-  if (it.k < ri.nq) {
-    if (KAXIS) {
-      const int npg = g.g_k / g.P;
-      const int lb0 = it.k * npg;
-      bool ok = lb0 + npg <= a.table_stride;
-      for (int j = 0; ok && j < npg; ++j) {
-        const int32_t b = ri.trow[lb0 + j];
-        ok = b >= 0 && b < g.num_blocks;
-      }
-      if (!ok) {
-        atomicOr(a.err, KVQ_DEVERR_BLOCK_ID);
-        mbar_arrive_expect_tx(bar, 0);
-        return;
-      }
-      mbar_arrive_expect_tx(bar, uint32_t(npg * g.chunk_used));
-      for (int j = 0; j < npg; ++j) {
-        const uint8_t* src = a.pool + int64_t(ri.trow[lb0 + j]) * g.block_bytes +
-                             int64_t(it.h) * g.chunk_bytes;
-        bulk_g2s(dst + j * g.chunk_used, src, uint32_t(g.chunk_used), bar);
-      }
-    } else {
-      const int T0 = 16 * it.k;
-      const int lb = T0 / g.P, u = (T0 % g.P) / 16;
-      const int32_t b = lb < a.table_stride ? ri.trow[lb] : -1;
-      if (b < 0 || b >= g.num_blocks) {
-        atomicOr(a.err, KVQ_DEVERR_BLOCK_ID);
-        mbar_arrive_expect_tx(bar, 0);
-        return;
-      }
-      const uint8_t* chunk = a.pool + int64_t(b) * g.block_bytes + int64_t(it.h) * g.chunk_bytes;
-      if (g.P == 16) {
-        mbar_arrive_expect_tx(bar, uint32_t(g.chunk_used));
-        bulk_g2s(dst, chunk, uint32_t(g.chunk_used), bar);
-      } else {
-        const int vrow = 16 * g.nvg * g.es, krow = 16 * g.nkg * g.es;
-        const uint32_t total = 2 * g.sub_bytes + (vrow + krow) * (1 + ASYM);
-        mbar_arrive_expect_tx(bar, total);
-        bulk_g2s(dst, chunk + u * g.sub_bytes, g.sub_bytes, bar);
-        bulk_g2s(dst + g.sub_bytes, chunk + g.off_V + u * g.sub_bytes, g.sub_bytes, bar);
-        const uint32_t vm = dst + 2 * g.sub_bytes, km = vm + g.vm16;
-        bulk_g2s(vm, chunk + g.off_Vm + int64_t(16 * u) * g.nvg * g.es, vrow, bar);
-        bulk_g2s(km, chunk + g.off_Km + int64_t(16 * u) * g.nkg * g.es, krow, bar);
-        if (ASYM) {
-          bulk_g2s(vm + vrow, chunk + g.off_Vm + int64_t(g.P + 16 * u) * g.nvg * g.es, vrow, bar);
-          bulk_g2s(km + krow, chunk + g.off_Km + int64_t(g.P + 16 * u) * g.nkg * g.es, krow, bar);
-        }
-      }
-    }
-  } else {
-    const int kr = it.k - ri.nq;
-    const int64_t base = ((int64_t(ri.seq) * g.h_kv + it.h) * g.R + 16 * kr) * kD;
-    mbar_arrive_expect_tx(bar, 2 * 16 * kD * 2);
-    bulk_g2s(dst, a.kres + base, 16 * kD * 2, bar);
-    bulk_g2s(dst + 16 * kD * 2, a.vres + base, 16 * kD * 2, bar);
-  }
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
+}
+
+// Barrier of the four consumer warps only (the producer warp never joins).
+__device__ __forceinline__ void consumer_sync() {
+  asm volatile("bar.sync 1, 128;\n" ::: "memory");
+}
+
+// Bounded wait that also gives up as soon as another warp has aborted.
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int32_t* abort_flag) {
+  return mbar_wait_bounded(bar, parity, kWaitNs, abort_flag);
 }
 
 // Per-thread accumulation state of one (row, kv head) pair.
@@ -210,7 +180,7 @@ __device__ __forceinline__ void state_reset(State& st) {
 }
 
 // Online softmax over the two scores (tokens gq, gq+8; head tq) of a 16-token
-// sub-tile; returns their weights p relative to the running max.
+// sub-tile; returns their weights relative to the running max.
 __device__ __forceinline__ void softmax_step(State& st, float s0, float s1, float& p0, float& p1) {
   float mx = fmaxf(s0, s1);
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
@@ -233,9 +203,8 @@ __device__ __forceinline__ void softmax_step(State& st, float s0, float s1, floa
   st.l += p0 + p1;
 }
 
-// Scores of a 16-token sub-tile of packed keys: acc[] += K_hat q'^T for the
-// k-steps of one key group; the caller folds groups.
-template <int BITS, bool SGN>
+// Key words of rows gq and gq + 8 of a packed 16-token sub-tile.
+template <int BITS>
 __device__ __forceinline__ void load_key_words(const uint8_t* ksub, int gq, int tq, uint32_t (&wa)[BITS],
                                                uint32_t (&wb)[BITS]) {
   constexpr int row = kD * BITS / 8, slice = 4 * BITS;
@@ -282,8 +251,8 @@ __device__ __forceinline__ void key_frag(const uint32_t (&wa)[BITS], const uint3
 
 // A operand of the value product for channel tile i from a lane record.
 template <int BITS, bool SGN>
-__device__ __forceinline__ void value_frag(const uint32_t (&w)[2 * BITS], int i, uint32_t& a0,
-                                           uint32_t& a1, uint32_t& a2, uint32_t& a3) {
+__device__ __forceinline__ void value_frag(const uint32_t (&w)[2 * BITS], int i, uint32_t& a0, uint32_t& a1,
+                                           uint32_t& a2, uint32_t& a3) {
   if (BITS == 4) {
     a0 = nib_pair<SGN>(w[i], 0);
     a1 = nib_pair<SGN>(w[i], 1);
@@ -313,45 +282,72 @@ __device__ __forceinline__ void load_value_words(const uint8_t* vsub, int lane, 
   }
 }
 
-__device__ __forceinline__ float vmeta(const uint8_t* base, int idx, int es) {
+__device__ __forceinline__ float meta_at(const uint8_t* base, int idx, int es) {
   return es == 4 ? reinterpret_cast<const float*>(base)[idx]
                  : __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(base)[idx]));
 }
 
-// B operand (token rows 2tq, 2tq+1, 2tq+8, 2tq+9; column gq = head gq/2,
-// hi|lo) of the value product, from the softmax weights pa0 (2tq), pb0
-// (2tq+1), pa1 (2tq+8), pb1 (2tq+9) times each token's value scale.
-__device__ __forceinline__ void pv_bfrag(float pa0, float pb0, float pa1, float pb1, float s0, float s1,
-                                         float s2, float s3, bool lo, bool dead, uint32_t& b0,
-                                         uint32_t& b1) {
-  b0 = split_pack(pa0 * s0, pb0 * s1, lo);
-  b1 = split_pack(pa1 * s2, pb1 * s3, lo);
-  if (dead) b0 = b1 = 0u;
+// Four consecutive metadata entries starting at a multiple of 4.
+__device__ __forceinline__ void meta4(const uint8_t* base, int idx, int es, float (&v)[4]) {
+  if (es == 4) {
+    const float4 x = *reinterpret_cast<const float4*>(base + idx * 4);
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+  } else {
+    const uint2 x = *reinterpret_cast<const uint2*>(base + idx * 2);
+    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&x.x));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&x.y));
+    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+  }
 }
 
+// Both bf16 parts of an fp32 pair: hi = bf16_rn(x), lo = bf16_rn(x - hi).
+__device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  const __nv_bfloat162 l =
+      __floats2bfloat162_rn(x0 - __uint_as_float(hi << 16), x1 - __uint_as_float(hi & 0xFFFF0000u));
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// Where one 16-token sub-tile sits in a stage.
+struct Sub {
+  const uint8_t* k;     // key codes
+  const uint8_t* v;     // value codes
+  const uint8_t* vms;   // value scales, row 0 of the sub-tile; index r * nvg + group
+  const uint8_t* vmz;   // value zero-points
+  const uint8_t* kms;   // token-axis key scales, row 0; index r * nkg + group
+  const uint8_t* kmz;
+};
+
 template <int BITS, int ASYM, int KAXIS>
-__global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const __grid_constant__ DecodeArgs a) {
+__global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_constant__ DecodeArgs a) {
   constexpr int D = kD;
   constexpr bool SGN = !ASYM;
   extern __shared__ __align__(128) uint8_t smem[];
   const Geo& g = a.g;
+  const DecodePipe& pp = a.pipe;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int gq = lane >> 2, tq = lane & 3;
-  const int hh = gq >> 1;               // head of this lane's B column
-  const bool is_lo = gq & 1;            // column carries the lo part
-  const bool dead_col = hh >= g.G;      // padding column (fewer than 4 heads)
-
+  const SmemLayout L = smem_layout(a.B, pp);
   int32_t* s_pre = reinterpret_cast<int32_t*>(smem);
   int32_t* s_scr = s_pre + (a.B + 1);
-  uint8_t* my_stages = smem + a.pre_bytes + size_t(warp) * a.nstages * a.stage_bytes;
-  uint64_t* my_bars = reinterpret_cast<uint64_t*>(smem + a.pre_bytes +
-                                                  size_t(kDecodeWarps) * a.nstages * a.stage_bytes) +
-                      warp * a.nstages;
+  uint8_t* stages = smem + L.stages;
+  const uint32_t stage0 = smem_addr(stages);
+  const uint32_t full0 = smem_addr(smem + L.bars);
+  const uint32_t empty0 = full0 + 8 * pp.nstages;
+  volatile int32_t* abort_flag = reinterpret_cast<int32_t*>(smem + L.flag);
 
-  // ---- work list: tiles per row, prefix over rows -------------------------
+  // ---- the work list: units per row, prefix over rows ---------------------
   for (int i = tid; i < a.B; i += blockDim.x) {
     const RowInfo ri = row_info(a, i, blockIdx.x == 0);
     s_pre[i + 1] = ri.nq + ri.nr;
+  }
+  if (tid == 0) {
+    for (int s = 0; s < pp.nstages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, kDecodeWarps);
+    }
+    *abort_flag = 0;
+    mbar_init_fence();
   }
   __syncthreads();
   block_scan(s_pre, a.B, s_scr);
@@ -359,61 +355,150 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const __grid_
     for (int i = tid; i <= a.B; i += blockDim.x) a.prefix[i] = s_pre[i];
 
   const int64_t U = int64_t(s_pre[a.B]) * g.h_kv;
-  const int gw = blockIdx.x * kDecodeWarps + warp;
-  const int64_t u0 = int64_t(gw) * U / a.nw, u1 = int64_t(gw + 1) * U / a.nw;
-  if (u0 >= u1) return;
+  const int64_t c0 = int64_t(blockIdx.x) * U / a.grid, c1 = int64_t(blockIdx.x + 1) * U / a.grid;
+  if (c0 >= c1) return;
+  const int N = int(c1 - c0);
 
-  const uint32_t stage0 = smem_addr(my_stages);
-  const uint32_t bar0 = smem_addr(my_bars);
-  if (lane == 0) {
-    for (int s = 0; s < a.nstages; ++s) mbar_init(bar0 + 8 * s, 1);
-    mbar_init_fence();
-  }
-  __syncwarp();
-
-  // ---- producer (lane 0): run ahead by nstages tiles ----------------------
-  It pit;
-  it_seek(pit, s_pre, a.B, g.h_kv, u0);
-  RowInfo pri = row_info(a, pit.i, false);
-  int64_t issued = u0;
-  if (lane == 0) {
-    for (int s = 0; s < a.nstages && issued < u1; ++s, ++issued) {
-      issue_tile<ASYM, KAXIS>(a, pit, pri, stage0 + s * a.stage_bytes, bar0 + 8 * s);
-      if (it_next(pit, s_pre, a.B, g.h_kv) && issued + 1 < u1) pri = row_info(a, pit.i, false);
+  if (warp == kDecodeWarps) {
+    // ---------------------------- producer ----------------------------------
+    // The whole warp: a window of 32 block-table entries is fetched with one
+    // coalesced load and read by shuffle, and a unit's copies are issued in
+    // parallel, one lane per page (or per 16-token sub-tile).
+    constexpr uint32_t FULL = 0xffffffffu;
+    It it;
+    it_seek(it, s_pre, a.B, g.h_kv, c0);
+    RowInfo ri = row_info(a, it.i, false);
+    int win_row = -1, win_base = 0;
+    int32_t win = -1;
+    int s = 0;
+    uint32_t ph = 0;
+    int issued = 0;
+    const int vrow = 16 * g.nvg * g.es, krow = 16 * g.nkg * g.es;
+    for (int n = 0; n < N; ++n) {
+      const uint32_t dst = stage0 + s * pp.stage_bytes;
+      const uint32_t bar = full0 + 8 * s;
+      bool bad = false;
+      uint32_t total = 0;
+      int ncopy = 0;          // lanes [0, ncopy) issue copies
+      int32_t blk = 0;        // this lane's block
+      int tok = 0;            // token axis: this lane's sub-tile's first token
+      if (it.k < ri.nq) {
+        const int T0 = it.k * pp.sup;
+        const int valid = min(pp.sup, ri.qa - T0);
+        const int lb0 = T0 >> g.lg_P;
+        int npg;
+        if (KAXIS) {
+          npg = ((valid + g.g_k - 1) >> g.lg_gk) << (g.lg_gk - g.lg_P);   // whole key groups
+          ncopy = npg;
+          total = uint32_t(npg * g.chunk_used);
+        } else {
+          const int nsub = (valid + 15) >> 4;
+          npg = ((T0 + 16 * nsub - 1) >> g.lg_P) - lb0 + 1;
+          ncopy = nsub;
+          total = uint32_t(nsub) * (g.P == 16 ? uint32_t(g.chunk_used)
+                                              : uint32_t(2 * g.sub_bytes + (vrow + krow) * (1 + ASYM)));
+          tok = T0 + 16 * min(lane, nsub - 1);
+        }
+        if (it.i != win_row || lb0 < win_base || lb0 + npg > win_base + 32) {
+          win_row = it.i;
+          win_base = lb0;
+          win = lb0 + lane < a.table_stride ? ri.trow[lb0 + lane] : -1;
+        }
+        const int pg = KAXIS ? lane : (tok >> g.lg_P) - lb0;
+        blk = __shfl_sync(FULL, win, (lb0 - win_base + pg) & 31);
+        bad = __any_sync(FULL, lane < ncopy && (blk < 0 || blk >= g.num_blocks));
+      } else {
+        ncopy = 2;
+        total = 2 * 16 * kD * 2;
+      }
+      // every lane waits; the verdict is made warp-uniform before anyone leaves
+      if (n >= pp.nstages && !__all_sync(FULL, wait_or_abort(empty0 + 8 * s, ph ^ 1u, abort_flag))) {
+        if (lane == 0) {
+          atomicOr(a.err, KVQ_DEVERR_TIMEOUT);
+          *abort_flag = 1;
+        }
+        break;
+      }
+      if (bad) {
+        if (lane == 0) {
+          atomicOr(a.err, KVQ_DEVERR_BLOCK_ID);
+          mbar_arrive_expect_tx(bar, 0);
+        }
+      } else {
+        if (lane == 0) mbar_arrive_expect_tx(bar, total);
+        __syncwarp();
+        if (lane < ncopy) {
+          if (it.k >= ri.nq) {
+            const int kr = it.k - ri.nq;
+            const int64_t base = ((int64_t(ri.seq) * g.h_kv + it.h) * g.R + 16 * kr) * kD;
+            bulk_g2s(dst + lane * (16 * kD * 2), (lane ? a.vres : a.kres) + base, 16 * kD * 2, bar);
+          } else {
+            const uint8_t* chunk = a.pool + int64_t(blk) * g.block_bytes + int64_t(it.h) * g.chunk_bytes;
+            if (KAXIS) {
+              bulk_g2s(dst + lane * g.chunk_used, chunk, uint32_t(g.chunk_used), bar);
+            } else if (g.P == 16) {
+              bulk_g2s(dst + lane * pp.qsub, chunk, uint32_t(g.chunk_used), bar);
+            } else {
+              const int u = (tok & (g.P - 1)) >> 4;
+              const uint32_t d = dst + lane * pp.qsub;
+              bulk_g2s(d, chunk + u * g.sub_bytes, g.sub_bytes, bar);
+              bulk_g2s(d + g.sub_bytes, chunk + g.off_V + u * g.sub_bytes, g.sub_bytes, bar);
+              const uint32_t vm = d + 2 * g.sub_bytes, km = vm + g.vm16;
+              bulk_g2s(vm, chunk + g.off_Vm + int64_t(16 * u) * g.nvg * g.es, vrow, bar);
+              bulk_g2s(km, chunk + g.off_Km + int64_t(16 * u) * g.nkg * g.es, krow, bar);
+              if (ASYM) {
+                bulk_g2s(vm + vrow, chunk + g.off_Vm + int64_t(g.P + 16 * u) * g.nvg * g.es, vrow, bar);
+                bulk_g2s(km + krow, chunk + g.off_Km + int64_t(g.P + 16 * u) * g.nkg * g.es, krow, bar);
+              }
+            }
+          }
+        }
+      }
+      ++issued;
+      if (it_next(it, s_pre, a.B, g.h_kv) && n + 1 < N) ri = row_info(a, it.i, false);
+      if (++s == pp.nstages) { s = 0; ph ^= 1u; }
     }
+    // keep the CTA until its last copies have landed (bounded)
+    if (lane == 0)
+      for (int k = 0; k < pp.nstages && k < issued; ++k) {
+        const int n = issued - 1 - k;
+        (void)mbar_wait_bounded(full0 + 8 * (n % pp.nstages), uint32_t((n / pp.nstages) & 1), kWaitNs);
+      }
+    return;
   }
 
-  // ---- consumer (all lanes) -----------------------------------------------
-  It cit;
-  it_seek(cit, s_pre, a.B, g.h_kv, u0);
-  RowInfo cri = row_info(a, cit.i, false);
+  // ------------------------------ consumers -----------------------------------
+  const int gq = lane >> 2, tq = lane & 3;
+  const int hh = gq >> 1;               // head of this lane's B column
+  const bool is_lo = gq & 1;            // the column carries the lo part
+  const bool dead_col = hh >= g.G;      // padding column (fewer than 4 heads)
+  const float C = a.qk_scale;
+  const int vg_shift = __ffs(g.g_v >> 4) - 1;          // channel tiles per value group, log2
+  const int kg_shift = KAXIS ? 3 : __ffs(g.g_k >> 4) - 1;   // k-steps per key group, log2
+
   State st;
   state_reset(st);
-  int cur_pair = -1;
   uint32_t bq[8][2];          // score B operand (q' hi|lo columns)
-  float qf[KAXIS ? 32 : 1];   // channel axis: q of head hh at this lane's 32 channels
-  float bias_t = 0.0f;        // channel-axis zero-point term of head tq (log2 units)
-  const float C = a.qk_scale;
+  bool bq_holds_q = false;    // bq carries q itself (token axis, BF16 window)
+  float bias_t = 0.0f;        // zero-point term of head tq for the loaded key group
+  float qv[4] = {0.0f, 0.0f, 0.0f, 0.0f};     // q of head `warp` at this thread's 4 channels
+  float qsum[4] = {0.0f, 0.0f, 0.0f, 0.0f};   // token-axis zero-points: sum of q per group
+  int chan_units = 0;         // channel-axis units seen: picks the q' buffer
 
-  auto load_q = [&](int row, int h, float* dst32) {
-    const uint16_t* qrow = a.q + (int64_t(row) * g.h_q + h * g.G + min(hh, g.G - 1)) * D;
-#pragma unroll
-    for (int m = 0; m < 32; m += 2) {
-      const uint32_t two = *reinterpret_cast<const uint32_t*>(qrow + key_channel(32 * tq + m));
-      dst32[m] = __uint_as_float(two << 16);
-      dst32[m + 1] = __uint_as_float(two & 0xFFFF0000u);
-    }
+  auto qrow = [&](int row, int h, int head) {
+    return a.q + (int64_t(row) * g.h_q + h * g.G + min(head, g.G - 1)) * D;
   };
-  // B operand from 32 fp32 values x[] in list order (4 per k-step)
-  auto make_bq = [&](const float* x) {
+  auto load_bq_from_q = [&](int row, int h) {
+    const uint16_t* qr = qrow(row, h, hh);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      bq[j][0] = dead_col ? 0u : split_pack(x[4 * j], x[4 * j + 1], is_lo);
-      bq[j][1] = dead_col ? 0u : split_pack(x[4 * j + 2], x[4 * j + 3], is_lo);
+      const uint32_t t0 = *reinterpret_cast<const uint32_t*>(qr + key_channel(32 * tq + 4 * j));
+      const uint32_t t1 = *reinterpret_cast<const uint32_t*>(qr + key_channel(32 * tq + 4 * j + 2));
+      // q is exact in bf16: its hi part is q itself and its lo part is zero
+      bq[j][0] = (dead_col || is_lo) ? 0u : t0;
+      bq[j][1] = (dead_col || is_lo) ? 0u : t1;
     }
   };
-  // token-axis asymmetric keys: sum of q over each key group, head tq
-  float qsum[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 
   auto emit = [&](int row, int h) {
     float l = st.l;
@@ -433,7 +518,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const __grid_
     }
     if (tq < g.G) {
       const int64_t pair = int64_t(row) * g.h_kv + h;
-      float* rec = a.partials + ((pair + gw) * g.G + tq) * (D + 2);
+      float* rec = a.partials + (((pair + blockIdx.x) * kDecodeWarps + warp) * g.G + tq) * (D + 2);
       if (gq == 0) {
         rec[0] = st.m;
         rec[1] = l;
@@ -446,261 +531,340 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const __grid_
     }
   };
 
-  bool bq_holds_q = false;    // bq currently carries q itself (token axis, BF16 window)
   auto setup_pair = [&](int row, int h) {
     state_reset(st);
-    bq_holds_q = !KAXIS;
-    float qv[32];
-    load_q(row, h, qv);
+    bq_holds_q = false;
+    bias_t = 0.0f;
     if (KAXIS) {
-#pragma unroll
-      for (int m = 0; m < 32; ++m) qf[m] = qv[m];
+      // this thread's share of the q' job: head `warp`, lane group lane>>3, k-step lane&7
+      const uint16_t* qr = qrow(row, h, warp);
+      const int f = 32 * (lane >> 3) + 4 * (lane & 7);
+      const uint32_t t0 = *reinterpret_cast<const uint32_t*>(qr + key_channel(f));
+      const uint32_t t1 = *reinterpret_cast<const uint32_t*>(qr + key_channel(f + 2));
+      const bool live = warp < g.G;
+      qv[0] = live ? __uint_as_float(t0 << 16) : 0.0f;
+      qv[1] = live ? __uint_as_float(t0 & 0xFFFF0000u) : 0.0f;
+      qv[2] = live ? __uint_as_float(t1 << 16) : 0.0f;
+      qv[3] = live ? __uint_as_float(t1 & 0xFFFF0000u) : 0.0f;
     } else {
-      make_bq(qv);
+      load_bq_from_q(row, h);
+      bq_holds_q = true;
       if (ASYM) {
-        // sum of q over each key group for head tq (token-axis zero-points)
-        const uint16_t* qrow = a.q + (int64_t(row) * g.h_q + h * g.G + min(tq, g.G - 1)) * D;
+        const uint16_t* qr = qrow(row, h, tq);
         for (int gi = 0; gi < g.nkg; ++gi) {
           float s = 0.0f;
-          for (int c = gi * g.g_k; c < (gi + 1) * g.g_k; ++c) s += bf16_bits_to_float(qrow[c]);
-          qsum[gi] = s;
+          for (int c = gi * g.g_k; c < (gi + 1) * g.g_k; ++c) s += bf16_bits_to_float(qr[c]);
+          qsum[gi & 3] = s;
         }
       }
     }
   };
 
-  const int mt_per_vg = g.g_v / 16;      // channel tiles per value group
-  bool timed_out = false;
+  // Scores, online softmax and the value product of one 16-token sub-tile.
+  auto process_sub = [&](const Sub& sb, int valid) {
+    uint32_t wa[BITS], wb[BITS];
+    load_key_words<BITS>(sb.k, gq, tq, wa, wb);
+    float acc0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, acc1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      uint32_t a0, a1, a2, a3;
+      key_frag<BITS, SGN>(wa, wb, j, a0, a1, a2, a3);
+      if (j & 1) mma_bf16(acc1, a0, a1, a2, a3, bq[j][0], bq[j][1]);
+      else mma_bf16(acc0, a0, a1, a2, a3, bq[j][0], bq[j][1]);
+      if (!KAXIS && ((j + 1) & ((1 << kg_shift) - 1)) == 0) {
+        const int gi = j >> kg_shift;
+        const float r0 = acc0[0] + acc0[1] + acc1[0] + acc1[1];
+        const float r1 = acc0[2] + acc0[3] + acc1[2] + acc1[3];
+        s0 = fmaf(meta_at(sb.kms, gq * g.nkg + gi, g.es), r0, s0);
+        s1 = fmaf(meta_at(sb.kms, (gq + 8) * g.nkg + gi, g.es), r1, s1);
+        if (ASYM) {
+          s0 = fmaf(meta_at(sb.kmz, gq * g.nkg + gi, g.es), qsum[gi & 3], s0);
+          s1 = fmaf(meta_at(sb.kmz, (gq + 8) * g.nkg + gi, g.es), qsum[gi & 3], s1);
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc0[c] = acc1[c] = 0.0f;
+      }
+    }
+    if (KAXIS) {
+      s0 = acc0[0] + acc0[1] + acc1[0] + acc1[1];
+      s1 = acc0[2] + acc0[3] + acc1[2] + acc1[3];
+    }
+    s0 = fmaf(s0, C, bias_t);
+    s1 = fmaf(s1, C, bias_t);
+    if (gq >= valid) s0 = -INFINITY;
+    if (gq + 8 >= valid) s1 = -INFINITY;
 
-  for (int64_t u = u0; u < u1; ++u) {
-    const int slot = int((u - u0) % a.nstages);
-    const uint32_t parity = uint32_t(((u - u0) / a.nstages) & 1);
-    const int pair_id = cit.i * g.h_kv + cit.h;
+    float p0, p1;
+    softmax_step(st, s0, s1, p0, p1);
+
+    // value product: P' V_hat with p' = p * s_value(token, group)
+    const int sa = 8 * tq + hh, sbl = sa + 4;
+    const float pa0 = __shfl_sync(0xffffffffu, p0, sa);
+    const float pa1 = __shfl_sync(0xffffffffu, p1, sa);
+    const float pb0 = __shfl_sync(0xffffffffu, p0, sbl);
+    const float pb1 = __shfl_sync(0xffffffffu, p1, sbl);
+    uint32_t vw[2 * BITS];
+    load_value_words<BITS>(sb.v, lane, vw);
+    const int n = g.nvg;
+    uint32_t b0 = 0, b1 = 0;
+    float zs = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if ((i & ((1 << vg_shift) - 1)) == 0) {
+        const int gi = i >> vg_shift;
+        uint32_t h0, l0, h1, l1;
+        split2(pa0 * meta_at(sb.vms, (2 * tq) * n + gi, g.es), pb0 * meta_at(sb.vms, (2 * tq + 1) * n + gi, g.es),
+               h0, l0);
+        split2(pa1 * meta_at(sb.vms, (2 * tq + 8) * n + gi, g.es),
+               pb1 * meta_at(sb.vms, (2 * tq + 9) * n + gi, g.es), h1, l1);
+        b0 = dead_col ? 0u : (is_lo ? l0 : h0);
+        b1 = dead_col ? 0u : (is_lo ? l1 : h1);
+        if (ASYM) zs = p0 * meta_at(sb.vmz, gq * n + gi, g.es) + p1 * meta_at(sb.vmz, (gq + 8) * n + gi, g.es);
+      }
+      uint32_t a0, a1, a2, a3;
+      value_frag<BITS, SGN>(vw, i, a0, a1, a2, a3);
+      mma_bf16(st.o[i], a0, a1, a2, a3, b0, b1);
+      if (ASYM) st.zacc[i] += zs;
+    }
+  };
+
+  // A 16-token tile of the BF16 window (natural row-major layout).
+  auto process_window = [&](const uint8_t* stg, int valid) {
+    const uint32_t kaddr = smem_addr(stg), vaddr = kaddr + 16 * D * 2;
+    float acc0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, acc1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    const int mi = lane >> 3;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int r = (lane & 7) + 8 * (mi & 1), c = 16 * j + 8 * (mi >> 1);
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4(kaddr + (r * D + c) * 2, a0, a1, a2, a3);
+      if (j & 1) mma_bf16(acc1, a0, a1, a2, a3, bq[j][0], bq[j][1]);
+      else mma_bf16(acc0, a0, a1, a2, a3, bq[j][0], bq[j][1]);
+    }
+    float s0 = (acc0[0] + acc0[1] + acc1[0] + acc1[1]) * C;
+    float s1 = (acc0[2] + acc0[3] + acc1[2] + acc1[3]) * C;
+    if (gq >= valid) s0 = -INFINITY;
+    if (gq + 8 >= valid) s1 = -INFINITY;
+    float p0, p1;
+    softmax_step(st, s0, s1, p0, p1);
+    const int sa = 8 * tq + hh, sbl = sa + 4;
+    const float pa0 = __shfl_sync(0xffffffffu, p0, sa);
+    const float pa1 = __shfl_sync(0xffffffffu, p1, sa);
+    const float pb0 = __shfl_sync(0xffffffffu, p0, sbl);
+    const float pb1 = __shfl_sync(0xffffffffu, p1, sbl);
+    uint32_t h0, l0, h1, l1;
+    split2(pa0, pb0, h0, l0);
+    split2(pa1, pb1, h1, l1);
+    const uint32_t b0 = dead_col ? 0u : (is_lo ? l0 : h0);
+    const uint32_t b1 = dead_col ? 0u : (is_lo ? l1 : h1);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = (lane & 7) + 8 * (mi >> 1), c = 16 * i + 8 * (mi & 1);
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4_t(vaddr + (r * D + c) * 2, a0, a1, a2, a3);
+      mma_bf16(st.o[i], a0, a1, a2, a3, b0, b1);
+    }
+  };
+
+  It it;
+  it_seek(it, s_pre, a.B, g.h_kv, c0);
+  RowInfo ri = row_info(a, it.i, false);
+  int cur_pair = -1;
+  int s = 0;
+  uint32_t ph = 0;
+  bool aborted = false;
+  for (int n = 0; n < N; ++n) {
+    const int pair_id = it.i * g.h_kv + it.h;
     if (pair_id != cur_pair) {
-      if (cur_pair >= 0) emit(cur_pair / g.h_kv, cur_pair % g.h_kv);
-      setup_pair(cit.i, cit.h);
+      if (cur_pair >= 0 && !aborted) emit(cur_pair / g.h_kv, cur_pair % g.h_kv);
+      setup_pair(it.i, it.h);
       cur_pair = pair_id;
     }
-    // every lane polls; the warp leaves together if any lane gave up
-    const bool arrived = mbar_wait_bounded(bar0 + 8 * slot, parity, kWaitPolls);
-    if (!__all_sync(0xffffffffu, arrived)) {
-      timed_out = true;
-      break;
+    // every lane polls; the warp gives up together, and once any warp has
+    // given up all of them skip the remaining work (but keep the barriers)
+    if (!aborted) {
+      const bool arrived = wait_or_abort(full0 + 8 * s, ph, abort_flag);
+      if (!__all_sync(0xffffffffu, arrived)) {
+        if (lane == 0) {
+          atomicOr(a.err, KVQ_DEVERR_TIMEOUT);
+          *abort_flag = 1;
+        }
+        aborted = true;
+      }
     }
-    const uint8_t* stg = my_stages + size_t(slot) * a.stage_bytes;
+    const uint8_t* stg = stages + size_t(s) * pp.stage_bytes;
 
-    if (cit.k < cri.nq) {
-      // ------------------------- quantized tile -----------------------------
-      const int nsub = KAXIS ? g.g_k / 16 : 1;
-      const int tile_start = cit.k * g.tileT;
+    if (it.k < ri.nq) {
+      const int T0 = it.k * pp.sup;
+      const int valid_unit = min(pp.sup, ri.qa - T0);
       if (KAXIS) {
-        // q' = q * s_channel for this key group (scales striped over its pages)
-        float xq[32];
-        float zdot = 0.0f;
+        // q' = q * s_channel for the unit's key groups, shared by the 4 warps
+        const int buf = chan_units++ & 1;
+        const int ngv = (valid_unit + g.g_k - 1) >> g.lg_gk;
+        const int f = 32 * (lane >> 3) + 4 * (lane & 7);
+        const int lg_ppg = g.lg_gk - g.lg_P;   // pages per key group, log2
+        for (int gi = 0; gi < ngv && !aborted; ++gi) {
+          const uint8_t* km = stg + ((gi << lg_ppg) + (f >> g.lg_kslice)) * g.chunk_used + g.off_Km;
+          const int off = f & (g.kslice - 1);
+          float sc[4];
+          meta4(km, off, g.es, sc);
+          uint32_t h0, l0, h1, l1;
+          split2(qv[0] * sc[0], qv[1] * sc[1], h0, l0);
+          split2(qv[2] * sc[2], qv[3] * sc[3], h1, l1);
+          uint8_t* qb = smem + L.qbuf + (buf * pp.ngr + gi) * kQbufBytes;
+          const int lane_hi = 4 * (2 * warp) + (lane >> 3);       // (gq = 2 * head, tq)
+          const int kk = 2 * (lane & 7);
+          *reinterpret_cast<uint2*>(qb + (lane_hi * 16 + kk) * 4) = make_uint2(h0, h1);
+          *reinterpret_cast<uint2*>(qb + ((lane_hi + 4) * 16 + kk) * 4) = make_uint2(l0, l1);
+          if (ASYM) {
+            float zc[4];
+            meta4(km, g.kslice + off, g.es, zc);
+            float dz = qv[0] * zc[0] + qv[1] * zc[1] + qv[2] * zc[2] + qv[3] * zc[3];
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          const int f0 = 32 * tq + 8 * c4;
-          const uint8_t* km = stg + (f0 / g.kslice) * g.chunk_used + g.off_Km;
-          const int off = f0 % g.kslice;
-#pragma unroll
-          for (int m = 0; m < 8; ++m) {
-            const float s = vmeta(km, off + m, g.es);
-            xq[8 * c4 + m] = qf[8 * c4 + m] * s;
-            if (ASYM) zdot = fmaf(qf[8 * c4 + m], vmeta(km, g.kslice + off + m, g.es), zdot);
+            for (int o = 1; o < 32; o <<= 1) dz += __shfl_xor_sync(0xffffffffu, dz, o);
+            if (lane == 0)
+              reinterpret_cast<float*>(smem + L.bias + (buf * pp.ngr + gi) * kBiasBytes)[warp] = dz;
           }
         }
-        make_bq(xq);
-        bq_holds_q = false;
-        if (ASYM) {
-          zdot += __shfl_xor_sync(0xffffffffu, zdot, 1);
-          zdot += __shfl_xor_sync(0xffffffffu, zdot, 2);
-          bias_t = C * __shfl_sync(0xffffffffu, zdot, 8 * tq);   // lane (gq=2tq, 0): head tq
-        }
-      }
-#pragma unroll 1
-      for (int sb = 0; sb < nsub; ++sb) {
-        const int pg = KAXIS ? sb / (g.P / 16) : 0;
-        const int us = KAXIS ? sb % (g.P / 16) : 0;
-        const uint8_t* cb = stg + pg * g.chunk_used;
-        const uint8_t* ksub = cb + us * g.sub_bytes;
-        const uint8_t* vsub = KAXIS ? cb + g.off_V + us * g.sub_bytes : stg + g.sub_bytes;
-        const uint8_t* vms = KAXIS ? cb + g.off_Vm + 16 * us * g.nvg * g.es : stg + 2 * g.sub_bytes;
-        const uint8_t* vmz = KAXIS ? cb + g.off_Vm + (g.P + 16 * us) * g.nvg * g.es
-                                   : stg + 2 * g.sub_bytes + 16 * g.nvg * g.es;
-        const uint8_t* kms = stg + 2 * g.sub_bytes + g.vm16;     // token axis only
-        const uint8_t* kmz = kms + 16 * g.nkg * g.es;
-
-        // scores
-        uint32_t wa[BITS], wb[BITS];
-        load_key_words<BITS, SGN>(ksub, gq, tq, wa, wb);
-        float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-        float s0 = 0.0f, s1 = 0.0f;
-        const int ks_per_group = KAXIS ? 8 : g.g_k / 16;
+        consumer_sync();
+        int loaded = -1;
+        for (int i = 0; i < pp.spw && !aborted; ++i) {
+          const int tok0 = 16 * (warp * pp.spw + i);
+          if (tok0 >= valid_unit) break;
+          const int gi = tok0 >> g.lg_gk;
+          if (gi != loaded) {
+            const uint4* qb = reinterpret_cast<const uint4*>(smem + L.qbuf + (buf * pp.ngr + gi) * kQbufBytes +
+                                                             lane * 64);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          uint32_t a0, a1, a2, a3;
-          key_frag<BITS, SGN>(wa, wb, j, a0, a1, a2, a3);
-          mma_bf16(acc, a0, a1, a2, a3, bq[j][0], bq[j][1]);
-          if ((j + 1) % ks_per_group == 0) {
-            if (KAXIS) {
-              s0 = acc[0] + acc[1];
-              s1 = acc[2] + acc[3];
-            } else {
-              const int gi = j / ks_per_group;
-              const float k0 = vmeta(kms, gq * g.nkg + gi, g.es);
-              const float k1 = vmeta(kms, (gq + 8) * g.nkg + gi, g.es);
-              s0 = fmaf(k0, acc[0] + acc[1], s0);
-              s1 = fmaf(k1, acc[2] + acc[3], s1);
-              if (ASYM) {
-                s0 = fmaf(vmeta(kmz, gq * g.nkg + gi, g.es), qsum[gi & 3], s0);
-                s1 = fmaf(vmeta(kmz, (gq + 8) * g.nkg + gi, g.es), qsum[gi & 3], s1);
-              }
-              acc[0] = acc[1] = acc[2] = acc[3] = 0.0f;
+            for (int v = 0; v < 4; ++v) {
+              const uint4 x = qb[v];
+              bq[2 * v][0] = x.x; bq[2 * v][1] = x.y; bq[2 * v + 1][0] = x.z; bq[2 * v + 1][1] = x.w;
             }
+            bias_t = ASYM ? C * reinterpret_cast<const float*>(smem + L.bias + (buf * pp.ngr + gi) *
+                                                                                  kBiasBytes)[min(tq, g.G - 1)]
+                          : 0.0f;
+            loaded = gi;
+            bq_holds_q = false;
           }
+          const int pg = tok0 >> g.lg_P, us = (tok0 & (g.P - 1)) >> 4;
+          const uint8_t* cb = stg + pg * g.chunk_used;
+          Sub sb;
+          sb.k = cb + us * g.sub_bytes;
+          sb.v = cb + g.off_V + us * g.sub_bytes;
+          sb.vms = cb + g.off_Vm + 16 * us * g.nvg * g.es;
+          sb.vmz = cb + g.off_Vm + (g.P + 16 * us) * g.nvg * g.es;
+          sb.kms = sb.kmz = nullptr;
+          process_sub(sb, valid_unit - tok0);
         }
-        s0 = fmaf(s0, C, bias_t);
-        s1 = fmaf(s1, C, bias_t);
-        const int valid = cri.qa - (tile_start + 16 * sb);
-        if (gq >= valid) s0 = -INFINITY;
-        if (gq + 8 >= valid) s1 = -INFINITY;
-
-        float p0, p1;
-        softmax_step(st, s0, s1, p0, p1);
-
-        // value product: P' V_hat, p' = p * s_value(token, group)
-        const int sa = 8 * tq + hh, sbl = sa + 4;
-        const float pa0 = __shfl_sync(0xffffffffu, p0, sa);
-        const float pa1 = __shfl_sync(0xffffffffu, p1, sa);
-        const float pb0 = __shfl_sync(0xffffffffu, p0, sbl);
-        const float pb1 = __shfl_sync(0xffffffffu, p1, sbl);
-        uint32_t vw[2 * BITS];
-        load_value_words<BITS>(vsub, lane, vw);
-        uint32_t b0 = 0, b1 = 0;
-        float zs = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          if (i % mt_per_vg == 0) {
-            const int gi = i / mt_per_vg;
-            const int n = g.nvg;
-            pv_bfrag(pa0, pb0, pa1, pb1, vmeta(vms, (2 * tq) * n + gi, g.es),
-                     vmeta(vms, (2 * tq + 1) * n + gi, g.es), vmeta(vms, (2 * tq + 8) * n + gi, g.es),
-                     vmeta(vms, (2 * tq + 9) * n + gi, g.es), is_lo, dead_col, b0, b1);
-            if (ASYM) zs = p0 * vmeta(vmz, gq * n + gi, g.es) + p1 * vmeta(vmz, (gq + 8) * n + gi, g.es);
-          }
-          uint32_t a0, a1, a2, a3;
-          value_frag<BITS, SGN>(vw, i, a0, a1, a2, a3);
-          mma_bf16(st.o[i], a0, a1, a2, a3, b0, b1);
-          if (ASYM) st.zacc[i] += zs;
+      } else if (!aborted) {
+        const int tok0 = 16 * warp;
+        if (tok0 < valid_unit) {
+          const uint8_t* sbase = stg + warp * pp.qsub;
+          Sub sb;
+          sb.k = sbase;
+          sb.v = sbase + g.sub_bytes;
+          sb.vms = sbase + 2 * g.sub_bytes;
+          sb.vmz = sb.vms + 16 * g.nvg * g.es;
+          sb.kms = sbase + 2 * g.sub_bytes + g.vm16;
+          sb.kmz = sb.kms + 16 * g.nkg * g.es;
+          process_sub(sb, valid_unit - tok0);
         }
       }
-    } else {
-      // ------------------------- BF16 residual tile -------------------------
-      if (!bq_holds_q) {
-        // B operand of q itself (exact in bf16: lo columns are zero)
-        float qv[32];
-        load_q(cit.i, cit.h, qv);
-        make_bq(qv);
-        bq_holds_q = true;
-      }
-      const uint32_t kaddr = smem_addr(stg), vaddr = kaddr + 16 * D * 2;
-      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int mi = lane >> 3;   // matrix 0..3: (rows 0-7 | 8-15) x (cols 0-7 | 8-15)
-        const int r = (lane & 7) + 8 * (mi & 1), c = 16 * j + 8 * (mi >> 1);
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4(kaddr + (r * D + c) * 2, a0, a1, a2, a3);
-        mma_bf16(acc, a0, a1, a2, a3, bq[j][0], bq[j][1]);
-      }
-      float s0 = (acc[0] + acc[1]) * C, s1 = (acc[2] + acc[3]) * C;
-      const int valid = cri.ra - 16 * (cit.k - cri.nq);
-      if (gq >= valid) s0 = -INFINITY;
-      if (gq + 8 >= valid) s1 = -INFINITY;
-      float p0, p1;
-      softmax_step(st, s0, s1, p0, p1);
-      const int sa = 8 * tq + hh, sbl = sa + 4;
-      const float pa0 = __shfl_sync(0xffffffffu, p0, sa);
-      const float pa1 = __shfl_sync(0xffffffffu, p1, sa);
-      const float pb0 = __shfl_sync(0xffffffffu, p0, sbl);
-      const float pb1 = __shfl_sync(0xffffffffu, p1, sbl);
-      uint32_t b0, b1;
-      pv_bfrag(pa0, pb0, pa1, pb1, 1.0f, 1.0f, 1.0f, 1.0f, is_lo, dead_col, b0, b1);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int mi = lane >> 3;   // (tok 0-7 | 8-15) x (ch +0 | +8) -> a0..a3
-        const int r = (lane & 7) + 8 * (mi >> 1), c = 16 * i + 8 * (mi & 1);
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4_t(vaddr + (r * D + c) * 2, a0, a1, a2, a3);
-        mma_bf16(st.o[i], a0, a1, a2, a3, b0, b1);
+    } else if (!aborted) {
+      const int r = it.k - ri.nq;
+      if ((r & (kDecodeWarps - 1)) == warp) {
+        if (!bq_holds_q) {
+          load_bq_from_q(it.i, it.h);
+          bq_holds_q = true;
+          bias_t = 0.0f;
+        }
+        process_window(stg, ri.ra - 16 * r);
       }
     }
 
-    // release the stage and refill it with the tile nstages ahead
+    // release the stage to the producer
     fence_proxy_async();
     __syncwarp();
-    if (lane == 0 && issued < u1) {
-      issue_tile<ASYM, KAXIS>(a, pit, pri, stage0 + slot * a.stage_bytes, bar0 + 8 * slot);
-      if (it_next(pit, s_pre, a.B, g.h_kv) && issued + 1 < u1) pri = row_info(a, pit.i, false);
-      ++issued;
-    }
-    if (it_next(cit, s_pre, a.B, g.h_kv) && u + 1 < u1) cri = row_info(a, cit.i, false);
+    if (lane == 0) mbar_arrive(empty0 + 8 * s);
+    if (++s == pp.nstages) { s = 0; ph ^= 1u; }
+    if (it_next(it, s_pre, a.B, g.h_kv) && n + 1 < N) ri = row_info(a, it.i, false);
   }
-
-  if (timed_out) {
-    if (lane == 0) atomicOr(a.err, KVQ_DEVERR_TIMEOUT);
-    // drain this warp's copies still in flight (bounded), then leave
-    for (int s = 0; s < a.nstages; ++s) {
-      // parity of the most recent phase issued on stage s is unknown here;
-      // poll both and stop at the limit
-      (void)mbar_wait_bounded(bar0 + 8 * s, 0, kWaitPolls >> 4);
-      (void)mbar_wait_bounded(bar0 + 8 * s, 1, kWaitPolls >> 4);
-    }
-    return;
-  }
-  if (cur_pair >= 0) emit(cur_pair / g.h_kv, cur_pair % g.h_kv);
+  if (!aborted && cur_pair >= 0) emit(cur_pair / g.h_kv, cur_pair % g.h_kv);
 }
 
-// Merge the per-warp partials of each (row, kv head) by log-sum-exp.
-__global__ void __launch_bounds__(128) reduce_kernel(const __grid_constant__ DecodeArgs a) {
+// Merge: one CTA per (row, kv head, query head), one thread per channel.  The
+// records of a pair are the consumer warps of every CTA whose range holds its
+// units, taken in CTA order (a fixed summation order).
+constexpr int kMergeThreads = 128;
+constexpr int kMaxRecords = kDecodeWarps * kMaxDecodeGrid;
+
+__global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_constant__ DecodeArgs a) {
   constexpr int D = kD;
+  __shared__ int32_t s_cta[kMaxDecodeGrid];
+  __shared__ float s_w[kMaxRecords];
+  __shared__ int32_t s_cnt[kMergeThreads / 32];
+  __shared__ float s_red[kMergeThreads / 32];
   const Geo& g = a.g;
-  const int p = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int G = g.G;
+  const int p = blockIdx.x / G, hd = blockIdx.x % G;
   const int i = p / g.h_kv, h = p % g.h_kv;
   const int32_t* pre = a.prefix;
   const int n = pre[i + 1] - pre[i];
-  const int64_t U = int64_t(pre[a.B]) * g.h_kv;
-  for (int idx = threadIdx.x; idx < g.G * D; idx += blockDim.x) {
-    const int hd = idx / D, c = idx % D;
-    float* out = a.out + (int64_t(i) * g.h_q + h * g.G + hd) * D + c;
-    if (n == 0) {
-      *out = 0.0f;
-      continue;
-    }
-    // warps whose ranges hold this pair's tiles: start at the owner of its
-    // first tile and jump from range end to range end (warps with empty
-    // ranges in between own nothing and wrote nothing)
-    const int64_t ua = int64_t(pre[i]) * g.h_kv + int64_t(h) * n, ub = ua + n - 1;
-    const int64_t w0 = ((ua + 1) * a.nw - 1) / U, w1 = ((ub + 1) * a.nw - 1) / U;
-    auto next_warp = [&](int64_t w) {
-      const int64_t end = ((w + 1) * U) / a.nw;     // first tile after warp w's range
-      return ((end + 1) * a.nw - 1) / U;
-    };
-    float M = -INFINITY;
-    for (int64_t w = w0;; w = next_warp(w)) {
-      M = fmaxf(M, a.partials[((p + w) * g.G + hd) * (D + 2)]);
-      if (w >= w1) break;
-    }
-    float num = 0.0f, den = 0.0f;
-    for (int64_t w = w0;; w = next_warp(w)) {
-      const float* rec = a.partials + ((p + w) * g.G + hd) * (D + 2);
-      const float sc = fast_exp2(rec[0] - M);
-      den = fmaf(sc, rec[1], den);
-      num = fmaf(sc, rec[2 + c], num);
-      if (w >= w1) break;
-    }
-    *out = num / den;
+  float* out = a.out + (int64_t(i) * g.h_q + h * G + hd) * D;
+  if (n == 0) {
+    out[tid] = 0.0f;
+    return;
   }
+  const int64_t U = int64_t(pre[a.B]) * g.h_kv;
+  const int64_t GR = a.grid;
+  const int64_t ua = int64_t(pre[i]) * g.h_kv + int64_t(h) * n, ub = ua + n - 1;
+  const int64_t k0 = ((ua + 1) * GR - 1) / U, k1 = ((ub + 1) * GR - 1) / U;
+  // CTAs with non-empty ranges from k0 to k1, in order
+  int count = 0;
+  for (int64_t base = k0; base <= k1; base += kMergeThreads) {
+    const int64_t k = base + tid;
+    const bool live = k <= k1 && (k * U) / GR < ((k + 1) * U) / GR;
+    const uint32_t m = __ballot_sync(0xffffffffu, live);
+    if (lane == 0) s_cnt[w] = __popc(m);
+    __syncthreads();
+    int before = count;
+    for (int q = 0; q < w; ++q) before += s_cnt[q];
+    if (live) s_cta[before + __popc(m & ((1u << lane) - 1u))] = int32_t(k);
+    int tot = 0;
+    for (int q = 0; q < kMergeThreads / 32; ++q) tot += s_cnt[q];
+    __syncthreads();
+    count += tot;
+  }
+  const int nrec = count * kDecodeWarps;
+  auto rec_of = [&](int r) {
+    const int64_t slot = (int64_t(p) + s_cta[r / kDecodeWarps]) * kDecodeWarps + (r % kDecodeWarps);
+    return a.partials + (slot * G + hd) * (D + 2);
+  };
+  float M = -INFINITY;
+  for (int r = tid; r < nrec; r += kMergeThreads) M = fmaxf(M, rec_of(r)[0]);
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  if (lane == 0) s_red[w] = M;
+  __syncthreads();
+  M = s_red[0];
+  for (int q = 1; q < kMergeThreads / 32; ++q) M = fmaxf(M, s_red[q]);
+  __syncthreads();
+  float den = 0.0f;
+  for (int r = tid; r < nrec; r += kMergeThreads) {
+    const float* rec = rec_of(r);
+    const float wgt = M == -INFINITY ? 0.0f : fast_exp2(rec[0] - M);
+    s_w[r] = wgt;
+    den = fmaf(wgt, rec[1], den);
+  }
+  for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  if (lane == 0) s_red[w] = den;
+  __syncthreads();
+  den = 0.0f;
+  for (int q = 0; q < kMergeThreads / 32; ++q) den += s_red[q];
+  float num = 0.0f;
+  for (int r = 0; r < nrec; ++r) num = fmaf(s_w[r], rec_of(r)[2 + tid], num);
+  out[tid] = den > 0.0f ? num / den : 0.0f;
 }
 
 template <int BITS, int ASYM, int KAXIS>
@@ -709,13 +873,6 @@ const void* kernel_of() {
 }
 
 }  // namespace
-
-int decode_prefix_bytes(int B) { return ((B + 1 + 32) * 4 + 127) / 128 * 128; }
-
-size_t decode_smem_bytes(int B, int nstages, int stage_bytes) {
-  return size_t(decode_prefix_bytes(B)) + size_t(kDecodeWarps) * nstages * stage_bytes +
-         size_t(kDecodeWarps) * nstages * 8;
-}
 
 const void* decode_kernel_ptr(const Geo& g) {
   const int key = (g.bits == 8 ? 0 : g.bits == 4 ? 1 : 2) * 4 + g.asym * 2 + g.k_axis;
@@ -735,20 +892,60 @@ const void* decode_kernel_ptr(const Geo& g) {
   }
 }
 
-cudaError_t launch_decode(const DecodeArgs& a, int grid, size_t smem, cudaStream_t s,
-                          cudaEvent_t between, int* launches) {
+size_t decode_smem_bytes(const Geo& g, const DecodePipe& p, int B) {
+  (void)g;
+  return size_t(smem_layout(B, p).total);
+}
+
+size_t decode_partials_bytes(const Geo& g, int B, int grid) {
+  return (size_t(B) * g.h_kv + size_t(grid)) * kDecodeWarps * g.G * (kD + 2) * sizeof(float);
+}
+
+cudaError_t plan_decode(const Geo& g, int max_B, DecodePipe* out) {
+  DecodePipe p{};
+  p.sup = g.k_axis ? (g.g_k > 64 ? g.g_k : 64) : 64;
+  p.spw = p.sup / 64;
+  p.lg_sup = p.sup == 128 ? 7 : 6;
+  p.ngr = g.k_axis ? (p.sup / g.g_k) : 1;
+  p.qsub = g.k_axis ? 0 : 2 * g.sub_bytes + g.vm16 + g.km16;
+  const int qunit = g.k_axis ? (p.sup / g.P) * g.chunk_used : kDecodeWarps * p.qsub;
+  const int res = g.R ? 2 * 16 * kD * 2 : 0;
+  p.stage_bytes = (((qunit > res ? qunit : res) + 127) / 128) * 128;
+  int dev = 0, max_optin = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e != cudaSuccess) return e;
+  // aim for three resident CTAs per SM: about 72 KB of shared memory each
+  p.nstages = 6;
+  while (p.nstages > 2 && size_t(smem_layout(max_B, p).total) > size_t(72 * 1024)) --p.nstages;
+  while (p.nstages > 1 && size_t(smem_layout(max_B, p).total) > size_t(max_optin)) --p.nstages;
+  const size_t smem = size_t(smem_layout(max_B, p).total);
+  if (smem > size_t(max_optin)) return cudaErrorInvalidConfiguration;
+  const void* kern = decode_kernel_ptr(g);
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&p.ctas_per_sm, kern, kDecodeThreads, smem);
+  if (e != cudaSuccess) return e;
+  if (p.ctas_per_sm < 1) return cudaErrorInvalidConfiguration;
+  *out = p;
+  return cudaSuccess;
+}
+
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s, cudaEvent_t between, int* launches) {
   const void* k = decode_kernel_ptr(a.g);
   void* args[] = {const_cast<DecodeArgs*>(&a)};
-  cudaError_t e = cudaLaunchKernel(k, dim3(grid), dim3(kDecodeWarps * 32), args, smem, s);
+  const size_t smem = decode_smem_bytes(a.g, a.pipe, a.B);
+  cudaError_t e = cudaLaunchKernel(k, dim3(a.grid), dim3(kDecodeThreads), args, smem, s);
   if (e != cudaSuccess) return e;
   ++*launches;
   if (between) {
     e = cudaEventRecord(between, s);
     if (e != cudaSuccess) return e;
   }
-  const int pairs = a.B * a.g.h_kv;
-  if (pairs == 0) return cudaSuccess;
-  e = cudaLaunchKernel(reinterpret_cast<const void*>(&reduce_kernel), dim3(pairs), dim3(128), args, 0, s);
+  const int items = a.B * a.g.h_kv * a.g.G;
+  if (items == 0) return cudaSuccess;
+  e = cudaLaunchKernel(reinterpret_cast<const void*>(&merge_kernel), dim3(items), dim3(kMergeThreads), args, 0, s);
   if (e == cudaSuccess) ++*launches;
   return e;
 }

@@ -12,7 +12,8 @@
 namespace kvq {
 
 constexpr int kD = 128;            // head dimension supported by the kernels
-constexpr int kDecodeWarps = 4;    // warps per decode CTA (independent pipelines)
+constexpr int kDecodeWarps = 4;    // consumer warps per decode CTA (plus one producer warp)
+constexpr int kDecodeThreads = (kDecodeWarps + 1) * 32;
 constexpr int kFlushThreads = 256;
 constexpr int kMaxPagesPerGroup = 8;
 // flush plan entry: seq, group, n_pages, blocks[kMaxPagesPerGroup]
@@ -33,6 +34,7 @@ struct Geo {
   int64_t chunk_bytes, block_bytes;
   int num_blocks, max_seqs, mbps;
   int tileT;                // tokens per quantized decode tile
+  int lg_P, lg_gk, lg_kslice;   // log2 of page, g_k and kslice (powers of two)
   int vm16, km16;           // token-axis stage: metadata bytes of 16 rows
   int qtile_bytes;          // bytes staged for one quantized tile
 };
@@ -53,6 +55,18 @@ struct DevState {
   uint32_t* err;
 };
 
+// Shape of the decode pipeline for a format (see kvq_decode.cu).
+struct DecodePipe {
+  int sup;          // tokens per quantized work unit (64, or g_k when larger)
+  int lg_sup;       // log2(sup)
+  int spw;          // 16-token sub-tiles per consumer warp in a unit (sup / 64)
+  int ngr;          // key groups per unit (channel axis), 1 on the token axis
+  int qsub;         // token axis: bytes of one staged 16-token sub-tile
+  int stage_bytes;  // one stage: a quantized unit or a 16-token BF16 window tile
+  int nstages;
+  int ctas_per_sm;  // resident CTAs per SM at the largest batch
+};
+
 struct DecodeArgs {
   const uint8_t* pool;
   const uint16_t* kres;
@@ -65,15 +79,13 @@ struct DecodeArgs {
   const int32_t* stored_len;
   const uint16_t* q;
   float* out;
-  float* partials;
+  float* partials;            // [(B * h_kv + grid) * kDecodeWarps * G][D + 2]
   int32_t* prefix;            // [B + 1], written by CTA 0
   uint32_t* err;
   int32_t B;
-  int32_t nstages;
-  int32_t stage_bytes;
-  int32_t pre_bytes;          // dynamic smem bytes of the prefix table
-  int32_t nw;                 // total warps of the launch
+  int32_t grid;
   float qk_scale;             // log2(e) / sqrt(D)
+  DecodePipe pipe;
   Geo g;
 };
 
@@ -90,10 +102,15 @@ cudaError_t launch_quant_token(const Geo& g, const DevState& d, const PlanView& 
                                int* launches);
 
 const void* decode_kernel_ptr(const Geo& g);
-cudaError_t launch_decode(const DecodeArgs& a, int grid, size_t smem, cudaStream_t s,
-                          cudaEvent_t between, int* launches);
-size_t decode_smem_bytes(int B, int nstages, int stage_bytes);
-int decode_prefix_bytes(int B);
+// Sizes the pipeline for batches up to max_B on the current device, sets the
+// kernel's shared-memory limit and finds its residency.
+cudaError_t plan_decode(const Geo& g, int max_B, DecodePipe* out);
+size_t decode_smem_bytes(const Geo& g, const DecodePipe& p, int B);
+size_t decode_partials_bytes(const Geo& g, int B, int grid);
+// Launches the attention kernel and the merge; `between` (optional) is
+// recorded between them.
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s, cudaEvent_t between, int* launches);
+constexpr int kMaxDecodeGrid = 1024;
 
 // Fixed decode scratch of kvq_decode_attn_noalloc (kvq_noalloc.cu).
 size_t noalloc_scratch_bytes();

@@ -17,7 +17,7 @@
 namespace kvq {
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;   // 4 MiB per device
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB per device
 
 __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
 

@@ -59,7 +59,8 @@ kvq_status validate(const kvq_config* c) {
   const int G = c->h_q / c->h_kv;
   if (G != 1 && G != 2 && G != 4) return fail(KVQ_ERR_UNSUPPORTED, "h_q / h_kv must be 1, 2 or 4");
   if (c->g_v != 32 && c->g_v != 64 && c->g_v != 128) return fail(KVQ_ERR_UNSUPPORTED, "g_v must be 32, 64 or 128");
-  if (c->page < 16 || c->page % 16 != 0) return fail(KVQ_ERR_INVALID_ARG, "page must be a positive multiple of 16");
+  if (c->page < 16 || (c->page & (c->page - 1)) != 0)
+    return fail(KVQ_ERR_INVALID_ARG, "page must be a power of two >= 16");
   if (c->k_axis == KVQ_AXIS_TOKEN) {
     if (c->g_k != 32 && c->g_k != 64 && c->g_k != 128)
       return fail(KVQ_ERR_UNSUPPORTED, "token-axis g_k must be 32, 64 or 128");
@@ -112,6 +113,10 @@ kvq::Geo make_geo(const kvq_config& c) {
   g.max_seqs = c.max_seqs;
   g.mbps = c.max_blocks_per_seq;
   g.tileT = c.k_axis == KVQ_AXIS_CHANNEL ? c.g_k : 16;
+  auto lg = [](int v) { int r = 0; while ((1 << r) < v) ++r; return r; };
+  g.lg_P = lg(c.page);
+  g.lg_gk = lg(c.g_k);
+  g.lg_kslice = g.kslice ? lg(g.kslice) : 0;
   g.vm16 = int(align_up(size_t(16) * g.nvg * g.es * A, 16));
   g.km16 = int(align_up(size_t(16) * g.nkg * g.es * A, 16));
   g.qtile_bytes = c.k_axis == KVQ_AXIS_CHANNEL ? (c.g_k / c.page) * g.chunk_used
@@ -160,9 +165,7 @@ struct kvq_handle_s {
   int sm_count = 0;
   int decode_ctas = 0;
   int decode_override = 0;
-  int nstages = 0;
-  int stage_bytes = 0;
-  size_t decode_smem = 0;
+  kvq::DecodePipe pipe{};
   size_t bytes_workspace = 0;
   cudaEvent_t decode_event = nullptr;
   int launches = 0;
@@ -297,31 +300,14 @@ kvq_status create_device(kvq_handle h) {
   KVQ_CUDA(cudaMemset(h->d_err, 0, sizeof(uint32_t)));
   for (auto& s : h->slots) KVQ_CUDA(cudaEventCreateWithFlags(&s.ev, cudaEventDisableTiming));
 
-  // decode pipeline: per-warp ring of stages, two resident CTAs per SM if possible
-  const int res_tile = c.residual ? 2 * 16 * kvq::kD * 2 : 0;
-  h->stage_bytes = int(align_up(size_t(std::max(g.qtile_bytes, res_tile)), 128));
-  const size_t budget = 113 * 1024;
-  const size_t fixed = size_t(kvq::decode_prefix_bytes(c.max_seqs));
-  int ns = int((budget > fixed ? budget - fixed : 0) / (size_t(kvq::kDecodeWarps) * (h->stage_bytes + 8)));
-  ns = std::max(1, std::min(ns, 8));
-  size_t smem = kvq::decode_smem_bytes(c.max_seqs, ns, h->stage_bytes);
-  int max_optin = 0;
-  KVQ_CUDA(cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, h->device));
-  while (smem > size_t(max_optin) && ns > 1) smem = kvq::decode_smem_bytes(c.max_seqs, --ns, h->stage_bytes);
-  if (smem > size_t(max_optin)) return fail(KVQ_ERR_UNSUPPORTED, "decode tile does not fit in shared memory");
-  h->nstages = ns;
-  h->decode_smem = smem;
-  const void* kern = kvq::decode_kernel_ptr(g);
-  KVQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
-  int per_sm = 0;
-  KVQ_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kvq::kDecodeWarps * 32, smem));
-  if (per_sm < 1) return fail(KVQ_ERR_UNSUPPORTED, "decode kernel cannot be resident");
-  h->decode_ctas = h->sm_count * per_sm;
+  // decode pipeline: stage ring of a producer warp and four consumer warps
+  cudaError_t pe = kvq::plan_decode(g, c.max_seqs, &h->pipe);
+  if (pe == cudaErrorInvalidConfiguration) return fail(KVQ_ERR_UNSUPPORTED, "decode tile does not fit on this device");
+  KVQ_CUDA(pe);
+  h->decode_ctas = std::min(h->sm_count * h->pipe.ctas_per_sm, kvq::kMaxDecodeGrid);
 
   // workspace: split partials for up to max_seqs rows and any grid we launch
-  const int max_grid = std::max(h->decode_ctas, 4096);
-  const size_t recs = (size_t(c.max_seqs) * c.h_kv + size_t(max_grid) * kvq::kDecodeWarps) * g.G;
-  h->part_bytes = recs * (kvq::kD + 2) * sizeof(float);
+  h->part_bytes = kvq::decode_partials_bytes(g, c.max_seqs, kvq::kMaxDecodeGrid);
   KVQ_CUDA(cudaMalloc(&h->d_part, h->part_bytes));
   // NaN-fill: a merge that ever read a slot no warp wrote shows up as NaN
   KVQ_CUDA(cudaMemset(h->d_part, 0xFF, h->part_bytes));
@@ -549,15 +535,11 @@ kvq_status kvq_decode_attn(kvq_handle h, const void* q_bf16, const int32_t* bloc
   a.prefix = h->d_prefix;
   a.err = h->d_err;
   a.B = batch;
-  a.nstages = h->nstages;
-  a.stage_bytes = h->stage_bytes;
-  a.pre_bytes = kvq::decode_prefix_bytes(batch);
-  const int grid = h->decode_override > 0 ? h->decode_override : h->decode_ctas;
-  a.nw = grid * kvq::kDecodeWarps;
+  a.grid = h->decode_override > 0 ? h->decode_override : h->decode_ctas;
   a.qk_scale = float(1.4426950408889634 / std::sqrt(double(kvq::kD)));
+  a.pipe = h->pipe;
   a.g = h->geo;
-  const size_t smem = kvq::decode_smem_bytes(batch, h->nstages, h->stage_bytes);
-  KVQ_CUDA(kvq::launch_decode(a, grid, smem, stream, h->decode_event, &h->launches));
+  KVQ_CUDA(kvq::launch_decode(a, stream, h->decode_event, &h->launches));
   return KVQ_OK;
 }
 
@@ -685,7 +667,7 @@ kvq_status kvq_set_decode_event(kvq_handle h, void* event) {
 
 kvq_status kvq_set_decode_grid(kvq_handle h, int32_t ctas) {
   if (!h) return fail(KVQ_ERR_INVALID_ARG, "handle is null");
-  if (ctas < 0 || ctas > 4096) return fail(KVQ_ERR_INVALID_ARG, "ctas must be in [0, 4096]");
+  if (ctas < 0 || ctas > kvq::kMaxDecodeGrid) return fail(KVQ_ERR_INVALID_ARG, "ctas must be in [0, 1024]");
   h->decode_override = ctas;
   return KVQ_OK;
 }
@@ -710,32 +692,19 @@ kvq_status kvq_decode_attn_noalloc(const kvq_config* cfg, const void* pool, cons
   const kvq::Geo g = make_geo(*cfg);
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
 
-  int dev = 0, sms = 0, max_optin = 0;
+  int dev = 0, sms = 0;
   KVQ_CUDA(cudaGetDevice(&dev));
   KVQ_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-  KVQ_CUDA(cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
-  // the same stage sizing as a handle's decode
-  const int res_tile = cfg->residual ? 2 * 16 * kvq::kD * 2 : 0;
-  const int stage_bytes = int(align_up(size_t(std::max(g.qtile_bytes, res_tile)), 128));
-  const size_t budget = 113 * 1024;
-  const size_t fixed = size_t(kvq::decode_prefix_bytes(cfg->max_seqs));
-  int ns = int((budget > fixed ? budget - fixed : 0) / (size_t(kvq::kDecodeWarps) * (stage_bytes + 8)));
-  ns = std::max(1, std::min(ns, 8));
-  size_t smem_max = kvq::decode_smem_bytes(cfg->max_seqs, ns, stage_bytes);
-  while (smem_max > size_t(max_optin) && ns > 1) smem_max = kvq::decode_smem_bytes(cfg->max_seqs, --ns, stage_bytes);
-  if (smem_max > size_t(max_optin)) return fail(KVQ_ERR_UNSUPPORTED, "decode tile does not fit in shared memory");
-  const void* kern = kvq::decode_kernel_ptr(g);
-  KVQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_max)));
-  int per_sm = 0;
-  KVQ_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kvq::kDecodeWarps * 32, smem_max));
-  if (per_sm < 1) return fail(KVQ_ERR_UNSUPPORTED, "decode kernel cannot be resident");
-  const int grid = sms * per_sm;
-  const int nw = grid * kvq::kDecodeWarps;
+  kvq::DecodePipe pipe{};
+  cudaError_t pe = kvq::plan_decode(g, cfg->max_seqs, &pipe);
+  if (pe == cudaErrorInvalidConfiguration) return fail(KVQ_ERR_UNSUPPORTED, "decode tile does not fit on this device");
+  KVQ_CUDA(pe);
+  const int grid = std::min(sms * pipe.ctas_per_sm, kvq::kMaxDecodeGrid);
 
   // scratch layout: [error word | pad to 256][prefix (batch + 1) | pad to 256][partials]
   const size_t off_prefix = 256;
   const size_t off_part = off_prefix + align_up(size_t(batch + 1) * 4, 256);
-  const size_t part_bytes = (size_t(batch) * g.h_kv + size_t(nw)) * g.G * (kvq::kD + 2) * sizeof(float);
+  const size_t part_bytes = kvq::decode_partials_bytes(g, batch, grid);
   if (off_part + part_bytes > kvq::noalloc_scratch_bytes())
     return fail(KVQ_ERR_INVALID_ARG,
                 "batch * h_kv too large for the fixed decode scratch of " +
@@ -762,15 +731,12 @@ kvq_status kvq_decode_attn_noalloc(const kvq_config* cfg, const void* pool, cons
   a.prefix = reinterpret_cast<int32_t*>(base + off_prefix);
   a.err = reinterpret_cast<uint32_t*>(base);
   a.B = batch;
-  a.nstages = ns;
-  a.stage_bytes = stage_bytes;
-  a.pre_bytes = kvq::decode_prefix_bytes(batch);
-  a.nw = nw;
+  a.grid = grid;
   a.qk_scale = float(1.4426950408889634 / std::sqrt(double(kvq::kD)));
+  a.pipe = pipe;
   a.g = g;
   int launches = 0;
-  KVQ_CUDA(kvq::launch_decode(a, grid, kvq::decode_smem_bytes(batch, ns, stage_bytes), stream, nullptr,
-                              &launches));
+  KVQ_CUDA(kvq::launch_decode(a, stream, nullptr, &launches));
   if (error_bits_dev)
     KVQ_CUDA(cudaMemcpyAsync(error_bits_dev, base, sizeof(uint32_t), cudaMemcpyDeviceToDevice, stream));
   return KVQ_OK;

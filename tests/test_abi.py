@@ -137,6 +137,7 @@ def test_fail_alloc_after_and_table_width():
     ("h_q", 3, kvq.KVQ_ERR_INVALID_ARG),
     ("residual", 32, kvq.KVQ_ERR_INVALID_ARG),
     ("page", 24, kvq.KVQ_ERR_INVALID_ARG),
+    ("page", 48, kvq.KVQ_ERR_INVALID_ARG),
     ("page", 128, kvq.KVQ_ERR_UNSUPPORTED),
     ("g_v", 48, kvq.KVQ_ERR_UNSUPPORTED),
     ("num_blocks", 0, kvq.KVQ_ERR_INVALID_ARG),
