@@ -217,11 +217,11 @@ def run_gpu(args, rank, ws, dist):
     dev = torch.device("cuda", torch.cuda.current_device())
     w = workload(args.workload)
     w.seed = w.seed + 1000 * rank        # each replica draws its own inputs
-    total_steps = args.warmup + args.steps
-    dr = Draws(w, steps=2 * total_steps)
+    total_steps = args.warmup + 3 * args.steps   # warm-up, decode pass, attention pass, e2e pass
+    dr = Draws(w, steps=total_steps)
     f = w.fmt
-    nb = pool_blocks(dr.lengths, 2 * total_steps + 2, f.page)
-    mbps = max((L + 2 * total_steps + 2) // f.page + 2 for L in dr.lengths)
+    nb = pool_blocks(dr.lengths, total_steps + 2, f.page)
+    mbps = max((L + total_steps + 2) // f.page + 2 for L in dr.lengths)
     cache = kvq.KVCache(kvq.Format(f.bits, f.asym, f.k_axis, f.g_k, f.g_v, f.scale_fp32,
                                    f.residual, f.page), w.h_q, w.h_kv, max_seqs=w.batch,
                         num_blocks=nb, max_blocks_per_seq=mbps, seed=w.seed,
@@ -235,7 +235,7 @@ def run_gpu(args, rank, ws, dist):
     lens = list(dr.lengths)
     B = w.batch
     ids = np.arange(B, dtype=np.int32)
-    steps_in = [dr.step() for _ in range(2 * total_steps)]
+    steps_in = [dr.step() for _ in range(total_steps)]
     dev_in = [(bf16_dev(k), bf16_dev(v), bf16_dev(q)) for k, v, q in steps_in]
     host_in = [tuple(torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
                      for a in s) for s in steps_in]
@@ -244,11 +244,6 @@ def run_gpu(args, rank, ws, dist):
     out = torch.empty((B, w.h_q, D), dtype=torch.float32, device=dev)
     out_host = torch.empty_like(out, device="cpu").pin_memory()
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    ev_mid = torch.cuda.Event(enable_timing=True)
-    ev_mid.record()               # torch creates the CUDA event on its first record
-    torch.cuda.synchronize()
-    assert ev_mid.cuda_event != 0
-    cache.set_decode_event(ev_mid)
     torch.cuda.synchronize()
     assert cache.sync_status() == 0
 
@@ -279,36 +274,60 @@ def run_gpu(args, rank, ws, dist):
     torch.cuda.synchronize()
     assert cache.sync_status() == 0
 
-    # timed: device-resident inputs
+    # timed: device-resident inputs, the decode call as a user makes it.  The
+    # host enqueues every step before waiting (as a serving loop runs ahead of
+    # the GPU), so the events see device time, not host launch gaps.
+    cache.set_decode_event(None)
     st0 = cache.stats()["kernel_launches"]
     sampler = ClockSampler(torch.cuda.current_device(), enabled=not args.no_clocks)
     time.sleep(0.15 if sampler.proc else 0)
     barrier(dist)
     torch.cuda.synchronize()
-    recs = []
     kv_bytes, app_bytes, seq_tokens = 0, 0, 0
-    for s in range(args.warmup, total_steps):
+    s0 = args.warmup
+    step_evs = []
+    for s in range(s0, s0 + args.steps):
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
         before = list(lens)
         one_step(s, False, evs)
-        evs[2].synchronize()
-        # ev_mid was recorded by the library between the attention kernel and the merge
-        recs.append((evs[0].elapsed_time(evs[1]), evs[1].elapsed_time(ev_mid),
-                     evs[1].elapsed_time(evs[2])))
+        step_evs.append(evs)
         kv_bytes += decode_bytes(w, lens)
         app_bytes += append_bytes(w, before)
         seq_tokens += sum(lens)
     torch.cuda.synchronize()
+    recs = [(e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2])) for e in step_evs]
     barrier(dist)
     launches = cache.stats()["kernel_launches"] - st0
     clocks = sampler.stop()
+    assert cache.sync_status() == 0
+
+    # timed: the attention kernel alone -- the library records an event between
+    # it and the merge (which then runs as a plain launch); one event per step
+    barrier(dist)
+    torch.cuda.synchronize()
+    attn_bytes = 0
+    s0 += args.steps
+    step_evs = []
+    for s in range(s0, s0 + args.steps):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        mid = torch.cuda.Event(enable_timing=True)
+        mid.record()              # creates the CUDA event; the library records it again
+        cache.set_decode_event(mid)
+        one_step(s, False, evs)
+        step_evs.append((evs, mid))
+        attn_bytes += decode_bytes(w, lens)
+    torch.cuda.synchronize()
+    t_attn = sum(e[1].elapsed_time(mid) for e, mid in step_evs)
+    barrier(dist)
+    cache.set_decode_event(None)
     assert cache.sync_status() == 0
 
     # timed: end to end through the C ABI with host buffers
     barrier(dist)
     torch.cuda.synchronize()
     e2e_ms, e2e_bytes = 0.0, 0
-    for s in range(total_steps, total_steps + args.steps):
+    s0 += args.steps
+    for s in range(s0, s0 + args.steps):
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
         one_step(s, True, evs)
         evs[2].synchronize()
@@ -320,8 +339,7 @@ def run_gpu(args, rank, ws, dist):
     cache.close()
 
     t_app = sum(r[0] for r in recs)
-    t_attn = sum(r[1] for r in recs)
-    t_dec = sum(r[2] for r in recs)
+    t_dec = sum(r[1] for r in recs)
     step_ms = t_app + t_dec
     mx = max_over_ranks(dist, [t_app, t_attn, t_dec, step_ms, e2e_ms])
     tot = sum_over_ranks(dist, [kv_bytes, app_bytes, seq_tokens, e2e_bytes])
@@ -329,7 +347,7 @@ def run_gpu(args, rank, ws, dist):
     res = {
         "w": w, "K": K, "ws": ws, "launches": launches, "clocks": clocks,
         "kv_gbs": tot[0] / (mx[2] * 1e-3) / 1e9,
-        "attn_gbs": (kv_bytes / K) / (t_attn / K * 1e-3) / 1e9,
+        "attn_gbs": (attn_bytes / K) / (t_attn / K * 1e-3) / 1e9,
         "attn_us": t_attn / K * 1e3,
         "decode_us": t_dec / K * 1e3,
         "append_us": t_app / K * 1e3,

@@ -40,19 +40,18 @@ namespace kvq {
 namespace {
 
 constexpr uint64_t kWaitNs = 2000000000ull;   // give up on a copy after 2 s
-constexpr int kQbufBytes = 32 * 16 * 4;   // one key group's q' operand: 32 lanes x 16 words
-constexpr int kBiasBytes = 16;            // one key group's zero-point bias of 4 heads
+constexpr int kQbufBytes = 32 * 16 * 4;   // one warp's q' operand: 32 lanes x 16 words
+constexpr int kScoreBytes = 8 * 32 * 4;   // one warp's scores / weights of a 64-token chunk
 
 struct SmemLayout {
-  int stages, qbuf, bias, bars, flag, total;
+  int stages, qbuf, bars, flag, total;
 };
 
 __host__ __device__ inline SmemLayout smem_layout(int B, const DecodePipe& p) {
   SmemLayout L;
   L.stages = ((B + 1 + 32) * 4 + 127) / 128 * 128;      // prefix table + scan scratch
   L.qbuf = L.stages + p.nstages * p.stage_bytes;
-  L.bias = L.qbuf + 2 * p.ngr * kQbufBytes;
-  L.bars = L.bias + 2 * p.ngr * kBiasBytes;
+  L.bars = L.qbuf + kDecodeWarps * (kQbufBytes + kScoreBytes);
   L.flag = L.bars + 2 * p.nstages * 8;
   L.total = L.flag + 16;
   return L;
@@ -151,11 +150,6 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
 }
 
-// Barrier of the four consumer warps only (the producer warp never joins).
-__device__ __forceinline__ void consumer_sync() {
-  asm volatile("bar.sync 1, 128;\n" ::: "memory");
-}
-
 // Bounded wait that also gives up as soon as another warp has aborted.
 __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int32_t* abort_flag) {
   return mbar_wait_bounded(bar, parity, kWaitNs, abort_flag);
@@ -177,30 +171,6 @@ __device__ __forceinline__ void state_reset(State& st) {
   }
   st.m = -INFINITY;
   st.l = 0.0f;
-}
-
-// Online softmax over the two scores (tokens gq, gq+8; head tq) of a 16-token
-// sub-tile; returns their weights relative to the running max.
-__device__ __forceinline__ void softmax_step(State& st, float s0, float s1, float& p0, float& p1) {
-  float mx = fmaxf(s0, s1);
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-  if (mx > st.m + 8.0f) {   // also taken from -inf
-    const float alpha = fast_exp2(st.m - mx);
-    st.l *= alpha;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-#pragma unroll
-      for (int c = 0; c < 4; ++c) st.o[i][c] *= alpha;
-      st.zacc[i] *= alpha;
-    }
-    st.m = mx;
-  }
-  const bool live = st.m != -INFINITY;
-  p0 = live ? fast_exp2(s0 - st.m) : 0.0f;
-  p1 = live ? fast_exp2(s1 - st.m) : 0.0f;
-  st.l += p0 + p1;
 }
 
 // Key words of rows gq and gq + 8 of a packed 16-token sub-tile.
@@ -319,12 +289,51 @@ struct Sub {
   const uint8_t* kmz;
 };
 
-template <int BITS, int ASYM, int KAXIS>
+// The KIVI-style INT4 format (symmetric, keys per channel in groups of 64,
+// values per token in groups of 64, fp16 scales, 16-token pages, a 64-token
+// BF16 window, 4 query heads per kv head) gets its own kernel instance with
+// every geometry field below a compile-time constant, so the per-sub-tile
+// address arithmetic folds into immediates.  The host dispatches to it only
+// when the runtime geometry equals these values field by field.
+struct SpecInt4Kivi {
+  static constexpr int bits = 4, asym = 0, k_axis = 1, g_k = 64, g_v = 64, scale_fp32 = 0, R = 64, P = 16, G = 4;
+  static constexpr int n = 8, row_bytes = 64, sub_bytes = 1024, es = 2, nvg = 2, kslice = 32;
+  static constexpr int off_V = 1024, off_Vm = 2048, off_Km = 2112, chunk_used = 2176;
+  static constexpr int lg_P = 4, lg_gk = 6, lg_kslice = 5;
+};
+
+template <int SPEC>
+__device__ __forceinline__ Geo geo_of(const Geo& rt) {
+  Geo g = rt;
+  if constexpr (SPEC == 1) {
+    using S = SpecInt4Kivi;
+    g.bits = S::bits; g.asym = S::asym; g.k_axis = S::k_axis; g.g_k = S::g_k; g.g_v = S::g_v;
+    g.scale_fp32 = S::scale_fp32; g.R = S::R; g.P = S::P; g.G = S::G; g.n = S::n;
+    g.row_bytes = S::row_bytes; g.sub_bytes = S::sub_bytes; g.es = S::es; g.nvg = S::nvg;
+    g.kslice = S::kslice; g.off_V = S::off_V; g.off_Vm = S::off_Vm; g.off_Km = S::off_Km;
+    g.chunk_used = S::chunk_used; g.lg_P = S::lg_P; g.lg_gk = S::lg_gk; g.lg_kslice = S::lg_kslice;
+  }
+  return g;
+}
+
+bool spec_int4_kivi(const Geo& g) {
+  using S = SpecInt4Kivi;
+  return g.bits == S::bits && g.asym == S::asym && g.k_axis == S::k_axis && g.g_k == S::g_k &&
+         g.g_v == S::g_v && g.scale_fp32 == S::scale_fp32 && g.R == S::R && g.P == S::P && g.G == S::G &&
+         g.n == S::n && g.row_bytes == S::row_bytes && g.sub_bytes == S::sub_bytes && g.es == S::es &&
+         g.nvg == S::nvg && g.kslice == S::kslice && g.off_V == S::off_V && g.off_Vm == S::off_Vm &&
+         g.off_Km == S::off_Km && g.chunk_used == S::chunk_used && g.lg_P == S::lg_P && g.lg_gk == S::lg_gk &&
+         g.lg_kslice == S::lg_kslice;
+}
+
+template <int BITS, int ASYM, int KAXIS, int SPEC>
 __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_constant__ DecodeArgs a) {
   constexpr int D = kD;
   constexpr bool SGN = !ASYM;
+  constexpr int kPair = 1;   // sub-tiles per trip of the chunk loops (2 measured slower)
   extern __shared__ __align__(128) uint8_t smem[];
-  const Geo& g = a.g;
+  const Geo gs = geo_of<SPEC>(a.g);
+  const Geo& g = SPEC ? gs : a.g;   // the generic instances read the geometry from the parameters
   const DecodePipe& pp = a.pipe;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const SmemLayout L = smem_layout(a.B, pp);
@@ -336,6 +345,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
   const uint32_t empty0 = full0 + 8 * pp.nstages;
   volatile int32_t* abort_flag = reinterpret_cast<int32_t*>(smem + L.flag);
 
+  // the merge grid may be scheduled now; it waits for this grid to complete
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+
   // ---- the work list: units per row, prefix over rows ---------------------
   for (int i = tid; i < a.B; i += blockDim.x) {
     const RowInfo ri = row_info(a, i, blockIdx.x == 0);
@@ -344,7 +356,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
   if (tid == 0) {
     for (int s = 0; s < pp.nstages; ++s) {
       mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, kDecodeWarps);
+      mbar_init(empty0 + 8 * s, 1);   // released by the one warp that owns the unit
     }
     *abort_flag = 0;
     mbar_init_fence();
@@ -468,22 +480,28 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
   }
 
   // ------------------------------ consumers -----------------------------------
+  // Consumer warp w owns the units n of the range with n % 4 == w: it waits for
+  // the unit's stage, computes all of it alone and releases the stage.  It
+  // walks every unit of the range to see the pair boundaries, so it leaves one
+  // (m, l, o) record for every pair the CTA touches (empty where it owned no
+  // unit of the pair), which is what the merge reads.
   const int gq = lane >> 2, tq = lane & 3;
   const int hh = gq >> 1;               // head of this lane's B column
   const bool is_lo = gq & 1;            // the column carries the lo part
   const bool dead_col = hh >= g.G;      // padding column (fewer than 4 heads)
   const float C = a.qk_scale;
-  const int vg_shift = __ffs(g.g_v >> 4) - 1;          // channel tiles per value group, log2
+  const int vg_shift = __ffs(g.g_v >> 4) - 1;               // channel tiles per value group, log2
   const int kg_shift = KAXIS ? 3 : __ffs(g.g_k >> 4) - 1;   // k-steps per key group, log2
+  uint32_t* qbw = reinterpret_cast<uint32_t*>(smem + L.qbuf + warp * kQbufBytes);   // this warp's q'
+  float* spw = reinterpret_cast<float*>(smem + L.qbuf + kDecodeWarps * kQbufBytes) + warp * 8 * 32;
 
   State st;
   state_reset(st);
-  uint32_t bq[8][2];          // score B operand (q' hi|lo columns)
-  bool bq_holds_q = false;    // bq carries q itself (token axis, BF16 window)
-  float bias_t = 0.0f;        // zero-point term of head tq for the loaded key group
-  float qv[4] = {0.0f, 0.0f, 0.0f, 0.0f};     // q of head `warp` at this thread's 4 channels
-  float qsum[4] = {0.0f, 0.0f, 0.0f, 0.0f};   // token-axis zero-points: sum of q per group
-  int chan_units = 0;         // channel-axis units seen: picks the q' buffer
+  uint32_t bq[8][2];          // score B operand: q' hi|lo columns, or q itself
+  bool bq_holds_q = false;    // bq carries q (token axis, BF16 window)
+  float bias_t = 0.0f;        // channel-axis zero-points: key bias of head tq for the loaded group
+  uint32_t qw[4][2];          // channel axis: q of head h at key-list channels 4*lane .. 4*lane+3
+  float qsum[4] = {0.0f, 0.0f, 0.0f, 0.0f};   // token-axis zero-points: sum of q per key group
 
   auto qrow = [&](int row, int h, int head) {
     return a.q + (int64_t(row) * g.h_q + h * g.G + min(head, g.G - 1)) * D;
@@ -536,16 +554,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
     bq_holds_q = false;
     bias_t = 0.0f;
     if (KAXIS) {
-      // this thread's share of the q' job: head `warp`, lane group lane>>3, k-step lane&7
-      const uint16_t* qr = qrow(row, h, warp);
-      const int f = 32 * (lane >> 3) + 4 * (lane & 7);
-      const uint32_t t0 = *reinterpret_cast<const uint32_t*>(qr + key_channel(f));
-      const uint32_t t1 = *reinterpret_cast<const uint32_t*>(qr + key_channel(f + 2));
-      const bool live = warp < g.G;
-      qv[0] = live ? __uint_as_float(t0 << 16) : 0.0f;
-      qv[1] = live ? __uint_as_float(t0 & 0xFFFF0000u) : 0.0f;
-      qv[2] = live ? __uint_as_float(t1 << 16) : 0.0f;
-      qv[3] = live ? __uint_as_float(t1 & 0xFFFF0000u) : 0.0f;
+      // this lane's share of the q' job: key-list channels 4*lane .. 4*lane+3 of every head
+      const int f = 4 * lane;
+#pragma unroll
+      for (int h2 = 0; h2 < 4; ++h2) {
+        const uint16_t* qr = qrow(row, h, h2);
+        const bool live = h2 < g.G;
+        qw[h2][0] = live ? *reinterpret_cast<const uint32_t*>(qr + key_channel(f)) : 0u;
+        qw[h2][1] = live ? *reinterpret_cast<const uint32_t*>(qr + key_channel(f + 2)) : 0u;
+      }
     } else {
       load_bq_from_q(row, h);
       bq_holds_q = true;
@@ -560,12 +577,62 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
     }
   };
 
-  // Scores, online softmax and the value product of one 16-token sub-tile.
-  auto process_sub = [&](const Sub& sb, int valid) {
+  // Channel axis: q' = q * s_channel of key group gi of the unit in `stg`, as
+  // this lane's score B operand.  Each lane scales 4 channels of every head and
+  // writes both bf16 parts into the warp's buffer in operand order (16-byte
+  // slots XOR-swizzled so the four 16-byte reads per lane are conflict-free).
+  auto qprime_job = [&](const uint8_t* stg, int gi) {
+    const int f = 4 * lane;
+    const int lg_ppg = g.lg_gk - g.lg_P;   // pages per key group, log2
+    const uint8_t* km = stg + ((gi << lg_ppg) + (f >> g.lg_kslice)) * g.chunk_used + g.off_Km;
+    const int off = f & (g.kslice - 1);
+    float sc[4];
+    meta4(km, off, g.es, sc);
+    float zc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    if (ASYM) meta4(km, g.kslice + off, g.es, zc);
+    const int t0 = lane >> 3, j = lane & 7;
+    float dz[4];
+    __syncwarp();   // every lane has read the previous operand
+#pragma unroll
+    for (int h2 = 0; h2 < 4; ++h2) {
+      const float q0 = __uint_as_float(qw[h2][0] << 16), q1 = __uint_as_float(qw[h2][0] & 0xFFFF0000u);
+      const float q2 = __uint_as_float(qw[h2][1] << 16), q3 = __uint_as_float(qw[h2][1] & 0xFFFF0000u);
+      uint32_t h0, l0, h1, l1;
+      split2(q0 * sc[0], q1 * sc[1], h0, l0);
+      split2(q2 * sc[2], q3 * sc[3], h1, l1);
+      const int thi = 8 * h2 + t0, tlo = thi + 4;   // lanes (gq = 2 h2 | 2 h2 + 1, tq = t0)
+      *reinterpret_cast<uint2*>(qbw + thi * 16 + 4 * ((j >> 1) ^ ((thi >> 1) & 3)) + 2 * (j & 1)) =
+          make_uint2(h0, h1);
+      *reinterpret_cast<uint2*>(qbw + tlo * 16 + 4 * ((j >> 1) ^ ((tlo >> 1) & 3)) + 2 * (j & 1)) =
+          make_uint2(l0, l1);
+      if (ASYM) dz[h2] = q0 * zc[0] + q1 * zc[1] + q2 * zc[2] + q3 * zc[3];
+    }
+    if (ASYM) {
+#pragma unroll
+      for (int h2 = 0; h2 < 4; ++h2)
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) dz[h2] += __shfl_xor_sync(0xffffffffu, dz[h2], o);
+      const int ht = min(tq, g.G - 1);
+      bias_t = C * (ht == 0 ? dz[0] : ht == 1 ? dz[1] : ht == 2 ? dz[2] : dz[3]);
+    }
+    __syncwarp();
+    const uint4* qb = reinterpret_cast<const uint4*>(qbw + lane * 16);
+    const int sw = (lane >> 1) & 3;
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const uint4 x = qb[v ^ sw];
+      bq[2 * v][0] = x.x; bq[2 * v][1] = x.y; bq[2 * v + 1][0] = x.z; bq[2 * v + 1][1] = x.w;
+    }
+    bq_holds_q = false;
+  };
+
+  // Scores of one 16-token quantized sub-tile: tokens gq, gq + 8 for head tq,
+  // scaled into the log2 domain; positions at or past `valid` are -inf.
+  auto score_sub = [&](const Sub& sb, int valid, float& s0, float& s1) {
     uint32_t wa[BITS], wb[BITS];
     load_key_words<BITS>(sb.k, gq, tq, wa, wb);
     float acc0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, acc1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    float s0 = 0.0f, s1 = 0.0f;
+    float r0 = 0.0f, r1 = 0.0f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       uint32_t a0, a1, a2, a3;
@@ -574,31 +641,28 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
       else mma_bf16(acc0, a0, a1, a2, a3, bq[j][0], bq[j][1]);
       if (!KAXIS && ((j + 1) & ((1 << kg_shift) - 1)) == 0) {
         const int gi = j >> kg_shift;
-        const float r0 = acc0[0] + acc0[1] + acc1[0] + acc1[1];
-        const float r1 = acc0[2] + acc0[3] + acc1[2] + acc1[3];
-        s0 = fmaf(meta_at(sb.kms, gq * g.nkg + gi, g.es), r0, s0);
-        s1 = fmaf(meta_at(sb.kms, (gq + 8) * g.nkg + gi, g.es), r1, s1);
+        const float t0 = acc0[0] + acc0[1] + acc1[0] + acc1[1];
+        const float t1 = acc0[2] + acc0[3] + acc1[2] + acc1[3];
+        r0 = fmaf(meta_at(sb.kms, gq * g.nkg + gi, g.es), t0, r0);
+        r1 = fmaf(meta_at(sb.kms, (gq + 8) * g.nkg + gi, g.es), t1, r1);
         if (ASYM) {
-          s0 = fmaf(meta_at(sb.kmz, gq * g.nkg + gi, g.es), qsum[gi & 3], s0);
-          s1 = fmaf(meta_at(sb.kmz, (gq + 8) * g.nkg + gi, g.es), qsum[gi & 3], s1);
+          r0 = fmaf(meta_at(sb.kmz, gq * g.nkg + gi, g.es), qsum[gi & 3], r0);
+          r1 = fmaf(meta_at(sb.kmz, (gq + 8) * g.nkg + gi, g.es), qsum[gi & 3], r1);
         }
 #pragma unroll
         for (int c = 0; c < 4; ++c) acc0[c] = acc1[c] = 0.0f;
       }
     }
     if (KAXIS) {
-      s0 = acc0[0] + acc0[1] + acc1[0] + acc1[1];
-      s1 = acc0[2] + acc0[3] + acc1[2] + acc1[3];
+      r0 = acc0[0] + acc0[1] + acc1[0] + acc1[1];
+      r1 = acc0[2] + acc0[3] + acc1[2] + acc1[3];
     }
-    s0 = fmaf(s0, C, bias_t);
-    s1 = fmaf(s1, C, bias_t);
-    if (gq >= valid) s0 = -INFINITY;
-    if (gq + 8 >= valid) s1 = -INFINITY;
+    s0 = gq < valid ? fmaf(r0, C, bias_t) : -INFINITY;
+    s1 = gq + 8 < valid ? fmaf(r1, C, bias_t) : -INFINITY;
+  };
 
-    float p0, p1;
-    softmax_step(st, s0, s1, p0, p1);
-
-    // value product: P' V_hat with p' = p * s_value(token, group)
+  // Value product of one sub-tile: P' V_hat with p' = p * s_value(token, group).
+  auto pv_sub = [&](const Sub& sb, float p0, float p1, bool live) {
     const int sa = 8 * tq + hh, sbl = sa + 4;
     const float pa0 = __shfl_sync(0xffffffffu, p0, sa);
     const float pa1 = __shfl_sync(0xffffffffu, p1, sa);
@@ -618,15 +682,44 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
                h0, l0);
         split2(pa1 * meta_at(sb.vms, (2 * tq + 8) * n + gi, g.es),
                pb1 * meta_at(sb.vms, (2 * tq + 9) * n + gi, g.es), h1, l1);
-        b0 = dead_col ? 0u : (is_lo ? l0 : h0);
-        b1 = dead_col ? 0u : (is_lo ? l1 : h1);
-        if (ASYM) zs = p0 * meta_at(sb.vmz, gq * n + gi, g.es) + p1 * meta_at(sb.vmz, (gq + 8) * n + gi, g.es);
+        b0 = (dead_col || !live) ? 0u : (is_lo ? l0 : h0);
+        b1 = (dead_col || !live) ? 0u : (is_lo ? l1 : h1);
+        if (ASYM)
+          zs = live ? p0 * meta_at(sb.vmz, gq * n + gi, g.es) + p1 * meta_at(sb.vmz, (gq + 8) * n + gi, g.es)
+                    : 0.0f;
       }
       uint32_t a0, a1, a2, a3;
       value_frag<BITS, SGN>(vw, i, a0, a1, a2, a3);
       mma_bf16(st.o[i], a0, a1, a2, a3, b0, b1);
       if (ASYM) st.zacc[i] += zs;
     }
+  };
+
+  // Online softmax over up to 64 tokens (4 sub-tiles x 2 scores per lane).
+  auto softmax_chunk = [&](const float (&s)[8], float (&p)[8]) {
+    float mx = fmaxf(fmaxf(fmaxf(s[0], s[1]), fmaxf(s[2], s[3])), fmaxf(fmaxf(s[4], s[5]), fmaxf(s[6], s[7])));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+    if (mx > st.m + 8.0f) {   // also taken from -inf
+      const float alpha = fast_exp2(st.m - mx);
+      st.l *= alpha;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) st.o[i][c] *= alpha;
+        st.zacc[i] *= alpha;
+      }
+      st.m = mx;
+    }
+    const bool live = st.m != -INFINITY;
+    float sum = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      p[k] = live ? fast_exp2(s[k] - st.m) : 0.0f;
+      sum += p[k];
+    }
+    st.l += sum;
   };
 
   // A 16-token tile of the BF16 window (natural row-major layout).
@@ -642,17 +735,17 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
       if (j & 1) mma_bf16(acc1, a0, a1, a2, a3, bq[j][0], bq[j][1]);
       else mma_bf16(acc0, a0, a1, a2, a3, bq[j][0], bq[j][1]);
     }
-    float s0 = (acc0[0] + acc0[1] + acc1[0] + acc1[1]) * C;
-    float s1 = (acc0[2] + acc0[3] + acc1[2] + acc1[3]) * C;
-    if (gq >= valid) s0 = -INFINITY;
-    if (gq + 8 >= valid) s1 = -INFINITY;
-    float p0, p1;
-    softmax_step(st, s0, s1, p0, p1);
+    float s[8], p[8];
+    s[0] = gq < valid ? (acc0[0] + acc0[1] + acc1[0] + acc1[1]) * C : -INFINITY;
+    s[1] = gq + 8 < valid ? (acc0[2] + acc0[3] + acc1[2] + acc1[3]) * C : -INFINITY;
+#pragma unroll
+    for (int k = 2; k < 8; ++k) s[k] = -INFINITY;
+    softmax_chunk(s, p);
     const int sa = 8 * tq + hh, sbl = sa + 4;
-    const float pa0 = __shfl_sync(0xffffffffu, p0, sa);
-    const float pa1 = __shfl_sync(0xffffffffu, p1, sa);
-    const float pb0 = __shfl_sync(0xffffffffu, p0, sbl);
-    const float pb1 = __shfl_sync(0xffffffffu, p1, sbl);
+    const float pa0 = __shfl_sync(0xffffffffu, p[0], sa);
+    const float pa1 = __shfl_sync(0xffffffffu, p[1], sa);
+    const float pb0 = __shfl_sync(0xffffffffu, p[0], sbl);
+    const float pb1 = __shfl_sync(0xffffffffu, p[1], sbl);
     uint32_t h0, l0, h1, l1;
     split2(pa0, pb0, h0, l0);
     split2(pa1, pb1, h1, l1);
@@ -666,6 +759,32 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
       mma_bf16(st.o[i], a0, a1, a2, a3, b0, b1);
     }
   };
+
+  // Where sub-tile `tok0 / 16` of a quantized unit sits in its stage.
+  auto sub_at = [&](const uint8_t* stg, int tok0) {
+    Sub sb;
+    if (KAXIS) {
+      const uint8_t* cb = stg + (tok0 >> g.lg_P) * g.chunk_used;
+      const int us = (tok0 & (g.P - 1)) >> 4;
+      sb.k = cb + us * g.sub_bytes;
+      sb.v = cb + g.off_V + us * g.sub_bytes;
+      sb.vms = cb + g.off_Vm + 16 * us * g.nvg * g.es;
+      sb.vmz = cb + g.off_Vm + (g.P + 16 * us) * g.nvg * g.es;
+      sb.kms = sb.kmz = nullptr;
+    } else {
+      const uint8_t* sbase = stg + (tok0 >> 4) * pp.qsub;
+      sb.k = sbase;
+      sb.v = sbase + g.sub_bytes;
+      sb.vms = sbase + 2 * g.sub_bytes;
+      sb.vmz = sb.vms + 16 * g.nvg * g.es;
+      sb.kms = sbase + 2 * g.sub_bytes + g.vm16;
+      sb.kmz = sb.kms + 16 * g.nkg * g.es;
+    }
+    return sb;
+  };
+
+  // sub-tiles per softmax chunk: 4, or one key group when groups are shorter
+  const int ch = KAXIS ? min(4, g.g_k >> 4) : 4;
 
   It it;
   it_seek(it, s_pre, a.B, g.h_kv, c0);
@@ -681,112 +800,78 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
       setup_pair(it.i, it.h);
       cur_pair = pair_id;
     }
-    // every lane polls; the warp gives up together, and once any warp has
-    // given up all of them skip the remaining work (but keep the barriers)
-    if (!aborted) {
-      const bool arrived = wait_or_abort(full0 + 8 * s, ph, abort_flag);
-      if (!__all_sync(0xffffffffu, arrived)) {
-        if (lane == 0) {
-          atomicOr(a.err, KVQ_DEVERR_TIMEOUT);
-          *abort_flag = 1;
-        }
-        aborted = true;
-      }
-    }
-    const uint8_t* stg = stages + size_t(s) * pp.stage_bytes;
-
-    if (it.k < ri.nq) {
-      const int T0 = it.k * pp.sup;
-      const int valid_unit = min(pp.sup, ri.qa - T0);
-      if (KAXIS) {
-        // q' = q * s_channel for the unit's key groups, shared by the 4 warps
-        const int buf = chan_units++ & 1;
-        const int ngv = (valid_unit + g.g_k - 1) >> g.lg_gk;
-        const int f = 32 * (lane >> 3) + 4 * (lane & 7);
-        const int lg_ppg = g.lg_gk - g.lg_P;   // pages per key group, log2
-        for (int gi = 0; gi < ngv && !aborted; ++gi) {
-          const uint8_t* km = stg + ((gi << lg_ppg) + (f >> g.lg_kslice)) * g.chunk_used + g.off_Km;
-          const int off = f & (g.kslice - 1);
-          float sc[4];
-          meta4(km, off, g.es, sc);
-          uint32_t h0, l0, h1, l1;
-          split2(qv[0] * sc[0], qv[1] * sc[1], h0, l0);
-          split2(qv[2] * sc[2], qv[3] * sc[3], h1, l1);
-          uint8_t* qb = smem + L.qbuf + (buf * pp.ngr + gi) * kQbufBytes;
-          const int lane_hi = 4 * (2 * warp) + (lane >> 3);       // (gq = 2 * head, tq)
-          const int kk = 2 * (lane & 7);
-          *reinterpret_cast<uint2*>(qb + (lane_hi * 16 + kk) * 4) = make_uint2(h0, h1);
-          *reinterpret_cast<uint2*>(qb + ((lane_hi + 4) * 16 + kk) * 4) = make_uint2(l0, l1);
-          if (ASYM) {
-            float zc[4];
-            meta4(km, g.kslice + off, g.es, zc);
-            float dz = qv[0] * zc[0] + qv[1] * zc[1] + qv[2] * zc[2] + qv[3] * zc[3];
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) dz += __shfl_xor_sync(0xffffffffu, dz, o);
-            if (lane == 0)
-              reinterpret_cast<float*>(smem + L.bias + (buf * pp.ngr + gi) * kBiasBytes)[warp] = dz;
+    if ((n & (kDecodeWarps - 1)) == warp) {
+      // every lane polls; the warp gives up together, and once any warp has
+      // given up all of them skip the remaining work (but keep the barriers)
+      if (!aborted) {
+        const bool arrived = wait_or_abort(full0 + 8 * s, ph, abort_flag);
+        if (!__all_sync(0xffffffffu, arrived)) {
+          if (lane == 0) {
+            atomicOr(a.err, KVQ_DEVERR_TIMEOUT);
+            *abort_flag = 1;
           }
+          aborted = true;
         }
-        consumer_sync();
+      }
+      const uint8_t* stg = stages + size_t(s) * pp.stage_bytes;
+      if (aborted) {
+      } else if (it.k < ri.nq) {
+        const int T0 = it.k * pp.sup;
+        const int valid_unit = min(pp.sup, ri.qa - T0);
+        const int nsub = (valid_unit + 15) >> 4;
         int loaded = -1;
-        for (int i = 0; i < pp.spw && !aborted; ++i) {
-          const int tok0 = 16 * (warp * pp.spw + i);
-          if (tok0 >= valid_unit) break;
-          const int gi = tok0 >> g.lg_gk;
-          if (gi != loaded) {
-            const uint4* qb = reinterpret_cast<const uint4*>(smem + L.qbuf + (buf * pp.ngr + gi) * kQbufBytes +
-                                                             lane * 64);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              const uint4 x = qb[v];
-              bq[2 * v][0] = x.x; bq[2 * v][1] = x.y; bq[2 * v + 1][0] = x.z; bq[2 * v + 1][1] = x.w;
-            }
-            bias_t = ASYM ? C * reinterpret_cast<const float*>(smem + L.bias + (buf * pp.ngr + gi) *
-                                                                                  kBiasBytes)[min(tq, g.G - 1)]
-                          : 0.0f;
-            loaded = gi;
-            bq_holds_q = false;
+        for (int c = 0; c < nsub; c += ch) {
+          if (KAXIS && ((16 * c) >> g.lg_gk) != loaded) {
+            loaded = (16 * c) >> g.lg_gk;
+            qprime_job(stg, loaded);
           }
-          const int pg = tok0 >> g.lg_P, us = (tok0 & (g.P - 1)) >> 4;
-          const uint8_t* cb = stg + pg * g.chunk_used;
-          Sub sb;
-          sb.k = cb + us * g.sub_bytes;
-          sb.v = cb + g.off_V + us * g.sub_bytes;
-          sb.vms = cb + g.off_Vm + 16 * us * g.nvg * g.es;
-          sb.vmz = cb + g.off_Vm + (g.P + 16 * us) * g.nvg * g.es;
-          sb.kms = sb.kmz = nullptr;
-          process_sub(sb, valid_unit - tok0);
+          // scores of the chunk's sub-tiles go through this lane's own slots of
+          // the warp scratch, which keeps the loops rolled (small code, no spills)
+          const int nt = min(ch, nsub - c);
+          // two sub-tiles per trip, as independent instruction streams, where
+          // registers allow (an odd last trip re-reads sub-tile nt - 1 and
+          // discards it); one per trip otherwise
+#pragma unroll 1
+          for (int t = 0; t < nt; t += kPair) {
+            const int tokA = 16 * (c + t);
+            float sA0, sA1;
+            score_sub(sub_at(stg, tokA), valid_unit - tokA, sA0, sA1);
+            spw[(2 * t) * 32 + lane] = sA0;
+            spw[(2 * t + 1) * 32 + lane] = sA1;
+            if (kPair == 2) {
+              const int tokB = 16 * (c + min(t + 1, nt - 1));
+              float sB0, sB1;
+              score_sub(sub_at(stg, tokB), t + 1 < nt ? valid_unit - tokB : 0, sB0, sB1);
+              spw[(2 * t + 2) * 32 + lane] = sB0;
+              spw[(2 * t + 3) * 32 + lane] = sB1;
+            }
+          }
+          float sc[8], pc[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) sc[k] = k < 2 * nt ? spw[k * 32 + lane] : -INFINITY;
+          softmax_chunk(sc, pc);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) spw[k * 32 + lane] = pc[k];
+#pragma unroll 1
+          for (int t = 0; t < nt; t += kPair) {
+            pv_sub(sub_at(stg, 16 * (c + t)), spw[(2 * t) * 32 + lane], spw[(2 * t + 1) * 32 + lane], true);
+            if (kPair == 2)
+              pv_sub(sub_at(stg, 16 * (c + min(t + 1, nt - 1))), spw[(2 * t + 2) * 32 + lane],
+                     spw[(2 * t + 3) * 32 + lane], t + 1 < nt);
+          }
         }
-      } else if (!aborted) {
-        const int tok0 = 16 * warp;
-        if (tok0 < valid_unit) {
-          const uint8_t* sbase = stg + warp * pp.qsub;
-          Sub sb;
-          sb.k = sbase;
-          sb.v = sbase + g.sub_bytes;
-          sb.vms = sbase + 2 * g.sub_bytes;
-          sb.vmz = sb.vms + 16 * g.nvg * g.es;
-          sb.kms = sbase + 2 * g.sub_bytes + g.vm16;
-          sb.kmz = sb.kms + 16 * g.nkg * g.es;
-          process_sub(sb, valid_unit - tok0);
-        }
-      }
-    } else if (!aborted) {
-      const int r = it.k - ri.nq;
-      if ((r & (kDecodeWarps - 1)) == warp) {
+      } else {
         if (!bq_holds_q) {
           load_bq_from_q(it.i, it.h);
           bq_holds_q = true;
           bias_t = 0.0f;
         }
-        process_window(stg, ri.ra - 16 * r);
+        process_window(stg, ri.ra - 16 * (it.k - ri.nq));
       }
+      // release the stage to the producer
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty0 + 8 * s);
     }
-
-    // release the stage to the producer
-    fence_proxy_async();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(empty0 + 8 * s);
     if (++s == pp.nstages) { s = 0; ph ^= 1u; }
     if (it_next(it, s_pre, a.B, g.h_kv) && n + 1 < N) ri = row_info(a, it.i, false);
   }
@@ -795,18 +880,18 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
 
 // Merge: one CTA per (row, kv head, query head), one thread per channel.  The
 // records of a pair are the consumer warps of every CTA whose range holds its
-// units, taken in CTA order (a fixed summation order).
+// units, visited in CTA order and warp order (a fixed summation order) with a
+// running log-sum-exp, so each thread issues every load of a CTA's four
+// records at once and no block-wide reduction is needed.
 constexpr int kMergeThreads = 128;
-constexpr int kMaxRecords = kDecodeWarps * kMaxDecodeGrid;
 
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_constant__ DecodeArgs a) {
   constexpr int D = kD;
-  __shared__ int32_t s_cta[kMaxDecodeGrid];
-  __shared__ float s_w[kMaxRecords];
-  __shared__ int32_t s_cnt[kMergeThreads / 32];
-  __shared__ float s_red[kMergeThreads / 32];
+  // launched as a programmatic dependent of the decode grid: wait until that
+  // grid has completed and its writes are visible (returns at once otherwise)
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
   const Geo& g = a.g;
-  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int tid = threadIdx.x;
   const int G = g.G;
   const int p = blockIdx.x / G, hd = blockIdx.x % G;
   const int i = p / g.h_kv, h = p % g.h_kv;
@@ -821,60 +906,46 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
   const int64_t GR = a.grid;
   const int64_t ua = int64_t(pre[i]) * g.h_kv + int64_t(h) * n, ub = ua + n - 1;
   const int64_t k0 = ((ua + 1) * GR - 1) / U, k1 = ((ub + 1) * GR - 1) / U;
-  // CTAs with non-empty ranges from k0 to k1, in order
-  int count = 0;
-  for (int64_t base = k0; base <= k1; base += kMergeThreads) {
-    const int64_t k = base + tid;
-    const bool live = k <= k1 && (k * U) / GR < ((k + 1) * U) / GR;
-    const uint32_t m = __ballot_sync(0xffffffffu, live);
-    if (lane == 0) s_cnt[w] = __popc(m);
-    __syncthreads();
-    int before = count;
-    for (int q = 0; q < w; ++q) before += s_cnt[q];
-    if (live) s_cta[before + __popc(m & ((1u << lane) - 1u))] = int32_t(k);
-    int tot = 0;
-    for (int q = 0; q < kMergeThreads / 32; ++q) tot += s_cnt[q];
-    __syncthreads();
-    count += tot;
+  const int64_t rec_stride = int64_t(G) * (D + 2);
+  float M = -INFINITY, den = 0.0f, num = 0.0f;
+#pragma unroll 2
+  for (int64_t k = k0; k <= k1; ++k) {
+    if ((k * U) / GR >= ((k + 1) * U) / GR) continue;   // a CTA with an empty range wrote nothing
+    const float* rec = a.partials + ((int64_t(p) + k) * kDecodeWarps * G + hd) * (D + 2);
+    float m[kDecodeWarps], l[kDecodeWarps], o[kDecodeWarps];
+#pragma unroll
+    for (int w = 0; w < kDecodeWarps; ++w) {
+      m[w] = rec[w * rec_stride];
+      l[w] = rec[w * rec_stride + 1];
+      o[w] = rec[w * rec_stride + 2 + tid];
+    }
+    float mx = M;
+#pragma unroll
+    for (int w = 0; w < kDecodeWarps; ++w) mx = fmaxf(mx, m[w]);
+    if (mx == -INFINITY) continue;
+    const float sc = fast_exp2(M - mx);   // 0 while M is -inf
+    den *= sc;
+    num *= sc;
+#pragma unroll
+    for (int w = 0; w < kDecodeWarps; ++w) {
+      const float wt = fast_exp2(m[w] - mx);
+      den = fmaf(wt, l[w], den);
+      num = fmaf(wt, o[w], num);
+    }
+    M = mx;
   }
-  const int nrec = count * kDecodeWarps;
-  auto rec_of = [&](int r) {
-    const int64_t slot = (int64_t(p) + s_cta[r / kDecodeWarps]) * kDecodeWarps + (r % kDecodeWarps);
-    return a.partials + (slot * G + hd) * (D + 2);
-  };
-  float M = -INFINITY;
-  for (int r = tid; r < nrec; r += kMergeThreads) M = fmaxf(M, rec_of(r)[0]);
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  if (lane == 0) s_red[w] = M;
-  __syncthreads();
-  M = s_red[0];
-  for (int q = 1; q < kMergeThreads / 32; ++q) M = fmaxf(M, s_red[q]);
-  __syncthreads();
-  float den = 0.0f;
-  for (int r = tid; r < nrec; r += kMergeThreads) {
-    const float* rec = rec_of(r);
-    const float wgt = M == -INFINITY ? 0.0f : fast_exp2(rec[0] - M);
-    s_w[r] = wgt;
-    den = fmaf(wgt, rec[1], den);
-  }
-  for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-  if (lane == 0) s_red[w] = den;
-  __syncthreads();
-  den = 0.0f;
-  for (int q = 0; q < kMergeThreads / 32; ++q) den += s_red[q];
-  float num = 0.0f;
-  for (int r = 0; r < nrec; ++r) num = fmaf(s_w[r], rec_of(r)[2 + tid], num);
   out[tid] = den > 0.0f ? num / den : 0.0f;
 }
 
-template <int BITS, int ASYM, int KAXIS>
+template <int BITS, int ASYM, int KAXIS, int SPEC = 0>
 const void* kernel_of() {
-  return reinterpret_cast<const void*>(&decode_kernel<BITS, ASYM, KAXIS>);
+  return reinterpret_cast<const void*>(&decode_kernel<BITS, ASYM, KAXIS, SPEC>);
 }
 
 }  // namespace
 
 const void* decode_kernel_ptr(const Geo& g) {
+  if (spec_int4_kivi(g)) return kernel_of<4, 0, 1, 1>();
   const int key = (g.bits == 8 ? 0 : g.bits == 4 ? 1 : 2) * 4 + g.asym * 2 + g.k_axis;
   switch (key) {
     case 0: return kernel_of<8, 0, 0>();
@@ -904,9 +975,7 @@ size_t decode_partials_bytes(const Geo& g, int B, int grid) {
 cudaError_t plan_decode(const Geo& g, int max_B, DecodePipe* out) {
   DecodePipe p{};
   p.sup = g.k_axis ? (g.g_k > 64 ? g.g_k : 64) : 64;
-  p.spw = p.sup / 64;
   p.lg_sup = p.sup == 128 ? 7 : 6;
-  p.ngr = g.k_axis ? (p.sup / g.g_k) : 1;
   p.qsub = g.k_axis ? 0 : 2 * g.sub_bytes + g.vm16 + g.km16;
   const int qunit = g.k_axis ? (p.sup / g.P) * g.chunk_used : kDecodeWarps * p.qsub;
   const int res = g.R ? 2 * 16 * kD * 2 : 0;
@@ -916,10 +985,12 @@ cudaError_t plan_decode(const Geo& g, int max_B, DecodePipe* out) {
   if (e != cudaSuccess) return e;
   e = cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   if (e != cudaSuccess) return e;
-  // aim for three resident CTAs per SM: about 72 KB of shared memory each
-  p.nstages = 6;
-  while (p.nstages > 2 && size_t(smem_layout(max_B, p).total) > size_t(72 * 1024)) --p.nstages;
-  while (p.nstages > 1 && size_t(smem_layout(max_B, p).total) > size_t(max_optin)) --p.nstages;
+  // aim for three resident CTAs per SM (about 72 KB of shared memory each)
+  // with two stages per consumer warp; the stage count stays a multiple of
+  // the warp count so warp w always owns stages w, w + 4, ...
+  p.nstages = 2 * kDecodeWarps;
+  if (size_t(smem_layout(max_B, p).total) > size_t(72 * 1024)) p.nstages = kDecodeWarps;
+  if (size_t(smem_layout(max_B, p).total) > size_t(max_optin)) return cudaErrorInvalidConfiguration;
   const size_t smem = size_t(smem_layout(max_B, p).total);
   if (smem > size_t(max_optin)) return cudaErrorInvalidConfiguration;
   const void* kern = decode_kernel_ptr(g);
@@ -945,7 +1016,19 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s, cudaEvent_t betwe
   }
   const int items = a.B * a.g.h_kv * a.g.G;
   if (items == 0) return cudaSuccess;
-  e = cudaLaunchKernel(reinterpret_cast<const void*>(&merge_kernel), dim3(items), dim3(kMergeThreads), args, 0, s);
+  // The merge is a programmatic dependent launch, so its launch overlaps the
+  // decode grid's tail; with an event between the two it is a plain launch.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(items);
+  cfg.blockDim = dim3(kMergeThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = between ? 0 : 1;
+  e = cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(&merge_kernel), args);
   if (e == cudaSuccess) ++*launches;
   return e;
 }

@@ -59,8 +59,6 @@ struct DevState {
 struct DecodePipe {
   int sup;          // tokens per quantized work unit (64, or g_k when larger)
   int lg_sup;       // log2(sup)
-  int spw;          // 16-token sub-tiles per consumer warp in a unit (sup / 64)
-  int ngr;          // key groups per unit (channel axis), 1 on the token axis
   int qsub;         // token axis: bytes of one staged 16-token sub-tile
   int stage_bytes;  // one stage: a quantized unit or a 16-token BF16 window tile
   int nstages;
