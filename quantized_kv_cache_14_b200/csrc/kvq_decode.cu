@@ -195,50 +195,64 @@ __device__ __forceinline__ void load_key_words(const uint8_t* ksub, int gq, int 
   }
 }
 
+// One operand register from two codes: fp16 (H) or bf16.
+template <bool SGN, bool H>
+__device__ __forceinline__ uint32_t nib2(uint32_t w, int x) {
+  return H ? nib_pair_h<SGN>(w, x) : nib_pair<SGN>(w, x);
+}
+template <bool SGN, bool H>
+__device__ __forceinline__ uint32_t crumb2(uint32_t w, int x) {
+  return H ? crumb_pair_h<SGN>(w, x) : crumb_pair<SGN>(w, x);
+}
+template <bool SGN, bool H>
+__device__ __forceinline__ uint32_t byte2(uint32_t w, int x) {
+  return H ? byte_pair_h<SGN>(w, x) : byte_pair<SGN>(w, x);
+}
+
 // A operand (rows gq / gq+8, k-step j) of the score product from key words.
-template <int BITS, bool SGN>
+template <int BITS, bool SGN, bool H>
 __device__ __forceinline__ void key_frag(const uint32_t (&wa)[BITS], const uint32_t (&wb)[BITS], int j,
                                          uint32_t& a0, uint32_t& a1, uint32_t& a2, uint32_t& a3) {
   if (BITS == 4) {
     const int jj = j >> 1, x = 2 * (j & 1);
-    a0 = nib_pair<SGN>(wa[jj], x);
-    a1 = nib_pair<SGN>(wb[jj], x);
-    a2 = nib_pair<SGN>(wa[jj], x + 1);
-    a3 = nib_pair<SGN>(wb[jj], x + 1);
+    a0 = nib2<SGN, H>(wa[jj], x);
+    a1 = nib2<SGN, H>(wb[jj], x);
+    a2 = nib2<SGN, H>(wa[jj], x + 1);
+    a3 = nib2<SGN, H>(wb[jj], x + 1);
   } else if (BITS == 2) {
     const int jj = j >> 2, x = 2 * (j & 3);
-    a0 = crumb_pair<SGN>(wa[jj], x);
-    a1 = crumb_pair<SGN>(wb[jj], x);
-    a2 = crumb_pair<SGN>(wa[jj], x + 1);
-    a3 = crumb_pair<SGN>(wb[jj], x + 1);
+    a0 = crumb2<SGN, H>(wa[jj], x);
+    a1 = crumb2<SGN, H>(wb[jj], x);
+    a2 = crumb2<SGN, H>(wa[jj], x + 1);
+    a3 = crumb2<SGN, H>(wb[jj], x + 1);
   } else {
-    a0 = byte_pair<SGN>(wa[j], 0);
-    a1 = byte_pair<SGN>(wb[j], 0);
-    a2 = byte_pair<SGN>(wa[j], 1);
-    a3 = byte_pair<SGN>(wb[j], 1);
+    a0 = byte2<SGN, H>(wa[j], 0);
+    a1 = byte2<SGN, H>(wb[j], 0);
+    a2 = byte2<SGN, H>(wa[j], 1);
+    a3 = byte2<SGN, H>(wb[j], 1);
   }
 }
 
 // A operand of the value product for channel tile i from a lane record.
-template <int BITS, bool SGN>
+template <int BITS, bool SGN, bool H>
 __device__ __forceinline__ void value_frag(const uint32_t (&w)[2 * BITS], int i, uint32_t& a0, uint32_t& a1,
                                            uint32_t& a2, uint32_t& a3) {
   if (BITS == 4) {
-    a0 = nib_pair<SGN>(w[i], 0);
-    a1 = nib_pair<SGN>(w[i], 1);
-    a2 = nib_pair<SGN>(w[i], 2);
-    a3 = nib_pair<SGN>(w[i], 3);
+    a0 = nib2<SGN, H>(w[i], 0);
+    a1 = nib2<SGN, H>(w[i], 1);
+    a2 = nib2<SGN, H>(w[i], 2);
+    a3 = nib2<SGN, H>(w[i], 3);
   } else if (BITS == 2) {
     const int b = 2 * (i & 1);
-    a0 = crumb_pair<SGN>(w[i >> 1], b);
-    a1 = crumb_pair<SGN>(w[i >> 1], b + 1);
-    a2 = crumb_pair<SGN>(w[i >> 1], b + 4);
-    a3 = crumb_pair<SGN>(w[i >> 1], b + 5);
+    a0 = crumb2<SGN, H>(w[i >> 1], b);
+    a1 = crumb2<SGN, H>(w[i >> 1], b + 1);
+    a2 = crumb2<SGN, H>(w[i >> 1], b + 4);
+    a3 = crumb2<SGN, H>(w[i >> 1], b + 5);
   } else {
-    a0 = byte_pair<SGN>(w[2 * i], 0);
-    a1 = byte_pair<SGN>(w[2 * i], 1);
-    a2 = byte_pair<SGN>(w[2 * i + 1], 0);
-    a3 = byte_pair<SGN>(w[2 * i + 1], 1);
+    a0 = byte2<SGN, H>(w[2 * i], 0);
+    a1 = byte2<SGN, H>(w[2 * i], 1);
+    a2 = byte2<SGN, H>(w[2 * i + 1], 0);
+    a3 = byte2<SGN, H>(w[2 * i + 1], 1);
   }
 }
 
@@ -278,6 +292,18 @@ __device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_
       __floats2bfloat162_rn(x0 - __uint_as_float(hi << 16), x1 - __uint_as_float(hi & 0xFFFF0000u));
   lo = *reinterpret_cast<const uint32_t*>(&l);
 }
+
+// Both fp16 parts of an fp32 pair: hi = f16_rn(x), lo = f16_rn(x - hi).
+__device__ __forceinline__ void split2h(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(x0, x1);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  const float2 hf = __half22float2(h);
+  const __half2 l = __floats2half2_rn(x0 - hf.x, x1 - hf.y);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// 2^e as a float, e in [-126, 127].
+__device__ __forceinline__ float pow2f(int e) { return __uint_as_float(uint32_t(e + 127) << 23); }
 
 // Where one 16-token sub-tile sits in a stage.
 struct Sub {
@@ -326,10 +352,14 @@ bool spec_int4_kivi(const Geo& g) {
          g.lg_kslice == S::lg_kslice;
 }
 
-template <int BITS, int ASYM, int KAXIS, int SPEC>
+template <int BITS, int ASYM, int KAXIS, int ES, int SPEC>
 __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_constant__ DecodeArgs a) {
   constexpr int D = kD;
   constexpr bool SGN = !ASYM;
+  // The value product runs on fp16 operands when the stored scales are fp16:
+  // with the running max exact (p <= 1), p' = p * s fits fp16's range.  Fp32
+  // scales keep bf16 operands (fp32 range).
+  constexpr bool PVH = ES == 2;
   constexpr int kPair = 1;   // sub-tiles per trip of the chunk loops (2 measured slower)
   extern __shared__ __align__(128) uint8_t smem[];
   const Geo gs = geo_of<SPEC>(a.g);
@@ -385,7 +415,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
     int s = 0;
     uint32_t ph = 0;
     int issued = 0;
-    const int vrow = 16 * g.nvg * g.es, krow = 16 * g.nkg * g.es;
+    const int vrow = 16 * g.nvg * ES, krow = 16 * g.nkg * ES;
     for (int n = 0; n < N; ++n) {
       const uint32_t dst = stage0 + s * pp.stage_bytes;
       const uint32_t bar = full0 + 8 * s;
@@ -456,11 +486,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
               bulk_g2s(d, chunk + u * g.sub_bytes, g.sub_bytes, bar);
               bulk_g2s(d + g.sub_bytes, chunk + g.off_V + u * g.sub_bytes, g.sub_bytes, bar);
               const uint32_t vm = d + 2 * g.sub_bytes, km = vm + g.vm16;
-              bulk_g2s(vm, chunk + g.off_Vm + int64_t(16 * u) * g.nvg * g.es, vrow, bar);
-              bulk_g2s(km, chunk + g.off_Km + int64_t(16 * u) * g.nkg * g.es, krow, bar);
+              bulk_g2s(vm, chunk + g.off_Vm + int64_t(16 * u) * g.nvg * ES, vrow, bar);
+              bulk_g2s(km, chunk + g.off_Km + int64_t(16 * u) * g.nkg * ES, krow, bar);
               if (ASYM) {
-                bulk_g2s(vm + vrow, chunk + g.off_Vm + int64_t(g.P + 16 * u) * g.nvg * g.es, vrow, bar);
-                bulk_g2s(km + krow, chunk + g.off_Km + int64_t(g.P + 16 * u) * g.nkg * g.es, krow, bar);
+                bulk_g2s(vm + vrow, chunk + g.off_Vm + int64_t(g.P + 16 * u) * g.nvg * ES, vrow, bar);
+                bulk_g2s(km + krow, chunk + g.off_Km + int64_t(g.P + 16 * u) * g.nkg * ES, krow, bar);
               }
             }
           }
@@ -497,8 +527,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
 
   State st;
   state_reset(st);
-  uint32_t bq[8][2];          // score B operand: q' hi|lo columns, or q itself
-  bool bq_holds_q = false;    // bq carries q (token axis, BF16 window)
+  uint32_t bq[8][2];          // score B operand: fp16 q' hi|lo columns, fp16 q, or bf16 q (window)
+  bool bq_bf16 = false;       // bq carries bf16 q for the BF16 window
+  float cs = C;               // score scale: C times the power of two taken out of the fp16 operand
   float bias_t = 0.0f;        // channel-axis zero-points: key bias of head tq for the loaded group
   uint32_t qw[4][2];          // channel axis: q of head h at key-list channels 4*lane .. 4*lane+3
   float qsum[4] = {0.0f, 0.0f, 0.0f, 0.0f};   // token-axis zero-points: sum of q per key group
@@ -516,6 +547,32 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
       bq[j][0] = (dead_col || is_lo) ? 0u : t0;
       bq[j][1] = (dead_col || is_lo) ? 0u : t1;
     }
+  };
+
+  // Token axis: q itself as the fp16 operand, scaled by a power of two per pair
+  // so the largest |q| of the kv head's query heads lies in [2^14, 2^15).
+  auto load_bq_f16 = [&](int row, int h) {
+    load_bq_from_q(row, h);
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int e = 0; e < 2; ++e)
+        amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(bq[j][e] << 16)), fabsf(__uint_as_float(bq[j][e] & 0xFFFF0000u))));
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const int ex = amax > 0.0f ? min(max(int((__float_as_uint(amax) >> 23) & 0xFF) - 127 - 14, -100), 100) : 0;
+    const float down = pow2f(-ex);
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const __half2 hq = __floats2half2_rn(__uint_as_float(bq[j][e] << 16) * down,
+                                             __uint_as_float(bq[j][e] & 0xFFFF0000u) * down);
+        bq[j][e] = *reinterpret_cast<const uint32_t*>(&hq);
+      }
+    cs = C * pow2f(ex);
+    return down;
   };
 
   auto emit = [&](int row, int h) {
@@ -551,7 +608,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
 
   auto setup_pair = [&](int row, int h) {
     state_reset(st);
-    bq_holds_q = false;
+    bq_bf16 = false;
     bias_t = 0.0f;
     if (KAXIS) {
       // this lane's share of the q' job: key-list channels 4*lane .. 4*lane+3 of every head
@@ -564,14 +621,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
         qw[h2][1] = live ? *reinterpret_cast<const uint32_t*>(qr + key_channel(f + 2)) : 0u;
       }
     } else {
-      load_bq_from_q(row, h);
-      bq_holds_q = true;
+      const float down = load_bq_f16(row, h);
       if (ASYM) {
+        // in the operand's scaled domain, like the products it is added to
         const uint16_t* qr = qrow(row, h, tq);
         for (int gi = 0; gi < g.nkg; ++gi) {
           float s = 0.0f;
           for (int c = gi * g.g_k; c < (gi + 1) * g.g_k; ++c) s += bf16_bits_to_float(qr[c]);
-          qsum[gi & 3] = s;
+          qsum[gi & 3] = s * down;
         }
       }
     }
@@ -587,25 +644,39 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
     const uint8_t* km = stg + ((gi << lg_ppg) + (f >> g.lg_kslice)) * g.chunk_used + g.off_Km;
     const int off = f & (g.kslice - 1);
     float sc[4];
-    meta4(km, off, g.es, sc);
+    meta4(km, off, ES, sc);
     float zc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    if (ASYM) meta4(km, g.kslice + off, g.es, zc);
+    if (ASYM) meta4(km, g.kslice + off, ES, zc);
     const int t0 = lane >> 3, j = lane & 7;
     float dz[4];
-    __syncwarp();   // every lane has read the previous operand
+    float x[4][4];
+    float amax = 0.0f;
 #pragma unroll
     for (int h2 = 0; h2 < 4; ++h2) {
       const float q0 = __uint_as_float(qw[h2][0] << 16), q1 = __uint_as_float(qw[h2][0] & 0xFFFF0000u);
       const float q2 = __uint_as_float(qw[h2][1] << 16), q3 = __uint_as_float(qw[h2][1] & 0xFFFF0000u);
+      x[h2][0] = q0 * sc[0]; x[h2][1] = q1 * sc[1]; x[h2][2] = q2 * sc[2]; x[h2][3] = q3 * sc[3];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(x[h2][e]));
+      if (ASYM) dz[h2] = q0 * zc[0] + q1 * zc[1] + q2 * zc[2] + q3 * zc[3];
+    }
+    // one power of two per group puts the largest |q'| in [2^14, 2^15)
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const int ex = amax > 0.0f ? min(max(int((__float_as_uint(amax) >> 23) & 0xFF) - 127 - 14, -100), 100) : 0;
+    const float down = pow2f(-ex);
+    cs = C * pow2f(ex);
+    __syncwarp();   // every lane has read the previous operand
+#pragma unroll
+    for (int h2 = 0; h2 < 4; ++h2) {
       uint32_t h0, l0, h1, l1;
-      split2(q0 * sc[0], q1 * sc[1], h0, l0);
-      split2(q2 * sc[2], q3 * sc[3], h1, l1);
+      split2h(x[h2][0] * down, x[h2][1] * down, h0, l0);
+      split2h(x[h2][2] * down, x[h2][3] * down, h1, l1);
       const int thi = 8 * h2 + t0, tlo = thi + 4;   // lanes (gq = 2 h2 | 2 h2 + 1, tq = t0)
       *reinterpret_cast<uint2*>(qbw + thi * 16 + 4 * ((j >> 1) ^ ((thi >> 1) & 3)) + 2 * (j & 1)) =
           make_uint2(h0, h1);
       *reinterpret_cast<uint2*>(qbw + tlo * 16 + 4 * ((j >> 1) ^ ((tlo >> 1) & 3)) + 2 * (j & 1)) =
           make_uint2(l0, l1);
-      if (ASYM) dz[h2] = q0 * zc[0] + q1 * zc[1] + q2 * zc[2] + q3 * zc[3];
     }
     if (ASYM) {
 #pragma unroll
@@ -623,7 +694,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
       const uint4 x = qb[v ^ sw];
       bq[2 * v][0] = x.x; bq[2 * v][1] = x.y; bq[2 * v + 1][0] = x.z; bq[2 * v + 1][1] = x.w;
     }
-    bq_holds_q = false;
+    bq_bf16 = false;
   };
 
   // Scores of one 16-token quantized sub-tile: tokens gq, gq + 8 for head tq,
@@ -636,18 +707,18 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       uint32_t a0, a1, a2, a3;
-      key_frag<BITS, SGN>(wa, wb, j, a0, a1, a2, a3);
-      if (j & 1) mma_bf16(acc1, a0, a1, a2, a3, bq[j][0], bq[j][1]);
-      else mma_bf16(acc0, a0, a1, a2, a3, bq[j][0], bq[j][1]);
+      key_frag<BITS, SGN, true>(wa, wb, j, a0, a1, a2, a3);
+      if (j & 1) mma_f16(acc1, a0, a1, a2, a3, bq[j][0], bq[j][1]);
+      else mma_f16(acc0, a0, a1, a2, a3, bq[j][0], bq[j][1]);
       if (!KAXIS && ((j + 1) & ((1 << kg_shift) - 1)) == 0) {
         const int gi = j >> kg_shift;
         const float t0 = acc0[0] + acc0[1] + acc1[0] + acc1[1];
         const float t1 = acc0[2] + acc0[3] + acc1[2] + acc1[3];
-        r0 = fmaf(meta_at(sb.kms, gq * g.nkg + gi, g.es), t0, r0);
-        r1 = fmaf(meta_at(sb.kms, (gq + 8) * g.nkg + gi, g.es), t1, r1);
+        r0 = fmaf(meta_at(sb.kms, gq * g.nkg + gi, ES), t0, r0);
+        r1 = fmaf(meta_at(sb.kms, (gq + 8) * g.nkg + gi, ES), t1, r1);
         if (ASYM) {
-          r0 = fmaf(meta_at(sb.kmz, gq * g.nkg + gi, g.es), qsum[gi & 3], r0);
-          r1 = fmaf(meta_at(sb.kmz, (gq + 8) * g.nkg + gi, g.es), qsum[gi & 3], r1);
+          r0 = fmaf(meta_at(sb.kmz, gq * g.nkg + gi, ES), qsum[gi & 3], r0);
+          r1 = fmaf(meta_at(sb.kmz, (gq + 8) * g.nkg + gi, ES), qsum[gi & 3], r1);
         }
 #pragma unroll
         for (int c = 0; c < 4; ++c) acc0[c] = acc1[c] = 0.0f;
@@ -657,8 +728,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
       r0 = acc0[0] + acc0[1] + acc1[0] + acc1[1];
       r1 = acc0[2] + acc0[3] + acc1[2] + acc1[3];
     }
-    s0 = gq < valid ? fmaf(r0, C, bias_t) : -INFINITY;
-    s1 = gq + 8 < valid ? fmaf(r1, C, bias_t) : -INFINITY;
+    s0 = gq < valid ? fmaf(r0, cs, bias_t) : -INFINITY;
+    s1 = gq + 8 < valid ? fmaf(r1, cs, bias_t) : -INFINITY;
   };
 
   // Value product of one sub-tile: P' V_hat with p' = p * s_value(token, group).
@@ -678,19 +749,27 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
       if ((i & ((1 << vg_shift) - 1)) == 0) {
         const int gi = i >> vg_shift;
         uint32_t h0, l0, h1, l1;
-        split2(pa0 * meta_at(sb.vms, (2 * tq) * n + gi, g.es), pb0 * meta_at(sb.vms, (2 * tq + 1) * n + gi, g.es),
-               h0, l0);
-        split2(pa1 * meta_at(sb.vms, (2 * tq + 8) * n + gi, g.es),
-               pb1 * meta_at(sb.vms, (2 * tq + 9) * n + gi, g.es), h1, l1);
+        const float x0 = pa0 * meta_at(sb.vms, (2 * tq) * n + gi, ES);
+        const float x1 = pb0 * meta_at(sb.vms, (2 * tq + 1) * n + gi, ES);
+        const float x2 = pa1 * meta_at(sb.vms, (2 * tq + 8) * n + gi, ES);
+        const float x3 = pb1 * meta_at(sb.vms, (2 * tq + 9) * n + gi, ES);
+        if (PVH) {
+          split2h(x0, x1, h0, l0);
+          split2h(x2, x3, h1, l1);
+        } else {
+          split2(x0, x1, h0, l0);
+          split2(x2, x3, h1, l1);
+        }
         b0 = (dead_col || !live) ? 0u : (is_lo ? l0 : h0);
         b1 = (dead_col || !live) ? 0u : (is_lo ? l1 : h1);
         if (ASYM)
-          zs = live ? p0 * meta_at(sb.vmz, gq * n + gi, g.es) + p1 * meta_at(sb.vmz, (gq + 8) * n + gi, g.es)
+          zs = live ? p0 * meta_at(sb.vmz, gq * n + gi, ES) + p1 * meta_at(sb.vmz, (gq + 8) * n + gi, ES)
                     : 0.0f;
       }
       uint32_t a0, a1, a2, a3;
-      value_frag<BITS, SGN>(vw, i, a0, a1, a2, a3);
-      mma_bf16(st.o[i], a0, a1, a2, a3, b0, b1);
+      value_frag<BITS, SGN, PVH>(vw, i, a0, a1, a2, a3);
+      if (PVH) mma_f16(st.o[i], a0, a1, a2, a3, b0, b1);
+      else mma_bf16(st.o[i], a0, a1, a2, a3, b0, b1);
       if (ASYM) st.zacc[i] += zs;
     }
   };
@@ -701,7 +780,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-    if (mx > st.m + 8.0f) {   // also taken from -inf
+    if (mx > st.m) {   // also taken from -inf; keeps p <= 1
       const float alpha = fast_exp2(st.m - mx);
       st.l *= alpha;
 #pragma unroll
@@ -768,17 +847,17 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
       const int us = (tok0 & (g.P - 1)) >> 4;
       sb.k = cb + us * g.sub_bytes;
       sb.v = cb + g.off_V + us * g.sub_bytes;
-      sb.vms = cb + g.off_Vm + 16 * us * g.nvg * g.es;
-      sb.vmz = cb + g.off_Vm + (g.P + 16 * us) * g.nvg * g.es;
+      sb.vms = cb + g.off_Vm + 16 * us * g.nvg * ES;
+      sb.vmz = cb + g.off_Vm + (g.P + 16 * us) * g.nvg * ES;
       sb.kms = sb.kmz = nullptr;
     } else {
       const uint8_t* sbase = stg + (tok0 >> 4) * pp.qsub;
       sb.k = sbase;
       sb.v = sbase + g.sub_bytes;
       sb.vms = sbase + 2 * g.sub_bytes;
-      sb.vmz = sb.vms + 16 * g.nvg * g.es;
+      sb.vmz = sb.vms + 16 * g.nvg * ES;
       sb.kms = sbase + 2 * g.sub_bytes + g.vm16;
-      sb.kmz = sb.kms + 16 * g.nkg * g.es;
+      sb.kmz = sb.kms + 16 * g.nkg * ES;
     }
     return sb;
   };
@@ -861,9 +940,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
           }
         }
       } else {
-        if (!bq_holds_q) {
+        if (!bq_bf16) {
           load_bq_from_q(it.i, it.h);
-          bq_holds_q = true;
+          bq_bf16 = true;
           bias_t = 0.0f;
         }
         process_window(stg, ri.ra - 16 * (it.k - ri.nq));
@@ -878,11 +957,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
   if (!aborted && cur_pair >= 0) emit(cur_pair / g.h_kv, cur_pair % g.h_kv);
 }
 
-// Merge: one CTA per (row, kv head, query head), one thread per channel.  The
-// records of a pair are the consumer warps of every CTA whose range holds its
-// units, visited in CTA order and warp order (a fixed summation order) with a
-// running log-sum-exp, so each thread issues every load of a CTA's four
-// records at once and no block-wide reduction is needed.
+// Merge: one CTA per (row, kv head, query head).  The records of a pair are
+// the consumer warps of every CTA whose range holds its units.  The CTA's four
+// warps split those CTAs into four contiguous runs; each lane keeps a running
+// log-sum-exp over four channels, and the four runs are then combined in warp
+// order -- a fixed summation order for a given grid.
 constexpr int kMergeThreads = 128;
 
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_constant__ DecodeArgs a) {
@@ -890,8 +969,10 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
   // launched as a programmatic dependent of the decode grid: wait until that
   // grid has completed and its writes are visible (returns at once otherwise)
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  __shared__ float s_m[4], s_den[4];
+  __shared__ float s_num[4][D];
   const Geo& g = a.g;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int G = g.G;
   const int p = blockIdx.x / G, hd = blockIdx.x % G;
   const int i = p / g.h_kv, h = p % g.h_kv;
@@ -906,60 +987,88 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
   const int64_t GR = a.grid;
   const int64_t ua = int64_t(pre[i]) * g.h_kv + int64_t(h) * n, ub = ua + n - 1;
   const int64_t k0 = ((ua + 1) * GR - 1) / U, k1 = ((ub + 1) * GR - 1) / U;
+  // With at least as many units as CTAs every CTA from k0 to k1 holds units of
+  // the pair.  With fewer, each unit has a CTA of its own and the others wrote
+  // nothing: walk the pair's units instead (then all values are below 2^20).
+  const bool by_unit = U < GR;
+  const int64_t nk = by_unit ? ub - ua + 1 : k1 - k0 + 1;
+  const int64_t kb = (int64_t(w) * nk) / 4, ke = (int64_t(w + 1) * nk) / 4;
   const int64_t rec_stride = int64_t(G) * (D + 2);
-  float M = -INFINITY, den = 0.0f, num = 0.0f;
-#pragma unroll 2
-  for (int64_t k = k0; k <= k1; ++k) {
-    if ((k * U) / GR >= ((k + 1) * U) / GR) continue;   // a CTA with an empty range wrote nothing
+  float M = -INFINITY, den = 0.0f;
+  float num[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  for (int64_t t = kb; t < ke; ++t) {
+    const int64_t k = by_unit ? int64_t((int(ua + t + 1) * int(GR) - 1) / int(U)) : k0 + t;
     const float* rec = a.partials + ((int64_t(p) + k) * kDecodeWarps * G + hd) * (D + 2);
-    float m[kDecodeWarps], l[kDecodeWarps], o[kDecodeWarps];
+    float m[kDecodeWarps], l[kDecodeWarps];
+    float2 o[kDecodeWarps][2];
 #pragma unroll
-    for (int w = 0; w < kDecodeWarps; ++w) {
-      m[w] = rec[w * rec_stride];
-      l[w] = rec[w * rec_stride + 1];
-      o[w] = rec[w * rec_stride + 2 + tid];
+    for (int r = 0; r < kDecodeWarps; ++r) {
+      const float* rr = rec + r * rec_stride;
+      m[r] = rr[0];
+      l[r] = rr[1];
+      o[r][0] = *reinterpret_cast<const float2*>(rr + 2 + 4 * lane);
+      o[r][1] = *reinterpret_cast<const float2*>(rr + 4 + 4 * lane);
     }
     float mx = M;
 #pragma unroll
-    for (int w = 0; w < kDecodeWarps; ++w) mx = fmaxf(mx, m[w]);
+    for (int r = 0; r < kDecodeWarps; ++r) mx = fmaxf(mx, m[r]);
     if (mx == -INFINITY) continue;
     const float sc = fast_exp2(M - mx);   // 0 while M is -inf
     den *= sc;
-    num *= sc;
 #pragma unroll
-    for (int w = 0; w < kDecodeWarps; ++w) {
-      const float wt = fast_exp2(m[w] - mx);
-      den = fmaf(wt, l[w], den);
-      num = fmaf(wt, o[w], num);
+    for (int c = 0; c < 4; ++c) num[c] *= sc;
+#pragma unroll
+    for (int r = 0; r < kDecodeWarps; ++r) {
+      const float wt = fast_exp2(m[r] - mx);
+      den = fmaf(wt, l[r], den);
+      num[0] = fmaf(wt, o[r][0].x, num[0]);
+      num[1] = fmaf(wt, o[r][0].y, num[1]);
+      num[2] = fmaf(wt, o[r][1].x, num[2]);
+      num[3] = fmaf(wt, o[r][1].y, num[3]);
     }
     M = mx;
   }
-  out[tid] = den > 0.0f ? num / den : 0.0f;
+  if (lane == 0) {
+    s_m[w] = M;
+    s_den[w] = den;
+  }
+#pragma unroll
+  for (int c = 0; c < 4; ++c) s_num[w][4 * lane + c] = num[c];
+  __syncthreads();
+  float Mt = -INFINITY;
+#pragma unroll
+  for (int r = 0; r < 4; ++r) Mt = fmaxf(Mt, s_m[r]);
+  float dt = 0.0f, nt = 0.0f;
+  if (Mt != -INFINITY) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float wt = fast_exp2(s_m[r] - Mt);   // 0 for a run with nothing
+      dt = fmaf(wt, s_den[r], dt);
+      nt = fmaf(wt, s_num[r][tid], nt);
+    }
+  }
+  out[tid] = dt > 0.0f ? nt / dt : 0.0f;
 }
 
-template <int BITS, int ASYM, int KAXIS, int SPEC = 0>
+template <int BITS, int ASYM, int KAXIS, int ES, int SPEC = 0>
 const void* kernel_of() {
-  return reinterpret_cast<const void*>(&decode_kernel<BITS, ASYM, KAXIS, SPEC>);
+  return reinterpret_cast<const void*>(&decode_kernel<BITS, ASYM, KAXIS, ES, SPEC>);
 }
 
 }  // namespace
 
 const void* decode_kernel_ptr(const Geo& g) {
-  if (spec_int4_kivi(g)) return kernel_of<4, 0, 1, 1>();
-  const int key = (g.bits == 8 ? 0 : g.bits == 4 ? 1 : 2) * 4 + g.asym * 2 + g.k_axis;
+  if (spec_int4_kivi(g)) return kernel_of<4, 0, 1, 2, 1>();
+  const int key = ((g.bits == 8 ? 0 : g.bits == 4 ? 1 : 2) * 4 + g.asym * 2 + g.k_axis) * 2 + (g.es == 4);
   switch (key) {
-    case 0: return kernel_of<8, 0, 0>();
-    case 1: return kernel_of<8, 0, 1>();
-    case 2: return kernel_of<8, 1, 0>();
-    case 3: return kernel_of<8, 1, 1>();
-    case 4: return kernel_of<4, 0, 0>();
-    case 5: return kernel_of<4, 0, 1>();
-    case 6: return kernel_of<4, 1, 0>();
-    case 7: return kernel_of<4, 1, 1>();
-    case 8: return kernel_of<2, 0, 0>();
-    case 9: return kernel_of<2, 0, 1>();
-    case 10: return kernel_of<2, 1, 0>();
-    default: return kernel_of<2, 1, 1>();
+#define KVQ_CASE(k, b, as, ax) \
+    case 2 * (k): return kernel_of<b, as, ax, 2>(); \
+    case 2 * (k) + 1: return kernel_of<b, as, ax, 4>();
+    KVQ_CASE(0, 8, 0, 0) KVQ_CASE(1, 8, 0, 1) KVQ_CASE(2, 8, 1, 0) KVQ_CASE(3, 8, 1, 1)
+    KVQ_CASE(4, 4, 0, 0) KVQ_CASE(5, 4, 0, 1) KVQ_CASE(6, 4, 1, 0) KVQ_CASE(7, 4, 1, 1)
+    KVQ_CASE(8, 2, 0, 0) KVQ_CASE(9, 2, 0, 1) KVQ_CASE(10, 2, 1, 0) KVQ_CASE(11, 2, 1, 1)
+#undef KVQ_CASE
+    default: return nullptr;
   }
 }
 

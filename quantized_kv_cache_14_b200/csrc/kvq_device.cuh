@@ -31,6 +31,14 @@ __host__ __device__ constexpr uint32_t bf16x2_of(float x) {
   return (__builtin_bit_cast(uint32_t, x) >> 16) * 0x10001u;
 }
 
+// fp16 bit pattern, twice, of a float exactly representable as a normal fp16
+// (compile time).
+__host__ __device__ constexpr uint32_t f16x2_of(float x) {
+  const uint32_t b = __builtin_bit_cast(uint32_t, x);
+  const uint32_t h = ((b >> 16) & 0x8000u) | ((((b >> 23) & 0xFFu) - 112u) << 10) | ((b >> 13) & 0x3FFu);
+  return (x == 0.0f ? 0u : h) * 0x10001u;
+}
+
 // ---------------------------------------------------------------------------
 // PTX wrappers.
 // ---------------------------------------------------------------------------
@@ -46,6 +54,22 @@ __device__ __forceinline__ uint32_t bf2_fma(uint32_t a, uint32_t b, uint32_t c) 
   uint32_t r;
   asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
   return r;
+}
+
+__device__ __forceinline__ uint32_t h2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t r;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+
+// D += A * B, m16n8k16, fp16 operands, fp32 accumulation.
+__device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                        uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 // D += A * B, m16n8k16, bf16 operands, fp32 accumulation.
@@ -204,6 +228,52 @@ __device__ __forceinline__ uint32_t byte_pair(uint32_t w, int x) {
   const uint32_t hr = and_xor(vhi, 0x000F000Fu, SIGNED ? 0x43084308u : 0x43004300u);
   const uint32_t hi16 = bf2_fma(hr, bf16x2_of(16.0f), SIGNED ? bf16x2_of(-2176.0f) : bf16x2_of(-2048.0f));
   return bf2_fma(lo, bf16x2_of(1.0f), hi16);
+}
+
+// ---------------------------------------------------------------------------
+// Unpacking codes into fp16x2 operand registers.
+//
+// An fp16 with exponent field 25 holds 1024 + m for a 10-bit integer m in its
+// mantissa bits, so OR-ing a field that sits anywhere inside the low 10 bits of
+// each half into 0x6400 gives 1024 + field * 2^pos exactly; one fp16x2 FMA
+// scales by 2^-pos and removes the 1024 (and a signed code's offset).  A
+// nibble at bit 4 or a byte at bit 0 therefore needs no shift, which leaves one
+// shift per word of nibbles or bytes.  Two's complement fields become offset
+// binary by flipping their top bit in the same LOP3.
+// ---------------------------------------------------------------------------
+
+// 4-bit fields at bit 4x (low half) and 16 + 4x (high half) -> fp16x2.
+template <bool SIGNED>
+__device__ __forceinline__ uint32_t nib_pair_h(uint32_t w, int x) {
+  const uint32_t v = x >= 2 ? (w >> 8) : w;
+  const int y = x & 1;   // field at bit 4y of v
+  const uint32_t r = and_xor(v, 0x000F000Fu << (4 * y), 0x64006400u | (SIGNED ? (0x00080008u << (4 * y)) : 0u));
+  // r = 1024 + 16^y f', f' the field (top bit flipped when signed)
+  return h2_fma(r, y ? f16x2_of(0.0625f) : f16x2_of(1.0f),
+                y ? f16x2_of(SIGNED ? -72.0f : -64.0f) : f16x2_of(SIGNED ? -1032.0f : -1024.0f));
+}
+
+// 2-bit fields at bit 2x and 16 + 2x, x in [0, 8) -> fp16x2.
+template <bool SIGNED>
+__device__ __forceinline__ uint32_t crumb_pair_h(uint32_t w, int x) {
+  // fields 0..4 read from w, 5..7 from w >> 10, at local position y
+  const uint32_t v = x >= 5 ? (w >> 10) : w;
+  const int y = x >= 5 ? x - 5 : x;
+  const uint32_t m = 0x00030003u << (2 * y);
+  const uint32_t k = 0x64006400u | (SIGNED ? (0x00020002u << (2 * y)) : 0u);
+  const uint32_t r = and_xor(v, m, k);
+  // r = 1024 + 4^y c'  ->  c - offset = r / 4^y - 1024 / 4^y - offset
+  const float off = SIGNED ? 2.0f : 0.0f;
+  const float inv = y == 0 ? 1.0f : y == 1 ? 0.25f : y == 2 ? 0.0625f : y == 3 ? 0.015625f : 0.00390625f;
+  return h2_fma(r, f16x2_of(inv), f16x2_of(-1024.0f * inv - off));
+}
+
+// 8-bit fields at byte x and byte x + 2 (x in {0, 1}) -> fp16x2.
+template <bool SIGNED>
+__device__ __forceinline__ uint32_t byte_pair_h(uint32_t w, int x) {
+  const uint32_t v = x ? (w >> 8) : w;
+  const uint32_t r = and_xor(v, 0x00FF00FFu, SIGNED ? 0x64806480u : 0x64006400u);
+  return h2_fma(r, f16x2_of(1.0f), f16x2_of(SIGNED ? -1152.0f : -1024.0f));
 }
 
 // ---------------------------------------------------------------------------
