@@ -532,6 +532,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
   float cs = C;               // score scale: C times the power of two taken out of the fp16 operand
   float bias_t = 0.0f;        // channel-axis zero-points: key bias of head tq for the loaded group
   uint32_t qw[4][2];          // channel axis: q of head h at key-list channels 4*lane .. 4*lane+3
+  uint32_t qh[4][2];          // the same as fp16, scaled by a power of two per pair (fp16 scales)
   float qsum[4] = {0.0f, 0.0f, 0.0f, 0.0f};   // token-axis zero-points: sum of q per key group
 
   auto qrow = [&](int row, int h, int head) {
@@ -620,6 +621,30 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
         qw[h2][0] = live ? *reinterpret_cast<const uint32_t*>(qr + key_channel(f)) : 0u;
         qw[h2][1] = live ? *reinterpret_cast<const uint32_t*>(qr + key_channel(f + 2)) : 0u;
       }
+      if (ES == 2) {
+        // q as fp16 with the largest |q| of the pair in [1/2, 1): then
+        // q * s stays below 65504 for every fp16 scale s
+        float amax = 0.0f;
+#pragma unroll
+        for (int h2 = 0; h2 < 4; ++h2)
+#pragma unroll
+          for (int e = 0; e < 2; ++e)
+            amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(qw[h2][e] << 16)),
+                                     fabsf(__uint_as_float(qw[h2][e] & 0xFFFF0000u))));
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const int ex = amax > 0.0f ? min(max(int((__float_as_uint(amax) >> 23) & 0xFF) - 127 + 1, -100), 100) : 0;
+        const float down = pow2f(-ex);
+#pragma unroll
+        for (int h2 = 0; h2 < 4; ++h2)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const __half2 v = __floats2half2_rn(__uint_as_float(qw[h2][e] << 16) * down,
+                                                __uint_as_float(qw[h2][e] & 0xFFFF0000u) * down);
+            qh[h2][e] = *reinterpret_cast<const uint32_t*>(&v);
+          }
+        cs = C * pow2f(ex);
+      }
     } else {
       const float down = load_bq_f16(row, h);
       if (ASYM) {
@@ -643,11 +668,60 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
     const int lg_ppg = g.lg_gk - g.lg_P;   // pages per key group, log2
     const uint8_t* km = stg + ((gi << lg_ppg) + (f >> g.lg_kslice)) * g.chunk_used + g.off_Km;
     const int off = f & (g.kslice - 1);
+    const int t0 = lane >> 3, j = lane & 7;
+    auto put = [&](int h2, uint32_t h0, uint32_t h1, uint32_t l0, uint32_t l1) {
+      const int thi = 8 * h2 + t0, tlo = thi + 4;   // lanes (gq = 2 h2 | 2 h2 + 1, tq = t0)
+      *reinterpret_cast<uint2*>(qbw + thi * 16 + 4 * ((j >> 1) ^ ((thi >> 1) & 3)) + 2 * (j & 1)) =
+          make_uint2(h0, h1);
+      *reinterpret_cast<uint2*>(qbw + tlo * 16 + 4 * ((j >> 1) ^ ((tlo >> 1) & 3)) + 2 * (j & 1)) =
+          make_uint2(l0, l1);
+    };
+    if constexpr (ES == 2) {
+      // fp16 scales: q'_hi = f16(q s) and q'_lo = f16(q s - q'_hi) by one fp16
+      // multiply and one fp16 FMA per pair (the FMA's residual is exact, so
+      // q'_hi + q'_lo = q s exactly unless a part underflows)
+      const uint2 sr = *reinterpret_cast<const uint2*>(km + off * 2);
+      const __half2 s01 = *reinterpret_cast<const __half2*>(&sr.x), s23 = *reinterpret_cast<const __half2*>(&sr.y);
+      __syncwarp();   // every lane has read the previous operand
+#pragma unroll
+      for (int h2 = 0; h2 < 4; ++h2) {
+        const __half2 qa = *reinterpret_cast<const __half2*>(&qh[h2][0]);
+        const __half2 qb = *reinterpret_cast<const __half2*>(&qh[h2][1]);
+        const __half2 ha = __hmul2(qa, s01), hb = __hmul2(qb, s23);
+        const __half2 la = __hfma2(qa, s01, __hneg2(ha)), lb = __hfma2(qb, s23, __hneg2(hb));
+        put(h2, *reinterpret_cast<const uint32_t*>(&ha), *reinterpret_cast<const uint32_t*>(&hb),
+            *reinterpret_cast<const uint32_t*>(&la), *reinterpret_cast<const uint32_t*>(&lb));
+      }
+      if (ASYM) {
+        const uint2 zr = *reinterpret_cast<const uint2*>(km + (g.kslice + off) * 2);
+        const float2 z01 = __half22float2(*reinterpret_cast<const __half2*>(&zr.x));
+        const float2 z23 = __half22float2(*reinterpret_cast<const __half2*>(&zr.y));
+        float dz[4];
+#pragma unroll
+        for (int h2 = 0; h2 < 4; ++h2) {
+          dz[h2] = __uint_as_float(qw[h2][0] << 16) * z01.x + __uint_as_float(qw[h2][0] & 0xFFFF0000u) * z01.y +
+                   __uint_as_float(qw[h2][1] << 16) * z23.x + __uint_as_float(qw[h2][1] & 0xFFFF0000u) * z23.y;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) dz[h2] += __shfl_xor_sync(0xffffffffu, dz[h2], o);
+        }
+        const int ht = min(tq, g.G - 1);
+        bias_t = C * (ht == 0 ? dz[0] : ht == 1 ? dz[1] : ht == 2 ? dz[2] : dz[3]);
+      }
+      __syncwarp();
+      const uint4* qb = reinterpret_cast<const uint4*>(qbw + lane * 16);
+      const int sw = (lane >> 1) & 3;
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const uint4 x = qb[v ^ sw];
+        bq[2 * v][0] = x.x; bq[2 * v][1] = x.y; bq[2 * v + 1][0] = x.z; bq[2 * v + 1][1] = x.w;
+      }
+      bq_bf16 = false;
+      return;
+    }
     float sc[4];
     meta4(km, off, ES, sc);
     float zc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     if (ASYM) meta4(km, g.kslice + off, ES, zc);
-    const int t0 = lane >> 3, j = lane & 7;
     float dz[4];
     float x[4][4];
     float amax = 0.0f;
@@ -672,11 +746,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
       uint32_t h0, l0, h1, l1;
       split2h(x[h2][0] * down, x[h2][1] * down, h0, l0);
       split2h(x[h2][2] * down, x[h2][3] * down, h1, l1);
-      const int thi = 8 * h2 + t0, tlo = thi + 4;   // lanes (gq = 2 h2 | 2 h2 + 1, tq = t0)
-      *reinterpret_cast<uint2*>(qbw + thi * 16 + 4 * ((j >> 1) ^ ((thi >> 1) & 3)) + 2 * (j & 1)) =
-          make_uint2(h0, h1);
-      *reinterpret_cast<uint2*>(qbw + tlo * 16 + 4 * ((j >> 1) ^ ((tlo >> 1) & 3)) + 2 * (j & 1)) =
-          make_uint2(l0, l1);
+      put(h2, h0, h1, l0, l1);
     }
     if (ASYM) {
 #pragma unroll
@@ -744,19 +814,39 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
     const int n = g.nvg;
     uint32_t b0 = 0, b1 = 0;
     float zs = 0.0f;
+    // fp16 value product: p = p_hi + p_lo in fp16 once per sub-tile; per value
+    // group p' = p s is then f16(p_hi s) plus f16(p_lo s + the exact residual
+    // of p_hi s), one multiply and two FMAs per pair (relative error 2^-21)
+    uint32_t pha = 0, pla = 0, phb = 0, plb = 0;
+    if (PVH) {
+      split2h(pa0, pb0, pha, pla);
+      split2h(pa1, pb1, phb, plb);
+    }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       if ((i & ((1 << vg_shift) - 1)) == 0) {
         const int gi = i >> vg_shift;
         uint32_t h0, l0, h1, l1;
-        const float x0 = pa0 * meta_at(sb.vms, (2 * tq) * n + gi, ES);
-        const float x1 = pb0 * meta_at(sb.vms, (2 * tq + 1) * n + gi, ES);
-        const float x2 = pa1 * meta_at(sb.vms, (2 * tq + 8) * n + gi, ES);
-        const float x3 = pb1 * meta_at(sb.vms, (2 * tq + 9) * n + gi, ES);
         if (PVH) {
-          split2h(x0, x1, h0, l0);
-          split2h(x2, x3, h1, l1);
+          const uint16_t* vs = reinterpret_cast<const uint16_t*>(sb.vms);
+          const __half2 sa2 = __halves2half2(__ushort_as_half(vs[(2 * tq) * n + gi]),
+                                             __ushort_as_half(vs[(2 * tq + 1) * n + gi]));
+          const __half2 sb2 = __halves2half2(__ushort_as_half(vs[(2 * tq + 8) * n + gi]),
+                                             __ushort_as_half(vs[(2 * tq + 9) * n + gi]));
+          auto two = [](uint32_t ph, uint32_t pl, __half2 sv, uint32_t& hi, uint32_t& lo) {
+            const __half2 a = *reinterpret_cast<const __half2*>(&ph), b = *reinterpret_cast<const __half2*>(&pl);
+            const __half2 h = __hmul2(a, sv);
+            const __half2 l = __hfma2(b, sv, __hfma2(a, sv, __hneg2(h)));
+            hi = *reinterpret_cast<const uint32_t*>(&h);
+            lo = *reinterpret_cast<const uint32_t*>(&l);
+          };
+          two(pha, pla, sa2, h0, l0);
+          two(phb, plb, sb2, h1, l1);
         } else {
+          const float x0 = pa0 * meta_at(sb.vms, (2 * tq) * n + gi, ES);
+          const float x1 = pb0 * meta_at(sb.vms, (2 * tq + 1) * n + gi, ES);
+          const float x2 = pa1 * meta_at(sb.vms, (2 * tq + 8) * n + gi, ES);
+          const float x3 = pb1 * meta_at(sb.vms, (2 * tq + 9) * n + gi, ES);
           split2(x0, x1, h0, l0);
           split2(x2, x3, h1, l1);
         }
