@@ -40,8 +40,10 @@ namespace kvq {
 namespace {
 
 constexpr uint64_t kWaitNs = 2000000000ull;   // give up on a copy after 2 s
-constexpr int kQbufBytes = 32 * 16 * 4;   // one warp's q' operand: 32 lanes x 16 words
-constexpr int kScoreBytes = 8 * 32 * 4;   // one warp's scores / weights of a 64-token chunk
+// One warp's scratch: half of its q' operand in flight (32 lanes x 8 words), or
+// the scores / weights of a 64-token chunk (8 x 32 floats); the two uses never
+// overlap in time.
+constexpr int kScratchBytes = 32 * 8 * 4;
 
 struct SmemLayout {
   int stages, qbuf, bars, flag, total;
@@ -51,7 +53,7 @@ __host__ __device__ inline SmemLayout smem_layout(int B, const DecodePipe& p) {
   SmemLayout L;
   L.stages = ((B + 1 + 32) * 4 + 127) / 128 * 128;      // prefix table + scan scratch
   L.qbuf = L.stages + p.nstages * p.stage_bytes;
-  L.bars = L.qbuf + kDecodeWarps * (kQbufBytes + kScoreBytes);
+  L.bars = L.qbuf + kDecodeWarps * kScratchBytes;
   L.flag = L.bars + 2 * p.nstages * 8;
   L.total = L.flag + 16;
   return L;
@@ -522,8 +524,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
   const float C = a.qk_scale;
   const int vg_shift = __ffs(g.g_v >> 4) - 1;               // channel tiles per value group, log2
   const int kg_shift = KAXIS ? 3 : __ffs(g.g_k >> 4) - 1;   // k-steps per key group, log2
-  uint32_t* qbw = reinterpret_cast<uint32_t*>(smem + L.qbuf + warp * kQbufBytes);   // this warp's q'
-  float* spw = reinterpret_cast<float*>(smem + L.qbuf + kDecodeWarps * kQbufBytes) + warp * 8 * 32;
+  uint32_t* qbw = reinterpret_cast<uint32_t*>(smem + L.qbuf + warp * kScratchBytes);   // this warp's scratch
+  float* spw = reinterpret_cast<float*>(qbw);
 
   State st;
   state_reset(st);
@@ -669,12 +671,41 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
     const uint8_t* km = stg + ((gi << lg_ppg) + (f >> g.lg_kslice)) * g.chunk_used + g.off_Km;
     const int off = f & (g.kslice - 1);
     const int t0 = lane >> 3, j = lane & 7;
+    uint32_t qv[4][4];   // per head: hi pair, hi pair, lo pair, lo pair of this lane's 4 channels
     auto put = [&](int h2, uint32_t h0, uint32_t h1, uint32_t l0, uint32_t l1) {
-      const int thi = 8 * h2 + t0, tlo = thi + 4;   // lanes (gq = 2 h2 | 2 h2 + 1, tq = t0)
-      *reinterpret_cast<uint2*>(qbw + thi * 16 + 4 * ((j >> 1) ^ ((thi >> 1) & 3)) + 2 * (j & 1)) =
-          make_uint2(h0, h1);
-      *reinterpret_cast<uint2*>(qbw + tlo * 16 + 4 * ((j >> 1) ^ ((tlo >> 1) & 3)) + 2 * (j & 1)) =
-          make_uint2(l0, l1);
+      qv[h2][0] = h0; qv[h2][1] = h1; qv[h2][2] = l0; qv[h2][3] = l1;
+    };
+    // Lane L's values of head h belong to lanes (gq = 2h | 2h + 1, tq = L / 8),
+    // k-step L % 8.  Two passes over the 1 KB scratch move k-steps 0-3, then
+    // 4-7; each reader's 8 words are two 16-byte slots, XOR-swizzled so the
+    // reads are conflict-free.
+    auto transpose = [&]() {
+#pragma unroll
+      for (int pass = 0; pass < 2; ++pass) {
+        __syncwarp();   // the scratch is free
+        if ((j >> 2) == pass) {
+          const int j4 = j & 3;
+#pragma unroll
+          for (int h2 = 0; h2 < 4; ++h2) {
+            const int thi = 8 * h2 + t0, tlo = thi + 4;
+            *reinterpret_cast<uint2*>(qbw + thi * 8 + 4 * ((j4 >> 1) ^ ((thi >> 2) & 1)) + 2 * (j4 & 1)) =
+                make_uint2(qv[h2][0], qv[h2][1]);
+            *reinterpret_cast<uint2*>(qbw + tlo * 8 + 4 * ((j4 >> 1) ^ ((tlo >> 2) & 1)) + 2 * (j4 & 1)) =
+                make_uint2(qv[h2][2], qv[h2][3]);
+          }
+        }
+        __syncwarp();
+        const uint4* qb = reinterpret_cast<const uint4*>(qbw + lane * 8);
+        const int sw = (lane >> 2) & 1;
+#pragma unroll
+        for (int v = 0; v < 2; ++v) {
+          const uint4 x = qb[v ^ sw];
+          bq[4 * pass + 2 * v][0] = x.x; bq[4 * pass + 2 * v][1] = x.y;
+          bq[4 * pass + 2 * v + 1][0] = x.z; bq[4 * pass + 2 * v + 1][1] = x.w;
+        }
+      }
+      __syncwarp();   // all reads done before the scratch holds scores
+      bq_bf16 = false;
     };
     if constexpr (ES == 2) {
       // fp16 scales: q'_hi = f16(q s) and q'_lo = f16(q s - q'_hi) by one fp16
@@ -682,7 +713,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
       // q'_hi + q'_lo = q s exactly unless a part underflows)
       const uint2 sr = *reinterpret_cast<const uint2*>(km + off * 2);
       const __half2 s01 = *reinterpret_cast<const __half2*>(&sr.x), s23 = *reinterpret_cast<const __half2*>(&sr.y);
-      __syncwarp();   // every lane has read the previous operand
 #pragma unroll
       for (int h2 = 0; h2 < 4; ++h2) {
         const __half2 qa = *reinterpret_cast<const __half2*>(&qh[h2][0]);
@@ -707,15 +737,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
         const int ht = min(tq, g.G - 1);
         bias_t = C * (ht == 0 ? dz[0] : ht == 1 ? dz[1] : ht == 2 ? dz[2] : dz[3]);
       }
-      __syncwarp();
-      const uint4* qb = reinterpret_cast<const uint4*>(qbw + lane * 16);
-      const int sw = (lane >> 1) & 3;
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        const uint4 x = qb[v ^ sw];
-        bq[2 * v][0] = x.x; bq[2 * v][1] = x.y; bq[2 * v + 1][0] = x.z; bq[2 * v + 1][1] = x.w;
-      }
-      bq_bf16 = false;
+      transpose();
       return;
     }
     float sc[4];
@@ -740,7 +762,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
     const int ex = amax > 0.0f ? min(max(int((__float_as_uint(amax) >> 23) & 0xFF) - 127 - 14, -100), 100) : 0;
     const float down = pow2f(-ex);
     cs = C * pow2f(ex);
-    __syncwarp();   // every lane has read the previous operand
 #pragma unroll
     for (int h2 = 0; h2 < 4; ++h2) {
       uint32_t h0, l0, h1, l1;
@@ -756,15 +777,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
       const int ht = min(tq, g.G - 1);
       bias_t = C * (ht == 0 ? dz[0] : ht == 1 ? dz[1] : ht == 2 ? dz[2] : dz[3]);
     }
-    __syncwarp();
-    const uint4* qb = reinterpret_cast<const uint4*>(qbw + lane * 16);
-    const int sw = (lane >> 1) & 3;
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const uint4 x = qb[v ^ sw];
-      bq[2 * v][0] = x.x; bq[2 * v][1] = x.y; bq[2 * v + 1][0] = x.z; bq[2 * v + 1][1] = x.w;
-    }
-    bq_bf16 = false;
+    transpose();
   };
 
   // Scores of one 16-token quantized sub-tile: tokens gq, gq + 8 for head tq,
@@ -1187,8 +1200,14 @@ cudaError_t plan_decode(const Geo& g, int max_B, DecodePipe* out) {
   // aim for three resident CTAs per SM (about 72 KB of shared memory each)
   // with two stages per consumer warp; the stage count stays a multiple of
   // the warp count so warp w always owns stages w, w + 4, ...
+  int per_sm = 0;
+  e = cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+  if (e != cudaSuccess) return e;
+  int reserved = 0;
+  e = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+  if (e != cudaSuccess) return e;
   p.nstages = 2 * kDecodeWarps;
-  if (size_t(smem_layout(max_B, p).total) > size_t(72 * 1024)) p.nstages = kDecodeWarps;
+  if (3 * (size_t(smem_layout(max_B, p).total) + size_t(reserved)) > size_t(per_sm)) p.nstages = kDecodeWarps;
   if (size_t(smem_layout(max_B, p).total) > size_t(max_optin)) return cudaErrorInvalidConfiguration;
   const size_t smem = size_t(smem_layout(max_B, p).total);
   if (smem > size_t(max_optin)) return cudaErrorInvalidConfiguration;
