@@ -8,7 +8,9 @@ Prints ONE JSON line (rank 0).  `value` is decode-attention KV GB/s: the
 algorithmic bytes of the decode call (codes, scales, zero-points, BF16 window
 rows, q, out, block-table entries) over its device time, summed over ranks and
 divided by the max over ranks.  Inputs live in HBM before the timed region; L2
-is flushed (256 MB write, untimed) before every timed step.  `e2e` is the same
+is flushed before every timed step (untimed): a 256 MB write, then a read of
+another 256 MB so that the write's dirty lines are written back before the
+timed region and the timed kernels start on a cold, clean L2.  `e2e` is the same
 metric through the C ABI with host buffers: pinned H2D of the step's new K/V
 and q and D2H of the attention output inside the timed region.  With N > 1 every
 rank runs its own replica (sequences shard across GPUs; no collective is on the
@@ -244,13 +246,15 @@ def run_gpu(args, rank, ws, dist):
     out = torch.empty((B, w.h_q, D), dtype=torch.float32, device=dev)
     out_host = torch.empty_like(out, device="cpu").pin_memory()
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_rd = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     torch.cuda.synchronize()
     assert cache.sync_status() == 0
 
     def one_step(s, e2e, evs):
         nonlocal lens
         ev0, ev1, ev2 = evs
-        flush.zero_()                                   # untimed: evicts L2
+        flush.zero_()                                   # untimed: evicts L2 ...
+        flush_rd.sum()                                  # ... and writes the dirty lines back
         ev0.record()
         if e2e:
             kh, vh, qh = host_in[s]
@@ -414,7 +418,7 @@ def workload_config(w, lens):
                   f"{'fp32' if f.scale_fp32 else 'fp16'} scales, page {f.page}, BF16 window {f.residual}",
         "batch": w.batch, "h_q": w.h_q, "h_kv": w.h_kv, "d_h": D,
         "seq_len_min": int(min(lens)), "seq_len_max": int(max(lens)),
-        "l2": "flushed before every timed step (256 MB write, untimed)",
+        "l2": "flushed before every timed step (256 MB write then 256 MB read, untimed)",
         "step": "append 1 token per sequence (quantize/window/flush) + decode attention",
         "parallelism": "replicas",
     }

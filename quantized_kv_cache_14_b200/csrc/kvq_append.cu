@@ -377,8 +377,16 @@ cudaError_t launch_flush(const Geo& g, const DevState& d, const PlanView& p, con
   const size_t smem = flush_smem_bytes(g);
   return by_format(g, [&](auto B, auto A) {
     auto kern = flush_kernel<decltype(B)::value, decltype(A)::value>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    // the shared-memory limit only grows: set it once per kernel, device and size
+    static thread_local size_t limit_set[32] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    if (dev >= 32 || smem > limit_set[dev]) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+      if (e != cudaSuccess) return e;
+      if (dev < 32) limit_set[dev] = smem;
+    }
     kern<<<dim3(p.n_flush, g.h_kv), kFlushThreads, smem, s>>>(g, d, p, k, v);
     ++*launches;
     return cudaGetLastError();

@@ -15,23 +15,21 @@
 //    tiles.  A persistent grid gives every CTA a contiguous, equal share of
 //    the whole list (split-K whose split points come from balance), so all SMs
 //    stay busy for any length mix.
-//  * A CTA is one producer warp and four consumer warps around a ring of
-//    shared-memory stages.  The producer's lane 0 fills a stage with bulk
-//    asynchronous copies (TMA, cp.async.bulk) of whole page chunks completing
-//    on the stage's "full" mbarrier; the consumers release it on its "empty"
-//    mbarrier.  Each consumer warp takes one 16-token sub-tile of a unit.
+//  * A CTA is four warps.  Warp w computes every fourth unit of the CTA's
+//    share and stages its own units: two shared-memory stages per warp, each
+//    filled by bulk asynchronous copies (TMA, cp.async.bulk) of whole page
+//    chunks completing on the stage's mbarrier, issued two units ahead with
+//    the block ids loaded one unit earlier still.
 //  * The g = h_q / h_kv query heads sharing a kv head are processed together:
 //    every cached byte is read once.  Scores K_hat q'^T and P' V_hat run on
-//    mma.sync m16n8k16 with bf16 operands and fp32 accumulation.  Codes are
-//    exact in bf16; the scale goes into the other operand (q' = q * s_channel
-//    per key group, computed once per unit by the four consumer warps into
-//    shared memory; p' = p * s_token per value group), split into bf16 hi + lo
-//    columns (4 heads x {hi, lo} = the 8 mma columns, 16 significant bits).
-//    Zero-points enter as a per-group key bias and a p-weighted value sum.
-//  * Online softmax in the log2 domain with warp-shuffle reductions; the
-//    running max moves only when it grows by more than 8 (p <= 256).  Each
-//    consumer warp leaves one (m, l, o) partial per pair its CTA touched; the
-//    merge kernel combines them by log-sum-exp in a fixed order.
+//    mma.sync m16n8k16 with fp32 accumulation.  Codes are exact small integers
+//    in fp16; the scale goes into the other operand (q' = q * s_channel per key
+//    group, p' = p * s_token per value group), split into hi + lo parts that
+//    take two of the 8 mma columns per head (4 heads x {hi, lo}).  Zero-points
+//    enter as a per-group key bias and a p-weighted value sum.
+//  * Online softmax in the log2 domain with warp-shuffle reductions, one step
+//    per 64 tokens.  Each warp leaves one (m, l, o) record per pair its CTA
+//    touched; the merge kernel combines them by log-sum-exp in a fixed order.
 #include <cstdint>
 
 #include "kvq_device.cuh"
@@ -51,10 +49,10 @@ struct SmemLayout {
 
 __host__ __device__ inline SmemLayout smem_layout(int B, const DecodePipe& p) {
   SmemLayout L;
-  L.stages = ((B + 1 + 32) * 4 + 127) / 128 * 128;      // prefix table + scan scratch
+  L.stages = ((B + 1 + 32 + 3 * B) * 4 + 127) / 128 * 128;   // prefix, scan scratch, per-row info
   L.qbuf = L.stages + p.nstages * p.stage_bytes;
   L.bars = L.qbuf + kDecodeWarps * kScratchBytes;
-  L.flag = L.bars + 2 * p.nstages * 8;
+  L.flag = L.bars + p.nstages * 8;
   L.total = L.flag + 16;
   return L;
 }
@@ -146,10 +144,6 @@ __device__ __forceinline__ bool it_next(It& it, const int32_t* pre, int B, int h
   do { ++it.i; } while (it.i < B && pre[it.i + 1] == pre[it.i]);
   if (it.i < B) it.n = pre[it.i + 1] - pre[it.i];
   return true;   // row changed
-}
-
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
 }
 
 // Bounded wait that also gives up as soon as another warp has aborted.
@@ -362,7 +356,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
   // with the running max exact (p <= 1), p' = p * s fits fp16's range.  Fp32
   // scales keep bf16 operands (fp32 range).
   constexpr bool PVH = ES == 2;
-  constexpr int kPair = 1;   // sub-tiles per trip of the chunk loops (2 measured slower)
   extern __shared__ __align__(128) uint8_t smem[];
   const Geo gs = geo_of<SPEC>(a.g);
   const Geo& g = SPEC ? gs : a.g;   // the generic instances read the geometry from the parameters
@@ -371,10 +364,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
   const SmemLayout L = smem_layout(a.B, pp);
   int32_t* s_pre = reinterpret_cast<int32_t*>(smem);
   int32_t* s_scr = s_pre + (a.B + 1);
+  int32_t* s_row = s_scr + 32;   // per row: sequence, quantized and window positions attended
   uint8_t* stages = smem + L.stages;
   const uint32_t stage0 = smem_addr(stages);
   const uint32_t full0 = smem_addr(smem + L.bars);
-  const uint32_t empty0 = full0 + 8 * pp.nstages;
   volatile int32_t* abort_flag = reinterpret_cast<int32_t*>(smem + L.flag);
 
   // the merge grid may be scheduled now; it waits for this grid to complete
@@ -384,12 +377,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
   for (int i = tid; i < a.B; i += blockDim.x) {
     const RowInfo ri = row_info(a, i, blockIdx.x == 0);
     s_pre[i + 1] = ri.nq + ri.nr;
+    s_row[3 * i] = ri.seq;
+    s_row[3 * i + 1] = ri.qa;
+    s_row[3 * i + 2] = ri.ra;
   }
   if (tid == 0) {
-    for (int s = 0; s < pp.nstages; ++s) {
-      mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, 1);   // released by the one warp that owns the unit
-    }
+    for (int s = 0; s < pp.nstages; ++s) mbar_init(full0 + 8 * s, 1);
     *abort_flag = 0;
     mbar_init_fence();
   }
@@ -402,114 +395,110 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
   const int64_t c0 = int64_t(blockIdx.x) * U / a.grid, c1 = int64_t(blockIdx.x + 1) * U / a.grid;
   if (c0 >= c1) return;
   const int N = int(c1 - c0);
-
-  if (warp == kDecodeWarps) {
-    // ---------------------------- producer ----------------------------------
-    // The whole warp: a window of 32 block-table entries is fetched with one
-    // coalesced load and read by shuffle, and a unit's copies are issued in
-    // parallel, one lane per page (or per 16-token sub-tile).
-    constexpr uint32_t FULL = 0xffffffffu;
-    It it;
-    it_seek(it, s_pre, a.B, g.h_kv, c0);
-    RowInfo ri = row_info(a, it.i, false);
-    int win_row = -1, win_base = 0;
-    int32_t win = -1;
-    int s = 0;
-    uint32_t ph = 0;
-    int issued = 0;
-    const int vrow = 16 * g.nvg * ES, krow = 16 * g.nkg * ES;
-    for (int n = 0; n < N; ++n) {
-      const uint32_t dst = stage0 + s * pp.stage_bytes;
-      const uint32_t bar = full0 + 8 * s;
-      bool bad = false;
-      uint32_t total = 0;
-      int ncopy = 0;          // lanes [0, ncopy) issue copies
-      int32_t blk = 0;        // this lane's block
-      int tok = 0;            // token axis: this lane's sub-tile's first token
-      if (it.k < ri.nq) {
-        const int T0 = it.k * pp.sup;
-        const int valid = min(pp.sup, ri.qa - T0);
-        const int lb0 = T0 >> g.lg_P;
-        int npg;
-        if (KAXIS) {
-          npg = ((valid + g.g_k - 1) >> g.lg_gk) << (g.lg_gk - g.lg_P);   // whole key groups
-          ncopy = npg;
-          total = uint32_t(npg * g.chunk_used);
-        } else {
-          const int nsub = (valid + 15) >> 4;
-          npg = ((T0 + 16 * nsub - 1) >> g.lg_P) - lb0 + 1;
-          ncopy = nsub;
-          total = uint32_t(nsub) * (g.P == 16 ? uint32_t(g.chunk_used)
-                                              : uint32_t(2 * g.sub_bytes + (vrow + krow) * (1 + ASYM)));
-          tok = T0 + 16 * min(lane, nsub - 1);
-        }
-        if (it.i != win_row || lb0 < win_base || lb0 + npg > win_base + 32) {
-          win_row = it.i;
-          win_base = lb0;
-          win = lb0 + lane < a.table_stride ? ri.trow[lb0 + lane] : -1;
-        }
-        const int pg = KAXIS ? lane : (tok >> g.lg_P) - lb0;
-        blk = __shfl_sync(FULL, win, (lb0 - win_base + pg) & 31);
-        bad = __any_sync(FULL, lane < ncopy && (blk < 0 || blk >= g.num_blocks));
-      } else {
-        ncopy = 2;
-        total = 2 * 16 * kD * 2;
-      }
-      // every lane waits; the verdict is made warp-uniform before anyone leaves
-      if (n >= pp.nstages && !__all_sync(FULL, wait_or_abort(empty0 + 8 * s, ph ^ 1u, abort_flag))) {
-        if (lane == 0) {
-          atomicOr(a.err, KVQ_DEVERR_TIMEOUT);
-          *abort_flag = 1;
-        }
-        break;
-      }
-      if (bad) {
-        if (lane == 0) {
-          atomicOr(a.err, KVQ_DEVERR_BLOCK_ID);
-          mbar_arrive_expect_tx(bar, 0);
-        }
-      } else {
-        if (lane == 0) mbar_arrive_expect_tx(bar, total);
-        __syncwarp();
-        if (lane < ncopy) {
-          if (it.k >= ri.nq) {
-            const int kr = it.k - ri.nq;
-            const int64_t base = ((int64_t(ri.seq) * g.h_kv + it.h) * g.R + 16 * kr) * kD;
-            bulk_g2s(dst + lane * (16 * kD * 2), (lane ? a.vres : a.kres) + base, 16 * kD * 2, bar);
-          } else {
-            const uint8_t* chunk = a.pool + int64_t(blk) * g.block_bytes + int64_t(it.h) * g.chunk_bytes;
-            if (KAXIS) {
-              bulk_g2s(dst + lane * g.chunk_used, chunk, uint32_t(g.chunk_used), bar);
-            } else if (g.P == 16) {
-              bulk_g2s(dst + lane * pp.qsub, chunk, uint32_t(g.chunk_used), bar);
-            } else {
-              const int u = (tok & (g.P - 1)) >> 4;
-              const uint32_t d = dst + lane * pp.qsub;
-              bulk_g2s(d, chunk + u * g.sub_bytes, g.sub_bytes, bar);
-              bulk_g2s(d + g.sub_bytes, chunk + g.off_V + u * g.sub_bytes, g.sub_bytes, bar);
-              const uint32_t vm = d + 2 * g.sub_bytes, km = vm + g.vm16;
-              bulk_g2s(vm, chunk + g.off_Vm + int64_t(16 * u) * g.nvg * ES, vrow, bar);
-              bulk_g2s(km, chunk + g.off_Km + int64_t(16 * u) * g.nkg * ES, krow, bar);
-              if (ASYM) {
-                bulk_g2s(vm + vrow, chunk + g.off_Vm + int64_t(g.P + 16 * u) * g.nvg * ES, vrow, bar);
-                bulk_g2s(km + krow, chunk + g.off_Km + int64_t(g.P + 16 * u) * g.nkg * ES, krow, bar);
-              }
-            }
-          }
-        }
-      }
-      ++issued;
-      if (it_next(it, s_pre, a.B, g.h_kv) && n + 1 < N) ri = row_info(a, it.i, false);
-      if (++s == pp.nstages) { s = 0; ph ^= 1u; }
-    }
-    // keep the CTA until its last copies have landed (bounded)
-    if (lane == 0)
-      for (int k = 0; k < pp.nstages && k < issued; ++k) {
-        const int n = issued - 1 - k;
-        (void)mbar_wait_bounded(full0 + 8 * (n % pp.nstages), uint32_t((n / pp.nstages) & 1), kWaitNs);
-      }
+  if (pp.nstages != kDecodeWarps && pp.nstages != 2 * kDecodeWarps) {   // stage indexing needs 4 or 8
+    if (tid == 0) atomicOr(a.err, KVQ_DEVERR_TIMEOUT);
     return;
   }
+
+  // row info from the shared cache (no global reads after the prologue)
+  auto rinfo = [&](int i) {
+    RowInfo r;
+    r.seq = s_row[3 * i];
+    r.qa = s_row[3 * i + 1];
+    r.ra = s_row[3 * i + 2];
+    r.nq = (r.qa + pp.sup - 1) >> pp.lg_sup;
+    r.nr = (r.ra + 15) >> 4;
+    r.trow = a.table + int64_t(a.table_by_seq ? r.seq : i) * a.table_stride;
+    return r;
+  };
+  // one unit forward; `n` counts units of the range, row info is refreshed
+  // only while inside it
+  auto step = [&](It& it, RowInfo& ri, int& n) {
+    const bool row_changed = it_next(it, s_pre, a.B, g.h_kv);
+    ++n;
+    if (row_changed && n < N) ri = rinfo(it.i);
+  };
+
+  // ---- staging: each warp fills its own two stages, two units ahead ---------
+  const int vrow = 16 * g.nvg * ES, krow = 16 * g.nkg * ES;
+  // this lane's block for the unit's copies (loaded early so the latency hides
+  // under a unit of compute); -1 when out of the table
+  auto load_blk = [&](const It& it, const RowInfo& ri) -> int32_t {
+    if (it.k >= ri.nq) return 0;   // a BF16 window tile
+    const int T0 = it.k * pp.sup;
+    const int valid = min(pp.sup, ri.qa - T0);
+    int pg, ncopy;
+    if (KAXIS) {
+      ncopy = ((valid + g.g_k - 1) >> g.lg_gk) << (g.lg_gk - g.lg_P);   // whole key groups
+      pg = (T0 >> g.lg_P) + lane;
+    } else {
+      ncopy = (valid + 15) >> 4;
+      pg = (T0 + 16 * min(lane, ncopy - 1)) >> g.lg_P;
+    }
+    if (lane >= ncopy) return 0;
+    return pg < a.table_stride ? ri.trow[pg] : -1;
+  };
+  auto issue = [&](const It& it, const RowInfo& ri, int32_t blk, int sidx) {
+    constexpr uint32_t FULL = 0xffffffffu;
+    const uint32_t dst = stage0 + sidx * pp.stage_bytes;
+    const uint32_t bar = full0 + 8 * sidx;
+    uint32_t total;
+    int ncopy, tok = 0;
+    const bool window = it.k >= ri.nq;
+    if (!window) {
+      const int T0 = it.k * pp.sup;
+      const int valid = min(pp.sup, ri.qa - T0);
+      if (KAXIS) {
+        ncopy = ((valid + g.g_k - 1) >> g.lg_gk) << (g.lg_gk - g.lg_P);
+        total = uint32_t(ncopy * g.chunk_used);
+      } else {
+        ncopy = (valid + 15) >> 4;
+        total = uint32_t(ncopy) * (g.P == 16 ? uint32_t(g.chunk_used)
+                                             : uint32_t(2 * g.sub_bytes + (vrow + krow) * (1 + ASYM)));
+        tok = T0 + 16 * min(lane, ncopy - 1);
+      }
+    } else {
+      ncopy = 2;
+      total = 2 * 16 * kD * 2;
+    }
+    const bool bad = !window && __any_sync(FULL, lane < ncopy && (blk < 0 || blk >= g.num_blocks));
+    // this warp's generic-proxy reads of the stage come before the copies' writes
+    fence_proxy_async();
+    if (bad) {
+      if (lane == 0) {
+        atomicOr(a.err, KVQ_DEVERR_BLOCK_ID);
+        mbar_arrive_expect_tx(bar, 0);
+      }
+      return;
+    }
+    if (lane == 0) mbar_arrive_expect_tx(bar, total);
+    __syncwarp();
+    if (lane >= ncopy) return;
+    if (window) {
+      const int kr = it.k - ri.nq;
+      const int64_t base = ((int64_t(ri.seq) * g.h_kv + it.h) * g.R + 16 * kr) * kD;
+      bulk_g2s(dst + lane * (16 * kD * 2), (lane ? a.vres : a.kres) + base, 16 * kD * 2, bar);
+      return;
+    }
+    const uint8_t* chunk = a.pool + int64_t(blk) * g.block_bytes + int64_t(it.h) * g.chunk_bytes;
+    if (KAXIS) {
+      bulk_g2s(dst + lane * g.chunk_used, chunk, uint32_t(g.chunk_used), bar);
+    } else if (g.P == 16) {
+      bulk_g2s(dst + lane * pp.qsub, chunk, uint32_t(g.chunk_used), bar);
+    } else {
+      const int u = (tok & (g.P - 1)) >> 4;
+      const uint32_t d = dst + lane * pp.qsub;
+      bulk_g2s(d, chunk + u * g.sub_bytes, g.sub_bytes, bar);
+      bulk_g2s(d + g.sub_bytes, chunk + g.off_V + u * g.sub_bytes, g.sub_bytes, bar);
+      const uint32_t vm = d + 2 * g.sub_bytes, km = vm + g.vm16;
+      bulk_g2s(vm, chunk + g.off_Vm + int64_t(16 * u) * g.nvg * ES, vrow, bar);
+      bulk_g2s(km, chunk + g.off_Km + int64_t(16 * u) * g.nkg * ES, krow, bar);
+      if (ASYM) {
+        bulk_g2s(vm + vrow, chunk + g.off_Vm + int64_t(g.P + 16 * u) * g.nvg * ES, vrow, bar);
+        bulk_g2s(km + krow, chunk + g.off_Km + int64_t(g.P + 16 * u) * g.nkg * ES, krow, bar);
+      }
+    }
+  };
 
   // ------------------------------ consumers -----------------------------------
   // Consumer warp w owns the units n of the range with n % 4 == w: it waits for
@@ -842,10 +831,20 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
         uint32_t h0, l0, h1, l1;
         if (PVH) {
           const uint16_t* vs = reinterpret_cast<const uint16_t*>(sb.vms);
-          const __half2 sa2 = __halves2half2(__ushort_as_half(vs[(2 * tq) * n + gi]),
-                                             __ushort_as_half(vs[(2 * tq + 1) * n + gi]));
-          const __half2 sb2 = __halves2half2(__ushort_as_half(vs[(2 * tq + 8) * n + gi]),
-                                             __ushort_as_half(vs[(2 * tq + 9) * n + gi]));
+          __half2 sa2, sb2;
+          if (n == 2) {
+            // rows 2tq, 2tq + 1 (and + 8) hold both groups' scales in 8 bytes
+            const uint2 ra = *reinterpret_cast<const uint2*>(vs + 4 * tq);
+            const uint2 rb = *reinterpret_cast<const uint2*>(vs + 4 * tq + 16);
+            const uint32_t sel = gi ? 0x7632u : 0x5410u;
+            const uint32_t xa = __byte_perm(ra.x, ra.y, sel), xb = __byte_perm(rb.x, rb.y, sel);
+            sa2 = *reinterpret_cast<const __half2*>(&xa);
+            sb2 = *reinterpret_cast<const __half2*>(&xb);
+          } else {
+            sa2 = __halves2half2(__ushort_as_half(vs[(2 * tq) * n + gi]), __ushort_as_half(vs[(2 * tq + 1) * n + gi]));
+            sb2 = __halves2half2(__ushort_as_half(vs[(2 * tq + 8) * n + gi]),
+                                 __ushort_as_half(vs[(2 * tq + 9) * n + gi]));
+          }
           auto two = [](uint32_t ph, uint32_t pl, __half2 sv, uint32_t& hi, uint32_t& lo) {
             const __half2 a = *reinterpret_cast<const __half2*>(&ph), b = *reinterpret_cast<const __half2*>(&pl);
             const __half2 h = __hmul2(a, sv);
@@ -968,96 +967,135 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
   // sub-tiles per softmax chunk: 4, or one key group when groups are shorter
   const int ch = KAXIS ? min(4, g.g_k >> 4) : 4;
 
-  It it;
-  it_seek(it, s_pre, a.B, g.h_kv, c0);
-  RowInfo ri = row_info(a, it.i, false);
-  int cur_pair = -1;
-  int s = 0;
-  uint32_t ph = 0;
-  bool aborted = false;
-  for (int n = 0; n < N; ++n) {
-    const int pair_id = it.i * g.h_kv + it.h;
-    if (pair_id != cur_pair) {
-      if (cur_pair >= 0 && !aborted) emit(cur_pair / g.h_kv, cur_pair % g.h_kv);
-      setup_pair(it.i, it.h);
-      cur_pair = pair_id;
-    }
-    if ((n & (kDecodeWarps - 1)) == warp) {
-      // every lane polls; the warp gives up together, and once any warp has
-      // given up all of them skip the remaining work (but keep the barriers)
-      if (!aborted) {
-        const bool arrived = wait_or_abort(full0 + 8 * s, ph, abort_flag);
-        if (!__all_sync(0xffffffffu, arrived)) {
-          if (lane == 0) {
-            atomicOr(a.err, KVQ_DEVERR_TIMEOUT);
-            *abort_flag = 1;
-          }
-          aborted = true;
-        }
-      }
-      const uint8_t* stg = stages + size_t(s) * pp.stage_bytes;
-      if (aborted) {
-      } else if (it.k < ri.nq) {
-        const int T0 = it.k * pp.sup;
-        const int valid_unit = min(pp.sup, ri.qa - T0);
-        const int nsub = (valid_unit + 15) >> 4;
-        int loaded = -1;
-        for (int c = 0; c < nsub; c += ch) {
-          if (KAXIS && ((16 * c) >> g.lg_gk) != loaded) {
-            loaded = (16 * c) >> g.lg_gk;
-            qprime_job(stg, loaded);
-          }
-          // scores of the chunk's sub-tiles go through this lane's own slots of
-          // the warp scratch, which keeps the loops rolled (small code, no spills)
-          const int nt = min(ch, nsub - c);
-          // two sub-tiles per trip, as independent instruction streams, where
-          // registers allow (an odd last trip re-reads sub-tile nt - 1 and
-          // discards it); one per trip otherwise
-#pragma unroll 1
-          for (int t = 0; t < nt; t += kPair) {
-            const int tokA = 16 * (c + t);
-            float sA0, sA1;
-            score_sub(sub_at(stg, tokA), valid_unit - tokA, sA0, sA1);
-            spw[(2 * t) * 32 + lane] = sA0;
-            spw[(2 * t + 1) * 32 + lane] = sA1;
-            if (kPair == 2) {
-              const int tokB = 16 * (c + min(t + 1, nt - 1));
-              float sB0, sB1;
-              score_sub(sub_at(stg, tokB), t + 1 < nt ? valid_unit - tokB : 0, sB0, sB1);
-              spw[(2 * t + 2) * 32 + lane] = sB0;
-              spw[(2 * t + 3) * 32 + lane] = sB1;
-            }
-          }
-          float sc[8], pc[8];
-#pragma unroll
-          for (int k = 0; k < 8; ++k) sc[k] = k < 2 * nt ? spw[k * 32 + lane] : -INFINITY;
-          softmax_chunk(sc, pc);
-#pragma unroll
-          for (int k = 0; k < 8; ++k) spw[k * 32 + lane] = pc[k];
-#pragma unroll 1
-          for (int t = 0; t < nt; t += kPair) {
-            pv_sub(sub_at(stg, 16 * (c + t)), spw[(2 * t) * 32 + lane], spw[(2 * t + 1) * 32 + lane], true);
-            if (kPair == 2)
-              pv_sub(sub_at(stg, 16 * (c + min(t + 1, nt - 1))), spw[(2 * t + 2) * 32 + lane],
-                     spw[(2 * t + 3) * 32 + lane], t + 1 < nt);
-          }
-        }
-      } else {
-        if (!bq_bf16) {
-          load_bq_from_q(it.i, it.h);
-          bq_bf16 = true;
-          bias_t = 0.0f;
-        }
-        process_window(stg, ri.ra - 16 * (it.k - ri.nq));
-      }
-      // release the stage to the producer
-      __syncwarp();
-      if (lane == 0) mbar_arrive(empty0 + 8 * s);
-    }
-    if (++s == pp.nstages) { s = 0; ph ^= 1u; }
-    if (it_next(it, s_pre, a.B, g.h_kv) && n + 1 < N) ri = row_info(a, it.i, false);
+  // This warp computes units n = warp, warp + 4, ... of the range (K of them);
+  // it owns SPW = nstages / 4 stages (2, or 1 when shared memory is short) and
+  // its k-th unit lives in stage SPW * warp + k % SPW.  The walk iterator
+  // `itc` visits every unit so that a record is left for every pair the CTA
+  // touches; `iti` runs SPW of this warp's units ahead for the copies.
+  const int SPW = pp.nstages / kDecodeWarps;   // 1 or 2 (the host guarantees it)
+  const int K = N > warp ? (N - warp + kDecodeWarps - 1) / kDecodeWarps : 0;
+  It itc;
+  it_seek(itc, s_pre, a.B, g.h_kv, c0);
+  RowInfo ric = rinfo(itc.i);
+  int nc = 0;
+  It iti = itc;
+  RowInfo rii = ric;
+  int ni = 0;
+  for (int t = 0; t < warp && t < N; ++t) step(iti, rii, ni);
+  int issued = 0;
+  if (K > 0) {
+    const int32_t b0 = load_blk(iti, rii);
+    issue(iti, rii, b0, SPW * warp);
+    ++issued;
   }
-  if (!aborted && cur_pair >= 0) emit(cur_pair / g.h_kv, cur_pair % g.h_kv);
+  if (SPW == 2 && K > 1) {
+    for (int t = 0; t < kDecodeWarps; ++t) step(iti, rii, ni);
+    const int32_t b1 = load_blk(iti, rii);
+    issue(iti, rii, b1, SPW * warp + 1);
+    ++issued;
+  }
+  int32_t blk_next = 0;
+  if (K > SPW) {
+    for (int t = 0; t < kDecodeWarps; ++t) step(iti, rii, ni);
+    blk_next = load_blk(iti, rii);
+  }
+
+  int cur_pair = itc.i * g.h_kv + itc.h;
+  bool needs_setup = true;
+  bool aborted = false;
+  // leaves the walk iterator on unit `target`, recording every pair it passes
+  auto walk_to = [&](int target) {
+    while (nc < target) {
+      step(itc, ric, nc);
+      const int pid = itc.i * g.h_kv + itc.h;
+      if (pid != cur_pair) {
+        emit(cur_pair / g.h_kv, cur_pair % g.h_kv);
+        state_reset(st);
+        cur_pair = pid;
+        needs_setup = true;
+      }
+    }
+  };
+  int consumed = 0;
+  for (int k = 0; k < K; ++k) {
+    walk_to(warp + kDecodeWarps * k);
+    if (needs_setup) {
+      setup_pair(itc.i, itc.h);
+      needs_setup = false;
+    }
+    const int use = SPW == 2 ? (k >> 1) : k;   // earlier uses of this unit's stage
+    const int sidx = SPW * warp + (SPW == 2 ? (k & 1) : 0);
+    // every lane polls; the warp gives up together
+    const bool arrived = wait_or_abort(full0 + 8 * sidx, uint32_t(use & 1), abort_flag);
+    if (!__all_sync(0xffffffffu, arrived)) {
+      if (lane == 0) {
+        atomicOr(a.err, KVQ_DEVERR_TIMEOUT);
+        *abort_flag = 1;
+      }
+      aborted = true;
+      break;
+    }
+    ++consumed;
+    const uint8_t* stg = stages + size_t(sidx) * pp.stage_bytes;
+    if (itc.k < ric.nq) {
+      const int T0 = itc.k * pp.sup;
+      const int valid_unit = min(pp.sup, ric.qa - T0);
+      const int nsub = (valid_unit + 15) >> 4;
+      int loaded = -1;
+      for (int c = 0; c < nsub; c += ch) {
+        if (KAXIS && ((16 * c) >> g.lg_gk) != loaded) {
+          loaded = (16 * c) >> g.lg_gk;
+          qprime_job(stg, loaded);
+        }
+        // scores of the chunk's sub-tiles go through this lane's own slots of
+        // the warp scratch, which keeps the loops rolled (small code, no spills)
+        const int nt = min(ch, nsub - c);
+#pragma unroll 1
+        for (int t = 0; t < nt; ++t) {
+          const int tok0 = 16 * (c + t);
+          float s0, s1;
+          score_sub(sub_at(stg, tok0), valid_unit - tok0, s0, s1);
+          spw[(2 * t) * 32 + lane] = s0;
+          spw[(2 * t + 1) * 32 + lane] = s1;
+        }
+        float sc[8], pc[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) sc[q] = q < 2 * nt ? spw[q * 32 + lane] : -INFINITY;
+        softmax_chunk(sc, pc);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) spw[q * 32 + lane] = pc[q];
+#pragma unroll 1
+        for (int t = 0; t < nt; ++t)
+          pv_sub(sub_at(stg, 16 * (c + t)), spw[(2 * t) * 32 + lane], spw[(2 * t + 1) * 32 + lane], true);
+      }
+    } else {
+      if (!bq_bf16) {
+        load_bq_from_q(itc.i, itc.h);
+        bq_bf16 = true;
+        bias_t = 0.0f;
+      }
+      process_window(stg, ric.ra - 16 * (itc.k - ric.nq));
+    }
+    __syncwarp();
+    if (k + SPW < K) {
+      issue(iti, rii, blk_next, sidx);   // the stage just read takes unit k + SPW
+      ++issued;
+      if (k + SPW + 1 < K) {
+        for (int t = 0; t < kDecodeWarps; ++t) step(iti, rii, ni);
+        blk_next = load_blk(iti, rii);
+      }
+    }
+  }
+  if (aborted) {
+    // keep the CTA until its copies in flight have landed (bounded)
+    for (int j = consumed; j < issued; ++j) {
+      const int sj = SPW * warp + (SPW == 2 ? (j & 1) : 0);
+      (void)mbar_wait_bounded(full0 + 8 * sj, uint32_t((SPW == 2 ? (j >> 1) : j) & 1), kWaitNs);
+    }
+    return;
+  }
+  walk_to(N - 1);
+  emit(cur_pair / g.h_kv, cur_pair % g.h_kv);
 }
 
 // Merge: one CTA per (row, kv head, query head).  The records of a pair are
@@ -1206,6 +1244,8 @@ cudaError_t plan_decode(const Geo& g, int max_B, DecodePipe* out) {
   int reserved = 0;
   e = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
   if (e != cudaSuccess) return e;
+  // two stages per warp when three CTAs still fit per SM, else one; the kernel
+  // indexes stages as (nstages / 4) * warp + ..., so nstages must be 4 or 8
   p.nstages = 2 * kDecodeWarps;
   if (3 * (size_t(smem_layout(max_B, p).total) + size_t(reserved)) > size_t(per_sm)) p.nstages = kDecodeWarps;
   if (size_t(smem_layout(max_B, p).total) > size_t(max_optin)) return cudaErrorInvalidConfiguration;

@@ -12,8 +12,8 @@
 namespace kvq {
 
 constexpr int kD = 128;            // head dimension supported by the kernels
-constexpr int kDecodeWarps = 4;    // consumer warps per decode CTA (plus one producer warp)
-constexpr int kDecodeThreads = (kDecodeWarps + 1) * 32;
+constexpr int kDecodeWarps = 4;    // warps per decode CTA; each stages and computes its own units
+constexpr int kDecodeThreads = kDecodeWarps * 32;
 constexpr int kFlushThreads = 256;
 constexpr int kMaxPagesPerGroup = 8;
 // flush plan entry: seq, group, n_pages, blocks[kMaxPagesPerGroup]
