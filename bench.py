@@ -48,7 +48,7 @@ def decode_bytes(w, lengths):
     block-table entry per page read."""
     f = w.fmt
     es = 4 if f.scale_fp32 else 2
-    meta = es * (1 + f.asym)
+    meta = es * (1 + f.asym) if f.bits < 16 else 0      # the BF16 control stores no metadata
     per_tok_q = w.h_kv * (2 * D * f.bits // 8 + D * meta // f.g_k + D * meta // f.g_v)
     per_tok_r = w.h_kv * 2 * D * 2
     total = 0
@@ -194,9 +194,11 @@ def kernel_source_sha():
     return h.hexdigest()[:16]
 
 
-def committed_traffic(workload_name):
+def committed_traffic(workload_name, algorithmic_bytes):
     """Per-launch DRAM bytes of the attention kernel from the committed ncu
-    summary, if it was taken from the current kernel source; else None."""
+    record, scaled from the captured launch to a launch moving
+    `algorithmic_bytes` (traffic grows with the units processed), if the record
+    was taken from the current kernel source; else None."""
     p = os.path.join(ROOT, "profiles", "decode_traffic.json")
     if not os.path.exists(p):
         return None
@@ -204,7 +206,11 @@ def committed_traffic(workload_name):
         rec = json.load(f)
     if rec.get("kernel_source_sha") != kernel_source_sha():
         return None
-    return rec.get("traffic_bytes_per_launch", {}).get(workload_name)
+    t = rec.get("traffic_bytes_per_launch", {}).get(workload_name)
+    a = rec.get("algorithmic_bytes_per_launch", {}).get(workload_name)
+    if t is None or not a:
+        return None
+    return t * algorithmic_bytes / a
 
 
 # ---------------------------------------------------------------------------
@@ -352,6 +358,7 @@ def run_gpu(args, rank, ws, dist):
         "w": w, "K": K, "ws": ws, "launches": launches, "clocks": clocks,
         "kv_gbs": tot[0] / (mx[2] * 1e-3) / 1e9,
         "attn_gbs": (attn_bytes / K) / (t_attn / K * 1e-3) / 1e9,
+        "attn_bytes_per_launch": attn_bytes / K,
         "attn_us": t_attn / K * 1e3,
         "decode_us": t_dec / K * 1e3,
         "append_us": t_app / K * 1e3,
@@ -365,6 +372,61 @@ def run_gpu(args, rank, ws, dist):
         "d2h": B * w.h_q * D * 4,
     }
     return res
+
+
+def run_control(args):
+    """The pages' trade-off, saved traffic versus dequantization work, on this
+    workload: decode alone (no appends) over the quantized cache and over the
+    BF16 control cache (same paged path, bf16 rows, no dequantization), both
+    filled from the same draws; L2 flushed clean before every call."""
+    import dataclasses
+    import torch
+    from quantized_kv_cache_14_b200 import kvq
+    from quantized_kv_cache_14_b200.workloads import CacheFormat
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = workload(args.workload)
+    K = max(5, min(args.steps, 50))
+    dr = Draws(w, steps=1)
+    k, v, q = dr.step()
+    lens = [L + 1 for L in dr.lengths]
+    bf = dataclasses.replace(w, fmt=CacheFormat(16, 0, 0, 128, 128, 0, 0, w.fmt.page))
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_rd = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    out = {}
+    for tag, ww in (("quantized", w), ("bf16", bf)):
+        f = ww.fmt
+        nb = pool_blocks(lens, 2, f.page)
+        mbps = max((L + 2) // f.page + 2 for L in lens)
+        cache = kvq.KVCache(kvq.Format(f.bits, f.asym, f.k_axis, f.g_k, f.g_v, f.scale_fp32, f.residual,
+                                       f.page), ww.h_q, ww.h_kv, max_seqs=ww.batch, num_blocks=nb,
+                            max_blocks_per_seq=mbps, seed=ww.seed, device=torch.cuda.current_device())
+
+        def dbf(a):
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+        cache.append(dbf(dr.k), dbf(dr.v), dr.seq_ids)
+        cache.append(dbf(k), dbf(v), np.arange(ww.batch, dtype=np.int32))
+        qd = dbf(q)
+        sl = torch.tensor(lens, dtype=torch.int32, device=dev)
+        o = torch.empty((ww.batch, ww.h_q, D), dtype=torch.float32, device=dev)
+        evs = []
+        for it in range(K + 3):
+            flush.zero_()
+            flush_rd.sum()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            cache.decode(qd, sl, o)
+            e1.record()
+            if it >= 3:
+                evs.append((e0, e1))
+        torch.cuda.synchronize()
+        assert cache.sync_status() == 0
+        us = float(np.median([a.elapsed_time(b) for a, b in evs])) * 1e3
+        nbytes = decode_bytes(ww, lens)
+        out[tag] = {"decode_us": us, "kv_bytes": nbytes, "gbs": nbytes / (us * 1e-6) / 1e9}
+        cache.close()
+    return {"format": "BF16 control: the same paged path over bf16 rows, no dequantization",
+            "calls": K, "quantized": out["quantized"], "bf16": out["bf16"],
+            "speedup_quantized_over_bf16": out["bf16"]["decode_us"] / out["quantized"]["decode_us"]}
 
 
 # ---------------------------------------------------------------------------
@@ -434,6 +496,7 @@ def main():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=0, help="rows of the CPU oracle sample")
+    ap.add_argument("--no-control", action="store_true", help="skip the BF16 control comparison")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -467,11 +530,13 @@ def main():
     peak, peak_kind = measured_peak()
     cpu = None
     if ws == 1 and not args.no_cpu_baseline:
-        gbs, secs, _, _ = run_oracle_sample(w, 2, 0, rows, threads)
+        n_cpu = 24   # about 10 s of oracle decode on the machine's host cores
+        gbs, secs, _, _ = run_oracle_sample(w, n_cpu, 0, rows, threads)
         cpu = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
-               "sample": f"2 steps of {rows}/{w.batch} sequences (append + fp64 decode), "
+               "sample": f"{n_cpu} steps of {rows}/{w.batch} sequences (append + fp64 decode), "
                          f"{secs:.1f} s timed"}
-    traffic = committed_traffic(w.name)
+    traffic = committed_traffic(w.name, res["attn_bytes_per_launch"])
+    control = run_control(args) if (ws == 1 and not args.no_control) else None
     line = {
         "metric": "decode-attn KV GB/s", "value": res["kv_gbs"], "unit": "GB/s",
         "n_gpus": ws, "steps": res["K"], "warmup": args.warmup,
@@ -492,6 +557,7 @@ def main():
         "kv_bytes_per_step": res["kv_bytes_per_step"],
         "frac_of_8TBps": res["kv_gbs"] / 8000.0,
         "frac_of_peak": res["kv_gbs"] / peak,
+        "bf16_control": control,
     }
     print(json.dumps(line))
     if dist is not None:

@@ -65,7 +65,12 @@ typedef enum kvq_status {
 enum { KVQ_AXIS_TOKEN = 0, KVQ_AXIS_CHANNEL = 1 };
 
 /* Storage format and capacity of one layer's cache.
- *   bits        8, 4 or 2 bits per stored element.
+ *   bits        8, 4 or 2 bits per stored element, or 16 for the BF16 control:
+ *               the same paged cache holding bf16 rows with no quantization (the
+ *               pages' BF16 baseline, "From BF16 to INT8, INT4, or even fewer
+ *               bits"); it needs k_axis 0, residual 0, asym 0, scale_fp32 0 and
+ *               g_k = g_v = 128, and stores each 16-token sub-tile of keys and of
+ *               values as 16 natural bf16 rows.
  *   asym        0: symmetric codes in [-Q, Q], Q = 2^(bits-1) - 1;
  *               1: unsigned codes in [0, 2^bits - 1] with a zero-point.
  *   k_axis      KVQ_AXIS_TOKEN: key groups are g_k consecutive channels of

@@ -187,7 +187,14 @@ Layout make_layout(const Cfg& c) {
   L.secK = (P / 16) * L.sub_bytes;
   L.secV = L.secK;
   L.secVm = align_up(P * L.nvg * L.es * A, 16);
-  if (c.k_axis == 0) {
+  if (c.bits == 16) {
+    // The pages' unquantized BF16 cache ("From BF16 to INT8, INT4, or even
+    // fewer bits"), kept as a control: rows only, no scales.
+    L.nkg = 1;
+    L.secVm = 0;
+    L.secKm = 0;
+    L.kslice = 0;
+  } else if (c.k_axis == 0) {
     L.nkg = D / size_t(c.g_k);
     L.secKm = align_up(P * L.nkg * L.es * A, 16);
     L.kslice = 0;
@@ -219,6 +226,8 @@ struct Loc { size_t byte; int shift; };
 
 // Byte/bit of key code (token-in-page, channel) inside the K section of a chunk.
 Loc k_loc(const Cfg& c, const Layout& L, const std::vector<int>& inv, int tok, int ch) {
+  if (c.bits == 16)   // BF16 control: natural rows, channel ch at bytes 2ch, 2ch+1
+    return {size_t(tok / 16) * L.sub_bytes + size_t(tok % 16) * L.row_bytes + size_t(2 * ch), 0};
   int f = inv[ch];
   int w = f / L.n, l = f % L.n, p = word_pos(l, L.n);
   size_t byte = size_t(tok / 16) * L.sub_bytes + size_t(tok % 16) * L.row_bytes +
@@ -238,6 +247,8 @@ Loc k_loc(const Cfg& c, const Layout& L, const std::vector<int>& inv, int tok, i
 //                     a2(2i'), a3(2i'), a2(2i'+1), a3(2i'+1)]
 // and register x of a word has its low element at field x, its high at x + n/2.
 Loc v_loc(const Cfg& c, const Layout& L, int tok, int ch) {
+  if (c.bits == 16)   // BF16 control: natural rows, like the keys
+    return {size_t(tok / 16) * L.sub_bytes + size_t(tok % 16) * L.row_bytes + size_t(2 * ch), 0};
   int sub = tok / 16, tau = tok % 16;
   int i = ch / 16, rr = ch % 16, g = rr % 8, upper = rr / 8;
   int tt = tau % 8, t = tt / 2, hi = tt % 2, second = tau / 8;
@@ -254,12 +265,18 @@ Loc v_loc(const Cfg& c, const Layout& L, int tok, int ch) {
 }
 
 void put_code(uint8_t* base, Loc loc, int bits, int32_t code) {
+  if (bits == 16) {   // a whole little-endian 16-bit field
+    base[loc.byte] = uint8_t(uint32_t(code) & 0xFFu);
+    base[loc.byte + 1] = uint8_t((uint32_t(code) >> 8) & 0xFFu);
+    return;
+  }
   uint8_t mask = uint8_t((1u << bits) - 1u);
   uint8_t v = uint8_t(uint32_t(code) & mask);
   base[loc.byte] = uint8_t((base[loc.byte] & ~(mask << loc.shift)) | (v << loc.shift));
 }
 
 int32_t get_code(const uint8_t* base, Loc loc, int bits, bool is_signed) {
+  if (bits == 16) return int32_t(uint32_t(base[loc.byte]) | (uint32_t(base[loc.byte + 1]) << 8));
   uint32_t mask = (1u << bits) - 1u;
   uint32_t v = (uint32_t(base[loc.byte]) >> loc.shift) & mask;
   if (is_signed && (v & (1u << (bits - 1)))) return int32_t(v) - (1 << bits);
@@ -319,6 +336,11 @@ void write_value_row(Cache& C, int32_t block, int tok_in_page, int h, const floa
   const Cfg& c = C.c;
   const Layout& L = C.L;
   uint8_t* ch = chunk_ptr(C, block, h);
+  if (c.bits == 16) {   // BF16 control: the row itself (x holds bf16 values exactly)
+    for (int e = 0; e < c.d_h; ++e)
+      put_code(ch + L.off_V, v_loc(c, L, tok_in_page, e), 16, int32_t(f32_bits(x[e]) >> 16));
+    return;
+  }
   int32_t codes[128];
   for (size_t gi = 0; gi < L.nvg; ++gi) {
     float s = 0, z = 0;
@@ -338,6 +360,11 @@ void write_key_row_token_axis(Cache& C, int32_t block, int tok_in_page, int h, c
   const Cfg& c = C.c;
   const Layout& L = C.L;
   uint8_t* ch = chunk_ptr(C, block, h);
+  if (c.bits == 16) {   // BF16 control: the row itself
+    for (int e = 0; e < c.d_h; ++e)
+      put_code(ch, k_loc(c, L, C.inv, tok_in_page, e), 16, int32_t(f32_bits(x[e]) >> 16));
+    return;
+  }
   int32_t codes[128];
   for (size_t gi = 0; gi < L.nkg; ++gi) {
     float s = 0, z = 0;
@@ -411,6 +438,13 @@ void dequant_token(const Cache& C, int s, int h, int64_t pos, double* kout, doub
   int32_t blk = C.table[s][size_t(pos / P)];
   int tok = int(pos % P);
   const uint8_t* ch = &C.pool[size_t(blk) * L.block_bytes + size_t(h) * L.chunk_bytes];
+  if (c.bits == 16) {   // BF16 control: the stored rows are the values
+    for (int e = 0; e < D; ++e) {
+      kout[e] = bf16_to_f32(uint16_t(get_code(ch, k_loc(c, L, C.inv, tok, e), 16, false)));
+      vout[e] = bf16_to_f32(uint16_t(get_code(ch + L.off_V, v_loc(c, L, tok, e), 16, false)));
+    }
+    return;
+  }
   bool sgn = !c.asym;
   for (int e = 0; e < D; ++e) {
     int32_t q = get_code(ch + L.off_V, v_loc(c, L, tok, e), c.bits, sgn);

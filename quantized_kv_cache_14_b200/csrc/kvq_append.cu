@@ -332,6 +332,26 @@ __global__ void residual_kernel(const Geo g, const DevState d, const PlanView p,
   }
 }
 
+// BF16 control: the token's key and value rows of each head go unchanged into
+// their page as natural bf16 rows (row r of sub-tile r / 16).  One warp per
+// (token, head); lane l copies channels 4l .. 4l+3.
+__global__ void __launch_bounds__(256) copy_token_kernel(const Geo g, const DevState d, const PlanView p,
+                                                         const uint16_t* kin, const uint16_t* vin) {
+  constexpr int D = kD;
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int64_t item = int64_t(blockIdx.x) * 8 + wib;
+  if (item >= int64_t(p.n_tok) * g.h_kv) return;
+  const int e = int(item / g.h_kv), h = int(item % g.h_kv);
+  const int32_t src = p.plan[p.off_tok + 3 * e];
+  const int32_t blk = p.plan[p.off_tok + 3 * e + 1];
+  const int32_t tok = p.plan[p.off_tok + 3 * e + 2];
+  uint8_t* chunk = d.pool + int64_t(blk) * g.block_bytes + int64_t(h) * g.chunk_bytes;
+  const int64_t row = int64_t(tok >> 4) * g.sub_bytes + (tok & 15) * (D * 2);
+  const int64_t in = (int64_t(src) * g.h_kv + h) * D + 4 * lane;
+  *reinterpret_cast<uint2*>(chunk + row + 8 * lane) = *reinterpret_cast<const uint2*>(kin + in);
+  *reinterpret_cast<uint2*>(chunk + g.off_V + row + 8 * lane) = *reinterpret_cast<const uint2*>(vin + in);
+}
+
 template <typename F>
 cudaError_t by_format(const Geo& g, F&& f) {
   if (g.bits == 8) return g.asym ? f(std::integral_constant<int, 8>(), std::integral_constant<int, 1>())
@@ -364,6 +384,11 @@ cudaError_t launch_quant_token(const Geo& g, const DevState& d, const PlanView& 
   if (p.n_tok == 0) return cudaSuccess;
   const int64_t items = int64_t(p.n_tok) * g.h_kv;
   const int blocks = int((items + 7) / 8);
+  if (g.bits == 16) {
+    copy_token_kernel<<<blocks, 256, 0, s>>>(g, d, p, k, v);
+    ++*launches;
+    return cudaGetLastError();
+  }
   return by_format(g, [&](auto B, auto A) {
     quant_token_kernel<decltype(B)::value, decltype(A)::value><<<blocks, 256, 0, s>>>(g, d, p, k, v);
     ++*launches;

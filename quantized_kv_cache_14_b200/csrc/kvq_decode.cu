@@ -356,6 +356,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
   // with the running max exact (p <= 1), p' = p * s fits fp16's range.  Fp32
   // scales keep bf16 operands (fp32 range).
   constexpr bool PVH = ES == 2;
+  // The BF16 control (16-bit "codes"): 16-token tiles of natural bf16 rows,
+  // computed like the BF16 window.
+  constexpr bool BF = BITS == 16;
   extern __shared__ __align__(128) uint8_t smem[];
   const Geo gs = geo_of<SPEC>(a.g);
   const Geo& g = SPEC ? gs : a.g;   // the generic instances read the geometry from the parameters
@@ -428,7 +431,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
     const int T0 = it.k * pp.sup;
     const int valid = min(pp.sup, ri.qa - T0);
     int pg, ncopy;
-    if (KAXIS) {
+    if (BF) {
+      ncopy = 2;                     // key tile and value tile of one page
+      pg = T0 >> g.lg_P;
+    } else if (KAXIS) {
       ncopy = ((valid + g.g_k - 1) >> g.lg_gk) << (g.lg_gk - g.lg_P);   // whole key groups
       pg = (T0 >> g.lg_P) + lane;
     } else {
@@ -448,7 +454,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
     if (!window) {
       const int T0 = it.k * pp.sup;
       const int valid = min(pp.sup, ri.qa - T0);
-      if (KAXIS) {
+      if (BF) {
+        ncopy = 2;
+        total = 2 * 16 * kD * 2;
+        tok = T0;
+      } else if (KAXIS) {
         ncopy = ((valid + g.g_k - 1) >> g.lg_gk) << (g.lg_gk - g.lg_P);
         total = uint32_t(ncopy * g.chunk_used);
       } else {
@@ -481,7 +491,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
       return;
     }
     const uint8_t* chunk = a.pool + int64_t(blk) * g.block_bytes + int64_t(it.h) * g.chunk_bytes;
-    if (KAXIS) {
+    if (BF) {
+      const int u = (tok & (g.P - 1)) >> 4;
+      bulk_g2s(dst + lane * (16 * kD * 2), chunk + (lane ? g.off_V : 0) + int64_t(u) * g.sub_bytes, 16 * kD * 2, bar);
+    } else if (KAXIS) {
       bulk_g2s(dst + lane * g.chunk_used, chunk, uint32_t(g.chunk_used), bar);
     } else if (g.P == 16) {
       bulk_g2s(dst + lane * pp.qsub, chunk, uint32_t(g.chunk_used), bar);
@@ -636,6 +649,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
           }
         cs = C * pow2f(ex);
       }
+    } else if (BF) {
+      load_bq_from_q(row, h);
+      bq_bf16 = true;
     } else {
       const float down = load_bq_f16(row, h);
       if (ASYM) {
@@ -1037,7 +1053,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
     }
     ++consumed;
     const uint8_t* stg = stages + size_t(sidx) * pp.stage_bytes;
-    if (itc.k < ric.nq) {
+    if (BF && itc.k < ric.nq) {
+      process_window(stg, min(16, ric.qa - itc.k * 16));
+    } else if (itc.k < ric.nq) {
       const int T0 = itc.k * pp.sup;
       const int valid_unit = min(pp.sup, ric.qa - T0);
       const int nsub = (valid_unit + 15) >> 4;
@@ -1200,6 +1218,7 @@ const void* kernel_of() {
 
 const void* decode_kernel_ptr(const Geo& g) {
   if (spec_int4_kivi(g)) return kernel_of<4, 0, 1, 2, 1>();
+  if (g.bits == 16) return kernel_of<16, 0, 0, 2>();
   const int key = ((g.bits == 8 ? 0 : g.bits == 4 ? 1 : 2) * 4 + g.asym * 2 + g.k_axis) * 2 + (g.es == 4);
   switch (key) {
 #define KVQ_CASE(k, b, as, ax) \
@@ -1224,10 +1243,12 @@ size_t decode_partials_bytes(const Geo& g, int B, int grid) {
 
 cudaError_t plan_decode(const Geo& g, int max_B, DecodePipe* out) {
   DecodePipe p{};
-  p.sup = g.k_axis ? (g.g_k > 64 ? g.g_k : 64) : 64;
-  p.lg_sup = p.sup == 128 ? 7 : 6;
+  p.sup = g.bits == 16 ? 16 : g.k_axis ? (g.g_k > 64 ? g.g_k : 64) : 64;
+  p.lg_sup = p.sup == 128 ? 7 : p.sup == 64 ? 6 : 4;
   p.qsub = g.k_axis ? 0 : 2 * g.sub_bytes + g.vm16 + g.km16;
-  const int qunit = g.k_axis ? (p.sup / g.P) * g.chunk_used : kDecodeWarps * p.qsub;
+  const int qunit = g.bits == 16 ? 2 * 16 * kD * 2
+                    : g.k_axis   ? (p.sup / g.P) * g.chunk_used
+                                 : kDecodeWarps * p.qsub;
   const int res = g.R ? 2 * 16 * kD * 2 : 0;
   p.stage_bytes = (((qunit > res ? qunit : res) + 127) / 128) * 128;
   int dev = 0, max_optin = 0;

@@ -50,7 +50,12 @@ bool is_group_size(int g) { return g == 16 || g == 32 || g == 64 || g == 128; }
 
 kvq_status validate(const kvq_config* c) {
   if (!c) return fail(KVQ_ERR_INVALID_ARG, "config is null");
-  if (c->bits != 2 && c->bits != 4 && c->bits != 8) return fail(KVQ_ERR_INVALID_ARG, "bits must be 2, 4 or 8");
+  if (c->bits != 2 && c->bits != 4 && c->bits != 8 && c->bits != 16)
+    return fail(KVQ_ERR_INVALID_ARG, "bits must be 2, 4, 8 or 16");
+  if (c->bits == 16 && (c->k_axis != KVQ_AXIS_TOKEN || c->residual != 0 || c->asym != 0 || c->scale_fp32 != 0 ||
+                        c->g_k != 128 || c->g_v != 128))
+    return fail(KVQ_ERR_INVALID_ARG,
+                "the BF16 control (bits 16) needs k_axis 0, residual 0, asym 0, scale_fp32 0, g_k = g_v = 128");
   if (c->asym != 0 && c->asym != 1) return fail(KVQ_ERR_INVALID_ARG, "asym must be 0 or 1");
   if (c->scale_fp32 != 0 && c->scale_fp32 != 1) return fail(KVQ_ERR_INVALID_ARG, "scale_fp32 must be 0 or 1");
   if (c->d_h != kvq::kD) return fail(KVQ_ERR_UNSUPPORTED, "d_h must be 128");
@@ -94,7 +99,12 @@ kvq::Geo make_geo(const kvq_config& c) {
   g.secK = (c.page / 16) * g.sub_bytes;
   g.secV = g.secK;
   g.secVm = int(align_up(size_t(c.page) * g.nvg * g.es * A, 16));
-  if (c.k_axis == KVQ_AXIS_TOKEN) {
+  if (c.bits == 16) {   // BF16 control: rows only, no metadata
+    g.nkg = 1;
+    g.kslice = 0;
+    g.secVm = 0;
+    g.secKm = 0;
+  } else if (c.k_axis == KVQ_AXIS_TOKEN) {
     g.nkg = D / c.g_k;
     g.kslice = 0;
     g.secKm = int(align_up(size_t(c.page) * g.nkg * g.es * A, 16));
@@ -341,10 +351,11 @@ kvq_status kvq_layout(const kvq_config* cfg, kvq_layout_info* out) {
 
 uint64_t kvq_cache_bytes(int32_t layers, int64_t tokens, int32_t h_kv, int32_t d_h, const kvq_config* cfg) {
   if (!cfg || layers < 0 || tokens < 0 || h_kv < 0 || d_h < 0) return 0;
-  if (cfg->bits != 2 && cfg->bits != 4 && cfg->bits != 8) return 0;
+  if (cfg->bits != 2 && cfg->bits != 4 && cfg->bits != 8 && cfg->bits != 16) return 0;
   if (cfg->g_k <= 0 || cfg->g_v <= 0) return 0;
   // M = 2 L T H_kv d_h b: codes for K and V, plus per-group metadata
   const uint64_t elems = uint64_t(layers) * uint64_t(tokens) * uint64_t(h_kv) * uint64_t(d_h);
+  if (cfg->bits == 16) return 2 * elems * 2;   // the BF16 control: b = 2, no metadata
   const uint64_t meta = uint64_t(cfg->scale_fp32 ? 4 : 2) * uint64_t(1 + cfg->asym);
   const uint64_t codes = 2 * elems * uint64_t(cfg->bits) / 8;
   const uint64_t kmeta = (elems * meta + uint64_t(cfg->g_k) - 1) / uint64_t(cfg->g_k);

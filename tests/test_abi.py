@@ -45,6 +45,7 @@ FMTS = {
     "int2_asym_chan32": dict(bits=2, asym=1, k_axis=1, g_k=32, g_v=32, scale_fp32=0, residual=32, page=16),
     "int4_chan64_p32": dict(bits=4, asym=0, k_axis=1, g_k=64, g_v=32, scale_fp32=0, residual=64, page=32),
     "int4_asym_tok32": dict(bits=4, asym=1, k_axis=0, g_k=32, g_v=32, scale_fp32=0, residual=0, page=32),
+    "bf16_control_p16": dict(bits=16, asym=0, k_axis=0, g_k=128, g_v=128, scale_fp32=0, residual=0, page=16),
 }
 
 
@@ -142,6 +143,7 @@ def test_fail_alloc_after_and_table_width():
     ("g_v", 48, kvq.KVQ_ERR_UNSUPPORTED),
     ("num_blocks", 0, kvq.KVQ_ERR_INVALID_ARG),
     ("k_axis", 2, kvq.KVQ_ERR_INVALID_ARG),
+    ("bits", 16, kvq.KVQ_ERR_INVALID_ARG),     # the BF16 control takes token-axis keys, no window
 ])
 def test_config_validation(field, value, status):
     cfg, _ = cfg_of("int4_chan64")
@@ -175,3 +177,17 @@ def test_cache_bytes_formula_worked_example():
     assert kvq.kvq_cache_bytes(32, 8192, 8, 128, cfg8) == 2 * elems + 2 * elems * 2 // 128
     cfg2, _ = cfg_of("int2_asym_chan32")
     assert kvq.kvq_cache_bytes(1, 100, 8, 128, cfg2) == 2 * 102400 // 4 + 2 * 102400 * 4 // 32
+    cfg16, _ = cfg_of("bf16_control_p16")      # BF16: 2 bytes per element, no metadata
+    assert kvq.kvq_cache_bytes(32, 8192, 8, 128, cfg16) == 2 * elems * 2
+
+
+def test_bf16_control_config_rules():
+    for field, value in (("residual", 64), ("asym", 1), ("scale_fp32", 1), ("g_k", 64), ("g_v", 64)):
+        cfg, _ = cfg_of("bf16_control_p16")
+        setattr(cfg, field, value)
+        if field == "residual":
+            cfg.k_axis = 1
+            cfg.g_k = 64
+        with pytest.raises(kvq.KvqError) as e:
+            kvq.kvq_create(cfg)
+        assert e.value.status == kvq.KVQ_ERR_INVALID_ARG

@@ -35,6 +35,9 @@ FMTS = {
     "int8_asym_chan128_p64": dict(bits=8, asym=1, k_axis=1, g_k=128, g_v=128, scale_fp32=0, residual=128, page=64),
     "int2_sym_tok64_fp32": dict(bits=2, asym=0, k_axis=0, g_k=64, g_v=64, scale_fp32=1, residual=0, page=16),
     "int4_chan16": dict(bits=4, asym=0, k_axis=1, g_k=16, g_v=128, scale_fp32=0, residual=16, page=16),
+    # the pages' unquantized BF16 cache on the same paged path (control)
+    "bf16_control_p16": dict(bits=16, asym=0, k_axis=0, g_k=128, g_v=128, scale_fp32=0, residual=0, page=16),
+    "bf16_control_p64": dict(bits=16, asym=0, k_axis=0, g_k=128, g_v=128, scale_fp32=0, residual=0, page=64),
 }
 
 
@@ -83,7 +86,7 @@ def test_incremental_appends_interleaved(name):
     p.close()
 
 
-@pytest.mark.parametrize("name", ["int4_chan64", "int8_tok_p16", "int2_asym_chan32"])
+@pytest.mark.parametrize("name", ["int4_chan64", "int8_tok_p16", "int2_asym_chan32", "bf16_control_p16"])
 def test_split_k_merge_is_invariant_to_grid(name):
     rng = np.random.default_rng(3)
     h_q, h_kv = 16, 4

@@ -356,3 +356,69 @@ def test_decode_dominant_score_picks_its_row():
     _, V = c.dequant(0, 0, T)
     assert np.allclose(out[0, 0], V[17], atol=1e-9)
     c.close()
+
+
+# ------------------------------------------------------------ BF16 control
+
+def _bf16_control(**kw):
+    cfg = dict(bits=16, asym=0, k_axis=0, g_k=128, g_v=128, scale_fp32=0, residual=0, page=16,
+               h_q=4, h_kv=2, d_h=D, max_seqs=3, num_blocks=64, max_blocks_per_seq=64, seed=5,
+               fail_alloc_after=-1)
+    cfg.update(kw)
+    return O.OracleCache(**cfg)
+
+
+@pytest.mark.parametrize("page", [16, 64])
+def test_bf16_control_stores_rows_unchanged(page):
+    """The control format is the pages' unquantized BF16 cache: the stored
+    bytes are the appended bf16 rows (natural order, 256 B per row, 16-row
+    sub-tiles), dequantization returns them exactly, and there is no metadata."""
+    rng = np.random.default_rng(2)
+    c = _bf16_control(page=page)
+    lay = c.layout
+    assert lay["row_bytes"] == 2 * D and lay["sub_bytes"] == 16 * 2 * D
+    assert lay["off_V"] == lay["secK"] == (page // 16) * 16 * 2 * D
+    assert lay["off_Vm"] == lay["off_Km"] == 2 * lay["secK"]          # no scales
+    T = 3 * page + 5
+    k = random_bf16(rng, (T, 2, D), 4.0)
+    v = random_bf16(rng, (T, 2, D))
+    assert c.append(k, v, np.zeros(T, np.int32)) == 0
+    pool = c.pool()
+    table = c.block_table(0)
+    for tok in (0, 1, 15, 16, page - 1, page, T - 1):
+        for ch in (0, 1, 77, D - 1):
+            b, sh = c.code_loc("k", tok % page, ch)
+            assert sh == 0 and b == (tok % page // 16) * 16 * 2 * D + (tok % 16) * 2 * D + 2 * ch
+            for h in range(2):
+                base = int(table[tok // page]) * lay["block_bytes"] + h * lay["chunk_bytes"]
+                kb = int(pool[base + b]) | (int(pool[base + b + 1]) << 8)
+                vb = int(pool[base + lay["off_V"] + b]) | (int(pool[base + lay["off_V"] + b + 1]) << 8)
+                assert kb == int(k[tok, h, ch]) and vb == int(v[tok, h, ch])
+    for h in range(2):
+        K, V = c.dequant(0, h, T)
+        assert np.array_equal(K, O.bf16_bits_to_f32(k[:, h, :]).astype(np.float64))
+        assert np.array_equal(V, O.bf16_bits_to_f32(v[:, h, :]).astype(np.float64))
+    # 2 bytes per element for K and for V, nothing else
+    assert O.cache_bytes_formula(32, 8192, 8, 128, 16, 128, 128, 0) == 2 * 32 * 8192 * 8 * 128 * 2
+    c.close()
+
+
+def test_bf16_control_decode_matches_torch_sdpa():
+    rng = np.random.default_rng(9)
+    c = _bf16_control()
+    lens = [1, 40, 97]
+    ids = np.repeat(np.arange(3, dtype=np.int32), lens)
+    k = random_bf16(rng, (ids.size, 2, D), 3.0)
+    v = random_bf16(rng, (ids.size, 2, D))
+    assert c.append(k, v, ids) == 0
+    q = random_bf16(rng, (3, 4, D))
+    got = c.decode(q, lens)
+    for i, L in enumerate(lens):
+        sel = ids == i
+        K = torch.from_numpy(O.bf16_bits_to_f32(k[sel]).astype(np.float64)).permute(1, 0, 2)
+        V = torch.from_numpy(O.bf16_bits_to_f32(v[sel]).astype(np.float64)).permute(1, 0, 2)
+        Q = torch.from_numpy(O.bf16_bits_to_f32(q[i]).astype(np.float64)).reshape(4, 1, D)
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            Q, K.repeat_interleave(2, dim=0), V.repeat_interleave(2, dim=0))
+        assert np.allclose(got[i], ref.reshape(4, D).numpy(), rtol=0, atol=1e-12)
+    c.close()
