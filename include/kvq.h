@@ -208,9 +208,26 @@ kvq_status kvq_seq_len(kvq_handle h, int32_t seq, int32_t* len);
  * appends in stream order (usable as seq_lens when rows are sequences). */
 kvq_status kvq_seq_lens_device(kvq_handle h, const int32_t** dev_ptr);
 
-/* Returns a sequence's blocks to the back of the free list, in logical order,
- * and resets its length to 0.  `stream` orders the device-side reset. */
+/* Releases a sequence's blocks in logical order and resets its length to 0.
+ * A block goes to the back of the free list when the last block-table row
+ * holding it lets go (blocks can be shared, see kvq_share_prefix).  `stream`
+ * orders the device-side reset. */
 kvq_status kvq_free_seq(kvq_handle h, int32_t seq, void* stream);
+
+/* Prefix sharing of quantized blocks (the paging section of the day-65 page,
+ * "How this connects to paging and prefix caching": blocks are what prefix
+ * caching shares).  Makes the empty sequence dst_seq start with the first
+ * `tokens` tokens of src_seq by pointing dst's block-table row at src's
+ * physical blocks (no copy; each shared block's holder count goes up).
+ * Format check: `tokens` must be a multiple of the page for per-token formats
+ * and of g_k (a whole key group, whole pages) for per-channel formats, so
+ * only full blocks that no later append writes are shared; dst's window
+ * starts empty.  Later appends to either sequence take fresh blocks.
+ * Errors (no state change): KVQ_ERR_BAD_SEQ for ids out of range;
+ * KVQ_ERR_INVALID_ARG for dst not empty, dst == src, tokens outside
+ * [0, len(src)] or not aligned; KVQ_ERR_OOM if dst's row is too short.
+ * `stream` orders the device-side table and length update. */
+kvq_status kvq_share_prefix(kvq_handle h, int32_t src_seq, int32_t dst_seq, int32_t tokens, void* stream);
 
 /* Capacity and usage counters (day-65 page's memory formula for bytes_formula;
  * oh-bug.com checklist item on monitoring KV-cache usage). */

@@ -312,6 +312,7 @@ struct Cache {
   std::vector<std::vector<int32_t>> table;
   std::deque<int32_t> freelist;
   int64_t alloc_count = 0;
+  std::vector<int32_t> holders;    // per block: table rows holding it (shared prefixes)
 };
 
 int64_t blocks_for_len(const Cfg& c, int64_t len) {
@@ -323,6 +324,7 @@ int32_t alloc_block(Cache& C) {
   int32_t b = C.freelist.front();
   C.freelist.pop_front();
   ++C.alloc_count;
+  C.holders[size_t(b)] = 1;
   std::memset(&C.pool[size_t(b) * C.L.block_bytes], 0, C.L.block_bytes);
   return b;
 }
@@ -540,6 +542,7 @@ void* orc_create(const Cfg* cfg) {
   std::vector<int32_t> perm(size_t(C->c.num_blocks));
   orc_free_list(C->c.num_blocks, C->c.seed, perm.data());
   C->freelist.assign(perm.begin(), perm.end());
+  C->holders.assign(size_t(C->c.num_blocks), 0);
   return C;
 }
 
@@ -625,9 +628,37 @@ void orc_v_loc(void* hh, int32_t tok, int32_t ch, int64_t* byte, int32_t* shift)
 int32_t orc_free_seq(void* hh, int32_t s) {
   Cache& C = *static_cast<Cache*>(hh);
   if (s < 0 || s >= C.c.max_seqs) return 3;
-  for (int32_t b : C.table[size_t(s)]) C.freelist.push_back(b);
+  // a block is free again when its last holder lets go; freed in logical order
+  for (int32_t b : C.table[size_t(s)])
+    if (--C.holders[size_t(b)] == 0) C.freelist.push_back(b);
   C.table[size_t(s)].clear();
   C.len[size_t(s)] = 0;
+  return 0;
+}
+
+// Prefix sharing (day-65 page, "How this connects to paging and prefix
+// caching"): the empty sequence dst starts with the first `tokens` tokens of
+// src by holding src's blocks too.  Only whole blocks that no append writes
+// again are shared: tokens a multiple of the page (no window) or of the window
+// length R = g_k (whole key groups).  Returns 0; 3 for bad ids; 4 for dst not
+// empty, dst == src, tokens out of [0, len(src)] or not aligned; 2 when dst's
+// table row is too short.  No state change on error.
+int32_t orc_share_prefix(void* hh, int32_t src, int32_t dst, int32_t tokens) {
+  Cache& C = *static_cast<Cache*>(hh);
+  const Cfg& c = C.c;
+  if (src < 0 || src >= c.max_seqs || dst < 0 || dst >= c.max_seqs) return 3;
+  if (src == dst || C.len[size_t(dst)] != 0) return 4;
+  if (tokens < 0 || tokens > C.len[size_t(src)]) return 4;
+  const int32_t unit = c.residual ? c.residual : c.page;
+  if (tokens % unit != 0) return 4;
+  const int64_t nb = blocks_for_len(c, tokens);
+  if (nb > c.max_blocks_per_seq) return 2;
+  for (int64_t j = 0; j < nb; ++j) {
+    const int32_t b = C.table[size_t(src)][size_t(j)];
+    C.table[size_t(dst)].push_back(b);
+    ++C.holders[size_t(b)];
+  }
+  C.len[size_t(dst)] = tokens;
   return 0;
 }
 

@@ -62,6 +62,8 @@ def lib():
         L.orc_append.argtypes = [P, P, P, P, ctypes.c_int32]
         L.orc_free_seq.restype = ctypes.c_int32
         L.orc_free_seq.argtypes = [P, ctypes.c_int32]
+        L.orc_share_prefix.restype = ctypes.c_int32
+        L.orc_share_prefix.argtypes = [P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]
         L.orc_seq_len.restype = ctypes.c_int32
         L.orc_seq_len.argtypes = [P, ctypes.c_int32]
         L.orc_pool_bytes.restype = ctypes.c_int64
@@ -173,6 +175,9 @@ class OracleCache:
 
     def free_seq(self, s: int) -> int:
         return lib().orc_free_seq(self.h, int(s))
+
+    def share_prefix(self, src: int, dst: int, tokens: int) -> int:
+        return lib().orc_share_prefix(self.h, int(src), int(dst), int(tokens))
 
     def seq_len(self, s: int) -> int:
         return lib().orc_seq_len(self.h, int(s))

@@ -154,6 +154,7 @@ struct kvq_handle_s {
   std::vector<int32_t> len;     // stored length per sequence
   std::vector<int32_t> table;   // [max_seqs][mbps], -1 = none
   std::vector<int32_t> nblk;    // blocks per sequence
+  std::vector<int32_t> refcnt;  // per block: block-table rows that hold it (0 = free)
   std::deque<int32_t> freelist;
   int64_t alloc_count = 0;
   // device
@@ -373,6 +374,7 @@ kvq_status kvq_create(const kvq_config* cfg, kvq_handle* out) {
   h->geo = make_geo(*cfg);
   h->len.assign(size_t(cfg->max_seqs), 0);
   h->nblk.assign(size_t(cfg->max_seqs), 0);
+  h->refcnt.assign(size_t(cfg->num_blocks), 0);
   h->table.assign(size_t(cfg->max_seqs) * cfg->max_blocks_per_seq, -1);
   // free list: Fisher-Yates over [0, num_blocks) driven by splitmix64(seed)
   std::vector<int32_t> perm(size_t(cfg->num_blocks));
@@ -502,6 +504,7 @@ kvq_status kvq_append(kvq_handle h, const void* k_bf16, const void* v_bf16, cons
   // ---- commit host state -----------------------------------------------------
   h->table.swap(tbl);
   h->nblk = nblk;
+  for (int64_t j = 0; j < allocs; ++j) h->refcnt[size_t(h->freelist[size_t(j)])] = 1;
   h->freelist.erase(h->freelist.begin(), h->freelist.begin() + allocs);
   h->alloc_count += allocs;
   for (int s = 0; s < S; ++s) h->len[size_t(s)] = cur[size_t(s)];
@@ -600,11 +603,48 @@ kvq_status kvq_free_seq(kvq_handle h, int32_t seq, void* stream_) {
   }
   for (int32_t j = 0; j < h->nblk[size_t(seq)]; ++j) {
     int32_t& e = h->table[size_t(seq) * MB + j];
-    h->freelist.push_back(e);
+    if (--h->refcnt[size_t(e)] == 0) h->freelist.push_back(e);   // last holder frees it
     e = -1;
   }
   h->nblk[size_t(seq)] = 0;
   h->len[size_t(seq)] = 0;
+  return KVQ_OK;
+}
+
+kvq_status kvq_share_prefix(kvq_handle h, int32_t src_seq, int32_t dst_seq, int32_t tokens, void* stream_) {
+  if (!h) return fail(KVQ_ERR_INVALID_ARG, "handle is null");
+  const kvq_config& c = h->cfg;
+  if (src_seq < 0 || src_seq >= c.max_seqs || dst_seq < 0 || dst_seq >= c.max_seqs)
+    return fail(KVQ_ERR_BAD_SEQ, "sequence id out of range");
+  if (src_seq == dst_seq) return fail(KVQ_ERR_INVALID_ARG, "source and destination are the same sequence");
+  if (h->len[size_t(dst_seq)] != 0) return fail(KVQ_ERR_INVALID_ARG, "destination sequence is not empty");
+  if (tokens < 0 || tokens > h->len[size_t(src_seq)])
+    return fail(KVQ_ERR_INVALID_ARG, "tokens must be in [0, source length]");
+  // only whole, full blocks are shared: whole pages of a per-token format, whole
+  // key groups (which are whole pages) of a per-channel format with a window
+  const int32_t unit = c.residual ? c.residual : c.page;
+  if (tokens % unit != 0)
+    return fail(KVQ_ERR_INVALID_ARG, "tokens must be a multiple of " + std::to_string(unit) +
+                                         " (whole blocks / key groups) to be shared");
+  const int MB = c.max_blocks_per_seq;
+  const int32_t nb = int32_t(blocks_for_len(c, tokens));
+  if (nb > MB) return fail(KVQ_ERR_OOM, "block-table row is too short");
+  Plan pl;
+  for (int32_t j = 0; j < nb; ++j) pl.tab.insert(pl.tab.end(), {dst_seq * MB + j, h->table[size_t(src_seq) * MB + j]});
+  pl.lens.insert(pl.lens.end(), {dst_seq, tokens});
+  if (!c.host_only) {
+    kvq_status st = device_guard(h);
+    if (st != KVQ_OK) return st;
+    st = run_plan(h, pl, nullptr, nullptr, static_cast<cudaStream_t>(stream_));
+    if (st != KVQ_OK) return st;
+  }
+  for (int32_t j = 0; j < nb; ++j) {
+    const int32_t b = h->table[size_t(src_seq) * MB + j];
+    h->table[size_t(dst_seq) * MB + j] = b;
+    ++h->refcnt[size_t(b)];
+  }
+  h->nblk[size_t(dst_seq)] = nb;
+  h->len[size_t(dst_seq)] = tokens;
   return KVQ_OK;
 }
 

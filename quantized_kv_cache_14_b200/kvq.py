@@ -37,7 +37,7 @@ KVQ_AXIS_CHANNEL = 1
 # Every symbol of include/kvq.h (checked by tests/test_abi.py).
 EXPORTS = (
     "kvq_create", "kvq_destroy", "kvq_append", "kvq_decode_attn", "kvq_block_table",
-    "kvq_block_table_host", "kvq_seq_len", "kvq_seq_lens_device", "kvq_free_seq",
+    "kvq_block_table_host", "kvq_seq_len", "kvq_seq_lens_device", "kvq_free_seq", "kvq_share_prefix",
     "kvq_stats", "kvq_cache_bytes", "kvq_layout", "kvq_read_pool", "kvq_read_residual",
     "kvq_sync_status", "kvq_set_decode_grid", "kvq_set_decode_event", "kvq_decode_attn_noalloc",
     "kvq_last_error",
@@ -97,6 +97,7 @@ def lib():
             "kvq_seq_len": (st, [P, I32, ctypes.POINTER(I32)]),
             "kvq_seq_lens_device": (st, [P, ctypes.POINTER(P)]),
             "kvq_free_seq": (st, [P, I32, P]),
+            "kvq_share_prefix": (st, [P, I32, I32, I32, P]),
             "kvq_stats": (st, [P, ctypes.POINTER(KvqStats)]),
             "kvq_cache_bytes": (U64, [I32, ctypes.c_int64, I32, I32, ctypes.POINTER(KvqConfig)]),
             "kvq_layout": (st, [ctypes.POINTER(KvqConfig), ctypes.POINTER(KvqLayoutInfo)]),
@@ -192,6 +193,10 @@ def kvq_seq_lens_device(h) -> int:
 
 def kvq_free_seq(h, seq: int, stream: int = 0):
     _check(lib().kvq_free_seq(h, int(seq), ctypes.c_void_p(stream)))
+
+
+def kvq_share_prefix(h, src_seq: int, dst_seq: int, tokens: int, stream: int = 0):
+    _check(lib().kvq_share_prefix(h, int(src_seq), int(dst_seq), int(tokens), ctypes.c_void_p(stream)))
 
 
 def kvq_stats(h) -> dict:
@@ -328,6 +333,9 @@ class KVCache:
 
     def free_seq(self, s, stream=None):
         kvq_free_seq(self.h, s, 0 if self.cfg.host_only else self._stream(stream))
+
+    def share_prefix(self, src, dst, tokens, stream=None):
+        kvq_share_prefix(self.h, src, dst, tokens, 0 if self.cfg.host_only else self._stream(stream))
 
     def pool(self, stream=None):
         return kvq_read_pool(self.h, self.cfg.num_blocks * self.layout["block_bytes"], self._stream(stream))

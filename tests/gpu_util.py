@@ -52,6 +52,10 @@ class Pair:
         self.gpu.append(bits_to_cuda_bf16(k_bits), bits_to_cuda_bf16(v_bits), ids)
         assert self.orc.append(k_bits, v_bits, ids) == 0
 
+    def share_prefix(self, src, dst, tokens):
+        self.gpu.share_prefix(src, dst, tokens)
+        assert self.orc.share_prefix(src, dst, tokens) == 0
+
     def check_state(self, pool=True):
         torch.cuda.synchronize()
         assert self.gpu.sync_status() == 0

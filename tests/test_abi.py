@@ -191,3 +191,44 @@ def test_bf16_control_config_rules():
         with pytest.raises(kvq.KvqError) as e:
             kvq.kvq_create(cfg)
         assert e.value.status == kvq.KVQ_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("name", ["int8_tok_p16", "int4_chan64", "int4_asym_tok32"])
+def test_share_prefix_planner_matches_oracle(name):
+    cfg, d = cfg_of(name, max_seqs=4, num_blocks=300)
+    h = kvq.kvq_create(cfg)
+    oc = O.OracleCache(**{k: v for k, v in d.items() if k not in ("host_only", "device")})
+    unit = d["residual"] or d["page"]
+    z = np.zeros((1, 2, 128), np.uint16)
+
+    def both_append(n, s):
+        ids = np.full(n, s, np.int32)
+        kb = np.zeros((n, 2, 128), np.uint16)
+        assert oc.append(kb, kb, ids) == 0
+        kvq.kvq_append(h, 0, 0, ids, n)
+
+    both_append(5 * unit + 7, 0)
+    kvq.kvq_share_prefix(h, 0, 1, 3 * unit)
+    assert oc.share_prefix(0, 1, 3 * unit) == 0
+    both_append(2 * unit + 1, 1)
+    both_append(unit, 0)
+    kvq.kvq_share_prefix(h, 1, 2, 2 * unit)
+    assert oc.share_prefix(1, 2, 2 * unit) == 0
+    for s in (0, 1, 2):
+        assert kvq.kvq_seq_len(h, s) == oc.seq_len(s)
+        assert kvq.kvq_block_table_host(h, s).tolist() == oc.block_table(s).tolist()
+    for s in (0, 2, 1):
+        kvq.kvq_free_seq(h, s)
+        assert oc.free_seq(s) == 0
+        assert kvq.kvq_stats(h)["blocks_free"] == oc.free_count()
+    both_append(4 * unit, 3)     # blocks come back in the same order on both sides
+    assert kvq.kvq_block_table_host(h, 3).tolist() == oc.block_table(3).tolist()
+    # format check and other errors, with no state change
+    for args, status in (((3, 0, unit + 1), kvq.KVQ_ERR_INVALID_ARG), ((3, 3, unit), kvq.KVQ_ERR_INVALID_ARG),
+                         ((3, 0, 99 * unit), kvq.KVQ_ERR_INVALID_ARG), ((3, 9, unit), kvq.KVQ_ERR_BAD_SEQ)):
+        with pytest.raises(kvq.KvqError) as e:
+            kvq.kvq_share_prefix(h, *args)
+        assert e.value.status == status
+    assert kvq.kvq_seq_len(h, 0) == 0
+    kvq.kvq_destroy(h)
+    oc.close()

@@ -107,6 +107,33 @@ def test_split_k_merge_is_invariant_to_grid(name):
     p.close()
 
 
+@pytest.mark.parametrize("name", ["int4_chan64", "int8_tok_p16", "int2_asym_chan32", "bf16_control_p16"])
+def test_shared_prefix_decode(name):
+    """Prefix sharing: a sequence holding another's quantized blocks decodes as
+    the oracle says, before and after both sequences grow past the share."""
+    rng = np.random.default_rng(8)
+    fmt = FMTS[name]
+    unit = fmt["residual"] or fmt["page"]
+    h_q, h_kv = 8, 2
+    p = Pair(fmt, h_q, h_kv, max_seqs=3, num_blocks=400, mbps=64, seed=6)
+    n0 = 6 * unit + 9
+    p.append(outlier_keys(rng, n0, h_kv), random_bf16(rng, (n0, h_kv, D)), np.zeros(n0, np.int32))
+    p.share_prefix(0, 1, 4 * unit)
+    p.share_prefix(0, 2, 2 * unit)
+    p.check_state()
+    p.check_decode(random_bf16(rng, (3, h_q, D)), [n0, 4 * unit, 2 * unit])
+    for s, n in ((1, 3 * unit + 2), (0, unit + 4), (2, 5)):
+        p.append(outlier_keys(rng, n, h_kv), random_bf16(rng, (n, h_kv, D)), np.full(n, s, np.int32))
+    p.check_state()
+    lens = [p.orc.seq_len(s) for s in range(3)]
+    p.check_decode(random_bf16(rng, (3, h_q, D)), lens)
+    p.gpu.free_seq(0)
+    assert p.orc.free_seq(0) == 0
+    p.check_state()
+    p.check_decode(random_bf16(rng, (3, h_q, D)), [0] + lens[1:])
+    p.close()
+
+
 def test_prefix_lengths_empty_rows_and_seq_map():
     rng = np.random.default_rng(4)
     fmt = FMTS["int4_chan64"]

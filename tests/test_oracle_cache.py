@@ -422,3 +422,69 @@ def test_bf16_control_decode_matches_torch_sdpa():
             Q, K.repeat_interleave(2, dim=0), V.repeat_interleave(2, dim=0))
         assert np.allclose(got[i], ref.reshape(4, D).numpy(), rtol=0, atol=1e-12)
     c.close()
+
+
+# ------------------------------------------------------------ prefix sharing
+
+@pytest.mark.parametrize("name", ["int8_tok_p16", "int4_chan64_p16", "int2_asym_chan32_p16", "int4_asym_tok32"])
+def test_shared_prefix_equals_an_unshared_copy(name):
+    """A sequence that starts from another's shared prefix holds exactly what a
+    sequence built by appending the same rows would hold (quantization works
+    per group, and only whole groups/pages are shared); appends after the
+    share go to fresh blocks and leave the other sequence unchanged."""
+    rng = np.random.default_rng(4)
+    bits, asym, k_axis, g_k, g_v, fp32, R, P = FORMATS[name]
+    unit = R or P
+    c = make(name, max_seqs=3, num_blocks=200)
+    ref = make(name, max_seqs=3, num_blocks=200)
+    T0 = 4 * unit + 3
+    k0, v0 = random_bf16(rng, (T0, 2, D), 3.0), random_bf16(rng, (T0, 2, D))
+    assert c.append(k0, v0, np.zeros(T0, np.int32)) == 0
+    shared = 3 * unit
+    assert c.share_prefix(0, 1, shared) == 0
+    assert c.seq_len(1) == shared
+    assert c.block_table(1).tolist() == c.block_table(0)[:len(c.block_table(1))].tolist()
+    # independent copy: seq 1 of `ref` gets the same prefix rows by appending
+    assert ref.append(k0[:shared], v0[:shared], np.ones(shared, np.int32)) == 0
+    k1, v1 = random_bf16(rng, (2 * unit + 5, 2, D)), random_bf16(rng, (2 * unit + 5, 2, D))
+    k2, v2 = random_bf16(rng, (unit + 1, 2, D)), random_bf16(rng, (unit + 1, 2, D))
+    for cache in (c, ref):
+        assert cache.append(k1, v1, np.ones(len(k1), np.int32)) == 0
+    assert c.append(k2, v2, np.zeros(len(k2), np.int32)) == 0
+    for h in range(2):
+        K1, V1 = c.dequant(1, h, c.seq_len(1))
+        Kr, Vr = ref.dequant(1, h, ref.seq_len(1))
+        assert np.array_equal(K1, Kr) and np.array_equal(V1, Vr)
+        # seq 0: its whole groups/pages from before are unchanged by everything
+        # done to seq 1 (its window tail was quantized later by its own appends)
+        T0w = (T0 // unit) * unit
+        K0, V0 = c.dequant(0, h, T0w)
+        solo = make(name, max_seqs=1, num_blocks=200)
+        assert solo.append(k0, v0, np.zeros(T0, np.int32)) == 0
+        Ks, Vs = solo.dequant(0, h, T0w)
+        assert np.array_equal(K0, Ks) and np.array_equal(V0, Vs)
+        solo.close()
+    c.close()
+    ref.close()
+
+
+def test_shared_blocks_are_freed_by_their_last_holder():
+    c = make("int8_tok_p16", max_seqs=3, num_blocks=40)
+    k = random_bf16(np.random.default_rng(1), (80, 2, D))
+    assert c.append(k, k, np.zeros(80, np.int32)) == 0          # 5 blocks
+    free0 = c.free_count()
+    assert c.share_prefix(0, 1, 64) == 0                         # 4 blocks shared
+    assert c.free_count() == free0
+    t0 = c.block_table(0).tolist()
+    assert c.free_seq(0) == 0                                    # only the unshared block frees
+    assert c.free_count() == free0 + 1
+    assert c.free_seq(1) == 0                                    # now the shared ones, in order
+    assert c.free_count() == free0 + 5
+    # errors leave the state alone
+    assert c.append(k[:20], k[:20], np.zeros(20, np.int32)) == 0
+    for args, code in (((0, 1, 17), 4), ((0, 0, 16), 4), ((0, 1, 32), 4), ((0, 5, 16), 3)):
+        if args[2] == 32:
+            assert c.share_prefix(0, 1, 16) == 0                 # dst no longer empty
+        assert c.share_prefix(*args) == code
+    assert t0 != []
+    c.close()
