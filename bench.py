@@ -48,7 +48,7 @@ def decode_bytes(w, lengths):
     block-table entry per page read."""
     f = w.fmt
     es = 4 if f.scale_fp32 else 2
-    meta = es * (1 + f.asym) if f.bits < 16 else 0      # the BF16 control stores no metadata
+    meta = 0 if (f.bits == 16 or f.fp8) else es * (1 + f.asym)   # BF16 control and FP8: no metadata
     per_tok_q = w.h_kv * (2 * D * f.bits // 8 + D * meta // f.g_k + D * meta // f.g_v)
     per_tok_r = w.h_kv * 2 * D * 2
     total = 0
@@ -390,16 +390,24 @@ def run_control(args):
     k, v, q = dr.step()
     lens = [L + 1 for L in dr.lengths]
     bf = dataclasses.replace(w, fmt=CacheFormat(16, 0, 0, 128, 128, 0, 0, w.fmt.page))
+    f8 = dataclasses.replace(w, fmt=CacheFormat(8, 0, 0, 128, 128, 0, 0, w.fmt.page, fp8=1))
+    # FP8 scales per kv head: amax of the prefill / 448 (no calibration)
+    kf = np.abs((dr.k.view(np.uint16).astype(np.uint32) << 16).view(np.float32))
+    vf = np.abs((dr.v.view(np.uint16).astype(np.uint32) << 16).view(np.float32))
+    f8_scales = ((np.maximum(kf.max(axis=(0, 2)), 1e-6) / 448.0).astype(np.float32),
+                 (np.maximum(vf.max(axis=(0, 2)), 1e-6) / 448.0).astype(np.float32))
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     flush_rd = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     out = {}
-    for tag, ww in (("quantized", w), ("bf16", bf)):
+    for tag, ww in (("quantized", w), ("bf16", bf), ("fp8", f8)):
         f = ww.fmt
         nb = pool_blocks(lens, 2, f.page)
         mbps = max((L + 2) // f.page + 2 for L in lens)
         cache = kvq.KVCache(kvq.Format(f.bits, f.asym, f.k_axis, f.g_k, f.g_v, f.scale_fp32, f.residual,
-                                       f.page), ww.h_q, ww.h_kv, max_seqs=ww.batch, num_blocks=nb,
+                                       f.page, f.fp8), ww.h_q, ww.h_kv, max_seqs=ww.batch, num_blocks=nb,
                             max_blocks_per_seq=mbps, seed=ww.seed, device=torch.cuda.current_device())
+        if f.fp8:
+            cache.set_fp8_scales(*f8_scales)
 
         def dbf(a):
             return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
@@ -424,9 +432,11 @@ def run_control(args):
         nbytes = decode_bytes(ww, lens)
         out[tag] = {"decode_us": us, "kv_bytes": nbytes, "gbs": nbytes / (us * 1e-6) / 1e9}
         cache.close()
-    return {"format": "BF16 control: the same paged path over bf16 rows, no dequantization",
-            "calls": K, "quantized": out["quantized"], "bf16": out["bf16"],
-            "speedup_quantized_over_bf16": out["bf16"]["decode_us"] / out["quantized"]["decode_us"]}
+    return {"format": "BF16 control: the same paged path over bf16 rows, no dequantization; FP8: E4M3 "
+                      "with one scale per kv head (amax / 448 of the prefill)",
+            "calls": K, "quantized": out["quantized"], "bf16": out["bf16"], "fp8": out["fp8"],
+            "speedup_quantized_over_bf16": out["bf16"]["decode_us"] / out["quantized"]["decode_us"],
+            "speedup_fp8_over_bf16": out["bf16"]["decode_us"] / out["fp8"]["decode_us"]}
 
 
 # ---------------------------------------------------------------------------

@@ -92,6 +92,15 @@ enum { KVQ_AXIS_TOKEN = 0, KVQ_AXIS_CHANNEL = 1 };
  *   fail_alloc_after  test hook: allocation number k (0-based, cumulative)
  *               fails when k >= fail_alloc_after; -1 disables it.
  *   host_only   1: no device memory and no kernels (host bookkeeping only;
+ *   fp8         1: the FP8 (E4M3) format, the oh-bug.com page's engineering
+ *               baseline ("FP8 / INT8: Engineering Baseline"): each element is
+ *               e4m3(x / s) (round to nearest even, saturating at +-448) with
+ *               one scale s per kv head for keys and one for values
+ *               (kvq_set_fp8_scales; 1.0 until set), no per-group metadata.
+ *               Needs bits 8, asym 0, k_axis 0, residual 0, scale_fp32 0,
+ *               g_k = g_v = 128.  Key rows keep the key-list order with bytes in
+ *               natural order; value lane records hold each operand register's
+ *               two tokens in adjacent bytes.  0 otherwise.
  *               for tests on machines without a GPU).
  *   device      CUDA device ordinal (ignored when host_only). */
 typedef struct kvq_config {
@@ -113,6 +122,7 @@ typedef struct kvq_config {
   int32_t fail_alloc_after;
   int32_t host_only;
   int32_t device;
+  int32_t fp8;
 } kvq_config;
 
 /* Byte geometry of the paged format.  A block holds `page` token slots of all
@@ -214,6 +224,15 @@ kvq_status kvq_seq_lens_device(kvq_handle h, const int32_t** dev_ptr);
  * orders the device-side reset. */
 kvq_status kvq_free_seq(kvq_handle h, int32_t seq, void* stream);
 
+/* Scales of the FP8 format (config fp8 = 1): k_scales and v_scales are host
+ * float arrays of h_kv entries, one per kv head (equal entries give a
+ * per-tensor scale).  Stored elements are e4m3(x / s) and read back as
+ * s * e4m3.  The pages leave calibration out; a caller typically passes
+ * amax / 448 of a sample of each head.  Must be called before the first
+ * append (KVQ_ERR_INVALID_ARG otherwise, or for a non-FP8 cache or a scale
+ * that is not positive and finite).  Synchronises the device. */
+kvq_status kvq_set_fp8_scales(kvq_handle h, const float* k_scales, const float* v_scales);
+
 /* Prefix sharing of quantized blocks (the paging section of the day-65 page,
  * "How this connects to paging and prefix caching": blocks are what prefix
  * caching shares).  Makes the empty sequence dst_seq start with the first
@@ -296,7 +315,8 @@ kvq_status kvq_set_decode_event(kvq_handle h, void* event);
  * capture.  All calls share the one array and it keeps the last call's
  * contents: calls whose work can overlap on the GPU (different streams
  * without ordering) race on it.  Returns KVQ_ERR_INVALID_ARG with a message
- * giving both sizes when batch * h_kv needs more scratch than the array holds.
+ * giving both sizes when batch * h_kv needs more scratch than the array holds;
+ * KVQ_ERR_UNSUPPORTED for the FP8 format (its per-head scales live in a handle).
  * The partials take (batch * h_kv + grid) * 4 * G * 520 bytes, G = h_q / h_kv
  * and grid = resident decode CTAs (3 per SM, 444 on 148 SMs): with G = 4 that
  * allows about 1,500 (row, kv head) pairs. */
@@ -305,6 +325,24 @@ kvq_status kvq_decode_attn_noalloc(const kvq_config* cfg, const void* pool, cons
                                    int32_t bt_stride, const int32_t* stored_lens,
                                    const int32_t* seq_lens, const void* q_bf16, int32_t batch,
                                    float* out, uint32_t* error_bits_dev, void* stream);
+
+/* Attention for a chunk of query tokens over the quantized cache (chunked
+ * prefill, which oh-bug.com "KV Cache Quantization in Practice" asks a
+ * quantized cache to stay compatible with: "Go-Live Checklist" and Step 1 of
+ * its four-step approach).  Row i is the query of a token whose
+ * keys and values are already appended: it attends positions 0 ..
+ * positions_host[i] of sequence seq_ids_host[i] (causal), with the attention
+ * of kvq_decode_attn.
+ *   q_bf16          device bf16 [n][h_q][d_h].
+ *   seq_ids_host    host int32 [n]; positions_host host int32 [n], each a
+ *                   stored position of its sequence.
+ *   out             device fp32 [n][h_q][d_h].
+ * Runs as decode launches of at most max_seqs rows, each row reading its own
+ * prefix (no reuse of a key tile across the chunk's rows).  Errors:
+ * KVQ_ERR_BAD_SEQ for an id out of range, KVQ_ERR_INVALID_ARG for a position
+ * that is not stored or null / unaligned pointers. */
+kvq_status kvq_prefill_attn(kvq_handle h, const void* q_bf16, const int32_t* seq_ids_host,
+                            const int32_t* positions_host, int32_t n, float* out, void* stream);
 
 /* Text of the last failure on the calling thread ("" if none). */
 const char* kvq_last_error(void);

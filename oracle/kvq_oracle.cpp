@@ -92,6 +92,40 @@ uint16_t f32_to_f16(float x) {
   return uint16_t(sign | uint32_t(r));    // r == 1024 carries into the exponent
 }
 
+// fp32 -> FP8 E4M3 (sign, 4 exponent bits with bias 7, 3 mantissa bits; no
+// infinities, S.1111.111 is NaN, largest finite 448), round to nearest even,
+// saturating: finite values and infinities beyond 448 become +-448, NaN stays
+// NaN.  This is the FP8 KV format the oh-bug.com page calls the engineering
+// baseline ("FP8 / INT8: Engineering Baseline").
+uint8_t f32_to_e4m3(float x) {
+  uint32_t u = f32_bits(x);
+  uint8_t sign = uint8_t((u >> 24) & 0x80u);
+  int exp = int((u >> 23) & 0xFF);
+  uint32_t man = u & 0x7FFFFFu;
+  if (exp == 0xFF) return man ? uint8_t(sign | 0x7Fu) : uint8_t(sign | 0x7Eu);
+  if (exp == 0) return sign;  // fp32 zero/subnormal: far below half of 2^-9
+  int e = exp - 127;          // value = m24 * 2^(e - 23)
+  uint64_t m24 = (uint64_t(1) << 23) | man;
+  if (e >= -6) {              // E4M3 normal range (before rounding)
+    uint64_t r = shift_rne(m24, 20);           // 1.mmm as an integer in [8, 16]
+    if (r == 16) { r = 8; ++e; }
+    if (e > 8 || (e == 8 && r > 14)) return uint8_t(sign | 0x7Eu);   // beyond 448
+    return uint8_t(sign | (uint32_t(e + 7) << 3) | (uint32_t(r) & 7u));
+  }
+  // subnormal: a count of 2^-9 units; a count of 8 is the smallest normal
+  uint64_t r = shift_rne(m24, 14 - e);
+  return uint8_t(sign | uint32_t(r));
+}
+
+float e4m3_to_f32(uint8_t c) {
+  const int E = (c >> 3) & 15, m = c & 7;
+  float v;
+  if (E == 15 && m == 7) v = std::nanf("");
+  else if (E == 0) v = float(m) * 0.001953125f;                    // m * 2^-9
+  else v = std::ldexp(float(8 + m), E - 10);                       // (1 + m/8) * 2^(E-7)
+  return (c & 0x80u) ? -v : v;
+}
+
 float f16_to_f32(uint16_t h) {
   uint32_t sign = uint32_t(h & 0x8000u) << 16;
   int exp = (h >> 10) & 0x1F;
@@ -165,6 +199,7 @@ struct Cfg {
   int32_t h_q, h_kv, d_h, max_seqs, num_blocks, max_blocks_per_seq;
   uint64_t seed;
   int32_t fail_alloc_after;
+  int32_t fp8;   // 1: FP8 E4M3 elements with one scale per kv head (bits 8, no metadata)
 };
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -187,7 +222,14 @@ Layout make_layout(const Cfg& c) {
   L.secK = (P / 16) * L.sub_bytes;
   L.secV = L.secK;
   L.secVm = align_up(P * L.nvg * L.es * A, 16);
-  if (c.bits == 16) {
+  if (c.fp8) {
+    // FP8 E4M3 (oh-bug.com, "FP8 / INT8: Engineering Baseline"): one scale per
+    // kv head for keys and for values, no per-group metadata
+    L.nkg = 1;
+    L.secVm = 0;
+    L.secKm = 0;
+    L.kslice = 0;
+  } else if (c.bits == 16) {
     // The pages' unquantized BF16 cache ("From BF16 to INT8, INT4, or even
     // fewer bits"), kept as a control: rows only, no scales.
     L.nkg = 1;
@@ -228,6 +270,8 @@ struct Loc { size_t byte; int shift; };
 Loc k_loc(const Cfg& c, const Layout& L, const std::vector<int>& inv, int tok, int ch) {
   if (c.bits == 16)   // BF16 control: natural rows, channel ch at bytes 2ch, 2ch+1
     return {size_t(tok / 16) * L.sub_bytes + size_t(tok % 16) * L.row_bytes + size_t(2 * ch), 0};
+  if (c.fp8)          // FP8: key-list order, one byte per element in natural order
+    return {size_t(tok / 16) * L.sub_bytes + size_t(tok % 16) * L.row_bytes + size_t(inv[ch]), 0};
   int f = inv[ch];
   int w = f / L.n, l = f % L.n, p = word_pos(l, L.n);
   size_t byte = size_t(tok / 16) * L.sub_bytes + size_t(tok % 16) * L.row_bytes +
@@ -255,6 +299,10 @@ Loc v_loc(const Cfg& c, const Layout& L, int tok, int ch) {
   int reg = 2 * second + upper;
   int lane = 4 * g + t;
   int word, x;
+  if (c.fp8) {   // FP8: word 2i = [a0 lo, a0 hi, a1 lo, a1 hi], word 2i+1 = a2, a3 likewise
+    word = 2 * i + (reg >> 1);
+    return {size_t(sub) * L.sub_bytes + size_t(lane) * 64u + size_t(4 * word) + size_t(2 * (reg & 1) + hi), 0};
+  }
   if (c.bits == 8) { word = 2 * i + (reg >> 1); x = reg & 1; }
   else if (c.bits == 4) { word = i; x = reg; }
   else { word = i / 2; x = 4 * (reg >> 1) + 2 * (i & 1) + (reg & 1); }
@@ -313,6 +361,7 @@ struct Cache {
   std::deque<int32_t> freelist;
   int64_t alloc_count = 0;
   std::vector<int32_t> holders;    // per block: table rows holding it (shared prefixes)
+  std::vector<float> fp8_k, fp8_v;  // FP8: per kv head scales (1.0 until set)
 };
 
 int64_t blocks_for_len(const Cfg& c, int64_t len) {
@@ -343,6 +392,11 @@ void write_value_row(Cache& C, int32_t block, int tok_in_page, int h, const floa
       put_code(ch + L.off_V, v_loc(c, L, tok_in_page, e), 16, int32_t(f32_bits(x[e]) >> 16));
     return;
   }
+  if (c.fp8) {          // FP8: e4m3(x / s_head), an IEEE fp32 division then RNE + saturation
+    for (int e = 0; e < c.d_h; ++e)
+      put_code(ch + L.off_V, v_loc(c, L, tok_in_page, e), 8, f32_to_e4m3(x[e] / C.fp8_v[size_t(h)]));
+    return;
+  }
   int32_t codes[128];
   for (size_t gi = 0; gi < L.nvg; ++gi) {
     float s = 0, z = 0;
@@ -365,6 +419,11 @@ void write_key_row_token_axis(Cache& C, int32_t block, int tok_in_page, int h, c
   if (c.bits == 16) {   // BF16 control: the row itself
     for (int e = 0; e < c.d_h; ++e)
       put_code(ch, k_loc(c, L, C.inv, tok_in_page, e), 16, int32_t(f32_bits(x[e]) >> 16));
+    return;
+  }
+  if (c.fp8) {
+    for (int e = 0; e < c.d_h; ++e)
+      put_code(ch, k_loc(c, L, C.inv, tok_in_page, e), 8, f32_to_e4m3(x[e] / C.fp8_k[size_t(h)]));
     return;
   }
   int32_t codes[128];
@@ -440,6 +499,15 @@ void dequant_token(const Cache& C, int s, int h, int64_t pos, double* kout, doub
   int32_t blk = C.table[s][size_t(pos / P)];
   int tok = int(pos % P);
   const uint8_t* ch = &C.pool[size_t(blk) * L.block_bytes + size_t(h) * L.chunk_bytes];
+  if (c.fp8) {          // FP8: s_head * e4m3 value
+    for (int e = 0; e < D; ++e) {
+      kout[e] = double(C.fp8_k[size_t(h)]) *
+                e4m3_to_f32(uint8_t(get_code(ch, k_loc(c, L, C.inv, tok, e), 8, false)));
+      vout[e] = double(C.fp8_v[size_t(h)]) *
+                e4m3_to_f32(uint8_t(get_code(ch + L.off_V, v_loc(c, L, tok, e), 8, false)));
+    }
+    return;
+  }
   if (c.bits == 16) {   // BF16 control: the stored rows are the values
     for (int e = 0; e < D; ++e) {
       kout[e] = bf16_to_f32(uint16_t(get_code(ch, k_loc(c, L, C.inv, tok, e), 16, false)));
@@ -482,6 +550,13 @@ extern "C" {
 
 // ---- scalar helpers (exported for the pin tests) ---------------------------
 uint16_t orc_f32_to_f16(float x) { return f32_to_f16(x); }
+uint8_t orc_f32_to_e4m3(float x) { return f32_to_e4m3(x); }
+
+// FP8 format: per kv head scales for keys and values (h_kv each).  Returns 0,
+// or 4 when the cache is not FP8, holds tokens already, or a scale is not a
+// positive finite number.
+int32_t orc_set_fp8_scales(void* hh, const float* k, const float* v);
+float orc_e4m3_to_f32(uint8_t c) { return e4m3_to_f32(c); }
 float orc_f16_to_f32(uint16_t h) { return f16_to_f32(h); }
 float orc_bf16_to_f32(uint16_t b) { return bf16_to_f32(b); }
 float orc_stored_value(float s, int32_t scale_fp32) { return stored_value(s, scale_fp32); }
@@ -543,6 +618,8 @@ void* orc_create(const Cfg* cfg) {
   orc_free_list(C->c.num_blocks, C->c.seed, perm.data());
   C->freelist.assign(perm.begin(), perm.end());
   C->holders.assign(size_t(C->c.num_blocks), 0);
+  C->fp8_k.assign(size_t(C->c.h_kv), 1.0f);
+  C->fp8_v.assign(size_t(C->c.h_kv), 1.0f);
   return C;
 }
 
@@ -643,6 +720,18 @@ int32_t orc_free_seq(void* hh, int32_t s) {
 // length R = g_k (whole key groups).  Returns 0; 3 for bad ids; 4 for dst not
 // empty, dst == src, tokens out of [0, len(src)] or not aligned; 2 when dst's
 // table row is too short.  No state change on error.
+int32_t orc_set_fp8_scales(void* hh, const float* k, const float* v) {
+  Cache& C = *static_cast<Cache*>(hh);
+  if (!C.c.fp8) return 4;
+  for (int32_t L : C.len)
+    if (L) return 4;
+  for (int h = 0; h < C.c.h_kv; ++h)
+    if (!(k[h] > 0.0f) || !(v[h] > 0.0f) || !std::isfinite(k[h]) || !std::isfinite(v[h])) return 4;
+  C.fp8_k.assign(k, k + C.c.h_kv);
+  C.fp8_v.assign(v, v + C.c.h_kv);
+  return 0;
+}
+
 int32_t orc_share_prefix(void* hh, int32_t src, int32_t dst, int32_t tokens) {
   Cache& C = *static_cast<Cache*>(hh);
   const Cfg& c = C.c;

@@ -30,7 +30,7 @@ class OracleConfig(ctypes.Structure):
         ("h_q", ctypes.c_int32), ("h_kv", ctypes.c_int32), ("d_h", ctypes.c_int32),
         ("max_seqs", ctypes.c_int32), ("num_blocks", ctypes.c_int32),
         ("max_blocks_per_seq", ctypes.c_int32), ("seed", ctypes.c_uint64),
-        ("fail_alloc_after", ctypes.c_int32),
+        ("fail_alloc_after", ctypes.c_int32), ("fp8", ctypes.c_int32),
     ]
 
 
@@ -60,6 +60,12 @@ def lib():
         L.orc_layout.argtypes = [P, P]
         L.orc_append.restype = ctypes.c_int32
         L.orc_append.argtypes = [P, P, P, P, ctypes.c_int32]
+        L.orc_f32_to_e4m3.restype = ctypes.c_uint8
+        L.orc_f32_to_e4m3.argtypes = [ctypes.c_float]
+        L.orc_e4m3_to_f32.restype = ctypes.c_float
+        L.orc_e4m3_to_f32.argtypes = [ctypes.c_uint8]
+        L.orc_set_fp8_scales.restype = ctypes.c_int32
+        L.orc_set_fp8_scales.argtypes = [P, P, P]
         L.orc_free_seq.restype = ctypes.c_int32
         L.orc_free_seq.argtypes = [P, ctypes.c_int32]
         L.orc_share_prefix.restype = ctypes.c_int32
@@ -90,6 +96,14 @@ def _ptr(a):
 
 def f32_to_f16_bits(x: float) -> int:
     return lib().orc_f32_to_f16(float(x))
+
+
+def f32_to_e4m3(x: float) -> int:
+    return int(lib().orc_f32_to_e4m3(float(x)))
+
+
+def e4m3_to_f32(c: int) -> float:
+    return float(lib().orc_e4m3_to_f32(int(c)))
 
 
 def f16_bits_to_f32(h: int) -> float:
@@ -147,7 +161,7 @@ class OracleCache:
     def __init__(self, **cfg):
         self.cfg = dict(cfg)
         c = OracleConfig()
-        defaults = dict(asym=0, scale_fp32=0, residual=0, seed=0, fail_alloc_after=-1)
+        defaults = dict(asym=0, scale_fp32=0, residual=0, seed=0, fail_alloc_after=-1, fp8=0)
         for k, _ in OracleConfig._fields_:
             setattr(c, k, int(cfg.get(k, defaults.get(k, 0))))
         self._c = c
@@ -175,6 +189,11 @@ class OracleCache:
 
     def free_seq(self, s: int) -> int:
         return lib().orc_free_seq(self.h, int(s))
+
+    def set_fp8_scales(self, k_scales, v_scales) -> int:
+        k = np.ascontiguousarray(k_scales, dtype=np.float32)
+        v = np.ascontiguousarray(v_scales, dtype=np.float32)
+        return lib().orc_set_fp8_scales(self.h, _ptr(k), _ptr(v))
 
     def share_prefix(self, src: int, dst: int, tokens: int) -> int:
         return lib().orc_share_prefix(self.h, int(src), int(dst), int(tokens))

@@ -352,6 +352,44 @@ __global__ void __launch_bounds__(256) copy_token_kernel(const Geo g, const DevS
   *reinterpret_cast<uint2*>(chunk + g.off_V + row + 8 * lane) = *reinterpret_cast<const uint2*>(vin + in);
 }
 
+// FP8 format: every element becomes e4m3(x / s_head) (an IEEE division, then
+// round to nearest even with saturation at +-448).  Keys keep the key-list
+// order with one byte per element in natural order; values go to lane records
+// where operand register x of tile i holds its two tokens in bytes 2x, 2x + 1
+// of word 2i + x / 2.  One warp per (token, head); each lane writes one key
+// word and four value bytes.
+__global__ void __launch_bounds__(256) fp8_token_kernel(const Geo g, const DevState d, const PlanView p,
+                                                        const uint16_t* kin, const uint16_t* vin) {
+  constexpr int D = kD;
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int64_t item = int64_t(blockIdx.x) * 8 + wib;
+  if (item >= int64_t(p.n_tok) * g.h_kv) return;
+  const int e = int(item / g.h_kv), h = int(item % g.h_kv);
+  const int32_t src = p.plan[p.off_tok + 3 * e];
+  const int32_t blk = p.plan[p.off_tok + 3 * e + 1];
+  const int32_t tok = p.plan[p.off_tok + 3 * e + 2];
+  uint8_t* chunk = d.pool + int64_t(blk) * g.block_bytes + int64_t(h) * g.chunk_bytes;
+  const int sub = tok >> 4, r = tok & 15;
+  const float sk = d.fp8[h], sv = d.fp8[g.h_kv + h];
+  const uint16_t* krow = kin + (int64_t(src) * g.h_kv + h) * D;
+  const uint16_t* vrow = vin + (int64_t(src) * g.h_kv + h) * D;
+  uint32_t word = 0;
+  for (int b = 0; b < 4; ++b) {
+    const float x = bf16_bits_to_float(krow[key_channel(4 * lane + b)]);
+    word |= uint32_t(__nv_cvt_float_to_fp8(__fdiv_rn(x, sk), __NV_SATFINITE, __NV_E4M3)) << (8 * b);
+  }
+  *reinterpret_cast<uint32_t*>(chunk + sub * g.sub_bytes + r * g.row_bytes + 4 * lane) = word;
+  const int tq = (r & 7) >> 1, hi = r & 1, second = r >> 3;
+  uint8_t* vsub = chunk + g.off_V + sub * g.sub_bytes;
+  for (int b = 0; b < 4; ++b) {
+    const int c = 4 * lane + b, i = c >> 4, rr = c & 15, gq = rr & 7, upper = rr >> 3;
+    const int reg = 2 * second + upper;
+    const float x = bf16_bits_to_float(vrow[c]);
+    vsub[(4 * gq + tq) * 64 + 4 * (2 * i + (reg >> 1)) + 2 * (reg & 1) + hi] =
+        uint8_t(__nv_cvt_float_to_fp8(__fdiv_rn(x, sv), __NV_SATFINITE, __NV_E4M3));
+  }
+}
+
 template <typename F>
 cudaError_t by_format(const Geo& g, F&& f) {
   if (g.bits == 8) return g.asym ? f(std::integral_constant<int, 8>(), std::integral_constant<int, 1>())
@@ -386,6 +424,11 @@ cudaError_t launch_quant_token(const Geo& g, const DevState& d, const PlanView& 
   const int blocks = int((items + 7) / 8);
   if (g.bits == 16) {
     copy_token_kernel<<<blocks, 256, 0, s>>>(g, d, p, k, v);
+    ++*launches;
+    return cudaGetLastError();
+  }
+  if (g.fp8) {
+    fp8_token_kernel<<<blocks, 256, 0, s>>>(g, d, p, k, v);
     ++*launches;
     return cudaGetLastError();
   }

@@ -355,7 +355,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
   // The value product runs on fp16 operands when the stored scales are fp16:
   // with the running max exact (p <= 1), p' = p * s fits fp16's range.  Fp32
   // scales keep bf16 operands (fp32 range).
-  constexpr bool PVH = ES == 2;
+  // The FP8 format (ES == 1): e4m3 elements with one scale per kv head,
+  // converted to fp16 operands; the scales are applied once per pair.
+  constexpr bool F8 = ES == 1;
+  constexpr bool PVH = ES == 2 || F8;
   // The BF16 control (16-bit "codes"): 16-token tiles of natural bf16 rows,
   // computed like the BF16 window.
   constexpr bool BF = BITS == 16;
@@ -423,7 +426,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
   };
 
   // ---- staging: each warp fills its own two stages, two units ahead ---------
-  const int vrow = 16 * g.nvg * ES, krow = 16 * g.nkg * ES;
+  // metadata rows of a 16-token sub-tile (none for FP8)
+  const int vrow = F8 ? 0 : 16 * g.nvg * ES, krow = F8 ? 0 : 16 * g.nkg * ES;
   // this lane's block for the unit's copies (loaded early so the latency hides
   // under a unit of compute); -1 when out of the table
   auto load_blk = [&](const It& it, const RowInfo& ri) -> int32_t {
@@ -504,8 +508,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
       bulk_g2s(d, chunk + u * g.sub_bytes, g.sub_bytes, bar);
       bulk_g2s(d + g.sub_bytes, chunk + g.off_V + u * g.sub_bytes, g.sub_bytes, bar);
       const uint32_t vm = d + 2 * g.sub_bytes, km = vm + g.vm16;
-      bulk_g2s(vm, chunk + g.off_Vm + int64_t(16 * u) * g.nvg * ES, vrow, bar);
-      bulk_g2s(km, chunk + g.off_Km + int64_t(16 * u) * g.nkg * ES, krow, bar);
+      if (!F8) {
+        bulk_g2s(vm, chunk + g.off_Vm + int64_t(16 * u) * g.nvg * ES, vrow, bar);
+        bulk_g2s(km, chunk + g.off_Km + int64_t(16 * u) * g.nkg * ES, krow, bar);
+      }
       if (ASYM) {
         bulk_g2s(vm + vrow, chunk + g.off_Vm + int64_t(g.P + 16 * u) * g.nvg * ES, vrow, bar);
         bulk_g2s(km + krow, chunk + g.off_Km + int64_t(g.P + 16 * u) * g.nkg * ES, krow, bar);
@@ -534,6 +540,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
   uint32_t bq[8][2];          // score B operand: fp16 q' hi|lo columns, fp16 q, or bf16 q (window)
   bool bq_bf16 = false;       // bq carries bf16 q for the BF16 window
   float cs = C;               // score scale: C times the power of two taken out of the fp16 operand
+  float vscale = 1.0f;        // FP8: the pair's value scale, applied to its record
   float bias_t = 0.0f;        // channel-axis zero-points: key bias of head tq for the loaded group
   uint32_t qw[4][2];          // channel axis: q of head h at key-list channels 4*lane .. 4*lane+3
   uint32_t qh[4][2];          // the same as fp16, scaled by a power of two per pair (fp16 scales)
@@ -605,8 +612,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
       }
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        rec[2 + 16 * i + gq] = st.o[i][0] + st.o[i][1] + zt[i];
-        rec[2 + 16 * i + gq + 8] = st.o[i][2] + st.o[i][3] + zt[i];
+        rec[2 + 16 * i + gq] = (st.o[i][0] + st.o[i][1] + zt[i]) * vscale;
+        rec[2 + 16 * i + gq + 8] = (st.o[i][2] + st.o[i][3] + zt[i]) * vscale;
       }
     }
   };
@@ -654,6 +661,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
       bq_bf16 = true;
     } else {
       const float down = load_bq_f16(row, h);
+      if (F8) {
+        cs *= a.fp8[h];             // keys: s_k[h] times the scores
+        vscale = a.fp8[g.h_kv + h]; // values: s_v[h] times the weighted sum
+      }
       if (ASYM) {
         // in the operand's scaled domain, like the products it is added to
         const uint16_t* qr = qrow(row, h, tq);
@@ -795,10 +806,17 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       uint32_t a0, a1, a2, a3;
-      key_frag<BITS, SGN, true>(wa, wb, j, a0, a1, a2, a3);
+      if (F8) {
+        a0 = fp8x2_to_h2(wa[j]);
+        a1 = fp8x2_to_h2(wb[j]);
+        a2 = fp8x2_to_h2(wa[j] >> 16);
+        a3 = fp8x2_to_h2(wb[j] >> 16);
+      } else {
+        key_frag<BITS, SGN, true>(wa, wb, j, a0, a1, a2, a3);
+      }
       if (j & 1) mma_f16(acc1, a0, a1, a2, a3, bq[j][0], bq[j][1]);
       else mma_f16(acc0, a0, a1, a2, a3, bq[j][0], bq[j][1]);
-      if (!KAXIS && ((j + 1) & ((1 << kg_shift) - 1)) == 0) {
+      if (!KAXIS && !F8 && ((j + 1) & ((1 << kg_shift) - 1)) == 0) {
         const int gi = j >> kg_shift;
         const float t0 = acc0[0] + acc0[1] + acc1[0] + acc1[1];
         const float t1 = acc0[2] + acc0[3] + acc1[2] + acc1[3];
@@ -812,7 +830,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
         for (int c = 0; c < 4; ++c) acc0[c] = acc1[c] = 0.0f;
       }
     }
-    if (KAXIS) {
+    if (KAXIS || F8) {
       r0 = acc0[0] + acc0[1] + acc1[0] + acc1[1];
       r1 = acc0[2] + acc0[3] + acc1[2] + acc1[3];
     }
@@ -845,7 +863,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
       if ((i & ((1 << vg_shift) - 1)) == 0) {
         const int gi = i >> vg_shift;
         uint32_t h0, l0, h1, l1;
-        if (PVH) {
+        if (F8) {   // one value scale per head, applied to the record: p' = p
+          h0 = pha; l0 = pla; h1 = phb; l1 = plb;
+        } else if (PVH) {
           const uint16_t* vs = reinterpret_cast<const uint16_t*>(sb.vms);
           __half2 sa2, sb2;
           if (n == 2) {
@@ -885,7 +905,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
                     : 0.0f;
       }
       uint32_t a0, a1, a2, a3;
-      value_frag<BITS, SGN, PVH>(vw, i, a0, a1, a2, a3);
+      if (F8) {
+        a0 = fp8x2_to_h2(vw[2 * i]);
+        a1 = fp8x2_to_h2(vw[2 * i] >> 16);
+        a2 = fp8x2_to_h2(vw[2 * i + 1]);
+        a3 = fp8x2_to_h2(vw[2 * i + 1] >> 16);
+      } else {
+        value_frag<BITS, SGN, PVH>(vw, i, a0, a1, a2, a3);
+      }
       if (PVH) mma_f16(st.o[i], a0, a1, a2, a3, b0, b1);
       else mma_bf16(st.o[i], a0, a1, a2, a3, b0, b1);
       if (ASYM) st.zacc[i] += zs;
@@ -1219,6 +1246,7 @@ const void* kernel_of() {
 const void* decode_kernel_ptr(const Geo& g) {
   if (spec_int4_kivi(g)) return kernel_of<4, 0, 1, 2, 1>();
   if (g.bits == 16) return kernel_of<16, 0, 0, 2>();
+  if (g.fp8) return kernel_of<8, 0, 0, 1>();
   const int key = ((g.bits == 8 ? 0 : g.bits == 4 ? 1 : 2) * 4 + g.asym * 2 + g.k_axis) * 2 + (g.es == 4);
   switch (key) {
 #define KVQ_CASE(k, b, as, ax) \

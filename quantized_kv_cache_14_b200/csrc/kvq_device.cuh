@@ -7,6 +7,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include "kvq_internal.h"
 
@@ -60,6 +61,13 @@ __device__ __forceinline__ uint32_t h2_fma(uint32_t a, uint32_t b, uint32_t c) {
   uint32_t r;
   asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
   return r;
+}
+
+// Two FP8 E4M3 values in the low 16 bits of v (low byte first) -> fp16x2,
+// exactly (every E4M3 value is an fp16 value).
+__device__ __forceinline__ uint32_t fp8x2_to_h2(uint32_t v) {
+  const __half2_raw r = __nv_cvt_fp8x2_to_halfraw2(__nv_fp8x2_storage_t(v & 0xFFFFu), __NV_E4M3);
+  return uint32_t(r.x) | (uint32_t(r.y) << 16);
 }
 
 // D += A * B, m16n8k16, fp16 operands, fp32 accumulation.

@@ -35,6 +35,7 @@ struct Geo {
   int num_blocks, max_seqs, mbps;
   int tileT;                // tokens per quantized decode tile
   int lg_P, lg_gk, lg_kslice;   // log2 of page, g_k and kslice (powers of two)
+  int fp8;                  // 1: FP8 E4M3 elements, one scale per kv head (no metadata)
   int vm16, km16;           // token-axis stage: metadata bytes of 16 rows
   int qtile_bytes;          // bytes staged for one quantized tile
 };
@@ -53,6 +54,7 @@ struct DevState {
   int32_t* table;
   int32_t* len;
   uint32_t* err;
+  const float* fp8;   // FP8 format: [2][h_kv] scales (keys, then values)
 };
 
 // Shape of the decode pipeline for a format (see kvq_decode.cu).
@@ -76,6 +78,7 @@ struct DecodeArgs {
   const int32_t* seqmap;      // may be null: row i = sequence i
   const int32_t* stored_len;
   const uint16_t* q;
+  const float* fp8;           // FP8 format: [2][h_kv] scales (keys, then values)
   float* out;
   float* partials;            // [(B * h_kv + grid) * kDecodeWarps * G][D + 2]
   int32_t* prefix;            // [B + 1], written by CTA 0

@@ -52,6 +52,11 @@ kvq_status validate(const kvq_config* c) {
   if (!c) return fail(KVQ_ERR_INVALID_ARG, "config is null");
   if (c->bits != 2 && c->bits != 4 && c->bits != 8 && c->bits != 16)
     return fail(KVQ_ERR_INVALID_ARG, "bits must be 2, 4, 8 or 16");
+  if (c->fp8 != 0 && c->fp8 != 1) return fail(KVQ_ERR_INVALID_ARG, "fp8 must be 0 or 1");
+  if (c->fp8 && (c->bits != 8 || c->k_axis != KVQ_AXIS_TOKEN || c->residual != 0 || c->asym != 0 ||
+                 c->scale_fp32 != 0 || c->g_k != 128 || c->g_v != 128))
+    return fail(KVQ_ERR_INVALID_ARG,
+                "the FP8 format needs bits 8, k_axis 0, residual 0, asym 0, scale_fp32 0, g_k = g_v = 128");
   if (c->bits == 16 && (c->k_axis != KVQ_AXIS_TOKEN || c->residual != 0 || c->asym != 0 || c->scale_fp32 != 0 ||
                         c->g_k != 128 || c->g_v != 128))
     return fail(KVQ_ERR_INVALID_ARG,
@@ -99,7 +104,8 @@ kvq::Geo make_geo(const kvq_config& c) {
   g.secK = (c.page / 16) * g.sub_bytes;
   g.secV = g.secK;
   g.secVm = int(align_up(size_t(c.page) * g.nvg * g.es * A, 16));
-  if (c.bits == 16) {   // BF16 control: rows only, no metadata
+  g.fp8 = c.fp8;
+  if (c.bits == 16 || c.fp8) {   // BF16 control and FP8: no per-group metadata
     g.nkg = 1;
     g.kslice = 0;
     g.secVm = 0;
@@ -127,8 +133,8 @@ kvq::Geo make_geo(const kvq_config& c) {
   g.lg_P = lg(c.page);
   g.lg_gk = lg(c.g_k);
   g.lg_kslice = g.kslice ? lg(g.kslice) : 0;
-  g.vm16 = int(align_up(size_t(16) * g.nvg * g.es * A, 16));
-  g.km16 = int(align_up(size_t(16) * g.nkg * g.es * A, 16));
+  g.vm16 = g.secVm ? int(align_up(size_t(16) * g.nvg * g.es * A, 16)) : 0;
+  g.km16 = g.secKm ? int(align_up(size_t(16) * g.nkg * g.es * A, 16)) : 0;
   g.qtile_bytes = c.k_axis == KVQ_AXIS_CHANNEL ? (c.g_k / c.page) * g.chunk_used
                                                : 2 * g.sub_bytes + g.vm16 + g.km16;
   return g;
@@ -171,6 +177,9 @@ struct kvq_handle_s {
   size_t part_bytes = 0;
   int32_t* d_prefix = nullptr;
   int32_t* d_seqmap = nullptr;
+  int32_t* d_rowlen = nullptr;  // per-row attended lengths of a prefill call
+  float* d_fp8 = nullptr;       // FP8 format: [2][h_kv] scales
+  std::vector<float> fp8;       // host copy
   PinnedSlot slots[4];
   int slot_next = 0;
   int sm_count = 0;
@@ -260,7 +269,7 @@ kvq_status run_plan(kvq_handle h, const Plan& pl, const uint16_t* k, const uint1
   st = stage_upload(h, flat.data(), off, h->d_plan, stream);
   if (st != KVQ_OK) return st;
   pv.plan = h->d_plan;
-  kvq::DevState d{h->d_pool, h->d_kres, h->d_vres, h->d_table, h->d_len, h->d_err};
+  kvq::DevState d{h->d_pool, h->d_kres, h->d_vres, h->d_table, h->d_len, h->d_err, h->d_fp8};
   KVQ_CUDA(kvq::launch_apply(h->geo, d, pv, stream, &h->launches));
   KVQ_CUDA(kvq::launch_quant_token(h->geo, d, pv, k, v, stream, &h->launches));
   KVQ_CUDA(kvq::launch_flush(h->geo, d, pv, k, v, stream, &h->launches));
@@ -282,6 +291,8 @@ void destroy_device(kvq_handle h) {
   cudaFree(h->d_part);
   cudaFree(h->d_prefix);
   cudaFree(h->d_seqmap);
+  cudaFree(h->d_rowlen);
+  cudaFree(h->d_fp8);
   for (auto& s : h->slots) {
     if (s.host) cudaFreeHost(s.host);
     if (s.ev) cudaEventDestroy(s.ev);
@@ -309,6 +320,8 @@ kvq_status create_device(kvq_handle h) {
   KVQ_CUDA(cudaMemset(h->d_len, 0, size_t(c.max_seqs) * sizeof(int32_t)));
   KVQ_CUDA(cudaMalloc(&h->d_err, sizeof(uint32_t)));
   KVQ_CUDA(cudaMemset(h->d_err, 0, sizeof(uint32_t)));
+  KVQ_CUDA(cudaMalloc(&h->d_fp8, size_t(2) * c.h_kv * sizeof(float)));
+  KVQ_CUDA(cudaMemcpy(h->d_fp8, h->fp8.data(), size_t(2) * c.h_kv * sizeof(float), cudaMemcpyHostToDevice));
   for (auto& s : h->slots) KVQ_CUDA(cudaEventCreateWithFlags(&s.ev, cudaEventDisableTiming));
 
   // decode pipeline: stage ring of a producer warp and four consumer warps
@@ -324,6 +337,7 @@ kvq_status create_device(kvq_handle h) {
   KVQ_CUDA(cudaMemset(h->d_part, 0xFF, h->part_bytes));
   KVQ_CUDA(cudaMalloc(&h->d_prefix, size_t(c.max_seqs + 1) * sizeof(int32_t)));
   KVQ_CUDA(cudaMalloc(&h->d_seqmap, size_t(c.max_seqs) * sizeof(int32_t)));
+  KVQ_CUDA(cudaMalloc(&h->d_rowlen, size_t(c.max_seqs) * sizeof(int32_t)));
   h->bytes_workspace = h->part_bytes + size_t(c.max_seqs + 1) * 4 + size_t(c.max_seqs) * 4 + 4;
   return ensure_plan_capacity(h, size_t(1) << 16);
 }
@@ -375,6 +389,7 @@ kvq_status kvq_create(const kvq_config* cfg, kvq_handle* out) {
   h->len.assign(size_t(cfg->max_seqs), 0);
   h->nblk.assign(size_t(cfg->max_seqs), 0);
   h->refcnt.assign(size_t(cfg->num_blocks), 0);
+  h->fp8.assign(size_t(2) * cfg->h_kv, 1.0f);
   h->table.assign(size_t(cfg->max_seqs) * cfg->max_blocks_per_seq, -1);
   // free list: Fisher-Yates over [0, num_blocks) driven by splitmix64(seed)
   std::vector<int32_t> perm(size_t(cfg->num_blocks));
@@ -511,6 +526,40 @@ kvq_status kvq_append(kvq_handle h, const void* k_bf16, const void* v_bf16, cons
   return KVQ_OK;
 }
 
+namespace {
+
+// Decode over the handle's pool and windows for `batch` rows (tables from the
+// caller or the handle's own rows by sequence).
+kvq_status launch_handle_decode(kvq_handle h, const void* q_bf16, const int32_t* block_table, int32_t bt_stride,
+                                const int32_t* seq_lens, const int32_t* seqmap, int32_t batch, float* out,
+                                cudaStream_t stream) {
+  kvq::DecodeArgs a{};
+  a.pool = h->d_pool;
+  a.kres = h->d_kres;
+  a.vres = h->d_vres;
+  a.table = block_table ? block_table : h->d_table;
+  a.table_stride = block_table ? bt_stride : h->cfg.max_blocks_per_seq;
+  a.table_by_seq = block_table ? 0 : 1;
+  a.seq_lens = seq_lens;
+  a.seqmap = seqmap;
+  a.stored_len = h->d_len;
+  a.q = static_cast<const uint16_t*>(q_bf16);
+  a.fp8 = h->d_fp8;
+  a.out = out;
+  a.partials = h->d_part;
+  a.prefix = h->d_prefix;
+  a.err = h->d_err;
+  a.B = batch;
+  a.grid = h->decode_override > 0 ? h->decode_override : h->decode_ctas;
+  a.qk_scale = float(1.4426950408889634 / std::sqrt(double(kvq::kD)));
+  a.pipe = h->pipe;
+  a.g = h->geo;
+  KVQ_CUDA(kvq::launch_decode(a, stream, h->decode_event, &h->launches));
+  return KVQ_OK;
+}
+
+}  // namespace
+
 kvq_status kvq_decode_attn(kvq_handle h, const void* q_bf16, const int32_t* block_table, int32_t bt_stride,
                            const int32_t* seq_lens, const int32_t* seq_ids_host, int32_t batch, float* out,
                            void* stream_) {
@@ -533,27 +582,44 @@ kvq_status kvq_decode_attn(kvq_handle h, const void* q_bf16, const int32_t* bloc
     if (st != KVQ_OK) return st;
     seqmap = h->d_seqmap;
   }
-  kvq::DecodeArgs a{};
-  a.pool = h->d_pool;
-  a.kres = h->d_kres;
-  a.vres = h->d_vres;
-  a.table = block_table ? block_table : h->d_table;
-  a.table_stride = block_table ? bt_stride : h->cfg.max_blocks_per_seq;
-  a.table_by_seq = block_table ? 0 : 1;
-  a.seq_lens = seq_lens;
-  a.seqmap = seqmap;
-  a.stored_len = h->d_len;
-  a.q = static_cast<const uint16_t*>(q_bf16);
-  a.out = out;
-  a.partials = h->d_part;
-  a.prefix = h->d_prefix;
-  a.err = h->d_err;
-  a.B = batch;
-  a.grid = h->decode_override > 0 ? h->decode_override : h->decode_ctas;
-  a.qk_scale = float(1.4426950408889634 / std::sqrt(double(kvq::kD)));
-  a.pipe = h->pipe;
-  a.g = h->geo;
-  KVQ_CUDA(kvq::launch_decode(a, stream, h->decode_event, &h->launches));
+  return launch_handle_decode(h, q_bf16, block_table, bt_stride, seq_lens, seqmap, batch, out, stream);
+}
+
+kvq_status kvq_prefill_attn(kvq_handle h, const void* q_bf16, const int32_t* seq_ids_host,
+                            const int32_t* positions_host, int32_t n, float* out, void* stream_) {
+  if (!h) return fail(KVQ_ERR_INVALID_ARG, "handle is null");
+  if (n < 0) return fail(KVQ_ERR_INVALID_ARG, "n must be >= 0");
+  if (n == 0) return KVQ_OK;
+  kvq_status st = device_guard(h);
+  if (st != KVQ_OK) return st;
+  if (!q_bf16 || !out || !seq_ids_host || !positions_host)
+    return fail(KVQ_ERR_INVALID_ARG, "q, out, seq_ids and positions are required");
+  if (!aligned16(q_bf16) || !aligned16(out)) return fail(KVQ_ERR_INVALID_ARG, "q/out must be 16-byte aligned");
+  const kvq_config& c = h->cfg;
+  for (int32_t i = 0; i < n; ++i) {
+    const int32_t s = seq_ids_host[i];
+    if (s < 0 || s >= c.max_seqs)
+      return fail(KVQ_ERR_BAD_SEQ, "sequence id " + std::to_string(s) + " out of range");
+    if (positions_host[i] < 0 || positions_host[i] >= h->len[size_t(s)])
+      return fail(KVQ_ERR_INVALID_ARG, "position " + std::to_string(positions_host[i]) + " of row " +
+                                           std::to_string(i) + " is not a stored position of its sequence");
+  }
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  // one decode row per query token, attending its own causal prefix; at most
+  // max_seqs rows per launch (the planned batch)
+  std::vector<int32_t> rowlen(size_t(std::min<int32_t>(n, c.max_seqs)));
+  const int64_t row = int64_t(c.h_q) * c.d_h;
+  for (int32_t base = 0; base < n; base += c.max_seqs) {
+    const int32_t m = std::min<int32_t>(c.max_seqs, n - base);
+    for (int32_t j = 0; j < m; ++j) rowlen[size_t(j)] = positions_host[base + j] + 1;
+    st = stage_upload(h, seq_ids_host + base, size_t(m), h->d_seqmap, stream);
+    if (st != KVQ_OK) return st;
+    st = stage_upload(h, rowlen.data(), size_t(m), h->d_rowlen, stream);
+    if (st != KVQ_OK) return st;
+    st = launch_handle_decode(h, static_cast<const uint16_t*>(q_bf16) + base * row, nullptr, 0, h->d_rowlen,
+                              h->d_seqmap, m, out + base * row, stream);
+    if (st != KVQ_OK) return st;
+  }
   return KVQ_OK;
 }
 
@@ -608,6 +674,29 @@ kvq_status kvq_free_seq(kvq_handle h, int32_t seq, void* stream_) {
   }
   h->nblk[size_t(seq)] = 0;
   h->len[size_t(seq)] = 0;
+  return KVQ_OK;
+}
+
+kvq_status kvq_set_fp8_scales(kvq_handle h, const float* k_scales, const float* v_scales) {
+  if (!h) return fail(KVQ_ERR_INVALID_ARG, "handle is null");
+  if (!h->cfg.fp8) return fail(KVQ_ERR_INVALID_ARG, "the cache is not in the FP8 format");
+  if (!k_scales || !v_scales) return fail(KVQ_ERR_INVALID_ARG, "scales are required");
+  for (int32_t L : h->len)
+    if (L) return fail(KVQ_ERR_INVALID_ARG, "scales must be set before the first append");
+  const int H = h->cfg.h_kv;
+  for (int i = 0; i < H; ++i)
+    if (!(k_scales[i] > 0.0f) || !(v_scales[i] > 0.0f) || !std::isfinite(k_scales[i]) || !std::isfinite(v_scales[i]))
+      return fail(KVQ_ERR_INVALID_ARG, "scales must be positive finite numbers");
+  std::vector<float> s(size_t(2) * H);
+  std::copy(k_scales, k_scales + H, s.begin());
+  std::copy(v_scales, v_scales + H, s.begin() + H);
+  if (!h->cfg.host_only) {
+    kvq_status st = device_guard(h);
+    if (st != KVQ_OK) return st;
+    KVQ_CUDA(cudaDeviceSynchronize());   // earlier work may still read the old scales
+    KVQ_CUDA(cudaMemcpy(h->d_fp8, s.data(), s.size() * sizeof(float), cudaMemcpyHostToDevice));
+  }
+  h->fp8 = s;
   return KVQ_OK;
 }
 
@@ -731,6 +820,7 @@ kvq_status kvq_decode_attn_noalloc(const kvq_config* cfg, const void* pool, cons
                                    int32_t batch, float* out, uint32_t* error_bits_dev, void* stream_) {
   kvq_status st = validate(cfg);
   if (st != KVQ_OK) return st;
+  if (cfg->fp8) return fail(KVQ_ERR_UNSUPPORTED, "the FP8 format is not served without a handle (its scales live there)");
   if (batch < 0 || batch > cfg->max_seqs) return fail(KVQ_ERR_INVALID_ARG, "batch must be in [0, max_seqs]");
   if (batch == 0) return KVQ_OK;
   if (!pool || !block_table || !stored_lens || !seq_lens || !q_bf16 || !out)

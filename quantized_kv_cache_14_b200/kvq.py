@@ -40,7 +40,7 @@ EXPORTS = (
     "kvq_block_table_host", "kvq_seq_len", "kvq_seq_lens_device", "kvq_free_seq", "kvq_share_prefix",
     "kvq_stats", "kvq_cache_bytes", "kvq_layout", "kvq_read_pool", "kvq_read_residual",
     "kvq_sync_status", "kvq_set_decode_grid", "kvq_set_decode_event", "kvq_decode_attn_noalloc",
-    "kvq_last_error",
+    "kvq_prefill_attn", "kvq_set_fp8_scales", "kvq_last_error",
 )
 
 
@@ -59,7 +59,7 @@ class KvqConfig(ctypes.Structure):
         ("max_seqs", ctypes.c_int32), ("num_blocks", ctypes.c_int32),
         ("max_blocks_per_seq", ctypes.c_int32), ("seed", ctypes.c_uint64),
         ("fail_alloc_after", ctypes.c_int32), ("host_only", ctypes.c_int32),
-        ("device", ctypes.c_int32),
+        ("device", ctypes.c_int32), ("fp8", ctypes.c_int32),
     ]
 
 
@@ -98,6 +98,8 @@ def lib():
             "kvq_seq_lens_device": (st, [P, ctypes.POINTER(P)]),
             "kvq_free_seq": (st, [P, I32, P]),
             "kvq_share_prefix": (st, [P, I32, I32, I32, P]),
+            "kvq_prefill_attn": (st, [P, P, P, P, I32, P, P]),
+            "kvq_set_fp8_scales": (st, [P, P, P]),
             "kvq_stats": (st, [P, ctypes.POINTER(KvqStats)]),
             "kvq_cache_bytes": (U64, [I32, ctypes.c_int64, I32, I32, ctypes.POINTER(KvqConfig)]),
             "kvq_layout": (st, [ctypes.POINTER(KvqConfig), ctypes.POINTER(KvqLayoutInfo)]),
@@ -132,10 +134,10 @@ def _host_i32(a):
 
 def make_config(bits, asym, k_axis, g_k, g_v, scale_fp32, residual, page, h_q, h_kv, d_h,
                 max_seqs, num_blocks, max_blocks_per_seq, seed=0, fail_alloc_after=-1,
-                host_only=0, device=0) -> KvqConfig:
+                host_only=0, device=0, fp8=0) -> KvqConfig:
     return KvqConfig(bits, asym, k_axis, g_k, g_v, scale_fp32, residual, page, h_q, h_kv, d_h,
                      max_seqs, num_blocks, max_blocks_per_seq, seed, fail_alloc_after,
-                     host_only, device)
+                     host_only, device, fp8)
 
 
 # ---- the C calls, same names --------------------------------------------------
@@ -193,6 +195,21 @@ def kvq_seq_lens_device(h) -> int:
 
 def kvq_free_seq(h, seq: int, stream: int = 0):
     _check(lib().kvq_free_seq(h, int(seq), ctypes.c_void_p(stream)))
+
+
+def kvq_prefill_attn(h, q_ptr: int, seq_ids, positions, out_ptr: int, stream: int = 0):
+    ids = np.ascontiguousarray(seq_ids, dtype=np.int32)
+    pos = np.ascontiguousarray(positions, dtype=np.int32)
+    assert ids.shape == pos.shape
+    V = ctypes.c_void_p
+    _check(lib().kvq_prefill_attn(h, V(q_ptr), V(ids.ctypes.data), V(pos.ctypes.data), int(ids.size), V(out_ptr),
+                                  V(stream)))
+
+
+def kvq_set_fp8_scales(h, k_scales, v_scales):
+    k = np.ascontiguousarray(k_scales, dtype=np.float32)
+    v = np.ascontiguousarray(v_scales, dtype=np.float32)
+    _check(lib().kvq_set_fp8_scales(h, ctypes.c_void_p(k.ctypes.data), ctypes.c_void_p(v.ctypes.data)))
 
 
 def kvq_share_prefix(h, src_seq: int, dst_seq: int, tokens: int, stream: int = 0):
@@ -275,6 +292,7 @@ class Format:
     scale_fp32: int
     residual: int
     page: int
+    fp8: int = 0
 
 
 class KVCache:
@@ -285,7 +303,8 @@ class KVCache:
         self.fmt = fmt
         self.cfg = make_config(fmt.bits, fmt.asym, fmt.k_axis, fmt.g_k, fmt.g_v, fmt.scale_fp32,
                                fmt.residual, fmt.page, h_q, h_kv, d_h, max_seqs, num_blocks,
-                               max_blocks_per_seq, seed, fail_alloc_after, int(host_only), device)
+                               max_blocks_per_seq, seed, fail_alloc_after, int(host_only), device,
+                               int(getattr(fmt, "fp8", 0)))
         self.h = kvq_create(self.cfg)
         self.h_q, self.h_kv, self.d_h = h_q, h_kv, d_h
         self.layout = kvq_layout(self.cfg)
@@ -333,6 +352,14 @@ class KVCache:
 
     def free_seq(self, s, stream=None):
         kvq_free_seq(self.h, s, 0 if self.cfg.host_only else self._stream(stream))
+
+    def prefill_attn(self, q, seq_ids, positions, out, stream=None):
+        """q: cuda bf16 [n, h_q, d_h]; out: cuda fp32 [n, h_q, d_h]; row i attends
+        positions 0..positions[i] of sequence seq_ids[i]."""
+        kvq_prefill_attn(self.h, q.data_ptr(), seq_ids, positions, out.data_ptr(), self._stream(stream))
+
+    def set_fp8_scales(self, k_scales, v_scales):
+        kvq_set_fp8_scales(self.h, k_scales, v_scales)
 
     def share_prefix(self, src, dst, tokens, stream=None):
         kvq_share_prefix(self.h, src, dst, tokens, 0 if self.cfg.host_only else self._stream(stream))

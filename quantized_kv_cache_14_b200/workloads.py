@@ -42,6 +42,7 @@ class CacheFormat:
     scale_fp32: int
     residual: int        # R (0 for per-token keys, == g_k for per-channel keys)
     page: int            # P tokens per block
+    fp8: int = 0         # 1: FP8 E4M3 elements with one scale per kv head
 
 
 @dataclass

@@ -23,7 +23,7 @@ def built():
 def header_functions():
     src = open(os.path.join(ROOT, "include", "kvq.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(kvq_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(kvq_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_exports_match_header():
@@ -31,7 +31,7 @@ def test_exports_match_header():
     assert declared == sorted(kvq.EXPORTS)
     out = subprocess.run(["nm", "-D", "--defined-only", kvq.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
-    exported = set(re.findall(r" T (kvq_[a-z_]+)$", out, flags=re.M))
+    exported = set(re.findall(r" T (kvq_[a-z0-9_]+)$", out, flags=re.M))
     assert set(declared) <= exported
     L = kvq.lib()
     for name in declared:
@@ -46,6 +46,7 @@ FMTS = {
     "int4_chan64_p32": dict(bits=4, asym=0, k_axis=1, g_k=64, g_v=32, scale_fp32=0, residual=64, page=32),
     "int4_asym_tok32": dict(bits=4, asym=1, k_axis=0, g_k=32, g_v=32, scale_fp32=0, residual=0, page=32),
     "bf16_control_p16": dict(bits=16, asym=0, k_axis=0, g_k=128, g_v=128, scale_fp32=0, residual=0, page=16),
+    "fp8_p32": dict(bits=8, asym=0, k_axis=0, g_k=128, g_v=128, scale_fp32=0, residual=0, page=32, fp8=1),
 }
 
 
@@ -179,6 +180,29 @@ def test_cache_bytes_formula_worked_example():
     assert kvq.kvq_cache_bytes(1, 100, 8, 128, cfg2) == 2 * 102400 // 4 + 2 * 102400 * 4 // 32
     cfg16, _ = cfg_of("bf16_control_p16")      # BF16: 2 bytes per element, no metadata
     assert kvq.kvq_cache_bytes(32, 8192, 8, 128, cfg16) == 2 * elems * 2
+
+
+def test_fp8_config_rules():
+    for field, value in (("bits", 4), ("asym", 1), ("scale_fp32", 1), ("g_k", 64), ("fp8", 2)):
+        cfg, _ = cfg_of("fp8_p32")
+        setattr(cfg, field, value)
+        with pytest.raises(kvq.KvqError) as e:
+            kvq.kvq_create(cfg)
+        assert e.value.status == kvq.KVQ_ERR_INVALID_ARG
+    cfg, _ = cfg_of("fp8_p32")
+    h = kvq.kvq_create(cfg)
+    kvq.kvq_set_fp8_scales(h, [0.5, 2.0], [1.0, 1.0])
+    with pytest.raises(kvq.KvqError):
+        kvq.kvq_set_fp8_scales(h, [0.0, 1.0], [1.0, 1.0])       # not positive
+    kvq.kvq_append(h, 0, 0, np.zeros(3, np.int32), 3)
+    with pytest.raises(kvq.KvqError):
+        kvq.kvq_set_fp8_scales(h, [1.0, 1.0], [1.0, 1.0])       # tokens stored already
+    kvq.kvq_destroy(h)
+    cfg, _ = cfg_of("int8_tok_p16")
+    h = kvq.kvq_create(cfg)
+    with pytest.raises(kvq.KvqError):
+        kvq.kvq_set_fp8_scales(h, [1.0, 1.0], [1.0, 1.0])       # not an FP8 cache
+    kvq.kvq_destroy(h)
 
 
 def test_bf16_control_config_rules():

@@ -10,6 +10,7 @@ import pytest
 import torch
 
 from quantized_kv_cache_14_b200 import build as kbuild
+from quantized_kv_cache_14_b200 import kvq
 from quantized_kv_cache_14_b200.workloads import Draws, random_bf16, workload
 from tests.gpu_util import ATOL, Pair, bits_to_cuda_bf16
 
@@ -38,6 +39,9 @@ FMTS = {
     # the pages' unquantized BF16 cache on the same paged path (control)
     "bf16_control_p16": dict(bits=16, asym=0, k_axis=0, g_k=128, g_v=128, scale_fp32=0, residual=0, page=16),
     "bf16_control_p64": dict(bits=16, asym=0, k_axis=0, g_k=128, g_v=128, scale_fp32=0, residual=0, page=64),
+    # FP8 E4M3 with one scale per kv head (1.0 unless a test sets them)
+    "fp8_p16": dict(bits=8, asym=0, k_axis=0, g_k=128, g_v=128, scale_fp32=0, residual=0, page=16, fp8=1),
+    "fp8_p32": dict(bits=8, asym=0, k_axis=0, g_k=128, g_v=128, scale_fp32=0, residual=0, page=32, fp8=1),
 }
 
 
@@ -86,7 +90,7 @@ def test_incremental_appends_interleaved(name):
     p.close()
 
 
-@pytest.mark.parametrize("name", ["int4_chan64", "int8_tok_p16", "int2_asym_chan32", "bf16_control_p16"])
+@pytest.mark.parametrize("name", ["int4_chan64", "int8_tok_p16", "int2_asym_chan32", "bf16_control_p16", "fp8_p16"])
 def test_split_k_merge_is_invariant_to_grid(name):
     rng = np.random.default_rng(3)
     h_q, h_kv = 16, 4
@@ -131,6 +135,63 @@ def test_shared_prefix_decode(name):
     assert p.orc.free_seq(0) == 0
     p.check_state()
     p.check_decode(random_bf16(rng, (3, h_q, D)), [0] + lens[1:])
+    p.close()
+
+
+@pytest.mark.parametrize("name", ["int4_chan64", "int8_tok_p16", "int2_asym_chan32"])
+def test_chunked_prefill_attention(name):
+    """Chunked prefill: append a chunk, then each chunk token attends its own
+    causal prefix (rows straddle the quantized/window boundary and span more
+    rows than max_seqs, so the call takes several launches)."""
+    rng = np.random.default_rng(12)
+    fmt = FMTS[name]
+    h_q, h_kv, S = 8, 2, 3
+    p = Pair(fmt, h_q, h_kv, max_seqs=S, num_blocks=300, mbps=64, seed=7)
+    pre = [150, 37, 64]
+    ids = np.repeat(np.arange(S, dtype=np.int32), pre)
+    p.append(outlier_keys(rng, ids.size, h_kv), random_bf16(rng, (ids.size, h_kv, D)), ids)
+    chunk = [45, 20, 9]
+    cids = np.repeat(np.arange(S, dtype=np.int32), chunk)
+    p.append(outlier_keys(rng, cids.size, h_kv), random_bf16(rng, (cids.size, h_kv, D)), cids)
+    pos = np.concatenate([np.arange(pre[s], pre[s] + chunk[s]) for s in range(S)]).astype(np.int32)
+    q = random_bf16(rng, (cids.size, h_q, D))
+    out = torch.full((cids.size, h_q, D), float("nan"), dtype=torch.float32, device="cuda")
+    p.gpu.prefill_attn(bits_to_cuda_bf16(q), cids, pos, out)
+    torch.cuda.synchronize()
+    assert p.gpu.sync_status() == 0
+    want = p.orc.decode(q, (pos + 1).tolist(), seq_ids=cids)
+    got = out.cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(got))
+    err = float(np.max(np.abs(got - want)))
+    assert err <= 2e-3, f"max abs error {err}"
+    with pytest.raises(kvq.KvqError):   # a position that is not stored yet
+        p.gpu.prefill_attn(bits_to_cuda_bf16(q[:1]), [0], [pre[0] + chunk[0]], out)
+    p.close()
+
+
+@pytest.mark.parametrize("page", [16, 32])
+def test_fp8_per_head_scales(page):
+    """FP8 with per-head scales from amax / 448 of a sample, keys with large
+    outliers, and values beyond the scaled range (saturation at +-448)."""
+    rng = np.random.default_rng(31)
+    fmt = dict(FMTS["fp8_p16"], page=page)
+    h_q, h_kv, S = 8, 2, 3
+    p = Pair(fmt, h_q, h_kv, max_seqs=S, num_blocks=200, mbps=64, seed=3)
+    lens = [300, 45, 129]
+    ids = np.repeat(np.arange(S, dtype=np.int32), lens)
+    k = outlier_keys(rng, ids.size, h_kv, gain=40.0)
+    v = random_bf16(rng, (ids.size, h_kv, D), 2.0)
+    from oracle import oracle as O
+    kf, vf = O.bf16_bits_to_f32(k), O.bf16_bits_to_f32(v)
+    ks = (np.abs(kf[:100]).max(axis=(0, 2)) / 448.0).astype(np.float32)   # amax of a sample per head
+    vs = (np.abs(vf[:100]).max(axis=(0, 2)) / 448.0 / 2.0).astype(np.float32)   # half: values saturate
+    p.gpu.set_fp8_scales(ks, vs)
+    assert p.orc.set_fp8_scales(ks, vs) == 0
+    p.append(k, v, ids)
+    p.check_state()
+    p.check_decode(random_bf16(rng, (S, h_q, D)), lens)
+    with pytest.raises(kvq.KvqError):          # scales are fixed once tokens are stored
+        p.gpu.set_fp8_scales(ks, vs)
     p.close()
 
 

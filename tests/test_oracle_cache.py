@@ -488,3 +488,45 @@ def test_shared_blocks_are_freed_by_their_last_holder():
         assert c.share_prefix(*args) == code
     assert t0 != []
     c.close()
+
+
+# ------------------------------------------------------------ FP8 format
+
+def test_fp8_dequant_is_scale_times_e4m3_of_the_scaled_input():
+    """FP8 E4M3 with one scale per kv head: the stored byte of element x is
+    e4m3(x / s) (pinned converter), read back as s * e4m3; keys keep the
+    key-list order one byte per element, values the lane records."""
+    rng = np.random.default_rng(6)
+    c = O.OracleCache(bits=8, asym=0, k_axis=0, g_k=128, g_v=128, scale_fp32=0, residual=0, page=16, fp8=1,
+                      h_q=4, h_kv=2, d_h=D, max_seqs=2, num_blocks=40, max_blocks_per_seq=40, seed=2,
+                      fail_alloc_after=-1)
+    ks, vs = np.array([0.25, 3.0], np.float32), np.array([1.5, 0.01], np.float32)
+    assert c.set_fp8_scales(ks, vs) == 0
+    T = 37
+    k = random_bf16(rng, (T, 2, D), 5.0)
+    v = random_bf16(rng, (T, 2, D), 5.0)
+    assert c.append(k, v, np.zeros(T, np.int32)) == 0
+    assert c.set_fp8_scales(ks, vs) == 4                     # fixed once tokens are stored
+    lay = c.layout
+    assert lay["off_Vm"] == lay["off_Km"] == 2 * lay["secK"]   # no metadata
+    kf, vf = O.bf16_bits_to_f32(k), O.bf16_bits_to_f32(v)
+    for h in range(2):
+        K, V = c.dequant(0, h, T)
+        for t in (0, 5, 36):
+            for ch in (0, 9, 77, 127):
+                ck = O.f32_to_e4m3(float(np.float32(kf[t, h, ch]) / ks[h]))
+                cv = O.f32_to_e4m3(float(np.float32(vf[t, h, ch]) / vs[h]))
+                assert K[t, ch] == float(ks[h]) * O.e4m3_to_f32(ck)
+                assert V[t, ch] == float(vs[h]) * O.e4m3_to_f32(cv)
+    # values beyond 448 s saturate
+    assert np.max(np.abs(c.dequant(0, 1, T)[1])) <= 448 * float(vs[1]) + 1e-12
+    # layout: every byte of a section belongs to one element, key rows in list order
+    for kind, sec in (("k", lay["secK"]), ("v", lay["secV"])):
+        seen = np.zeros(sec, np.int32)
+        for tok in range(16):
+            for ch in range(D):
+                b, sh = c.code_loc(kind, tok, ch)
+                assert sh == 0
+                seen[b] += 1
+        assert np.all(seen == 1)
+    c.close()

@@ -4,6 +4,7 @@ published generator vectors and brute force.  CPU only."""
 import math
 
 import numpy as np
+import torch
 import pytest
 
 from oracle import oracle as O
@@ -246,3 +247,55 @@ def test_free_list_is_fisher_yates_permutation():
     j = x2 % 2
     p[1], p[j] = p[j], p[1]
     assert O.free_list(3, 9).tolist() == p
+
+
+# ------------------------------------------------------------------ FP8 E4M3
+
+def _e4m3_value(c):
+    """The E4M3 code table written from its definition: sign, 4-bit exponent
+    with bias 7, 3-bit mantissa, subnormals at exponent 0, S.1111.111 NaN."""
+    sign = -1.0 if c & 0x80 else 1.0
+    E, m = (c >> 3) & 15, c & 7
+    if E == 15 and m == 7:
+        return float("nan")
+    if E == 0:
+        return sign * m / 8.0 * 2.0 ** -6
+    return sign * (1.0 + m / 8.0) * 2.0 ** (E - 7)
+
+
+def test_e4m3_code_table_and_exact_values():
+    for c in range(256):
+        want = _e4m3_value(c)
+        got = O.e4m3_to_f32(c)
+        if np.isnan(want):
+            assert np.isnan(got)
+            continue
+        assert got == want, (c, got, want)
+        assert O.f32_to_e4m3(want) == c      # every value encodes to its own code (-0 keeps its sign)
+    assert _e4m3_value(0x7E) == 448.0 and _e4m3_value(0x08) == 2.0 ** -6 and _e4m3_value(0x01) == 2.0 ** -9
+
+
+def test_e4m3_round_to_nearest_even_and_saturation():
+    vals = sorted({_e4m3_value(c) for c in range(0x7F)})            # non-negative finite values
+    codes = {v: O.f32_to_e4m3(v) for v in vals}
+    for lo, hi in zip(vals, vals[1:]):
+        mid = np.float32((lo + hi) / 2.0)
+        assert float(mid) == (lo + hi) / 2.0                          # midpoints are exact in fp32
+        even = lo if (codes[lo] & 1) == 0 else hi
+        assert O.f32_to_e4m3(float(mid)) == codes[even]
+        assert O.f32_to_e4m3(float(np.nextafter(mid, np.float32(0)))) == codes[lo]
+        assert O.f32_to_e4m3(float(np.nextafter(mid, np.float32(np.inf)))) == codes[hi]
+    for x in (448.0, 449.0, 463.9, 464.0, 1e6, float("inf")):
+        assert O.f32_to_e4m3(x) == 0x7E and O.f32_to_e4m3(-x) == 0xFE
+    assert O.f32_to_e4m3(float("nan")) & 0x7F == 0x7F
+
+
+def test_e4m3_matches_torch_float8_in_range():
+    """Independent library check inside the finite range (torch's e4m3fn cast
+    rounds to nearest even; beyond 448 it does not saturate, so stay inside)."""
+    rng = np.random.default_rng(5)
+    x = np.concatenate([rng.uniform(-448, 448, 20000), rng.normal(0, 1, 20000),
+                        rng.normal(0, 2.0 ** -8, 20000)]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([O.f32_to_e4m3(float(v)) for v in x], dtype=np.uint8)
+    assert np.array_equal(got, ref)
