@@ -150,7 +150,11 @@ __global__ void __launch_bounds__(256) quant_token_kernel(const Geo g, const Dev
 }
 
 // ---------------------------------------------------------------------------
-// Per-channel key flush: one CTA per (flushed group, head).
+// Per-channel key flush: one CTA per (flushed group, head, 16-token sub-tile).
+// Every CTA gathers the group's R key rows and computes all channel scales
+// (they need every row), then writes only its own sub-tile's key and value
+// codes, value scales, and -- when its sub-tile starts a page -- that page's
+// slice of the key scales.
 template <int BITS, int ASYM>
 __global__ void __launch_bounds__(kFlushThreads) flush_kernel(const Geo g, const DevState d,
                                                               const PlanView p,
@@ -168,17 +172,20 @@ __global__ void __launch_bounds__(kFlushThreads) flush_kernel(const Geo g, const
   float* vsc = kzp + D;                                              // [R][nvg]
   float* vzp = vsc + R * g.nvg;                                      // [R][nvg]
 
-  const int e = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+  const int e = blockIdx.x, h = blockIdx.y, zs = blockIdx.z, tid = threadIdx.x;
+  const int r_lo = 16 * zs;   // this CTA's rows [r_lo, r_lo + 16)
   const int32_t* ent = p.plan + p.off_flush + e * kFlushEntryInts;
   const int seq = ent[0];
   const int npg = ent[2];
   const int32_t* srcs = p.plan + p.off_src + int64_t(e) * R;
 
-  // 1. gather the group's K and V rows (bf16) into shared memory
+  // 1. gather the group's K rows and this sub-tile's V rows (bf16) into
+  //    shared memory
   for (int idx = tid; idx < R * (D / 8) * 2; idx += blockDim.x) {
     const int which = idx / (R * (D / 8));
     const int rem = idx % (R * (D / 8));
     const int r = rem / (D / 8), c8 = rem % (D / 8);
+    if (which && (r < r_lo || r >= r_lo + 16)) continue;
     const int32_t s = srcs[r];
     const uint16_t* src;
     if (s >= 0) src = (which ? vin : kin) + (int64_t(s) * g.h_kv + h) * D;
@@ -207,7 +214,7 @@ __global__ void __launch_bounds__(kFlushThreads) flush_kernel(const Geo g, const
   } else {
     const int w = (tid - D) >> 5, lane = tid & 31;
     const int lanes_per_group = g.g_v / 4;
-    for (int r = w; r < R; r += (blockDim.x - D) / 32) {
+    for (int r = r_lo + w; r < r_lo + 16; r += (blockDim.x - D) / 32) {
       float x[4];
       for (int i = 0; i < 4; ++i) x[i] = bf16_bits_to_float(vt[r * D + 4 * lane + i]);
       float a = 0.0f, mn = x[0], mx = x[0];
@@ -254,9 +261,9 @@ __global__ void __launch_bounds__(kFlushThreads) flush_kernel(const Geo g, const
 
   // 3. key codes: word W of the group -> (sub-tile, row, word in row)
   const int row_words = D * BITS / 32;
-  const int k_words = R * row_words;
+  const int k_words = 16 * row_words;
   for (int W = tid; W < k_words; W += blockDim.x) {
-    const int rowi = W / row_words, w = W % row_words;       // rowi = token in group
+    const int rowi = r_lo + W / row_words, w = W % row_words;   // rowi = token in group
     uint32_t word = 0;
     for (int l = 0; l < N; ++l) word |= kcode(rowi, key_channel(w * N + l)) << (BITS * word_field(l, N));
     const int sub = rowi >> 4, rr = rowi & 15;
@@ -270,9 +277,9 @@ __global__ void __launch_bounds__(kFlushThreads) flush_kernel(const Geo g, const
   //    16-channel tile i: a0 = (ch 16i+gq, tok 2tq | 2tq+1), a1 = ch + 8,
   //    a2 = tokens + 8, a3 = both.
   const int rec_words = 2 * BITS;
-  const int v_words = (R / 16) * 32 * rec_words;
+  const int v_words = 32 * rec_words;
   for (int W = tid; W < v_words; W += blockDim.x) {
-    const int sub = W / (32 * rec_words), rem = W % (32 * rec_words);
+    const int sub = zs, rem = W;
     const int lam = rem / rec_words, w = rem % rec_words;
     const int gq = lam >> 2, tq = lam & 3;
     uint32_t word = 0;
@@ -291,16 +298,19 @@ __global__ void __launch_bounds__(kFlushThreads) flush_kernel(const Geo g, const
     *reinterpret_cast<uint32_t*>(dst) = word;
   }
 
-  // 5. metadata: key scales in list order, striped over the group's pages;
-  //    value scales per token row
-  for (int f = tid; f < D; f += blockDim.x) {
-    const int c = key_channel(f);
-    const int page = f / g.kslice, off = f % g.kslice;
-    uint8_t* km = chunk_of(page) + g.off_Km;
-    store_meta(km + off * g.es, ksc[c], g.scale_fp32);
-    if (ASYM) store_meta(km + (g.kslice + off) * g.es, kzp[c], g.scale_fp32);
+  // 5. metadata: key scales in list order, striped over the group's pages
+  //    (the CTA of a page's first sub-tile writes that page's slice); value
+  //    scales of this sub-tile's rows
+  if (r_lo % g.P == 0) {
+    const int page = r_lo / g.P;
+    for (int off = tid; off < g.kslice; off += blockDim.x) {
+      const int c = key_channel(page * g.kslice + off);
+      uint8_t* km = chunk_of(page) + g.off_Km;
+      store_meta(km + off * g.es, ksc[c], g.scale_fp32);
+      if (ASYM) store_meta(km + (g.kslice + off) * g.es, kzp[c], g.scale_fp32);
+    }
   }
-  for (int idx = tid; idx < R * g.nvg; idx += blockDim.x) {
+  for (int idx = r_lo * g.nvg + tid; idx < (r_lo + 16) * g.nvg; idx += blockDim.x) {
     const int r = idx / g.nvg, gi = idx % g.nvg;
     const int page = r / g.P, rp = r % g.P;
     uint8_t* vm = chunk_of(page) + g.off_Vm;
@@ -455,7 +465,7 @@ cudaError_t launch_flush(const Geo& g, const DevState& d, const PlanView& p, con
       if (e != cudaSuccess) return e;
       if (dev < 32) limit_set[dev] = smem;
     }
-    kern<<<dim3(p.n_flush, g.h_kv), kFlushThreads, smem, s>>>(g, d, p, k, v);
+    kern<<<dim3(p.n_flush, g.h_kv, g.R / 16), kFlushThreads, smem, s>>>(g, d, p, k, v);
     ++*launches;
     return cudaGetLastError();
   });
