@@ -16,7 +16,11 @@
  *    (section "Why compression may also improve speed");
  *  - oh-bug.com "KV Cache Quantization in Practice": keys per channel, values
  *    per token (the KIVI paragraph), asymmetric 2-bit (the list under
- *    "4-bit / 3-bit / 2-bit").
+ *    "4-bit / 3-bit / 2-bit"), the FP8 engineering baseline with per-head
+ *    scales ("FP8 / INT8: Engineering Baseline", Step 3), and compatibility
+ *    with prefix caching and chunked prefill ("Go-Live Checklist").
+ * Besides the quantized formats the cache also holds the pages' unquantized
+ * BF16 baseline (bits = 16) on the same paged path, as a control.
  *
  * Conventions for every call:
  *  - Plain pointers and sizes only.  "device" pointers are CUDA global memory

@@ -27,9 +27,31 @@ namespace kvq {
 namespace {
 
 // ---------------------------------------------------------------------------
-__global__ void apply_kernel(const Geo g, const DevState d, const PlanView p) {
+// Table and length updates and zeroing of new partial blocks; with `kin`
+// given (a call that flushes no group and quantizes no token) it also copies
+// the new rows into the BF16 window, which saves the residual launch.
+__global__ void apply_kernel(const Geo g, const DevState d, const PlanView p, const uint16_t* kin,
+                             const uint16_t* vin) {
   const int64_t tid = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t nthr = int64_t(gridDim.x) * blockDim.x;
+  if (kin) {
+    constexpr int D = kD;
+    const int64_t total = int64_t(p.n_res) * g.h_kv * 2 * (D / 8);
+    for (int64_t idx = tid; idx < total; idx += nthr) {
+      const int c8 = int(idx % (D / 8));
+      int64_t rest = idx / (D / 8);
+      const int which = int(rest % 2);
+      rest /= 2;
+      const int h = int(rest % g.h_kv);
+      const int e = int(rest / g.h_kv);
+      const int32_t src = p.plan[p.off_res + 3 * e];
+      const int32_t seq = p.plan[p.off_res + 3 * e + 1];
+      const int32_t slot = p.plan[p.off_res + 3 * e + 2];
+      const uint16_t* s = (which ? vin : kin) + (int64_t(src) * g.h_kv + h) * D;
+      uint16_t* dst = (which ? d.vres : d.kres) + ((int64_t(seq) * g.h_kv + h) * g.R + slot) * D;
+      reinterpret_cast<uint4*>(dst)[c8] = reinterpret_cast<const uint4*>(s)[c8];
+    }
+  }
   // zero whole blocks (16-byte stores)
   const int64_t per_block = g.block_bytes / 16;
   const int64_t zero_items = int64_t(p.n_zero) * per_block;
@@ -416,13 +438,13 @@ size_t flush_smem_bytes(const Geo& g) {
 
 }  // namespace
 
-cudaError_t launch_apply(const Geo& g, const DevState& d, const PlanView& p, cudaStream_t s,
-                         int* launches) {
-  const int64_t work = std::max<int64_t>(int64_t(p.n_zero) * (g.block_bytes / 16),
-                                         std::max(p.n_tab, p.n_len));
+cudaError_t launch_apply(const Geo& g, const DevState& d, const PlanView& p, const uint16_t* k,
+                         const uint16_t* v, cudaStream_t s, int* launches) {
+  int64_t work = std::max<int64_t>(int64_t(p.n_zero) * (g.block_bytes / 16), std::max(p.n_tab, p.n_len));
+  if (k) work = std::max<int64_t>(work, int64_t(p.n_res) * g.h_kv * 2 * (kD / 8));
   if (work == 0) return cudaSuccess;
   const int blocks = int(std::min<int64_t>((work + 255) / 256, 4096));
-  apply_kernel<<<blocks, 256, 0, s>>>(g, d, p);
+  apply_kernel<<<blocks, 256, 0, s>>>(g, d, p, k, v);
   ++*launches;
   return cudaGetLastError();
 }

@@ -425,6 +425,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
     if (row_changed && n < N) ri = rinfo(it.i);
   };
 
+  // four units forward at once when that stays inside one (row, head)
+  auto advance4 = [&](It& it, RowInfo& ri, int& n) {
+    if (it.k + kDecodeWarps < it.n) {
+      it.k += kDecodeWarps;
+      n += kDecodeWarps;
+      return;
+    }
+    for (int t = 0; t < kDecodeWarps; ++t) step(it, ri, n);
+  };
+
   // ---- staging: each warp fills its own two stages, two units ahead ---------
   // metadata rows of a 16-token sub-tile (none for FP8)
   const int vrow = F8 ? 0 : 16 * g.nvg * ES, krow = F8 ? 0 : 16 * g.nkg * ES;
@@ -1032,14 +1042,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
     ++issued;
   }
   if (SPW == 2 && K > 1) {
-    for (int t = 0; t < kDecodeWarps; ++t) step(iti, rii, ni);
+    advance4(iti, rii, ni);
     const int32_t b1 = load_blk(iti, rii);
     issue(iti, rii, b1, SPW * warp + 1);
     ++issued;
   }
   int32_t blk_next = 0;
   if (K > SPW) {
-    for (int t = 0; t < kDecodeWarps; ++t) step(iti, rii, ni);
+    advance4(iti, rii, ni);
     blk_next = load_blk(iti, rii);
   }
 
@@ -1048,6 +1058,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
   bool aborted = false;
   // leaves the walk iterator on unit `target`, recording every pair it passes
   auto walk_to = [&](int target) {
+    if (itc.k + (target - nc) < itc.n) {   // still inside the same (row, head): no boundary
+      itc.k += target - nc;
+      nc = target;
+      return;
+    }
     while (nc < target) {
       step(itc, ric, nc);
       const int pid = itc.i * g.h_kv + itc.h;
@@ -1126,7 +1141,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
       issue(iti, rii, blk_next, sidx);   // the stage just read takes unit k + SPW
       ++issued;
       if (k + SPW + 1 < K) {
-        for (int t = 0; t < kDecodeWarps; ++t) step(iti, rii, ni);
+        advance4(iti, rii, ni);
         blk_next = load_blk(iti, rii);
       }
     }

@@ -92,8 +92,10 @@ struct DecodeArgs {
 
 // Host-side launchers (defined in the .cu files).
 // Each launcher adds the number of kernels it launched to *launches.
-cudaError_t launch_apply(const Geo& g, const DevState& d, const PlanView& p, cudaStream_t s,
-                         int* launches);
+// Table, length and zeroing updates of a plan; given k and v it also copies
+// the plan's window rows (only for a plan with no flush and no token rows).
+cudaError_t launch_apply(const Geo& g, const DevState& d, const PlanView& p, const uint16_t* k,
+                         const uint16_t* v, cudaStream_t s, int* launches);
 cudaError_t launch_flush(const Geo& g, const DevState& d, const PlanView& p,
                          const uint16_t* k, const uint16_t* v, cudaStream_t s, int* launches);
 cudaError_t launch_residual(const Geo& g, const DevState& d, const PlanView& p,

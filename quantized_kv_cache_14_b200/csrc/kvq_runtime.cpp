@@ -270,10 +270,13 @@ kvq_status run_plan(kvq_handle h, const Plan& pl, const uint16_t* k, const uint1
   if (st != KVQ_OK) return st;
   pv.plan = h->d_plan;
   kvq::DevState d{h->d_pool, h->d_kres, h->d_vres, h->d_table, h->d_len, h->d_err, h->d_fp8};
-  KVQ_CUDA(kvq::launch_apply(h->geo, d, pv, stream, &h->launches));
+  // The window copy must follow a flush's reads of the window slots it
+  // replaces; with no flush (and no token rows) it rides in the apply launch.
+  const bool fused = k && pl.flush.empty() && pl.tok.empty();
+  KVQ_CUDA(kvq::launch_apply(h->geo, d, pv, fused ? k : nullptr, fused ? v : nullptr, stream, &h->launches));
   KVQ_CUDA(kvq::launch_quant_token(h->geo, d, pv, k, v, stream, &h->launches));
   KVQ_CUDA(kvq::launch_flush(h->geo, d, pv, k, v, stream, &h->launches));
-  KVQ_CUDA(kvq::launch_residual(h->geo, d, pv, k, v, stream, &h->launches));
+  if (!fused) KVQ_CUDA(kvq::launch_residual(h->geo, d, pv, k, v, stream, &h->launches));
   return KVQ_OK;
 }
 
