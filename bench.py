@@ -248,7 +248,6 @@ def run_gpu(args, rank, ws, dist):
     host_in = [tuple(torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
                      for a in s) for s in steps_in]
     del dr
-    seq_lens = torch.tensor(lens, dtype=torch.int32, device=dev)
     out = torch.empty((B, w.h_q, D), dtype=torch.float32, device=dev)
     out_host = torch.empty_like(out, device="cpu").pin_memory()
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
@@ -271,9 +270,8 @@ def run_gpu(args, rank, ws, dist):
             k, v, q = dev_in[s]
         cache.append(k, v, ids)
         lens = [L + 1 for L in lens]
-        seq_lens.add_(1)
         ev1.record()
-        cache.decode(q, seq_lens, out)
+        cache.decode(q, None, out)              # attends over the stored lengths
         if e2e:
             out_host.copy_(out, non_blocking=True)
         ev2.record()

@@ -26,14 +26,22 @@
 namespace kvq {
 namespace {
 
+// Every launch of this file fits the classic 4 KB kernel-parameter space.
+static_assert(sizeof(Geo) + sizeof(DevState) + sizeof(PlanView) + 3 * sizeof(void*) + 16 <= 4096,
+              "append kernel parameters exceed 4 KB");
+
+// The plan's entries: inline in the launch parameters or uploaded.
+__device__ __forceinline__ const int32_t* plan_of(const PlanView& p) { return p.plan ? p.plan : p.inl; }
+
 // ---------------------------------------------------------------------------
-// Table and length updates and zeroing of new partial blocks; with `kin`
-// given (a call that flushes no group and quantizes no token) it also copies
-// the new rows into the BF16 window, which saves the residual launch.
-__global__ void apply_kernel(const Geo g, const DevState d, const PlanView p, const uint16_t* kin,
-                             const uint16_t* vin) {
-  const int64_t tid = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t nthr = int64_t(gridDim.x) * blockDim.x;
+// Table and length updates and zeroing of new partial blocks, done by threads
+// tid, tid + nthr, ...; with `kin` given it also copies the plan's window rows
+// into the BF16 window (a call whose window writes touch no slot that a flush
+// of the same call reads).
+__device__ __forceinline__ void apply_body(const Geo& g, const DevState& d, const PlanView& p,
+                                           const uint16_t* kin, const uint16_t* vin, int64_t tid,
+                                           int64_t nthr) {
+  const int32_t* plan = plan_of(p);
   if (kin) {
     constexpr int D = kD;
     const int64_t total = int64_t(p.n_res) * g.h_kv * 2 * (D / 8);
@@ -44,9 +52,9 @@ __global__ void apply_kernel(const Geo g, const DevState d, const PlanView p, co
       rest /= 2;
       const int h = int(rest % g.h_kv);
       const int e = int(rest / g.h_kv);
-      const int32_t src = p.plan[p.off_res + 3 * e];
-      const int32_t seq = p.plan[p.off_res + 3 * e + 1];
-      const int32_t slot = p.plan[p.off_res + 3 * e + 2];
+      const int32_t src = plan[p.off_res + 3 * e];
+      const int32_t seq = plan[p.off_res + 3 * e + 1];
+      const int32_t slot = plan[p.off_res + 3 * e + 2];
       const uint16_t* s = (which ? vin : kin) + (int64_t(src) * g.h_kv + h) * D;
       uint16_t* dst = (which ? d.vres : d.kres) + ((int64_t(seq) * g.h_kv + h) * g.R + slot) * D;
       reinterpret_cast<uint4*>(dst)[c8] = reinterpret_cast<const uint4*>(s)[c8];
@@ -56,14 +64,25 @@ __global__ void apply_kernel(const Geo g, const DevState d, const PlanView p, co
   const int64_t per_block = g.block_bytes / 16;
   const int64_t zero_items = int64_t(p.n_zero) * per_block;
   for (int64_t i = tid; i < zero_items; i += nthr) {
-    const int32_t blk = p.plan[p.off_zero + i / per_block];
+    const int32_t blk = plan[p.off_zero + i / per_block];
     reinterpret_cast<uint4*>(d.pool + int64_t(blk) * g.block_bytes)[i % per_block] =
         make_uint4(0, 0, 0, 0);
   }
-  for (int64_t i = tid; i < p.n_tab; i += nthr)
-    d.table[p.plan[p.off_tab + 2 * i]] = p.plan[p.off_tab + 2 * i + 1];
-  for (int64_t i = tid; i < p.n_len; i += nthr)
-    d.len[p.plan[p.off_len + 2 * i]] = p.plan[p.off_len + 2 * i + 1];
+  for (int64_t i = tid; i < p.n_tab; i += nthr) d.table[plan[p.off_tab + 2 * i]] = plan[p.off_tab + 2 * i + 1];
+  for (int64_t i = tid; i < p.n_len; i += nthr) d.len[plan[p.off_len + 2 * i]] = plan[p.off_len + 2 * i + 1];
+}
+
+// Threads an apply body needs for a plan (window rows copied or not).
+inline int64_t apply_work(const Geo& g, const PlanView& p, bool copy_rows) {
+  int64_t work = std::max<int64_t>(int64_t(p.n_zero) * (g.block_bytes / 16), std::max(p.n_tab, p.n_len));
+  if (copy_rows) work = std::max<int64_t>(work, int64_t(p.n_res) * g.h_kv * 2 * (kD / 8));
+  return work;
+}
+
+__global__ void apply_kernel(const Geo g, const DevState d, const __grid_constant__ PlanView p,
+                             const uint16_t* kin, const uint16_t* vin) {
+  apply_body(g, d, p, kin, vin, int64_t(blockIdx.x) * blockDim.x + threadIdx.x,
+             int64_t(gridDim.x) * blockDim.x);
 }
 
 // ---------------------------------------------------------------------------
@@ -71,7 +90,7 @@ __global__ void apply_kernel(const Geo g, const DevState d, const PlanView p, co
 // 4l .. 4l+3.
 template <int BITS, int ASYM>
 __global__ void __launch_bounds__(256) quant_token_kernel(const Geo g, const DevState d,
-                                                          const PlanView p, const uint16_t* kin,
+                                                          const __grid_constant__ PlanView p, const uint16_t* kin,
                                                           const uint16_t* vin) {
   constexpr int D = kD;
   constexpr int N = 32 / BITS;                 // codes per word
@@ -81,9 +100,9 @@ __global__ void __launch_bounds__(256) quant_token_kernel(const Geo g, const Dev
   const int64_t item = int64_t(blockIdx.x) * 8 + wib;
   if (item >= int64_t(p.n_tok) * g.h_kv) return;
   const int e = int(item / g.h_kv), h = int(item % g.h_kv);
-  const int32_t src = p.plan[p.off_tok + 3 * e];
-  const int32_t blk = p.plan[p.off_tok + 3 * e + 1];
-  const int32_t tok = p.plan[p.off_tok + 3 * e + 2];
+  const int32_t src = plan_of(p)[p.off_tok + 3 * e];
+  const int32_t blk = plan_of(p)[p.off_tok + 3 * e + 1];
+  const int32_t tok = plan_of(p)[p.off_tok + 3 * e + 2];
   uint8_t* chunk = d.pool + int64_t(blk) * g.block_bytes + int64_t(h) * g.chunk_bytes;
   const int sub = tok >> 4, r = tok & 15;
 
@@ -176,12 +195,21 @@ __global__ void __launch_bounds__(256) quant_token_kernel(const Geo g, const Dev
 // Every CTA gathers the group's R key rows and computes all channel scales
 // (they need every row), then writes only its own sub-tile's key and value
 // codes, value scales, and -- when its sub-tile starts a page -- that page's
-// slice of the key scales.
+// slice of the key scales.  CTAs with blockIdx.x >= n_flush run the plan's
+// apply body instead (with the window copy when `fuse_rows` is set), so a
+// decode-sized append is one launch.
 template <int BITS, int ASYM>
 __global__ void __launch_bounds__(kFlushThreads) flush_kernel(const Geo g, const DevState d,
-                                                              const PlanView p,
+                                                              const __grid_constant__ PlanView p,
                                                               const uint16_t* kin,
-                                                              const uint16_t* vin) {
+                                                              const uint16_t* vin, int fuse_rows) {
+  if (int(blockIdx.x) >= p.n_flush) {
+    const int64_t cta =
+        (int64_t(blockIdx.x - p.n_flush) * gridDim.y + blockIdx.y) * gridDim.z + blockIdx.z;
+    const int64_t ctas = int64_t(gridDim.x - p.n_flush) * gridDim.y * gridDim.z;
+    apply_body(g, d, p, fuse_rows ? kin : nullptr, vin, cta * blockDim.x + threadIdx.x, ctas * blockDim.x);
+    return;
+  }
   constexpr int D = kD;
   constexpr int N = 32 / BITS;
   constexpr int Q = ASYM ? (1 << BITS) - 1 : (1 << (BITS - 1)) - 1;
@@ -196,10 +224,10 @@ __global__ void __launch_bounds__(kFlushThreads) flush_kernel(const Geo g, const
 
   const int e = blockIdx.x, h = blockIdx.y, zs = blockIdx.z, tid = threadIdx.x;
   const int r_lo = 16 * zs;   // this CTA's rows [r_lo, r_lo + 16)
-  const int32_t* ent = p.plan + p.off_flush + e * kFlushEntryInts;
+  const int32_t* ent = plan_of(p) + p.off_flush + e * kFlushEntryInts;
   const int seq = ent[0];
   const int npg = ent[2];
-  const int32_t* srcs = p.plan + p.off_src + int64_t(e) * R;
+  const int32_t* srcs = plan_of(p) + p.off_src + int64_t(e) * R;
 
   // 1. gather the group's K rows and this sub-tile's V rows (bf16) into
   //    shared memory
@@ -343,7 +371,7 @@ __global__ void __launch_bounds__(kFlushThreads) flush_kernel(const Geo g, const
 }
 
 // ---------------------------------------------------------------------------
-__global__ void residual_kernel(const Geo g, const DevState d, const PlanView p,
+__global__ void residual_kernel(const Geo g, const DevState d, const __grid_constant__ PlanView p,
                                 const uint16_t* kin, const uint16_t* vin) {
   constexpr int D = kD;
   const int64_t total = int64_t(p.n_res) * g.h_kv * 2 * (D / 8);
@@ -355,9 +383,9 @@ __global__ void residual_kernel(const Geo g, const DevState d, const PlanView p,
     rest /= 2;
     const int h = int(rest % g.h_kv);
     const int e = int(rest / g.h_kv);
-    const int32_t src = p.plan[p.off_res + 3 * e];
-    const int32_t seq = p.plan[p.off_res + 3 * e + 1];
-    const int32_t slot = p.plan[p.off_res + 3 * e + 2];
+    const int32_t src = plan_of(p)[p.off_res + 3 * e];
+    const int32_t seq = plan_of(p)[p.off_res + 3 * e + 1];
+    const int32_t slot = plan_of(p)[p.off_res + 3 * e + 2];
     const uint16_t* s = (which ? vin : kin) + (int64_t(src) * g.h_kv + h) * D;
     uint16_t* dst = (which ? d.vres : d.kres) + ((int64_t(seq) * g.h_kv + h) * g.R + slot) * D;
     reinterpret_cast<uint4*>(dst)[c8] = reinterpret_cast<const uint4*>(s)[c8];
@@ -367,16 +395,17 @@ __global__ void residual_kernel(const Geo g, const DevState d, const PlanView p,
 // BF16 control: the token's key and value rows of each head go unchanged into
 // their page as natural bf16 rows (row r of sub-tile r / 16).  One warp per
 // (token, head); lane l copies channels 4l .. 4l+3.
-__global__ void __launch_bounds__(256) copy_token_kernel(const Geo g, const DevState d, const PlanView p,
+__global__ void __launch_bounds__(256) copy_token_kernel(const Geo g, const DevState d,
+                                                         const __grid_constant__ PlanView p,
                                                          const uint16_t* kin, const uint16_t* vin) {
   constexpr int D = kD;
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int64_t item = int64_t(blockIdx.x) * 8 + wib;
   if (item >= int64_t(p.n_tok) * g.h_kv) return;
   const int e = int(item / g.h_kv), h = int(item % g.h_kv);
-  const int32_t src = p.plan[p.off_tok + 3 * e];
-  const int32_t blk = p.plan[p.off_tok + 3 * e + 1];
-  const int32_t tok = p.plan[p.off_tok + 3 * e + 2];
+  const int32_t src = plan_of(p)[p.off_tok + 3 * e];
+  const int32_t blk = plan_of(p)[p.off_tok + 3 * e + 1];
+  const int32_t tok = plan_of(p)[p.off_tok + 3 * e + 2];
   uint8_t* chunk = d.pool + int64_t(blk) * g.block_bytes + int64_t(h) * g.chunk_bytes;
   const int64_t row = int64_t(tok >> 4) * g.sub_bytes + (tok & 15) * (D * 2);
   const int64_t in = (int64_t(src) * g.h_kv + h) * D + 4 * lane;
@@ -390,16 +419,17 @@ __global__ void __launch_bounds__(256) copy_token_kernel(const Geo g, const DevS
 // where operand register x of tile i holds its two tokens in bytes 2x, 2x + 1
 // of word 2i + x / 2.  One warp per (token, head); each lane writes one key
 // word and four value bytes.
-__global__ void __launch_bounds__(256) fp8_token_kernel(const Geo g, const DevState d, const PlanView p,
+__global__ void __launch_bounds__(256) fp8_token_kernel(const Geo g, const DevState d,
+                                                        const __grid_constant__ PlanView p,
                                                         const uint16_t* kin, const uint16_t* vin) {
   constexpr int D = kD;
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int64_t item = int64_t(blockIdx.x) * 8 + wib;
   if (item >= int64_t(p.n_tok) * g.h_kv) return;
   const int e = int(item / g.h_kv), h = int(item % g.h_kv);
-  const int32_t src = p.plan[p.off_tok + 3 * e];
-  const int32_t blk = p.plan[p.off_tok + 3 * e + 1];
-  const int32_t tok = p.plan[p.off_tok + 3 * e + 2];
+  const int32_t src = plan_of(p)[p.off_tok + 3 * e];
+  const int32_t blk = plan_of(p)[p.off_tok + 3 * e + 1];
+  const int32_t tok = plan_of(p)[p.off_tok + 3 * e + 2];
   uint8_t* chunk = d.pool + int64_t(blk) * g.block_bytes + int64_t(h) * g.chunk_bytes;
   const int sub = tok >> 4, r = tok & 15;
   const float sk = d.fp8[h], sv = d.fp8[g.h_kv + h];
@@ -440,8 +470,7 @@ size_t flush_smem_bytes(const Geo& g) {
 
 cudaError_t launch_apply(const Geo& g, const DevState& d, const PlanView& p, const uint16_t* k,
                          const uint16_t* v, cudaStream_t s, int* launches) {
-  int64_t work = std::max<int64_t>(int64_t(p.n_zero) * (g.block_bytes / 16), std::max(p.n_tab, p.n_len));
-  if (k) work = std::max<int64_t>(work, int64_t(p.n_res) * g.h_kv * 2 * (kD / 8));
+  const int64_t work = apply_work(g, p, k != nullptr);
   if (work == 0) return cudaSuccess;
   const int blocks = int(std::min<int64_t>((work + 255) / 256, 4096));
   apply_kernel<<<blocks, 256, 0, s>>>(g, d, p, k, v);
@@ -472,9 +501,13 @@ cudaError_t launch_quant_token(const Geo& g, const DevState& d, const PlanView& 
 }
 
 cudaError_t launch_flush(const Geo& g, const DevState& d, const PlanView& p, const uint16_t* k,
-                         const uint16_t* v, cudaStream_t s, int* launches) {
+                         const uint16_t* v, bool with_apply, bool fuse_rows, cudaStream_t s, int* launches) {
   if (p.n_flush == 0) return cudaSuccess;
   const size_t smem = flush_smem_bytes(g);
+  // extra columns of (h_kv x R/16) CTAs for the apply body
+  const int64_t per_col = int64_t(g.h_kv) * (g.R / 16) * kFlushThreads;
+  const int64_t work = with_apply ? apply_work(g, p, fuse_rows) : 0;
+  const int extra = int(std::min<int64_t>((work + per_col - 1) / per_col, 64));
   return by_format(g, [&](auto B, auto A) {
     auto kern = flush_kernel<decltype(B)::value, decltype(A)::value>;
     // the shared-memory limit only grows: set it once per kernel, device and size
@@ -487,7 +520,8 @@ cudaError_t launch_flush(const Geo& g, const DevState& d, const PlanView& p, con
       if (e != cudaSuccess) return e;
       if (dev < 32) limit_set[dev] = smem;
     }
-    kern<<<dim3(p.n_flush, g.h_kv, g.R / 16), kFlushThreads, smem, s>>>(g, d, p, k, v);
+    kern<<<dim3(p.n_flush + extra, g.h_kv, g.R / 16), kFlushThreads, smem, s>>>(g, d, p, k, v,
+                                                                              fuse_rows ? 1 : 0);
     ++*launches;
     return cudaGetLastError();
   });

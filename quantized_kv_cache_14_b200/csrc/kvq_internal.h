@@ -40,11 +40,16 @@ struct Geo {
   int qtile_bytes;          // bytes staged for one quantized tile
 };
 
-// Device view of an append plan: one int32 array with sections.
+// Device view of an append plan: one int32 array with sections.  A plan of
+// at most kPlanInline entries travels inside the launch parameters (`inl`,
+// `plan` null), so a decode-sized append needs no host-to-device copy; a
+// larger one is uploaded first and read through `plan`.
+constexpr int kPlanInline = 880;
 struct PlanView {
   const int32_t* plan;
   int n_tok, n_flush, n_res, n_tab, n_len, n_zero;
   int off_tok, off_flush, off_src, off_res, off_tab, off_len, off_zero;
+  int32_t inl[kPlanInline];
 };
 
 struct DevState {
@@ -93,11 +98,15 @@ struct DecodeArgs {
 // Host-side launchers (defined in the .cu files).
 // Each launcher adds the number of kernels it launched to *launches.
 // Table, length and zeroing updates of a plan; given k and v it also copies
-// the plan's window rows (only for a plan with no flush and no token rows).
+// the plan's window rows (only for a plan with no token rows whose flushes,
+// if any, read none of the slots those rows fill).
 cudaError_t launch_apply(const Geo& g, const DevState& d, const PlanView& p, const uint16_t* k,
                          const uint16_t* v, cudaStream_t s, int* launches);
+// Flush launch; with `with_apply` it also runs the plan's apply body (and the
+// window rows when `fuse_rows` is set) in extra CTAs of the same launch.
 cudaError_t launch_flush(const Geo& g, const DevState& d, const PlanView& p,
-                         const uint16_t* k, const uint16_t* v, cudaStream_t s, int* launches);
+                         const uint16_t* k, const uint16_t* v, bool with_apply, bool fuse_rows,
+                         cudaStream_t s, int* launches);
 cudaError_t launch_residual(const Geo& g, const DevState& d, const PlanView& p,
                             const uint16_t* k, const uint16_t* v, cudaStream_t s, int* launches);
 cudaError_t launch_quant_token(const Geo& g, const DevState& d, const PlanView& p,

@@ -12,6 +12,7 @@
 #include <cstring>
 #include <deque>
 #include <string>
+#include <unordered_set>
 #include <vector>
 
 #include <cuda_runtime.h>
@@ -260,23 +261,53 @@ kvq_status run_plan(kvq_handle h, const Plan& pl, const uint16_t* k, const uint1
   pv.off_len = int(off); off += pl.lens.size();
   pv.off_zero = int(off); off += pl.zero.size();
   if (off == 0) return KVQ_OK;
-  std::vector<int32_t> flat;
-  flat.reserve(off);
-  for (const auto* sec : {&pl.tok, &pl.flush, &pl.src, &pl.res, &pl.tab, &pl.lens, &pl.zero})
-    flat.insert(flat.end(), sec->begin(), sec->end());
-  kvq_status st = ensure_plan_capacity(h, off);
-  if (st != KVQ_OK) return st;
-  st = stage_upload(h, flat.data(), off, h->d_plan, stream);
-  if (st != KVQ_OK) return st;
-  pv.plan = h->d_plan;
+  if (off <= size_t(kvq::kPlanInline)) {
+    // small plans ride in the launch parameters: no upload on the stream
+    int32_t* o = pv.inl;
+    for (const auto* sec : {&pl.tok, &pl.flush, &pl.src, &pl.res, &pl.tab, &pl.lens, &pl.zero})
+      o = std::copy(sec->begin(), sec->end(), o);
+    pv.plan = nullptr;
+  } else {
+    std::vector<int32_t> flat;
+    flat.reserve(off);
+    for (const auto* sec : {&pl.tok, &pl.flush, &pl.src, &pl.res, &pl.tab, &pl.lens, &pl.zero})
+      flat.insert(flat.end(), sec->begin(), sec->end());
+    kvq_status st = ensure_plan_capacity(h, off);
+    if (st != KVQ_OK) return st;
+    st = stage_upload(h, flat.data(), off, h->d_plan, stream);
+    if (st != KVQ_OK) return st;
+    pv.plan = h->d_plan;
+  }
   kvq::DevState d{h->d_pool, h->d_kres, h->d_vres, h->d_table, h->d_len, h->d_err, h->d_fp8};
-  // The window copy must follow a flush's reads of the window slots it
-  // replaces; with no flush (and no token rows) it rides in the apply launch.
-  const bool fused = k && pl.flush.empty() && pl.tok.empty();
-  KVQ_CUDA(kvq::launch_apply(h->geo, d, pv, fused ? k : nullptr, fused ? v : nullptr, stream, &h->launches));
-  KVQ_CUDA(kvq::launch_quant_token(h->geo, d, pv, k, v, stream, &h->launches));
-  KVQ_CUDA(kvq::launch_flush(h->geo, d, pv, k, v, stream, &h->launches));
-  if (!fused) KVQ_CUDA(kvq::launch_residual(h->geo, d, pv, k, v, stream, &h->launches));
+  // The window rows go into the first launch unless one of them would land in
+  // a window slot that a flush of this call still reads (a multi-token append
+  // that completes a group and leaves tokens behind); token rows keep their
+  // own order (zeroing first).
+  const bool tok = !pl.tok.empty(), flush = !pl.flush.empty();
+  bool rows_in = k && !tok;
+  if (rows_in && flush && !pl.res.empty()) {
+    const int R = h->geo.R;
+    std::unordered_set<int64_t> reads;
+    for (int e = 0; e < pv.n_flush; ++e) {
+      const int64_t seq = pl.flush[size_t(e) * kvq::kFlushEntryInts];
+      for (int r = 0; r < R; ++r) {
+        const int32_t src = pl.src[size_t(e) * R + r];
+        if (src < 0) reads.insert(seq * R + (-1 - src));
+      }
+    }
+    for (size_t i = 0; i + 2 < pl.res.size() && rows_in; i += 3)
+      if (reads.count(int64_t(pl.res[i + 1]) * R + pl.res[i + 2])) rows_in = false;
+  }
+  if (flush && !tok) {
+    // one launch: flush CTAs plus apply CTAs (tables, lengths, window rows)
+    KVQ_CUDA(kvq::launch_flush(h->geo, d, pv, k, v, true, rows_in, stream, &h->launches));
+  } else {
+    KVQ_CUDA(kvq::launch_apply(h->geo, d, pv, rows_in ? k : nullptr, rows_in ? v : nullptr, stream,
+                               &h->launches));
+    KVQ_CUDA(kvq::launch_quant_token(h->geo, d, pv, k, v, stream, &h->launches));
+    KVQ_CUDA(kvq::launch_flush(h->geo, d, pv, k, v, false, false, stream, &h->launches));
+  }
+  if (!rows_in) KVQ_CUDA(kvq::launch_residual(h->geo, d, pv, k, v, stream, &h->launches));
   return KVQ_OK;
 }
 

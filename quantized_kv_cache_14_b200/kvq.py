@@ -338,10 +338,19 @@ class KVCache:
         kvq_append(self.h, kp, vp, ids, n, 0 if self.cfg.host_only else self._stream(stream))
 
     def decode(self, q, seq_lens, out, block_table=None, bt_stride=0, seq_ids=None, stream=None):
-        """q: CUDA bf16 [B, h_q, d_h]; seq_lens: CUDA int32 [B]; out: CUDA fp32 [B, h_q, d_h]."""
+        """q: CUDA bf16 [B, h_q, d_h]; seq_lens: CUDA int32 [B], or None to attend
+        over every stored token of sequences 0..B-1 (the library's own device
+        lengths, so no length update is needed between appends and decodes);
+        out: CUDA fp32 [B, h_q, d_h]."""
         B = int(q.shape[0])
         bt = block_table.data_ptr() if block_table is not None else 0
-        kvq_decode_attn(self.h, q.data_ptr(), bt, bt_stride, seq_lens.data_ptr(), seq_ids, B,
+        if seq_lens is None:
+            if seq_ids is not None or block_table is not None:
+                raise ValueError("seq_lens=None needs rows 0..B-1 to be sequences 0..B-1")
+            sl = kvq_seq_lens_device(self.h)
+        else:
+            sl = seq_lens.data_ptr()
+        kvq_decode_attn(self.h, q.data_ptr(), bt, bt_stride, sl, seq_ids, B,
                         out.data_ptr(), self._stream(stream))
 
     def seq_len(self, s):

@@ -90,6 +90,46 @@ def test_incremental_appends_interleaved(name):
     p.close()
 
 
+@pytest.mark.parametrize("name", ["int4_chan64", "int2_asym_chan32", "int4_chan16", "int8_asym_chan128_p64"])
+def test_append_launch_shapes(name):
+    """The append's launch shapes give the oracle's bytes: decode steps where
+    some sequences complete a key group (flush and window rows in one launch,
+    plan in the launch parameters), a multi-token append that completes a
+    group and leaves tokens of the same sequence behind (window rows after the
+    flush), and a bulk append whose plan is uploaded.  Decode over the
+    library's own stored lengths equals decode over explicit lengths."""
+    rng = np.random.default_rng(11)
+    R = FMTS[name]["residual"]
+    h_q, h_kv, S = 8, 2, 4
+    p = Pair(FMTS[name], h_q, h_kv, max_seqs=S, num_blocks=400, mbps=128, seed=2)
+    # bulk (plan uploaded): lengths R-2, R-1, 2R-1, 3
+    lens = [R - 2, R - 1, 2 * R - 1, 3]
+    ids = np.repeat(np.arange(S, dtype=np.int32), lens)
+    p.append(outlier_keys(rng, ids.size, h_kv), random_bf16(rng, (ids.size, h_kv, D)), ids)
+    p.check_state()
+    # decode steps: one token per sequence; sequences 1 and 2 flush at once
+    for _ in range(3):
+        ids = np.arange(S, dtype=np.int32)
+        p.append(outlier_keys(rng, S, h_kv), random_bf16(rng, (S, h_kv, D)), ids)
+        lens = [L + 1 for L in lens]
+        p.check_state()
+    # sequence 0 completes its group and keeps 5 tokens in one call; sequence 3 gains 2
+    ids = np.array([0] * (R - lens[0] % R + 5) + [3, 3], dtype=np.int32)
+    p.append(outlier_keys(rng, ids.size, h_kv), random_bf16(rng, (ids.size, h_kv, D)), ids)
+    lens[0] += R - lens[0] % R + 5
+    lens[3] += 2
+    p.check_state()
+    q = random_bf16(rng, (S, h_q, D))
+    got, want = p.decode(q, lens)
+    assert np.max(np.abs(got - want)) <= ATOL
+    out = torch.full((S, h_q, D), float("nan"), dtype=torch.float32, device="cuda")
+    p.gpu.decode(bits_to_cuda_bf16(q), None, out)
+    torch.cuda.synchronize()
+    assert p.gpu.sync_status() == 0
+    assert np.array_equal(out.cpu().numpy(), got.astype(np.float32))
+    p.close()
+
+
 @pytest.mark.parametrize("name", ["int4_chan64", "int8_tok_p16", "int2_asym_chan32", "bf16_control_p16", "fp8_p16"])
 def test_split_k_merge_is_invariant_to_grid(name):
     rng = np.random.default_rng(3)
