@@ -11,8 +11,9 @@ divided by the max over ranks.  Inputs live in HBM before the timed region; L2
 is flushed before every timed step (untimed): a 256 MB write, then a read of
 another 256 MB so that the write's dirty lines are written back before the
 timed region and the timed kernels start on a cold, clean L2.  `e2e` is the same
-metric through the C ABI with host buffers: pinned H2D of the step's new K/V
-and q and D2H of the attention output inside the timed region.  With N > 1 every
+metric through the C ABI with host buffers: one kvq_step_host call per step
+(pinned H2D of the step's new K/V and q, append, decode, D2H of the attention
+output) inside the timed region, synchronised every step.  With N > 1 every
 rank runs its own replica (sequences shard across GPUs; no collective is on the
 data path; the only collectives are the barrier and the max-over-ranks timing).
 `--impl reference` times the CPU oracle (test infrastructure) on a bounded
@@ -261,19 +262,19 @@ def run_gpu(args, rank, ws, dist):
         flush.zero_()                                   # untimed: evicts L2 ...
         flush_rd.sum()                                  # ... and writes the dirty lines back
         ev0.record()
-        if e2e:
-            kh, vh, qh = host_in[s]
-            k = kh.to(dev, non_blocking=True)
-            v = vh.to(dev, non_blocking=True)
-            q = qh.to(dev, non_blocking=True)
-        else:
-            k, v, q = dev_in[s]
-        cache.append(k, v, ids)
         lens = [L + 1 for L in lens]
+        if e2e:
+            # one C-ABI call from pinned host buffers: H2D of k, v, q, append,
+            # decode over the stored lengths, D2H of the output
+            kh, vh, qh = host_in[s]
+            cache.step_host(kh, vh, ids, qh, out_host)
+            ev1.record()
+            ev2.record()
+            return
+        k, v, q = dev_in[s]
+        cache.append(k, v, ids)
         ev1.record()
         cache.decode(q, None, out)              # attends over the stored lengths
-        if e2e:
-            out_host.copy_(out, non_blocking=True)
         ev2.record()
 
     # warm-up
@@ -437,6 +438,103 @@ def run_control(args):
             "speedup_fp8_over_bf16": out["bf16"]["decode_us"] / out["fp8"]["decode_us"]}
 
 
+def _timed_calls(fn, K, flush, flush_rd):
+    """Median device time (µs) of fn() over K calls after 3 warm-up calls,
+    with a clean L2 flush before each."""
+    import torch
+    evs = []
+    for it in range(K + 3):
+        flush.zero_()
+        flush_rd.sum()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        if it >= 3:
+            evs.append((e0, e1))
+    torch.cuda.synchronize()
+    return float(np.median([a.elapsed_time(b) for a, b in evs])) * 1e3
+
+
+def run_next_rows(args):
+    """The widened rows on the workload's format:
+    prefix sharing -- 16 sequences over one 8192-token prefix (whole key
+    groups) plus 64 tokens of their own, the prefix held once through
+    kvq_share_prefix, against 16 unshared copies of the same tokens: pool
+    blocks and decode time (outputs must agree bit for bit);
+    chunked prefill -- one sequence with an 8192-token context and a new chunk
+    of 256 tokens, each chunk token attending its causal prefix through
+    kvq_prefill_attn: time per chunk and query tokens per second."""
+    import torch
+    from quantized_kv_cache_14_b200 import kvq
+    from quantized_kv_cache_14_b200.workloads import random_bf16
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = workload(args.workload)
+    f = w.fmt
+    K = max(5, min(args.steps, 30))
+    rng = np.random.default_rng(w.seed + 77)
+    fmt = kvq.Format(f.bits, f.asym, f.k_axis, f.g_k, f.g_v, f.scale_fp32, f.residual, f.page, f.fp8)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_rd = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def dbf(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    B, Lp, Ls = w.batch, 8192, 64
+    kp, vp = random_bf16(rng, (Lp, w.h_kv, D)), random_bf16(rng, (Lp, w.h_kv, D))
+    ks, vs = random_bf16(rng, (B * Ls, w.h_kv, D)), random_bf16(rng, (B * Ls, w.h_kv, D))
+    sid = np.repeat(np.arange(B, dtype=np.int32), Ls)
+    q = dbf(random_bf16(rng, (B, w.h_q, D)))
+    lens = [Lp + Ls] * B
+    mbps = (Lp + Ls) // f.page + 4
+    share = {}
+    outs = {}
+    for tag in ("shared", "unshared"):
+        nb = (B if tag == "unshared" else 1) * (Lp // f.page) + B * (Ls // f.page + 2) + 64
+        c = kvq.KVCache(fmt, w.h_q, w.h_kv, max_seqs=B, num_blocks=nb, max_blocks_per_seq=mbps,
+                        seed=w.seed, device=torch.cuda.current_device())
+        if tag == "shared":
+            c.append(dbf(kp), dbf(vp), np.zeros(Lp, np.int32))
+            for s in range(1, B):
+                c.share_prefix(0, s, Lp)
+        else:
+            c.append(dbf(np.tile(kp, (B, 1, 1))), dbf(np.tile(vp, (B, 1, 1))),
+                     np.repeat(np.arange(B, dtype=np.int32), Lp))
+        c.append(dbf(ks), dbf(vs), sid)
+        o = torch.empty((B, w.h_q, D), dtype=torch.float32, device=dev)
+        us = _timed_calls(lambda: c.decode(q, None, o), K, flush, flush_rd)
+        assert c.sync_status() == 0
+        outs[tag] = o.cpu()
+        st = c.stats()
+        share[tag] = {"decode_us": us, "blocks_used": int(st["blocks_used"]),
+                      "pool_bytes_used": int(st["blocks_used"]) * c.layout["block_bytes"]}
+        c.close()
+    share["outputs_equal"] = bool(torch.equal(outs["shared"], outs["unshared"]))
+    share["memory_ratio"] = share["unshared"]["blocks_used"] / share["shared"]["blocks_used"]
+    share["speedup"] = share["unshared"]["decode_us"] / share["shared"]["decode_us"]
+    share["workload"] = f"{B} sequences x ({Lp} shared + {Ls} own) tokens"
+
+    Lc, C = 8192, 256
+    c = kvq.KVCache(fmt, w.h_q, w.h_kv, max_seqs=C, num_blocks=(Lc + C) // f.page + 64,
+                    max_blocks_per_seq=(Lc + C) // f.page + 4, seed=w.seed, device=torch.cuda.current_device())
+    c.append(dbf(random_bf16(rng, (Lc + C, w.h_kv, D))), dbf(random_bf16(rng, (Lc + C, w.h_kv, D))),
+             np.zeros(Lc + C, np.int32))
+    qc = dbf(random_bf16(rng, (C, w.h_q, D)))
+    oc = torch.empty((C, w.h_q, D), dtype=torch.float32, device=dev)
+    ids = np.zeros(C, np.int32)
+    pos = np.arange(Lc, Lc + C, dtype=np.int32)
+    us = _timed_calls(lambda: c.prefill_attn(qc, ids, pos, oc), K, flush, flush_rd)
+    assert c.sync_status() == 0
+    c.close()
+    row_bytes = decode_bytes(w, [int(p) + 1 for p in pos])
+    prefill = {"workload": f"one sequence, {Lc}-token context, chunk of {C} new tokens",
+               "chunk_us": us, "query_tokens_per_s": C / (us * 1e-6),
+               "row_bytes": row_bytes, "row_gbs": row_bytes / (us * 1e-6) / 1e9,
+               "note": "each chunk token is a decode row over its own causal prefix (rows re-read "
+                       "the shared context, mostly from L2)"}
+    return {"calls": K, "prefix_sharing": share, "chunked_prefill": prefill}
+
+
 # ---------------------------------------------------------------------------
 # the CPU oracle (baseline / reference arm)
 # ---------------------------------------------------------------------------
@@ -504,7 +602,7 @@ def main():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=0, help="rows of the CPU oracle sample")
-    ap.add_argument("--no-control", action="store_true", help="skip the BF16 control comparison")
+    ap.add_argument("--no-control", action="store_true", help="skip the BF16 / FP8 comparison and the prefix-sharing and chunked-prefill measurements")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -545,6 +643,7 @@ def main():
                          f"{secs:.1f} s timed"}
     traffic = committed_traffic(w.name, res["attn_bytes_per_launch"])
     control = run_control(args) if (ws == 1 and not args.no_control) else None
+    next_rows = run_next_rows(args) if (ws == 1 and not args.no_control) else None
     line = {
         "metric": "decode-attn KV GB/s", "value": res["kv_gbs"], "unit": "GB/s",
         "n_gpus": ws, "steps": res["K"], "warmup": args.warmup,
@@ -566,6 +665,7 @@ def main():
         "frac_of_8TBps": res["kv_gbs"] / 8000.0,
         "frac_of_peak": res["kv_gbs"] / peak,
         "bf16_control": control,
+        "next_rows": next_rows,
     }
     print(json.dumps(line))
     if dist is not None:

@@ -205,6 +205,26 @@ kvq_status kvq_decode_attn(kvq_handle h, const void* q_bf16,
                            const int32_t* seq_lens, const int32_t* seq_ids_host,
                            int32_t batch, float* out, void* stream);
 
+/* One decode step from host memory, all enqueued on `stream`:
+ *   1. the n new rows k_host, v_host (host bf16 [n][h_kv][d_h]) go to
+ *      library-owned device buffers and are appended to sequences
+ *      seq_ids_host[i] exactly as kvq_append does;
+ *   2. q_host (host bf16 [batch][h_q][d_h]) goes to the device and row i
+ *      attends over every stored token of sequence i (kvq_decode_attn with the
+ *      library's own lengths, rows 0..batch-1 = sequences 0..batch-1);
+ *   3. the output comes back to out_host (host fp32 [batch][h_q][d_h]).
+ * out_host holds the result once the stream reaches that point.  Page-locked
+ * host buffers let the copies run asynchronously; pageable ones work with the
+ * copy semantics CUDA gives them.  n = 0 skips the append, batch = 0 the decode.
+ * The device buffers grow on demand (a device synchronize, then a reallocation)
+ * and live until kvq_destroy; the host buffers stay the caller's and must
+ * stay valid until the stream has reached the end of the step.
+ * Errors: KVQ_ERR_INVALID_ARG, KVQ_ERR_BAD_SEQ (nothing enqueued), those of
+ * kvq_append (state unchanged) and KVQ_ERR_CUDA. */
+kvq_status kvq_step_host(kvq_handle h, const void* k_host, const void* v_host,
+                         const int32_t* seq_ids_host, int32_t n, const void* q_host,
+                         int32_t batch, float* out_host, void* stream);
+
 /* Library-owned device block table: int32 [max_seqs][*stride], entry
  * [s][j] = physical block of logical block j of sequence s, -1 if none.
  * Valid until kvq_destroy; updated by appends in stream order. */

@@ -190,6 +190,13 @@ struct kvq_handle_s {
   size_t bytes_workspace = 0;
   cudaEvent_t decode_event = nullptr;
   int launches = 0;
+  // device staging of kvq_step_host: new K/V rows, q, output (grown on demand)
+  uint16_t* d_kin = nullptr;
+  uint16_t* d_vin = nullptr;
+  uint16_t* d_qin = nullptr;
+  float* d_out = nullptr;
+  int32_t io_rows = 0;    // K/V rows the staging holds
+  int32_t io_batch = 0;   // q / output rows the staging holds
 };
 
 namespace {
@@ -327,6 +334,10 @@ void destroy_device(kvq_handle h) {
   cudaFree(h->d_seqmap);
   cudaFree(h->d_rowlen);
   cudaFree(h->d_fp8);
+  cudaFree(h->d_kin);
+  cudaFree(h->d_vin);
+  cudaFree(h->d_qin);
+  cudaFree(h->d_out);
   for (auto& s : h->slots) {
     if (s.host) cudaFreeHost(s.host);
     if (s.ev) cudaEventDestroy(s.ev);
@@ -490,8 +501,13 @@ kvq_status kvq_append(kvq_handle h, const void* k_bf16, const void* v_bf16, cons
   std::vector<int32_t> first(h->len.begin(), h->len.end());   // length before the call
   std::vector<int32_t> cur(first);
   std::vector<int32_t> nblk(h->nblk);
-  std::vector<int32_t> tbl(h->table);                           // table after the call
+  // New table entries go straight into h->table (they were -1) and are
+  // listed here, so a failure below can put the -1 back; the planner never
+  // copies the whole table.
   std::vector<std::pair<int32_t, int32_t>> tab_changes;        // (index, block)
+  auto undo_table = [&]() {
+    for (const auto& tc : tab_changes) h->table[size_t(tc.first)] = -1;
+  };
   std::vector<std::vector<int32_t>> arrivals(static_cast<size_t>(S));  // input rows per sequence
   int64_t allocs = 0;
   auto take = [&]() { return h->freelist[size_t(allocs++)]; };  // front of the free list, in order
@@ -503,11 +519,11 @@ kvq_status kvq_append(kvq_handle h, const void* k_bf16, const void* v_bf16, cons
       if (lb == nblk[size_t(s)]) {
         const int32_t b = take();
         tab_changes.push_back({s * MB + lb, b});
-        tbl[size_t(s) * MB + lb] = b;
+        h->table[size_t(s) * MB + lb] = b;
         ++nblk[size_t(s)];
         if (newlen[size_t(s)] < int64_t(lb + 1) * P) pl.zero.push_back(b);
       }
-      pl.tok.insert(pl.tok.end(), {i, tbl[size_t(s) * MB + lb], pos % P});
+      pl.tok.insert(pl.tok.end(), {i, h->table[size_t(s) * MB + lb], pos % P});
     } else {
       arrivals[size_t(s)].push_back(i);
       if (pos % R == R - 1) {
@@ -516,7 +532,7 @@ kvq_status kvq_append(kvq_handle h, const void* k_bf16, const void* v_bf16, cons
         for (int j = 0; j < npg; ++j) {
           const int32_t b = take();
           tab_changes.push_back({s * MB + nblk[size_t(s)], b});
-          tbl[size_t(s) * MB + nblk[size_t(s)]] = b;
+          h->table[size_t(s) * MB + nblk[size_t(s)]] = b;
           ++nblk[size_t(s)];
           ent.push_back(b);
         }
@@ -545,13 +561,15 @@ kvq_status kvq_append(kvq_handle h, const void* k_bf16, const void* v_bf16, cons
 
   if (!c.host_only) {
     kvq_status st = device_guard(h);
-    if (st != KVQ_OK) return st;
-    st = run_plan(h, pl, static_cast<const uint16_t*>(k_bf16), static_cast<const uint16_t*>(v_bf16),
-                  static_cast<cudaStream_t>(stream_));
-    if (st != KVQ_OK) return st;
+    if (st == KVQ_OK)
+      st = run_plan(h, pl, static_cast<const uint16_t*>(k_bf16), static_cast<const uint16_t*>(v_bf16),
+                    static_cast<cudaStream_t>(stream_));
+    if (st != KVQ_OK) {
+      undo_table();
+      return st;
+    }
   }
   // ---- commit host state -----------------------------------------------------
-  h->table.swap(tbl);
   h->nblk = nblk;
   for (int64_t j = 0; j < allocs; ++j) h->refcnt[size_t(h->freelist[size_t(j)])] = 1;
   h->freelist.erase(h->freelist.begin(), h->freelist.begin() + allocs);
@@ -617,6 +635,68 @@ kvq_status kvq_decode_attn(kvq_handle h, const void* q_bf16, const int32_t* bloc
     seqmap = h->d_seqmap;
   }
   return launch_handle_decode(h, q_bf16, block_table, bt_stride, seq_lens, seqmap, batch, out, stream);
+}
+
+namespace {
+
+// Grows the staging of kvq_step_host to at least `rows` K/V rows and `batch`
+// q / output rows.  Earlier steps may still read the old buffers: growing
+// waits for the device first.
+kvq_status ensure_io(kvq_handle h, int32_t rows, int32_t batch) {
+  if (rows <= h->io_rows && batch <= h->io_batch) return KVQ_OK;
+  KVQ_CUDA(cudaDeviceSynchronize());
+  const int32_t r = std::max(rows, h->io_rows), b = std::max(batch, h->io_batch);
+  const kvq_config& c = h->cfg;
+  const size_t kv = size_t(r) * c.h_kv * c.d_h, qo = size_t(b) * c.h_q * c.d_h;
+  for (void* p : {static_cast<void*>(h->d_kin), static_cast<void*>(h->d_vin), static_cast<void*>(h->d_qin),
+                  static_cast<void*>(h->d_out)})
+    if (p) KVQ_CUDA(cudaFree(p));
+  h->d_kin = h->d_vin = h->d_qin = nullptr;
+  h->d_out = nullptr;
+  h->bytes_workspace -= (size_t(h->io_rows) * c.h_kv * c.d_h * 4 + size_t(h->io_batch) * c.h_q * c.d_h * 6);
+  h->io_rows = h->io_batch = 0;
+  KVQ_CUDA(cudaMalloc(&h->d_kin, std::max<size_t>(kv, 1) * 2));
+  KVQ_CUDA(cudaMalloc(&h->d_vin, std::max<size_t>(kv, 1) * 2));
+  KVQ_CUDA(cudaMalloc(&h->d_qin, std::max<size_t>(qo, 1) * 2));
+  KVQ_CUDA(cudaMalloc(&h->d_out, std::max<size_t>(qo, 1) * 4));
+  h->io_rows = r;
+  h->io_batch = b;
+  h->bytes_workspace += kv * 4 + qo * 6;
+  return KVQ_OK;
+}
+
+}  // namespace
+
+kvq_status kvq_step_host(kvq_handle h, const void* k_host, const void* v_host, const int32_t* seq_ids_host,
+                         int32_t n, const void* q_host, int32_t batch, float* out_host, void* stream_) {
+  if (!h) return fail(KVQ_ERR_INVALID_ARG, "handle is null");
+  if (n < 0 || batch < 0) return fail(KVQ_ERR_INVALID_ARG, "n and batch must be >= 0");
+  if (batch > h->cfg.max_seqs) return fail(KVQ_ERR_INVALID_ARG, "batch exceeds max_seqs");
+  if (n > 0 && (!k_host || !v_host || !seq_ids_host))
+    return fail(KVQ_ERR_INVALID_ARG, "k, v and seq_ids are required when n > 0");
+  if (batch > 0 && (!q_host || !out_host)) return fail(KVQ_ERR_INVALID_ARG, "q and out are required when batch > 0");
+  kvq_status st = device_guard(h);
+  if (st != KVQ_OK) return st;
+  const kvq_config& c = h->cfg;
+  for (int32_t i = 0; i < n; ++i)   // checked here so that a bad id enqueues nothing
+    if (seq_ids_host[i] < 0 || seq_ids_host[i] >= c.max_seqs)
+      return fail(KVQ_ERR_BAD_SEQ, "sequence id " + std::to_string(seq_ids_host[i]) + " out of range");
+  st = ensure_io(h, n, batch);
+  if (st != KVQ_OK) return st;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  const size_t kv_bytes = size_t(n) * c.h_kv * c.d_h * 2, q_bytes = size_t(batch) * c.h_q * c.d_h * 2;
+  if (n > 0) {
+    KVQ_CUDA(cudaMemcpyAsync(h->d_kin, k_host, kv_bytes, cudaMemcpyHostToDevice, stream));
+    KVQ_CUDA(cudaMemcpyAsync(h->d_vin, v_host, kv_bytes, cudaMemcpyHostToDevice, stream));
+    st = kvq_append(h, h->d_kin, h->d_vin, seq_ids_host, n, stream_);
+    if (st != KVQ_OK) return st;
+  }
+  if (batch == 0) return KVQ_OK;
+  KVQ_CUDA(cudaMemcpyAsync(h->d_qin, q_host, q_bytes, cudaMemcpyHostToDevice, stream));
+  st = launch_handle_decode(h, h->d_qin, nullptr, 0, h->d_len, nullptr, batch, h->d_out, stream);
+  if (st != KVQ_OK) return st;
+  KVQ_CUDA(cudaMemcpyAsync(out_host, h->d_out, q_bytes * 2, cudaMemcpyDeviceToHost, stream));
+  return KVQ_OK;
 }
 
 kvq_status kvq_prefill_attn(kvq_handle h, const void* q_bf16, const int32_t* seq_ids_host,

@@ -40,7 +40,7 @@ EXPORTS = (
     "kvq_block_table_host", "kvq_seq_len", "kvq_seq_lens_device", "kvq_free_seq", "kvq_share_prefix",
     "kvq_stats", "kvq_cache_bytes", "kvq_layout", "kvq_read_pool", "kvq_read_residual",
     "kvq_sync_status", "kvq_set_decode_grid", "kvq_set_decode_event", "kvq_decode_attn_noalloc",
-    "kvq_prefill_attn", "kvq_set_fp8_scales", "kvq_last_error",
+    "kvq_prefill_attn", "kvq_set_fp8_scales", "kvq_step_host", "kvq_last_error",
 )
 
 
@@ -99,6 +99,7 @@ def lib():
             "kvq_free_seq": (st, [P, I32, P]),
             "kvq_share_prefix": (st, [P, I32, I32, I32, P]),
             "kvq_prefill_attn": (st, [P, P, P, P, I32, P, P]),
+            "kvq_step_host": (st, [P, P, P, P, I32, P, I32, P, P]),
             "kvq_set_fp8_scales": (st, [P, P, P]),
             "kvq_stats": (st, [P, ctypes.POINTER(KvqStats)]),
             "kvq_cache_bytes": (U64, [I32, ctypes.c_int64, I32, I32, ctypes.POINTER(KvqConfig)]),
@@ -204,6 +205,16 @@ def kvq_prefill_attn(h, q_ptr: int, seq_ids, positions, out_ptr: int, stream: in
     V = ctypes.c_void_p
     _check(lib().kvq_prefill_attn(h, V(q_ptr), V(ids.ctypes.data), V(pos.ctypes.data), int(ids.size), V(out_ptr),
                                   V(stream)))
+
+
+def kvq_step_host(h, k_ptr: int, v_ptr: int, seq_ids, q_ptr: int, batch: int, out_ptr: int,
+                  stream: int = 0):
+    """Host pointers: k, v bf16 [n][h_kv][d_h]; q bf16 [batch][h_q][d_h]; out fp32."""
+    arr, p = _host_i32(seq_ids)
+    n = 0 if arr is None else int(arr.size)
+    V = ctypes.c_void_p
+    _check(lib().kvq_step_host(h, V(k_ptr or None), V(v_ptr or None), p, n, V(q_ptr or None), int(batch),
+                               V(out_ptr or None), V(stream)))
 
 
 def kvq_set_fp8_scales(h, k_scales, v_scales):
@@ -352,6 +363,17 @@ class KVCache:
             sl = seq_lens.data_ptr()
         kvq_decode_attn(self.h, q.data_ptr(), bt, bt_stride, sl, seq_ids, B,
                         out.data_ptr(), self._stream(stream))
+
+    def step_host(self, k, v, seq_ids, q, out, stream=None):
+        """One decode step from host memory (kvq_step_host): CPU tensors k, v
+        bf16 [n, h_kv, d_h] (pinned for asynchronous copies), seq_ids int32 [n],
+        q bf16 [B, h_q, d_h]; out, CPU fp32 [B, h_q, d_h], is written once the
+        stream reaches the end of the step."""
+        for t in (k, v, q, out):
+            if t.is_cuda or not t.is_contiguous():
+                raise ValueError("step_host takes contiguous CPU tensors")
+        kvq_step_host(self.h, k.data_ptr(), v.data_ptr(), seq_ids, q.data_ptr(), int(q.shape[0]),
+                      out.data_ptr(), self._stream(stream))
 
     def seq_len(self, s):
         return kvq_seq_len(self.h, s)

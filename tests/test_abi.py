@@ -163,6 +163,14 @@ def test_null_and_host_only_guards():
     with pytest.raises(kvq.KvqError):
         kvq.kvq_append(h, 0, 0, None, 3)                     # null seq ids
     kvq.kvq_append(h, 0, 0, np.zeros(0, np.int32), 0)        # empty append is fine
+    for args in [(16, 16, np.zeros(1, np.int32), 16, 1, 16),       # host-only handle
+                 (0, 0, np.zeros(1, np.int32), 16, 1, 16),         # rows without k / v
+                 (16, 16, np.zeros(1, np.int32), 16, 99, 16),      # batch above max_seqs
+                 (16, 16, np.zeros(1, np.int32), 0, 1, 0)]:        # decode rows without q / out
+        with pytest.raises(kvq.KvqError) as e:
+            kvq.kvq_step_host(h, *args)
+        assert e.value.status == kvq.KVQ_ERR_INVALID_ARG
+    assert kvq.kvq_seq_len(h, 0) == 0
     kvq.kvq_destroy(h)
 
 

@@ -130,6 +130,44 @@ def test_append_launch_shapes(name):
     p.close()
 
 
+@pytest.mark.parametrize("name", ["int4_chan64", "int8_tok_p16", "fp8_p16"])
+def test_step_host_equals_device_calls(name):
+    """kvq_step_host (host buffers in, host output back, one call) appends the
+    same bytes and returns the same output as kvq_append + kvq_decode_attn on
+    device buffers, and both match the oracle."""
+    rng = np.random.default_rng(21)
+    h_q, h_kv, S = 8, 2, 3
+    fmt = FMTS[name]
+    a = Pair(fmt, h_q, h_kv, max_seqs=S, num_blocks=300, mbps=128, seed=4)
+    b = kvq.KVCache(kvq.Format(**fmt), h_q, h_kv, S, 300, 128, seed=4)
+    lens = [70, 5, 129]
+    ids = np.repeat(np.arange(S, dtype=np.int32), lens)
+    k0, v0 = outlier_keys(rng, ids.size, h_kv), random_bf16(rng, (ids.size, h_kv, D))
+    a.append(k0, v0, ids)
+    b.append(bits_to_cuda_bf16(k0), bits_to_cuda_bf16(v0), ids)
+
+    def host(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).pin_memory()
+
+    for step in range(70):   # crosses group boundaries of every sequence
+        ids = np.arange(S, dtype=np.int32)
+        k, v, q = outlier_keys(rng, S, h_kv), random_bf16(rng, (S, h_kv, D)), random_bf16(rng, (S, h_q, D))
+        lens = [L + 1 for L in lens]
+        a.append(k, v, ids)
+        out_h = torch.full((S, h_q, D), float("nan"), dtype=torch.float32).pin_memory()
+        b.step_host(host(k), host(v), ids, host(q), out_h)
+        torch.cuda.synchronize()
+        if step % 23 == 0 or step == 69:
+            got, want = a.decode(q, lens)
+            assert np.array_equal(out_h.numpy(), got.astype(np.float32))
+            assert np.max(np.abs(got - want)) <= ATOL
+    a.check_state()
+    assert np.array_equal(b.pool(), a.gpu.pool())
+    assert b.sync_status() == 0
+    b.close()
+    a.close()
+
+
 @pytest.mark.parametrize("name", ["int4_chan64", "int8_tok_p16", "int2_asym_chan32", "bf16_control_p16", "fp8_p16"])
 def test_split_k_merge_is_invariant_to_grid(name):
     rng = np.random.default_rng(3)
