@@ -189,7 +189,7 @@ def measured_peak():
 
 def kernel_source_sha():
     h = hashlib.sha256()
-    for f in ("kvq_decode.cu", "kvq_device.cuh", "kvq_internal.h"):
+    for f in ("kvq_decode.cu", "kvq_device.cuh", "kvq_tiles.cuh", "kvq_internal.h"):
         with open(os.path.join(ROOT, "quantized_kv_cache_14_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -527,11 +527,14 @@ def run_next_rows(args):
     assert c.sync_status() == 0
     c.close()
     row_bytes = decode_bytes(w, [int(p) + 1 for p in pos])
+    flops = 4.0 * w.h_q * D * float(sum(int(p) + 1 for p in pos))   # QK^T and PV, 2 flops per MAC
     prefill = {"workload": f"one sequence, {Lc}-token context, chunk of {C} new tokens",
                "chunk_us": us, "query_tokens_per_s": C / (us * 1e-6),
+               "attention_tflops": flops / (us * 1e-6) / 1e12,
                "row_bytes": row_bytes, "row_gbs": row_bytes / (us * 1e-6) / 1e9,
-               "note": "each chunk token is a decode row over its own causal prefix (rows re-read "
-                       "the shared context, mostly from L2)"}
+               "note": "the prefill kernel: 64 / g query tokens of the chunk share every staged tile "
+                       "(rows in the mma M dimension), key range split over CTAs; row_gbs counts the "
+                       "bytes each row would read on its own"}
     return {"calls": K, "prefix_sharing": share, "chunked_prefill": prefill}
 
 

@@ -361,8 +361,13 @@ kvq_status kvq_decode_attn_noalloc(const kvq_config* cfg, const void* pool, cons
  *   seq_ids_host    host int32 [n]; positions_host host int32 [n], each a
  *                   stored position of its sequence.
  *   out             device fp32 [n][h_q][d_h].
- * Runs as decode launches of at most max_seqs rows, each row reading its own
- * prefix (no reuse of a key tile across the chunk's rows).  Errors:
+ * Channel-axis formats with the window (2/4/8-bit codes, fp16 scales) run
+ * the prefill kernel: up to 64 / g query tokens of one sequence share every
+ * staged tile (their rows are the mma M dimension), the key range split over
+ * CTAs and merged by log-sum-exp.  Other formats run as decode launches of at
+ * most max_seqs rows, each row reading its own prefix.  Rows may come in any
+ * order; the call uploads a small plan (rows sorted by sequence and position)
+ * and may grow a workspace (with a device synchronize).  Errors:
  * KVQ_ERR_BAD_SEQ for an id out of range, KVQ_ERR_INVALID_ARG for a position
  * that is not stored or null / unaligned pointers. */
 kvq_status kvq_prefill_attn(kvq_handle h, const void* q_bf16, const int32_t* seq_ids_host,

@@ -95,6 +95,36 @@ struct DecodeArgs {
   Geo g;
 };
 
+// Chunked-prefill attention (kvq_prefill.cu).  The plan holds three int32
+// sections: rows [n][2] = (row, position) sorted by sequence and position;
+// blocks [nb][4] = (sequence, first row entry, rows, quantized length); tasks
+// [n_tasks][5] = (block, kv head, split, first unit, end unit), one CTA each.
+constexpr int kPrefillMaxPages = 1024;   // block ids one task caches in shared memory
+struct PrefillArgs {
+  const uint8_t* pool;
+  const uint16_t* kres;
+  const uint16_t* vres;
+  const int32_t* table;       // the handle's block table [max_seqs][table_stride]
+  int32_t table_stride;
+  const uint16_t* q;          // bf16 [n][h_q][D]
+  float* out;                 // fp32 [n][h_q][D]
+  float* part;                // with splits > 1: records [n][h_q][splits][D + 2]
+  const int32_t* plan;
+  int32_t off_rows, off_blocks, off_tasks;
+  int32_t n_tasks, splits;
+  uint32_t* err;
+  float qk_scale;             // log2(e) / sqrt(D)
+  int32_t sup, lg_sup;        // tokens per unit (whole key groups) and its log2
+  int32_t stage_bytes;
+  Geo g;
+};
+// Formats with a prefill kernel: channel-axis keys with the window, 2/4/8-bit
+// codes, fp16 scales.  Others run their chunk as decode rows.
+bool prefill_supported(const Geo& g);
+int prefill_stage_bytes(const Geo& g, int sup);
+size_t prefill_smem_bytes(int stage_bytes);
+cudaError_t launch_prefill(const PrefillArgs& a, int64_t n_rows, cudaStream_t s, int* launches);
+
 // Host-side launchers (defined in the .cu files).
 // Each launcher adds the number of kernels it launched to *launches.
 // Table, length and zeroing updates of a plan; given k and v it also copies

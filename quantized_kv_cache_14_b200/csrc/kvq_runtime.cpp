@@ -197,6 +197,11 @@ struct kvq_handle_s {
   float* d_out = nullptr;
   int32_t io_rows = 0;    // K/V rows the staging holds
   int32_t io_batch = 0;   // q / output rows the staging holds
+  // chunked prefill: plan and split records (grown on demand)
+  int32_t* d_pfplan = nullptr;
+  size_t pfplan_cap = 0;  // int32 entries
+  float* d_pfpart = nullptr;
+  size_t pfpart_cap = 0;  // floats
 };
 
 namespace {
@@ -338,6 +343,8 @@ void destroy_device(kvq_handle h) {
   cudaFree(h->d_vin);
   cudaFree(h->d_qin);
   cudaFree(h->d_out);
+  cudaFree(h->d_pfplan);
+  cudaFree(h->d_pfpart);
   for (auto& s : h->slots) {
     if (s.host) cudaFreeHost(s.host);
     if (s.ev) cudaEventDestroy(s.ev);
@@ -699,6 +706,114 @@ kvq_status kvq_step_host(kvq_handle h, const void* k_host, const void* v_host, c
   return KVQ_OK;
 }
 
+namespace {
+
+// Grows a device buffer of `elem`-byte entries to at least `need` entries
+// (earlier launches may still read it: growing waits for the device first).
+kvq_status ensure_buffer(kvq_handle h, void** buf, size_t& cap, size_t need, size_t elem) {
+  if (need <= cap) return KVQ_OK;
+  KVQ_CUDA(cudaDeviceSynchronize());
+  if (*buf) KVQ_CUDA(cudaFree(*buf));
+  *buf = nullptr;
+  const size_t c = std::max(need, cap * 2);
+  KVQ_CUDA(cudaMalloc(buf, c * elem));
+  h->bytes_workspace += (c - cap) * elem;
+  cap = c;
+  return KVQ_OK;
+}
+
+// Chunked prefill with shared tiles: rows sorted by (sequence, position) form
+// blocks of at most 64 / g query tokens of one sequence; each block is split
+// over the key range into `splits` tasks per kv head, one CTA each.
+kvq_status prefill_blocks(kvq_handle h, const uint16_t* q, const int32_t* seq_ids, const int32_t* pos,
+                          int32_t n, float* out, cudaStream_t stream) {
+  const kvq::Geo& g = h->geo;
+  const int G = g.G, QB = 4 * (16 / G);
+  std::vector<int32_t> order(static_cast<size_t>(n));
+  for (int32_t i = 0; i < n; ++i) order[size_t(i)] = i;
+  std::stable_sort(order.begin(), order.end(), [&](int32_t x, int32_t y) {
+    return seq_ids[x] != seq_ids[y] ? seq_ids[x] < seq_ids[y] : pos[x] < pos[y];
+  });
+  std::vector<int32_t> rows, blocks, tasks;
+  rows.reserve(size_t(n) * 2);
+  std::vector<int32_t> nq;   // quantized units per block
+  const int sup = h->pipe.sup;
+  for (int32_t i = 0; i < n;) {
+    const int32_t s = seq_ids[order[size_t(i)]];
+    int32_t j = i;
+    while (j < n && j - i < QB && seq_ids[order[size_t(j)]] == s) ++j;
+    const int32_t Lq = (h->len[size_t(s)] / g.g_k) * g.g_k;
+    const int32_t bmax = pos[order[size_t(j - 1)]];
+    blocks.insert(blocks.end(), {s, int32_t(rows.size() / 2), j - i, Lq});
+    for (int32_t k = i; k < j; ++k) rows.insert(rows.end(), {order[size_t(k)], pos[order[size_t(k)]]});
+    nq.push_back((std::min(bmax + 1, Lq) + sup - 1) / sup);
+    i = j;
+  }
+  const int nb = int(nq.size());
+  const int cap_units = kvq::kPrefillMaxPages / (sup / g.P);
+  int max_nq = 1;
+  for (int x : nq) max_nq = std::max(max_nq, x);
+  // Two CTAs fit per SM.  Pick the split count that minimises (waves of
+  // resident CTAs) x (units per task), with a small charge per split for the
+  // merge; no task may outgrow its block-id cache.
+  const int slots = 2 * h->sm_count;
+  const int smin = std::max(1, (max_nq + cap_units - 1) / cap_units);
+  const int smax = std::max(smin, std::min(64, max_nq));
+  int splits = smin;
+  double best = 1e300;
+  for (int sp = smin; sp <= smax; ++sp) {
+    const int64_t waves = (int64_t(nb) * g.h_kv * sp + slots - 1) / slots;
+    const double cost = double(waves) * double((max_nq + sp - 1) / sp) + 0.02 * sp;
+    if (cost < best) {
+      best = cost;
+      splits = sp;
+    }
+  }
+  for (int b = 0; b < nb; ++b)
+    for (int hk = 0; hk < g.h_kv; ++hk)
+      for (int sp = 0; sp < splits; ++sp)
+        tasks.insert(tasks.end(), {b, hk, sp, int32_t(int64_t(sp) * nq[size_t(b)] / splits),
+                                   int32_t(int64_t(sp + 1) * nq[size_t(b)] / splits)});
+  kvq::PrefillArgs a{};
+  a.off_rows = 0;
+  a.off_blocks = int32_t(rows.size());
+  a.off_tasks = a.off_blocks + int32_t(blocks.size());
+  const size_t total = size_t(a.off_tasks) + tasks.size();
+  std::vector<int32_t> flat;
+  flat.reserve(total);
+  for (const auto* sec : {&rows, &blocks, &tasks}) flat.insert(flat.end(), sec->begin(), sec->end());
+  kvq_status st = ensure_buffer(h, reinterpret_cast<void**>(&h->d_pfplan), h->pfplan_cap, total, 4);
+  if (st != KVQ_OK) return st;
+  if (splits > 1) {
+    st = ensure_buffer(h, reinterpret_cast<void**>(&h->d_pfpart), h->pfpart_cap,
+                       size_t(n) * g.h_q * splits * (kvq::kD + 2), 4);
+    if (st != KVQ_OK) return st;
+  }
+  st = stage_upload(h, flat.data(), total, h->d_pfplan, stream);
+  if (st != KVQ_OK) return st;
+  a.pool = h->d_pool;
+  a.kres = h->d_kres;
+  a.vres = h->d_vres;
+  a.table = h->d_table;
+  a.table_stride = h->cfg.max_blocks_per_seq;
+  a.q = q;
+  a.out = out;
+  a.part = h->d_pfpart;
+  a.plan = h->d_pfplan;
+  a.n_tasks = int32_t(tasks.size() / 5);
+  a.splits = splits;
+  a.err = h->d_err;
+  a.qk_scale = float(1.4426950408889634 / std::sqrt(double(kvq::kD)));
+  a.sup = sup;
+  a.lg_sup = h->pipe.lg_sup;
+  a.stage_bytes = kvq::prefill_stage_bytes(g, sup);
+  a.g = g;
+  KVQ_CUDA(kvq::launch_prefill(a, n, stream, &h->launches));
+  return KVQ_OK;
+}
+
+}  // namespace
+
 kvq_status kvq_prefill_attn(kvq_handle h, const void* q_bf16, const int32_t* seq_ids_host,
                             const int32_t* positions_host, int32_t n, float* out, void* stream_) {
   if (!h) return fail(KVQ_ERR_INVALID_ARG, "handle is null");
@@ -719,8 +834,10 @@ kvq_status kvq_prefill_attn(kvq_handle h, const void* q_bf16, const int32_t* seq
                                            std::to_string(i) + " is not a stored position of its sequence");
   }
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
-  // one decode row per query token, attending its own causal prefix; at most
-  // max_seqs rows per launch (the planned batch)
+  if (kvq::prefill_supported(h->geo))
+    return prefill_blocks(h, static_cast<const uint16_t*>(q_bf16), seq_ids_host, positions_host, n, out, stream);
+  // other formats: one decode row per query token, attending its own causal
+  // prefix; at most max_seqs rows per launch (the planned batch)
   std::vector<int32_t> rowlen(size_t(std::min<int32_t>(n, c.max_seqs)));
   const int64_t row = int64_t(c.h_q) * c.d_h;
   for (int32_t base = 0; base < n; base += c.max_seqs) {

@@ -247,6 +247,48 @@ def test_chunked_prefill_attention(name):
     p.close()
 
 
+@pytest.mark.parametrize("name,h_q,h_kv", [
+    ("int4_chan64", 8, 2), ("int4_chan64", 4, 2), ("int4_chan64", 2, 2), ("int2_asym_chan32", 8, 2),
+    ("int4_chan64_p32_gv32", 8, 2), ("int8_asym_chan128_p64", 4, 1), ("int4_chan16", 8, 2)])
+def test_prefill_kernel_blocks(name, h_q, h_kv):
+    """The shared-tile prefill kernel: chunks of several sequences with rows in
+    shuffled order, long prefixes (the key range split over CTAs and merged),
+    a sequence whose chunk sits only in the window, and a single-split call."""
+    rng = np.random.default_rng(31)
+    fmt = FMTS[name]
+    S = 3
+    p = Pair(fmt, h_q, h_kv, max_seqs=S, num_blocks=900, mbps=256, seed=3)
+    pre = [1500, 64, 0]
+    ids = np.repeat(np.arange(S, dtype=np.int32), pre)
+    p.append(outlier_keys(rng, ids.size, h_kv), random_bf16(rng, (ids.size, h_kv, D)), ids)
+    chunk = [100, 70, 9]
+    cids = np.concatenate([np.full(c, s, np.int32) for s, c in enumerate(chunk)])
+    p.append(outlier_keys(rng, cids.size, h_kv), random_bf16(rng, (cids.size, h_kv, D)), cids)
+    pos = np.concatenate([np.arange(pre[s], pre[s] + chunk[s]) for s in range(S)]).astype(np.int32)
+    perm = rng.permutation(cids.size)
+    cids, pos = cids[perm], pos[perm]
+    q = random_bf16(rng, (cids.size, h_q, D))
+    out = torch.full((cids.size, h_q, D), float("nan"), dtype=torch.float32, device="cuda")
+    p.gpu.prefill_attn(bits_to_cuda_bf16(q), cids, pos, out)
+    torch.cuda.synchronize()
+    assert p.gpu.sync_status() == 0
+    want = p.orc.decode(q, (pos + 1).tolist(), seq_ids=cids)
+    got = out.cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(got))
+    err = float(np.max(np.abs(got - want)))
+    assert err <= ATOL, f"max abs error {err}"
+    # one short chunk of one sequence: a single split writes the output directly
+    q1 = random_bf16(rng, (5, h_q, D))
+    ids1 = np.full(5, 1, np.int32)
+    pos1 = np.arange(60, 65, dtype=np.int32)
+    out1 = torch.full((5, h_q, D), float("nan"), dtype=torch.float32, device="cuda")
+    p.gpu.prefill_attn(bits_to_cuda_bf16(q1), ids1, pos1, out1)
+    torch.cuda.synchronize()
+    want1 = p.orc.decode(q1, (pos1 + 1).tolist(), seq_ids=ids1)
+    assert np.max(np.abs(out1.cpu().numpy().astype(np.float64) - want1)) <= ATOL
+    p.close()
+
+
 @pytest.mark.parametrize("page", [16, 32])
 def test_fp8_per_head_scales(page):
     """FP8 with per-head scales from amax / 448 of a sample, keys with large
