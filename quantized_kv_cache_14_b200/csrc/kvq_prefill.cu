@@ -517,16 +517,19 @@ __global__ void __launch_bounds__(kD) prefill_merge_kernel(const float* __restri
                                                           int splits) {
   const int c = threadIdx.x;
   const float* rec = part + int64_t(blockIdx.x) * splits * (kD + 2);
+  // the loops are unrolled so that their independent loads overlap
   float M = -INFINITY;
+#pragma unroll 8
   for (int s = 0; s < splits; ++s) M = fmaxf(M, rec[s * (kD + 2) + kD]);
   float num = 0.0f, den = 0.0f;
   if (M != -INFINITY) {
+#pragma unroll 8
     for (int s = 0; s < splits; ++s) {
       const float m = rec[s * (kD + 2) + kD];
-      if (m == -INFINITY) continue;
-      const float w = fast_exp2(m - M);
-      num = fmaf(w, rec[s * (kD + 2) + c], num);
-      den = fmaf(w, rec[s * (kD + 2) + kD + 1], den);
+      const float x = rec[s * (kD + 2) + c], y = rec[s * (kD + 2) + kD + 1];
+      const float w = m == -INFINITY ? 0.0f : fast_exp2(m - M);
+      num = fmaf(w, x, num);
+      den = fmaf(w, y, den);
     }
   }
   out[int64_t(blockIdx.x) * kD + c] = den > 0.0f ? num / den : 0.0f;

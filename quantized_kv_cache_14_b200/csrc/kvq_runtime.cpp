@@ -753,27 +753,41 @@ kvq_status prefill_blocks(kvq_handle h, const uint16_t* q, const int32_t* seq_id
   const int cap_units = kvq::kPrefillMaxPages / (sup / g.P);
   int max_nq = 1;
   for (int x : nq) max_nq = std::max(max_nq, x);
-  // Two CTAs fit per SM.  Pick the split count that minimises (waves of
-  // resident CTAs) x (units per task), with a small charge per split for the
-  // merge; no task may outgrow its block-id cache.
+  // Two CTAs fit per SM.  Pick the split count that minimises the makespan
+  // estimate max(waves of resident CTAs x (mean units per task + a task's
+  // fixed cost), the longest task + that cost); a task's setup, pipeline fill
+  // and records cost about as much as 8 units.  No task may outgrow its
+  // block-id cache.
   const int slots = 2 * h->sm_count;
+  double units = 0.0;
+  for (int x : nq) units += double(x) * g.h_kv;
   const int smin = std::max(1, (max_nq + cap_units - 1) / cap_units);
   const int smax = std::max(smin, std::min(64, max_nq));
   int splits = smin;
   double best = 1e300;
   for (int sp = smin; sp <= smax; ++sp) {
-    const int64_t waves = (int64_t(nb) * g.h_kv * sp + slots - 1) / slots;
-    const double cost = double(waves) * double((max_nq + sp - 1) / sp) + 0.02 * sp;
+    const int64_t ntask = int64_t(nb) * g.h_kv * sp;
+    const double waves = double((ntask + slots - 1) / slots);
+    constexpr double kTaskUnits = 8.0;
+    const double cost = std::max(waves * (units / double(ntask) + kTaskUnits),
+                                 double((max_nq + sp - 1) / sp) + kTaskUnits);
     if (cost < best) {
       best = cost;
       splits = sp;
     }
   }
+  struct Task { int32_t b, hk, sp, u0, u1; };
+  std::vector<Task> tl;
+  tl.reserve(size_t(nb) * g.h_kv * splits);
   for (int b = 0; b < nb; ++b)
     for (int hk = 0; hk < g.h_kv; ++hk)
       for (int sp = 0; sp < splits; ++sp)
-        tasks.insert(tasks.end(), {b, hk, sp, int32_t(int64_t(sp) * nq[size_t(b)] / splits),
-                                   int32_t(int64_t(sp + 1) * nq[size_t(b)] / splits)});
+        tl.push_back({b, hk, sp, int32_t(int64_t(sp) * nq[size_t(b)] / splits),
+                      int32_t(int64_t(sp + 1) * nq[size_t(b)] / splits)});
+  // longest tasks first: CTAs start roughly in index order, so this packs the
+  // resident slots like a longest-processing-time schedule
+  std::stable_sort(tl.begin(), tl.end(), [](const Task& x, const Task& y) { return x.u1 - x.u0 > y.u1 - y.u0; });
+  for (const Task& t : tl) tasks.insert(tasks.end(), {t.b, t.hk, t.sp, t.u0, t.u1});
   kvq::PrefillArgs a{};
   a.off_rows = 0;
   a.off_blocks = int32_t(rows.size());
