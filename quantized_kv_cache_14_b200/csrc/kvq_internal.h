@@ -123,6 +123,8 @@ struct PrefillArgs {
 bool prefill_supported(const Geo& g);
 int prefill_stage_bytes(const Geo& g, int sup);
 size_t prefill_smem_bytes(int stage_bytes);
+// Resident prefill CTAs per SM for the format (occupancy API; at least 1).
+int prefill_ctas_per_sm(const Geo& g, int stage_bytes);
 cudaError_t launch_prefill(const PrefillArgs& a, int64_t n_rows, cudaStream_t s, int* launches);
 
 // Host-side launchers (defined in the .cu files).

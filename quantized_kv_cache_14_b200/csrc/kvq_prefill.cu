@@ -15,15 +15,18 @@
 //    a tile is read from memory once for up to 64 rows.
 //  * Thread 0 stages whole page chunks of units (whole key groups, 64 tokens
 //    or one group when longer) and 16-row tiles of the BF16 window with
-//    cp.async.bulk into a 4-stage ring that completes on mbarriers; the CTA
+//    cp.async.bulk into a 2-stage ring that completes on mbarriers; the CTA
 //    frees a stage with one barrier per item.  The task's block ids are read
-//    into shared memory once.
+//    into shared memory once.  Up to three CTAs (12 warps) fit on an SM (two
+//    with 128-token units): the context is mostly in L2, so more warps hide
+//    latency better than a deeper ring would.
 //  * Scores S = Q' C^T: the codes C are exact small integers in fp16 (the B
 //    operand, from the packed words exactly as in decode) and Q' = q s_key of
-//    the key group, split into fp16 hi + lo parts (two A operands).  Each
-//    row's q is first scaled by a power of two (max |q| in [1/2, 1)) so that
-//    Q' stays inside the fp16 range; the power goes back into the row's score
-//    scale.  Window tiles multiply q and the bf16 rows directly (exact).
+//    the key group, split into fp16 hi + lo parts kept in shared memory and
+//    read per k-step with ldmatrix (two A operands).  Each row's q is first
+//    scaled by a power of two (max |q| in [1/2, 1)) so that Q' stays inside
+//    the fp16 range; the power goes back into the row's score scale.  Window
+//    tiles multiply q and the bf16 rows directly (exact).
 //  * Online softmax per 16-token sub-tile in the log2 domain with the exact
 //    running max (p <= 1); P' = p s_value of each value group as fp16 hi + lo
 //    A operands against the value codes.  Zero-points enter as a per-row key
@@ -41,21 +44,22 @@ namespace {
 
 constexpr int kPfWarps = 4;
 constexpr int kPfThreads = 32 * kPfWarps;
-constexpr int kPfStages = 4;
+constexpr int kPfStages = 2;
 constexpr uint64_t kPfWaitNs = 2000000000ull;   // give up on a copy after 2 s
 constexpr uint32_t kFull = 0xffffffffu;
 
 struct PfSmem {
-  int stages, qs, qn, cs, blk, bars, flag, total;
+  int stages, qs, qp, cs, dn, blk, bars, flag, total;
 };
 
 __host__ __device__ inline PfSmem pf_smem(int stage_bytes) {
   PfSmem L;
   L.stages = 0;
-  L.qs = kPfStages * stage_bytes;                   // bf16 q rows, 16-byte chunks swizzled
-  L.qn = L.qs + kPfWarps * 16 * kD * 2;             // fp16 scaled q rows, key-row position order
-  L.cs = L.qn + kPfWarps * 16 * kD * 2;             // per-row score scale
-  L.blk = L.cs + kPfWarps * 16 * 4;                 // the task's block ids
+  L.qs = kPfStages * stage_bytes;                   // bf16 q rows, 16-byte chunks swizzled by row
+  L.qp = L.qs + kPfWarps * 16 * kD * 2;             // Q' hi and lo tiles per warp, swizzled likewise
+  L.cs = L.qp + kPfWarps * 2 * 16 * kD * 2;         // per-row score scale
+  L.dn = L.cs + kPfWarps * 16 * 4;                  // per-row q scaling 2^-e
+  L.blk = L.dn + kPfWarps * 16 * 4;                 // the task's block ids
   L.bars = L.blk + kPrefillMaxPages * 4;
   L.flag = L.bars + kPfStages * 8;
   L.total = L.flag + 16;
@@ -85,7 +89,7 @@ __device__ __forceinline__ void ps_split(uint32_t ph, uint32_t pl, uint32_t s2, 
 }
 
 template <int BITS, int ASYM>
-__global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_constant__ PrefillArgs a) {
+__global__ void __launch_bounds__(kPfThreads, 3) prefill_kernel(const __grid_constant__ PrefillArgs a) {
   constexpr int D = kD;
   constexpr bool SGN = !ASYM;
   const Geo& g = a.g;
@@ -115,8 +119,10 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
   const int K = nu + nw;
 
   uint16_t* qs = reinterpret_cast<uint16_t*>(smem + L.qs) + warp * 16 * D;
-  __half* qn = reinterpret_cast<__half*>(smem + L.qn) + warp * 16 * D;
+  __half* qph = reinterpret_cast<__half*>(smem + L.qp) + warp * 2 * 16 * D;
+  __half* qpl = qph + 16 * D;
   float* cs = reinterpret_cast<float*>(smem + L.cs) + warp * 16;
+  float* dn = reinterpret_cast<float*>(smem + L.dn) + warp * 16;
   int32_t* sblk = reinterpret_cast<int32_t*>(smem + L.blk);
   volatile int32_t* abort_flag = reinterpret_cast<int32_t*>(smem + L.flag);
   const uint32_t stage0 = smem_addr(smem + L.stages);
@@ -161,22 +167,14 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
     // 2^-ex puts max |q| in [1/2, 1)
     const int ex = amax > 0.0f ? min(max(int((__float_as_uint(amax) >> 23) & 0xFF) - 126, -126), 126) : 0;
     const float down = __uint_as_float(uint32_t(127 - ex) << 23);
-    if (half == 0) cs[r] = a.qk_scale * __uint_as_float(uint32_t(127 + ex) << 23);
+    if (half == 0) {
+      cs[r] = a.qk_scale * __uint_as_float(uint32_t(127 + ex) << 23);
+      dn[r] = down;
+    }
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
       const int ch = 8 * half + c;   // 16-byte chunk of the row
       *reinterpret_cast<uint4*>(qs + r * D + 8 * (ch ^ (r & 7))) = v[c];
-      const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const __half2 x = __floats2half2_rn(__uint_as_float(w[e] << 16) * down,
-                                            __uint_as_float(w[e] & 0xFFFF0000u) * down);
-        // channels (c, c + 1) go to key-row positions (f, f + 1), the order of
-        // the packed key words and of the stored key scales
-        const int c = 8 * ch + 2 * e, cw = c & 15;
-        const int f = 32 * ((cw & 7) >> 1) + 4 * (c >> 4) + 2 * (cw >> 3);
-        *reinterpret_cast<__half2*>(qn + r * D + f) = x;
-      }
     }
   }
   __syncthreads();
@@ -224,7 +222,6 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
   for (int d = 0; d < 16; ++d) o[d][0] = o[d][1] = o[d][2] = o[d][3] = 0.0f;
   float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.0f, l_b = 0.0f;
   float za[4] = {0.0f, 0.0f, 0.0f, 0.0f}, zb[4] = {0.0f, 0.0f, 0.0f, 0.0f};   // value zero sums per group
-  uint32_t qh[8][4], ql[8][4];   // Q' of the current key group, hi and lo A operands
   float bias_a = 0.0f, bias_b = 0.0f;
   const int vg_shift = g.g_v == 32 ? 1 : g.g_v == 64 ? 2 : 3;   // channel tiles per value group, log2
 
@@ -263,37 +260,58 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
     }
   };
 
-  // Q' = q s of key group gi (of the unit in `stg`) at the lane's key-row
-  // positions 32tq + 4j + {0..3} (channels 16j + 2tq + {0, 1, 8, 9}: the k
-  // indices 2tq, 2tq + 1, 2tq + 8, 2tq + 9 of k-step j), both rows; with
-  // zero-points, the rows' key bias.
+  // Q' = q s of key group gi (of the unit in `stg`) for the warp's 16 rows,
+  // written as fp16 hi and lo tiles in natural channel order (16-byte chunks
+  // swizzled by row, as qs) for ldmatrix.  The lane covers channels 16j + 2tq
+  // + {0, 1, 8, 9} of rows gq and gq + 8: the k indices 2tq, 2tq + 1, 2tq + 8,
+  // 2tq + 9 of k-step j, whose scales sit at key-row positions 32tq + 4j +
+  // {0..3}.  With zero-points, also the rows' key bias.
   auto qprime = [&](const uint8_t* stg, int gi) {
     const int lg_ppg = g.lg_gk - g.lg_P;
+    const float dna = dn[gq], dnb = dn[gq + 8];
+    const int sw = gq & 7;   // rows gq and gq + 8 share their swizzle
     float da = 0.0f, db = 0.0f;
+    auto scaled = [](uint32_t w, float d, float& x0, float& x1) {
+      x0 = __uint_as_float(w << 16) * d;
+      x1 = __uint_as_float(w & 0xFFFF0000u) * d;
+      const __half2 h = __floats2half2_rn(x0, x1);
+      return *reinterpret_cast<const uint32_t*>(&h);
+    };
+    __syncwarp();   // the previous group's tiles are no longer read
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const int c = 32 * tq + 4 * j;
-      const uint8_t* km = stg + ((gi << lg_ppg) + (c >> g.lg_kslice)) * g.chunk_used + g.off_Km;
-      const int off = c & (g.kslice - 1);
+      const int f = 32 * tq + 4 * j;
+      const uint8_t* km = stg + ((gi << lg_ppg) + (f >> g.lg_kslice)) * g.chunk_used + g.off_Km;
+      const int off = f & (g.kslice - 1);
       const uint2 s = *reinterpret_cast<const uint2*>(km + 2 * off);
-      const uint2 xa = *reinterpret_cast<const uint2*>(qn + gq * D + c);
-      const uint2 xb = *reinterpret_cast<const uint2*>(qn + (gq + 8) * D + c);
-      qs_split(xa.x, s.x, qh[j][0], ql[j][0]);
-      qs_split(xb.x, s.x, qh[j][1], ql[j][1]);
-      qs_split(xa.y, s.y, qh[j][2], ql[j][2]);
-      qs_split(xb.y, s.y, qh[j][3], ql[j][3]);
+      const int e0 = 8 * ((2 * j) ^ sw) + 2 * tq, e1 = 8 * ((2 * j + 1) ^ sw) + 2 * tq;
+      float x[8];
+      const uint32_t qa0 = scaled(*reinterpret_cast<const uint32_t*>(qs + gq * D + e0), dna, x[0], x[1]);
+      const uint32_t qa1 = scaled(*reinterpret_cast<const uint32_t*>(qs + gq * D + e1), dna, x[2], x[3]);
+      const uint32_t qb0 = scaled(*reinterpret_cast<const uint32_t*>(qs + (gq + 8) * D + e0), dnb, x[4], x[5]);
+      const uint32_t qb1 = scaled(*reinterpret_cast<const uint32_t*>(qs + (gq + 8) * D + e1), dnb, x[6], x[7]);
+      uint32_t hi, lo;
+      qs_split(qa0, s.x, hi, lo);
+      *reinterpret_cast<uint32_t*>(qph + gq * D + e0) = hi;
+      *reinterpret_cast<uint32_t*>(qpl + gq * D + e0) = lo;
+      qs_split(qa1, s.y, hi, lo);
+      *reinterpret_cast<uint32_t*>(qph + gq * D + e1) = hi;
+      *reinterpret_cast<uint32_t*>(qpl + gq * D + e1) = lo;
+      qs_split(qb0, s.x, hi, lo);
+      *reinterpret_cast<uint32_t*>(qph + (gq + 8) * D + e0) = hi;
+      *reinterpret_cast<uint32_t*>(qpl + (gq + 8) * D + e0) = lo;
+      qs_split(qb1, s.y, hi, lo);
+      *reinterpret_cast<uint32_t*>(qph + (gq + 8) * D + e1) = hi;
+      *reinterpret_cast<uint32_t*>(qpl + (gq + 8) * D + e1) = lo;
       if (ASYM) {
         const uint2 z = *reinterpret_cast<const uint2*>(km + 2 * (g.kslice + off));
         const float2 z0 = __half22float2(*reinterpret_cast<const __half2*>(&z.x));
         const float2 z1 = __half22float2(*reinterpret_cast<const __half2*>(&z.y));
-        const float2 a0 = __half22float2(*reinterpret_cast<const __half2*>(&xa.x));
-        const float2 a1 = __half22float2(*reinterpret_cast<const __half2*>(&xa.y));
-        const float2 b0 = __half22float2(*reinterpret_cast<const __half2*>(&xb.x));
-        const float2 b1 = __half22float2(*reinterpret_cast<const __half2*>(&xb.y));
-        da += a0.x * z0.x + a0.y * z0.y + a1.x * z1.x + a1.y * z1.y;
-        db += b0.x * z0.x + b0.y * z0.y + b1.x * z1.x + b1.y * z1.y;
+        da += x[0] * z0.x + x[1] * z0.y + x[2] * z1.x + x[3] * z1.y;
+        db += x[4] * z0.x + x[5] * z0.y + x[6] * z1.x + x[7] * z1.y;
       }
     }
+    __syncwarp();   // the tiles are complete before any lane reads them
     if (ASYM) {
       da += __shfl_xor_sync(kFull, da, 1);
       da += __shfl_xor_sync(kFull, da, 2);
@@ -314,14 +332,22 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
     // dependency chains short
     float s0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, s1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     float r0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, r1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    // ldmatrix row addresses of the Q' tiles: lane L gives row (L & 7) + 8 ((L >> 3) & 1)
+    // of chunk 2j + (L >> 4)
+    const int lr = (lane & 7) + 8 * ((lane >> 3) & 1), lc = lane >> 4;
+    const uint32_t qh_base = smem_addr(qph) + lr * D * 2, ql_base = smem_addr(qpl) + lr * D * 2;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
+      const uint32_t off = 16 * (((2 * j + lc) ^ (lr & 7)));
+      uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
+      ldsm_x4(qh_base + off, h0, h1, h2, h3);
+      ldsm_x4(ql_base + off, l0, l1, l2, l3);
       uint32_t k0, k1, k2, k3;
       key_frag<BITS, SGN, true>(wa, wb, j, k0, k1, k2, k3);
-      mma_f16(s0, qh[j][0], qh[j][1], qh[j][2], qh[j][3], k0, k2);
-      mma_f16(s1, qh[j][0], qh[j][1], qh[j][2], qh[j][3], k1, k3);
-      mma_f16(r0, ql[j][0], ql[j][1], ql[j][2], ql[j][3], k0, k2);
-      mma_f16(r1, ql[j][0], ql[j][1], ql[j][2], ql[j][3], k1, k3);
+      mma_f16(s0, h0, h1, h2, h3, k0, k2);
+      mma_f16(s1, h0, h1, h2, h3, k1, k3);
+      mma_f16(r0, l0, l1, l2, l3, k0, k2);
+      mma_f16(r1, l0, l1, l2, l3, k1, k3);
     }
     const int t0 = T + 2 * tq;
     float xa[4] = {s0[0] + r0[0], s0[1] + r0[1], s1[0] + r1[0], s1[1] + r1[1]};
@@ -568,6 +594,19 @@ int prefill_stage_bytes(const Geo& g, int sup) {
 }
 
 size_t prefill_smem_bytes(int stage_bytes) { return size_t(pf_smem(stage_bytes).total); }
+
+int prefill_ctas_per_sm(const Geo& g, int stage_bytes) {
+  const int smem = pf_smem(stage_bytes).total;
+  auto occ = [&](auto kern) {
+    int n = 0;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kPfThreads, smem) != cudaSuccess) return 1;
+    return n > 0 ? n : 1;
+  };
+  if (g.bits == 4) return g.asym ? occ(prefill_kernel<4, 1>) : occ(prefill_kernel<4, 0>);
+  if (g.bits == 2) return g.asym ? occ(prefill_kernel<2, 1>) : occ(prefill_kernel<2, 0>);
+  return g.asym ? occ(prefill_kernel<8, 1>) : occ(prefill_kernel<8, 0>);
+}
 
 cudaError_t launch_prefill(const PrefillArgs& a, int64_t n_rows, cudaStream_t s, int* launches) {
   const Geo& g = a.g;

@@ -202,6 +202,7 @@ struct kvq_handle_s {
   size_t pfplan_cap = 0;  // int32 entries
   float* d_pfpart = nullptr;
   size_t pfpart_cap = 0;  // floats
+  int pf_ctas_per_sm = 0; // resident prefill CTAs per SM (0: not queried yet)
 };
 
 namespace {
@@ -753,12 +754,14 @@ kvq_status prefill_blocks(kvq_handle h, const uint16_t* q, const int32_t* seq_id
   const int cap_units = kvq::kPrefillMaxPages / (sup / g.P);
   int max_nq = 1;
   for (int x : nq) max_nq = std::max(max_nq, x);
-  // Two CTAs fit per SM.  Pick the split count that minimises the makespan
+  // Pick the split count that minimises the makespan
   // estimate max(waves of resident CTAs x (mean units per task + a task's
   // fixed cost), the longest task + that cost); a task's setup, pipeline fill
   // and records cost about as much as 8 units.  No task may outgrow its
   // block-id cache.
-  const int slots = 2 * h->sm_count;
+  const int stage_bytes = kvq::prefill_stage_bytes(g, sup);
+  if (h->pf_ctas_per_sm == 0) h->pf_ctas_per_sm = kvq::prefill_ctas_per_sm(g, stage_bytes);
+  const int slots = h->pf_ctas_per_sm * h->sm_count;
   double units = 0.0;
   for (int x : nq) units += double(x) * g.h_kv;
   const int smin = std::max(1, (max_nq + cap_units - 1) / cap_units);
@@ -820,7 +823,7 @@ kvq_status prefill_blocks(kvq_handle h, const uint16_t* q, const int32_t* seq_id
   a.qk_scale = float(1.4426950408889634 / std::sqrt(double(kvq::kD)));
   a.sup = sup;
   a.lg_sup = h->pipe.lg_sup;
-  a.stage_bytes = kvq::prefill_stage_bytes(g, sup);
+  a.stage_bytes = stage_bytes;
   a.g = g;
   KVQ_CUDA(kvq::launch_prefill(a, n, stream, &h->launches));
   return KVQ_OK;
