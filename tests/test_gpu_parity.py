@@ -36,6 +36,7 @@ FMTS = {
     "int8_asym_chan128_p64": dict(bits=8, asym=1, k_axis=1, g_k=128, g_v=128, scale_fp32=0, residual=128, page=64),
     "int2_sym_tok64_fp32": dict(bits=2, asym=0, k_axis=0, g_k=64, g_v=64, scale_fp32=1, residual=0, page=16),
     "int4_chan16": dict(bits=4, asym=0, k_axis=1, g_k=16, g_v=128, scale_fp32=0, residual=16, page=16),
+    "int4_chan64_fp32": dict(bits=4, asym=0, k_axis=1, g_k=64, g_v=64, scale_fp32=1, residual=64, page=16),
     # the pages' unquantized BF16 cache on the same paged path (control)
     "bf16_control_p16": dict(bits=16, asym=0, k_axis=0, g_k=128, g_v=128, scale_fp32=0, residual=0, page=16),
     "bf16_control_p64": dict(bits=16, asym=0, k_axis=0, g_k=128, g_v=128, scale_fp32=0, residual=0, page=64),
@@ -286,6 +287,35 @@ def test_prefill_kernel_blocks(name, h_q, h_kv):
     torch.cuda.synchronize()
     want1 = p.orc.decode(q1, (pos1 + 1).tolist(), seq_ids=ids1)
     assert np.max(np.abs(out1.cpu().numpy().astype(np.float64) - want1)) <= ATOL
+    p.close()
+
+
+@pytest.mark.parametrize("name", ["int4_chan64", "int2_asym_chan32", "int4_chan64_fp32", "int8_tok_p16"])
+def test_prefill_over_shared_prefix(name):
+    """Chunked prefill of sequences that hold another sequence's blocks: the
+    rows read the shared pages through their own block tables (the prefill
+    kernel for the channel-axis fp16-scale formats, decode rows for the
+    others) and match the oracle."""
+    rng = np.random.default_rng(41)
+    fmt = FMTS[name]
+    unit = fmt["residual"] or fmt["page"]
+    h_q, h_kv = 8, 2
+    p = Pair(fmt, h_q, h_kv, max_seqs=3, num_blocks=600, mbps=128, seed=8)
+    n0 = 12 * unit + 5
+    p.append(outlier_keys(rng, n0, h_kv), random_bf16(rng, (n0, h_kv, D)), np.zeros(n0, np.int32))
+    p.share_prefix(0, 1, 8 * unit)
+    p.share_prefix(0, 2, 3 * unit)
+    chunk = [(1, 2 * unit + 7), (2, 40)]
+    ids = np.concatenate([np.full(c, s, np.int32) for s, c in chunk])
+    p.append(outlier_keys(rng, ids.size, h_kv), random_bf16(rng, (ids.size, h_kv, D)), ids)
+    pos = np.concatenate([np.arange(b, b + c) for b, (s, c) in zip((8 * unit, 3 * unit), chunk)]).astype(np.int32)
+    q = random_bf16(rng, (ids.size, h_q, D))
+    out = torch.full((ids.size, h_q, D), float("nan"), dtype=torch.float32, device="cuda")
+    p.gpu.prefill_attn(bits_to_cuda_bf16(q), ids, pos, out)
+    torch.cuda.synchronize()
+    assert p.gpu.sync_status() == 0
+    want = p.orc.decode(q, (pos + 1).tolist(), seq_ids=ids)
+    assert np.max(np.abs(out.cpu().numpy().astype(np.float64) - want)) <= ATOL
     p.close()
 
 
