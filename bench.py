@@ -18,6 +18,12 @@ rank runs its own replica (sequences shard across GPUs; no collective is on the
 data path; the only collectives are the barrier and the max-over-ranks timing).
 `--impl reference` times the CPU oracle (test infrastructure) on a bounded
 sample of the same workload.
+
+Beside the headline, on one GPU (skipped with --no-control): `bf16_control`
+times decode alone over the same draws for the quantized, BF16 and FP8 caches,
+and `next_rows` measures prefix sharing (pool blocks and decode time against
+unshared copies) and chunked prefill (a 256-token chunk over an 8192-token
+context through the prefill kernel).
 """
 import argparse
 import hashlib
