@@ -3,27 +3,35 @@ K/V token per sequence (quantize, residual window, flush when a key group
 fills) + decode attention for every sequence over the packed paged cache.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 3] [--impl kvq|reference]
+    python bench.py --floor            # the HBM read floor of one decode pass (own JSON)
 
-Prints ONE JSON line (rank 0).  `value` is decode-attention KV GB/s: the
+Prints ONE JSON line (rank 0).  `value` is decode-attention KV GB/s of the
+headline workload (--workload, default 3: the INT4 KIVI-style cache): the
 algorithmic bytes of the decode call (codes, scales, zero-points, BF16 window
 rows, q, out, block-table entries) over its device time, summed over ranks and
-divided by the max over ranks.  Inputs live in HBM before the timed region; L2
-is flushed before every timed step (untimed): a 256 MB write, then a read of
-another 256 MB so that the write's dirty lines are written back before the
-timed region and the timed kernels start on a cold, clean L2.  `e2e` is the same
-metric through the C ABI with host buffers: one kvq_step_host call per step
-(pinned H2D of the step's new K/V and q, append, decode, D2H of the attention
-output) inside the timed region, synchronised every step.  With N > 1 every
-rank runs its own replica (sequences shard across GPUs; no collective is on the
-data path; the only collectives are the barrier and the max-over-ranks timing).
-`--impl reference` times the CPU oracle (test infrastructure) on a bounded
-sample of the same workload.
+divided by the max over ranks.  The decode call is two launches (attention,
+then the split-K merge); `roofline.achieved` is the same bytes over the
+attention kernel alone (an event recorded between the two).  Inputs live in HBM before the timed region; L2 is flushed before
+every timed step (untimed): a 256 MB write, then a read of another 256 MB so
+that the write's dirty lines are written back before the timed region and the
+timed kernels start on a cold, clean L2.  `e2e` is the same metric through the
+C ABI with host buffers: one kvq_step_host call per step (one page-locked
+host-to-device copy of the step's k | v | q, append, decode, the attention
+output written into page-locked host memory) inside the timed region,
+synchronised every step.  With N > 1 every rank runs its own replica
+(sequences shard across GPUs; no collective is on the data path; the only
+collectives are the barrier and the max-over-ranks timing).  `--impl
+reference` times the CPU oracle (test infrastructure) on a bounded sample of
+the same workload.
 
-Beside the headline, on one GPU (skipped with --no-control): `bf16_control`
-times decode alone over the same draws for the quantized, BF16 and FP8 caches,
-and `next_rows` measures prefix sharing (pool blocks and decode time against
-unshared copies) and chunked prefill (a 256-token chunk over an 8192-token
-context through the prefill kernel).
+Beside the headline (skipped with --no-workloads): `workloads` gives the same
+measurement for the other four workloads with min(K, 20) steps each.  On one
+GPU (skipped with --no-control): `bulk_append` times the headline workload's
+bulk prefill append; `bf16_control` times decode alone over the same draws for
+the quantized, BF16 and FP8 caches; and `next_rows` measures prefix sharing
+(pool blocks and decode time against unshared copies) and chunked prefill (a
+256-token chunk over an 8192-token context through the prefill kernel).
+NVTX ranges mark every append, decode and step_host call.
 """
 import argparse
 import hashlib
@@ -224,36 +232,101 @@ def committed_traffic(workload_name, algorithmic_bytes):
 # the CUDA arm
 # ---------------------------------------------------------------------------
 
-def run_gpu(args, rank, ws, dist):
+def bulk_append_bytes(w, lengths):
+    """Bytes a bulk prefill append must move: every new bf16 K/V row read once,
+    codes and scales (+ zero-points) of the tokens that land in quantized
+    groups written, and the BF16 window rows written (groups that complete
+    within the call are quantized from the input rows)."""
+    f = w.fmt
+    es = 4 if f.scale_fp32 else 2
+    meta = 0 if (f.bits == 16 or f.fp8) else es * (1 + f.asym)
+    row = w.h_kv * D * 2
+    per_tok_q = w.h_kv * (2 * D * f.bits // 8 + D * meta // f.g_k + D * meta // f.g_v)
+    total = 0
+    for L in lengths:
+        Lq = (L // f.residual) * f.residual if f.residual else L
+        total += 2 * row * L + per_tok_q * Lq + 2 * row * (L - Lq)
+    return total
+
+
+def nvtx(name):
+    import torch
+    torch.cuda.nvtx.range_push(name)
+
+
+def nvtx_pop():
+    import torch
+    torch.cuda.nvtx.range_pop()
+
+
+def run_gpu(args, rank, ws, dist, widx, steps, warmup, bulk_calls=0):
+    """One workload: prefill (bulk append, untimed), then `warmup` steps and
+    three timed passes of `steps` steps each -- device-resident inputs (the
+    append + decode calls as a user makes them) for `value`; the same with an
+    event recorded between the attention kernel and the split-K merge, for
+    `roofline` (the attention kernel alone); and host inputs through
+    kvq_step_host for `e2e`.  With bulk_calls > 0 it also times the bulk
+    prefill append itself (a fresh cache each call)."""
     import torch
     from quantized_kv_cache_14_b200 import kvq
 
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", rank)) if ws > 1 else 0)
     dev = torch.device("cuda", torch.cuda.current_device())
-    w = workload(args.workload)
+    w = workload(widx)
     w.seed = w.seed + 1000 * rank        # each replica draws its own inputs
-    total_steps = args.warmup + 3 * args.steps   # warm-up, decode pass, attention pass, e2e pass
+    total_steps = warmup + 3 * steps     # warm-up, device pass, attention pass, e2e pass
     dr = Draws(w, steps=total_steps)
     f = w.fmt
     nb = pool_blocks(dr.lengths, total_steps + 2, f.page)
     mbps = max((L + total_steps + 2) // f.page + 2 for L in dr.lengths)
-    cache = kvq.KVCache(kvq.Format(f.bits, f.asym, f.k_axis, f.g_k, f.g_v, f.scale_fp32,
-                                   f.residual, f.page), w.h_q, w.h_kv, max_seqs=w.batch,
-                        num_blocks=nb, max_blocks_per_seq=mbps, seed=w.seed,
-                        device=torch.cuda.current_device())
+    fmt = kvq.Format(f.bits, f.asym, f.k_axis, f.g_k, f.g_v, f.scale_fp32, f.residual, f.page)
+
+    def new_cache():
+        return kvq.KVCache(fmt, w.h_q, w.h_kv, max_seqs=w.batch, num_blocks=nb, max_blocks_per_seq=mbps,
+                           seed=w.seed, device=torch.cuda.current_device())
 
     def bf16_dev(a):
         return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
 
-    # prefill (bulk append), untimed
-    cache.append(bf16_dev(dr.k), bf16_dev(dr.v), dr.seq_ids)
+    k_all, v_all = bf16_dev(dr.k), bf16_dev(dr.v)
+    bulk = None
+    if bulk_calls > 0:
+        # the bulk prefill append alone: the GPU is held by a sleep while the
+        # host plans, so the events see device time only
+        ts = []
+        for it in range(bulk_calls + 1):
+            c = new_cache()
+            torch.cuda.synchronize()
+            torch.cuda._sleep(60_000_000)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            c.append(k_all, v_all, dr.seq_ids)
+            e1.record()
+            torch.cuda.synchronize()
+            assert c.sync_status() == 0
+            if it:
+                ts.append(e0.elapsed_time(e1) * 1e3)
+            c.close()
+        us = float(np.median(ts))
+        nbytes = bulk_append_bytes(w, dr.lengths)
+        bulk = {"us": us, "bytes": nbytes, "gbs": nbytes / (us * 1e-6) / 1e9, "tokens": int(sum(dr.lengths)),
+                "calls": bulk_calls, "what": "bulk prefill append of every prefill token, device time"}
+    cache = new_cache()
+    cache.append(k_all, v_all, dr.seq_ids)      # prefill, untimed
+    del k_all, v_all
     lens = list(dr.lengths)
     B = w.batch
     ids = np.arange(B, dtype=np.int32)
     steps_in = [dr.step() for _ in range(total_steps)]
     dev_in = [(bf16_dev(k), bf16_dev(v), bf16_dev(q)) for k, v, q in steps_in]
-    host_in = [tuple(torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
-                     for a in s) for s in steps_in]
+    # host inputs of a step in one page-locked buffer, k | v | q back to back,
+    # so kvq_step_host issues one host-to-device copy
+    host_in = []
+    for k, v, q in steps_in:
+        flat = np.concatenate([k.ravel(), v.ravel(), q.ravel()]).view(np.int16)
+        buf = torch.from_numpy(flat).view(torch.bfloat16).pin_memory()
+        nk = k.size
+        host_in.append((buf[:nk].view(k.shape), buf[nk:2 * nk].view(v.shape), buf[2 * nk:].view(q.shape)))
     del dr
     out = torch.empty((B, w.h_q, D), dtype=torch.float32, device=dev)
     out_host = torch.empty_like(out, device="cpu").pin_memory()
@@ -270,38 +343,43 @@ def run_gpu(args, rank, ws, dist):
         ev0.record()
         lens = [L + 1 for L in lens]
         if e2e:
-            # one C-ABI call from pinned host buffers: H2D of k, v, q, append,
-            # decode over the stored lengths, D2H of the output
+            # one C-ABI call from page-locked host buffers: one H2D copy of
+            # k | v | q, append, decode over the stored lengths, output written
+            # into page-locked host memory
             kh, vh, qh = host_in[s]
+            nvtx("step_host")
             cache.step_host(kh, vh, ids, qh, out_host)
+            nvtx_pop()
             ev1.record()
             ev2.record()
             return
         k, v, q = dev_in[s]
+        nvtx("append")
         cache.append(k, v, ids)
+        nvtx_pop()
         ev1.record()
+        nvtx("decode")
         cache.decode(q, None, out)              # attends over the stored lengths
+        nvtx_pop()
         ev2.record()
 
-    # warm-up
-    for s in range(args.warmup):
+    for s in range(warmup):
         one_step(s, False, [torch.cuda.Event(enable_timing=True) for _ in range(3)])
     torch.cuda.synchronize()
     assert cache.sync_status() == 0
 
-    # timed: device-resident inputs, the decode call as a user makes it.  The
+    # timed: device-resident inputs, the calls as a user makes them.  The
     # host enqueues every step before waiting (as a serving loop runs ahead of
     # the GPU), so the events see device time, not host launch gaps.
-    cache.set_decode_event(None)
     st0 = cache.stats()["kernel_launches"]
     sampler = ClockSampler(torch.cuda.current_device(), enabled=not args.no_clocks)
     time.sleep(0.15 if sampler.proc else 0)
     barrier(dist)
     torch.cuda.synchronize()
     kv_bytes, app_bytes, seq_tokens = 0, 0, 0
-    s0 = args.warmup
+    s0 = warmup
     step_evs = []
-    for s in range(s0, s0 + args.steps):
+    for s in range(s0, s0 + steps):
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
         before = list(lens)
         one_step(s, False, evs)
@@ -321,18 +399,18 @@ def run_gpu(args, rank, ws, dist):
     barrier(dist)
     torch.cuda.synchronize()
     attn_bytes = 0
-    s0 += args.steps
-    step_evs = []
-    for s in range(s0, s0 + args.steps):
+    s0 += steps
+    attn_evs = []
+    for s in range(s0, s0 + steps):
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
         mid = torch.cuda.Event(enable_timing=True)
         mid.record()              # creates the CUDA event; the library records it again
         cache.set_decode_event(mid)
         one_step(s, False, evs)
-        step_evs.append((evs, mid))
+        attn_evs.append((evs, mid))
         attn_bytes += decode_bytes(w, lens)
     torch.cuda.synchronize()
-    t_attn = sum(e[1].elapsed_time(mid) for e, mid in step_evs)
+    t_attn = sum(e[1].elapsed_time(mid) for e, mid in attn_evs)
     barrier(dist)
     cache.set_decode_event(None)
     assert cache.sync_status() == 0
@@ -341,8 +419,8 @@ def run_gpu(args, rank, ws, dist):
     barrier(dist)
     torch.cuda.synchronize()
     e2e_ms, e2e_bytes = 0.0, 0
-    s0 += args.steps
-    for s in range(s0, s0 + args.steps):
+    s0 += steps
+    for s in range(s0, s0 + steps):
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
         one_step(s, True, evs)
         evs[2].synchronize()
@@ -356,27 +434,27 @@ def run_gpu(args, rank, ws, dist):
     t_app = sum(r[0] for r in recs)
     t_dec = sum(r[1] for r in recs)
     step_ms = t_app + t_dec
-    mx = max_over_ranks(dist, [t_app, t_attn, t_dec, step_ms, e2e_ms])
+    mx = max_over_ranks(dist, [t_app, t_dec, step_ms, e2e_ms])
     tot = sum_over_ranks(dist, [kv_bytes, app_bytes, seq_tokens, e2e_bytes])
-    K = args.steps
-    res = {
+    K = steps
+    return {
         "w": w, "K": K, "ws": ws, "launches": launches, "clocks": clocks,
-        "kv_gbs": tot[0] / (mx[2] * 1e-3) / 1e9,
+        "kv_gbs": tot[0] / (mx[1] * 1e-3) / 1e9,
         "attn_gbs": (attn_bytes / K) / (t_attn / K * 1e-3) / 1e9,
         "attn_bytes_per_launch": attn_bytes / K,
         "attn_us": t_attn / K * 1e3,
         "decode_us": t_dec / K * 1e3,
         "append_us": t_app / K * 1e3,
         "append_gbs": tot[1] / (mx[0] * 1e-3) / 1e9,
-        "seq_tok_s": tot[2] / (mx[3] * 1e-3),
-        "ms_per_step": mx[3] / K,
-        "e2e_gbs": tot[3] / (mx[4] * 1e-3) / 1e9,
+        "seq_tok_s": tot[2] / (mx[2] * 1e-3),
+        "ms_per_step": mx[2] / K,
+        "e2e_gbs": tot[3] / (mx[3] * 1e-3) / 1e9,
         "kv_bytes_per_step": kv_bytes / K,
         "lens_final": lens,
         "h2d": B * w.h_kv * D * 2 * 2 + B * w.h_q * D * 2,
         "d2h": B * w.h_q * D * 4,
+        "bulk": bulk,
     }
-    return res
 
 
 def run_control(args):
@@ -544,6 +622,135 @@ def run_next_rows(args):
     return {"calls": K, "prefix_sharing": share, "chunked_prefill": prefill}
 
 
+def chunk_used_bytes(w, layout):
+    """Bytes a decode stage copies per page chunk: codes and metadata, without
+    the chunk's tail padding."""
+    f = w.fmt
+    es = 4 if f.scale_fp32 else 2
+    if f.bits == 16 or f.fp8:
+        meta = 0
+    elif f.k_axis:
+        meta = layout["kslice"] * es * (1 + f.asym)
+    else:
+        meta = f.page * (D // f.g_k) * es * (1 + f.asym)
+    return layout["off_kmeta"] + (meta + 15) // 16 * 16
+
+
+def run_floor(args):
+    """HBM read floor of one decode pass (kvq_read_floor): the time a single
+    launch needs just to read bytes, with no compute.  Three byte sets:
+    `paged`, the page chunks a decode call of the workload stages, in decode
+    order, at their block-table addresses (the same bytes as the decode call's
+    quantized part); `linear`, the same number of chunks back to back; and
+    contiguous buffers of 1 and 2 GB.  Two ways of reading: `bulk`, the decode
+    kernel's scheme (cp.async.bulk into per-warp stages, persistent grid of
+    four-warp CTAs) over a sweep of CTAs per SM, stages per warp and chunks
+    per unit; `stream`, 128-bit loads by every thread.  Median and best of
+    `calls` launches, L2 flushed clean before each."""
+    import torch
+    from quantized_kv_cache_14_b200 import kvq
+    dev = torch.device("cuda", torch.cuda.current_device())
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    w = workload(args.workload)
+    f = w.fmt
+    dr = Draws(w, steps=1)
+    nb = pool_blocks(dr.lengths, 2, f.page)
+    mbps = max((L + 2) // f.page + 2 for L in dr.lengths)
+    cache = kvq.KVCache(kvq.Format(f.bits, f.asym, f.k_axis, f.g_k, f.g_v, f.scale_fp32, f.residual, f.page),
+                        w.h_q, w.h_kv, max_seqs=w.batch, num_blocks=nb, max_blocks_per_seq=mbps, seed=w.seed,
+                        device=torch.cuda.current_device())
+
+    def dbf(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+    cache.append(dbf(dr.k), dbf(dr.v), dr.seq_ids)
+    torch.cuda.synchronize()
+    lay = cache.layout
+    chunk = chunk_used_bytes(w, lay)
+    offs = []
+    for i, L in enumerate(dr.lengths):
+        Lq = (L // f.residual) * f.residual if f.residual else L
+        npg = (Lq + f.page - 1) // f.page
+        tab = cache.block_table_host(i)[:npg].astype(np.int64)
+        for h in range(w.h_kv):
+            offs.append(tab * lay["block_bytes"] + h * lay["chunk_bytes"])
+    offs = torch.from_numpy(np.concatenate(offs)).to(dev)
+    n = int(offs.numel())
+    pool_ptr, pool_bytes = cache.pool_device()
+    sink = torch.zeros(2, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_rd = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    K = max(10, min(args.steps, 50))
+    smem_per_sm = torch.cuda.get_device_properties(dev).shared_memory_per_multiprocessor
+
+    def timed(fn):
+        evs = []
+        for it in range(K + 3):
+            flush.zero_()
+            flush_rd.sum()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            if it >= 3:
+                evs.append((e0, e1))
+        torch.cuda.synchronize()
+        t = [a.elapsed_time(b) * 1e3 for a, b in evs]
+        return float(np.median(t)), float(min(t))
+
+    peak, peak_kind = measured_peak()
+    rows = []
+
+    def record(kind, nbytes, mode, ctas, stages, per_unit, fn):
+        med, best = timed(fn)
+        rows.append({"bytes": kind, "nbytes": nbytes, "mode": mode, "ctas": ctas,
+                     "ctas_per_sm": ctas / sms, "stages": stages, "per_unit": per_unit,
+                     "us_median": med, "us_best": best, "gbs_median": nbytes / med / 1e3,
+                     "frac_median": nbytes / med / 1e3 / peak})
+
+    sweep = [(3, 2, 4), (3, 1, 8), (2, 3, 4), (2, 2, 8), (1, 6, 4), (1, 4, 8), (4, 1, 4), (2, 2, 4), (1, 2, 4)]
+    lin = torch.empty(n * chunk + 16, dtype=torch.uint8, device=dev)
+    lin.random_(0, 255)
+    for per_sm, S, U in sweep:
+        smem = 4 * S * ((U * chunk + 127) // 128 * 128 + 8)
+        if per_sm * (smem + 1024) > smem_per_sm:
+            continue
+        ctas = per_sm * sms
+        record("paged", n * chunk, "bulk", ctas, S, U, lambda: kvq.kvq_read_floor(
+            pool_ptr, offs.data_ptr(), n, pool_bytes, chunk, 0, ctas, S, U, sink.data_ptr(),
+            torch.cuda.current_stream().cuda_stream))
+        record("linear", n * chunk, "bulk", ctas, S, U, lambda: kvq.kvq_read_floor(
+            lin.data_ptr(), 0, n, lin.numel() // 16 * 16, chunk, 0, ctas, S, U, sink.data_ptr(),
+            torch.cuda.current_stream().cuda_stream))
+    span_lin = n * chunk // 16 * 16
+    for mult in (2, 4, 8, 16):
+        ctas = mult * sms
+        record("linear", span_lin, "stream", ctas, 0, 0, lambda: kvq.kvq_read_floor(
+            lin.data_ptr(), 0, 0, span_lin, 16, 1, ctas, 1, 1, sink.data_ptr(),
+            torch.cuda.current_stream().cuda_stream))
+    del lin
+    for gb in (1, 2):
+        big = torch.empty(gb << 30, dtype=torch.uint8, device=dev)
+        big.random_(0, 255)
+        nbig = big.numel() // chunk
+        for per_sm, S, U in ((3, 2, 4), (1, 6, 4)):
+            ctas = per_sm * sms
+            record(f"{gb}GB", nbig * chunk, "bulk", ctas, S, U, lambda: kvq.kvq_read_floor(
+                big.data_ptr(), 0, nbig, big.numel(), chunk, 0, ctas, S, U, sink.data_ptr(),
+                torch.cuda.current_stream().cuda_stream))
+        for mult in (4, 8):
+            ctas = mult * sms
+            record(f"{gb}GB", big.numel(), "stream", ctas, 0, 0, lambda: kvq.kvq_read_floor(
+                big.data_ptr(), 0, 0, big.numel(), 16, 1, ctas, 1, 1, sink.data_ptr(),
+                torch.cuda.current_stream().cuda_stream))
+        del big
+    torch.cuda.synchronize()
+    err = int(sink[1].item())
+    cache.close()
+    return {"floor": rows, "workload": w.name, "chunk_bytes": chunk, "chunks": n, "sms": sms,
+            "peak": peak, "peak_kind": peak_kind, "calls": K, "error_flags": err,
+            "l2": "flushed before every call (256 MB write then 256 MB read, untimed)"}
+
+
 # ---------------------------------------------------------------------------
 # the CPU oracle (baseline / reference arm)
 # ---------------------------------------------------------------------------
@@ -612,8 +819,15 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=0, help="rows of the CPU oracle sample")
     ap.add_argument("--no-control", action="store_true", help="skip the BF16 / FP8 comparison and the prefix-sharing and chunked-prefill measurements")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="time only --workload (skip the other four workloads' lines)")
+    ap.add_argument("--floor", action="store_true",
+                    help="measure the HBM read floor of one decode pass instead (one GPU; prints its own JSON)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.floor:
+        print(json.dumps(run_floor(args)))
+        return
 
     rank, ws, dist = dist_setup(args.gpus)
     w = workload(args.workload)
@@ -639,7 +853,15 @@ def main():
         print(json.dumps(line))
         return
 
-    res = run_gpu(args, rank, ws, dist)
+    res = run_gpu(args, rank, ws, dist, args.workload, args.steps, args.warmup,
+                  bulk_calls=0 if args.no_control else 5)
+    others = {}
+    if not args.no_workloads:
+        for widx in (1, 2, 3, 4, 5):
+            if widx == args.workload:
+                continue
+            r = run_gpu(args, rank, ws, dist, widx, max(5, min(args.steps, 20)), args.warmup)
+            others[workload(widx).name] = r
     if rank != 0:
         return
     peak, peak_kind = measured_peak()
@@ -653,6 +875,18 @@ def main():
     traffic = committed_traffic(w.name, res["attn_bytes_per_launch"])
     control = run_control(args) if (ws == 1 and not args.no_control) else None
     next_rows = run_next_rows(args) if (ws == 1 and not args.no_control) else None
+    per_workload = {}
+    for name, r in others.items():
+        per_workload[name] = {
+            "steps": r["K"], "attn_us": r["attn_us"], "decode_us": r["decode_us"], "kv_gbs": r["kv_gbs"],
+            "frac": r["attn_gbs"] / peak, "kv_bytes_per_step": r["kv_bytes_per_step"],
+            "e2e_gbs": r["e2e_gbs"], "append_us": r["append_us"], "append_gbs": r["append_gbs"],
+            "seq_tokens_per_s": r["seq_tok_s"], "clocks": r["clocks"],
+            "config": workload_config(r["w"], r["lens_final"])["workload"],
+        }
+    bulk = res["bulk"]
+    if bulk is not None:
+        bulk["frac"] = bulk["gbs"] / peak
     line = {
         "metric": "decode-attn KV GB/s", "value": res["kv_gbs"], "unit": "GB/s",
         "n_gpus": ws, "steps": res["K"], "warmup": args.warmup,
@@ -661,7 +895,8 @@ def main():
         "config": workload_config(w, res["lens_final"]),
         "roofline": {"bound": "hbm", "achieved": res["attn_gbs"], "peak": peak, "unit": "GB/s",
                      "frac": res["attn_gbs"] / peak, "traffic": traffic,
-                     "peak_kind": peak_kind, "kernel": "decode_kernel (attention, without the merge)"},
+                     "peak_kind": peak_kind,
+                     "kernel": "decode_kernel (attention, without the merge)"},
         "cpu_baseline": cpu,
         "e2e": {"value": res["e2e_gbs"], "unit": "GB/s", "h2d_bytes_per_step": res["h2d"],
                 "d2h_bytes_per_step": res["d2h"]},
@@ -669,10 +904,12 @@ def main():
         "clocks": res["clocks"],
         "seq_tokens_per_s": res["seq_tok_s"],
         "append_gbs": res["append_gbs"],
+        "bulk_append": bulk,
         "attn_us": res["attn_us"], "decode_us": res["decode_us"], "append_us": res["append_us"],
         "kv_bytes_per_step": res["kv_bytes_per_step"],
         "frac_of_8TBps": res["kv_gbs"] / 8000.0,
         "frac_of_peak": res["kv_gbs"] / peak,
+        "workloads": per_workload,
         "bf16_control": control,
         "next_rows": next_rows,
     }

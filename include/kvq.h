@@ -95,7 +95,9 @@ enum { KVQ_AXIS_TOKEN = 0, KVQ_AXIS_CHANNEL = 1 };
  *               from its front and freed blocks return to its back.
  *   fail_alloc_after  test hook: allocation number k (0-based, cumulative)
  *               fails when k >= fail_alloc_after; -1 disables it.
- *   host_only   1: no device memory and no kernels (host bookkeeping only;
+ *   host_only   1: no device memory and no kernels (host bookkeeping only,
+ *               for tests on machines without a GPU).
+ *   device      CUDA device ordinal (ignored when host_only).
  *   fp8         1: the FP8 (E4M3) format, the oh-bug.com page's engineering
  *               baseline ("FP8 / INT8: Engineering Baseline"): each element is
  *               e4m3(x / s) (round to nearest even, saturating at +-448) with
@@ -104,9 +106,7 @@ enum { KVQ_AXIS_TOKEN = 0, KVQ_AXIS_CHANNEL = 1 };
  *               Needs bits 8, asym 0, k_axis 0, residual 0, scale_fp32 0,
  *               g_k = g_v = 128.  Key rows keep the key-list order with bytes in
  *               natural order; value lane records hold each operand register's
- *               two tokens in adjacent bytes.  0 otherwise.
- *               for tests on machines without a GPU).
- *   device      CUDA device ordinal (ignored when host_only). */
+ *               two tokens in adjacent bytes.  0 otherwise. */
 typedef struct kvq_config {
   int32_t bits;
   int32_t asym;
@@ -197,8 +197,10 @@ kvq_status kvq_append(kvq_handle h, const void* k_bf16, const void* v_bf16,
  *   seq_ids_host host int32 [batch] mapping rows to sequence ids, or NULL for
  *               row i = sequence i.
  *   out         device fp32 [batch][h_q][d_h]; empty rows give zeros.
- * The library's split-K partials live in its workspace; one call at a time per
- * handle may be in flight on the GPU.
+ * The key range of every (row, kv head) is split over a persistent grid; a
+ * second kernel merges the split partials by log-sum-exp.  The partials live
+ * in the handle's workspace; one call at a time per handle may be in flight
+ * on the GPU.
  * Errors: KVQ_ERR_INVALID_ARG, KVQ_ERR_BAD_SEQ, KVQ_ERR_CUDA. */
 kvq_status kvq_decode_attn(kvq_handle h, const void* q_bf16,
                            const int32_t* block_table, int32_t bt_stride,
@@ -215,7 +217,13 @@ kvq_status kvq_decode_attn(kvq_handle h, const void* q_bf16,
  *   3. the output comes back to out_host (host fp32 [batch][h_q][d_h]).
  * out_host holds the result once the stream reaches that point.  Page-locked
  * host buffers let the copies run asynchronously; pageable ones work with the
- * copy semantics CUDA gives them.  n = 0 skips the append, batch = 0 the decode.
+ * copy semantics CUDA gives them.  When k_host, v_host and q_host lie back to
+ * back in host memory (v right after the n K rows, q right after the n V rows)
+ * the step issues one host-to-device copy instead of three; when out_host is
+ * page-locked memory the device can address (cudaPointerGetAttributes gives a
+ * device pointer), the decode kernel writes the output there directly instead
+ * of a device buffer plus a device-to-host copy.  n = 0 skips the append,
+ * batch = 0 the decode.
  * The device buffers grow on demand (a device synchronize, then a reallocation)
  * and live until kvq_destroy; the host buffers stay the caller's and must
  * stay valid until the stream has reached the end of the step.
@@ -301,6 +309,41 @@ kvq_status kvq_read_residual(kvq_handle h, void* k_host, void* v_host, uint64_t 
  * check fired, KVQ_ERR_CUDA on a CUDA error, else KVQ_OK. */
 kvq_status kvq_sync_status(kvq_handle h, void* stream, uint32_t* bits_out);
 
+/* Library-owned device view of the block pool: *dev_ptr receives its address
+ * and *bytes its size (num_blocks * block_bytes).  Valid until kvq_destroy;
+ * for measurement (kvq_read_floor over the pages a decode reads) and
+ * debugging.  KVQ_ERR_INVALID_ARG for a host-only handle. */
+kvq_status kvq_pool_device(kvq_handle h, const void** dev_ptr, uint64_t* bytes);
+
+/* Measurement hook: the HBM read floor of a decode pass.  Decode over a
+ * compressed cache is meant to be bound by memory traffic (llmdaily.org
+ * day-65, "Why compression may also improve speed"); this call reads bytes
+ * and does nothing else with them, so its device time is the floor a single
+ * launch can reach for the same bytes and the same way of reading.
+ *   base        device, 16-byte aligned; span_bytes (a multiple of 16)
+ *               readable bytes from it.
+ *   mode 0      bulk: a grid of `ctas` CTAs of four warps; each CTA takes a
+ *               contiguous share of the chunk list and each warp every fourth
+ *               unit of `per_unit` chunks (1..32), copying it with
+ *               cp.async.bulk into one of its `stages` (1..16) shared-memory
+ *               stages, as the decode kernel stages pages.  Chunk i is
+ *               chunk_bytes (a multiple of 16, <= 65536) at base + offsets[i]
+ *               (offsets: device int64 [n_chunks]) or, with offsets NULL, at
+ *               base + i * chunk_bytes.
+ *   mode 1      stream: 256-thread CTAs read [base, base + span_bytes) with
+ *               128-bit loads, eight in flight per thread (chunk arguments
+ *               ignored).
+ *   sink        device uint32 [2]: sink[0] receives an XOR checksum of one
+ *               word per chunk (mode 0) or of every word (mode 1); sink[1]
+ *               gets bit 0 for an offset that is negative, unaligned or past
+ *               span_bytes (that unit is skipped) and bit 1 for a copy wait
+ *               that gave up after 2 s.  Neither is cleared by the call.
+ * Asynchronous on `stream`.  KVQ_ERR_INVALID_ARG for out-of-range arguments or
+ * stages that do not fit in shared memory. */
+kvq_status kvq_read_floor(const void* base, const int64_t* offsets, int64_t n_chunks, int64_t span_bytes,
+                          int32_t chunk_bytes, int32_t mode, int32_t ctas, int32_t stages,
+                          int32_t per_unit, uint32_t* sink, void* stream);
+
 /* Overrides the decode kernel's grid (number of CTAs); 0 restores the default
  * (one resident wave on every SM).  Changes how the key range is split across
  * CTAs, never the result beyond rounding. */
@@ -321,7 +364,8 @@ kvq_status kvq_set_decode_event(kvq_handle h, void* event);
  * (split-K partials, tile prefix, error word) is a fixed 16 MiB array in the
  * library's device image, held by every GPU that loads the library until the
  * process exits; calls size-check against it and never call cudaMalloc,
- * cudaFree or an allocating library routine.
+ * cudaFree or an allocating library routine.  Each call clears the array's
+ * error word with cudaMemsetAsync (no allocation).
  *   cfg          format and capacity; max_seqs bounds batch.  Not a handle.
  *   pool         device, num_blocks * block_bytes in the kvq_layout format.
  *   k_window, v_window  device bf16 [batch][h_kv][residual][d_h] BF16 windows
@@ -333,11 +377,14 @@ kvq_status kvq_set_decode_event(kvq_handle h, void* event);
  *   q_bf16, out  as in kvq_decode_attn (row i uses window row i).
  *   error_bits_dev  optional device uint32: receives this call's device
  *                check bits (KVQ_DEVERR_*), 0 if none fired.
- * Runs on the current CUDA device.  The first call on a device looks up the
- * scratch array's device address (cudaGetSymbolAddress) and sets the decode
- * kernel's shared-memory limit; make that first call before any stream
- * capture.  All calls share the one array and it keeps the last call's
- * contents: calls whose work can overlap on the GPU (different streams
+ * Runs on the current CUDA device.  Every call looks up the scratch array's
+ * device address in the current context (cudaGetSymbolAddress).  The first
+ * call for a (device, format, max_seqs) sizes the decode pipeline, queries
+ * residency and may raise the decode kernel's shared-memory limit (the limit
+ * only ever rises, so a small plan never breaks a handle planned for a larger
+ * batch); later calls reuse that plan.  Make that first call before any
+ * stream capture.  All calls share the one array and it keeps the last
+ * call's contents: calls whose work can overlap on the GPU (different streams
  * without ordering) race on it.  Returns KVQ_ERR_INVALID_ARG with a message
  * giving both sizes when batch * h_kv needs more scratch than the array holds;
  * KVQ_ERR_UNSUPPORTED for the FP8 format (its per-head scales live in a handle).

@@ -713,13 +713,10 @@ int32_t orc_free_seq(void* hh, int32_t s) {
   return 0;
 }
 
-// Prefix sharing (day-65 page, "How this connects to paging and prefix
-// caching"): the empty sequence dst starts with the first `tokens` tokens of
-// src by holding src's blocks too.  Only whole blocks that no append writes
-// again are shared: tokens a multiple of the page (no window) or of the window
-// length R = g_k (whole key groups).  Returns 0; 3 for bad ids; 4 for dst not
-// empty, dst == src, tokens out of [0, len(src)] or not aligned; 2 when dst's
-// table row is too short.  No state change on error.
+// FP8 scales (oh-bug.com, "FP8 / INT8: Engineering Baseline"): one per kv
+// head for keys and one for values, set before the first append.  Returns 0;
+// 4 for a cache not in the FP8 format, a non-empty cache or a scale that is
+// not positive and finite.
 int32_t orc_set_fp8_scales(void* hh, const float* k, const float* v) {
   Cache& C = *static_cast<Cache*>(hh);
   if (!C.c.fp8) return 4;
@@ -732,6 +729,13 @@ int32_t orc_set_fp8_scales(void* hh, const float* k, const float* v) {
   return 0;
 }
 
+// Prefix sharing (day-65 page, "How this connects to paging and prefix
+// caching"): the empty sequence dst starts with the first `tokens` tokens of
+// src by holding src's blocks too.  Only whole blocks that no append writes
+// again are shared: tokens a multiple of the page (no window) or of the window
+// length R = g_k (whole key groups).  Returns 0; 3 for bad ids; 4 for dst not
+// empty, dst == src, tokens out of [0, len(src)] or not aligned; 2 when dst's
+// table row is too short.  No state change on error.
 int32_t orc_share_prefix(void* hh, int32_t src, int32_t dst, int32_t tokens) {
   Cache& C = *static_cast<Cache*>(hh);
   const Cfg& c = C.c;

@@ -31,6 +31,8 @@
 //    per 64 tokens.  Each warp leaves one (m, l, o) record per pair its CTA
 //    touched; the merge kernel combines them by log-sum-exp in a fixed order.
 #include <cstdint>
+#include <mutex>
+#include <vector>
 
 #include "kvq_device.cuh"
 #include "kvq_tiles.cuh"
@@ -1153,6 +1155,31 @@ size_t decode_partials_bytes(const Geo& g, int B, int grid) {
   return (size_t(B) * g.h_kv + size_t(grid)) * kDecodeWarps * g.G * (kD + 2) * sizeof(float);
 }
 
+// The dynamic shared-memory limit is an attribute of the kernel on a device,
+// shared by every handle and every allocation-free call.  Plans for different
+// batch sizes need different amounts, so the limit only ever rises: lowering
+// it for a small plan would make a live plan's larger launches fail.
+static cudaError_t raise_smem_limit(int dev, const void* kern, size_t smem) {
+  struct Entry {
+    int dev;
+    const void* kern;
+    size_t smem;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> set;
+  std::lock_guard<std::mutex> lock(mu);
+  for (Entry& en : set)
+    if (en.dev == dev && en.kern == kern) {
+      if (smem <= en.smem) return cudaSuccess;
+      const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+      if (e == cudaSuccess) en.smem = smem;
+      return e;
+    }
+  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e == cudaSuccess) set.push_back({dev, kern, smem});
+  return e;
+}
+
 cudaError_t plan_decode(const Geo& g, int max_B, DecodePipe* out) {
   DecodePipe p{};
   p.sup = g.bits == 16 ? 16 : g.k_axis ? (g.g_k > 64 ? g.g_k : 64) : 64;
@@ -1185,7 +1212,7 @@ cudaError_t plan_decode(const Geo& g, int max_B, DecodePipe* out) {
   const size_t smem = size_t(smem_layout(max_B, p).total);
   if (smem > size_t(max_optin)) return cudaErrorInvalidConfiguration;
   const void* kern = decode_kernel_ptr(g);
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  e = raise_smem_limit(dev, kern, smem);
   if (e != cudaSuccess) return e;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&p.ctas_per_sm, kern, kDecodeThreads, smem);
   if (e != cudaSuccess) return e;

@@ -156,6 +156,14 @@ size_t decode_partials_bytes(const Geo& g, int B, int grid);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s, cudaEvent_t between, int* launches);
 constexpr int kMaxDecodeGrid = 1024;
 
+// HBM read-floor measurement kernels (kvq_floor.cu).  mode 0: bulk copies of
+// chunks into per-warp shared-memory stages; mode 1: a 128-bit load stream
+// over [base, base + span).
+size_t floor_smem_bytes(int chunk_bytes, int per_unit, int stages);
+cudaError_t launch_floor(const void* base, const int64_t* offsets, int64_t n_chunks, int64_t span,
+                         int chunk_bytes, int mode, int ctas, int stages, int per_unit, uint32_t* sink,
+                         cudaStream_t s);
+
 // Fixed decode scratch of kvq_decode_attn_noalloc (kvq_noalloc.cu).
 size_t noalloc_scratch_bytes();
 cudaError_t noalloc_scratch(void** out);

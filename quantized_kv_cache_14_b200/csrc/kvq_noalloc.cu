@@ -8,7 +8,6 @@
 // device array instead of handle-owned memory.  Every GPU that loads the
 // library keeps this array until the process exits.
 #include <cstddef>
-#include <mutex>
 
 #include <cuda_runtime.h>
 
@@ -21,30 +20,20 @@ constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB per device
 
 __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
-
 }  // namespace
 
 size_t noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
 
-// Device address of the scratch array on the current device.  The first call
-// on a device looks it up with cudaGetSymbolAddress (host code cannot use the
-// array's name as a device address); later calls reuse the cached pointer.
+// Device address of the scratch array in the current context.  Host code
+// cannot use the array's name as a device address, so every call looks it up
+// with cudaGetSymbolAddress: the lookup is cheap, and it stays right when the
+// context is torn down and rebuilt (the module then loads again and the array
+// may move).
 cudaError_t noalloc_scratch(void** out) {
-  int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_decode_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_ptr[dev] = p;
-  }
-  *out = g_scratch_ptr[dev];
+  *out = p;
   return cudaSuccess;
 }
 

@@ -11,6 +11,7 @@
 #include <cstdio>
 #include <cstring>
 #include <deque>
+#include <mutex>
 #include <string>
 #include <unordered_set>
 #include <vector>
@@ -191,9 +192,7 @@ struct kvq_handle_s {
   cudaEvent_t decode_event = nullptr;
   int launches = 0;
   // device staging of kvq_step_host: new K/V rows, q, output (grown on demand)
-  uint16_t* d_kin = nullptr;
-  uint16_t* d_vin = nullptr;
-  uint16_t* d_qin = nullptr;
+  uint8_t* d_in = nullptr;   // one buffer: a call's K rows, V rows and q, back to back
   float* d_out = nullptr;
   int32_t io_rows = 0;    // K/V rows the staging holds
   int32_t io_batch = 0;   // q / output rows the staging holds
@@ -340,9 +339,7 @@ void destroy_device(kvq_handle h) {
   cudaFree(h->d_seqmap);
   cudaFree(h->d_rowlen);
   cudaFree(h->d_fp8);
-  cudaFree(h->d_kin);
-  cudaFree(h->d_vin);
-  cudaFree(h->d_qin);
+  cudaFree(h->d_in);
   cudaFree(h->d_out);
   cudaFree(h->d_pfplan);
   cudaFree(h->d_pfpart);
@@ -656,16 +653,13 @@ kvq_status ensure_io(kvq_handle h, int32_t rows, int32_t batch) {
   const int32_t r = std::max(rows, h->io_rows), b = std::max(batch, h->io_batch);
   const kvq_config& c = h->cfg;
   const size_t kv = size_t(r) * c.h_kv * c.d_h, qo = size_t(b) * c.h_q * c.d_h;
-  for (void* p : {static_cast<void*>(h->d_kin), static_cast<void*>(h->d_vin), static_cast<void*>(h->d_qin),
-                  static_cast<void*>(h->d_out)})
-    if (p) KVQ_CUDA(cudaFree(p));
-  h->d_kin = h->d_vin = h->d_qin = nullptr;
+  if (h->d_in) KVQ_CUDA(cudaFree(h->d_in));
+  if (h->d_out) KVQ_CUDA(cudaFree(h->d_out));
+  h->d_in = nullptr;
   h->d_out = nullptr;
   h->bytes_workspace -= (size_t(h->io_rows) * c.h_kv * c.d_h * 4 + size_t(h->io_batch) * c.h_q * c.d_h * 6);
   h->io_rows = h->io_batch = 0;
-  KVQ_CUDA(cudaMalloc(&h->d_kin, std::max<size_t>(kv, 1) * 2));
-  KVQ_CUDA(cudaMalloc(&h->d_vin, std::max<size_t>(kv, 1) * 2));
-  KVQ_CUDA(cudaMalloc(&h->d_qin, std::max<size_t>(qo, 1) * 2));
+  KVQ_CUDA(cudaMalloc(&h->d_in, std::max<size_t>(2 * kv + qo, 1) * 2));
   KVQ_CUDA(cudaMalloc(&h->d_out, std::max<size_t>(qo, 1) * 4));
   h->io_rows = r;
   h->io_batch = b;
@@ -693,17 +687,44 @@ kvq_status kvq_step_host(kvq_handle h, const void* k_host, const void* v_host, c
   if (st != KVQ_OK) return st;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   const size_t kv_bytes = size_t(n) * c.h_kv * c.d_h * 2, q_bytes = size_t(batch) * c.h_q * c.d_h * 2;
+  // this call's rows back to back in the device staging: K | V | q
+  uint8_t* d_k = h->d_in;
+  uint8_t* d_v = d_k + kv_bytes;
+  uint8_t* d_q = d_v + kv_bytes;
+  const uint8_t* hk = static_cast<const uint8_t*>(k_host);
+  const uint8_t* hv = static_cast<const uint8_t*>(v_host);
+  const uint8_t* hq = static_cast<const uint8_t*>(q_host);
+  // a caller whose k, v and q are back to back in host memory gets one copy
+  const bool packed = n > 0 && batch > 0 && hv == hk + kv_bytes && hq == hv + kv_bytes;
+  if (packed) {
+    KVQ_CUDA(cudaMemcpyAsync(d_k, hk, 2 * kv_bytes + q_bytes, cudaMemcpyHostToDevice, stream));
+  } else {
+    if (n > 0) {
+      KVQ_CUDA(cudaMemcpyAsync(d_k, hk, kv_bytes, cudaMemcpyHostToDevice, stream));
+      KVQ_CUDA(cudaMemcpyAsync(d_v, hv, kv_bytes, cudaMemcpyHostToDevice, stream));
+    }
+    if (batch > 0) KVQ_CUDA(cudaMemcpyAsync(d_q, hq, q_bytes, cudaMemcpyHostToDevice, stream));
+  }
   if (n > 0) {
-    KVQ_CUDA(cudaMemcpyAsync(h->d_kin, k_host, kv_bytes, cudaMemcpyHostToDevice, stream));
-    KVQ_CUDA(cudaMemcpyAsync(h->d_vin, v_host, kv_bytes, cudaMemcpyHostToDevice, stream));
-    st = kvq_append(h, h->d_kin, h->d_vin, seq_ids_host, n, stream_);
+    st = kvq_append(h, d_k, d_v, seq_ids_host, n, stream_);
     if (st != KVQ_OK) return st;
   }
   if (batch == 0) return KVQ_OK;
-  KVQ_CUDA(cudaMemcpyAsync(h->d_qin, q_host, q_bytes, cudaMemcpyHostToDevice, stream));
-  st = launch_handle_decode(h, h->d_qin, nullptr, 0, h->d_len, nullptr, batch, h->d_out, stream);
+  // page-locked output the device can write (mapped pinned memory) takes the
+  // attention output straight from the decode kernel; else one D2H copy
+  cudaPointerAttributes pa{};
+  float* d_out = h->d_out;
+  bool direct = false;
+  if (cudaPointerGetAttributes(&pa, out_host) == cudaSuccess && pa.type == cudaMemoryTypeHost &&
+      pa.devicePointer != nullptr && aligned16(pa.devicePointer)) {
+    d_out = static_cast<float*>(pa.devicePointer);
+    direct = true;
+  } else {
+    (void)cudaGetLastError();   // an unregistered host pointer is not an error here
+  }
+  st = launch_handle_decode(h, d_q, nullptr, 0, h->d_len, nullptr, batch, d_out, stream);
   if (st != KVQ_OK) return st;
-  KVQ_CUDA(cudaMemcpyAsync(out_host, h->d_out, q_bytes * 2, cudaMemcpyDeviceToHost, stream));
+  if (!direct) KVQ_CUDA(cudaMemcpyAsync(out_host, h->d_out, q_bytes * 2, cudaMemcpyDeviceToHost, stream));
   return KVQ_OK;
 }
 
@@ -1053,12 +1074,99 @@ kvq_status kvq_set_decode_event(kvq_handle h, void* event) {
   return KVQ_OK;
 }
 
+kvq_status kvq_pool_device(kvq_handle h, const void** dev_ptr, uint64_t* bytes) {
+  if (!h || !dev_ptr || !bytes) return fail(KVQ_ERR_INVALID_ARG, "null argument");
+  if (h->cfg.host_only) return fail(KVQ_ERR_INVALID_ARG, "handle is host-only");
+  *dev_ptr = h->d_pool;
+  *bytes = uint64_t(h->cfg.num_blocks) * uint64_t(h->geo.block_bytes);
+  return KVQ_OK;
+}
+
+kvq_status kvq_read_floor(const void* base, const int64_t* offsets, int64_t n_chunks, int64_t span_bytes,
+                          int32_t chunk_bytes, int32_t mode, int32_t ctas, int32_t stages, int32_t per_unit,
+                          uint32_t* sink, void* stream_) {
+  if (!base || !sink) return fail(KVQ_ERR_INVALID_ARG, "base and sink are required");
+  if (!aligned16(base) || (reinterpret_cast<uintptr_t>(sink) & 3u))
+    return fail(KVQ_ERR_INVALID_ARG, "base must be 16-byte aligned and sink 4-byte aligned");
+  if (mode != 0 && mode != 1) return fail(KVQ_ERR_INVALID_ARG, "mode must be 0 (bulk) or 1 (stream)");
+  if (ctas < 1 || ctas > 65535) return fail(KVQ_ERR_INVALID_ARG, "ctas must be in [1, 65535]");
+  if (span_bytes < 0 || span_bytes % 16) return fail(KVQ_ERR_INVALID_ARG, "span_bytes must be a non-negative multiple of 16");
+  if (mode == 0) {
+    if (chunk_bytes < 16 || chunk_bytes > 65536 || chunk_bytes % 16)
+      return fail(KVQ_ERR_INVALID_ARG, "chunk_bytes must be a multiple of 16 in [16, 65536]");
+    if (per_unit < 1 || per_unit > 32) return fail(KVQ_ERR_INVALID_ARG, "per_unit must be in [1, 32]");
+    if (stages < 1 || stages > 16) return fail(KVQ_ERR_INVALID_ARG, "stages must be in [1, 16]");
+    if (n_chunks < 0) return fail(KVQ_ERR_INVALID_ARG, "n_chunks must be >= 0");
+    if (!offsets && n_chunks * int64_t(chunk_bytes) > span_bytes)
+      return fail(KVQ_ERR_INVALID_ARG, "n_chunks * chunk_bytes exceeds span_bytes");
+    int dev = 0, optin = 0;
+    KVQ_CUDA(cudaGetDevice(&dev));
+    KVQ_CUDA(cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
+    if (kvq::floor_smem_bytes(chunk_bytes, per_unit, stages) > size_t(optin))
+      return fail(KVQ_ERR_INVALID_ARG, "stages * per_unit * chunk_bytes does not fit in shared memory");
+  }
+  KVQ_CUDA(kvq::launch_floor(base, offsets, n_chunks, span_bytes, chunk_bytes, mode, ctas, stages, per_unit, sink,
+                             static_cast<cudaStream_t>(stream_)));
+  return KVQ_OK;
+}
+
 kvq_status kvq_set_decode_grid(kvq_handle h, int32_t ctas) {
   if (!h) return fail(KVQ_ERR_INVALID_ARG, "handle is null");
   if (ctas < 0 || ctas > kvq::kMaxDecodeGrid) return fail(KVQ_ERR_INVALID_ARG, "ctas must be in [0, 1024]");
   h->decode_override = ctas;
   return KVQ_OK;
 }
+
+}  // extern "C"
+
+namespace {
+
+// Decode plans of kvq_decode_attn_noalloc, one per (device, format, max_seqs):
+// the first call for a key sizes the pipeline and queries residency, later
+// calls reuse the result.
+struct NoallocPlan {
+  int dev, max_seqs;
+  kvq_config fmt;
+  kvq::DecodePipe pipe;
+  int grid;
+};
+
+bool same_format(const kvq_config& a, const kvq_config& b) {
+  return a.bits == b.bits && a.asym == b.asym && a.k_axis == b.k_axis && a.g_k == b.g_k && a.g_v == b.g_v &&
+         a.scale_fp32 == b.scale_fp32 && a.residual == b.residual && a.page == b.page && a.h_q == b.h_q &&
+         a.h_kv == b.h_kv && a.d_h == b.d_h && a.num_blocks == b.num_blocks && a.fp8 == b.fp8;
+}
+
+kvq_status noalloc_plan(int dev, const kvq::Geo& g, int max_seqs, kvq::DecodePipe* pipe, int* grid) {
+  static std::mutex mu;
+  static std::vector<NoallocPlan> plans;
+  kvq_config key{};
+  key.bits = g.bits; key.asym = g.asym; key.k_axis = g.k_axis; key.g_k = g.g_k; key.g_v = g.g_v;
+  key.scale_fp32 = g.scale_fp32; key.residual = g.R; key.page = g.P; key.h_q = g.h_q; key.h_kv = g.h_kv;
+  key.d_h = kvq::kD; key.num_blocks = g.num_blocks; key.fp8 = g.fp8;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const NoallocPlan& p : plans)
+    if (p.dev == dev && p.max_seqs == max_seqs && same_format(p.fmt, key)) {
+      *pipe = p.pipe;
+      *grid = p.grid;
+      return KVQ_OK;
+    }
+  int sms = 0;
+  KVQ_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  kvq::DecodePipe pp{};
+  const cudaError_t pe = kvq::plan_decode(g, max_seqs, &pp);
+  if (pe == cudaErrorInvalidConfiguration) return fail(KVQ_ERR_UNSUPPORTED, "decode tile does not fit on this device");
+  KVQ_CUDA(pe);
+  const int gr = std::min(sms * pp.ctas_per_sm, kvq::kMaxDecodeGrid);
+  plans.push_back({dev, max_seqs, key, pp, gr});
+  *pipe = pp;
+  *grid = gr;
+  return KVQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
 
 // Decode over caller-owned buffers with the library's fixed scratch array:
 // allocates nothing (see include/kvq.h).
@@ -1081,14 +1189,12 @@ kvq_status kvq_decode_attn_noalloc(const kvq_config* cfg, const void* pool, cons
   const kvq::Geo g = make_geo(*cfg);
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
 
-  int dev = 0, sms = 0;
+  int dev = 0;
   KVQ_CUDA(cudaGetDevice(&dev));
-  KVQ_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
   kvq::DecodePipe pipe{};
-  cudaError_t pe = kvq::plan_decode(g, cfg->max_seqs, &pipe);
-  if (pe == cudaErrorInvalidConfiguration) return fail(KVQ_ERR_UNSUPPORTED, "decode tile does not fit on this device");
-  KVQ_CUDA(pe);
-  const int grid = std::min(sms * pipe.ctas_per_sm, kvq::kMaxDecodeGrid);
+  int grid = 0;
+  st = noalloc_plan(dev, g, cfg->max_seqs, &pipe, &grid);
+  if (st != KVQ_OK) return st;
 
   // scratch layout: [error word | pad to 256][prefix (batch + 1) | pad to 256][partials]
   const size_t off_prefix = 256;

@@ -41,6 +41,7 @@ EXPORTS = (
     "kvq_stats", "kvq_cache_bytes", "kvq_layout", "kvq_read_pool", "kvq_read_residual",
     "kvq_sync_status", "kvq_set_decode_grid", "kvq_set_decode_event", "kvq_decode_attn_noalloc",
     "kvq_prefill_attn", "kvq_set_fp8_scales", "kvq_step_host", "kvq_last_error",
+    "kvq_pool_device", "kvq_read_floor",
 )
 
 
@@ -112,6 +113,8 @@ def lib():
             "kvq_decode_attn_noalloc": (st, [ctypes.POINTER(KvqConfig), P, P, P, P, I32, P, P, P, I32,
                                              P, P, P]),
             "kvq_last_error": (ctypes.c_char_p, []),
+            "kvq_pool_device": (st, [P, ctypes.POINTER(P), ctypes.POINTER(U64)]),
+            "kvq_read_floor": (st, [P, P, ctypes.c_int64, ctypes.c_int64, I32, I32, I32, I32, I32, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -287,6 +290,22 @@ def kvq_decode_attn_noalloc(cfg: KvqConfig, pool_ptr: int, k_window_ptr: int, v_
                                          V(out_ptr), V(error_bits_ptr or None), V(stream)))
 
 
+def kvq_pool_device(h):
+    """(device address, bytes) of the handle's block pool."""
+    p, n = ctypes.c_void_p(), ctypes.c_uint64()
+    _check(lib().kvq_pool_device(h, ctypes.byref(p), ctypes.byref(n)))
+    return p.value, n.value
+
+
+def kvq_read_floor(base_ptr: int, offsets_ptr: int, n_chunks: int, span_bytes: int, chunk_bytes: int,
+                   mode: int, ctas: int, stages: int, per_unit: int, sink_ptr: int, stream: int = 0):
+    """The HBM read-floor measurement kernel (device pointers as ints)."""
+    V = ctypes.c_void_p
+    _check(lib().kvq_read_floor(V(base_ptr), V(offsets_ptr or None), int(n_chunks), int(span_bytes),
+                                int(chunk_bytes), int(mode), int(ctas), int(stages), int(per_unit),
+                                V(sink_ptr), V(stream)))
+
+
 def kvq_last_error() -> str:
     return lib().kvq_last_error().decode()
 
@@ -410,6 +429,9 @@ class KVCache:
 
     def stats(self):
         return kvq_stats(self.h)
+
+    def pool_device(self):
+        return kvq_pool_device(self.h)
 
     def set_decode_grid(self, ctas):
         kvq_set_decode_grid(self.h, ctas)

@@ -55,3 +55,14 @@ def test_algorithmic_bytes_of_the_int4_workload():
     assert 16 * 8192 * 8 * 136 == 142_606_336
     # 63 window tokens are bf16 rows of K and V
     assert bench.decode_bytes(w, [8192 + 63]) - b == 63 * 8 * 2 * 128 * 2
+
+
+def test_bulk_append_bytes_of_the_int4_workload():
+    import bench
+    from quantized_kv_cache_14_b200.workloads import workload
+    w = workload(3)
+    # 8192 + 17 tokens: every K and V row read once (8 heads x 128 bf16), the
+    # 8192 tokens of whole key groups written as codes + scales (136 B per
+    # token-head), the 17 window tokens written as bf16 K and V rows
+    row = 8 * 128 * 2
+    assert bench.bulk_append_bytes(w, [8192 + 17]) == 2 * row * (8192 + 17) + 8192 * 8 * 136 + 2 * row * 17
