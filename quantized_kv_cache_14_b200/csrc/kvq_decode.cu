@@ -158,7 +158,9 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, vol
 struct State {
   float o[8][4];     // channel tile i: (ch 16i+gq | +8) x (head tq hi | lo)
   float zacc[8];     // asymmetric values: p-weighted zero-point sums per tile
+  float zc[2][4];    // INT4 KIVI subnormal path: value offset terms per value group
   float m, l;        // running max (log2 domain) and partial sum, head tq
+  bool raw;          // o holds subnormal-path sums not yet normalised
 };
 
 __device__ __forceinline__ void state_reset(State& st) {
@@ -168,8 +170,13 @@ __device__ __forceinline__ void state_reset(State& st) {
     for (int c = 0; c < 4; ++c) st.o[i][c] = 0.0f;
     st.zacc[i] = 0.0f;
   }
+#pragma unroll
+  for (int gi = 0; gi < 2; ++gi)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) st.zc[gi][c] = 0.0f;
   st.m = -INFINITY;
   st.l = 0.0f;
+  st.raw = false;
 }
 
 // Where one 16-token sub-tile sits in a stage.
@@ -468,7 +475,26 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
     return down;
   };
 
+  // subnormal-path sums -> ordinary sums: drop the offset terms, undo the
+  // 2^-24 (rows gq) and 2^-20 (rows gq + 8) scales
+  auto normalize = [&]() {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int gi = i >> 2;
+      st.o[i][0] = (st.o[i][0] - st.zc[gi][0]) * 16777216.0f;
+      st.o[i][1] = (st.o[i][1] - st.zc[gi][1]) * 16777216.0f;
+      st.o[i][2] = (st.o[i][2] - st.zc[gi][2]) * 1048576.0f;
+      st.o[i][3] = (st.o[i][3] - st.zc[gi][3]) * 1048576.0f;
+    }
+#pragma unroll
+    for (int gi = 0; gi < 2; ++gi)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) st.zc[gi][c] = 0.0f;
+    st.raw = false;
+  };
+
   auto emit = [&](int row, int h) {
+    if (SPEC && st.raw) normalize();
     float l = st.l;
     l += __shfl_xor_sync(0xffffffffu, l, 4);
     l += __shfl_xor_sync(0xffffffffu, l, 8);
@@ -562,7 +588,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
   // this lane's score B operand.  Each lane scales 4 channels of every head and
   // writes both bf16 parts into the warp's buffer in operand order (16-byte
   // slots XOR-swizzled so the four 16-byte reads per lane are conflict-free).
-  auto qprime_job = [&](const uint8_t* stg, int gi) {
+  auto qprime_job = [&](const uint8_t* stg, int gi, bool b0x16 = false) {
     const int f = 4 * lane;
     const int lg_ppg = g.lg_gk - g.lg_P;   // pages per key group, log2
     const uint8_t* km = stg + ((gi << lg_ppg) + (f >> g.lg_kslice)) * g.chunk_used + g.off_Km;
@@ -612,7 +638,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
       const __half2 s01 = *reinterpret_cast<const __half2*>(&sr.x), s23 = *reinterpret_cast<const __half2*>(&sr.y);
 #pragma unroll
       for (int h2 = 0; h2 < 4; ++h2) {
-        const __half2 qa = *reinterpret_cast<const __half2*>(&qh[h2][0]);
+        // key-list positions 4L, 4L + 1 feed the b0 register of the score
+        // product; the subnormal path wants them 16 times larger (exact)
+        const __half2 qa = b0x16 ? __hmul2(*reinterpret_cast<const __half2*>(&qh[h2][0]), __float2half2_rn(16.0f))
+                                 : *reinterpret_cast<const __half2*>(&qh[h2][0]);
         const __half2 qb = *reinterpret_cast<const __half2*>(&qh[h2][1]);
         const __half2 ha = __hmul2(qa, s01), hb = __hmul2(qb, s23);
         const __half2 la = __hfma2(qa, s01, __hneg2(ha)), lb = __hfma2(qb, s23, __hneg2(hb));
@@ -679,7 +708,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
 
   // Scores of one 16-token quantized sub-tile: tokens gq, gq + 8 for head tq,
   // scaled into the log2 domain; positions at or past `valid` are -inf.
-  auto score_sub = [&](const Sub& sb, int valid, float& s0, float& s1) {
+  auto score_sub = [&](const Sub& sb, int valid, float& s0, float& s1, bool one_chain = false) {
     uint32_t wa[BITS], wb[BITS];
     load_key_words<BITS>(sb.k, gq, tq, wa, wb);
     float acc0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, acc1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
@@ -695,7 +724,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
       } else {
         key_frag<BITS, SGN, true>(wa, wb, j, a0, a1, a2, a3);
       }
-      if (j & 1) mma_f16(acc1, a0, a1, a2, a3, bq[j][0], bq[j][1]);
+      if ((j & 1) && !one_chain) mma_f16(acc1, a0, a1, a2, a3, bq[j][0], bq[j][1]);
       else mma_f16(acc0, a0, a1, a2, a3, bq[j][0], bq[j][1]);
       if (!KAXIS && !F8 && ((j + 1) & ((1 << kg_shift) - 1)) == 0) {
         const int gi = j >> kg_shift;
@@ -711,7 +740,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
         for (int c = 0; c < 4; ++c) acc0[c] = acc1[c] = 0.0f;
       }
     }
-    if (KAXIS || F8) {
+    if (one_chain) {
+      r0 = acc0[0] + acc0[1];
+      r1 = acc0[2] + acc0[3];
+    } else if (KAXIS || F8) {
       r0 = acc0[0] + acc0[1] + acc1[0] + acc1[1];
       r1 = acc0[2] + acc0[3] + acc1[2] + acc1[3];
     }
@@ -815,6 +847,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
         for (int c = 0; c < 4; ++c) st.o[i][c] *= alpha;
         st.zacc[i] *= alpha;
       }
+      if (SPEC) {
+#pragma unroll
+        for (int gi = 0; gi < 2; ++gi)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) st.zc[gi][c] *= alpha;
+      }
       st.m = mx;
     }
     const bool live = st.m != -INFINITY;
@@ -827,6 +865,75 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
     st.l += sum;
   };
 
+  // ---- INT4 KIVI, whole 64-token units: codes as fp16 subnormals ----------
+  // A nibble masked into the low mantissa bits of an fp16 half, exponent field
+  // zero, is the subnormal u * 2^-24 (bits 0-3) or u * 2^-20 (bits 4-7), u the
+  // field read as unsigned: one LOP3 per operand register, no FMA.  Flipping
+  // the field's top bit makes u = code + 8.  The constant 8 is removed exactly
+  // by the same products over all-zero codes (u = 8): per unit for the keys,
+  // per sub-tile and value group for the values.  Operand registers at bits
+  // 4-7 carry the extra 16: on the key side they are the k-half fed by the b1
+  // register, so q' of the b0 half is 16 times larger; on the value side they
+  // are channel rows gq + 8, rescaled when the sums are normalised.
+  constexpr uint32_t ZA0 = 0x00080008u, ZA1 = 0x00800080u;   // all-zero codes, bits 0-3 / 4-7
+  auto score_sub_sn = [&](const Sub& sb, float cs20, float bias, float& s0, float& s1) {
+    uint32_t wa[4], wb[4];
+    load_key_words<4>(sb.k, gq, tq, wa, wb);
+    float acc0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, acc1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int jj = j >> 1;
+      const uint32_t va = (j & 1) ? (wa[jj] >> 8) : wa[jj], vb = (j & 1) ? (wb[jj] >> 8) : wb[jj];
+      const uint32_t a0 = and_xor(va, 0x000F000Fu, ZA0), a1 = and_xor(vb, 0x000F000Fu, ZA0);
+      const uint32_t a2 = and_xor(va, 0x00F000F0u, ZA1), a3 = and_xor(vb, 0x00F000F0u, ZA1);
+      if (j & 1) mma_f16(acc1, a0, a1, a2, a3, bq[j][0], bq[j][1]);
+      else mma_f16(acc0, a0, a1, a2, a3, bq[j][0], bq[j][1]);
+    }
+    s0 = fmaf(acc0[0] + acc0[1] + acc1[0] + acc1[1], cs20, bias);
+    s1 = fmaf(acc0[2] + acc0[3] + acc1[2] + acc1[3], cs20, bias);
+  };
+  auto pv_sub_sn = [&](const Sub& sb, float p0, float p1) {
+    const int sa = 8 * tq + hh, sbl = sa + 4;
+    const float pa0 = __shfl_sync(0xffffffffu, p0, sa);
+    const float pa1 = __shfl_sync(0xffffffffu, p1, sa);
+    const float pb0 = __shfl_sync(0xffffffffu, p0, sbl);
+    const float pb1 = __shfl_sync(0xffffffffu, p1, sbl);
+    uint32_t vw[8];
+    load_value_words<4>(sb.v, lane, vw);
+    uint32_t pha, pla, phb, plb;
+    split2h(pa0, pb0, pha, pla);
+    split2h(pa1, pb1, phb, plb);
+    const uint16_t* vs = reinterpret_cast<const uint16_t*>(sb.vms);
+    // rows 2tq, 2tq + 1 (and + 8) hold both groups' scales in 8 bytes
+    const uint2 ra = *reinterpret_cast<const uint2*>(vs + 4 * tq);
+    const uint2 rb = *reinterpret_cast<const uint2*>(vs + 4 * tq + 16);
+    uint32_t b0 = 0, b1 = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if ((i & 3) == 0) {
+        const int gi = i >> 2;
+        const uint32_t sel = gi ? 0x7632u : 0x5410u;
+        const uint32_t xa = __byte_perm(ra.x, ra.y, sel), xb = __byte_perm(rb.x, rb.y, sel);
+        const __half2 sa2 = *reinterpret_cast<const __half2*>(&xa), sb2 = *reinterpret_cast<const __half2*>(&xb);
+        auto two = [](uint32_t ph, uint32_t pl, __half2 sv, uint32_t& hi, uint32_t& lo) {
+          const __half2 a = *reinterpret_cast<const __half2*>(&ph), b = *reinterpret_cast<const __half2*>(&pl);
+          const __half2 h = __hmul2(a, sv);
+          const __half2 l = __hfma2(b, sv, __hfma2(a, sv, __hneg2(h)));
+          hi = *reinterpret_cast<const uint32_t*>(&h);
+          lo = *reinterpret_cast<const uint32_t*>(&l);
+        };
+        uint32_t h0, l0, h1, l1;
+        two(pha, pla, sa2, h0, l0);
+        two(phb, plb, sb2, h1, l1);
+        b0 = is_lo ? l0 : h0;
+        b1 = is_lo ? l1 : h1;
+        mma_f16(st.zc[gi], ZA0, ZA1, ZA0, ZA1, b0, b1);   // the offset 8 of every code
+      }
+      const uint32_t w = vw[i], w8 = w >> 8;
+      mma_f16(st.o[i], and_xor(w, 0x000F000Fu, ZA0), and_xor(w, 0x00F000F0u, ZA1), and_xor(w8, 0x000F000Fu, ZA0),
+              and_xor(w8, 0x00F000F0u, ZA1), b0, b1);
+    }
+  };
   // A 16-token tile of the BF16 window (natural row-major layout).
   auto process_window = [&](const uint8_t* stg, int valid) {
     const uint32_t kaddr = smem_addr(stg), vaddr = kaddr + 16 * D * 2;
@@ -973,7 +1080,26 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
       const int valid_unit = min(pp.sup, ric.qa - T0);
       const int nsub = (valid_unit + 15) >> 4;
       int loaded = -1;
-      for (int c = 0; c < nsub; c += ch) {
+      if (SPEC && valid_unit == 64) {
+        // A whole 64-token unit of the INT4 KIVI format: one key group, four
+        // 16-token pages in the stage at fixed offsets; straight-line code
+        // with scores and weights in registers, codes as fp16 subnormals.
+        qprime_job(stg, 0, true);
+        float accb[4] = {0.0f, 0.0f, 0.0f, 0.0f};   // the key offset: q' against all-zero codes
+#pragma unroll
+        for (int j = 0; j < 8; ++j) mma_f16(accb, ZA0, ZA0, ZA1, ZA1, bq[j][0], bq[j][1]);
+        const float cs20 = cs * 1048576.0f, bias = -(accb[0] + accb[1]) * cs20;
+        float sc[8], pc[8];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) score_sub_sn(sub_at(stg, 16 * t), cs20, bias, sc[2 * t], sc[2 * t + 1]);
+        softmax_chunk(sc, pc);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) pv_sub_sn(sub_at(stg, 16 * t), pc[2 * t], pc[2 * t + 1]);
+        st.raw = true;
+      } else if (SPEC && st.raw) {
+        normalize();
+      }
+      for (int c = 0; c < nsub && !(SPEC && valid_unit == 64); c += ch) {
         if (KAXIS && ((16 * c) >> g.lg_gk) != loaded) {
           loaded = (16 * c) >> g.lg_gk;
           qprime_job(stg, loaded);
@@ -1000,6 +1126,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
           pv_sub(sub_at(stg, 16 * (c + t)), spw[(2 * t) * 32 + lane], spw[(2 * t + 1) * 32 + lane], true);
       }
     } else {
+      if (SPEC && st.raw) normalize();
       if (!bq_bf16) {
         load_bq_from_q(itc.i, itc.h);
         bq_bf16 = true;
