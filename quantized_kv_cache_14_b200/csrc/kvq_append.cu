@@ -371,6 +371,189 @@ __global__ void __launch_bounds__(kFlushThreads) flush_kernel(const Geo g, const
 }
 
 // ---------------------------------------------------------------------------
+// Per-channel key flush for calls that flush many groups (bulk prefill): one
+// CTA per (flushed group, head).  The group's R key and value rows are
+// gathered once, the channel statistics use every thread, every code is
+// quantized once into shared memory, and the packing passes then write all
+// of the group's pages.  The bytes are those of flush_kernel.
+template <int BITS, int ASYM>
+__global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g, const DevState d,
+                                                                    const __grid_constant__ PlanView p,
+                                                                    const uint16_t* kin, const uint16_t* vin,
+                                                                    int fuse_rows) {
+  if (int(blockIdx.x) >= p.n_flush) {
+    const int64_t cta = int64_t(blockIdx.x - p.n_flush) * gridDim.y + blockIdx.y;
+    const int64_t ctas = int64_t(gridDim.x - p.n_flush) * gridDim.y;
+    apply_body(g, d, p, fuse_rows ? kin : nullptr, vin, cta * blockDim.x + threadIdx.x, ctas * blockDim.x);
+    return;
+  }
+  constexpr int D = kD;
+  constexpr int N = 32 / BITS;
+  constexpr int Q = ASYM ? (1 << BITS) - 1 : (1 << (BITS - 1)) - 1;
+  constexpr uint32_t MASK = (1u << BITS) - 1;
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int R = g.R;
+  uint16_t* kt = reinterpret_cast<uint16_t*>(smem);                 // [R][D] bf16
+  uint16_t* vt = kt + R * D;                                        // [R][D] bf16
+  uint8_t* kq = reinterpret_cast<uint8_t*>(vt + R * D);             // [R][D] key codes (low BITS bits)
+  uint8_t* vq = kq + R * D;                                         // [R][D] value codes
+  float* ksc = reinterpret_cast<float*>(vq + R * D);                // [D]
+  float* kzp = ksc + D;                                             // [D]
+  float* vsc = kzp + D;                                             // [R][nvg]
+  float* vzp = vsc + R * g.nvg;                                     // [R][nvg]
+  float* part = vzp + R * g.nvg;                                    // [3][D] second half's key statistics
+  int32_t* ssrc = reinterpret_cast<int32_t*>(part + 3 * D);         // [R]
+
+  const int e = blockIdx.x, h = blockIdx.y, tid = threadIdx.x, T = blockDim.x;
+  const int32_t* ent = plan_of(p) + p.off_flush + e * kFlushEntryInts;
+  const int seq = ent[0];
+  const int32_t* srcs = plan_of(p) + p.off_src + int64_t(e) * R;
+  for (int r = tid; r < R; r += T) ssrc[r] = srcs[r];
+  __syncthreads();
+
+  // 1. the group's K and V rows (bf16): from the input, or the window
+  for (int idx = tid; idx < 2 * R * (D / 8); idx += T) {
+    const int which = idx / (R * (D / 8));
+    const int rem = idx % (R * (D / 8));
+    const int r = rem / (D / 8), c8 = rem % (D / 8);
+    const int32_t s = ssrc[r];
+    const uint16_t* src;
+    if (s >= 0) src = (which ? vin : kin) + (int64_t(s) * g.h_kv + h) * D;
+    else src = (which ? d.vres : d.kres) + ((int64_t(seq) * g.h_kv + h) * R + (-1 - s)) * D;
+    reinterpret_cast<uint4*>((which ? vt : kt) + r * D)[c8] = reinterpret_cast<const uint4*>(src)[c8];
+  }
+  __syncthreads();
+
+  // 2. key channel statistics: thread (half, c) scans half of the rows
+  {
+    const int c = tid % D, half = tid / D, nh = T / D;
+    const int r0 = half * R / nh, r1 = (half + 1) * R / nh;
+    float a = 0.0f, mn = INFINITY, mx = -INFINITY;
+    for (int r = r0; r < r1; ++r) {
+      const float x = bf16_bits_to_float(kt[r * D + c]);
+      a = fmaxf(a, fabsf(x));
+      mn = fminf(mn, x);
+      mx = fmaxf(mx, x);
+    }
+    if (half == 1) {
+      part[c] = a;
+      part[D + c] = mn;
+      part[2 * D + c] = mx;
+    }
+    __syncthreads();
+    if (half == 0) {
+      a = fmaxf(a, part[c]);
+      mn = fminf(mn, part[D + c]);
+      mx = fmaxf(mx, part[2 * D + c]);
+      if (ASYM) {
+        kzp[c] = stored_value(mn, g.scale_fp32);
+        ksc[c] = stored_value(__fdiv_rn(__fsub_rn(mx, mn), float(Q)), g.scale_fp32);
+      } else {
+        ksc[c] = stored_value(__fdiv_rn(a, float(Q)), g.scale_fp32);
+        kzp[c] = 0.0f;
+      }
+    }
+  }
+  // value (token, group) statistics: warp w takes rows w, w + 8, ...
+  {
+    const int w = tid >> 5, lane = tid & 31;
+    const int lanes_per_group = g.g_v / 4;
+    for (int r = w; r < R; r += T / 32) {
+      float x[4];
+      for (int i = 0; i < 4; ++i) x[i] = bf16_bits_to_float(vt[r * D + 4 * lane + i]);
+      float a = 0.0f, mn = x[0], mx = x[0];
+      for (int i = 0; i < 4; ++i) {
+        a = fmaxf(a, fabsf(x[i]));
+        mn = fminf(mn, x[i]);
+        mx = fmaxf(mx, x[i]);
+      }
+      for (int off = 1; off < lanes_per_group; off <<= 1) {
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      }
+      if ((4 * lane) % g.g_v == 0) {
+        const int gi = (4 * lane) / g.g_v;
+        if (ASYM) {
+          vzp[r * g.nvg + gi] = stored_value(mn, g.scale_fp32);
+          vsc[r * g.nvg + gi] = stored_value(__fdiv_rn(__fsub_rn(mx, mn), float(Q)), g.scale_fp32);
+        } else {
+          vsc[r * g.nvg + gi] = stored_value(__fdiv_rn(a, float(Q)), g.scale_fp32);
+          vzp[r * g.nvg + gi] = 0.0f;
+        }
+      }
+    }
+  }
+  __syncthreads();
+
+  // 3. every code once
+  for (int idx = tid; idx < R * D; idx += T) {
+    const int r = idx / D, c = idx % D, gi = c / g.g_v;
+    const float xk = bf16_bits_to_float(kt[idx]), xv = bf16_bits_to_float(vt[idx]);
+    const int qk = ASYM ? quant_asym(xk, ksc[c], kzp[c], Q) : quant_sym(xk, ksc[c], Q);
+    const int qv = ASYM ? quant_asym(xv, vsc[r * g.nvg + gi], vzp[r * g.nvg + gi], Q)
+                        : quant_sym(xv, vsc[r * g.nvg + gi], Q);
+    kq[idx] = uint8_t(uint32_t(qk) & MASK);
+    vq[idx] = uint8_t(uint32_t(qv) & MASK);
+  }
+  __syncthreads();
+
+  auto chunk_of = [&](int page) -> uint8_t* {
+    return d.pool + int64_t(ent[3 + page]) * g.block_bytes + int64_t(h) * g.chunk_bytes;
+  };
+  const int subs_per_page = g.P / 16;
+
+  // 4. key words: (row, word in row), element l of word w is list position w N + l
+  const int row_words = D * BITS / 32;
+  for (int W = tid; W < R * row_words; W += T) {
+    const int rowi = W / row_words, w = W % row_words;
+    uint32_t word = 0;
+    for (int l = 0; l < N; ++l) word |= uint32_t(kq[rowi * D + key_channel(w * N + l)]) << (BITS * word_field(l, N));
+    const int sub = rowi >> 4, rr = rowi & 15;
+    *reinterpret_cast<uint32_t*>(chunk_of(sub / subs_per_page) + (sub % subs_per_page) * g.sub_bytes +
+                                 rr * g.row_bytes + 4 * w) = word;
+  }
+
+  // 5. value words: (sub-tile, lane record, word in record) as in flush_kernel
+  const int rec_words = 2 * BITS;
+  for (int W = tid; W < (R / 16) * 32 * rec_words; W += T) {
+    const int sub = W / (32 * rec_words), rem = W % (32 * rec_words);
+    const int lam = rem / rec_words, w = rem % rec_words;
+    const int gq = lam >> 2, tq = lam & 3;
+    uint32_t word = 0;
+    for (int x = 0; x < N / 2; ++x) {
+      int i, reg;
+      if (BITS == 8) { i = w >> 1; reg = 2 * (w & 1) + x; }
+      else if (BITS == 4) { i = w; reg = x; }
+      else { i = 2 * w + ((x >> 1) & 1); reg = 2 * (x >> 2) + (x & 1); }
+      const int c = 16 * i + gq + 8 * (reg & 1);
+      const int t0 = 16 * sub + 2 * tq + 8 * (reg >> 1);
+      word |= uint32_t(vq[t0 * D + c]) << (BITS * x);
+      word |= uint32_t(vq[(t0 + 1) * D + c]) << (BITS * (x + N / 2));
+    }
+    *reinterpret_cast<uint32_t*>(chunk_of(sub / subs_per_page) + g.off_V + (sub % subs_per_page) * g.sub_bytes +
+                                 lam * (8 * BITS) + 4 * w) = word;
+  }
+
+  // 6. metadata: each page's slice of the key scales (list order), value scales
+  const int npg = R / g.P;
+  for (int idx = tid; idx < npg * g.kslice; idx += T) {
+    const int page = idx / g.kslice, off = idx % g.kslice;
+    const int c = key_channel(page * g.kslice + off);
+    uint8_t* km = chunk_of(page) + g.off_Km;
+    store_meta(km + off * g.es, ksc[c], g.scale_fp32);
+    if (ASYM) store_meta(km + (g.kslice + off) * g.es, kzp[c], g.scale_fp32);
+  }
+  for (int idx = tid; idx < R * g.nvg; idx += T) {
+    const int r = idx / g.nvg, gi = idx % g.nvg;
+    const int page = r / g.P, rp = r % g.P;
+    uint8_t* vm = chunk_of(page) + g.off_Vm;
+    store_meta(vm + (rp * g.nvg + gi) * g.es, vsc[idx], g.scale_fp32);
+    if (ASYM) store_meta(vm + (g.P * g.nvg + rp * g.nvg + gi) * g.es, vzp[idx], g.scale_fp32);
+  }
+}
+
+// ---------------------------------------------------------------------------
 __global__ void residual_kernel(const Geo g, const DevState d, const __grid_constant__ PlanView p,
                                 const uint16_t* kin, const uint16_t* vin) {
   constexpr int D = kD;
@@ -466,6 +649,15 @@ size_t flush_smem_bytes(const Geo& g) {
   return size_t(2) * g.R * kD * 2 + size_t(2) * kD * 4 + size_t(2) * g.R * g.nvg * 4;
 }
 
+size_t flush_group_smem_bytes(const Geo& g) {
+  return size_t(2) * g.R * kD * 2 + size_t(2) * g.R * kD + size_t(2) * kD * 4 + size_t(2) * g.R * g.nvg * 4 +
+         size_t(3) * kD * 4 + size_t(g.R) * 4;
+}
+
+// Calls that flush at least this many groups use one CTA per (group, head);
+// fewer (a decode step) keep one CTA per (group, head, sub-tile).
+constexpr int kBulkFlushGroups = 16;
+
 }  // namespace
 
 cudaError_t launch_apply(const Geo& g, const DevState& d, const PlanView& p, const uint16_t* k,
@@ -503,6 +695,27 @@ cudaError_t launch_quant_token(const Geo& g, const DevState& d, const PlanView& 
 cudaError_t launch_flush(const Geo& g, const DevState& d, const PlanView& p, const uint16_t* k,
                          const uint16_t* v, bool with_apply, bool fuse_rows, cudaStream_t s, int* launches) {
   if (p.n_flush == 0) return cudaSuccess;
+  if (p.n_flush >= kBulkFlushGroups) {
+    const size_t smem = flush_group_smem_bytes(g);
+    const int64_t per_col = int64_t(g.h_kv) * kFlushThreads;
+    const int64_t work = with_apply ? apply_work(g, p, fuse_rows) : 0;
+    const int extra = int(std::min<int64_t>((work + per_col - 1) / per_col, 256));
+    return by_format(g, [&](auto B, auto A) {
+      auto kern = flush_group_kernel<decltype(B)::value, decltype(A)::value>;
+      static thread_local size_t limit_set[32] = {};
+      int dev = 0;
+      cudaError_t e = cudaGetDevice(&dev);
+      if (e != cudaSuccess) return e;
+      if (dev >= 32 || smem > limit_set[dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e != cudaSuccess) return e;
+        if (dev < 32) limit_set[dev] = smem;
+      }
+      kern<<<dim3(p.n_flush + extra, g.h_kv), kFlushThreads, smem, s>>>(g, d, p, k, v, fuse_rows ? 1 : 0);
+      ++*launches;
+      return cudaGetLastError();
+    });
+  }
   const size_t smem = flush_smem_bytes(g);
   // extra columns of (h_kv x R/16) CTAs for the apply body
   const int64_t per_col = int64_t(g.h_kv) * (g.R / 16) * kFlushThreads;

@@ -131,6 +131,29 @@ def test_append_launch_shapes(name):
     p.close()
 
 
+@pytest.mark.parametrize("name", ["int4_chan64", "int2_asym_chan32", "int8_asym_chan128_p64", "int4_chan16",
+                                  "int4_chan64_p32_gv32", "int4_chan64_fp32"])
+def test_bulk_flush_matches_oracle(name):
+    """Calls that complete many key groups at once (the bulk prefill shape:
+    one CTA per group and head) give the oracle's bytes, with groups whose
+    tokens come partly from the window and partly from the call."""
+    rng = np.random.default_rng(31)
+    R = FMTS[name]["residual"]
+    h_q, h_kv, S = 8, 2, 20
+    p = Pair(FMTS[name], h_q, h_kv, max_seqs=S, num_blocks=S * (3 * R // 16 + 4), mbps=3 * R // 16 + 4, seed=6)
+    lens = [int(x) for x in rng.integers(R // 2, R, size=S)]     # every window partly filled
+    ids = np.repeat(np.arange(S, dtype=np.int32), lens)
+    p.append(outlier_keys(rng, ids.size, h_kv), random_bf16(rng, (ids.size, h_kv, D)), ids)
+    add = [int(x) for x in rng.integers(R, 2 * R, size=S)]       # each call completes 1-2 groups per sequence
+    ids = np.repeat(np.arange(S, dtype=np.int32), add)
+    rng.shuffle(ids)
+    p.append(outlier_keys(rng, ids.size, h_kv), random_bf16(rng, (ids.size, h_kv, D)), ids)
+    lens = [a + b for a, b in zip(lens, add)]
+    p.check_state()
+    p.check_decode(random_bf16(rng, (S, h_q, D)), lens)
+    p.close()
+
+
 @pytest.mark.parametrize("name", ["int4_chan64", "int8_tok_p16", "fp8_p16"])
 def test_step_host_equals_device_calls(name):
     """kvq_step_host (host buffers in, host output back, one call) appends the
@@ -150,13 +173,22 @@ def test_step_host_equals_device_calls(name):
     def host(bits):
         return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).pin_memory()
 
+    def packed(k, v, q):
+        # one page-locked buffer holding k | v | q back to back (one H2D copy)
+        buf = host(np.concatenate([k.ravel(), v.ravel(), q.ravel()]))
+        return buf[:k.size].view(k.shape), buf[k.size:2 * k.size].view(v.shape), buf[2 * k.size:].view(q.shape)
+
     for step in range(70):   # crosses group boundaries of every sequence
         ids = np.arange(S, dtype=np.int32)
         k, v, q = outlier_keys(rng, S, h_kv), random_bf16(rng, (S, h_kv, D)), random_bf16(rng, (S, h_q, D))
         lens = [L + 1 for L in lens]
         a.append(k, v, ids)
-        out_h = torch.full((S, h_q, D), float("nan"), dtype=torch.float32).pin_memory()
-        b.step_host(host(k), host(v), ids, host(q), out_h)
+        if step % 2 == 0:   # packed inputs, output written straight into page-locked memory
+            out_h = torch.full((S, h_q, D), float("nan"), dtype=torch.float32).pin_memory()
+            b.step_host(*packed(k, v, q)[:2], ids, packed(k, v, q)[2], out_h)
+        else:               # separate inputs, pageable output (one copy back)
+            out_h = torch.full((S, h_q, D), float("nan"), dtype=torch.float32)
+            b.step_host(host(k), host(v), ids, host(q), out_h)
         torch.cuda.synchronize()
         if step % 23 == 0 or step == 69:
             got, want = a.decode(q, lens)
