@@ -30,6 +30,9 @@ namespace {
 static_assert(sizeof(Geo) + sizeof(DevState) + sizeof(PlanView) + 3 * sizeof(void*) + 16 <= 4096,
               "append kernel parameters exceed 4 KB");
 
+// Row stride of the bulk flush's code arrays in shared memory (bytes).
+constexpr int kFlushCodeStride = kD + 8;
+
 // The plan's entries: inline in the launch parameters or uploaded.
 __device__ __forceinline__ const int32_t* plan_of(const PlanView& p) { return p.plan ? p.plan : p.inl; }
 
@@ -132,9 +135,10 @@ __global__ void __launch_bounds__(256) quant_token_kernel(const Geo g, const Dev
     } else {
       sh = stored_value(__fdiv_rn(a, float(Q)), g.scale_fp32);
     }
+    const float inv = quant_inv(sh);
     for (int i = 0; i < 4; ++i)
       s_codes[wib][4 * lane + i] =
-          int8_t(ASYM ? quant_asym(x[i], sh, zh, Q) : quant_sym(x[i], sh, Q));
+          int8_t(ASYM ? quant_asym_fast(x[i], sh, inv, zh, Q) : quant_sym_fast(x[i], sh, inv, Q));
     const int gi = (4 * lane) / gsz;
     if ((4 * lane) % gsz == 0) {
       const int off_meta = which ? g.off_Vm : g.off_Km;
@@ -221,6 +225,8 @@ __global__ void __launch_bounds__(kFlushThreads) flush_kernel(const Geo g, const
   float* kzp = ksc + D;                                              // [D]
   float* vsc = kzp + D;                                              // [R][nvg]
   float* vzp = vsc + R * g.nvg;                                      // [R][nvg]
+  float* kinv = vzp + R * g.nvg;                                     // [D] RN(1 / key scale)
+  float* vinv = kinv + D;                                            // [R][nvg]
 
   const int e = blockIdx.x, h = blockIdx.y, zs = blockIdx.z, tid = threadIdx.x;
   const int r_lo = 16 * zs;   // this CTA's rows [r_lo, r_lo + 16)
@@ -261,6 +267,7 @@ __global__ void __launch_bounds__(kFlushThreads) flush_kernel(const Geo g, const
       ksc[c] = stored_value(__fdiv_rn(a, float(Q)), g.scale_fp32);
       kzp[c] = 0.0f;
     }
+    kinv[c] = quant_inv(ksc[c]);
   } else {
     const int w = (tid - D) >> 5, lane = tid & 31;
     const int lanes_per_group = g.g_v / 4;
@@ -287,6 +294,7 @@ __global__ void __launch_bounds__(kFlushThreads) flush_kernel(const Geo g, const
           vsc[r * g.nvg + gi] = stored_value(__fdiv_rn(a, float(Q)), g.scale_fp32);
           vzp[r * g.nvg + gi] = 0.0f;
         }
+        vinv[r * g.nvg + gi] = quant_inv(vsc[r * g.nvg + gi]);
       }
     }
   }
@@ -295,16 +303,16 @@ __global__ void __launch_bounds__(kFlushThreads) flush_kernel(const Geo g, const
   auto chunk_of = [&](int page) -> uint8_t* {
     return d.pool + int64_t(ent[3 + page]) * g.block_bytes + int64_t(h) * g.chunk_bytes;
   };
+  const int lg_gv = __ffs(g.g_v) - 1;
   auto kcode = [&](int r, int c) -> uint32_t {
     const float x = bf16_bits_to_float(kt[r * D + c]);
-    const int q = ASYM ? quant_asym(x, ksc[c], kzp[c], Q) : quant_sym(x, ksc[c], Q);
+    const int q = ASYM ? quant_asym_fast(x, ksc[c], kinv[c], kzp[c], Q) : quant_sym_fast(x, ksc[c], kinv[c], Q);
     return uint32_t(q) & ((1u << BITS) - 1);
   };
   auto vcode = [&](int r, int c) -> uint32_t {
     const float x = bf16_bits_to_float(vt[r * D + c]);
-    const int gi = c / g.g_v;
-    const int q = ASYM ? quant_asym(x, vsc[r * g.nvg + gi], vzp[r * g.nvg + gi], Q)
-                       : quant_sym(x, vsc[r * g.nvg + gi], Q);
+    const int m = r * g.nvg + (c >> lg_gv);
+    const int q = ASYM ? quant_asym_fast(x, vsc[m], vinv[m], vzp[m], Q) : quant_sym_fast(x, vsc[m], vinv[m], Q);
     return uint32_t(q) & ((1u << BITS) - 1);
   };
   const int subs_per_page = g.P / 16;
@@ -391,17 +399,20 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
   constexpr int N = 32 / BITS;
   constexpr int Q = ASYM ? (1 << BITS) - 1 : (1 << (BITS - 1)) - 1;
   constexpr uint32_t MASK = (1u << BITS) - 1;
+  constexpr int CS = kFlushCodeStride;   // code row stride: 8 bytes of padding spread the banks
   extern __shared__ __align__(16) uint8_t smem[];
   const int R = g.R;
   uint16_t* kt = reinterpret_cast<uint16_t*>(smem);                 // [R][D] bf16
   uint16_t* vt = kt + R * D;                                        // [R][D] bf16
-  uint8_t* kq = reinterpret_cast<uint8_t*>(vt + R * D);             // [R][D] key codes (low BITS bits)
-  uint8_t* vq = kq + R * D;                                         // [R][D] value codes
-  float* ksc = reinterpret_cast<float*>(vq + R * D);                // [D]
+  uint8_t* kq = reinterpret_cast<uint8_t*>(vt + R * D);             // [R][CS] key codes (low BITS bits)
+  uint8_t* vq = kq + R * CS;                                        // [R][CS] value codes
+  float* ksc = reinterpret_cast<float*>(vq + R * CS);               // [D]
   float* kzp = ksc + D;                                             // [D]
   float* vsc = kzp + D;                                             // [R][nvg]
   float* vzp = vsc + R * g.nvg;                                     // [R][nvg]
-  float* part = vzp + R * g.nvg;                                    // [3][D] second half's key statistics
+  float* kinv = vzp + R * g.nvg;                                    // [D] RN(1 / key scale)
+  float* vinv = kinv + D;                                           // [R][nvg]
+  float* part = vinv + R * g.nvg;                                   // [3][D] second half's key statistics
   int32_t* ssrc = reinterpret_cast<int32_t*>(part + 3 * D);         // [R]
 
   const int e = blockIdx.x, h = blockIdx.y, tid = threadIdx.x, T = blockDim.x;
@@ -452,49 +463,116 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
         ksc[c] = stored_value(__fdiv_rn(a, float(Q)), g.scale_fp32);
         kzp[c] = 0.0f;
       }
+      kinv[c] = quant_inv(ksc[c]);
     }
   }
-  // value (token, group) statistics: warp w takes rows w, w + 8, ...
+  // value (token, group) extremes: warp w takes rows w, w + 8, ...; lane l
+  // holds channels 4l .. 4l + 3 (one 64-bit load), reduced over the g_v / 4
+  // lanes of its group; the scales follow once every row is reduced
   {
     const int w = tid >> 5, lane = tid & 31;
-    const int lanes_per_group = g.g_v / 4;
+    const int lanes_per_group = g.g_v / 4;   // a power of two
     for (int r = w; r < R; r += T / 32) {
-      float x[4];
-      for (int i = 0; i < 4; ++i) x[i] = bf16_bits_to_float(vt[r * D + 4 * lane + i]);
-      float a = 0.0f, mn = x[0], mx = x[0];
-      for (int i = 0; i < 4; ++i) {
-        a = fmaxf(a, fabsf(x[i]));
-        mn = fminf(mn, x[i]);
-        mx = fmaxf(mx, x[i]);
-      }
-      for (int off = 1; off < lanes_per_group; off <<= 1) {
-        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-      }
-      if ((4 * lane) % g.g_v == 0) {
-        const int gi = (4 * lane) / g.g_v;
-        if (ASYM) {
-          vzp[r * g.nvg + gi] = stored_value(mn, g.scale_fp32);
-          vsc[r * g.nvg + gi] = stored_value(__fdiv_rn(__fsub_rn(mx, mn), float(Q)), g.scale_fp32);
-        } else {
-          vsc[r * g.nvg + gi] = stored_value(__fdiv_rn(a, float(Q)), g.scale_fp32);
-          vzp[r * g.nvg + gi] = 0.0f;
+      const uint2 raw = *reinterpret_cast<const uint2*>(vt + r * D + 4 * lane);
+      const float x0 = bf16_bits_to_float(uint16_t(raw.x)), x1 = bf16_bits_to_float(uint16_t(raw.x >> 16));
+      const float x2 = bf16_bits_to_float(uint16_t(raw.y)), x3 = bf16_bits_to_float(uint16_t(raw.y >> 16));
+      if (ASYM) {
+        float mn = fminf(fminf(x0, x1), fminf(x2, x3)), mx = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
+        for (int off = 1; off < lanes_per_group; off <<= 1) {
+          mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
         }
+        if ((lane & (lanes_per_group - 1)) == 0) {
+          vzp[r * g.nvg + lane / lanes_per_group] = mn;   // raw extremes for now
+          vsc[r * g.nvg + lane / lanes_per_group] = mx;
+        }
+      } else {
+        float a = fmaxf(fmaxf(fabsf(x0), fabsf(x1)), fmaxf(fabsf(x2), fabsf(x3)));
+        for (int off = 1; off < lanes_per_group; off <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+        if ((lane & (lanes_per_group - 1)) == 0) vsc[r * g.nvg + lane / lanes_per_group] = a;
       }
     }
   }
   __syncthreads();
+  for (int m = tid; m < R * g.nvg; m += T) {   // the value scales, one (row, group) per thread
+    if (ASYM) {
+      const float mn = vzp[m], mx = vsc[m];
+      vzp[m] = stored_value(mn, g.scale_fp32);
+      vsc[m] = stored_value(__fdiv_rn(__fsub_rn(mx, mn), float(Q)), g.scale_fp32);
+    } else {
+      vsc[m] = stored_value(__fdiv_rn(vsc[m], float(Q)), g.scale_fp32);
+      vzp[m] = 0.0f;
+    }
+    vinv[m] = quant_inv(vsc[m]);
+  }
+  __syncthreads();
 
-  // 3. every code once
-  for (int idx = tid; idx < R * D; idx += T) {
-    const int r = idx / D, c = idx % D, gi = c / g.g_v;
-    const float xk = bf16_bits_to_float(kt[idx]), xv = bf16_bits_to_float(vt[idx]);
-    const int qk = ASYM ? quant_asym(xk, ksc[c], kzp[c], Q) : quant_sym(xk, ksc[c], Q);
-    const int qv = ASYM ? quant_asym(xv, vsc[r * g.nvg + gi], vzp[r * g.nvg + gi], Q)
-                        : quant_sym(xv, vsc[r * g.nvg + gi], Q);
-    kq[idx] = uint8_t(uint32_t(qk) & MASK);
-    vq[idx] = uint8_t(uint32_t(qv) & MASK);
+  // 3. every code once, eight consecutive channels of one row per item (one
+  //    128-bit load of the row, the scales as vectors, one 64-bit store)
+  const int lg_gv = __ffs(g.g_v) - 1;
+  for (int it = tid; it < 2 * R * (D / 8); it += T) {
+    const bool val = it >= R * (D / 8);
+    const int rem = val ? it - R * (D / 8) : it;
+    const int r = rem / (D / 8), c0 = 8 * (rem % (D / 8));
+    const uint4 raw = *reinterpret_cast<const uint4*>((val ? vt : kt) + r * D + c0);
+    const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+    uint32_t lo = 0, hi = 0;
+    uint32_t ties = 0;   // elements whose code the exact division must decide
+    float xs[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) xs[i] = bf16_bits_to_float(uint16_t(wv[i >> 1] >> (16 * (i & 1))));
+    if (val) {
+      const int m = r * g.nvg + (c0 >> lg_gv);   // one value group covers the 8 channels
+      const float sh = vsc[m], inv = vinv[m], zh = vzp[m];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        bool tie;
+        const int q = ASYM ? quant_code_nb(__fsub_rn(xs[i], zh) * inv, 0, Q, tie)
+                           : quant_code_nb(xs[i] * inv, -Q, Q, tie);
+        ties |= uint32_t(tie) << i;
+        const uint32_t b = (uint32_t(q) & MASK) << (8 * (i & 3));
+        if (i < 4) lo |= b; else hi |= b;
+      }
+      if (__any_sync(0xffffffffu, ties != 0)) {
+        for (int i = 0; i < 8; ++i)
+          if (ties & (1u << i)) {
+            const int q = ASYM ? quant_asym_exact(xs[i], sh, zh, Q) : quant_sym_exact(xs[i], sh, Q);
+            uint32_t& wd = i < 4 ? lo : hi;
+            wd = (wd & ~(0xFFu << (8 * (i & 3)))) | ((uint32_t(q) & MASK) << (8 * (i & 3)));
+          }
+      }
+    } else {
+      float sc[8], iv[8], zp[8];
+#pragma unroll
+      for (int v4 = 0; v4 < 2; ++v4) {
+        const float4 a4 = reinterpret_cast<const float4*>(ksc + c0)[v4];
+        const float4 b4 = reinterpret_cast<const float4*>(kinv + c0)[v4];
+        sc[4 * v4] = a4.x; sc[4 * v4 + 1] = a4.y; sc[4 * v4 + 2] = a4.z; sc[4 * v4 + 3] = a4.w;
+        iv[4 * v4] = b4.x; iv[4 * v4 + 1] = b4.y; iv[4 * v4 + 2] = b4.z; iv[4 * v4 + 3] = b4.w;
+        if (ASYM) {
+          const float4 z4 = reinterpret_cast<const float4*>(kzp + c0)[v4];
+          zp[4 * v4] = z4.x; zp[4 * v4 + 1] = z4.y; zp[4 * v4 + 2] = z4.z; zp[4 * v4 + 3] = z4.w;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        bool tie;
+        const int q = ASYM ? quant_code_nb(__fsub_rn(xs[i], zp[i]) * iv[i], 0, Q, tie)
+                           : quant_code_nb(xs[i] * iv[i], -Q, Q, tie);
+        ties |= uint32_t(tie) << i;
+        const uint32_t b = (uint32_t(q) & MASK) << (8 * (i & 3));
+        if (i < 4) lo |= b; else hi |= b;
+      }
+      if (__any_sync(0xffffffffu, ties != 0)) {
+        for (int i = 0; i < 8; ++i)
+          if (ties & (1u << i)) {
+            const int q = ASYM ? quant_asym_exact(xs[i], sc[i], zp[i], Q) : quant_sym_exact(xs[i], sc[i], Q);
+            uint32_t& wd = i < 4 ? lo : hi;
+            wd = (wd & ~(0xFFu << (8 * (i & 3)))) | ((uint32_t(q) & MASK) << (8 * (i & 3)));
+          }
+      }
+    }
+    *reinterpret_cast<uint2*>((val ? vq : kq) + r * CS + c0) = make_uint2(lo, hi);
   }
   __syncthreads();
 
@@ -508,7 +586,8 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
   for (int W = tid; W < R * row_words; W += T) {
     const int rowi = W / row_words, w = W % row_words;
     uint32_t word = 0;
-    for (int l = 0; l < N; ++l) word |= uint32_t(kq[rowi * D + key_channel(w * N + l)]) << (BITS * word_field(l, N));
+#pragma unroll
+    for (int l = 0; l < N; ++l) word |= uint32_t(kq[rowi * CS + key_channel(w * N + l)]) << (BITS * word_field(l, N));
     const int sub = rowi >> 4, rr = rowi & 15;
     *reinterpret_cast<uint32_t*>(chunk_of(sub / subs_per_page) + (sub % subs_per_page) * g.sub_bytes +
                                  rr * g.row_bytes + 4 * w) = word;
@@ -528,8 +607,8 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
       else { i = 2 * w + ((x >> 1) & 1); reg = 2 * (x >> 2) + (x & 1); }
       const int c = 16 * i + gq + 8 * (reg & 1);
       const int t0 = 16 * sub + 2 * tq + 8 * (reg >> 1);
-      word |= uint32_t(vq[t0 * D + c]) << (BITS * x);
-      word |= uint32_t(vq[(t0 + 1) * D + c]) << (BITS * (x + N / 2));
+      word |= uint32_t(vq[t0 * CS + c]) << (BITS * x);
+      word |= uint32_t(vq[(t0 + 1) * CS + c]) << (BITS * (x + N / 2));
     }
     *reinterpret_cast<uint32_t*>(chunk_of(sub / subs_per_page) + g.off_V + (sub % subs_per_page) * g.sub_bytes +
                                  lam * (8 * BITS) + 4 * w) = word;
@@ -646,12 +725,12 @@ cudaError_t by_format(const Geo& g, F&& f) {
 }
 
 size_t flush_smem_bytes(const Geo& g) {
-  return size_t(2) * g.R * kD * 2 + size_t(2) * kD * 4 + size_t(2) * g.R * g.nvg * 4;
+  return size_t(2) * g.R * kD * 2 + size_t(3) * kD * 4 + size_t(3) * g.R * g.nvg * 4;
 }
 
 size_t flush_group_smem_bytes(const Geo& g) {
-  return size_t(2) * g.R * kD * 2 + size_t(2) * g.R * kD + size_t(2) * kD * 4 + size_t(2) * g.R * g.nvg * 4 +
-         size_t(3) * kD * 4 + size_t(g.R) * 4;
+  return size_t(2) * g.R * kD * 2 + size_t(2) * g.R * kFlushCodeStride + size_t(3) * kD * 4 +
+         size_t(3) * g.R * g.nvg * 4 + size_t(3) * kD * 4 + size_t(g.R) * 4;
 }
 
 // Calls that flush at least this many groups use one CTA per (group, head);

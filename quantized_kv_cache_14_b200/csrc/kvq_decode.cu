@@ -1157,19 +1157,22 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
 }
 
 // Merge: one CTA per (row, kv head, query head).  The records of a pair are
-// the consumer warps of every CTA whose range holds its units.  The CTA's four
-// warps split those CTAs into four contiguous runs; each lane keeps a running
-// log-sum-exp over four channels, and the four runs are then combined in warp
-// order -- a fixed summation order for a given grid.
-constexpr int kMergeThreads = 128;
+// the consumer warps of every CTA whose range holds its units.  The CTA's
+// warps (4, 8 or 16: more when few pairs share the grid, so a long sequence's
+// pair, held by dozens of CTAs, is merged in few rounds) split those CTAs
+// into contiguous runs; each lane keeps a running log-sum-exp over four
+// channels, and the runs are then combined in warp order -- a fixed summation
+// order for a given grid and batch.
+constexpr int kMergeWarps = 16;
+constexpr int kMergeThreads = kMergeWarps * 32;
 
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_constant__ DecodeArgs a) {
   constexpr int D = kD;
   // launched as a programmatic dependent of the decode grid: wait until that
   // grid has completed and its writes are visible (returns at once otherwise)
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
-  __shared__ float s_m[4], s_den[4];
-  __shared__ float s_num[4][D];
+  __shared__ float s_m[kMergeWarps], s_den[kMergeWarps];
+  __shared__ float s_num[kMergeWarps][D];
   const Geo& g = a.g;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int G = g.G;
@@ -1179,7 +1182,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
   const int n = pre[i + 1] - pre[i];
   float* out = a.out + (int64_t(i) * g.h_q + h * G + hd) * D;
   if (n == 0) {
-    out[tid] = 0.0f;
+    if (tid < D) out[tid] = 0.0f;
     return;
   }
   const int64_t U = int64_t(pre[a.B]) * g.h_kv;
@@ -1191,7 +1194,8 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
   // nothing: walk the pair's units instead (then all values are below 2^20).
   const bool by_unit = U < GR;
   const int64_t nk = by_unit ? ub - ua + 1 : k1 - k0 + 1;
-  const int64_t kb = (int64_t(w) * nk) / 4, ke = (int64_t(w + 1) * nk) / 4;
+  const int nw = blockDim.x >> 5;
+  const int64_t kb = (int64_t(w) * nk) / nw, ke = (int64_t(w + 1) * nk) / nw;
   const int64_t rec_stride = int64_t(G) * (D + 2);
   float M = -INFINITY, den = 0.0f;
   float num[4] = {0.0f, 0.0f, 0.0f, 0.0f};
@@ -1234,13 +1238,16 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
 #pragma unroll
   for (int c = 0; c < 4; ++c) s_num[w][4 * lane + c] = num[c];
   __syncthreads();
+  if (tid >= D) return;
   float Mt = -INFINITY;
 #pragma unroll
-  for (int r = 0; r < 4; ++r) Mt = fmaxf(Mt, s_m[r]);
+  for (int r = 0; r < kMergeWarps; ++r)
+    if (r < nw) Mt = fmaxf(Mt, s_m[r]);
   float dt = 0.0f, nt = 0.0f;
   if (Mt != -INFINITY) {
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
+    for (int r = 0; r < kMergeWarps; ++r) {
+      if (r >= nw) break;
       const float wt = fast_exp2(s_m[r] - Mt);   // 0 for a run with nothing
       dt = fmaf(wt, s_den[r], dt);
       nt = fmaf(wt, s_num[r][tid], nt);
@@ -1364,8 +1371,12 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s, cudaEvent_t betwe
   // The merge is a programmatic dependent launch, so its launch overlaps the
   // decode grid's tail; with an event between the two it is a plain launch.
   cudaLaunchConfig_t cfg = {};
+  // about grid / (B h_kv) CTAs hold each pair: 4 warps up to 4 of them, 8 up
+  // to 8, else 16
+  const int per_pair = (a.grid + a.B * a.g.h_kv - 1) / (a.B * a.g.h_kv);
+  const int merge_warps = per_pair <= 4 ? 4 : per_pair <= 8 ? 8 : kMergeWarps;
   cfg.gridDim = dim3(items);
-  cfg.blockDim = dim3(kMergeThreads);
+  cfg.blockDim = dim3(32 * merge_warps);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];

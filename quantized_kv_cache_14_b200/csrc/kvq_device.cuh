@@ -322,6 +322,62 @@ __device__ __forceinline__ int quant_asym(float x, float sh, float zh, int Qa) {
   return q < 0 ? 0 : (q > Qa ? Qa : q);
 }
 
+// The same codes through a multiply by inv = RN(1 / sh) (__frcp_rn, once per
+// scale).  y = fl(x * inv) is within (2^-23 + 2^-24) |x / sh| of the IEEE
+// quotient fl(x / sh) (each of the reciprocal, the product and the quotient
+// is one rounding, relative error <= 2^-24).  For |y| < 256 that is below
+// 2^-13.4, so when y lies farther than 2^-13 from the half-integer between
+// its two neighbouring integers, y and fl(x / sh) round to the same integer;
+// |y| >= 256 clips to +-Q either way (Q <= 255).  Only the rare y near a
+// half-integer, a zero scale, or a non-finite product (NaN, or an infinite
+// reciprocal of a tiny fp32 scale) takes the exact division.
+// The exact fallbacks of the fast quantizers below, out of line so that the
+// rare call stays a branch instead of being computed for every element.
+static __device__ __noinline__ int quant_sym_exact(float x, float sh, int Q) { return quant_sym(x, sh, Q); }
+static __device__ __noinline__ int quant_asym_exact(float x, float sh, float zh, int Qa) { return quant_asym(x, sh, zh, Qa); }
+
+__device__ __forceinline__ int quant_sym_fast(float x, float sh, float inv, int Q) {
+  const float y = x * inv;
+  const float ay = fabsf(y);
+  if (ay >= 256.0f) return y > 0.0f ? Q : -Q;   // infinite y included
+  const float f = y - floorf(y);                 // exact for |y| < 2^23
+  if (sh != 0.0f && fabsf(f - 0.5f) > 0.0001220703125f) {
+    const int q = __float2int_rn(y);
+    return q < -Q ? -Q : (q > Q ? Q : q);
+  }
+  return quant_sym_exact(x, sh, Q);
+}
+
+__device__ __forceinline__ int quant_asym_fast(float x, float sh, float inv, float zh, int Qa) {
+  const float y = __fsub_rn(x, zh) * inv;
+  const float ay = fabsf(y);
+  if (ay >= 256.0f) return y > 0.0f ? Qa : 0;
+  const float f = y - floorf(y);
+  if (sh != 0.0f && fabsf(f - 0.5f) > 0.0001220703125f) {
+    const int q = __float2int_rn(y);
+    return q < 0 ? 0 : (q > Qa ? Qa : q);
+  }
+  return quant_asym_exact(x, sh, zh, Qa);
+}
+
+// Branch-free form of the fast quantizers for bulk work: the code of y =
+// x * inv (or (x - zh) * inv) clipped to [lo, hi], and `tie` set when |y| <
+// 256 lies within 2^-13 of a half-integer -- then (and only then) the caller
+// must take quant_sym / quant_asym instead.  |y| >= 256 needs no test: the
+// code clips either way.  With a zero scale inv is 0, so y = 0 and the code 0
+// (the exact quantizer's zero group) for every finite x; a NaN y gives code 0,
+// as the conversion of the exact quotient does.
+__device__ __forceinline__ int quant_code_nb(float y, int lo, int hi, bool& tie) {
+  const float r = rintf(y);
+  const float d = fabsf(y - r);
+  tie = !(d <= 0.4998779296875f) && fabsf(y) < 256.0f;   // 0.5 - 2^-13
+  const int q = __float2int_rn(r);
+  return q < lo ? lo : (q > hi ? hi : q);
+}
+
+// RN(1 / sh) for the fast quantizers (0 for a zero scale: those codes are 0).
+__device__ __forceinline__ float quant_inv(float sh) { return sh != 0.0f ? __frcp_rn(sh) : 0.0f; }
+
 __device__ __forceinline__ void store_meta(uint8_t* p, float v, int scale_fp32) {
   if (scale_fp32) *reinterpret_cast<float*>(p) = v;
   else *reinterpret_cast<uint16_t*>(p) = __half_as_ushort(__float2half_rn(v));
