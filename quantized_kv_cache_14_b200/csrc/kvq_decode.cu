@@ -1256,6 +1256,577 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
   out[tid] = dt > 0.0f ? nt / dt : 0.0f;
 }
 
+// ---------------------------------------------------------------------------
+// Warp-specialised decode of the INT4 KIVI format.  A CTA holds four pairs of
+// warps; pair p takes the units n = p, p + 4, ... of the CTA's share (as warp
+// p of decode_kernel does) through three shared-memory stages of its own.
+//  * The score warp waits for a unit's stage, forms q' (and the key offset)
+//    for its key group, computes the 64 scores with the subnormal-code path,
+//    takes the online-softmax step, and hands the unit's weights p and the
+//    rescale factor alpha of its running max to the value warp through a
+//    slot in shared memory (its next unit's scores are computed while the
+//    value warp still reads the slot; only the write waits).
+//  * The value warp takes the weights, rescales its accumulators by alpha,
+//    runs the value products, frees the slot and the stage, and issues the
+//    bulk copies of the pair's unit three ahead into that stage.
+// Each warp keeps half the state of a decode_kernel warp (the score warp q'
+// and q, the value warp the accumulators), so two CTAs of eight warps fit per
+// SM: four warps per scheduler, each running a shorter dependency chain.
+// Every wait is bounded; the pair leaves the same (m, l, o) records as
+// decode_kernel (m, l from the score warp, o from the value warp).
+constexpr int kWsPairs = kDecodeWarps;
+constexpr int kWsThreads = 2 * kWsPairs * 32;
+constexpr int kWsStages = 3;                                  // stages per pair
+constexpr int kWsStageBytes = 4 * SpecInt4Kivi::chunk_used;   // one 64-token unit
+constexpr int kWsPbufFloats = 4 * 4 * 16;                     // weights of a unit: [sub-tile][head][token]
+
+struct WsLayout {
+  int stages, qbuf, pbuf, alpha, bars, flag, total;
+};
+
+__host__ __device__ inline WsLayout ws_layout(int B) {
+  WsLayout L;
+  L.stages = ((B + 1 + 32 + 3 * B) * 4 + 127) / 128 * 128;   // prefix, scan scratch, per-row info
+  L.qbuf = L.stages + kWsPairs * kWsStages * kWsStageBytes;
+  L.pbuf = L.qbuf + kWsPairs * kScratchBytes;
+  L.alpha = L.pbuf + kWsPairs * kWsPbufFloats * 4;
+  L.bars = L.alpha + kWsPairs * 4 * 4;
+  L.flag = L.bars + kWsPairs * (kWsStages + 2) * 8;
+  L.total = L.flag + 16;
+  return L;
+}
+
+__global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_constant__ DecodeArgs a) {
+  constexpr int D = kD;
+  using S = SpecInt4Kivi;
+  constexpr uint32_t FULL = 0xffffffffu;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const Geo& g = a.g;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const bool vwarp = warp >= kWsPairs;
+  const int pr = warp & (kWsPairs - 1);
+  const WsLayout L = ws_layout(a.B);
+  int32_t* s_pre = reinterpret_cast<int32_t*>(smem);
+  int32_t* s_scr = s_pre + (a.B + 1);
+  int32_t* s_row = s_scr + 32;
+  const uint32_t sbase = smem_addr(smem);
+  const uint32_t bars = sbase + L.bars + 8u * uint32_t(pr * (kWsStages + 2));
+  auto full_bar = [&](int s) { return bars + 8u * s; };
+  const uint32_t pfull_bar = bars + 8u * kWsStages, pempty_bar = pfull_bar + 8u;
+  auto stage_of = [&](int s) { return smem + L.stages + (pr * kWsStages + s) * kWsStageBytes; };
+  float* pbuf = reinterpret_cast<float*>(smem + L.pbuf) + pr * kWsPbufFloats;
+  float* alphas = reinterpret_cast<float*>(smem + L.alpha) + pr * 4;
+  volatile int32_t* abort_flag = reinterpret_cast<int32_t*>(smem + L.flag);
+
+  // the merge grid may be scheduled now; it waits for this grid to complete
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+
+  // ---- the work list: units per row, prefix over rows ---------------------
+  for (int i = tid; i < a.B; i += blockDim.x) {
+    const RowInfo ri = row_info(a, i, blockIdx.x == 0);
+    s_pre[i + 1] = ri.nq + ri.nr;
+    s_row[3 * i] = ri.seq;
+    s_row[3 * i + 1] = ri.qa;
+    s_row[3 * i + 2] = ri.ra;
+  }
+  if (tid == 0) {
+    for (int b = 0; b < kWsPairs * (kWsStages + 2); ++b) mbar_init(sbase + L.bars + 8u * b, 1);
+    *abort_flag = 0;
+    mbar_init_fence();
+  }
+  __syncthreads();
+  block_scan(s_pre, a.B, s_scr);
+  if (blockIdx.x == 0)
+    for (int i = tid; i <= a.B; i += blockDim.x) a.prefix[i] = s_pre[i];
+
+  const int64_t U = int64_t(s_pre[a.B]) * g.h_kv;
+  const int64_t c0 = int64_t(blockIdx.x) * U / a.grid, c1 = int64_t(blockIdx.x + 1) * U / a.grid;
+  if (c0 >= c1) return;
+  const int N = int(c1 - c0);
+  const int K = N > pr ? (N - pr + kWsPairs - 1) / kWsPairs : 0;   // units of this pair
+
+  auto rinfo = [&](int i) {
+    RowInfo r;
+    r.seq = s_row[3 * i];
+    r.qa = s_row[3 * i + 1];
+    r.ra = s_row[3 * i + 2];
+    r.nq = (r.qa + 63) >> 6;
+    r.nr = (r.ra + 15) >> 4;
+    r.trow = a.table + int64_t(a.table_by_seq ? r.seq : i) * a.table_stride;
+    return r;
+  };
+  auto step = [&](It& it, RowInfo& ri, int& n) {
+    const bool row_changed = it_next(it, s_pre, a.B, g.h_kv);
+    ++n;
+    if (row_changed && n < N) ri = rinfo(it.i);
+  };
+  auto advance4 = [&](It& it, RowInfo& ri, int& n) {
+    if (it.k + kWsPairs < it.n) {
+      it.k += kWsPairs;
+      n += kWsPairs;
+      return;
+    }
+    for (int t = 0; t < kWsPairs; ++t) step(it, ri, n);
+  };
+
+  const int gq = lane >> 2, tq = lane & 3;
+  const int hh = gq >> 1;               // head of this lane's B column
+  const bool is_lo = gq & 1;            // the column carries the lo part
+  const float C = a.qk_scale;
+  constexpr uint32_t ZA0 = 0x00080008u, ZA1 = 0x00800080u;   // all-zero codes, bits 0-3 / 4-7
+
+  It itc;
+  it_seek(itc, s_pre, a.B, g.h_kv, c0);
+  RowInfo ric = rinfo(itc.i);
+  int nc = 0;
+  int cur_pair = itc.i * g.h_kv + itc.h;
+  bool needs_setup = true;
+  auto rec_of = [&](int pair, int head) {
+    return a.partials + (((int64_t(pair) + blockIdx.x) * kWsPairs + pr) * S::G + head) * (D + 2);
+  };
+  // Sub-tile t of a quantized unit's stage: page t of the unit.
+  auto page_of = [&](const uint8_t* stg, int t) { return stg + t * S::chunk_used; };
+
+  if (!vwarp) {
+    // ============================ score warp ================================
+    float m = -INFINITY, l = 0.0f;
+    uint32_t bq[8][2];
+    uint32_t qh[4][2];
+    float cs = C;
+    bool bq_bf16 = false;
+    uint32_t* qbw = reinterpret_cast<uint32_t*>(smem + L.qbuf + pr * kScratchBytes);
+    auto qrow = [&](int row, int h, int head) { return a.q + (int64_t(row) * g.h_q + h * S::G + head) * D; };
+    auto emit_k = [&](int pair) {
+      float lt = l;
+      lt += __shfl_xor_sync(FULL, lt, 4);
+      lt += __shfl_xor_sync(FULL, lt, 8);
+      lt += __shfl_xor_sync(FULL, lt, 16);
+      if (gq == 0) {
+        float* rec = rec_of(pair, tq);
+        rec[0] = m;
+        rec[1] = lt;
+      }
+    };
+    auto walk_to = [&](int target) {
+      if (itc.k + (target - nc) < itc.n) {
+        itc.k += target - nc;
+        nc = target;
+        return;
+      }
+      while (nc < target) {
+        step(itc, ric, nc);
+        const int pid = itc.i * g.h_kv + itc.h;
+        if (pid != cur_pair) {
+          emit_k(cur_pair);
+          m = -INFINITY;
+          l = 0.0f;
+          cur_pair = pid;
+          needs_setup = true;
+        }
+      }
+    };
+    // q of the pair's heads as fp16 with the largest |q| in [1/2, 1) (then q s
+    // stays below 65504 for every fp16 scale s): this lane's share of the q'
+    // job, key-list channels 4 lane .. 4 lane + 3 of every head
+    auto setup = [&](int row, int h) {
+      const int f = 4 * lane;
+      uint32_t qw[4][2];
+#pragma unroll
+      for (int h2 = 0; h2 < 4; ++h2) {
+        const uint16_t* qr = qrow(row, h, h2);
+        qw[h2][0] = *reinterpret_cast<const uint32_t*>(qr + key_channel(f));
+        qw[h2][1] = *reinterpret_cast<const uint32_t*>(qr + key_channel(f + 2));
+      }
+      float amax = 0.0f;
+#pragma unroll
+      for (int h2 = 0; h2 < 4; ++h2)
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+          amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(qw[h2][e] << 16)), fabsf(__uint_as_float(qw[h2][e] & 0xFFFF0000u))));
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, o));
+      const int ex = amax > 0.0f ? min(max(int((__float_as_uint(amax) >> 23) & 0xFF) - 127 + 1, -100), 100) : 0;
+      const float down = pow2f(-ex);
+#pragma unroll
+      for (int h2 = 0; h2 < 4; ++h2)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const __half2 v = __floats2half2_rn(__uint_as_float(qw[h2][e] << 16) * down,
+                                              __uint_as_float(qw[h2][e] & 0xFFFF0000u) * down);
+          qh[h2][e] = *reinterpret_cast<const uint32_t*>(&v);
+        }
+      cs = C * pow2f(ex);
+      bq_bf16 = false;
+    };
+    // q' = q s_channel of the unit's key group as the score B operand (the
+    // b0-half channels 16 times larger for the subnormal codes): each lane
+    // scales 4 channels of every head, then the warp scratch transposes them
+    // into operand order (XOR-swizzled 16-byte slots, conflict-free reads)
+    auto qprime = [&](const uint8_t* stg) {
+      const int f = 4 * lane;
+      const uint8_t* km = stg + (f >> S::lg_kslice) * S::chunk_used + S::off_Km;
+      const int off = f & (S::kslice - 1);
+      const int t0 = lane >> 3, j = lane & 7;
+      const uint2 sr = *reinterpret_cast<const uint2*>(km + off * 2);
+      const __half2 s01 = *reinterpret_cast<const __half2*>(&sr.x), s23 = *reinterpret_cast<const __half2*>(&sr.y);
+      uint32_t qv[4][4];
+#pragma unroll
+      for (int h2 = 0; h2 < 4; ++h2) {
+        const __half2 qa = __hmul2(*reinterpret_cast<const __half2*>(&qh[h2][0]), __float2half2_rn(16.0f));
+        const __half2 qb = *reinterpret_cast<const __half2*>(&qh[h2][1]);
+        const __half2 ha = __hmul2(qa, s01), hb = __hmul2(qb, s23);
+        const __half2 la = __hfma2(qa, s01, __hneg2(ha)), lb = __hfma2(qb, s23, __hneg2(hb));
+        qv[h2][0] = *reinterpret_cast<const uint32_t*>(&ha);
+        qv[h2][1] = *reinterpret_cast<const uint32_t*>(&hb);
+        qv[h2][2] = *reinterpret_cast<const uint32_t*>(&la);
+        qv[h2][3] = *reinterpret_cast<const uint32_t*>(&lb);
+      }
+#pragma unroll
+      for (int pass = 0; pass < 2; ++pass) {
+        __syncwarp();
+        if ((j >> 2) == pass) {
+          const int j4 = j & 3;
+#pragma unroll
+          for (int h2 = 0; h2 < 4; ++h2) {
+            const int thi = 8 * h2 + t0, tlo = thi + 4;
+            *reinterpret_cast<uint2*>(qbw + thi * 8 + 4 * ((j4 >> 1) ^ ((thi >> 2) & 1)) + 2 * (j4 & 1)) =
+                make_uint2(qv[h2][0], qv[h2][1]);
+            *reinterpret_cast<uint2*>(qbw + tlo * 8 + 4 * ((j4 >> 1) ^ ((tlo >> 2) & 1)) + 2 * (j4 & 1)) =
+                make_uint2(qv[h2][2], qv[h2][3]);
+          }
+        }
+        __syncwarp();
+        const uint4* qb = reinterpret_cast<const uint4*>(qbw + lane * 8);
+        const int sw = (lane >> 2) & 1;
+#pragma unroll
+        for (int v = 0; v < 2; ++v) {
+          const uint4 x = qb[v ^ sw];
+          bq[4 * pass + 2 * v][0] = x.x; bq[4 * pass + 2 * v][1] = x.y;
+          bq[4 * pass + 2 * v + 1][0] = x.z; bq[4 * pass + 2 * v + 1][1] = x.w;
+        }
+      }
+      __syncwarp();
+      bq_bf16 = false;
+    };
+    auto score_sub = [&](const uint8_t* ksub, float cs20, float bias, int valid, float& s0, float& s1) {
+      uint32_t wa[4], wb[4];
+      load_key_words<4>(ksub, gq, tq, wa, wb);
+      float acc0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, acc1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int jj = j >> 1;
+        const uint32_t va = (j & 1) ? (wa[jj] >> 8) : wa[jj], vb = (j & 1) ? (wb[jj] >> 8) : wb[jj];
+        const uint32_t a0 = and_xor(va, 0x000F000Fu, ZA0), a1 = and_xor(vb, 0x000F000Fu, ZA0);
+        const uint32_t a2 = and_xor(va, 0x00F000F0u, ZA1), a3 = and_xor(vb, 0x00F000F0u, ZA1);
+        if (j & 1) mma_f16(acc1, a0, a1, a2, a3, bq[j][0], bq[j][1]);
+        else mma_f16(acc0, a0, a1, a2, a3, bq[j][0], bq[j][1]);
+      }
+      s0 = gq < valid ? fmaf(acc0[0] + acc0[1] + acc1[0] + acc1[1], cs20, bias) : -INFINITY;
+      s1 = gq + 8 < valid ? fmaf(acc0[2] + acc0[3] + acc1[2] + acc1[3], cs20, bias) : -INFINITY;
+    };
+    for (int k = 0; k < K; ++k) {
+      walk_to(pr + kWsPairs * k);
+      if (needs_setup) {
+        setup(itc.i, itc.h);
+        needs_setup = false;
+      }
+      const int s = k % kWsStages;
+      if (!__all_sync(FULL, wait_or_abort(full_bar(s), uint32_t((k / kWsStages) & 1), abort_flag))) {
+        if (lane == 0) {
+          atomicOr(a.err, KVQ_DEVERR_TIMEOUT);
+          *abort_flag = 1;
+        }
+        return;
+      }
+      const uint8_t* stg = stage_of(s);
+      float sc[8];
+      if (itc.k < ric.nq) {
+        const int valid = min(64, ric.qa - itc.k * 64);
+        qprime(stg);
+        float accb[4] = {0.0f, 0.0f, 0.0f, 0.0f};   // the key offset: q' against all-zero codes
+#pragma unroll
+        for (int j = 0; j < 8; ++j) mma_f16(accb, ZA0, ZA0, ZA1, ZA1, bq[j][0], bq[j][1]);
+        const float cs20 = cs * 1048576.0f, bias = -(accb[0] + accb[1]) * cs20;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) score_sub(page_of(stg, t), cs20, bias, valid - 16 * t, sc[2 * t], sc[2 * t + 1]);
+      } else {
+        // a 16-token tile of the BF16 window: q in bf16 against natural rows
+        if (!bq_bf16) {
+          const uint16_t* qr = qrow(itc.i, itc.h, hh);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint32_t t0 = *reinterpret_cast<const uint32_t*>(qr + key_channel(32 * tq + 4 * j));
+            const uint32_t t1 = *reinterpret_cast<const uint32_t*>(qr + key_channel(32 * tq + 4 * j + 2));
+            bq[j][0] = is_lo ? 0u : t0;   // q is exact in bf16: its lo part is zero
+            bq[j][1] = is_lo ? 0u : t1;
+          }
+          bq_bf16 = true;
+        }
+        const int valid = ric.ra - 16 * (itc.k - ric.nq);
+        const uint32_t kaddr = smem_addr(stg);
+        float acc0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, acc1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        const int mi = lane >> 3;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int r = (lane & 7) + 8 * (mi & 1), c = 16 * j + 8 * (mi >> 1);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(kaddr + (r * D + c) * 2, a0, a1, a2, a3);
+          if (j & 1) mma_bf16(acc1, a0, a1, a2, a3, bq[j][0], bq[j][1]);
+          else mma_bf16(acc0, a0, a1, a2, a3, bq[j][0], bq[j][1]);
+        }
+        sc[0] = gq < valid ? (acc0[0] + acc0[1] + acc1[0] + acc1[1]) * C : -INFINITY;
+        sc[1] = gq + 8 < valid ? (acc0[2] + acc0[3] + acc1[2] + acc1[3]) * C : -INFINITY;
+#pragma unroll
+        for (int t = 2; t < 8; ++t) sc[t] = -INFINITY;
+      }
+      // online softmax over the unit (log2 domain); alpha rescales what came before
+      float mx = fmaxf(fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3])), fmaxf(fmaxf(sc[4], sc[5]), fmaxf(sc[6], sc[7])));
+      mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 16));
+      float alpha = 1.0f;
+      if (mx > m) {   // also taken from -inf; keeps p <= 1
+        alpha = fast_exp2(m - mx);
+        l *= alpha;
+        m = mx;
+      }
+      const bool live = m != -INFINITY;
+      float pc[8], sum = 0.0f;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        pc[t] = live ? fast_exp2(sc[t] - m) : 0.0f;
+        sum += pc[t];
+      }
+      l += sum;
+      // hand the weights to the value warp (the slot is free once it took k - 1)
+      if (k >= 1 && !__all_sync(FULL, wait_or_abort(pempty_bar, uint32_t((k - 1) & 1), abort_flag))) {
+        if (lane == 0) {
+          atomicOr(a.err, KVQ_DEVERR_TIMEOUT);
+          *abort_flag = 1;
+        }
+        return;
+      }
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        pbuf[t * 64 + tq * 16 + gq] = pc[2 * t];
+        pbuf[t * 64 + tq * 16 + gq + 8] = pc[2 * t + 1];
+      }
+      if (gq == 0) alphas[tq] = alpha;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(pfull_bar);
+    }
+    walk_to(N - 1);
+    emit_k(cur_pair);
+  } else {
+    // ============================ value warp ================================
+    State st;
+    state_reset(st);
+    auto normalize = [&]() {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int gi = i >> 2;
+        st.o[i][0] = (st.o[i][0] - st.zc[gi][0]) * 16777216.0f;
+        st.o[i][1] = (st.o[i][1] - st.zc[gi][1]) * 16777216.0f;
+        st.o[i][2] = (st.o[i][2] - st.zc[gi][2]) * 1048576.0f;
+        st.o[i][3] = (st.o[i][3] - st.zc[gi][3]) * 1048576.0f;
+      }
+#pragma unroll
+      for (int gi = 0; gi < 2; ++gi)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) st.zc[gi][c] = 0.0f;
+      st.raw = false;
+    };
+    auto emit_v = [&](int pair) {
+      if (st.raw) normalize();
+      float* rec = rec_of(pair, tq);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        rec[2 + 16 * i + gq] = st.o[i][0] + st.o[i][1];
+        rec[2 + 16 * i + gq + 8] = st.o[i][2] + st.o[i][3];
+      }
+    };
+    auto walk_to = [&](int target) {
+      if (itc.k + (target - nc) < itc.n) {
+        itc.k += target - nc;
+        nc = target;
+        return;
+      }
+      while (nc < target) {
+        step(itc, ric, nc);
+        const int pid = itc.i * g.h_kv + itc.h;
+        if (pid != cur_pair) {
+          emit_v(cur_pair);
+          state_reset(st);
+          cur_pair = pid;
+        }
+      }
+    };
+    // this lane's block for a unit's copies (-1 when out of the table)
+    auto load_blk = [&](const It& it, const RowInfo& ri) -> int32_t {
+      if (it.k >= ri.nq || lane >= 4) return 0;   // a window tile, or no page for this lane
+      const int pg = ((it.k * 64) >> 4) + lane;
+      return pg < a.table_stride ? ri.trow[pg] : -1;
+    };
+    auto issue = [&](const It& it, const RowInfo& ri, int32_t blk, int s) {
+      const uint32_t dst = sbase + L.stages + uint32_t((pr * kWsStages + s) * kWsStageBytes);
+      const uint32_t bar = full_bar(s);
+      const bool window = it.k >= ri.nq;
+      const int ncopy = window ? 2 : 4;
+      const uint32_t total = window ? 2 * 16 * D * 2 : 4 * S::chunk_used;
+      const bool bad = !window && __any_sync(FULL, lane < 4 && (blk < 0 || blk >= g.num_blocks));
+      // the pair's generic-proxy reads of the stage come before the copies' writes
+      fence_proxy_async();
+      if (bad) {
+        if (lane == 0) {
+          atomicOr(a.err, KVQ_DEVERR_BLOCK_ID);
+          mbar_arrive_expect_tx(bar, 0);
+        }
+        return;
+      }
+      if (lane == 0) mbar_arrive_expect_tx(bar, total);
+      __syncwarp();
+      if (lane >= ncopy) return;
+      if (window) {
+        const int kr = it.k - ri.nq;
+        const int64_t base = ((int64_t(ri.seq) * g.h_kv + it.h) * S::R + 16 * kr) * D;
+        bulk_g2s(dst + lane * (16 * D * 2), (lane ? a.vres : a.kres) + base, 16 * D * 2, bar);
+        return;
+      }
+      const uint8_t* chunk = a.pool + int64_t(blk) * g.block_bytes + int64_t(it.h) * g.chunk_bytes;
+      bulk_g2s(dst + lane * S::chunk_used, chunk, uint32_t(S::chunk_used), bar);
+    };
+    // the value product of one 16-token page: weights p of tokens (2tq, 2tq + 1)
+    // and (2tq + 8, 2tq + 9) of head hh as fp16 hi + lo, times each value group's
+    // per-token scale; codes as fp16 subnormals (see score warp)
+    auto pv_sub = [&](const uint8_t* page, float pa0, float pb0, float pa1, float pb1) {
+      uint32_t vw[8];
+      load_value_words<4>(page + S::off_V, lane, vw);
+      uint32_t pha, pla, phb, plb;
+      split2h(pa0, pb0, pha, pla);
+      split2h(pa1, pb1, phb, plb);
+      const uint16_t* vs = reinterpret_cast<const uint16_t*>(page + S::off_Vm);
+      // rows 2tq, 2tq + 1 (and + 8) hold both groups' scales in 8 bytes
+      const uint2 ra = *reinterpret_cast<const uint2*>(vs + 4 * tq);
+      const uint2 rb = *reinterpret_cast<const uint2*>(vs + 4 * tq + 16);
+      uint32_t b0 = 0, b1 = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if ((i & 3) == 0) {
+          const int gi = i >> 2;
+          const uint32_t sel = gi ? 0x7632u : 0x5410u;
+          const uint32_t xa = __byte_perm(ra.x, ra.y, sel), xb = __byte_perm(rb.x, rb.y, sel);
+          const __half2 sa2 = *reinterpret_cast<const __half2*>(&xa), sb2 = *reinterpret_cast<const __half2*>(&xb);
+          auto two = [](uint32_t ph, uint32_t pl, __half2 sv, uint32_t& hi, uint32_t& lo) {
+            const __half2 x = *reinterpret_cast<const __half2*>(&ph), y = *reinterpret_cast<const __half2*>(&pl);
+            const __half2 h = __hmul2(x, sv);
+            const __half2 lw = __hfma2(y, sv, __hfma2(x, sv, __hneg2(h)));
+            hi = *reinterpret_cast<const uint32_t*>(&h);
+            lo = *reinterpret_cast<const uint32_t*>(&lw);
+          };
+          uint32_t h0, l0, h1, l1;
+          two(pha, pla, sa2, h0, l0);
+          two(phb, plb, sb2, h1, l1);
+          b0 = is_lo ? l0 : h0;
+          b1 = is_lo ? l1 : h1;
+          mma_f16(st.zc[gi], ZA0, ZA1, ZA0, ZA1, b0, b1);   // the offset 8 of every code
+        }
+        const uint32_t w = vw[i], w8 = w >> 8;
+        mma_f16(st.o[i], and_xor(w, 0x000F000Fu, ZA0), and_xor(w, 0x00F000F0u, ZA1), and_xor(w8, 0x000F000Fu, ZA0),
+                and_xor(w8, 0x00F000F0u, ZA1), b0, b1);
+      }
+    };
+
+    // copies: the pair's first three units, then one unit three ahead per unit
+    It iti = itc;
+    RowInfo rii = ric;
+    int ni = 0;
+    for (int t = 0; t < pr && t < N; ++t) step(iti, rii, ni);
+    int issued = 0, consumed = 0;
+    for (; issued < K && issued < kWsStages; ++issued) {
+      if (issued) advance4(iti, rii, ni);
+      issue(iti, rii, load_blk(iti, rii), issued);
+    }
+    int32_t blk_next = 0;
+    if (K > kWsStages) {
+      advance4(iti, rii, ni);
+      blk_next = load_blk(iti, rii);
+    }
+    bool aborted = false;
+    for (int k = 0; k < K; ++k) {
+      walk_to(pr + kWsPairs * k);
+      const int s = k % kWsStages;
+      const bool ok = wait_or_abort(pfull_bar, uint32_t(k & 1), abort_flag) &&
+                      wait_or_abort(full_bar(s), uint32_t((k / kWsStages) & 1), abort_flag);
+      if (!__all_sync(FULL, ok)) {
+        if (lane == 0) {
+          atomicOr(a.err, KVQ_DEVERR_TIMEOUT);
+          *abort_flag = 1;
+        }
+        aborted = true;
+        break;
+      }
+      ++consumed;
+      const float alpha = alphas[tq];
+      if (__any_sync(FULL, alpha != 1.0f)) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) st.o[i][c] *= alpha;
+#pragma unroll
+        for (int gi = 0; gi < 2; ++gi)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) st.zc[gi][c] *= alpha;
+      }
+      const float* pb = pbuf;
+      const uint8_t* stg = stage_of(s);
+      if (itc.k < ric.nq) {
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float2 x = *reinterpret_cast<const float2*>(pb + t * 64 + hh * 16 + 2 * tq);
+          const float2 y = *reinterpret_cast<const float2*>(pb + t * 64 + hh * 16 + 2 * tq + 8);
+          pv_sub(page_of(stg, t), x.x, x.y, y.x, y.y);
+        }
+        st.raw = true;
+      } else {
+        if (st.raw) normalize();
+        const float2 x = *reinterpret_cast<const float2*>(pb + hh * 16 + 2 * tq);
+        const float2 y = *reinterpret_cast<const float2*>(pb + hh * 16 + 2 * tq + 8);
+        uint32_t h0, l0, h1, l1;
+        split2(x.x, x.y, h0, l0);
+        split2(y.x, y.y, h1, l1);
+        const uint32_t b0 = is_lo ? l0 : h0, b1 = is_lo ? l1 : h1;
+        const uint32_t vaddr = smem_addr(stg) + 16 * D * 2;
+        const int mi = lane >> 3;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = (lane & 7) + 8 * (mi >> 1), c = 16 * i + 8 * (mi & 1);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_t(vaddr + (r * D + c) * 2, a0, a1, a2, a3);
+          mma_bf16(st.o[i], a0, a1, a2, a3, b0, b1);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(pempty_bar);
+      if (k + kWsStages < K) {   // the stage just read takes unit k + 3
+        issue(iti, rii, blk_next, s);
+        ++issued;
+        if (k + kWsStages + 1 < K) {
+          advance4(iti, rii, ni);
+          blk_next = load_blk(iti, rii);
+        }
+      }
+    }
+    if (aborted) {
+      // keep the CTA until this pair's copies in flight have landed (bounded)
+      for (int u = consumed; u < issued; ++u)
+        (void)mbar_wait_bounded(full_bar(u % kWsStages), uint32_t((u / kWsStages) & 1), kWaitNs);
+      return;
+    }
+    walk_to(N - 1);
+    emit_v(cur_pair);
+  }
+}
+
 template <int BITS, int ASYM, int KAXIS, int ES, int SPEC = 0>
 const void* kernel_of() {
   return reinterpret_cast<const void*>(&decode_kernel<BITS, ASYM, KAXIS, ES, SPEC>);
@@ -1282,7 +1853,7 @@ const void* decode_kernel_ptr(const Geo& g) {
 
 size_t decode_smem_bytes(const Geo& g, const DecodePipe& p, int B) {
   (void)g;
-  return size_t(smem_layout(B, p).total);
+  return p.ws ? size_t(ws_layout(B).total) : size_t(smem_layout(B, p).total);
 }
 
 size_t decode_partials_bytes(const Geo& g, int B, int grid) {
@@ -1351,15 +1922,33 @@ cudaError_t plan_decode(const Geo& g, int max_B, DecodePipe* out) {
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&p.ctas_per_sm, kern, kDecodeThreads, smem);
   if (e != cudaSuccess) return e;
   if (p.ctas_per_sm < 1) return cudaErrorInvalidConfiguration;
+  p.ws = 0;
+  if (spec_int4_kivi(g)) {
+    // the warp-specialised kernel when two of its CTAs fit per SM
+    const size_t wsm = size_t(ws_layout(max_B).total);
+    if (2 * (wsm + size_t(reserved)) <= size_t(per_sm) && wsm <= size_t(max_optin)) {
+      const void* wk = reinterpret_cast<const void*>(&decode_ws_kernel);
+      e = raise_smem_limit(dev, wk, wsm);
+      if (e != cudaSuccess) return e;
+      int occ = 0;
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, wk, kWsThreads, wsm);
+      if (e != cudaSuccess) return e;
+      if (occ >= 2) {
+        p.ws = 1;
+        p.ctas_per_sm = occ;
+      }
+    }
+  }
   *out = p;
   return cudaSuccess;
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s, cudaEvent_t between, int* launches) {
-  const void* k = decode_kernel_ptr(a.g);
+  const void* k = a.pipe.ws ? reinterpret_cast<const void*>(&decode_ws_kernel) : decode_kernel_ptr(a.g);
   void* args[] = {const_cast<DecodeArgs*>(&a)};
   const size_t smem = decode_smem_bytes(a.g, a.pipe, a.B);
-  cudaError_t e = cudaLaunchKernel(k, dim3(a.grid), dim3(kDecodeThreads), args, smem, s);
+  cudaError_t e =
+      cudaLaunchKernel(k, dim3(a.grid), dim3(a.pipe.ws ? kWsThreads : kDecodeThreads), args, smem, s);
   if (e != cudaSuccess) return e;
   ++*launches;
   if (between) {

@@ -70,6 +70,7 @@ struct DecodePipe {
   int stage_bytes;  // one stage: a quantized unit or a 16-token BF16 window tile
   int nstages;
   int ctas_per_sm;  // resident CTAs per SM at the largest batch
+  int ws;           // 1: the warp-specialised kernel of the INT4 KIVI format
 };
 
 struct DecodeArgs {
