@@ -200,6 +200,18 @@ struct SpecInt4Kivi {
   static constexpr int n = 8, row_bytes = 64, sub_bytes = 1024, es = 2, nvg = 2, kslice = 32;
   static constexpr int off_V = 1024, off_Vm = 2048, off_Km = 2112, chunk_used = 2176;
   static constexpr int lg_P = 4, lg_gk = 6, lg_kslice = 5;
+  static constexpr int ws_stages = 3;   // warp-specialised kernel: stages per warp pair
+};
+
+// The INT2 asymmetric KIVI format (keys per channel G = 32, values per token
+// G = 32, fp16 scale and zero-point, BF16 window 32, page 16, 4 query heads per
+// kv head): only the warp-specialised kernel has a path of its own for it.
+struct SpecInt2Kivi {
+  static constexpr int bits = 2, asym = 1, k_axis = 1, g_k = 32, g_v = 32, scale_fp32 = 0, R = 32, P = 16, G = 4;
+  static constexpr int n = 16, row_bytes = 32, sub_bytes = 512, es = 2, nvg = 4, kslice = 64;
+  static constexpr int off_V = 512, off_Vm = 1024, off_Km = 1280, chunk_used = 1536;
+  static constexpr int lg_P = 4, lg_gk = 5, lg_kslice = 6;
+  static constexpr int ws_stages = 3;
 };
 
 template <int SPEC>
@@ -216,8 +228,8 @@ __device__ __forceinline__ Geo geo_of(const Geo& rt) {
   return g;
 }
 
-bool spec_int4_kivi(const Geo& g) {
-  using S = SpecInt4Kivi;
+template <class S>
+bool spec_matches(const Geo& g) {
   return g.bits == S::bits && g.asym == S::asym && g.k_axis == S::k_axis && g.g_k == S::g_k &&
          g.g_v == S::g_v && g.scale_fp32 == S::scale_fp32 && g.R == S::R && g.P == S::P && g.G == S::G &&
          g.n == S::n && g.row_bytes == S::row_bytes && g.sub_bytes == S::sub_bytes && g.es == S::es &&
@@ -225,6 +237,9 @@ bool spec_int4_kivi(const Geo& g) {
          g.off_Km == S::off_Km && g.chunk_used == S::chunk_used && g.lg_P == S::lg_P && g.lg_gk == S::lg_gk &&
          g.lg_kslice == S::lg_kslice;
 }
+
+bool spec_int4_kivi(const Geo& g) { return spec_matches<SpecInt4Kivi>(g); }
+bool spec_int2_kivi(const Geo& g) { return spec_matches<SpecInt2Kivi>(g); }
 
 template <int BITS, int ASYM, int KAXIS, int ES, int SPEC>
 __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_constant__ DecodeArgs a) {
@@ -541,7 +556,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
       }
       if (ES == 2) {
         // q as fp16 with the largest |q| of the pair in [1/2, 1): then
-        // q * s stays below 65504 for every fp16 scale s
+        // q * s stays below 65504 for every fp16 scale s.  The subnormal-code
+        // path multiplies half of q by 16, so it takes [2^-5, 2^-4) instead.
         float amax = 0.0f;
 #pragma unroll
         for (int h2 = 0; h2 < 4; ++h2)
@@ -551,7 +567,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
                                      fabsf(__uint_as_float(qw[h2][e] & 0xFFFF0000u))));
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        const int ex = amax > 0.0f ? min(max(int((__float_as_uint(amax) >> 23) & 0xFF) - 127 + 1, -100), 100) : 0;
+        const int ex = amax > 0.0f ? min(max(int((__float_as_uint(amax) >> 23) & 0xFF) - 127 + (SPEC ? 5 : 1), -100), 100)
+                                   : 0;
         const float down = pow2f(-ex);
 #pragma unroll
         for (int h2 = 0; h2 < 4; ++h2)
@@ -1257,9 +1274,14 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
 }
 
 // ---------------------------------------------------------------------------
-// Warp-specialised decode of the INT4 KIVI format.  A CTA holds four pairs of
-// warps; pair p takes the units n = p, p + 4, ... of the CTA's share (as warp
-// p of decode_kernel does) through three shared-memory stages of its own.
+// Warp-specialised decode of the two KIVI-style formats that have whole-unit
+// straight-line paths: INT4 symmetric (keys per channel G = 64, values per
+// token G = 64, BF16 window 64) and INT2 asymmetric (G = 32 for both, fp16
+// scale and zero-point, BF16 window 32), 4 query heads per kv head, page 16.
+// A unit is 64 tokens (one INT4 key group, two INT2 key groups).  A CTA holds
+// four pairs of warps; pair p takes the units n = p, p + 4, ... of the CTA's
+// share (as warp p of decode_kernel does) through three shared-memory stages
+// of its own.
 //  * The score warp waits for a unit's stage, forms q' (and the key offset)
 //    for its key group, computes the 64 scores with the subnormal-code path,
 //    takes the online-softmax step, and hands the unit's weights p and the
@@ -1276,36 +1298,46 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
 // decode_kernel (m, l from the score warp, o from the value warp).
 constexpr int kWsPairs = kDecodeWarps;
 constexpr int kWsThreads = 2 * kWsPairs * 32;
-constexpr int kWsStages = 3;                                  // stages per pair
-constexpr int kWsStageBytes = 4 * SpecInt4Kivi::chunk_used;   // one 64-token unit
-constexpr int kWsPbufFloats = 4 * 4 * 16;                     // weights of a unit: [sub-tile][head][token]
+constexpr int kWsPbufFloats = 4 * 4 * 16;   // weights of a unit: [sub-tile][head][token]
 
 struct WsLayout {
   int stages, qbuf, pbuf, alpha, bars, flag, total;
 };
 
+// A stage holds a unit's 4 pages or a 16-token window tile (K and V rows).
+template <class S>
+__host__ __device__ constexpr int ws_stage_bytes() {
+  return 4 * S::chunk_used > 2 * 16 * kD * 2 ? 4 * S::chunk_used : 2 * 16 * kD * 2;
+}
+
+// S::ws_stages stages per pair; the q' transposition scratch only for INT4
+// (INT2 keeps q in operand order instead).
+template <class S>
 __host__ __device__ inline WsLayout ws_layout(int B) {
   WsLayout L;
   L.stages = ((B + 1 + 32 + 3 * B) * 4 + 127) / 128 * 128;   // prefix, scan scratch, per-row info
-  L.qbuf = L.stages + kWsPairs * kWsStages * kWsStageBytes;
-  L.pbuf = L.qbuf + kWsPairs * kScratchBytes;
+  L.qbuf = L.stages + kWsPairs * S::ws_stages * ws_stage_bytes<S>();
+  L.pbuf = L.qbuf + (S::bits == 4 ? kWsPairs * kScratchBytes : 0);
   L.alpha = L.pbuf + kWsPairs * kWsPbufFloats * 4;
   L.bars = L.alpha + kWsPairs * 4 * 4;
-  L.flag = L.bars + kWsPairs * (kWsStages + 2) * 8;
+  L.flag = L.bars + kWsPairs * (S::ws_stages + 2) * 8;
   L.total = L.flag + 16;
   return L;
 }
 
+template <class S>
 __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_constant__ DecodeArgs a) {
   constexpr int D = kD;
-  using S = SpecInt4Kivi;
+  constexpr bool I2 = S::bits == 2;
+  constexpr int kWsStages = S::ws_stages;                 // stages per pair
+  constexpr int kWsStageBytes = ws_stage_bytes<S>();      // one 64-token unit or window tile
   constexpr uint32_t FULL = 0xffffffffu;
   extern __shared__ __align__(128) uint8_t smem[];
   const Geo& g = a.g;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool vwarp = warp >= kWsPairs;
   const int pr = warp & (kWsPairs - 1);
-  const WsLayout L = ws_layout(a.B);
+  const WsLayout L = ws_layout<S>(a.B);
   int32_t* s_pre = reinterpret_cast<int32_t*>(smem);
   int32_t* s_scr = s_pre + (a.B + 1);
   int32_t* s_row = s_scr + 32;
@@ -1391,7 +1423,8 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
     // ============================ score warp ================================
     float m = -INFINITY, l = 0.0f;
     uint32_t bq[8][2];
-    uint32_t qh[4][2];
+    uint32_t qh[4][2];   // INT4: this lane's q' job share, fp16
+    uint32_t qF[8][2];   // INT2: q in score-operand order, fp16, times the code weights
     float cs = C;
     bool bq_bf16 = false;
     uint32_t* qbw = reinterpret_cast<uint32_t*>(smem + L.qbuf + pr * kScratchBytes);
@@ -1425,9 +1458,11 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
         }
       }
     };
-    // q of the pair's heads as fp16 with the largest |q| in [1/2, 1) (then q s
-    // stays below 65504 for every fp16 scale s): this lane's share of the q'
-    // job, key-list channels 4 lane .. 4 lane + 3 of every head
+    // q of the pair's heads as fp16 with the largest |q| in [2^-5, 2^-4): then
+    // 16 q s stays below 65504 for every fp16 scale s, and an element that
+    // falls to an fp16 subnormal is off by at most 2^-25, 2^-20 of the largest.
+    // This lane's share of the q' job: key-list channels 4 lane .. 4 lane + 3
+    // of every head.
     auto setup = [&](int row, int h) {
       const int f = 4 * lane;
       uint32_t qw[4][2];
@@ -1445,7 +1480,7 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
           amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(qw[h2][e] << 16)), fabsf(__uint_as_float(qw[h2][e] & 0xFFFF0000u))));
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, o));
-      const int ex = amax > 0.0f ? min(max(int((__float_as_uint(amax) >> 23) & 0xFF) - 127 + 1, -100), 100) : 0;
+      const int ex = amax > 0.0f ? min(max(int((__float_as_uint(amax) >> 23) & 0xFF) - 127 + 5, -100), 100) : 0;
       const float down = pow2f(-ex);
 #pragma unroll
       for (int h2 = 0; h2 < 4; ++h2)
@@ -1457,6 +1492,103 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
         }
       cs = C * pow2f(ex);
       bq_bf16 = false;
+    };
+    // INT2: the 2-bit codes enter the products as fp16 subnormals, the code at
+    // bits 2y..2y+1 of a half-word worth c 4^y 2^-24 (y = 0..3, one shift by 8
+    // bringing the upper byte down).  Score product j takes its b0 half from
+    // y = 0 (j even) or 2 (j odd) and its b1 half from y + 1, so this lane's
+    // q in operand order carries the factors 2^-18 / weight: 64 and 16 (j
+    // even), 4 and 1 (j odd), and the products come out in units of 2^-18.
+    // The largest |q| lies in [2^-7, 2^-6): then 64 q s stays below 65504.
+    auto setup2 = [&](int row, int h) {
+      const uint16_t* qr = qrow(row, h, hh);
+      uint32_t t[8][2];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        t[j][0] = *reinterpret_cast<const uint32_t*>(qr + key_channel(32 * tq + 4 * j));
+        t[j][1] = *reinterpret_cast<const uint32_t*>(qr + key_channel(32 * tq + 4 * j + 2));
+      }
+      float amax = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+          amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(t[j][e] << 16)), fabsf(__uint_as_float(t[j][e] & 0xFFFF0000u))));
+      amax = __uint_as_float(__reduce_max_sync(FULL, __float_as_uint(amax)));
+      const int ex = amax > 0.0f ? min(max(int((__float_as_uint(amax) >> 23) & 0xFF) - 127 + 7, -100), 100) : 0;
+      const float down = pow2f(-ex);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float f = down * ((j & 1) ? (e ? 1.0f : 4.0f) : (e ? 16.0f : 64.0f));
+          const __half2 v = __floats2half2_rn(__uint_as_float(t[j][e] << 16) * f, __uint_as_float(t[j][e] & 0xFFFF0000u) * f);
+          qF[j][e] = *reinterpret_cast<const uint32_t*>(&v);
+        }
+      cs = C * pow2f(ex);
+      bq_bf16 = false;
+    };
+    // INT2, key group gk of a unit (pages 2 gk, 2 gk + 1): q' = q s as the score
+    // operand (hi in the even columns, lo in the odd ones) and the zero-point
+    // term sum_c q_c z_c of head tq, from this lane's 32 key-list positions
+    // 32 tq .. 32 tq + 31 (scales, then zero-points, in operand order).  The
+    // zero-point product runs on the tensor cores: z over the factors against
+    // the operand-order q.
+    auto group_q2 = [&](const uint8_t* stg, int gk) -> float {
+      const uint8_t* km = stg + (2 * gk + (tq >> 1)) * S::chunk_used + S::off_Km + 64 * (tq & 1);
+      const uint4* ks = reinterpret_cast<const uint4*>(km);
+      const uint4* kz = reinterpret_cast<const uint4*>(km + 2 * S::kslice);
+      float za0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, za1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const uint4 sv = ks[v], zv = kz[v];
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+          const int j = 2 * v + jj;
+          const uint32_t sw[2] = {jj ? sv.z : sv.x, jj ? sv.w : sv.y};
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const __half2 x = *reinterpret_cast<const __half2*>(&qF[j][e]), sc2 = *reinterpret_cast<const __half2*>(&sw[e]);
+            const __half2 hi = __hmul2(x, sc2);
+            const __half2 lo = __hfma2(x, sc2, __hneg2(hi));
+            bq[j][e] = is_lo ? *reinterpret_cast<const uint32_t*>(&lo) : *reinterpret_cast<const uint32_t*>(&hi);
+          }
+          const uint32_t z0 = jj ? zv.z : zv.x, z1 = jj ? zv.w : zv.y;
+          uint32_t zs0, zs1;
+          if (jj) {   // factors 4 and 1
+            const __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&z0), __float2half2_rn(0.25f));
+            zs0 = *reinterpret_cast<const uint32_t*>(&r);
+            zs1 = z1;
+          } else {    // factors 64 and 16
+            const __half2 r0 = __hmul2(*reinterpret_cast<const __half2*>(&z0), __float2half2_rn(0.015625f));
+            const __half2 r1 = __hmul2(*reinterpret_cast<const __half2*>(&z1), __float2half2_rn(0.0625f));
+            zs0 = *reinterpret_cast<const uint32_t*>(&r0);
+            zs1 = *reinterpret_cast<const uint32_t*>(&r1);
+          }
+          mma_f16(jj ? za1 : za0, zs0, zs0, zs1, zs1, qF[j][0], qF[j][1]);
+        }
+      }
+      bq_bf16 = false;
+      return za0[0] + za1[0];
+    };
+    // INT2 scores of one 16-token page: rows gq, gq + 8 hold 32 bytes of codes
+    // each, this lane's 8 at byte 8 tq
+    auto score_sub2 = [&](const uint8_t* ksub, float cs18, float csb, int valid, float& s0, float& s1) {
+      const uint2 x = *reinterpret_cast<const uint2*>(ksub + gq * S::row_bytes + 8 * tq);
+      const uint2 y = *reinterpret_cast<const uint2*>(ksub + (gq + 8) * S::row_bytes + 8 * tq);
+      const uint32_t wa[2] = {x.x, x.y}, wb[2] = {y.x, y.y};
+      const uint32_t ua[2] = {x.x >> 8, x.y >> 8}, ub[2] = {y.x >> 8, y.y >> 8};
+      float acc0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, acc1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int jj = j >> 2;
+        const uint32_t va = (j & 2) ? ua[jj] : wa[jj], vb = (j & 2) ? ub[jj] : wb[jj];
+        const uint32_t m0 = (j & 1) ? 0x00300030u : 0x00030003u, m1 = (j & 1) ? 0x00C000C0u : 0x000C000Cu;
+        if (j & 1) mma_f16(acc1, va & m0, vb & m0, va & m1, vb & m1, bq[j][0], bq[j][1]);
+        else mma_f16(acc0, va & m0, vb & m0, va & m1, vb & m1, bq[j][0], bq[j][1]);
+      }
+      s0 = gq < valid ? fmaf(acc0[0] + acc0[1] + acc1[0] + acc1[1], cs18, csb) : -INFINITY;
+      s1 = gq + 8 < valid ? fmaf(acc0[2] + acc0[3] + acc1[2] + acc1[3], cs18, csb) : -INFINITY;
     };
     // q' = q s_channel of the unit's key group as the score B operand (the
     // b0-half channels 16 times larger for the subnormal codes): each lane
@@ -1527,7 +1659,8 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
     for (int k = 0; k < K; ++k) {
       walk_to(pr + kWsPairs * k);
       if (needs_setup) {
-        setup(itc.i, itc.h);
+        if constexpr (I2) setup2(itc.i, itc.h);
+        else setup(itc.i, itc.h);
         needs_setup = false;
       }
       const int s = k % kWsStages;
@@ -1542,13 +1675,29 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
       float sc[8];
       if (itc.k < ric.nq) {
         const int valid = min(64, ric.qa - itc.k * 64);
-        qprime(stg);
-        float accb[4] = {0.0f, 0.0f, 0.0f, 0.0f};   // the key offset: q' against all-zero codes
+        if constexpr (I2) {
+          // one or two key groups of 32 tokens (the quantized length is a
+          // multiple of 32); a missing second group scores -inf
+          const float cs18 = cs * 262144.0f;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) mma_f16(accb, ZA0, ZA0, ZA1, ZA1, bq[j][0], bq[j][1]);
-        const float cs20 = cs * 1048576.0f, bias = -(accb[0] + accb[1]) * cs20;
+          for (int gk = 0; gk < 2; ++gk) {
+            if (gk == 0 || valid > 32) {
+              const float csb = cs * group_q2(stg, gk);
+              score_sub2(page_of(stg, 2 * gk), cs18, csb, valid - 32 * gk, sc[4 * gk], sc[4 * gk + 1]);
+              score_sub2(page_of(stg, 2 * gk + 1), cs18, csb, valid - 32 * gk - 16, sc[4 * gk + 2], sc[4 * gk + 3]);
+            } else {
+              sc[4] = sc[5] = sc[6] = sc[7] = -INFINITY;
+            }
+          }
+        } else {
+          qprime(stg);
+          float accb[4] = {0.0f, 0.0f, 0.0f, 0.0f};   // the key offset: q' against all-zero codes
 #pragma unroll
-        for (int t = 0; t < 4; ++t) score_sub(page_of(stg, t), cs20, bias, valid - 16 * t, sc[2 * t], sc[2 * t + 1]);
+          for (int j = 0; j < 8; ++j) mma_f16(accb, ZA0, ZA0, ZA1, ZA1, bq[j][0], bq[j][1]);
+          const float cs20 = cs * 1048576.0f, bias = -(accb[0] + accb[1]) * cs20;
+#pragma unroll
+          for (int t = 0; t < 4; ++t) score_sub(page_of(stg, t), cs20, bias, valid - 16 * t, sc[2 * t], sc[2 * t + 1]);
+        }
       } else {
         // a 16-token tile of the BF16 window: q in bf16 against natural rows
         if (!bq_bf16) {
@@ -1621,19 +1770,41 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
     // ============================ value warp ================================
     State st;
     state_reset(st);
+    float zv[4][4];   // INT2: p-weighted value zero-point sums per value group
+    auto zv_reset = [&]() {
+#pragma unroll
+      for (int gv = 0; gv < 4; ++gv)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) zv[gv][c] = 0.0f;
+    };
+    zv_reset();
     auto normalize = [&]() {
+      if constexpr (I2) {
+        // row gq of channel tile i holds codes worth 2^-24 (i even) or 2^-20
+        // (i odd), row gq + 8 four times that; then the zero-point terms
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int gi = i >> 2;
-        st.o[i][0] = (st.o[i][0] - st.zc[gi][0]) * 16777216.0f;
-        st.o[i][1] = (st.o[i][1] - st.zc[gi][1]) * 16777216.0f;
-        st.o[i][2] = (st.o[i][2] - st.zc[gi][2]) * 1048576.0f;
-        st.o[i][3] = (st.o[i][3] - st.zc[gi][3]) * 1048576.0f;
+        for (int i = 0; i < 8; ++i) {
+          const float fa = (i & 1) ? 1048576.0f : 16777216.0f, fb = (i & 1) ? 262144.0f : 4194304.0f;
+          st.o[i][0] = fmaf(st.o[i][0], fa, zv[i >> 1][0]);
+          st.o[i][1] = fmaf(st.o[i][1], fa, zv[i >> 1][1]);
+          st.o[i][2] = fmaf(st.o[i][2], fb, zv[i >> 1][2]);
+          st.o[i][3] = fmaf(st.o[i][3], fb, zv[i >> 1][3]);
+        }
+        zv_reset();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int gi = i >> 2;
+          st.o[i][0] = (st.o[i][0] - st.zc[gi][0]) * 16777216.0f;
+          st.o[i][1] = (st.o[i][1] - st.zc[gi][1]) * 16777216.0f;
+          st.o[i][2] = (st.o[i][2] - st.zc[gi][2]) * 1048576.0f;
+          st.o[i][3] = (st.o[i][3] - st.zc[gi][3]) * 1048576.0f;
+        }
+#pragma unroll
+        for (int gi = 0; gi < 2; ++gi)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) st.zc[gi][c] = 0.0f;
       }
-#pragma unroll
-      for (int gi = 0; gi < 2; ++gi)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) st.zc[gi][c] = 0.0f;
       st.raw = false;
     };
     auto emit_v = [&](int pair) {
@@ -1657,13 +1828,20 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
         if (pid != cur_pair) {
           emit_v(cur_pair);
           state_reset(st);
+          if constexpr (I2) zv_reset();
           cur_pair = pid;
         }
       }
     };
     // this lane's block for a unit's copies (-1 when out of the table)
+    // pages of a quantized unit: 4, or 2 for an INT2 unit whose attended
+    // tokens all lie in its first key group (a key group's scales span both
+    // of its pages, so pages follow whole groups)
+    auto unit_pages = [&](const It& it, const RowInfo& ri) {
+      return I2 && ri.qa - 64 * it.k <= 32 ? 2 : 4;
+    };
     auto load_blk = [&](const It& it, const RowInfo& ri) -> int32_t {
-      if (it.k >= ri.nq || lane >= 4) return 0;   // a window tile, or no page for this lane
+      if (it.k >= ri.nq || lane >= unit_pages(it, ri)) return 0;   // a window tile, or no page for this lane
       const int pg = ((it.k * 64) >> 4) + lane;
       return pg < a.table_stride ? ri.trow[pg] : -1;
     };
@@ -1671,9 +1849,10 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
       const uint32_t dst = sbase + L.stages + uint32_t((pr * kWsStages + s) * kWsStageBytes);
       const uint32_t bar = full_bar(s);
       const bool window = it.k >= ri.nq;
-      const int ncopy = window ? 2 : 4;
-      const uint32_t total = window ? 2 * 16 * D * 2 : 4 * S::chunk_used;
-      const bool bad = !window && __any_sync(FULL, lane < 4 && (blk < 0 || blk >= g.num_blocks));
+      const int npg = window ? 0 : unit_pages(it, ri);
+      const int ncopy = window ? 2 : npg;
+      const uint32_t total = window ? 2 * 16 * D * 2 : npg * S::chunk_used;
+      const bool bad = !window && __any_sync(FULL, lane < npg && (blk < 0 || blk >= g.num_blocks));
       // the pair's generic-proxy reads of the stage come before the copies' writes
       fence_proxy_async();
       if (bad) {
@@ -1736,6 +1915,53 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
       }
     };
 
+    // INT2 value product of one 16-token page: this lane's 16 bytes of codes
+    // (one word per value group of 32 channels, two channel tiles each), the
+    // weights p' = p s of each value group as fp16 hi + lo, and the zero-point
+    // term: z of tokens (2tq, 2tq + 1) and (2tq + 8, 2tq + 9) against p hi + lo,
+    // the same for every channel of the group.  Tile 2 gv takes the codes at
+    // y = 0, 1 (rows gq, gq + 8), tile 2 gv + 1 those at y = 2, 3, each from the
+    // word and from the word shifted down by 8 (the second half of the tokens).
+    auto pv_sub2 = [&](const uint8_t* page, float pa0, float pb0, float pa1, float pb1) {
+      const uint4 vq = *reinterpret_cast<const uint4*>(page + S::off_V + 16 * lane);
+      const uint32_t vw[4] = {vq.x, vq.y, vq.z, vq.w};
+      uint32_t pha, pla, phb, plb;
+      split2h(pa0, pb0, pha, pla);
+      split2h(pa1, pb1, phb, plb);
+      // token rows of 4 scales: rows 2tq, 2tq + 1 in 16 bytes, rows 2tq + 8,
+      // 2tq + 9 likewise; the zero-points follow the 16 rows of scales
+      const uint16_t* vs = reinterpret_cast<const uint16_t*>(page + S::off_Vm);
+      const uint4 ra = *reinterpret_cast<const uint4*>(vs + 8 * tq);
+      const uint4 rb = *reinterpret_cast<const uint4*>(vs + 8 * tq + 32);
+      const uint4 qa = *reinterpret_cast<const uint4*>(vs + 64 + 8 * tq);
+      const uint4 qb = *reinterpret_cast<const uint4*>(vs + 64 + 8 * tq + 32);
+      const uint32_t bza = is_lo ? pla : pha, bzb = is_lo ? plb : phb;
+      auto two = [](uint32_t ph, uint32_t pl, uint32_t svb, uint32_t& hi, uint32_t& lo) {
+        const __half2 x = *reinterpret_cast<const __half2*>(&ph), y = *reinterpret_cast<const __half2*>(&pl);
+        const __half2 sv = *reinterpret_cast<const __half2*>(&svb);
+        const __half2 h = __hmul2(x, sv);
+        const __half2 lw = __hfma2(y, sv, __hfma2(x, sv, __hneg2(h)));
+        hi = *reinterpret_cast<const uint32_t*>(&h);
+        lo = *reinterpret_cast<const uint32_t*>(&lw);
+      };
+#pragma unroll
+      for (int gv = 0; gv < 4; ++gv) {
+        const uint32_t sel = (gv & 1) ? 0x7632u : 0x5410u;
+        const uint32_t sa = __byte_perm(gv < 2 ? ra.x : ra.y, gv < 2 ? ra.z : ra.w, sel);
+        const uint32_t sb = __byte_perm(gv < 2 ? rb.x : rb.y, gv < 2 ? rb.z : rb.w, sel);
+        const uint32_t za = __byte_perm(gv < 2 ? qa.x : qa.y, gv < 2 ? qa.z : qa.w, sel);
+        const uint32_t zb = __byte_perm(gv < 2 ? qb.x : qb.y, gv < 2 ? qb.z : qb.w, sel);
+        uint32_t h0, l0, h1, l1;
+        two(pha, pla, sa, h0, l0);
+        two(phb, plb, sb, h1, l1);
+        const uint32_t b0 = is_lo ? l0 : h0, b1 = is_lo ? l1 : h1;
+        mma_f16(zv[gv], za, za, zb, zb, bza, bzb);
+        const uint32_t w = vw[gv], w8 = w >> 8;
+        mma_f16(st.o[2 * gv], w & 0x00030003u, w & 0x000C000Cu, w8 & 0x00030003u, w8 & 0x000C000Cu, b0, b1);
+        mma_f16(st.o[2 * gv + 1], w & 0x00300030u, w & 0x00C000C0u, w8 & 0x00300030u, w8 & 0x00C000C0u, b0, b1);
+      }
+    };
+
     // copies: the pair's first three units, then one unit three ahead per unit
     It iti = itc;
     RowInfo rii = ric;
@@ -1772,19 +1998,38 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
         for (int i = 0; i < 8; ++i)
 #pragma unroll
           for (int c = 0; c < 4; ++c) st.o[i][c] *= alpha;
+        if constexpr (I2) {
 #pragma unroll
-        for (int gi = 0; gi < 2; ++gi)
+          for (int gv = 0; gv < 4; ++gv)
 #pragma unroll
-          for (int c = 0; c < 4; ++c) st.zc[gi][c] *= alpha;
+            for (int c = 0; c < 4; ++c) zv[gv][c] *= alpha;
+        } else {
+#pragma unroll
+          for (int gi = 0; gi < 2; ++gi)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) st.zc[gi][c] *= alpha;
+        }
       }
       const float* pb = pbuf;
       const uint8_t* stg = stage_of(s);
       if (itc.k < ric.nq) {
+        if constexpr (I2) {
+          const int nt = unit_pages(itc, ric);   // 2 or 4 pages
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const float2 x = *reinterpret_cast<const float2*>(pb + t * 64 + hh * 16 + 2 * tq);
-          const float2 y = *reinterpret_cast<const float2*>(pb + t * 64 + hh * 16 + 2 * tq + 8);
-          pv_sub(page_of(stg, t), x.x, x.y, y.x, y.y);
+          for (int t = 0; t < 4; ++t) {
+            if (t < nt) {
+              const float2 x = *reinterpret_cast<const float2*>(pb + t * 64 + hh * 16 + 2 * tq);
+              const float2 y = *reinterpret_cast<const float2*>(pb + t * 64 + hh * 16 + 2 * tq + 8);
+              pv_sub2(page_of(stg, t), x.x, x.y, y.x, y.y);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const float2 x = *reinterpret_cast<const float2*>(pb + t * 64 + hh * 16 + 2 * tq);
+            const float2 y = *reinterpret_cast<const float2*>(pb + t * 64 + hh * 16 + 2 * tq + 8);
+            pv_sub(page_of(stg, t), x.x, x.y, y.x, y.y);
+          }
         }
         st.raw = true;
       } else {
@@ -1851,9 +2096,19 @@ const void* decode_kernel_ptr(const Geo& g) {
   }
 }
 
+// The warp-specialised kernel of a plan (pipe.ws: 1 INT4 KIVI, 2 INT2 KIVI).
+static const void* ws_kernel_ptr(int ws) {
+  return ws == 2 ? reinterpret_cast<const void*>(&decode_ws_kernel<SpecInt2Kivi>)
+                 : reinterpret_cast<const void*>(&decode_ws_kernel<SpecInt4Kivi>);
+}
+
+static size_t ws_smem_bytes(int ws, int B) {
+  return size_t(ws == 2 ? ws_layout<SpecInt2Kivi>(B).total : ws_layout<SpecInt4Kivi>(B).total);
+}
+
 size_t decode_smem_bytes(const Geo& g, const DecodePipe& p, int B) {
   (void)g;
-  return p.ws ? size_t(ws_layout(B).total) : size_t(smem_layout(B, p).total);
+  return p.ws ? ws_smem_bytes(p.ws, B) : size_t(smem_layout(B, p).total);
 }
 
 size_t decode_partials_bytes(const Geo& g, int B, int grid) {
@@ -1923,18 +2178,19 @@ cudaError_t plan_decode(const Geo& g, int max_B, DecodePipe* out) {
   if (e != cudaSuccess) return e;
   if (p.ctas_per_sm < 1) return cudaErrorInvalidConfiguration;
   p.ws = 0;
-  if (spec_int4_kivi(g)) {
+  const int ws = spec_int4_kivi(g) ? 1 : spec_int2_kivi(g) ? 2 : 0;
+  if (ws) {
     // the warp-specialised kernel when two of its CTAs fit per SM
-    const size_t wsm = size_t(ws_layout(max_B).total);
+    const size_t wsm = ws_smem_bytes(ws, max_B);
     if (2 * (wsm + size_t(reserved)) <= size_t(per_sm) && wsm <= size_t(max_optin)) {
-      const void* wk = reinterpret_cast<const void*>(&decode_ws_kernel);
+      const void* wk = ws_kernel_ptr(ws);
       e = raise_smem_limit(dev, wk, wsm);
       if (e != cudaSuccess) return e;
       int occ = 0;
       e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, wk, kWsThreads, wsm);
       if (e != cudaSuccess) return e;
       if (occ >= 2) {
-        p.ws = 1;
+        p.ws = ws;
         p.ctas_per_sm = occ;
       }
     }
@@ -1944,7 +2200,7 @@ cudaError_t plan_decode(const Geo& g, int max_B, DecodePipe* out) {
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s, cudaEvent_t between, int* launches) {
-  const void* k = a.pipe.ws ? reinterpret_cast<const void*>(&decode_ws_kernel) : decode_kernel_ptr(a.g);
+  const void* k = a.pipe.ws ? ws_kernel_ptr(a.pipe.ws) : decode_kernel_ptr(a.g);
   void* args[] = {const_cast<DecodeArgs*>(&a)};
   const size_t smem = decode_smem_bytes(a.g, a.pipe, a.B);
   cudaError_t e =

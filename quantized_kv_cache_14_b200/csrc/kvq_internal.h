@@ -70,7 +70,7 @@ struct DecodePipe {
   int stage_bytes;  // one stage: a quantized unit or a 16-token BF16 window tile
   int nstages;
   int ctas_per_sm;  // resident CTAs per SM at the largest batch
-  int ws;           // 1: the warp-specialised kernel of the INT4 KIVI format
+  int ws;           // the warp-specialised kernel: 1 for the INT4 KIVI format, 2 for INT2 KIVI
 };
 
 struct DecodeArgs {

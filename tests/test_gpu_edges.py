@@ -59,3 +59,25 @@ def test_quantizer_edges_bit_exact(name):
     q = random_bf16(rng, (1, h_q, D))
     p.check_decode(q, [L])
     p.close()
+
+
+@pytest.mark.parametrize("name", ["int4_chan64", "int2_asym_chan32"])
+def test_large_key_scales_decode(name):
+    """Keys of a few times 2^14 (fp16 scales in the thousands, well short of
+    saturation) with q near 2^-14, so the scores are ordinary: the key scale times q must
+    not overflow fp16 on any decode path, including the whole-unit paths of the
+    KIVI formats that weight parts of q by powers of two."""
+    fmt = FMTS[name]
+    rng = np.random.default_rng(11)
+    h_q, h_kv = 8, 2
+    p = Pair(fmt, h_q, h_kv, max_seqs=2, num_blocks=200, mbps=64, seed=5)
+    lens = [3 * fmt["g_k"] + 7, 2 * fmt["g_k"] + 40]
+    ids = np.repeat(np.arange(2, dtype=np.int32), lens)
+    k = random_bf16(rng, (ids.size, h_kv, D), 2.0 ** 14)
+    v = random_bf16(rng, (ids.size, h_kv, D))
+    p.append(k, v, ids)
+    p.check_state()
+    q = random_bf16(rng, (2, h_q, D), 2.0 ** -14)
+    p.check_decode(q, lens)
+    p.check_decode(q, [lens[0] - 20, lens[1] - 45])   # prefixes that end inside key groups
+    p.close()
