@@ -65,6 +65,14 @@ typedef enum kvq_status {
 #define KVQ_DEVERR_SEQ_LEN  0x2u   /* seq_lens[i] < 0 or > the stored length      */
 #define KVQ_DEVERR_TIMEOUT  0x4u   /* a bounded wait on a copy gave up            */
 #define KVQ_DEVERR_SEQ_ID   0x8u   /* decode row names an invalid sequence        */
+/* Debug build only (libkvq_debug.so, compiled with KVQ_DEBUG=1): the kernels
+ * check every index they compute against the buffer it addresses and skip
+ * the access instead of making it. */
+#define KVQ_DEVERR_SMEM     0x10u  /* a shared-memory stage read or copy outside
+                                      what the unit's copies filled          */
+#define KVQ_DEVERR_INDEX    0x20u  /* a global index (plan entry, window slot,
+                                      split-K record, pool chunk) outside its
+                                      buffer                                  */
 
 enum { KVQ_AXIS_TOKEN = 0, KVQ_AXIS_CHANNEL = 1 };
 

@@ -36,6 +36,19 @@ constexpr int kFlushCodeStride = kD + 8;
 // The plan's entries: inline in the launch parameters or uploaded.
 __device__ __forceinline__ const int32_t* plan_of(const PlanView& p) { return p.plan ? p.plan : p.inl; }
 
+// Debug build: the indices of one flush entry (sequence, page blocks, window
+// slots of the group's rows) lie inside their buffers.  Every thread of the
+// CTA reads the same entry, so the answer is uniform over the CTA.
+__device__ __forceinline__ bool flush_entry_ok(const Geo& g, const DevState& d, const int32_t* ent,
+                                               const int32_t* srcs) {
+  if (!KVQ_DEBUG) return true;
+  bool ok = ent[0] >= 0 && ent[0] < g.max_seqs && ent[2] >= 1 && ent[2] <= kFlushEntryInts - 3;
+  for (int j = 0; ok && j < ent[2]; ++j) ok = ent[3 + j] >= 0 && ent[3 + j] < g.num_blocks;
+  for (int r = 0; ok && r < g.R; ++r) ok = srcs[r] >= -g.R;
+  if (!ok && threadIdx.x == 0) atomicOr(d.err, KVQ_DEVERR_INDEX);
+  return ok;
+}
+
 // ---------------------------------------------------------------------------
 // Table and length updates and zeroing of new partial blocks, done by threads
 // tid, tid + nthr, ...; with `kin` given it also copies the plan's window rows
@@ -58,6 +71,8 @@ __device__ __forceinline__ void apply_body(const Geo& g, const DevState& d, cons
       const int32_t src = plan[p.off_res + 3 * e];
       const int32_t seq = plan[p.off_res + 3 * e + 1];
       const int32_t slot = plan[p.off_res + 3 * e + 2];
+      if (!dcheck(src >= 0 && seq >= 0 && seq < g.max_seqs && slot >= 0 && slot < g.R, d.err, KVQ_DEVERR_INDEX))
+        continue;
       const uint16_t* s = (which ? vin : kin) + (int64_t(src) * g.h_kv + h) * D;
       uint16_t* dst = (which ? d.vres : d.kres) + ((int64_t(seq) * g.h_kv + h) * g.R + slot) * D;
       reinterpret_cast<uint4*>(dst)[c8] = reinterpret_cast<const uint4*>(s)[c8];
@@ -68,11 +83,22 @@ __device__ __forceinline__ void apply_body(const Geo& g, const DevState& d, cons
   const int64_t zero_items = int64_t(p.n_zero) * per_block;
   for (int64_t i = tid; i < zero_items; i += nthr) {
     const int32_t blk = plan[p.off_zero + i / per_block];
+    if (!dcheck(blk >= 0 && blk < g.num_blocks, d.err, KVQ_DEVERR_INDEX)) continue;
     reinterpret_cast<uint4*>(d.pool + int64_t(blk) * g.block_bytes)[i % per_block] =
         make_uint4(0, 0, 0, 0);
   }
-  for (int64_t i = tid; i < p.n_tab; i += nthr) d.table[plan[p.off_tab + 2 * i]] = plan[p.off_tab + 2 * i + 1];
-  for (int64_t i = tid; i < p.n_len; i += nthr) d.len[plan[p.off_len + 2 * i]] = plan[p.off_len + 2 * i + 1];
+  for (int64_t i = tid; i < p.n_tab; i += nthr) {
+    const int32_t ti = plan[p.off_tab + 2 * i], tv = plan[p.off_tab + 2 * i + 1];
+    if (!dcheck(ti >= 0 && int64_t(ti) < int64_t(g.max_seqs) * g.mbps && tv >= -1 && tv < g.num_blocks, d.err,
+                KVQ_DEVERR_INDEX))
+      continue;
+    d.table[ti] = tv;
+  }
+  for (int64_t i = tid; i < p.n_len; i += nthr) {
+    const int32_t li = plan[p.off_len + 2 * i];
+    if (!dcheck(li >= 0 && li < g.max_seqs, d.err, KVQ_DEVERR_INDEX)) continue;
+    d.len[li] = plan[p.off_len + 2 * i + 1];
+  }
 }
 
 // Threads an apply body needs for a plan (window rows copied or not).
@@ -106,6 +132,8 @@ __global__ void __launch_bounds__(256) quant_token_kernel(const Geo g, const Dev
   const int32_t src = plan_of(p)[p.off_tok + 3 * e];
   const int32_t blk = plan_of(p)[p.off_tok + 3 * e + 1];
   const int32_t tok = plan_of(p)[p.off_tok + 3 * e + 2];
+  if (!dcheck(src >= 0 && blk >= 0 && blk < g.num_blocks && tok >= 0 && tok < g.P, d.err, KVQ_DEVERR_INDEX))
+    return;   // the warp's item, uniform over the warp
   uint8_t* chunk = d.pool + int64_t(blk) * g.block_bytes + int64_t(h) * g.chunk_bytes;
   const int sub = tok >> 4, r = tok & 15;
 
@@ -234,6 +262,7 @@ __global__ void __launch_bounds__(kFlushThreads) flush_kernel(const Geo g, const
   const int seq = ent[0];
   const int npg = ent[2];
   const int32_t* srcs = plan_of(p) + p.off_src + int64_t(e) * R;
+  if (!flush_entry_ok(g, d, ent, srcs)) return;
 
   // 1. gather the group's K rows and this sub-tile's V rows (bf16) into
   //    shared memory
@@ -419,6 +448,7 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
   const int32_t* ent = plan_of(p) + p.off_flush + e * kFlushEntryInts;
   const int seq = ent[0];
   const int32_t* srcs = plan_of(p) + p.off_src + int64_t(e) * R;
+  if (!flush_entry_ok(g, d, ent, srcs)) return;
   for (int r = tid; r < R; r += T) ssrc[r] = srcs[r];
   __syncthreads();
 
@@ -648,6 +678,8 @@ __global__ void residual_kernel(const Geo g, const DevState d, const __grid_cons
     const int32_t src = plan_of(p)[p.off_res + 3 * e];
     const int32_t seq = plan_of(p)[p.off_res + 3 * e + 1];
     const int32_t slot = plan_of(p)[p.off_res + 3 * e + 2];
+    if (!dcheck(src >= 0 && seq >= 0 && seq < g.max_seqs && slot >= 0 && slot < g.R, d.err, KVQ_DEVERR_INDEX))
+      continue;
     const uint16_t* s = (which ? vin : kin) + (int64_t(src) * g.h_kv + h) * D;
     uint16_t* dst = (which ? d.vres : d.kres) + ((int64_t(seq) * g.h_kv + h) * g.R + slot) * D;
     reinterpret_cast<uint4*>(dst)[c8] = reinterpret_cast<const uint4*>(s)[c8];
@@ -668,6 +700,8 @@ __global__ void __launch_bounds__(256) copy_token_kernel(const Geo g, const DevS
   const int32_t src = plan_of(p)[p.off_tok + 3 * e];
   const int32_t blk = plan_of(p)[p.off_tok + 3 * e + 1];
   const int32_t tok = plan_of(p)[p.off_tok + 3 * e + 2];
+  if (!dcheck(src >= 0 && blk >= 0 && blk < g.num_blocks && tok >= 0 && tok < g.P, d.err, KVQ_DEVERR_INDEX))
+    return;   // the warp's item, uniform over the warp
   uint8_t* chunk = d.pool + int64_t(blk) * g.block_bytes + int64_t(h) * g.chunk_bytes;
   const int64_t row = int64_t(tok >> 4) * g.sub_bytes + (tok & 15) * (D * 2);
   const int64_t in = (int64_t(src) * g.h_kv + h) * D + 4 * lane;
@@ -692,6 +726,8 @@ __global__ void __launch_bounds__(256) fp8_token_kernel(const Geo g, const DevSt
   const int32_t src = plan_of(p)[p.off_tok + 3 * e];
   const int32_t blk = plan_of(p)[p.off_tok + 3 * e + 1];
   const int32_t tok = plan_of(p)[p.off_tok + 3 * e + 2];
+  if (!dcheck(src >= 0 && blk >= 0 && blk < g.num_blocks && tok >= 0 && tok < g.P, d.err, KVQ_DEVERR_INDEX))
+    return;   // the warp's item, uniform over the warp
   uint8_t* chunk = d.pool + int64_t(blk) * g.block_bytes + int64_t(h) * g.chunk_bytes;
   const int sub = tok >> 4, r = tok & 15;
   const float sk = d.fp8[h], sv = d.fp8[g.h_kv + h];

@@ -378,12 +378,20 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
       ncopy = 2;
       total = 2 * 16 * kD * 2;
     }
-    const bool bad = !window && __any_sync(FULL, lane < ncopy && (blk < 0 || blk >= g.num_blocks));
+    bool bad = !window && __any_sync(FULL, lane < ncopy && (blk < 0 || blk >= g.num_blocks));
+    bool dbad = false;
+    if (KVQ_DEBUG && !bad) {
+      // the copies fit the stage, and a window tile's rows lie in the window
+      dbad = !dcheck(total <= uint32_t(pp.stage_bytes), a.err, KVQ_DEVERR_SMEM) ||
+             !dcheck(!window || (ri.seq >= 0 && ri.seq < g.max_seqs && 16 * (it.k - ri.nq) + 16 <= g.R), a.err,
+                     KVQ_DEVERR_INDEX);
+      dbad = __any_sync(FULL, dbad);
+    }
     // this warp's generic-proxy reads of the stage come before the copies' writes
     fence_proxy_async();
-    if (bad) {
+    if (bad || dbad) {
       if (lane == 0) {
-        atomicOr(a.err, KVQ_DEVERR_BLOCK_ID);
+        if (bad) atomicOr(a.err, KVQ_DEVERR_BLOCK_ID);
         mbar_arrive_expect_tx(bar, 0);
       }
       return;
@@ -525,7 +533,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
       }
       zt[i] = z;
     }
-    if (tq < g.G) {
+    if (tq < g.G && dcheck(int64_t(row) * g.h_kv + h + blockIdx.x < int64_t(a.B) * g.h_kv + a.grid, a.err,
+                           KVQ_DEVERR_INDEX)) {
       const int64_t pair = int64_t(row) * g.h_kv + h;
       float* rec = a.partials + (((pair + blockIdx.x) * kDecodeWarps + warp) * g.G + tq) * (D + 2);
       if (gq == 0) {
@@ -1218,6 +1227,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
   float num[4] = {0.0f, 0.0f, 0.0f, 0.0f};
   for (int64_t t = kb; t < ke; ++t) {
     const int64_t k = by_unit ? int64_t((int(ua + t + 1) * int(GR) - 1) / int(U)) : k0 + t;
+    if (!dcheck(k >= 0 && k < GR && int64_t(p) + k < int64_t(a.B) * g.h_kv + GR, a.err, KVQ_DEVERR_INDEX)) continue;
     const float* rec = a.partials + ((int64_t(p) + k) * kDecodeWarps * G + hd) * (D + 2);
     float m[kDecodeWarps], l[kDecodeWarps];
     float2 o[kDecodeWarps][2];
@@ -1301,7 +1311,7 @@ constexpr int kWsThreads = 2 * kWsPairs * 32;
 constexpr int kWsPbufFloats = 4 * 4 * 16;   // weights of a unit: [sub-tile][head][token]
 
 struct WsLayout {
-  int stages, qbuf, pbuf, alpha, bars, flag, total;
+  int stages, qbuf, pbuf, alpha, bars, flag, fill, total;
 };
 
 // A stage holds a unit's 4 pages or a 16-token window tile (K and V rows).
@@ -1321,7 +1331,8 @@ __host__ __device__ inline WsLayout ws_layout(int B) {
   L.alpha = L.pbuf + kWsPairs * kWsPbufFloats * 4;
   L.bars = L.alpha + kWsPairs * 4 * 4;
   L.flag = L.bars + kWsPairs * (S::ws_stages + 2) * 8;
-  L.total = L.flag + 16;
+  L.fill = L.flag + 16;   // debug build: pages each stage's copies filled (-1: a window tile)
+  L.total = L.fill + (KVQ_DEBUG ? (kWsPairs * S::ws_stages * 4 + 15) / 16 * 16 : 0);
   return L;
 }
 
@@ -1349,6 +1360,12 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
   float* pbuf = reinterpret_cast<float*>(smem + L.pbuf) + pr * kWsPbufFloats;
   float* alphas = reinterpret_cast<float*>(smem + L.alpha) + pr * 4;
   volatile int32_t* abort_flag = reinterpret_cast<int32_t*>(smem + L.flag);
+  int32_t* fill = reinterpret_cast<int32_t*>(smem + L.fill) + pr * kWsStages;   // debug build only
+  // debug build: a read of page t of stage s (t = -1: a window tile) must find
+  // it filled by the copies of the unit being read
+  auto page_filled = [&](int s, int t) {
+    return dcheck(t < 0 ? fill[s] == -1 : fill[s] > t, a.err, KVQ_DEVERR_SMEM);
+  };
 
   // the merge grid may be scheduled now; it waits for this grid to complete
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
@@ -1434,7 +1451,7 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
       lt += __shfl_xor_sync(FULL, lt, 4);
       lt += __shfl_xor_sync(FULL, lt, 8);
       lt += __shfl_xor_sync(FULL, lt, 16);
-      if (gq == 0) {
+      if (gq == 0 && dcheck(int64_t(pair) + blockIdx.x < int64_t(a.B) * g.h_kv + a.grid, a.err, KVQ_DEVERR_INDEX)) {
         float* rec = rec_of(pair, tq);
         rec[0] = m;
         rec[1] = lt;
@@ -1675,6 +1692,7 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
       float sc[8];
       if (itc.k < ric.nq) {
         const int valid = min(64, ric.qa - itc.k * 64);
+        (void)page_filled(s, I2 && valid <= 32 ? 1 : 3);
         if constexpr (I2) {
           // one or two key groups of 32 tokens (the quantized length is a
           // multiple of 32); a missing second group scores -inf
@@ -1700,6 +1718,7 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
         }
       } else {
         // a 16-token tile of the BF16 window: q in bf16 against natural rows
+        (void)page_filled(s, -1);
         if (!bq_bf16) {
           const uint16_t* qr = qrow(itc.i, itc.h, hh);
 #pragma unroll
@@ -1809,6 +1828,7 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
     };
     auto emit_v = [&](int pair) {
       if (st.raw) normalize();
+      if (!dcheck(int64_t(pair) + blockIdx.x < int64_t(a.B) * g.h_kv + a.grid, a.err, KVQ_DEVERR_INDEX)) return;
       float* rec = rec_of(pair, tq);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -1853,11 +1873,21 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
       const int ncopy = window ? 2 : npg;
       const uint32_t total = window ? 2 * 16 * D * 2 : npg * S::chunk_used;
       const bool bad = !window && __any_sync(FULL, lane < npg && (blk < 0 || blk >= g.num_blocks));
+      bool dbad = false;
+      if (KVQ_DEBUG) {
+        // the copies fit the stage, a window tile's rows lie in the window;
+        // record what the stage will hold for the readers' checks
+        dbad = !dcheck(s >= 0 && s < kWsStages && total <= uint32_t(kWsStageBytes), a.err, KVQ_DEVERR_SMEM) ||
+               !dcheck(!window || (ri.seq >= 0 && ri.seq < g.max_seqs && 16 * (it.k - ri.nq) + 16 <= S::R), a.err,
+                       KVQ_DEVERR_INDEX);
+        dbad = __any_sync(FULL, dbad);
+        if (lane == 0 && s >= 0 && s < kWsStages) fill[s] = bad || dbad ? 0 : (window ? -1 : npg);
+      }
       // the pair's generic-proxy reads of the stage come before the copies' writes
       fence_proxy_async();
-      if (bad) {
+      if (bad || dbad) {
         if (lane == 0) {
-          atomicOr(a.err, KVQ_DEVERR_BLOCK_ID);
+          if (bad) atomicOr(a.err, KVQ_DEVERR_BLOCK_ID);
           mbar_arrive_expect_tx(bar, 0);
         }
         return;
@@ -2013,6 +2043,7 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
       const float* pb = pbuf;
       const uint8_t* stg = stage_of(s);
       if (itc.k < ric.nq) {
+        (void)page_filled(s, unit_pages(itc, ric) - 1);
         if constexpr (I2) {
           const int nt = unit_pages(itc, ric);   // 2 or 4 pages
 #pragma unroll
@@ -2033,6 +2064,7 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
         }
         st.raw = true;
       } else {
+        (void)page_filled(s, -1);
         if (st.raw) normalize();
         const float2 x = *reinterpret_cast<const float2*>(pb + hh * 16 + 2 * tq);
         const float2 y = *reinterpret_cast<const float2*>(pb + hh * 16 + 2 * tq + 8);

@@ -41,6 +41,24 @@ __host__ __device__ constexpr uint32_t f16x2_of(float x) {
 }
 
 // ---------------------------------------------------------------------------
+// Debug-build checks.  With KVQ_DEBUG set (libkvq_debug.so) dcheck sets `bit`
+// in the device error word and returns false when `ok` fails, and the caller
+// skips the access; in the release build it is the constant true and compiles
+// away.
+// ---------------------------------------------------------------------------
+#ifndef KVQ_DEBUG
+#define KVQ_DEBUG 0
+#endif
+
+__device__ __forceinline__ bool dcheck(bool ok, uint32_t* err, uint32_t bit) {
+  if (KVQ_DEBUG && !ok) {
+    atomicOr(err, bit);
+    return false;
+  }
+  return true;
+}
+
+// ---------------------------------------------------------------------------
 // PTX wrappers.
 // ---------------------------------------------------------------------------
 

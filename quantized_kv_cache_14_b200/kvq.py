@@ -16,7 +16,9 @@ from dataclasses import dataclass
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libkvq.so")
+# KVQ_DEBUG=1 in the environment selects the debug build (kernels check every
+# index they compute; build.py --debug)
+LIB_PATH = os.path.join(_HERE, "libkvq_debug.so" if os.environ.get("KVQ_DEBUG") == "1" else "libkvq.so")
 
 KVQ_OK = 0
 KVQ_ERR_INVALID_ARG = 1
@@ -30,6 +32,8 @@ KVQ_DEVERR_BLOCK_ID = 0x1
 KVQ_DEVERR_SEQ_LEN = 0x2
 KVQ_DEVERR_TIMEOUT = 0x4
 KVQ_DEVERR_SEQ_ID = 0x8
+KVQ_DEVERR_SMEM = 0x10
+KVQ_DEVERR_INDEX = 0x20
 
 KVQ_AXIS_TOKEN = 0
 KVQ_AXIS_CHANNEL = 1

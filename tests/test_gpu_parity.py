@@ -513,3 +513,64 @@ def test_workload_5_continuous_batching():
     steps = int(os.environ.get("KVQ_CB_STEPS", "100"))
     checked = set(range(steps)) if os.environ.get("KVQ_CB_FULL") else {0, 1, 2, 49, 98, 99}
     run_full(5, steps_checked={s for s in checked if s < steps}, max_steps=steps)
+
+
+@pytest.mark.parametrize("name", ["int4_chan64", "int2_asym_chan32"])
+def test_merge_rows_and_repeats(name):
+    """Split-K merge of the warp-specialised KIVI kernels: rows that attend
+    nothing sit between live rows, and calls alternate batch size and grid
+    (pairs move between CTAs, a grid may exceed the resident CTAs and the unit
+    count); every call must match the oracle, empty rows giving zeros."""
+    rng = np.random.default_rng(12)
+    fmt = FMTS[name]
+    h_q, h_kv = 8, 2
+    p = Pair(fmt, h_q, h_kv, max_seqs=5, num_blocks=700, mbps=128, seed=2)
+    lens = [700, 1, 0, 333, 97]
+    ids = np.repeat(np.arange(5, dtype=np.int32), lens)
+    n = int(ids.size)
+    p.append(outlier_keys(rng, n, h_kv), random_bf16(rng, (n, h_kv, D)), ids)
+    for grid, attend in ((0, [700, 0, 0, 333, 97]), (3, [0, 1, 0, 0, 97]), (0, [700, 1, 0, 333]),
+                         (1024, [650, 1, 0, 300, 0]), (0, [700, 1, 0, 333, 97]), (7, [0, 0])):
+        p.gpu.set_decode_grid(grid)
+        q = random_bf16(rng, (len(attend), h_q, D))
+        got, want = p.decode(q, attend)
+        assert np.all(np.isfinite(got))
+        assert np.max(np.abs(got - want)) <= ATOL, (grid, attend)
+        for r, L in enumerate(attend):
+            if L == 0:
+                assert not np.any(got[r]), (grid, r)
+    assert p.gpu.sync_status() == 0
+    p.close()
+
+
+@pytest.mark.parametrize("name", ["int4_chan64", "int2_asym_chan32", "int8_tok_p16"])
+def test_device_check_flags_corrupted_caller_table(name):
+    """A caller block table with entries outside [0, num_blocks) sets
+    KVQ_DEVERR_BLOCK_ID: the kernels skip those copies instead of faulting,
+    and the next call on the same context decodes as the oracle says."""
+    rng = np.random.default_rng(9)
+    fmt = FMTS[name]
+    h_q, h_kv, S, stride = 8, 2, 2, 40
+    p = Pair(fmt, h_q, h_kv, max_seqs=S, num_blocks=120, mbps=stride, seed=4)
+    lens = [300, 170]
+    ids = np.repeat(np.arange(S, dtype=np.int32), lens)
+    p.append(outlier_keys(rng, ids.size, h_kv), random_bf16(rng, (ids.size, h_kv, D)), ids)
+    bt = np.full((S, stride), -1, np.int32)
+    for s in range(S):
+        row = p.gpu.block_table_host(s)
+        bt[s, :len(row)] = row
+    bad = bt.copy()
+    bad[0, 1] = -5
+    bad[1, 2] = 120 + 3
+    q = random_bf16(rng, (S, h_q, D))
+    p.gpu.decode(bits_to_cuda_bf16(q), torch.tensor(lens, dtype=torch.int32, device="cuda"),
+                 torch.zeros((S, h_q, D), dtype=torch.float32, device="cuda"),
+                 block_table=torch.from_numpy(bad).cuda(), bt_stride=stride)
+    from quantized_kv_cache_14_b200 import kvq
+    bits = p.gpu.sync_status()
+    assert bits & kvq.KVQ_DEVERR_BLOCK_ID, bits
+    assert p.gpu.sync_status() == 0
+    got, want = p.decode(q, lens, block_table=torch.from_numpy(bt).cuda(), bt_stride=stride)
+    assert np.max(np.abs(got - want)) <= ATOL
+    assert p.gpu.sync_status() == 0
+    p.close()
