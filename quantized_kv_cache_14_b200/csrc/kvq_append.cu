@@ -33,6 +33,13 @@ static_assert(sizeof(Geo) + sizeof(DevState) + sizeof(PlanView) + 3 * sizeof(voi
 // Row stride of the bulk flush's code arrays in shared memory (bytes).
 constexpr int kFlushCodeStride = kD + 8;
 
+// A decode launched right after an append is a programmatic dependent launch:
+// letting it be scheduled at the start of every append kernel hides its launch
+// behind the append (it waits for this grid on the device before it reads).
+__device__ __forceinline__ void launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
 // The plan's entries: inline in the launch parameters or uploaded.
 __device__ __forceinline__ const int32_t* plan_of(const PlanView& p) { return p.plan ? p.plan : p.inl; }
 
@@ -110,6 +117,7 @@ inline int64_t apply_work(const Geo& g, const PlanView& p, bool copy_rows) {
 
 __global__ void apply_kernel(const Geo g, const DevState d, const __grid_constant__ PlanView p,
                              const uint16_t* kin, const uint16_t* vin) {
+  launch_dependents();
   apply_body(g, d, p, kin, vin, int64_t(blockIdx.x) * blockDim.x + threadIdx.x,
              int64_t(gridDim.x) * blockDim.x);
 }
@@ -121,6 +129,7 @@ template <int BITS, int ASYM>
 __global__ void __launch_bounds__(256) quant_token_kernel(const Geo g, const DevState d,
                                                           const __grid_constant__ PlanView p, const uint16_t* kin,
                                                           const uint16_t* vin) {
+  launch_dependents();
   constexpr int D = kD;
   constexpr int N = 32 / BITS;                 // codes per word
   constexpr int Q = ASYM ? (1 << BITS) - 1 : (1 << (BITS - 1)) - 1;
@@ -235,6 +244,7 @@ __global__ void __launch_bounds__(kFlushThreads) flush_kernel(const Geo g, const
                                                               const __grid_constant__ PlanView p,
                                                               const uint16_t* kin,
                                                               const uint16_t* vin, int fuse_rows) {
+  launch_dependents();
   if (int(blockIdx.x) >= p.n_flush) {
     const int64_t cta =
         (int64_t(blockIdx.x - p.n_flush) * gridDim.y + blockIdx.y) * gridDim.z + blockIdx.z;
@@ -418,6 +428,7 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
                                                                     const __grid_constant__ PlanView p,
                                                                     const uint16_t* kin, const uint16_t* vin,
                                                                     int fuse_rows) {
+  launch_dependents();
   if (int(blockIdx.x) >= p.n_flush) {
     const int64_t cta = int64_t(blockIdx.x - p.n_flush) * gridDim.y + blockIdx.y;
     const int64_t ctas = int64_t(gridDim.x - p.n_flush) * gridDim.y;
@@ -665,6 +676,7 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
 // ---------------------------------------------------------------------------
 __global__ void residual_kernel(const Geo g, const DevState d, const __grid_constant__ PlanView p,
                                 const uint16_t* kin, const uint16_t* vin) {
+  launch_dependents();
   constexpr int D = kD;
   const int64_t total = int64_t(p.n_res) * g.h_kv * 2 * (D / 8);
   for (int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
@@ -692,6 +704,7 @@ __global__ void residual_kernel(const Geo g, const DevState d, const __grid_cons
 __global__ void __launch_bounds__(256) copy_token_kernel(const Geo g, const DevState d,
                                                          const __grid_constant__ PlanView p,
                                                          const uint16_t* kin, const uint16_t* vin) {
+  launch_dependents();
   constexpr int D = kD;
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int64_t item = int64_t(blockIdx.x) * 8 + wib;
@@ -718,6 +731,7 @@ __global__ void __launch_bounds__(256) copy_token_kernel(const Geo g, const DevS
 __global__ void __launch_bounds__(256) fp8_token_kernel(const Geo g, const DevState d,
                                                         const __grid_constant__ PlanView p,
                                                         const uint16_t* kin, const uint16_t* vin) {
+  launch_dependents();
   constexpr int D = kD;
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int64_t item = int64_t(blockIdx.x) * 8 + wib;

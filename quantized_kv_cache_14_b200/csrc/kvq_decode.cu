@@ -269,7 +269,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
   const uint32_t full0 = smem_addr(smem + L.bars);
   volatile int32_t* abort_flag = reinterpret_cast<int32_t*>(smem + L.flag);
 
-  // the merge grid may be scheduled now; it waits for this grid to complete
+  // Launched as a programmatic dependent of the previous kernel on the stream
+  // (the append of a decode step): wait until that grid has completed and its
+  // writes are visible before reading anything (returns at once when launched
+  // plainly).  Then the merge grid may be scheduled; it waits for this one.
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
 
   // ---- the work list: units per row, prefix over rows ---------------------
@@ -1367,7 +1371,11 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
     return dcheck(t < 0 ? fill[s] == -1 : fill[s] > t, a.err, KVQ_DEVERR_SMEM);
   };
 
-  // the merge grid may be scheduled now; it waits for this grid to complete
+  // Launched as a programmatic dependent of the previous kernel on the stream
+  // (the append of a decode step): wait until that grid has completed and its
+  // writes are visible before reading anything (returns at once when launched
+  // plainly).  Then the merge grid may be scheduled; it waits for this one.
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
 
   // ---- the work list: units per row, prefix over rows ---------------------
@@ -2235,8 +2243,19 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s, cudaEvent_t betwe
   const void* k = a.pipe.ws ? ws_kernel_ptr(a.pipe.ws) : decode_kernel_ptr(a.g);
   void* args[] = {const_cast<DecodeArgs*>(&a)};
   const size_t smem = decode_smem_bytes(a.g, a.pipe, a.B);
-  cudaError_t e =
-      cudaLaunchKernel(k, dim3(a.grid), dim3(a.pipe.ws ? kWsThreads : kDecodeThreads), args, smem, s);
+  // a programmatic dependent launch: the grid is scheduled while the previous
+  // kernel on the stream (an append) runs, and waits for it on the device
+  cudaLaunchConfig_t dcfg = {};
+  dcfg.gridDim = dim3(a.grid);
+  dcfg.blockDim = dim3(a.pipe.ws ? kWsThreads : kDecodeThreads);
+  dcfg.dynamicSmemBytes = smem;
+  dcfg.stream = s;
+  cudaLaunchAttribute dattr[1];
+  dattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  dattr[0].val.programmaticStreamSerializationAllowed = 1;
+  dcfg.attrs = dattr;
+  dcfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelExC(&dcfg, k, args);
   if (e != cudaSuccess) return e;
   ++*launches;
   if (between) {
