@@ -33,6 +33,9 @@ static_assert(sizeof(Geo) + sizeof(DevState) + sizeof(PlanView) + 3 * sizeof(voi
 // Row stride of the bulk flush's code arrays in shared memory (bytes).
 constexpr int kFlushCodeStride = kD + 8;
 
+// The bulk flush gives up on its row copies after 2 s (a device error bit).
+constexpr uint64_t kFlushWaitNs = 2000000000ull;
+
 // A decode launched right after an append is a programmatic dependent launch:
 // letting it be scheduled at the start of every append kernel hides its launch
 // behind the append (it waits for this grid on the device before it reads).
@@ -454,6 +457,7 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
   float* vinv = kinv + D;                                           // [R][nvg]
   float* part = vinv + R * g.nvg;                                   // [3][D] second half's key statistics
   int32_t* ssrc = reinterpret_cast<int32_t*>(part + 3 * D);         // [R]
+  const uint32_t gbar = smem_addr(ssrc + ((R + 1) & ~1));           // 8-byte mbarrier of the row copies
 
   const int e = blockIdx.x, h = blockIdx.y, tid = threadIdx.x, T = blockDim.x;
   const int32_t* ent = plan_of(p) + p.off_flush + e * kFlushEntryInts;
@@ -461,20 +465,28 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
   const int32_t* srcs = plan_of(p) + p.off_src + int64_t(e) * R;
   if (!flush_entry_ok(g, d, ent, srcs)) return;
   for (int r = tid; r < R; r += T) ssrc[r] = srcs[r];
-  __syncthreads();
-
-  // 1. the group's K and V rows (bf16): from the input, or the window
-  for (int idx = tid; idx < 2 * R * (D / 8); idx += T) {
-    const int which = idx / (R * (D / 8));
-    const int rem = idx % (R * (D / 8));
-    const int r = rem / (D / 8), c8 = rem % (D / 8);
-    const int32_t s = ssrc[r];
-    const uint16_t* src;
-    if (s >= 0) src = (which ? vin : kin) + (int64_t(s) * g.h_kv + h) * D;
-    else src = (which ? d.vres : d.kres) + ((int64_t(seq) * g.h_kv + h) * R + (-1 - s)) * D;
-    reinterpret_cast<uint4*>((which ? vt : kt) + r * D)[c8] = reinterpret_cast<const uint4*>(src)[c8];
+  if (tid == 0) {
+    mbar_init(gbar, 1);
+    mbar_init_fence();
+    mbar_arrive_expect_tx(gbar, uint32_t(2 * R * D * 2));
   }
   __syncthreads();
+
+  // 1. the group's K and V rows (bf16, 256 bytes each) from the input, or the
+  //    window for rows appended earlier: one bulk copy per row, all 2R in
+  //    flight at once on one mbarrier (R <= 128, so one row per thread)
+  if (tid < 2 * R) {
+    const int which = tid >= R, r = which ? tid - R : tid;
+    const int32_t s = ssrc[r];
+    const uint16_t* src = s >= 0 ? (which ? vin : kin) + (int64_t(s) * g.h_kv + h) * D
+                                 : (which ? d.vres : d.kres) + ((int64_t(seq) * g.h_kv + h) * R + (-1 - s)) * D;
+    bulk_g2s(smem_addr((which ? vt : kt) + r * D), src, uint32_t(D * 2), gbar);
+  }
+  if (!__syncthreads_and(mbar_wait_bounded(gbar, 0, kFlushWaitNs))) {
+    if (tid == 0) atomicOr(d.err, KVQ_DEVERR_TIMEOUT);
+    (void)mbar_wait_bounded(gbar, 0, kFlushWaitNs);   // keep the CTA until its copies land (bounded)
+    return;
+  }
 
   // 2. key channel statistics: thread (half, c) scans half of the rows
   {
@@ -780,7 +792,7 @@ size_t flush_smem_bytes(const Geo& g) {
 
 size_t flush_group_smem_bytes(const Geo& g) {
   return size_t(2) * g.R * kD * 2 + size_t(2) * g.R * kFlushCodeStride + size_t(3) * kD * 4 +
-         size_t(3) * g.R * g.nvg * 4 + size_t(3) * kD * 4 + size_t(g.R) * 4;
+         size_t(3) * g.R * g.nvg * 4 + size_t(3) * kD * 4 + size_t((g.R + 1) & ~1) * 4 + 8;
 }
 
 // Calls that flush at least this many groups use one CTA per (group, head);
