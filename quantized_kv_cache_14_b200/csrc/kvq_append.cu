@@ -30,9 +30,6 @@ namespace {
 static_assert(sizeof(Geo) + sizeof(DevState) + sizeof(PlanView) + 3 * sizeof(void*) + 16 <= 4096,
               "append kernel parameters exceed 4 KB");
 
-// Row stride of the bulk flush's code arrays in shared memory (bytes).
-constexpr int kFlushCodeStride = kD + 8;
-
 // The bulk flush gives up on its row copies after 2 s (a device error bit).
 constexpr uint64_t kFlushWaitNs = 2000000000ull;
 
@@ -442,14 +439,11 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
   constexpr int N = 32 / BITS;
   constexpr int Q = ASYM ? (1 << BITS) - 1 : (1 << (BITS - 1)) - 1;
   constexpr uint32_t MASK = (1u << BITS) - 1;
-  constexpr int CS = kFlushCodeStride;   // code row stride: 8 bytes of padding spread the banks
   extern __shared__ __align__(16) uint8_t smem[];
   const int R = g.R;
   uint16_t* kt = reinterpret_cast<uint16_t*>(smem);                 // [R][D] bf16
   uint16_t* vt = kt + R * D;                                        // [R][D] bf16
-  uint8_t* kq = reinterpret_cast<uint8_t*>(vt + R * D);             // [R][CS] key codes (low BITS bits)
-  uint8_t* vq = kq + R * CS;                                        // [R][CS] value codes
-  float* ksc = reinterpret_cast<float*>(vq + R * CS);               // [D]
+  float* ksc = reinterpret_cast<float*>(vt + R * D);                // [D]
   float* kzp = ksc + D;                                             // [D]
   float* vsc = kzp + D;                                             // [R][nvg]
   float* vzp = vsc + R * g.nvg;                                     // [R][nvg]
@@ -560,111 +554,110 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
   }
   __syncthreads();
 
-  // 3. every code once, eight consecutive channels of one row per item (one
-  //    128-bit load of the row, the scales as vectors, one 64-bit store)
-  const int lg_gv = __ffs(g.g_v) - 1;
-  for (int it = tid; it < 2 * R * (D / 8); it += T) {
-    const bool val = it >= R * (D / 8);
-    const int rem = val ? it - R * (D / 8) : it;
-    const int r = rem / (D / 8), c0 = 8 * (rem % (D / 8));
-    const uint4 raw = *reinterpret_cast<const uint4*>((val ? vt : kt) + r * D + c0);
-    const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
-    uint32_t lo = 0, hi = 0;
-    uint32_t ties = 0;   // elements whose code the exact division must decide
-    float xs[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) xs[i] = bf16_bits_to_float(uint16_t(wv[i >> 1] >> (16 * (i & 1))));
-    if (val) {
-      const int m = r * g.nvg + (c0 >> lg_gv);   // one value group covers the 8 channels
-      const float sh = vsc[m], inv = vinv[m], zh = vzp[m];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        bool tie;
-        const int q = ASYM ? quant_code_nb(__fsub_rn(xs[i], zh) * inv, 0, Q, tie)
-                           : quant_code_nb(xs[i] * inv, -Q, Q, tie);
-        ties |= uint32_t(tie) << i;
-        const uint32_t b = (uint32_t(q) & MASK) << (8 * (i & 3));
-        if (i < 4) lo |= b; else hi |= b;
-      }
-      if (__any_sync(0xffffffffu, ties != 0)) {
-        for (int i = 0; i < 8; ++i)
-          if (ties & (1u << i)) {
-            const int q = ASYM ? quant_asym_exact(xs[i], sh, zh, Q) : quant_sym_exact(xs[i], sh, Q);
-            uint32_t& wd = i < 4 ? lo : hi;
-            wd = (wd & ~(0xFFu << (8 * (i & 3)))) | ((uint32_t(q) & MASK) << (8 * (i & 3)));
-          }
-      }
-    } else {
-      float sc[8], iv[8], zp[8];
-#pragma unroll
-      for (int v4 = 0; v4 < 2; ++v4) {
-        const float4 a4 = reinterpret_cast<const float4*>(ksc + c0)[v4];
-        const float4 b4 = reinterpret_cast<const float4*>(kinv + c0)[v4];
-        sc[4 * v4] = a4.x; sc[4 * v4 + 1] = a4.y; sc[4 * v4 + 2] = a4.z; sc[4 * v4 + 3] = a4.w;
-        iv[4 * v4] = b4.x; iv[4 * v4 + 1] = b4.y; iv[4 * v4 + 2] = b4.z; iv[4 * v4 + 3] = b4.w;
-        if (ASYM) {
-          const float4 z4 = reinterpret_cast<const float4*>(kzp + c0)[v4];
-          zp[4 * v4] = z4.x; zp[4 * v4 + 1] = z4.y; zp[4 * v4 + 2] = z4.z; zp[4 * v4 + 3] = z4.w;
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        bool tie;
-        const int q = ASYM ? quant_code_nb(__fsub_rn(xs[i], zp[i]) * iv[i], 0, Q, tie)
-                           : quant_code_nb(xs[i] * iv[i], -Q, Q, tie);
-        ties |= uint32_t(tie) << i;
-        const uint32_t b = (uint32_t(q) & MASK) << (8 * (i & 3));
-        if (i < 4) lo |= b; else hi |= b;
-      }
-      if (__any_sync(0xffffffffu, ties != 0)) {
-        for (int i = 0; i < 8; ++i)
-          if (ties & (1u << i)) {
-            const int q = ASYM ? quant_asym_exact(xs[i], sc[i], zp[i], Q) : quant_sym_exact(xs[i], sc[i], Q);
-            uint32_t& wd = i < 4 ? lo : hi;
-            wd = (wd & ~(0xFFu << (8 * (i & 3)))) | ((uint32_t(q) & MASK) << (8 * (i & 3)));
-          }
-      }
-    }
-    *reinterpret_cast<uint2*>((val ? vq : kq) + r * CS + c0) = make_uint2(lo, hi);
-  }
-  __syncthreads();
-
   auto chunk_of = [&](int page) -> uint8_t* {
     return d.pool + int64_t(ent[3 + page]) * g.block_bytes + int64_t(h) * g.chunk_bytes;
   };
   const int subs_per_page = g.P / 16;
 
-  // 4. key words: (row, word in row), element l of word w is list position w N + l
-  const int row_words = D * BITS / 32;
-  for (int W = tid; W < R * row_words; W += T) {
-    const int rowi = W / row_words, w = W % row_words;
-    uint32_t word = 0;
+  // 3. key words, straight from the bf16 rows: word kw of a row holds the
+  //    codes of key-list positions kw N .. kw N + N - 1, i.e. N / 2 pairs of
+  //    adjacent channels.  A thread keeps one word column (the block size is
+  //    a multiple of the words per row), so its channels' reciprocal scales
+  //    and zero-points stay in registers across its rows.
+  {
+    constexpr int RW = D * BITS / 32;                 // words per key row
+    static_assert(kFlushThreads % RW == 0, "one word column per thread");
+    const int kw = tid % RW;
+    int cp[N / 2];
+    float iv[N], zq[N];
 #pragma unroll
-    for (int l = 0; l < N; ++l) word |= uint32_t(kq[rowi * CS + key_channel(w * N + l)]) << (BITS * word_field(l, N));
-    const int sub = rowi >> 4, rr = rowi & 15;
-    *reinterpret_cast<uint32_t*>(chunk_of(sub / subs_per_page) + (sub % subs_per_page) * g.sub_bytes +
-                                 rr * g.row_bytes + 4 * w) = word;
+    for (int l = 0; l < N; ++l) {
+      const int c = key_channel(kw * N + l);
+      if ((l & 1) == 0) cp[l >> 1] = c;
+      iv[l] = kinv[c];
+      zq[l] = ASYM ? kzp[c] : 0.0f;
+    }
+    for (int rowi = tid / RW; rowi < R; rowi += kFlushThreads / RW) {   // warp-uniform trip count
+      float xs[N];
+#pragma unroll
+      for (int m = 0; m < N / 2; ++m) {
+        const uint32_t pr = *reinterpret_cast<const uint32_t*>(kt + rowi * D + cp[m]);
+        xs[2 * m] = __uint_as_float(pr << 16);
+        xs[2 * m + 1] = __uint_as_float(pr & 0xFFFF0000u);
+      }
+      uint32_t word = 0, ties = 0;
+#pragma unroll
+      for (int l = 0; l < N; ++l) {
+        bool tie;
+        const int q = ASYM ? quant_code_nb(__fsub_rn(xs[l], zq[l]) * iv[l], 0, Q, tie)
+                           : quant_code_nb(xs[l] * iv[l], -Q, Q, tie);
+        ties |= uint32_t(tie) << l;
+        word |= (uint32_t(q) & MASK) << (BITS * word_field(l, N));
+      }
+      if (__any_sync(0xffffffffu, ties != 0)) {
+        for (int l = 0; l < N; ++l)
+          if (ties & (1u << l)) {
+            const int c = key_channel(kw * N + l);
+            const int q = ASYM ? quant_asym_exact(xs[l], ksc[c], kzp[c], Q) : quant_sym_exact(xs[l], ksc[c], Q);
+            const int sh = BITS * word_field(l, N);
+            word = (word & ~(MASK << sh)) | ((uint32_t(q) & MASK) << sh);
+          }
+      }
+      const int sub = rowi >> 4, rr = rowi & 15;
+      *reinterpret_cast<uint32_t*>(chunk_of(sub / subs_per_page) + (sub % subs_per_page) * g.sub_bytes +
+                                   rr * g.row_bytes + 4 * kw) = word;
+    }
   }
 
-  // 5. value words: (sub-tile, lane record, word in record) as in flush_kernel
-  const int rec_words = 2 * BITS;
-  for (int W = tid; W < (R / 16) * 32 * rec_words; W += T) {
-    const int sub = W / (32 * rec_words), rem = W % (32 * rec_words);
-    const int lam = rem / rec_words, w = rem % rec_words;
-    const int gq = lam >> 2, tq = lam & 3;
-    uint32_t word = 0;
-    for (int x = 0; x < N / 2; ++x) {
-      int i, reg;
-      if (BITS == 8) { i = w >> 1; reg = 2 * (w & 1) + x; }
-      else if (BITS == 4) { i = w; reg = x; }
-      else { i = 2 * w + ((x >> 1) & 1); reg = 2 * (x >> 2) + (x & 1); }
-      const int c = 16 * i + gq + 8 * (reg & 1);
-      const int t0 = 16 * sub + 2 * tq + 8 * (reg >> 1);
-      word |= uint32_t(vq[t0 * CS + c]) << (BITS * x);
-      word |= uint32_t(vq[(t0 + 1) * CS + c]) << (BITS * (x + N / 2));
+  // 4. value words, straight from the bf16 rows: word w of lane record lam
+  //    (gq = lam / 4, tq = lam % 4) of a sub-tile holds operand register reg
+  //    of channel tile i for tokens (2tq, 2tq + 1) + 8 (reg / 2) and channel
+  //    16 i + gq + 8 (reg % 2), each code with its token's scale for the
+  //    channel's value group
+  {
+    constexpr int RECW = 2 * BITS;                    // words per lane record
+    const int lg_gv = __ffs(g.g_v) - 1;
+    for (int W = tid; W < (R / 16) * 32 * RECW; W += kFlushThreads) {   // warp-uniform trip count
+      const int sub = W / (32 * RECW), rem = W % (32 * RECW);
+      const int lam = rem / RECW, w = rem % RECW;
+      const int gq = lam >> 2, tq = lam & 3;
+      float xs[N];
+      int tk[N / 2], cc[N / 2];
+      uint32_t word = 0, ties = 0;
+#pragma unroll
+      for (int x = 0; x < N / 2; ++x) {
+        int i, reg;
+        if (BITS == 8) { i = w >> 1; reg = 2 * (w & 1) + x; }
+        else if (BITS == 4) { i = w; reg = x; }
+        else { i = 2 * w + ((x >> 1) & 1); reg = 2 * (x >> 2) + (x & 1); }
+        const int c = 16 * i + gq + 8 * (reg & 1);
+        const int t0 = 16 * sub + 2 * tq + 8 * (reg >> 1);
+        tk[x] = t0;
+        cc[x] = c;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int t = t0 + u, l = x + u * (N / 2);
+          xs[l] = bf16_bits_to_float(vt[t * D + c]);
+          const int m = t * g.nvg + (c >> lg_gv);
+          bool tie;
+          const int q = ASYM ? quant_code_nb(__fsub_rn(xs[l], vzp[m]) * vinv[m], 0, Q, tie)
+                             : quant_code_nb(xs[l] * vinv[m], -Q, Q, tie);
+          ties |= uint32_t(tie) << l;
+          word |= (uint32_t(q) & MASK) << (BITS * l);
+        }
+      }
+      if (__any_sync(0xffffffffu, ties != 0)) {
+        for (int l = 0; l < N; ++l)
+          if (ties & (1u << l)) {
+            const int x = l % (N / 2), t = tk[x] + l / (N / 2), c = cc[x];
+            const int m = t * g.nvg + (c >> lg_gv);
+            const int q = ASYM ? quant_asym_exact(xs[l], vsc[m], vzp[m], Q) : quant_sym_exact(xs[l], vsc[m], Q);
+            word = (word & ~(MASK << (BITS * l))) | ((uint32_t(q) & MASK) << (BITS * l));
+          }
+      }
+      *reinterpret_cast<uint32_t*>(chunk_of(sub / subs_per_page) + g.off_V + (sub % subs_per_page) * g.sub_bytes +
+                                   lam * (8 * BITS) + 4 * w) = word;
     }
-    *reinterpret_cast<uint32_t*>(chunk_of(sub / subs_per_page) + g.off_V + (sub % subs_per_page) * g.sub_bytes +
-                                 lam * (8 * BITS) + 4 * w) = word;
   }
 
   // 6. metadata: each page's slice of the key scales (list order), value scales
@@ -791,7 +784,7 @@ size_t flush_smem_bytes(const Geo& g) {
 }
 
 size_t flush_group_smem_bytes(const Geo& g) {
-  return size_t(2) * g.R * kD * 2 + size_t(2) * g.R * kFlushCodeStride + size_t(3) * kD * 4 +
+  return size_t(2) * g.R * kD * 2 + size_t(3) * kD * 4 +
          size_t(3) * g.R * g.nvg * 4 + size_t(3) * kD * 4 + size_t((g.R + 1) & ~1) * 4 + 8;
 }
 
