@@ -449,8 +449,8 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
   float* vzp = vsc + R * g.nvg;                                     // [R][nvg]
   float* kinv = vzp + R * g.nvg;                                    // [D] RN(1 / key scale)
   float* vinv = kinv + D;                                           // [R][nvg]
-  float* part = vinv + R * g.nvg;                                   // [3][D] second half's key statistics
-  int32_t* ssrc = reinterpret_cast<int32_t*>(part + 3 * D);         // [R]
+  float* part = vinv + R * g.nvg;                                   // [3][3][D] key statistics of row quarters 1-3
+  int32_t* ssrc = reinterpret_cast<int32_t*>(part + 9 * D);         // [R]
   const uint32_t gbar = smem_addr(ssrc + ((R + 1) & ~1));           // 8-byte mbarrier of the row copies
 
   const int e = blockIdx.x, h = blockIdx.y, tid = threadIdx.x, T = blockDim.x;
@@ -482,35 +482,58 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
     return;
   }
 
-  // 2. key channel statistics: thread (half, c) scans half of the rows
+  // 2. key channel statistics: thread (quarter, pair) scans channels 2 pair,
+  //    2 pair + 1 (one 32-bit load per row) over a quarter of the rows; the
+  //    first quarter's threads combine and make the pair's scales
   {
-    const int c = tid % D, half = tid / D, nh = T / D;
-    const int r0 = half * R / nh, r1 = (half + 1) * R / nh;
-    float a = 0.0f, mn = INFINITY, mx = -INFINITY;
+    static_assert(kFlushThreads == 2 * D, "64 channel pairs x 4 row quarters");
+    const int cp = tid % (D / 2), qt = tid / (D / 2);
+    const int r0 = qt * (R / 4), r1 = r0 + R / 4;
+    float a[2] = {0.0f, 0.0f}, mn[2] = {INFINITY, INFINITY}, mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll 4
     for (int r = r0; r < r1; ++r) {
-      const float x = bf16_bits_to_float(kt[r * D + c]);
-      a = fmaxf(a, fabsf(x));
-      mn = fminf(mn, x);
-      mx = fmaxf(mx, x);
+      const uint32_t pr = *reinterpret_cast<const uint32_t*>(kt + r * D + 2 * cp);
+      const float x[2] = {__uint_as_float(pr << 16), __uint_as_float(pr & 0xFFFF0000u)};
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        if (ASYM) {
+          mn[e] = fminf(mn[e], x[e]);
+          mx[e] = fmaxf(mx[e], x[e]);
+        } else {
+          a[e] = fmaxf(a[e], fabsf(x[e]));
+        }
+      }
     }
-    if (half == 1) {
-      part[c] = a;
-      part[D + c] = mn;
-      part[2 * D + c] = mx;
+    if (qt > 0) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float* pq = part + (qt - 1) * 3 * D;
+        pq[2 * cp + e] = a[e];
+        pq[D + 2 * cp + e] = mn[e];
+        pq[2 * D + 2 * cp + e] = mx[e];
+      }
     }
     __syncthreads();
-    if (half == 0) {
-      a = fmaxf(a, part[c]);
-      mn = fminf(mn, part[D + c]);
-      mx = fmaxf(mx, part[2 * D + c]);
-      if (ASYM) {
-        kzp[c] = stored_value(mn, g.scale_fp32);
-        ksc[c] = stored_value(__fdiv_rn(__fsub_rn(mx, mn), float(Q)), g.scale_fp32);
-      } else {
-        ksc[c] = stored_value(__fdiv_rn(a, float(Q)), g.scale_fp32);
-        kzp[c] = 0.0f;
+    if (qt == 0) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int c = 2 * cp + e;
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+          const float* pq = part + k * 3 * D;
+          a[e] = fmaxf(a[e], pq[c]);
+          mn[e] = fminf(mn[e], pq[D + c]);
+          mx[e] = fmaxf(mx[e], pq[2 * D + c]);
+        }
+        if (ASYM) {
+          kzp[c] = stored_value(mn[e], g.scale_fp32);
+          ksc[c] = stored_value(__fdiv_rn(__fsub_rn(mx[e], mn[e]), float(Q)), g.scale_fp32);
+        } else {
+          ksc[c] = stored_value(__fdiv_rn(a[e], float(Q)), g.scale_fp32);
+          kzp[c] = 0.0f;
+        }
+        kinv[c] = quant_inv(ksc[c]);
       }
-      kinv[c] = quant_inv(ksc[c]);
     }
   }
   // value (token, group) extremes: warp w takes rows w, w + 8, ...; lane l
@@ -785,7 +808,7 @@ size_t flush_smem_bytes(const Geo& g) {
 
 size_t flush_group_smem_bytes(const Geo& g) {
   return size_t(2) * g.R * kD * 2 + size_t(3) * kD * 4 +
-         size_t(3) * g.R * g.nvg * 4 + size_t(3) * kD * 4 + size_t((g.R + 1) & ~1) * 4 + 8;
+         size_t(3) * g.R * g.nvg * 4 + size_t(9) * kD * 4 + size_t((g.R + 1) & ~1) * 4 + 8;
 }
 
 // Calls that flush at least this many groups use one CTA per (group, head);

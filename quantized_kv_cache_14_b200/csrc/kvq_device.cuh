@@ -384,16 +384,15 @@ __device__ __forceinline__ int quant_asym_fast(float x, float sh, float inv, flo
 }
 
 // Branch-free form of the fast quantizers for bulk work: the code of y =
-// x * inv (or (x - zh) * inv) clipped to [lo, hi], and `tie` set when |y| <
-// 256 lies within 2^-13 of a half-integer -- then (and only then) the caller
-// must take quant_sym / quant_asym instead.  |y| >= 256 needs no test: the
-// code clips either way.  With a zero scale inv is 0, so y = 0 and the code 0
-// (the exact quantizer's zero group) for every finite x; a NaN y gives code 0,
-// as the conversion of the exact quotient does.
+// x * inv (or (x - zh) * inv) clipped to [lo, hi], and `tie` set when y lies
+// within 2^-13 of a half-integer, or is NaN or infinite -- then the caller
+// must take quant_sym / quant_asym instead (exact, and rare).  For |y| < 256
+// the fast code is right whenever `tie` is clear; beyond, the code clips
+// either way.  With a zero scale inv is 0, so y = 0 and the code 0 (the exact
+// quantizer's zero group) for every finite x.
 __device__ __forceinline__ int quant_code_nb(float y, int lo, int hi, bool& tie) {
   const float r = rintf(y);
-  const float d = fabsf(y - r);
-  tie = !(d <= 0.4998779296875f) && fabsf(y) < 256.0f;   // 0.5 - 2^-13
+  tie = !(fabsf(y - r) <= 0.4998779296875f);   // 0.5 - 2^-13; NaN and inf included
   const int q = __float2int_rn(r);
   return q < lo ? lo : (q > hi ? hi : q);
 }
