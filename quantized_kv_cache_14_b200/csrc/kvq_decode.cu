@@ -1324,14 +1324,13 @@ __host__ __device__ constexpr int ws_stage_bytes() {
   return 4 * S::chunk_used > 2 * 16 * kD * 2 ? 4 * S::chunk_used : 2 * 16 * kD * 2;
 }
 
-// S::ws_stages stages per pair; the q' transposition scratch only for INT4
-// (INT2 keeps q in operand order instead).
+// S::ws_stages stages per pair, the weight slots, the barriers.
 template <class S>
 __host__ __device__ inline WsLayout ws_layout(int B) {
   WsLayout L;
   L.stages = ((B + 1 + 32 + 3 * B) * 4 + 127) / 128 * 128;   // prefix, scan scratch, per-row info
   L.qbuf = L.stages + kWsPairs * S::ws_stages * ws_stage_bytes<S>();
-  L.pbuf = L.qbuf + (S::bits == 4 ? kWsPairs * kScratchBytes : 0);
+  L.pbuf = L.qbuf;
   L.alpha = L.pbuf + kWsPairs * kWsPbufFloats * 4;
   L.bars = L.alpha + kWsPairs * 4 * 4;
   L.flag = L.bars + kWsPairs * (S::ws_stages + 2) * 8;
@@ -1448,11 +1447,9 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
     // ============================ score warp ================================
     float m = -INFINITY, l = 0.0f;
     uint32_t bq[8][2];
-    uint32_t qh[4][2];   // INT4: this lane's q' job share, fp16
-    uint32_t qF[8][2];   // INT2: q in score-operand order, fp16, times the code weights
+    uint32_t qF[8][2];   // q in score-operand order, fp16, times the code weights
     float cs = C;
     bool bq_bf16 = false;
-    uint32_t* qbw = reinterpret_cast<uint32_t*>(smem + L.qbuf + pr * kScratchBytes);
     auto qrow = [&](int row, int h, int head) { return a.q + (int64_t(row) * g.h_q + h * S::G + head) * D; };
     auto emit_k = [&](int pair) {
       float lt = l;
@@ -1483,49 +1480,20 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
         }
       }
     };
-    // q of the pair's heads as fp16 with the largest |q| in [2^-5, 2^-4): then
-    // 16 q s stays below 65504 for every fp16 scale s, and an element that
-    // falls to an fp16 subnormal is off by at most 2^-25, 2^-20 of the largest.
-    // This lane's share of the q' job: key-list channels 4 lane .. 4 lane + 3
-    // of every head.
-    auto setup = [&](int row, int h) {
-      const int f = 4 * lane;
-      uint32_t qw[4][2];
-#pragma unroll
-      for (int h2 = 0; h2 < 4; ++h2) {
-        const uint16_t* qr = qrow(row, h, h2);
-        qw[h2][0] = *reinterpret_cast<const uint32_t*>(qr + key_channel(f));
-        qw[h2][1] = *reinterpret_cast<const uint32_t*>(qr + key_channel(f + 2));
-      }
-      float amax = 0.0f;
-#pragma unroll
-      for (int h2 = 0; h2 < 4; ++h2)
-#pragma unroll
-        for (int e = 0; e < 2; ++e)
-          amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(qw[h2][e] << 16)), fabsf(__uint_as_float(qw[h2][e] & 0xFFFF0000u))));
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, o));
-      const int ex = amax > 0.0f ? min(max(int((__float_as_uint(amax) >> 23) & 0xFF) - 127 + 5, -100), 100) : 0;
-      const float down = pow2f(-ex);
-#pragma unroll
-      for (int h2 = 0; h2 < 4; ++h2)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const __half2 v = __floats2half2_rn(__uint_as_float(qw[h2][e] << 16) * down,
-                                              __uint_as_float(qw[h2][e] & 0xFFFF0000u) * down);
-          qh[h2][e] = *reinterpret_cast<const uint32_t*>(&v);
-        }
-      cs = C * pow2f(ex);
-      bq_bf16 = false;
-    };
-    // INT2: the 2-bit codes enter the products as fp16 subnormals, the code at
-    // bits 2y..2y+1 of a half-word worth c 4^y 2^-24 (y = 0..3, one shift by 8
-    // bringing the upper byte down).  Score product j takes its b0 half from
-    // y = 0 (j even) or 2 (j odd) and its b1 half from y + 1, so this lane's
-    // q in operand order carries the factors 2^-18 / weight: 64 and 16 (j
-    // even), 4 and 1 (j odd), and the products come out in units of 2^-18.
-    // The largest |q| lies in [2^-7, 2^-6): then 64 q s stays below 65504.
-    auto setup2 = [&](int row, int h) {
+    // q of the pair's heads in score-operand order (lane (gq, tq) holds, for
+    // product j, channels 16 j + 2 tq + {0, 1} and + {8, 9} of head gq / 2),
+    // fp16, times the code weights of its fields.
+    //  * INT4: a nibble at bits 0-3 is worth c 2^-24, at bits 4-7 c 2^-20, so
+    //    the b0 half carries the factor 16 and the products come out in units
+    //    of 2^-20; the largest |q| lies in [2^-5, 2^-4), so 16 q s < 65504.
+    //  * INT2: the code at bits 2y..2y+1 of a half-word is worth c 4^y 2^-24
+    //    (y = 0..3, one shift by 8 bringing the upper byte down).  Product j
+    //    takes its b0 half from y = 0 (j even) or 2 (j odd) and its b1 half
+    //    from y + 1, so q carries the factors 2^-18 / weight: 64 and 16 (j
+    //    even), 4 and 1 (j odd), and the products come out in units of 2^-18.
+    //    The largest |q| lies in [2^-7, 2^-6): then 64 q s stays below 65504.
+    // An element pushed into the fp16 subnormal range is off by at most 2^-25.
+    auto setup_op = [&](int row, int h) {
       const uint16_t* qr = qrow(row, h, hh);
       uint32_t t[8][2];
 #pragma unroll
@@ -1540,17 +1508,41 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
         for (int e = 0; e < 2; ++e)
           amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(t[j][e] << 16)), fabsf(__uint_as_float(t[j][e] & 0xFFFF0000u))));
       amax = __uint_as_float(__reduce_max_sync(FULL, __float_as_uint(amax)));
-      const int ex = amax > 0.0f ? min(max(int((__float_as_uint(amax) >> 23) & 0xFF) - 127 + 7, -100), 100) : 0;
+      constexpr int kExUp = I2 ? 7 : 5;
+      const int ex = amax > 0.0f ? min(max(int((__float_as_uint(amax) >> 23) & 0xFF) - 127 + kExUp, -100), 100) : 0;
       const float down = pow2f(-ex);
 #pragma unroll
       for (int j = 0; j < 8; ++j)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const float f = down * ((j & 1) ? (e ? 1.0f : 4.0f) : (e ? 16.0f : 64.0f));
+          const float f = down * (I2 ? ((j & 1) ? (e ? 1.0f : 4.0f) : (e ? 16.0f : 64.0f)) : (e ? 1.0f : 16.0f));
           const __half2 v = __floats2half2_rn(__uint_as_float(t[j][e] << 16) * f, __uint_as_float(t[j][e] & 0xFFFF0000u) * f);
           qF[j][e] = *reinterpret_cast<const uint32_t*>(&v);
         }
       cs = C * pow2f(ex);
+      bq_bf16 = false;
+    };
+    // INT4: q' = q s of the unit's key group as the score operand (hi in the
+    // even columns, lo in the odd ones); this lane's 32 key-list positions
+    // 32 tq .. 32 tq + 31 have their scales on page tq (32 per page)
+    auto group_q4 = [&](const uint8_t* stg) {
+      const uint4* ks = reinterpret_cast<const uint4*>(stg + tq * S::chunk_used + S::off_Km);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const uint4 sv = ks[v];
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+          const int j = 2 * v + jj;
+          const uint32_t sw[2] = {jj ? sv.z : sv.x, jj ? sv.w : sv.y};
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const __half2 x = *reinterpret_cast<const __half2*>(&qF[j][e]), sc2 = *reinterpret_cast<const __half2*>(&sw[e]);
+            const __half2 hi = __hmul2(x, sc2);
+            const __half2 lo = __hfma2(x, sc2, __hneg2(hi));
+            bq[j][e] = is_lo ? *reinterpret_cast<const uint32_t*>(&lo) : *reinterpret_cast<const uint32_t*>(&hi);
+          }
+        }
+      }
       bq_bf16 = false;
     };
     // INT2, key group gk of a unit (pages 2 gk, 2 gk + 1): q' = q s as the score
@@ -1615,56 +1607,6 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
       s0 = gq < valid ? fmaf(acc0[0] + acc0[1] + acc1[0] + acc1[1], cs18, csb) : -INFINITY;
       s1 = gq + 8 < valid ? fmaf(acc0[2] + acc0[3] + acc1[2] + acc1[3], cs18, csb) : -INFINITY;
     };
-    // q' = q s_channel of the unit's key group as the score B operand (the
-    // b0-half channels 16 times larger for the subnormal codes): each lane
-    // scales 4 channels of every head, then the warp scratch transposes them
-    // into operand order (XOR-swizzled 16-byte slots, conflict-free reads)
-    auto qprime = [&](const uint8_t* stg) {
-      const int f = 4 * lane;
-      const uint8_t* km = stg + (f >> S::lg_kslice) * S::chunk_used + S::off_Km;
-      const int off = f & (S::kslice - 1);
-      const int t0 = lane >> 3, j = lane & 7;
-      const uint2 sr = *reinterpret_cast<const uint2*>(km + off * 2);
-      const __half2 s01 = *reinterpret_cast<const __half2*>(&sr.x), s23 = *reinterpret_cast<const __half2*>(&sr.y);
-      uint32_t qv[4][4];
-#pragma unroll
-      for (int h2 = 0; h2 < 4; ++h2) {
-        const __half2 qa = __hmul2(*reinterpret_cast<const __half2*>(&qh[h2][0]), __float2half2_rn(16.0f));
-        const __half2 qb = *reinterpret_cast<const __half2*>(&qh[h2][1]);
-        const __half2 ha = __hmul2(qa, s01), hb = __hmul2(qb, s23);
-        const __half2 la = __hfma2(qa, s01, __hneg2(ha)), lb = __hfma2(qb, s23, __hneg2(hb));
-        qv[h2][0] = *reinterpret_cast<const uint32_t*>(&ha);
-        qv[h2][1] = *reinterpret_cast<const uint32_t*>(&hb);
-        qv[h2][2] = *reinterpret_cast<const uint32_t*>(&la);
-        qv[h2][3] = *reinterpret_cast<const uint32_t*>(&lb);
-      }
-#pragma unroll
-      for (int pass = 0; pass < 2; ++pass) {
-        __syncwarp();
-        if ((j >> 2) == pass) {
-          const int j4 = j & 3;
-#pragma unroll
-          for (int h2 = 0; h2 < 4; ++h2) {
-            const int thi = 8 * h2 + t0, tlo = thi + 4;
-            *reinterpret_cast<uint2*>(qbw + thi * 8 + 4 * ((j4 >> 1) ^ ((thi >> 2) & 1)) + 2 * (j4 & 1)) =
-                make_uint2(qv[h2][0], qv[h2][1]);
-            *reinterpret_cast<uint2*>(qbw + tlo * 8 + 4 * ((j4 >> 1) ^ ((tlo >> 2) & 1)) + 2 * (j4 & 1)) =
-                make_uint2(qv[h2][2], qv[h2][3]);
-          }
-        }
-        __syncwarp();
-        const uint4* qb = reinterpret_cast<const uint4*>(qbw + lane * 8);
-        const int sw = (lane >> 2) & 1;
-#pragma unroll
-        for (int v = 0; v < 2; ++v) {
-          const uint4 x = qb[v ^ sw];
-          bq[4 * pass + 2 * v][0] = x.x; bq[4 * pass + 2 * v][1] = x.y;
-          bq[4 * pass + 2 * v + 1][0] = x.z; bq[4 * pass + 2 * v + 1][1] = x.w;
-        }
-      }
-      __syncwarp();
-      bq_bf16 = false;
-    };
     auto score_sub = [&](const uint8_t* ksub, float cs20, float bias, int valid, float& s0, float& s1) {
       uint32_t wa[4], wb[4];
       load_key_words<4>(ksub, gq, tq, wa, wb);
@@ -1684,8 +1626,7 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
     for (int k = 0; k < K; ++k) {
       walk_to(pr + kWsPairs * k);
       if (needs_setup) {
-        if constexpr (I2) setup2(itc.i, itc.h);
-        else setup(itc.i, itc.h);
+        setup_op(itc.i, itc.h);
         needs_setup = false;
       }
       const int s = k % kWsStages;
@@ -1716,7 +1657,7 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
             }
           }
         } else {
-          qprime(stg);
+          group_q4(stg);
           float accb[4] = {0.0f, 0.0f, 0.0f, 0.0f};   // the key offset: q' against all-zero codes
 #pragma unroll
           for (int j = 0; j < 8; ++j) mma_f16(accb, ZA0, ZA0, ZA1, ZA1, bq[j][0], bq[j][1]);
