@@ -200,7 +200,8 @@ struct SpecInt4Kivi {
   static constexpr int n = 8, row_bytes = 64, sub_bytes = 1024, es = 2, nvg = 2, kslice = 32;
   static constexpr int off_V = 1024, off_Vm = 2048, off_Km = 2112, chunk_used = 2176;
   static constexpr int lg_P = 4, lg_gk = 6, lg_kslice = 5;
-  static constexpr int ws_stages = 3;   // warp-specialised kernel: stages per warp pair
+  static constexpr int ws_stages = 3;     // warp-specialised kernel: stages per warp pair
+  static constexpr int unit_tokens = 64;  // its unit: one key group
 };
 
 // The INT2 asymmetric KIVI format (keys per channel G = 32, values per token
@@ -212,6 +213,20 @@ struct SpecInt2Kivi {
   static constexpr int off_V = 512, off_Vm = 1024, off_Km = 1280, chunk_used = 1536;
   static constexpr int lg_P = 4, lg_gk = 5, lg_kslice = 6;
   static constexpr int ws_stages = 3;
+  static constexpr int unit_tokens = 64;  // two key groups
+};
+
+// The INT8 format with keys and values per token (G = 128 = d_h: one fp16
+// scale per token and head for each), no window, page 16, 4 query heads per
+// kv head: the warp-specialised kernel takes units of 32 tokens (two pages of
+// 4160 bytes) so that three stages per warp pair still fit two CTAs per SM.
+struct SpecInt8Tok {
+  static constexpr int bits = 8, asym = 0, k_axis = 0, g_k = 128, g_v = 128, scale_fp32 = 0, R = 0, P = 16, G = 4;
+  static constexpr int n = 4, row_bytes = 128, sub_bytes = 2048, es = 2, nvg = 1, kslice = 0;
+  static constexpr int off_V = 2048, off_Vm = 4096, off_Km = 4128, chunk_used = 4160;
+  static constexpr int lg_P = 4, lg_gk = 7, lg_kslice = 0;
+  static constexpr int ws_stages = 3;
+  static constexpr int unit_tokens = 32;
 };
 
 template <int SPEC>
@@ -240,6 +255,7 @@ bool spec_matches(const Geo& g) {
 
 bool spec_int4_kivi(const Geo& g) { return spec_matches<SpecInt4Kivi>(g); }
 bool spec_int2_kivi(const Geo& g) { return spec_matches<SpecInt2Kivi>(g); }
+bool spec_int8_tok(const Geo& g) { return spec_matches<SpecInt8Tok>(g); }
 
 template <int BITS, int ASYM, int KAXIS, int ES, int SPEC>
 __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_constant__ DecodeArgs a) {
@@ -1321,7 +1337,8 @@ struct WsLayout {
 // A stage holds a unit's 4 pages or a 16-token window tile (K and V rows).
 template <class S>
 __host__ __device__ constexpr int ws_stage_bytes() {
-  return 4 * S::chunk_used > 2 * 16 * kD * 2 ? 4 * S::chunk_used : 2 * 16 * kD * 2;
+  return (S::unit_tokens / 16) * S::chunk_used > 2 * 16 * kD * 2 ? (S::unit_tokens / 16) * S::chunk_used
+                                                                  : 2 * 16 * kD * 2;
 }
 
 // S::ws_stages stages per pair, the weight slots, the barriers.
@@ -1343,6 +1360,8 @@ template <class S>
 __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_constant__ DecodeArgs a) {
   constexpr int D = kD;
   constexpr bool I2 = S::bits == 2;
+  constexpr bool I8 = S::bits == 8;
+  constexpr int UT = S::unit_tokens;                      // tokens per quantized unit
   constexpr int kWsStages = S::ws_stages;                 // stages per pair
   constexpr int kWsStageBytes = ws_stage_bytes<S>();      // one 64-token unit or window tile
   constexpr uint32_t FULL = 0xffffffffu;
@@ -1406,7 +1425,7 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
     r.seq = s_row[3 * i];
     r.qa = s_row[3 * i + 1];
     r.ra = s_row[3 * i + 2];
-    r.nq = (r.qa + 63) >> 6;
+    r.nq = (r.qa + UT - 1) / UT;
     r.nr = (r.ra + 15) >> 4;
     r.trow = a.table + int64_t(a.table_by_seq ? r.seq : i) * a.table_stride;
     return r;
@@ -1430,6 +1449,7 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
   const bool is_lo = gq & 1;            // the column carries the lo part
   const float C = a.qk_scale;
   constexpr uint32_t ZA0 = 0x00080008u, ZA1 = 0x00800080u;   // all-zero codes, bits 0-3 / 4-7
+  constexpr uint32_t ZB8 = 0x00800080u;                       // INT8: the zero code, sign bit flipped
 
   It itc;
   it_seek(itc, s_pre, a.B, g.h_kv, c0);
@@ -1448,6 +1468,7 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
     float m = -INFINITY, l = 0.0f;
     uint32_t bq[8][2];
     uint32_t qF[8][2];   // q in score-operand order, fp16, times the code weights
+    float bias8 = 0.0f;  // INT8: q against all-128 codes, head tq
     float cs = C;
     bool bq_bf16 = false;
     auto qrow = [&](int row, int h, int head) { return a.q + (int64_t(row) * g.h_q + h * S::G + head) * D; };
@@ -1492,6 +1513,11 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
     //    from y + 1, so q carries the factors 2^-18 / weight: 64 and 16 (j
     //    even), 4 and 1 (j odd), and the products come out in units of 2^-18.
     //    The largest |q| lies in [2^-7, 2^-6): then 64 q s stays below 65504.
+    //  * INT8 (keys per token): a byte at bits 0-7 of a half-word is worth
+    //    c 2^-24 in either byte of the word (one shift by 8), so no factor;
+    //    the key scale multiplies the score per token, so q itself is the
+    //    operand for every unit of the pair (lo columns zero: q is exact in
+    //    fp16 once scaled so that its largest |q| lies in [1/2, 1)).
     // An element pushed into the fp16 subnormal range is off by at most 2^-25.
     auto setup_op = [&](int row, int h) {
       const uint16_t* qr = qrow(row, h, hh);
@@ -1508,19 +1534,31 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
         for (int e = 0; e < 2; ++e)
           amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(t[j][e] << 16)), fabsf(__uint_as_float(t[j][e] & 0xFFFF0000u))));
       amax = __uint_as_float(__reduce_max_sync(FULL, __float_as_uint(amax)));
-      constexpr int kExUp = I2 ? 7 : 5;
+      constexpr int kExUp = I2 ? 7 : I8 ? 1 : 5;
       const int ex = amax > 0.0f ? min(max(int((__float_as_uint(amax) >> 23) & 0xFF) - 127 + kExUp, -100), 100) : 0;
       const float down = pow2f(-ex);
 #pragma unroll
       for (int j = 0; j < 8; ++j)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const float f = down * (I2 ? ((j & 1) ? (e ? 1.0f : 4.0f) : (e ? 16.0f : 64.0f)) : (e ? 1.0f : 16.0f));
+          const float f = down * (I2 ? ((j & 1) ? (e ? 1.0f : 4.0f) : (e ? 16.0f : 64.0f)) : I8 ? 1.0f : (e ? 1.0f : 16.0f));
           const __half2 v = __floats2half2_rn(__uint_as_float(t[j][e] << 16) * f, __uint_as_float(t[j][e] & 0xFFFF0000u) * f);
           qF[j][e] = *reinterpret_cast<const uint32_t*>(&v);
         }
       cs = C * pow2f(ex);
       bq_bf16 = false;
+      if constexpr (I8) {
+        // the operand of every unit of the pair, and the offset term: the
+        // codes carry 128 (sign bit flipped), q against all-128 codes
+        float accb[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          bq[j][0] = is_lo ? 0u : qF[j][0];
+          bq[j][1] = is_lo ? 0u : qF[j][1];
+          mma_f16(accb, ZB8, ZB8, ZB8, ZB8, bq[j][0], bq[j][1]);
+        }
+        bias8 = accb[0];
+      }
     };
     // INT4: q' = q s of the unit's key group as the score operand (hi in the
     // even columns, lo in the odd ones); this lane's 32 key-list positions
@@ -1607,6 +1645,28 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
       s0 = gq < valid ? fmaf(acc0[0] + acc0[1] + acc1[0] + acc1[1], cs18, csb) : -INFINITY;
       s1 = gq + 8 < valid ? fmaf(acc0[2] + acc0[3] + acc1[2] + acc1[3], cs18, csb) : -INFINITY;
     };
+    // INT8 scores of one 16-token page: rows gq, gq + 8 hold 128 bytes of
+    // codes each, this lane's 32 at byte 32 tq; word j feeds product j (bytes
+    // 0, 2 its b0 half, bytes 1, 3 its b1 half); then the token's key scale
+    auto score_sub8 = [&](const uint8_t* page, float cs24, int valid, float& s0, float& s1) {
+      const uint4* ra = reinterpret_cast<const uint4*>(page + gq * S::row_bytes + 32 * tq);
+      const uint4* rb = reinterpret_cast<const uint4*>(page + (gq + 8) * S::row_bytes + 32 * tq);
+      const uint4 x0 = ra[0], x1 = ra[1], y0 = rb[0], y1 = rb[1];
+      const uint32_t wa[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+      const uint32_t wb[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+      float acc0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, acc1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t a0 = and_xor(wa[j], 0x00FF00FFu, ZB8), a1 = and_xor(wb[j], 0x00FF00FFu, ZB8);
+        const uint32_t a2 = and_xor(wa[j] >> 8, 0x00FF00FFu, ZB8), a3 = and_xor(wb[j] >> 8, 0x00FF00FFu, ZB8);
+        if (j & 1) mma_f16(acc1, a0, a1, a2, a3, bq[j][0], bq[j][1]);
+        else mma_f16(acc0, a0, a1, a2, a3, bq[j][0], bq[j][1]);
+      }
+      const uint16_t* ks = reinterpret_cast<const uint16_t*>(page + S::off_Km);
+      const float sa = __half2float(__ushort_as_half(ks[gq])), sb = __half2float(__ushort_as_half(ks[gq + 8]));
+      s0 = gq < valid ? (acc0[0] + acc1[0] - bias8) * (cs24 * sa) : -INFINITY;
+      s1 = gq + 8 < valid ? (acc0[2] + acc1[2] - bias8) * (cs24 * sb) : -INFINITY;
+    };
     auto score_sub = [&](const uint8_t* ksub, float cs20, float bias, int valid, float& s0, float& s1) {
       uint32_t wa[4], wb[4];
       load_key_words<4>(ksub, gq, tq, wa, wb);
@@ -1640,9 +1700,18 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
       const uint8_t* stg = stage_of(s);
       float sc[8];
       if (itc.k < ric.nq) {
-        const int valid = min(64, ric.qa - itc.k * 64);
-        (void)page_filled(s, I2 && valid <= 32 ? 1 : 3);
-        if constexpr (I2) {
+        const int valid = min(UT, ric.qa - itc.k * UT);
+        (void)page_filled(s, I8 ? (valid <= 16 ? 0 : 1) : I2 && valid <= 32 ? 1 : 3);
+        if constexpr (I8) {
+          // one or two pages (keys per token: the last unit of a row may end
+          // inside its first page); the unit's other scores are -inf
+          const float cs24 = cs * 16777216.0f;
+          score_sub8(page_of(stg, 0), cs24, valid, sc[0], sc[1]);
+          if (valid > 16) score_sub8(page_of(stg, 1), cs24, valid - 16, sc[2], sc[3]);
+          else sc[2] = sc[3] = -INFINITY;
+#pragma unroll
+          for (int t = 4; t < 8; ++t) sc[t] = -INFINITY;
+        } else if constexpr (I2) {
           // one or two key groups of 32 tokens (the quantized length is a
           // multiple of 32); a missing second group scores -inf
           const float cs18 = cs * 262144.0f;
@@ -1759,6 +1828,14 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
           st.o[i][3] = fmaf(st.o[i][3], fb, zv[i >> 1][3]);
         }
         zv_reset();
+      } else if constexpr (I8) {
+        // every code at 2^-24, with the offset 128 of the flipped sign bit
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) st.o[i][c] = (st.o[i][c] - st.zc[0][c]) * 16777216.0f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) st.zc[0][c] = 0.0f;
       } else {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -1807,11 +1884,12 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
     // tokens all lie in its first key group (a key group's scales span both
     // of its pages, so pages follow whole groups)
     auto unit_pages = [&](const It& it, const RowInfo& ri) {
+      if constexpr (I8) return ri.qa - UT * it.k <= 16 ? 1 : 2;   // token axis: pages as far as tokens go
       return I2 && ri.qa - 64 * it.k <= 32 ? 2 : 4;
     };
     auto load_blk = [&](const It& it, const RowInfo& ri) -> int32_t {
       if (it.k >= ri.nq || lane >= unit_pages(it, ri)) return 0;   // a window tile, or no page for this lane
-      const int pg = ((it.k * 64) >> 4) + lane;
+      const int pg = ((it.k * UT) >> 4) + lane;
       return pg < a.table_stride ? ri.trow[pg] : -1;
     };
     auto issue = [&](const It& it, const RowInfo& ri, int32_t blk, int s) {
@@ -1941,6 +2019,44 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
       }
     };
 
+    // INT8 value product of one 16-token page: this lane's 64-byte record
+    // (words 2i, 2i + 1 the operand registers of channel tile i, bytes 0, 2
+    // and 1, 3 of each), the weights p' = p s of the token's scale as fp16
+    // hi + lo, and the offset 128 of every code against all-128 codes
+    auto pv_sub8 = [&](const uint8_t* page, float pa0, float pb0, float pa1, float pb1) {
+      const uint4* vr = reinterpret_cast<const uint4*>(page + S::off_V + 64 * lane);
+      uint32_t w[16];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const uint4 x = vr[v];
+        w[4 * v] = x.x; w[4 * v + 1] = x.y; w[4 * v + 2] = x.z; w[4 * v + 3] = x.w;
+      }
+      uint32_t pha, pla, phb, plb;
+      split2h(pa0, pb0, pha, pla);
+      split2h(pa1, pb1, phb, plb);
+      const uint16_t* vs = reinterpret_cast<const uint16_t*>(page + S::off_Vm);   // one scale per token
+      const uint32_t sa = *reinterpret_cast<const uint32_t*>(vs + 2 * tq), sb = *reinterpret_cast<const uint32_t*>(vs + 2 * tq + 8);
+      auto two = [](uint32_t ph, uint32_t pl, uint32_t svb, uint32_t& hi, uint32_t& lo) {
+        const __half2 x = *reinterpret_cast<const __half2*>(&ph), y = *reinterpret_cast<const __half2*>(&pl);
+        const __half2 sv = *reinterpret_cast<const __half2*>(&svb);
+        const __half2 h = __hmul2(x, sv);
+        const __half2 lw = __hfma2(y, sv, __hfma2(x, sv, __hneg2(h)));
+        hi = *reinterpret_cast<const uint32_t*>(&h);
+        lo = *reinterpret_cast<const uint32_t*>(&lw);
+      };
+      uint32_t h0, l0, h1, l1;
+      two(pha, pla, sa, h0, l0);
+      two(phb, plb, sb, h1, l1);
+      const uint32_t b0 = is_lo ? l0 : h0, b1 = is_lo ? l1 : h1;
+      mma_f16(st.zc[0], ZB8, ZB8, ZB8, ZB8, b0, b1);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t w0 = w[2 * i], w1 = w[2 * i + 1];
+        mma_f16(st.o[i], and_xor(w0, 0x00FF00FFu, ZB8), and_xor(w0 >> 8, 0x00FF00FFu, ZB8),
+                and_xor(w1, 0x00FF00FFu, ZB8), and_xor(w1 >> 8, 0x00FF00FFu, ZB8), b0, b1);
+      }
+    };
+
     // copies: the pair's first three units, then one unit three ahead per unit
     It iti = itc;
     RowInfo rii = ric;
@@ -1993,7 +2109,17 @@ __global__ void __launch_bounds__(kWsThreads, 2) decode_ws_kernel(const __grid_c
       const uint8_t* stg = stage_of(s);
       if (itc.k < ric.nq) {
         (void)page_filled(s, unit_pages(itc, ric) - 1);
-        if constexpr (I2) {
+        if constexpr (I8) {
+          const int nt = unit_pages(itc, ric);   // 1 or 2 pages
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (t < nt) {
+              const float2 x = *reinterpret_cast<const float2*>(pb + t * 64 + hh * 16 + 2 * tq);
+              const float2 y = *reinterpret_cast<const float2*>(pb + t * 64 + hh * 16 + 2 * tq + 8);
+              pv_sub8(page_of(stg, t), x.x, x.y, y.x, y.y);
+            }
+          }
+        } else if constexpr (I2) {
           const int nt = unit_pages(itc, ric);   // 2 or 4 pages
 #pragma unroll
           for (int t = 0; t < 4; ++t) {
@@ -2077,14 +2203,18 @@ const void* decode_kernel_ptr(const Geo& g) {
   }
 }
 
-// The warp-specialised kernel of a plan (pipe.ws: 1 INT4 KIVI, 2 INT2 KIVI).
+// The warp-specialised kernel of a plan (pipe.ws: 1 INT4 KIVI, 2 INT2 KIVI,
+// 3 INT8 with keys per token).
 static const void* ws_kernel_ptr(int ws) {
-  return ws == 2 ? reinterpret_cast<const void*>(&decode_ws_kernel<SpecInt2Kivi>)
-                 : reinterpret_cast<const void*>(&decode_ws_kernel<SpecInt4Kivi>);
+  return ws == 3   ? reinterpret_cast<const void*>(&decode_ws_kernel<SpecInt8Tok>)
+         : ws == 2 ? reinterpret_cast<const void*>(&decode_ws_kernel<SpecInt2Kivi>)
+                   : reinterpret_cast<const void*>(&decode_ws_kernel<SpecInt4Kivi>);
 }
 
 static size_t ws_smem_bytes(int ws, int B) {
-  return size_t(ws == 2 ? ws_layout<SpecInt2Kivi>(B).total : ws_layout<SpecInt4Kivi>(B).total);
+  return size_t(ws == 3   ? ws_layout<SpecInt8Tok>(B).total
+                : ws == 2 ? ws_layout<SpecInt2Kivi>(B).total
+                          : ws_layout<SpecInt4Kivi>(B).total);
 }
 
 size_t decode_smem_bytes(const Geo& g, const DecodePipe& p, int B) {
@@ -2159,7 +2289,7 @@ cudaError_t plan_decode(const Geo& g, int max_B, DecodePipe* out) {
   if (e != cudaSuccess) return e;
   if (p.ctas_per_sm < 1) return cudaErrorInvalidConfiguration;
   p.ws = 0;
-  const int ws = spec_int4_kivi(g) ? 1 : spec_int2_kivi(g) ? 2 : 0;
+  const int ws = spec_int4_kivi(g) ? 1 : spec_int2_kivi(g) ? 2 : spec_int8_tok(g) ? 3 : 0;
   if (ws) {
     // the warp-specialised kernel when two of its CTAs fit per SM
     const size_t wsm = ws_smem_bytes(ws, max_B);
@@ -2173,6 +2303,10 @@ cudaError_t plan_decode(const Geo& g, int max_B, DecodePipe* out) {
       if (occ >= 2) {
         p.ws = ws;
         p.ctas_per_sm = occ;
+        if (ws == 3) {   // its units are 32 tokens: the per-row unit counts follow
+          p.sup = 32;
+          p.lg_sup = 5;
+        }
       }
     }
   }

@@ -70,7 +70,7 @@ struct DecodePipe {
   int stage_bytes;  // one stage: a quantized unit or a 16-token BF16 window tile
   int nstages;
   int ctas_per_sm;  // resident CTAs per SM at the largest batch
-  int ws;           // the warp-specialised kernel: 1 for the INT4 KIVI format, 2 for INT2 KIVI
+  int ws;           // the warp-specialised kernel: 1 INT4 KIVI, 2 INT2 KIVI, 3 INT8 keys per token
 };
 
 struct DecodeArgs {
