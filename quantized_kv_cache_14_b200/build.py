@@ -20,7 +20,8 @@ LIB_DEBUG = os.path.join(PKG, "libkvq_debug.so")
 BUILD_DEBUG = os.path.join(PKG, "_build_debug")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
-SOURCES = ["kvq_runtime.cpp", "kvq_append.cu", "kvq_decode.cu", "kvq_prefill.cu", "kvq_noalloc.cu", "kvq_floor.cu"]
+SOURCES = ["kvq_runtime.cpp", "kvq_append.cu", "kvq_decode.cu", "kvq_prefill.cu", "kvq_prefill_tc.cu", "kvq_noalloc.cu",
+           "kvq_floor.cu"]
 HEADERS = ["kvq_internal.h", "kvq_device.cuh", "kvq_tiles.cuh"]
 
 FLAGS = ["-std=c++17", "-O3", "-lineinfo", "-gencode", "arch=compute_100a,code=sm_100a",

@@ -127,6 +127,15 @@ size_t prefill_smem_bytes(int stage_bytes);
 // Resident prefill CTAs per SM for the format (occupancy API; at least 1).
 int prefill_ctas_per_sm(const Geo& g, int stage_bytes);
 cudaError_t launch_prefill(const PrefillArgs& a, int64_t n_rows, cudaStream_t s, int* launches);
+// The split records' log-sum-exp merge of a prefill plan with splits > 1.
+cudaError_t launch_prefill_merge(const PrefillArgs& a, int64_t n_rows, cudaStream_t s, int* launches);
+// The tensor-core (tcgen05) prefill of the INT4 KIVI format with 4 query heads
+// per kv head (kvq_prefill_tc.cu): blocks of 32 query tokens, one CTA per task.
+bool prefill_tc_supported(const Geo& g);
+size_t prefill_tc_smem_bytes();
+int prefill_tc_stage_bytes();
+int prefill_tc_ctas_per_sm();
+cudaError_t launch_prefill_tc(const PrefillArgs& a, int64_t n_rows, cudaStream_t s, int* launches);
 
 // Host-side launchers (defined in the .cu files).
 // Each launcher adds the number of kernels it launched to *launches.

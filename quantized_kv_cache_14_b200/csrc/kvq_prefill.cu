@@ -578,12 +578,16 @@ cudaError_t launch_prefill_t(const PrefillArgs& a, int64_t n_rows, cudaStream_t 
   ++*launches;
   e = cudaGetLastError();
   if (e != cudaSuccess || a.splits == 1) return e;
+  return launch_prefill_merge(a, n_rows, s, launches);
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_merge(const PrefillArgs& a, int64_t n_rows, cudaStream_t s, int* launches) {
   prefill_merge_kernel<<<unsigned(n_rows * a.g.h_q), kD, 0, s>>>(a.part, a.out, a.splits);
   ++*launches;
   return cudaGetLastError();
 }
-
-}  // namespace
 
 bool prefill_supported(const Geo& g) {
   return g.k_axis == 1 && g.R == g.g_k && !g.fp8 && g.bits != 16 && !g.scale_fp32;

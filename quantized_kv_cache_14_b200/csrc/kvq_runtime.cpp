@@ -745,12 +745,15 @@ kvq_status ensure_buffer(kvq_handle h, void** buf, size_t& cap, size_t need, siz
 }
 
 // Chunked prefill with shared tiles: rows sorted by (sequence, position) form
-// blocks of at most 64 / g query tokens of one sequence; each block is split
-// over the key range into `splits` tasks per kv head, one CTA each.
+// blocks of at most 64 / g query tokens of one sequence (32 for the
+// tensor-core kernel of the INT4 KIVI format: 128 rows of 4 heads); each
+// block is split over the key range into `splits` tasks per kv head, one CTA
+// each.
 kvq_status prefill_blocks(kvq_handle h, const uint16_t* q, const int32_t* seq_ids, const int32_t* pos,
                           int32_t n, float* out, cudaStream_t stream) {
   const kvq::Geo& g = h->geo;
-  const int G = g.G, QB = 4 * (16 / G);
+  const bool tc = kvq::prefill_tc_supported(g) && h->pipe.sup == 64;
+  const int G = g.G, QB = tc ? 32 : 4 * (16 / G);
   std::vector<int32_t> order(static_cast<size_t>(n));
   for (int32_t i = 0; i < n; ++i) order[size_t(i)] = i;
   std::stable_sort(order.begin(), order.end(), [&](int32_t x, int32_t y) {
@@ -780,8 +783,8 @@ kvq_status prefill_blocks(kvq_handle h, const uint16_t* q, const int32_t* seq_id
   // fixed cost), the longest task + that cost); a task's setup, pipeline fill
   // and records cost about as much as 8 units.  No task may outgrow its
   // block-id cache.
-  const int stage_bytes = kvq::prefill_stage_bytes(g, sup);
-  if (h->pf_ctas_per_sm == 0) h->pf_ctas_per_sm = kvq::prefill_ctas_per_sm(g, stage_bytes);
+  const int stage_bytes = tc ? kvq::prefill_tc_stage_bytes() : kvq::prefill_stage_bytes(g, sup);
+  if (h->pf_ctas_per_sm == 0) h->pf_ctas_per_sm = tc ? kvq::prefill_tc_ctas_per_sm() : kvq::prefill_ctas_per_sm(g, stage_bytes);
   const int slots = h->pf_ctas_per_sm * h->sm_count;
   double units = 0.0;
   for (int x : nq) units += double(x) * g.h_kv;
@@ -846,7 +849,8 @@ kvq_status prefill_blocks(kvq_handle h, const uint16_t* q, const int32_t* seq_id
   a.lg_sup = h->pipe.lg_sup;
   a.stage_bytes = stage_bytes;
   a.g = g;
-  KVQ_CUDA(kvq::launch_prefill(a, n, stream, &h->launches));
+  if (tc) KVQ_CUDA(kvq::launch_prefill_tc(a, n, stream, &h->launches));
+  else KVQ_CUDA(kvq::launch_prefill(a, n, stream, &h->launches));
   return KVQ_OK;
 }
 
