@@ -465,12 +465,20 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const __grid_
         for (int j = 32; j < 64; ++j) sv[j] = 0.0f;
       }
     }
+    // raw scores; the row scale cs > 0 goes into the exponent's FMA below.
+    // A unit wholly before every position of the warp's rows needs no mask.
     float mx = -INFINITY;
+    if (__all_sync(0xffffffffu, nt == 64 && T0 + 63 <= pos)) {
 #pragma unroll
-    for (int j = 0; j < 64; ++j) {
-      sv[j] = (j < nt && T0 + j <= pos) ? sv[j] * cs : -INFINITY;
-      mx = fmaxf(mx, sv[j]);
+      for (int j = 0; j < 64; ++j) mx = fmaxf(mx, sv[j]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 64; ++j) {
+        sv[j] = (j < nt && T0 + j <= pos) ? sv[j] : -INFINITY;
+        mx = fmaxf(mx, sv[j]);
+      }
     }
+    mx = mx == -INFINITY ? mx : mx * cs;
     const bool raise = mx > m_run + 8.0f || (m_run == -INFINITY && mx != -INFINITY);
     float alpha = 1.0f;
     if (raise) {
@@ -490,16 +498,21 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const __grid_
       }
     }
     {
+      // p = 2^(s cs - m): a masked score is -inf and gives 0 (as does a row
+      // with nothing attended, m = -inf, whose scores are all -inf); l sums
+      // the fp32 p (its fp16 rounding moves the sum by 2^-12 at most)
       uint32_t pw[32];
+      const float nm = m_run == -INFINITY ? 0.0f : -m_run;
+      float lsum = 0.0f;
 #pragma unroll
       for (int j = 0; j < 64; j += 2) {
-        const float p0 = sv[j] == -INFINITY ? 0.0f : fast_exp2(sv[j] - m_run);
-        const float p1 = sv[j + 1] == -INFINITY ? 0.0f : fast_exp2(sv[j + 1] - m_run);
+        const float p0 = fast_exp2(fmaf(sv[j], cs, nm));
+        const float p1 = fast_exp2(fmaf(sv[j + 1], cs, nm));
         const __half2 ph = __floats2half2_rn(p0, p1);
-        const float2 pf = __half22float2(ph);
-        l_run += pf.x + pf.y;
+        lsum += p0 + p1;
         pw[j >> 1] = *reinterpret_cast<const uint32_t*>(&ph);
       }
+      l_run += lsum;
 #pragma unroll
       for (int c = 0; c < 8; ++c)
         *reinterpret_cast<uint4*>(smem + L.p + sw128_off(tid, c)) =
@@ -586,11 +599,22 @@ size_t prefill_tc_smem_bytes() { return size_t(tc_smem().total) + 1024; }
 
 int prefill_tc_stage_bytes() { return kTcStageBytes; }
 
+// Resident CTAs per SM from the kernel's own resources: shared memory (with the
+// per-CTA reservation), registers (allocated per warp in units of 256), and
+// tensor memory (512 columns per SM, kTcCols per CTA).  The occupancy API
+// reports one CTA for this kernel where its resources allow two.
 int prefill_tc_ctas_per_sm() {
-  const int smem = int(prefill_tc_smem_bytes());
-  int n = 0;
-  if (cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return 1;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, prefill_tc_kernel, kTcThreads, smem) != cudaSuccess) return 1;
+  int dev = 0, per_sm = 0, reserved = 0, regs_sm = 0;
+  cudaFuncAttributes fa{};
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaFuncGetAttributes(&fa, prefill_tc_kernel) != cudaSuccess ||
+      cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev) != cudaSuccess)
+    return 1;
+  const int by_smem = per_sm / (int(prefill_tc_smem_bytes()) + reserved);
+  const int warp_regs = (fa.numRegs * 32 + 255) / 256 * 256;
+  const int by_regs = regs_sm / (warp_regs * (kTcThreads / 32));
+  const int n = std::min(std::min(by_smem, by_regs), 512 / kTcCols);
   return n > 0 ? n : 1;
 }
 
