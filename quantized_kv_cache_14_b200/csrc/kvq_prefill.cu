@@ -539,26 +539,38 @@ __global__ void __launch_bounds__(kPfThreads, 3) prefill_kernel(const __grid_con
 
 // out[row][hq] = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s over the
 // splits in order (records of splits that saw no position have m = -inf).
-__global__ void __launch_bounds__(kD) prefill_merge_kernel(const float* __restrict__ part, float* __restrict__ out,
-                                                          int splits) {
-  const int c = threadIdx.x;
-  const float* rec = part + int64_t(blockIdx.x) * splits * (kD + 2);
-  // the loops are unrolled so that their independent loads overlap
+// One warp per (row, query head): lane c holds channels 4c .. 4c + 3, and the
+// loads of every split are issued before any is used.
+constexpr int kMergeRowsPerCta = 4;
+__global__ void __launch_bounds__(32 * kMergeRowsPerCta) prefill_merge_kernel(const float* __restrict__ part,
+                                                                             float* __restrict__ out, int splits,
+                                                                             int64_t items) {
+  const int lane = threadIdx.x & 31;
+  const int64_t item = int64_t(blockIdx.x) * kMergeRowsPerCta + (threadIdx.x >> 5);
+  if (item >= items) return;
+  const float* rec = part + item * splits * (kD + 2);
   float M = -INFINITY;
 #pragma unroll 8
   for (int s = 0; s < splits; ++s) M = fmaxf(M, rec[s * (kD + 2) + kD]);
-  float num = 0.0f, den = 0.0f;
+  float4 num = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  float den = 0.0f;
   if (M != -INFINITY) {
 #pragma unroll 8
     for (int s = 0; s < splits; ++s) {
-      const float m = rec[s * (kD + 2) + kD];
-      const float x = rec[s * (kD + 2) + c], y = rec[s * (kD + 2) + kD + 1];
+      const float* r = rec + s * (kD + 2);
+      const float m = r[kD];
+      const float2 x0 = *reinterpret_cast<const float2*>(r + 4 * lane);
+      const float2 x1 = *reinterpret_cast<const float2*>(r + 4 * lane + 2);
       const float w = m == -INFINITY ? 0.0f : fast_exp2(m - M);
-      num = fmaf(w, x, num);
-      den = fmaf(w, y, den);
+      num.x = fmaf(w, x0.x, num.x);
+      num.y = fmaf(w, x0.y, num.y);
+      num.z = fmaf(w, x1.x, num.z);
+      num.w = fmaf(w, x1.y, num.w);
+      den = fmaf(w, r[kD + 1], den);
     }
   }
-  out[int64_t(blockIdx.x) * kD + c] = den > 0.0f ? num / den : 0.0f;
+  const float inv = den > 0.0f ? 1.0f / den : 0.0f;
+  reinterpret_cast<float4*>(out + item * kD)[lane] = make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
 }
 
 template <int BITS, int ASYM>
@@ -584,7 +596,9 @@ cudaError_t launch_prefill_t(const PrefillArgs& a, int64_t n_rows, cudaStream_t 
 }  // namespace
 
 cudaError_t launch_prefill_merge(const PrefillArgs& a, int64_t n_rows, cudaStream_t s, int* launches) {
-  prefill_merge_kernel<<<unsigned(n_rows * a.g.h_q), kD, 0, s>>>(a.part, a.out, a.splits);
+  const int64_t items = n_rows * a.g.h_q;
+  prefill_merge_kernel<<<unsigned((items + kMergeRowsPerCta - 1) / kMergeRowsPerCta), 32 * kMergeRowsPerCta, 0, s>>>(
+      a.part, a.out, a.splits, items);
   ++*launches;
   return cudaGetLastError();
 }
