@@ -259,6 +259,60 @@ def nvtx_pop():
     torch.cuda.nvtx.range_pop()
 
 
+def time_bulk_append(w, new_cache, k_all, v_all, dr, calls):
+    """The bulk prefill append alone, on one cache whose sequences are freed
+    between calls; the first calls grow the library's plan buffer and
+    page-locked plan slots (four of them), so they are not timed.  The GPU is
+    held by a sleep while the host plans, so the events see device time only."""
+    import torch
+    c = new_cache()
+    ts = []
+    for it in range(calls + 4):
+        for sq in range(w.batch):
+            c.free_seq(sq)
+        torch.cuda.synchronize()
+        torch.cuda._sleep(60_000_000)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        c.append(k_all, v_all, dr.seq_ids)
+        e1.record()
+        torch.cuda.synchronize()
+        assert c.sync_status() == 0
+        if it >= 4:
+            ts.append(e0.elapsed_time(e1) * 1e3)
+    c.close()
+    us = float(np.median(ts))
+    nbytes = bulk_append_bytes(w, dr.lengths)
+    return {"us": us, "bytes": nbytes, "gbs": nbytes / (us * 1e-6) / 1e9, "tokens": int(sum(dr.lengths)),
+            "calls": calls, "what": "bulk prefill append of every prefill token, device time"}
+
+
+def run_bulk_only(args):
+    """The workload's bulk prefill append alone (every prefill token of its
+    sequences through one kvq_append call): device time per call."""
+    import torch
+    from quantized_kv_cache_14_b200 import kvq
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    w = workload(args.workload)
+    dr = Draws(w, steps=1)
+    f = w.fmt
+    nb = pool_blocks(dr.lengths, 4, f.page)
+    mbps = max((L + 4) // f.page + 2 for L in dr.lengths)
+    fmt = kvq.Format(f.bits, f.asym, f.k_axis, f.g_k, f.g_v, f.scale_fp32, f.residual, f.page)
+
+    def new_cache():
+        return kvq.KVCache(fmt, w.h_q, w.h_kv, max_seqs=w.batch, num_blocks=nb, max_blocks_per_seq=mbps,
+                           seed=w.seed, device=0)
+
+    def bf16_dev(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    bulk = time_bulk_append(w, new_cache, bf16_dev(dr.k), bf16_dev(dr.v), dr, max(1, min(args.steps, 10)))
+    bulk["workload"] = w.name
+    return bulk
+
+
 def run_gpu(args, rank, ws, dist, widx, steps, warmup, bulk_calls=0):
     """One workload: prefill (bulk append, untimed), then `warmup` steps and
     three timed passes of `steps` steps each -- device-resident inputs (the
@@ -289,33 +343,7 @@ def run_gpu(args, rank, ws, dist, widx, steps, warmup, bulk_calls=0):
         return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
 
     k_all, v_all = bf16_dev(dr.k), bf16_dev(dr.v)
-    bulk = None
-    if bulk_calls > 0:
-        # the bulk prefill append alone, on one cache whose sequences are
-        # freed between calls; the first calls grow the library's plan buffer
-        # and page-locked plan slots (four of them), so they are not timed.
-        # The GPU is held by a sleep while the host plans, so the events see
-        # device time only.
-        c = new_cache()
-        ts = []
-        for it in range(bulk_calls + 4):
-            for sq in range(w.batch):
-                c.free_seq(sq)
-            torch.cuda.synchronize()
-            torch.cuda._sleep(60_000_000)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            c.append(k_all, v_all, dr.seq_ids)
-            e1.record()
-            torch.cuda.synchronize()
-            assert c.sync_status() == 0
-            if it >= 4:
-                ts.append(e0.elapsed_time(e1) * 1e3)
-        c.close()
-        us = float(np.median(ts))
-        nbytes = bulk_append_bytes(w, dr.lengths)
-        bulk = {"us": us, "bytes": nbytes, "gbs": nbytes / (us * 1e-6) / 1e9, "tokens": int(sum(dr.lengths)),
-                "calls": bulk_calls, "what": "bulk prefill append of every prefill token, device time"}
+    bulk = time_bulk_append(w, new_cache, k_all, v_all, dr, bulk_calls) if bulk_calls > 0 else None
     cache = new_cache()
     cache.append(k_all, v_all, dr.seq_ids)      # prefill, untimed
     del k_all, v_all
@@ -551,9 +579,7 @@ def run_next_rows(args):
     groups) plus 64 tokens of their own, the prefix held once through
     kvq_share_prefix, against 16 unshared copies of the same tokens: pool
     blocks and decode time (outputs must agree bit for bit);
-    chunked prefill -- one sequence with an 8192-token context and a new chunk
-    of 256 tokens, each chunk token attending its causal prefix through
-    kvq_prefill_attn: time per chunk and query tokens per second."""
+    chunked prefill -- run_chunked_prefill."""
     import torch
     from quantized_kv_cache_14_b200 import kvq
     from quantized_kv_cache_14_b200.workloads import random_bf16
@@ -603,6 +629,30 @@ def run_next_rows(args):
     share["speedup"] = share["unshared"]["decode_us"] / share["shared"]["decode_us"]
     share["workload"] = f"{B} sequences x ({Lp} shared + {Ls} own) tokens"
 
+    return {"calls": K, "prefix_sharing": share, "chunked_prefill": run_chunked_prefill(args)}
+
+
+def run_chunked_prefill(args):
+    """Chunked prefill on the workload's format: one sequence with an
+    8192-token context and a new chunk of 256 tokens, each chunk token
+    attending its causal prefix through kvq_prefill_attn (a user's call:
+    host planning, plan upload, attention and split merge inside the timed
+    region): time per chunk, query tokens per second and attention TFLOP/s."""
+    import torch
+    from quantized_kv_cache_14_b200 import kvq
+    from quantized_kv_cache_14_b200.workloads import random_bf16
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = workload(args.workload)
+    f = w.fmt
+    K = max(5, min(args.steps, 30))
+    rng = np.random.default_rng(w.seed + 78)
+    fmt = kvq.Format(f.bits, f.asym, f.k_axis, f.g_k, f.g_v, f.scale_fp32, f.residual, f.page, f.fp8)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_rd = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def dbf(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
     Lc, C = 8192, 256
     c = kvq.KVCache(fmt, w.h_q, w.h_kv, max_seqs=C, num_blocks=(Lc + C) // f.page + 64,
                     max_blocks_per_seq=(Lc + C) // f.page + 4, seed=w.seed, device=torch.cuda.current_device())
@@ -621,10 +671,12 @@ def run_next_rows(args):
                "chunk_us": us, "query_tokens_per_s": C / (us * 1e-6),
                "attention_tflops": flops / (us * 1e-6) / 1e12,
                "row_bytes": row_bytes, "row_gbs": row_bytes / (us * 1e-6) / 1e9,
-               "note": "the prefill kernel: 64 / g query tokens of the chunk share every staged tile "
-                       "(rows in the mma M dimension), key range split over CTAs; row_gbs counts the "
-                       "bytes each row would read on its own"}
-    return {"calls": K, "prefix_sharing": share, "chunked_prefill": prefill}
+               "note": "a block of query tokens (32 x 4 heads = 128 rows of the tcgen05 M dimension on "
+                       "the tensor-core path, 64 / g tokens on the mma.sync path) shares every staged "
+                       "tile, key range split over CTAs; row_gbs counts the bytes each row would read "
+                       "on its own"}
+    prefill["calls"] = K
+    return prefill
 
 
 def chunk_used_bytes(w, layout):
@@ -826,12 +878,21 @@ def main():
     ap.add_argument("--no-control", action="store_true", help="skip the BF16 / FP8 comparison and the prefix-sharing and chunked-prefill measurements")
     ap.add_argument("--no-workloads", action="store_true",
                     help="time only --workload (skip the other four workloads' lines)")
+    ap.add_argument("--only", choices=["prefill", "bulk"],
+                    help="measure one row alone and print its own JSON: prefill = chunked prefill, "
+                         "bulk = the workload's bulk prefill append")
     ap.add_argument("--floor", action="store_true",
                     help="measure the HBM read floor of one decode pass instead (one GPU; prints its own JSON)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.floor:
         print(json.dumps(run_floor(args)))
+        return
+    if args.only == "prefill":
+        print(json.dumps(run_chunked_prefill(args)))
+        return
+    if args.only == "bulk":
+        print(json.dumps(run_bulk_only(args)))
         return
 
     rank, ws, dist = dist_setup(args.gpus)

@@ -414,4 +414,35 @@ __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
   return __uint_as_float(uint32_t(b) << 16);
 }
 
+// One row of a split prefill: the records (o[D], m, l) of its `splits` key
+// ranges, back to back, combined by log-sum-exp in split order into
+// out[D] = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s (M the largest m_s;
+// a record with m = -inf saw no position).  Called by a whole warp: lane c
+// holds channels 4c .. 4c + 3, and every split's loads are issued before any
+// is used.  The loads go through L2 only: other CTAs wrote the records.
+__device__ __forceinline__ void prefill_merge_row(const float* rec, int splits, int lane, float* out) {
+  float M = -INFINITY;
+#pragma unroll 8
+  for (int s = 0; s < splits; ++s) M = fmaxf(M, __ldcg(rec + s * (kD + 2) + kD));
+  float4 num = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  float den = 0.0f;
+  if (M != -INFINITY) {
+#pragma unroll 8
+    for (int s = 0; s < splits; ++s) {
+      const float* r = rec + s * (kD + 2);
+      const float m = __ldcg(r + kD);
+      const float2 x0 = __ldcg(reinterpret_cast<const float2*>(r + 4 * lane));
+      const float2 x1 = __ldcg(reinterpret_cast<const float2*>(r + 4 * lane + 2));
+      const float w = m == -INFINITY ? 0.0f : fast_exp2(m - M);
+      num.x = fmaf(w, x0.x, num.x);
+      num.y = fmaf(w, x0.y, num.y);
+      num.z = fmaf(w, x1.x, num.z);
+      num.w = fmaf(w, x1.y, num.w);
+      den = fmaf(w, __ldcg(r + kD + 1), den);
+    }
+  }
+  const float inv = den > 0.0f ? 1.0f / den : 0.0f;
+  reinterpret_cast<float4*>(out)[lane] = make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
+}
+
 }  // namespace kvq

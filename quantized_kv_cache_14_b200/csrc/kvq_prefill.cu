@@ -545,32 +545,13 @@ constexpr int kMergeRowsPerCta = 4;
 __global__ void __launch_bounds__(32 * kMergeRowsPerCta) prefill_merge_kernel(const float* __restrict__ part,
                                                                              float* __restrict__ out, int splits,
                                                                              int64_t items) {
+  // a programmatic dependent launch: the records are complete once the
+  // attention grid is (a no-op after a plain launch)
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
   const int lane = threadIdx.x & 31;
   const int64_t item = int64_t(blockIdx.x) * kMergeRowsPerCta + (threadIdx.x >> 5);
   if (item >= items) return;
-  const float* rec = part + item * splits * (kD + 2);
-  float M = -INFINITY;
-#pragma unroll 8
-  for (int s = 0; s < splits; ++s) M = fmaxf(M, rec[s * (kD + 2) + kD]);
-  float4 num = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  float den = 0.0f;
-  if (M != -INFINITY) {
-#pragma unroll 8
-    for (int s = 0; s < splits; ++s) {
-      const float* r = rec + s * (kD + 2);
-      const float m = r[kD];
-      const float2 x0 = *reinterpret_cast<const float2*>(r + 4 * lane);
-      const float2 x1 = *reinterpret_cast<const float2*>(r + 4 * lane + 2);
-      const float w = m == -INFINITY ? 0.0f : fast_exp2(m - M);
-      num.x = fmaf(w, x0.x, num.x);
-      num.y = fmaf(w, x0.y, num.y);
-      num.z = fmaf(w, x1.x, num.z);
-      num.w = fmaf(w, x1.y, num.w);
-      den = fmaf(w, r[kD + 1], den);
-    }
-  }
-  const float inv = den > 0.0f ? 1.0f / den : 0.0f;
-  reinterpret_cast<float4*>(out + item * kD)[lane] = make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
+  prefill_merge_row(part + item * splits * (kD + 2), splits, lane, out + item * kD);
 }
 
 template <int BITS, int ASYM>
@@ -597,10 +578,22 @@ cudaError_t launch_prefill_t(const PrefillArgs& a, int64_t n_rows, cudaStream_t 
 
 cudaError_t launch_prefill_merge(const PrefillArgs& a, int64_t n_rows, cudaStream_t s, int* launches) {
   const int64_t items = n_rows * a.g.h_q;
-  prefill_merge_kernel<<<unsigned((items + kMergeRowsPerCta - 1) / kMergeRowsPerCta), 32 * kMergeRowsPerCta, 0, s>>>(
-      a.part, a.out, a.splits, items);
-  ++*launches;
-  return cudaGetLastError();
+  // a programmatic dependent launch: scheduled while the attention grid
+  // finishes, waiting for it on the device
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned((items + kMergeRowsPerCta - 1) / kMergeRowsPerCta));
+  cfg.blockDim = dim3(32 * kMergeRowsPerCta);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_merge_kernel, static_cast<const float*>(a.part), a.out,
+                                           int(a.splits), items);
+  if (e == cudaSuccess) ++*launches;
+  return e;
 }
 
 bool prefill_supported(const Geo& g) {

@@ -1,7 +1,8 @@
 // kvq_prefill_tc.cu -- chunked-prefill attention of the INT4 KIVI format (keys
 // per channel G = 64, values per token G = 64, fp16 scales, page 16, BF16
 // window 64, 4 query heads per kv head) on the fifth-generation tensor cores:
-// tcgen05.mma with operands in shared memory and accumulators in tensor memory.
+// tcgen05.mma with operands in shared and tensor memory, accumulators in tensor
+// memory.
 //
 // The attention is that of kvq_decode_attn for every query token of a chunk
 // over its causal prefix (oh-bug.com "KV Cache Quantization in Practice",
@@ -25,16 +26,21 @@
 //    causally, and takes an online-softmax step whose running max only moves
 //    when a score passes it by more than 8 (log2): p = 2^(s - m) <= 256 stays
 //    in fp16, and the accumulator in tensor memory is rescaled only then.
-//    P (fp16) goes to shared memory and O += P V^ is 4 more products into 128
-//    columns of tensor memory.  BF16 window tiles (16 tokens) take the same
-//    path with N = 16.
+//    P (fp16) replaces the scores in tensor memory and O += P V^ is 4 more
+//    products (A from tensor memory) into 128 columns.  BF16 window tiles (16
+//    tokens) take the same path with N = 16.
+//  * The score block is double-buffered in tensor memory, so the products
+//    overlap the CUDA-core work: an item's scores run while its values are
+//    dequantized, its P V while the next item's keys are.
 //  * Thread 0 stages units and window tiles with cp.async.bulk into a
 //    2-stage ring and issues the tensor-core products; tcgen05.commit
 //    signals their completion on mbarriers.  Every wait is bounded (an error
 //    bit, then the CTA drains and leaves); the tensor memory is freed on
 //    every exit path.
 //  * With one split the CTA writes the output; with several it writes (o, m,
-//    l) records that prefill_merge_kernel combines, as the mma.sync kernel's.
+//    l) records that prefill_merge_kernel combines, as the mma.sync kernel's;
+//    the merge is a programmatic dependent launch, scheduled once every CTA
+//    has left its item loop.
 //
 // Shared-memory tiles use the 128-byte swizzle of the tensor-core operand
 // descriptors: a tile is 8-row groups of 128-byte rows (64 fp16 along K),
@@ -57,11 +63,12 @@ constexpr int kTcRows = 128;            // 32 query tokens x 4 heads
 constexpr int kTcStages = 2;
 constexpr int kTcStageBytes = 4 * kTcChunk;   // >= a window tile's 2 x 4096 bytes
 constexpr uint64_t kTcWaitNs = 2000000000ull;
-constexpr int kTcCols = 256;            // tensor-memory columns: S at 0, O at 64
-constexpr int kTcColO = 64;
+constexpr int kTcCols = 256;            // tensor-memory columns: O at 0, two score blocks at 128 and 192
+constexpr int kTcColO = 0;
+constexpr int kTcColS = 128;
 
 struct TcSmem {
-  int q, kh, kl, vt, p, stages, blk, bars, misc, total;
+  int q, kh, kl, vt, stages, blk, bars, misc, total;
 };
 
 __host__ __device__ constexpr TcSmem tc_smem() {
@@ -70,8 +77,6 @@ __host__ __device__ constexpr TcSmem tc_smem() {
   L.kh = L.q + 2 * kTcRows * 128;           // B: [2][64 rows][128 B], hi parts
   L.kl = L.kh + 2 * 64 * 128;               // lo parts
   L.vt = L.kl + 2 * 64 * 128;               // B of P V: [128 rows (channels)][128 B (64 tokens)]
-  L.p = L.kl;                               // A of P V: [128 rows][128 B], over the lo key tile (free
-                                            // once the scores are done; the next keys wait for P V)
   L.stages = L.vt + kD * 128;
   L.blk = L.stages + kTcStages * kTcStageBytes;
   L.bars = L.blk + kPrefillMaxPages * 4;    // stage barriers, then S and O barriers
@@ -106,6 +111,16 @@ __device__ __forceinline__ void tc_mma_f16(uint32_t d_tmem, uint64_t adesc, uint
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
       " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// D[tmem] (+)= A[tmem] B[smem]^T: A's rows are the tensor-memory lanes, two
+// fp16 elements of K per 32-bit column (the lower K index in the low half).
+__device__ __forceinline__ void tc_mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(acc)
       : "memory");
 }
 // Arrive on an mbarrier once every earlier tcgen05.mma of this thread is done.
@@ -147,6 +162,13 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
   asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
 }
 
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[32]) {
+  float f[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
+  tmem_st32(taddr, f);
+}
+
 // Shared-memory operand descriptor of a K-major tile with the 128-byte
 // swizzle: start address (16-byte units), leading offset 1 (unused by this
 // layout), stride offset 1024 bytes (one 8-row group), version 1, layout 2.
@@ -177,6 +199,22 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const __grid_
   volatile int32_t* abort_flag = reinterpret_cast<int32_t*>(smem + L.misc + 4);
   int32_t* sblk = reinterpret_cast<int32_t*>(smem + L.blk);
 
+  // ---- once per CTA: barriers, tensor memory ------------------------------------
+  if (tid == 0) {
+    for (int b = 0; b < kTcStages + 2; ++b) mbar_init(bar_st + 8 * b, 1);
+    mbar_init_fence();
+    *abort_flag = 0;
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_addr(tmem_slot), kTcCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t trow_addr = tmem + (uint32_t(warp * 32) << 16);   // this warp's 32 lanes
+
   // ---- the task: a block of query tokens, a kv head, a range of key units ----
   const int32_t* task = a.plan + a.off_tasks + 5 * blockIdx.x;
   const int bi = task[0], h = task[1], split = task[2], u0 = task[3], u1 = task[4];
@@ -191,16 +229,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const __grid_
   const int tok = tid >> 2, hd = tid & 3;              // this thread's row: token tok of the block, head hd
   const int pos = tok < nrow ? rows[2 * tok + 1] : -1;
 
-  // ---- setup: barriers, tensor memory, block ids, Q ---------------------------
-  if (tid == 0) {
-    for (int b = 0; b < kTcStages + 2; ++b) mbar_init(bar_st + 8 * b, 1);
-    mbar_init_fence();
-    *abort_flag = 0;
-  }
-  if (warp == 0) {
-    tmem_alloc(smem_addr(tmem_slot), kTcCols);
-    tmem_relinquish();
-  }
+  // ---- setup: block ids, Q --------------------------------------------------------
   const int page0 = u0 * 4;                            // 4 pages per 64-token unit
   const int qg = ((qa + 63) >> 6) << 6;                // every page of each key group touched
   const int npages = min(nu * 4, (qg >> 4) - page0);
@@ -249,8 +278,6 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const __grid_
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t trow_addr = tmem + (uint32_t(warp * 32) << 16);   // this warp's 32 lanes
 
   // ---- staging (thread 0) ---------------------------------------------------------
   int issued = 0;
@@ -304,20 +331,10 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const __grid_
     const bool quant = k < nu;
     const int T0 = quant ? (u0 + k) * 64 : Lq + 16 * (k - nu);   // position of the item's first key
     const int nt = quant ? 64 : 16;                               // its keys (N of the score product)
+    const uint32_t s_col = kTcColS + uint32_t(k & 1) * 64;       // its scores, then its P
 
-    // 1. keys: K^ hi and lo tiles [keys][key-list positions], once the previous
-    //    item's P V products (which read P, over the lo tile, and V^T) are done
-    if (k > 0) {
-      const bool okv = mbar_wait_bounded(bar_o, uint32_t((k - 1) & 1), kTcWaitNs, abort_flag);
-      if (__syncthreads_or(!okv)) {
-        if (tid == 0) {
-          atomicOr(a.err, KVQ_DEVERR_TIMEOUT);
-          *abort_flag = 1;
-        }
-        aborted = true;
-        break;
-      }
-    }
+    // 1. keys: K^ hi and lo tiles [keys][key-list positions] (their last
+    //    reader, the previous item's score product, was waited for)
     if (quant) {
       const int w = tid & 15;   // word w of a key row: positions 8w .. 8w + 7, scales on page w / 4
       const uint4 sr = *reinterpret_cast<const uint4*>(stg + (w >> 2) * kTcChunk + kTcOffKm + ((8 * w) & 31) * 2);
@@ -371,7 +388,40 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const __grid_
         *reinterpret_cast<uint4*>(smem + L.kl + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
     }
-    // 2. values: V^T tile [channels][keys]
+    fence_proxy_async();   // the tiles' generic writes before the tensor core's reads
+    tc_fence_before();
+    __syncthreads();
+    // 2. the scores S = Q K^T into this item's column block; they run while
+    //    the values are dequantized
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t idesc = tc_idesc(kTcRows, nt);
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        const uint32_t bt = sb + (part ? L.kl : L.kh);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {   // K = 128 positions in steps of 16 (32 bytes)
+          const uint32_t oa = (ks >> 2) * (kTcRows * 128) + (ks & 3) * 32;
+          const uint32_t ob = (ks >> 2) * (64 * 128) + (ks & 3) * 32;
+          tc_mma_f16(tmem + s_col, sw128_desc(sb + L.q + oa), sw128_desc(bt + ob), idesc, (part | ks) != 0);
+        }
+      }
+      tc_commit(bar_s);
+    }
+    ++s_commits;
+    // 3. values: V^T tile [channels][keys], once the previous item's P V
+    //    product (their last reader) is done
+    if (k > 0) {
+      const bool okv = mbar_wait_bounded(bar_o, uint32_t((k - 1) & 1), kTcWaitNs, abort_flag);
+      if (__syncthreads_or(!okv)) {
+        if (tid == 0) {
+          atomicOr(a.err, KVQ_DEVERR_TIMEOUT);
+          *abort_flag = 1;
+        }
+        aborted = true;
+        break;
+      }
+    }
     if (quant) {
       // lane record (sub-tile st, lane gq * 4 + tq): word i holds channel tile i,
       // register x (x = 0..3) the channel 16 i + gq + 8 (x % 2) for keys
@@ -418,27 +468,6 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const __grid_
             *reinterpret_cast<const uint32_t*>(&pv);
       }
     }
-    fence_proxy_async();   // the tiles' generic writes before the tensor core's reads
-    tc_fence_before();
-    __syncthreads();
-    // 3. the stage is consumed: its next item; the scores
-    if (tid == 0) {
-      if (k + kTcStages < K) issue(k + kTcStages);
-      tc_fence_after();
-      const uint32_t idesc = tc_idesc(kTcRows, nt);
-#pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        const uint32_t bt = sb + (part ? L.kl : L.kh);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {   // K = 128 positions in steps of 16 (32 bytes)
-          const uint32_t oa = (ks >> 2) * (kTcRows * 128) + (ks & 3) * 32;
-          const uint32_t ob = (ks >> 2) * (64 * 128) + (ks & 3) * 32;
-          tc_mma_f16(tmem, sw128_desc(sb + L.q + oa), sw128_desc(bt + ob), idesc, (part | ks) != 0);
-        }
-      }
-      tc_commit(bar_s);
-    }
-    ++s_commits;
     // 4. this row's scores, masked causally; online softmax with a lazy max
     const bool oks = mbar_wait_bounded(bar_s, uint32_t(k & 1), kTcWaitNs, abort_flag);
     if (__syncthreads_or(!oks)) {
@@ -453,11 +482,11 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const __grid_
     float sv[64];
     {
       float h32[32];
-      tmem_ld32(trow_addr, h32);
+      tmem_ld32(trow_addr + s_col, h32);
 #pragma unroll
       for (int j = 0; j < 32; ++j) sv[j] = h32[j];
       if (nt == 64) {
-        tmem_ld32(trow_addr + 32, h32);
+        tmem_ld32(trow_addr + s_col + 32, h32);
 #pragma unroll
         for (int j = 0; j < 32; ++j) sv[32 + j] = h32[j];
       } else {
@@ -487,7 +516,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const __grid_
       m_run = mx;
     }
     if (k > 0 && __any_sync(0xffffffffu, raise)) {
-      // rescale the accumulator rows of this warp (complete: its last products were waited for)
+      // rescale the accumulator rows of this warp (complete: the previous P V was waited for)
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) {
         float ov[32];
@@ -500,7 +529,9 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const __grid_
     {
       // p = 2^(s cs - m): a masked score is -inf and gives 0 (as does a row
       // with nothing attended, m = -inf, whose scores are all -inf); l sums
-      // the fp32 p (its fp16 rounding moves the sum by 2^-12 at most)
+      // the fp32 p (its fp16 rounding moves the sum by 2^-12 at most).  P
+      // (fp16 pairs, key 2c in the low half of column c) replaces the scores
+      // in tensor memory, the A operand of the P V product.
       uint32_t pw[32];
       const float nm = m_run == -INFINITY ? 0.0f : -m_run;
       float lsum = 0.0f;
@@ -513,31 +544,33 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const __grid_
         pw[j >> 1] = *reinterpret_cast<const uint32_t*>(&ph);
       }
       l_run += lsum;
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(smem + L.p + sw128_off(tid, c)) =
-            make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+      tmem_st32u(trow_addr + s_col, pw);
     }
-    fence_proxy_async();
+    fence_proxy_async();   // the V^T tile's generic writes before the tensor core's reads
     tc_fence_before();
     __syncthreads();
-    // 5. O += P V^ (the item's keys in steps of 16)
+    // 5. the stage is consumed: its next item; O += P V^ (the item's keys in
+    //    steps of 16, P from tensor memory); it runs while the next keys are
+    //    dequantized
     if (tid == 0) {
+      if (k + kTcStages < K) issue(k + kTcStages);
       tc_fence_after();
       const uint32_t idesc = tc_idesc(kTcRows, D);
       for (int ks = 0; ks < nt / 16; ++ks)
-        tc_mma_f16(tmem + kTcColO, sw128_desc(sb + L.p + ks * 32), sw128_desc(sb + L.vt + ks * 32), idesc,
-                   (k > 0 || ks > 0) ? 1u : 0u);
+        tc_mma_f16_ts(tmem + kTcColO, tmem + s_col + 8 * ks, sw128_desc(sb + L.vt + ks * 32), idesc,
+                      (k > 0 || ks > 0) ? 1u : 0u);
       tc_commit(bar_o);
     }
     ++o_commits;
   }
 
+  // the merge grid may be scheduled now (it waits on the device for this grid)
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   if (aborted) {
     // bounded: the copies in flight land, the committed products finish
     if (tid == 0)
-      for (int k = consumed; k < issued; ++k)
-        (void)mbar_wait_bounded(bar_st + 8 * (k % kTcStages), uint32_t((k / kTcStages) & 1), kTcWaitNs);
+      for (int j = consumed; j < issued; ++j)
+        (void)mbar_wait_bounded(bar_st + 8 * (j % kTcStages), uint32_t((j / kTcStages) & 1), kTcWaitNs);
     if (s_commits > 0) (void)mbar_wait_bounded(bar_s, uint32_t((s_commits - 1) & 1), kTcWaitNs);
     if (o_commits > 0) (void)mbar_wait_bounded(bar_o, uint32_t((o_commits - 1) & 1), kTcWaitNs);
   } else if (K > 0) {

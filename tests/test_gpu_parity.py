@@ -322,6 +322,45 @@ def test_prefill_kernel_blocks(name, h_q, h_kv):
     p.close()
 
 
+@pytest.mark.parametrize("name", ["int4_chan64", "int2_asym_chan32"])
+def test_prefill_repeated_split_calls(name):
+    """Repeated split prefill calls on one cache give bit-identical outputs
+    (plan buffers and split records reused across calls, the merge a
+    programmatic dependent launch), with a smaller call in between, and match
+    the oracle."""
+    rng = np.random.default_rng(53)
+    fmt = FMTS[name]
+    h_q, h_kv = 8, 2
+    p = Pair(fmt, h_q, h_kv, max_seqs=2, num_blocks=900, mbps=256, seed=5)
+    pre = [2000, 700]
+    ids = np.repeat(np.arange(2, dtype=np.int32), pre)
+    p.append(outlier_keys(rng, ids.size, h_kv), random_bf16(rng, (ids.size, h_kv, D)), ids)
+    chunk = [96, 40]
+    cids = np.concatenate([np.full(c, s, np.int32) for s, c in enumerate(chunk)])
+    p.append(outlier_keys(rng, cids.size, h_kv), random_bf16(rng, (cids.size, h_kv, D)), cids)
+    pos = np.concatenate([np.arange(pre[s], pre[s] + chunk[s]) for s in range(2)]).astype(np.int32)
+    q = random_bf16(rng, (cids.size, h_q, D))
+    qd = bits_to_cuda_bf16(q)
+    outs = []
+    for it in range(3):
+        if it == 1:
+            small = torch.empty((8, h_q, D), dtype=torch.float32, device="cuda")
+            p.gpu.prefill_attn(bits_to_cuda_bf16(q[-8:]), cids[-8:], pos[-8:], small)
+        out = torch.full((cids.size, h_q, D), float("nan"), dtype=torch.float32, device="cuda")
+        p.gpu.prefill_attn(qd, cids, pos, out)
+        outs.append(out)
+    torch.cuda.synchronize()
+    assert p.gpu.sync_status() == 0
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0])
+    want = p.orc.decode(q, (pos + 1).tolist(), seq_ids=cids)
+    got = outs[0].cpu().numpy().astype(np.float64)
+    assert np.max(np.abs(got - want)) <= ATOL
+    want_small = p.orc.decode(q[-8:], (pos[-8:] + 1).tolist(), seq_ids=cids[-8:])
+    assert np.max(np.abs(small.cpu().numpy().astype(np.float64) - want_small)) <= ATOL
+    p.close()
+
+
 @pytest.mark.parametrize("name", ["int4_chan64", "int2_asym_chan32", "int4_chan64_fp32", "int8_tok_p16"])
 def test_prefill_over_shared_prefix(name):
     """Chunked prefill of sequences that hold another sequence's blocks: the
