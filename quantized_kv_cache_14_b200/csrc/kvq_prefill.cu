@@ -539,8 +539,7 @@ __global__ void __launch_bounds__(kPfThreads, 3) prefill_kernel(const __grid_con
 
 // out[row][hq] = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s over the
 // splits in order (records of splits that saw no position have m = -inf).
-// One warp per (row, query head): lane c holds channels 4c .. 4c + 3, and the
-// loads of every split are issued before any is used.
+// One warp per (row, query head): lane c holds channels 4c .. 4c + 3.
 constexpr int kMergeRowsPerCta = 4;
 __global__ void __launch_bounds__(32 * kMergeRowsPerCta) prefill_merge_kernel(const float* __restrict__ part,
                                                                              float* __restrict__ out, int splits,
