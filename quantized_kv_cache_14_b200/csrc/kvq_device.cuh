@@ -414,55 +414,4 @@ __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
   return __uint_as_float(uint32_t(b) << 16);
 }
 
-// One row of a split prefill: the records (o[D], m, l) of its `splits` key
-// ranges, back to back, combined by log-sum-exp in split order into
-// out[D] = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s (M the largest m_s;
-// a record with m = -inf saw no position).  Called by a whole warp: lane c
-// holds channels 4c .. 4c + 3.  The loads of up to 8 records are in flight
-// together (one round trip for 8 splits or fewer; beyond that the running
-// sums are rescaled to each batch's max).  The loads go through L2 only:
-// another grid wrote the records.
-__device__ __forceinline__ void prefill_merge_row(const float* rec, int splits, int lane, float* out) {
-  constexpr int kBatch = 8;
-  float M = -INFINITY, den = 0.0f;
-  float4 num = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  for (int s0 = 0; s0 < splits; s0 += kBatch) {
-    float m[kBatch], l[kBatch];
-    float2 x0[kBatch], x1[kBatch];
-#pragma unroll
-    for (int i = 0; i < kBatch; ++i) {
-      if (s0 + i < splits) {
-        const float* r = rec + (s0 + i) * (kD + 2);
-        m[i] = __ldcg(r + kD);
-        l[i] = __ldcg(r + kD + 1);
-        x0[i] = __ldcg(reinterpret_cast<const float2*>(r + 4 * lane));
-        x1[i] = __ldcg(reinterpret_cast<const float2*>(r + 4 * lane + 2));
-      } else {
-        m[i] = -INFINITY;
-        l[i] = 0.0f;
-        x0[i] = x1[i] = make_float2(0.0f, 0.0f);
-      }
-    }
-    float Mb = M;
-#pragma unroll
-    for (int i = 0; i < kBatch; ++i) Mb = fmaxf(Mb, m[i]);
-    if (Mb == -INFINITY) continue;
-    const float c = M == -INFINITY ? 0.0f : fast_exp2(M - Mb);
-    num = make_float4(num.x * c, num.y * c, num.z * c, num.w * c);
-    den *= c;
-#pragma unroll
-    for (int i = 0; i < kBatch; ++i) {
-      const float w = m[i] == -INFINITY ? 0.0f : fast_exp2(m[i] - Mb);
-      num.x = fmaf(w, x0[i].x, num.x);
-      num.y = fmaf(w, x0[i].y, num.y);
-      num.z = fmaf(w, x1[i].x, num.z);
-      num.w = fmaf(w, x1[i].y, num.w);
-      den = fmaf(w, l[i], den);
-    }
-    M = Mb;
-  }
-  const float inv = den > 0.0f ? 1.0f / den : 0.0f;
-  reinterpret_cast<float4*>(out)[lane] = make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
-}
-
 }  // namespace kvq

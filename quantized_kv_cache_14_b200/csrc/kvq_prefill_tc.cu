@@ -313,20 +313,18 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const __grid_
 
   // ---- items: quantized units, then window tiles -------------------------------------
   float m_run = -INFINITY, l_run = 0.0f;
-  int consumed = 0, s_commits = 0, o_commits = 0;
+  int consumed = 0, s_commits = 0, o_commits = 0;   // consumed: this thread's completed stage waits
   bool aborted = false;
+  auto raise_abort = [&]() {
+    atomicOr(a.err, KVQ_DEVERR_TIMEOUT);
+    *abort_flag = 1;
+  };
   for (int k = 0; k < K; ++k) {
     const int sidx = k % kTcStages;
-    const bool ok = mbar_wait_bounded(bar_st + 8 * sidx, uint32_t((k / kTcStages) & 1), kTcWaitNs, abort_flag);
-    if (__syncthreads_or(!ok)) {
-      if (tid == 0) {
-        atomicOr(a.err, KVQ_DEVERR_TIMEOUT);
-        *abort_flag = 1;
-      }
-      aborted = true;
-      break;
-    }
-    ++consumed;
+    // A wait that gives up raises the abort flag and carries on; the CTA
+    // leaves together at the next barrier (steps 1 and 4 end in one).
+    if (mbar_wait_bounded(bar_st + 8 * sidx, uint32_t((k / kTcStages) & 1), kTcWaitNs, abort_flag)) ++consumed;
+    else raise_abort();
     const uint8_t* stg = smem + L.stages + sidx * kTcStageBytes;
     const bool quant = k < nu;
     const int T0 = quant ? (u0 + k) * 64 : Lq + 16 * (k - nu);   // position of the item's first key
@@ -390,7 +388,10 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const __grid_
     }
     fence_proxy_async();   // the tiles' generic writes before the tensor core's reads
     tc_fence_before();
-    __syncthreads();
+    if (__syncthreads_or(*abort_flag != 0)) {
+      aborted = true;
+      break;
+    }
     // 2. the scores S = Q K^T into this item's column block; they run while
     //    the values are dequantized
     if (tid == 0) {
@@ -411,17 +412,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const __grid_
     ++s_commits;
     // 3. values: V^T tile [channels][keys], once the previous item's P V
     //    product (their last reader) is done
-    if (k > 0) {
-      const bool okv = mbar_wait_bounded(bar_o, uint32_t((k - 1) & 1), kTcWaitNs, abort_flag);
-      if (__syncthreads_or(!okv)) {
-        if (tid == 0) {
-          atomicOr(a.err, KVQ_DEVERR_TIMEOUT);
-          *abort_flag = 1;
-        }
-        aborted = true;
-        break;
-      }
-    }
+    if (k > 0 && !mbar_wait_bounded(bar_o, uint32_t((k - 1) & 1), kTcWaitNs, abort_flag)) raise_abort();
     if (quant) {
       // lane record (sub-tile st, lane gq * 4 + tq): word i holds channel tile i,
       // register x (x = 0..3) the channel 16 i + gq + 8 (x % 2) for keys
@@ -469,15 +460,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const __grid_
       }
     }
     // 4. this row's scores, masked causally; online softmax with a lazy max
-    const bool oks = mbar_wait_bounded(bar_s, uint32_t(k & 1), kTcWaitNs, abort_flag);
-    if (__syncthreads_or(!oks)) {
-      if (tid == 0) {
-        atomicOr(a.err, KVQ_DEVERR_TIMEOUT);
-        *abort_flag = 1;
-      }
-      aborted = true;
-      break;
-    }
+    if (!mbar_wait_bounded(bar_s, uint32_t(k & 1), kTcWaitNs, abort_flag)) raise_abort();
     tc_fence_after();
     float sv[64];
     {
@@ -548,7 +531,10 @@ __global__ void __launch_bounds__(kTcThreads, 2) prefill_tc_kernel(const __grid_
     }
     fence_proxy_async();   // the V^T tile's generic writes before the tensor core's reads
     tc_fence_before();
-    __syncthreads();
+    if (__syncthreads_or(*abort_flag != 0)) {
+      aborted = true;
+      break;
+    }
     // 5. the stage is consumed: its next item; O += P V^ (the item's keys in
     //    steps of 16, P from tensor memory); it runs while the next keys are
     //    dequantized

@@ -170,27 +170,36 @@ def test_step_host_equals_device_calls(name):
     a.append(k0, v0, ids)
     b.append(bits_to_cuda_bf16(k0), bits_to_cuda_bf16(v0), ids)
 
-    def host(bits):
-        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).pin_memory()
+    def host(bits, pinned=True):
+        t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+        return t.pin_memory() if pinned else t.clone()
 
-    def packed(k, v, q):
-        # one page-locked buffer holding k | v | q back to back (one H2D copy)
-        buf = host(np.concatenate([k.ravel(), v.ravel(), q.ravel()]))
+    def packed(k, v, q, pinned=True):
+        # one host buffer holding k | v | q back to back
+        buf = host(np.concatenate([k.ravel(), v.ravel(), q.ravel()]), pinned)
         return buf[:k.size].view(k.shape), buf[k.size:2 * k.size].view(v.shape), buf[2 * k.size:].view(q.shape)
 
-    for step in range(70):   # crosses group boundaries of every sequence
+    for step in range(72):   # crosses group boundaries of every sequence
         ids = np.arange(S, dtype=np.int32)
         k, v, q = outlier_keys(rng, S, h_kv), random_bf16(rng, (S, h_kv, D)), random_bf16(rng, (S, h_q, D))
         lens = [L + 1 for L in lens]
         a.append(k, v, ids)
-        if step % 2 == 0:   # packed inputs, output written straight into page-locked memory
-            out_h = torch.full((S, h_q, D), float("nan"), dtype=torch.float32).pin_memory()
-            b.step_host(*packed(k, v, q)[:2], ids, packed(k, v, q)[2], out_h)
-        else:               # separate inputs, pageable output (one copy back)
-            out_h = torch.full((S, h_q, D), float("nan"), dtype=torch.float32)
-            b.step_host(host(k), host(v), ids, host(q), out_h)
+        mode = step % 4
+        pinned_out = mode in (0, 2)
+        out_h = torch.full((S, h_q, D), float("nan"), dtype=torch.float32)
+        if pinned_out:   # the output written straight into page-locked memory
+            out_h = out_h.pin_memory()
+        if mode == 0:    # page-locked k | v | q back to back: one copy
+            kh, vh, qh = packed(k, v, q)
+        elif mode == 1:  # separate page-locked buffers
+            kh, vh, qh = host(k), host(v), host(q)
+        elif mode == 2:  # pageable k | v | q back to back: one copy of all three
+            kh, vh, qh = packed(k, v, q, pinned=False)
+        else:            # separate pageable buffers: three copies
+            kh, vh, qh = host(k, False), host(v, False), host(q, False)
+        b.step_host(kh, vh, ids, qh, out_h)
         torch.cuda.synchronize()
-        if step % 23 == 0 or step == 69:
+        if step % 23 == 0 or step >= 68:
             got, want = a.decode(q, lens)
             assert np.array_equal(out_h.numpy(), got.astype(np.float32))
             assert np.max(np.abs(got - want)) <= ATOL
