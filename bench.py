@@ -865,6 +865,18 @@ def workload_config(w, lens):
     }
 
 
+def attention_kernel_name(w):
+    """The decode attention kernel the library picks for the workload's format
+    (the warp-specialised kernel's three specs, else the generic kernel)."""
+    f = w.fmt
+    if (w.h_q // w.h_kv == 4 and f.page == 16 and not f.scale_fp32 and not f.fp8 and
+            (f.bits, f.asym, f.k_axis, f.g_k, f.g_v, f.residual) in
+            ((4, 0, 1, 64, 64, 64), (2, 1, 1, 32, 32, 32), (8, 0, 0, 128, 128, 0))):
+        spec = {4: "SpecInt4Kivi", 2: "SpecInt2Kivi", 8: "SpecInt8Tok"}[f.bits]
+        return f"decode_ws_kernel<{spec}>"
+    return "decode_kernel"
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -962,7 +974,7 @@ def main():
         "roofline": {"bound": "hbm", "achieved": res["attn_gbs"], "peak": peak, "unit": "GB/s",
                      "frac": res["attn_gbs"] / peak, "traffic": traffic,
                      "peak_kind": peak_kind,
-                     "kernel": "decode_kernel (attention, without the merge)"},
+                     "kernel": attention_kernel_name(w) + " (attention, without the merge)"},
         "cpu_baseline": cpu,
         "e2e": {"value": res["e2e_gbs"], "unit": "GB/s", "h2d_bytes_per_step": res["h2d"],
                 "d2h_bytes_per_step": res["d2h"]},
