@@ -32,6 +32,10 @@ static_assert(sizeof(Geo) + sizeof(DevState) + sizeof(PlanView) + 3 * sizeof(voi
 
 // The bulk flush gives up on its row copies after 2 s (a device error bit).
 constexpr uint64_t kFlushWaitNs = 2000000000ull;
+// Row stride (bf16 elements) of the bulk flush's gathered K and V rows: 16
+// bytes of padding per 256-byte row move consecutive rows by four banks (and
+// keep every row 16-byte aligned for its bulk copy).
+constexpr int kFlushRowStride = kD + 8;
 
 // A decode launched right after an append is a programmatic dependent launch:
 // letting it be scheduled at the start of every append kernel hides its launch
@@ -441,9 +445,10 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
   constexpr uint32_t MASK = (1u << BITS) - 1;
   extern __shared__ __align__(16) uint8_t smem[];
   const int R = g.R;
-  uint16_t* kt = reinterpret_cast<uint16_t*>(smem);                 // [R][D] bf16
-  uint16_t* vt = kt + R * D;                                        // [R][D] bf16
-  float* ksc = reinterpret_cast<float*>(vt + R * D);                // [D]
+  constexpr int RS = kFlushRowStride;
+  uint16_t* kt = reinterpret_cast<uint16_t*>(smem);                 // [R][RS] bf16 (D used)
+  uint16_t* vt = kt + R * RS;                                       // [R][RS] bf16
+  float* ksc = reinterpret_cast<float*>(vt + R * RS);               // [D]
   float* kzp = ksc + D;                                             // [D]
   float* vsc = kzp + D;                                             // [R][nvg]
   float* vzp = vsc + R * g.nvg;                                     // [R][nvg]
@@ -474,7 +479,7 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
     const int32_t s = ssrc[r];
     const uint16_t* src = s >= 0 ? (which ? vin : kin) + (int64_t(s) * g.h_kv + h) * D
                                  : (which ? d.vres : d.kres) + ((int64_t(seq) * g.h_kv + h) * R + (-1 - s)) * D;
-    bulk_g2s(smem_addr((which ? vt : kt) + r * D), src, uint32_t(D * 2), gbar);
+    bulk_g2s(smem_addr((which ? vt : kt) + r * RS), src, uint32_t(D * 2), gbar);
   }
   if (!__syncthreads_and(mbar_wait_bounded(gbar, 0, kFlushWaitNs))) {
     if (tid == 0) atomicOr(d.err, KVQ_DEVERR_TIMEOUT);
@@ -492,7 +497,7 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
     float a[2] = {0.0f, 0.0f}, mn[2] = {INFINITY, INFINITY}, mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll 4
     for (int r = r0; r < r1; ++r) {
-      const uint32_t pr = *reinterpret_cast<const uint32_t*>(kt + r * D + 2 * cp);
+      const uint32_t pr = *reinterpret_cast<const uint32_t*>(kt + r * RS + 2 * cp);
       const float x[2] = {__uint_as_float(pr << 16), __uint_as_float(pr & 0xFFFF0000u)};
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
@@ -543,7 +548,7 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
     const int w = tid >> 5, lane = tid & 31;
     const int lanes_per_group = g.g_v / 4;   // a power of two
     for (int r = w; r < R; r += T / 32) {
-      const uint2 raw = *reinterpret_cast<const uint2*>(vt + r * D + 4 * lane);
+      const uint2 raw = *reinterpret_cast<const uint2*>(vt + r * RS + 4 * lane);
       const float x0 = bf16_bits_to_float(uint16_t(raw.x)), x1 = bf16_bits_to_float(uint16_t(raw.x >> 16));
       const float x2 = bf16_bits_to_float(uint16_t(raw.y)), x3 = bf16_bits_to_float(uint16_t(raw.y >> 16));
       if (ASYM) {
@@ -604,7 +609,7 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
       float xs[N];
 #pragma unroll
       for (int m = 0; m < N / 2; ++m) {
-        const uint32_t pr = *reinterpret_cast<const uint32_t*>(kt + rowi * D + cp[m]);
+        const uint32_t pr = *reinterpret_cast<const uint32_t*>(kt + rowi * RS + cp[m]);
         xs[2 * m] = __uint_as_float(pr << 16);
         xs[2 * m + 1] = __uint_as_float(pr & 0xFFFF0000u);
       }
@@ -638,48 +643,66 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
   //    16 i + gq + 8 (reg % 2), each code with its token's scale for the
   //    channel's value group
   {
+    // Thread (sub, lam, half) makes the record's words half·WPT .. half·WPT +
+    // WPT - 1 and stores them at once: a warp writes 16 records, 512
+    // contiguous bytes.  Its reads of the bf16 rows (channels 16 i + gq, token
+    // rows 2 tq apart) fall in distinct banks up to a factor 2 thanks to the
+    // padded row stride.
     constexpr int RECW = 2 * BITS;                    // words per lane record
+    constexpr int WPT = RECW / 2;                     // words per thread
     const int lg_gv = __ffs(g.g_v) - 1;
-    for (int W = tid; W < (R / 16) * 32 * RECW; W += kFlushThreads) {   // warp-uniform trip count
-      const int sub = W / (32 * RECW), rem = W % (32 * RECW);
-      const int lam = rem / RECW, w = rem % RECW;
+    for (int W = tid; W < (R / 16) * 64; W += kFlushThreads) {   // warp-uniform trip count
+      const int sub = W >> 6, lam = (W >> 1) & 31, half = W & 1;
       const int gq = lam >> 2, tq = lam & 3;
-      float xs[N];
-      int tk[N / 2], cc[N / 2];
-      uint32_t word = 0, ties = 0;
+      uint32_t wd[WPT];
 #pragma unroll
-      for (int x = 0; x < N / 2; ++x) {
-        int i, reg;
-        if (BITS == 8) { i = w >> 1; reg = 2 * (w & 1) + x; }
-        else if (BITS == 4) { i = w; reg = x; }
-        else { i = 2 * w + ((x >> 1) & 1); reg = 2 * (x >> 2) + (x & 1); }
-        const int c = 16 * i + gq + 8 * (reg & 1);
-        const int t0 = 16 * sub + 2 * tq + 8 * (reg >> 1);
-        tk[x] = t0;
-        cc[x] = c;
+      for (int j = 0; j < WPT; ++j) {
+        const int w = half * WPT + j;
+        float xs[N];
+        int tk[N / 2], cc[N / 2];
+        uint32_t word = 0, ties = 0;
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int t = t0 + u, l = x + u * (N / 2);
-          xs[l] = bf16_bits_to_float(vt[t * D + c]);
-          const int m = t * g.nvg + (c >> lg_gv);
-          bool tie;
-          const int q = ASYM ? quant_code_nb(__fsub_rn(xs[l], vzp[m]) * vinv[m], 0, Q, tie)
-                             : quant_code_nb(xs[l] * vinv[m], -Q, Q, tie);
-          ties |= uint32_t(tie) << l;
-          word |= (uint32_t(q) & MASK) << (BITS * l);
-        }
-      }
-      if (__any_sync(0xffffffffu, ties != 0)) {
-        for (int l = 0; l < N; ++l)
-          if (ties & (1u << l)) {
-            const int x = l % (N / 2), t = tk[x] + l / (N / 2), c = cc[x];
+        for (int x = 0; x < N / 2; ++x) {
+          int i, reg;
+          if (BITS == 8) { i = w >> 1; reg = 2 * (w & 1) + x; }
+          else if (BITS == 4) { i = w; reg = x; }
+          else { i = 2 * w + ((x >> 1) & 1); reg = 2 * (x >> 2) + (x & 1); }
+          const int c = 16 * i + gq + 8 * (reg & 1);
+          const int t0 = 16 * sub + 2 * tq + 8 * (reg >> 1);
+          tk[x] = t0;
+          cc[x] = c;
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int t = t0 + u, l = x + u * (N / 2);
+            xs[l] = bf16_bits_to_float(vt[t * RS + c]);
             const int m = t * g.nvg + (c >> lg_gv);
-            const int q = ASYM ? quant_asym_exact(xs[l], vsc[m], vzp[m], Q) : quant_sym_exact(xs[l], vsc[m], Q);
-            word = (word & ~(MASK << (BITS * l))) | ((uint32_t(q) & MASK) << (BITS * l));
+            bool tie;
+            const int q = ASYM ? quant_code_nb(__fsub_rn(xs[l], vzp[m]) * vinv[m], 0, Q, tie)
+                               : quant_code_nb(xs[l] * vinv[m], -Q, Q, tie);
+            ties |= uint32_t(tie) << l;
+            word |= (uint32_t(q) & MASK) << (BITS * l);
           }
+        }
+        if (__any_sync(0xffffffffu, ties != 0)) {
+          for (int l = 0; l < N; ++l)
+            if (ties & (1u << l)) {
+              const int x = l % (N / 2), t = tk[x] + l / (N / 2), c = cc[x];
+              const int m = t * g.nvg + (c >> lg_gv);
+              const int q = ASYM ? quant_asym_exact(xs[l], vsc[m], vzp[m], Q) : quant_sym_exact(xs[l], vsc[m], Q);
+              word = (word & ~(MASK << (BITS * l))) | ((uint32_t(q) & MASK) << (BITS * l));
+            }
+        }
+        wd[j] = word;
       }
-      *reinterpret_cast<uint32_t*>(chunk_of(sub / subs_per_page) + g.off_V + (sub % subs_per_page) * g.sub_bytes +
-                                   lam * (8 * BITS) + 4 * w) = word;
+      uint8_t* dst = chunk_of(sub / subs_per_page) + g.off_V + (sub % subs_per_page) * g.sub_bytes +
+                     lam * (8 * BITS) + half * (4 * WPT);
+      if constexpr (WPT >= 4) {
+#pragma unroll
+        for (int v = 0; v < WPT / 4; ++v)
+          reinterpret_cast<uint4*>(dst)[v] = make_uint4(wd[4 * v], wd[4 * v + 1], wd[4 * v + 2], wd[4 * v + 3]);
+      } else {
+        *reinterpret_cast<uint2*>(dst) = make_uint2(wd[0], wd[1]);
+      }
     }
   }
 
@@ -807,7 +830,7 @@ size_t flush_smem_bytes(const Geo& g) {
 }
 
 size_t flush_group_smem_bytes(const Geo& g) {
-  return size_t(2) * g.R * kD * 2 + size_t(3) * kD * 4 +
+  return size_t(2) * g.R * kFlushRowStride * 2 + size_t(3) * kD * 4 +
          size_t(3) * g.R * g.nvg * 4 + size_t(9) * kD * 4 + size_t((g.R + 1) & ~1) * 4 + 8;
 }
 
