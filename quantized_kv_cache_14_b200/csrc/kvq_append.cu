@@ -541,30 +541,44 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
       }
     }
   }
-  // value (token, group) extremes: warp w takes rows w, w + 8, ...; lane l
-  // holds channels 4l .. 4l + 3 (one 64-bit load), reduced over the g_v / 4
-  // lanes of its group; the scales follow once every row is reduced
+  // value (token, group) extremes: warp w takes rows 2w, 2w + 1, 2w + 16, ...
+  // (a half-warp per row); lane l holds channels 8 (l mod 16) .. + 7 (one
+  // 16-byte load), reduced over the g_v / 8 lanes of its group; the scales
+  // follow once every row is reduced
   {
-    const int w = tid >> 5, lane = tid & 31;
-    const int lanes_per_group = g.g_v / 4;   // a power of two
-    for (int r = w; r < R; r += T / 32) {
-      const uint2 raw = *reinterpret_cast<const uint2*>(vt + r * RS + 4 * lane);
-      const float x0 = bf16_bits_to_float(uint16_t(raw.x)), x1 = bf16_bits_to_float(uint16_t(raw.x >> 16));
-      const float x2 = bf16_bits_to_float(uint16_t(raw.y)), x3 = bf16_bits_to_float(uint16_t(raw.y >> 16));
+    const int w = tid >> 5, lane = tid & 31, cl = lane & 15;
+    const int lanes_per_group = g.g_v / 8;   // 4, 8 or 16: inside the half-warp
+    for (int r0 = 2 * w; r0 < R; r0 += 2 * (T / 32)) {   // R is even: warp-uniform
+      const int r = r0 + (lane >> 4);
+      const uint4 raw = *reinterpret_cast<const uint4*>(vt + r * RS + 8 * cl);
+      const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
+      float x[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        x[2 * i] = __uint_as_float(rw[i] << 16);
+        x[2 * i + 1] = __uint_as_float(rw[i] & 0xFFFF0000u);
+      }
       if (ASYM) {
-        float mn = fminf(fminf(x0, x1), fminf(x2, x3)), mx = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
+        float mn = x[0], mx = x[0];
+#pragma unroll
+        for (int i = 1; i < 8; ++i) {
+          mn = fminf(mn, x[i]);
+          mx = fmaxf(mx, x[i]);
+        }
         for (int off = 1; off < lanes_per_group; off <<= 1) {
           mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
         }
-        if ((lane & (lanes_per_group - 1)) == 0) {
-          vzp[r * g.nvg + lane / lanes_per_group] = mn;   // raw extremes for now
-          vsc[r * g.nvg + lane / lanes_per_group] = mx;
+        if ((cl & (lanes_per_group - 1)) == 0) {
+          vzp[r * g.nvg + cl / lanes_per_group] = mn;   // raw extremes for now
+          vsc[r * g.nvg + cl / lanes_per_group] = mx;
         }
       } else {
-        float a = fmaxf(fmaxf(fabsf(x0), fabsf(x1)), fmaxf(fabsf(x2), fabsf(x3)));
+        float a = fabsf(x[0]);
+#pragma unroll
+        for (int i = 1; i < 8; ++i) a = fmaxf(a, fabsf(x[i]));
         for (int off = 1; off < lanes_per_group; off <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
-        if ((lane & (lanes_per_group - 1)) == 0) vsc[r * g.nvg + lane / lanes_per_group] = a;
+        if ((cl & (lanes_per_group - 1)) == 0) vsc[r * g.nvg + cl / lanes_per_group] = a;
       }
     }
   }
@@ -658,8 +672,11 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
 #pragma unroll
       for (int j = 0; j < WPT; ++j) {
         const int w = half * WPT + j;
+        // the word's channels lie in 16 (32 for 2-bit codes) aligned
+        // channels, inside one value group (g_v is 32, 64 or 128)
+        const int gi = ((BITS == 2 ? 32 : BITS == 4 ? 16 : 8) * w) >> lg_gv;
         float xs[N];
-        int tk[N / 2], cc[N / 2];
+        int tk[N / 2];
         uint32_t word = 0, ties = 0;
 #pragma unroll
         for (int x = 0; x < N / 2; ++x) {
@@ -670,12 +687,11 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
           const int c = 16 * i + gq + 8 * (reg & 1);
           const int t0 = 16 * sub + 2 * tq + 8 * (reg >> 1);
           tk[x] = t0;
-          cc[x] = c;
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const int t = t0 + u, l = x + u * (N / 2);
             xs[l] = bf16_bits_to_float(vt[t * RS + c]);
-            const int m = t * g.nvg + (c >> lg_gv);
+            const int m = t * g.nvg + gi;
             bool tie;
             const int q = ASYM ? quant_code_nb(__fsub_rn(xs[l], vzp[m]) * vinv[m], 0, Q, tie)
                                : quant_code_nb(xs[l] * vinv[m], -Q, Q, tie);
@@ -686,8 +702,8 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
         if (__any_sync(0xffffffffu, ties != 0)) {
           for (int l = 0; l < N; ++l)
             if (ties & (1u << l)) {
-              const int x = l % (N / 2), t = tk[x] + l / (N / 2), c = cc[x];
-              const int m = t * g.nvg + (c >> lg_gv);
+              const int t = tk[l % (N / 2)] + l / (N / 2);
+              const int m = t * g.nvg + gi;
               const int q = ASYM ? quant_asym_exact(xs[l], vsc[m], vzp[m], Q) : quant_sym_exact(xs[l], vsc[m], Q);
               word = (word & ~(MASK << (BITS * l))) | ((uint32_t(q) & MASK) << (BITS * l));
             }
