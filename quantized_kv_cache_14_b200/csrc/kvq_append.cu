@@ -358,7 +358,7 @@ __global__ void __launch_bounds__(kFlushThreads) flush_kernel(const Geo g, const
     const int q = ASYM ? quant_asym_fast(x, vsc[m], vinv[m], vzp[m], Q) : quant_sym_fast(x, vsc[m], vinv[m], Q);
     return uint32_t(q) & ((1u << BITS) - 1);
   };
-  const int subs_per_page = g.P / 16;
+  const int lg_spp = g.lg_P - 4, spp_mask = (1 << lg_spp) - 1;   // 16-token sub-tiles per page (a power of two)
 
   // 3. key codes: word W of the group -> (sub-tile, row, word in row)
   const int row_words = D * BITS / 32;
@@ -368,7 +368,7 @@ __global__ void __launch_bounds__(kFlushThreads) flush_kernel(const Geo g, const
     uint32_t word = 0;
     for (int l = 0; l < N; ++l) word |= kcode(rowi, key_channel(w * N + l)) << (BITS * word_field(l, N));
     const int sub = rowi >> 4, rr = rowi & 15;
-    uint8_t* dst = chunk_of(sub / subs_per_page) + (sub % subs_per_page) * g.sub_bytes +
+    uint8_t* dst = chunk_of(sub >> lg_spp) + (sub & spp_mask) * g.sub_bytes +
                    rr * g.row_bytes + 4 * w;
     *reinterpret_cast<uint32_t*>(dst) = word;
   }
@@ -394,7 +394,7 @@ __global__ void __launch_bounds__(kFlushThreads) flush_kernel(const Geo g, const
       word |= vcode(t0, c) << (BITS * x);
       word |= vcode(t0 + 1, c) << (BITS * (x + N / 2));
     }
-    uint8_t* dst = chunk_of(sub / subs_per_page) + g.off_V + (sub % subs_per_page) * g.sub_bytes +
+    uint8_t* dst = chunk_of(sub >> lg_spp) + g.off_V + (sub & spp_mask) * g.sub_bytes +
                    lam * (8 * BITS) + 4 * w;
     *reinterpret_cast<uint32_t*>(dst) = word;
   }
@@ -599,7 +599,7 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
   auto chunk_of = [&](int page) -> uint8_t* {
     return d.pool + int64_t(ent[3 + page]) * g.block_bytes + int64_t(h) * g.chunk_bytes;
   };
-  const int subs_per_page = g.P / 16;
+  const int lg_spp = g.lg_P - 4, spp_mask = (1 << lg_spp) - 1;   // 16-token sub-tiles per page (a power of two)
 
   // 3. key words, straight from the bf16 rows: word kw of a row holds the
   //    codes of key-list positions kw N .. kw N + N - 1, i.e. N / 2 pairs of
@@ -646,7 +646,7 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
           }
       }
       const int sub = rowi >> 4, rr = rowi & 15;
-      *reinterpret_cast<uint32_t*>(chunk_of(sub / subs_per_page) + (sub % subs_per_page) * g.sub_bytes +
+      *reinterpret_cast<uint32_t*>(chunk_of(sub >> lg_spp) + (sub & spp_mask) * g.sub_bytes +
                                    rr * g.row_bytes + 4 * kw) = word;
     }
   }
@@ -710,7 +710,7 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
         }
         wd[j] = word;
       }
-      uint8_t* dst = chunk_of(sub / subs_per_page) + g.off_V + (sub % subs_per_page) * g.sub_bytes +
+      uint8_t* dst = chunk_of(sub >> lg_spp) + g.off_V + (sub & spp_mask) * g.sub_bytes +
                      lam * (8 * BITS) + half * (4 * WPT);
       if constexpr (WPT >= 4) {
 #pragma unroll
@@ -723,17 +723,18 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
   }
 
   // 6. metadata: each page's slice of the key scales (list order), value scales
-  const int npg = R / g.P;
+  //    (page, kslice and nvg = D / g_v are powers of two)
+  const int npg = R >> g.lg_P, lg_nvg = __ffs(g.nvg) - 1;
   for (int idx = tid; idx < npg * g.kslice; idx += T) {
-    const int page = idx / g.kslice, off = idx % g.kslice;
+    const int page = idx >> g.lg_kslice, off = idx & (g.kslice - 1);
     const int c = key_channel(page * g.kslice + off);
     uint8_t* km = chunk_of(page) + g.off_Km;
     store_meta(km + off * g.es, ksc[c], g.scale_fp32);
     if (ASYM) store_meta(km + (g.kslice + off) * g.es, kzp[c], g.scale_fp32);
   }
   for (int idx = tid; idx < R * g.nvg; idx += T) {
-    const int r = idx / g.nvg, gi = idx % g.nvg;
-    const int page = r / g.P, rp = r % g.P;
+    const int r = idx >> lg_nvg, gi = idx & (g.nvg - 1);
+    const int page = r >> g.lg_P, rp = r & (g.P - 1);
     uint8_t* vm = chunk_of(page) + g.off_Vm;
     store_meta(vm + (rp * g.nvg + gi) * g.es, vsc[idx], g.scale_fp32);
     if (ASYM) store_meta(vm + (g.P * g.nvg + rp * g.nvg + gi) * g.es, vzp[idx], g.scale_fp32);
