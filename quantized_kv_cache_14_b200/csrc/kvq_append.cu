@@ -402,8 +402,9 @@ __global__ void __launch_bounds__(kFlushThreads) flush_kernel(const Geo g, const
   // 5. metadata: key scales in list order, striped over the group's pages
   //    (the CTA of a page's first sub-tile writes that page's slice); value
   //    scales of this sub-tile's rows
-  if (r_lo % g.P == 0) {
-    const int page = r_lo / g.P;
+  //    (page and nvg are powers of two)
+  if ((r_lo & (g.P - 1)) == 0) {
+    const int page = r_lo >> g.lg_P;
     for (int off = tid; off < g.kslice; off += blockDim.x) {
       const int c = key_channel(page * g.kslice + off);
       uint8_t* km = chunk_of(page) + g.off_Km;
@@ -411,9 +412,10 @@ __global__ void __launch_bounds__(kFlushThreads) flush_kernel(const Geo g, const
       if (ASYM) store_meta(km + (g.kslice + off) * g.es, kzp[c], g.scale_fp32);
     }
   }
+  const int lg_nvg = __ffs(g.nvg) - 1;
   for (int idx = r_lo * g.nvg + tid; idx < (r_lo + 16) * g.nvg; idx += blockDim.x) {
-    const int r = idx / g.nvg, gi = idx % g.nvg;
-    const int page = r / g.P, rp = r % g.P;
+    const int r = idx >> lg_nvg, gi = idx & (g.nvg - 1);
+    const int page = r >> g.lg_P, rp = r & (g.P - 1);
     uint8_t* vm = chunk_of(page) + g.off_Vm;
     store_meta(vm + (rp * g.nvg + gi) * g.es, vsc[idx], g.scale_fp32);
     if (ASYM) store_meta(vm + (g.P * g.nvg + rp * g.nvg + gi) * g.es, vzp[idx], g.scale_fp32);
