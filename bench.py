@@ -34,6 +34,7 @@ the quantized, BF16 and FP8 caches; and `next_rows` measures prefix sharing
 NVTX ranges mark every append, decode and step_host call.
 """
 import argparse
+import gc
 import hashlib
 import json
 import os
@@ -328,7 +329,7 @@ def run_gpu(args, rank, ws, dist, widx, steps, warmup, bulk_calls=0):
     dev = torch.device("cuda", torch.cuda.current_device())
     w = workload(widx)
     w.seed = w.seed + 1000 * rank        # each replica draws its own inputs
-    total_steps = warmup + 3 * steps     # warm-up, device pass, attention pass, e2e pass
+    total_steps = warmup + 3 * steps + 1   # warm-up, device pass, attention pass, e2e warm-up + pass
     dr = Draws(w, steps=total_steps)
     f = w.fmt
     nb = pool_blocks(dr.lengths, total_steps + 2, f.page)
@@ -404,6 +405,8 @@ def run_gpu(args, rank, ws, dist, widx, steps, warmup, bulk_calls=0):
     # timed: device-resident inputs, the calls as a user makes them.  The
     # host enqueues every step before waiting (as a serving loop runs ahead of
     # the GPU), so the events see device time, not host launch gaps.
+    gc.collect()
+    gc.disable()   # no collector pause inside a timed region (enabled again below)
     st0 = cache.stats()["kernel_launches"]
     sampler = ClockSampler(torch.cuda.current_device(), enabled=not args.no_clocks)
     time.sleep(0.15 if sampler.proc else 0)
@@ -448,11 +451,15 @@ def run_gpu(args, rank, ws, dist, widx, steps, warmup, bulk_calls=0):
     cache.set_decode_event(None)
     assert cache.sync_status() == 0
 
-    # timed: end to end through the C ABI with host buffers
+    # timed: end to end through the C ABI with host buffers, after one untimed
+    # step through the same call (its first use grows the library's host-step
+    # buffers: a device synchronize and an allocation)
+    s0 += steps
+    one_step(s0, True, [torch.cuda.Event(enable_timing=True) for _ in range(3)])
+    s0 += 1
     barrier(dist)
     torch.cuda.synchronize()
     e2e_ms, e2e_bytes = 0.0, 0
-    s0 += steps
     for s in range(s0, s0 + steps):
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
         one_step(s, True, evs)
@@ -460,6 +467,7 @@ def run_gpu(args, rank, ws, dist, widx, steps, warmup, bulk_calls=0):
         e2e_ms += evs[0].elapsed_time(evs[2])
         e2e_bytes += decode_bytes(w, lens)
     torch.cuda.synchronize()
+    gc.enable()
     barrier(dist)
     assert cache.sync_status() == 0
     cache.close()
