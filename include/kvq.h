@@ -417,8 +417,11 @@ kvq_status kvq_decode_attn_noalloc(const kvq_config* cfg, const void* pool, cons
  *                   stored position of its sequence.
  *   out             device fp32 [n][h_q][d_h].
  * Channel-axis formats with the window (2/4/8-bit codes, fp16 scales) run
- * the prefill kernel: up to 64 / g query tokens of one sequence share every
- * staged tile (their rows are the mma M dimension), the key range split over
+ * a prefill kernel whose query tokens of one sequence share every staged
+ * tile: the INT4 format with keys per channel G = 64, values per token G = 64,
+ * page 16, window 64 and 4 query heads per kv head on the tensor-core kernel
+ * (blocks of 32 tokens, 128 rows of the tcgen05 M dimension), the others on
+ * the mma.sync kernel (blocks of 64 / g tokens); the key range is split over
  * CTAs and merged by log-sum-exp.  Other formats run as decode launches of at
  * most max_seqs rows, each row reading its own prefix.  Rows may come in any
  * order; the call uploads a small plan (rows sorted by sequence and position)
