@@ -629,23 +629,28 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
         xs[2 * m] = __uint_as_float(pr << 16);
         xs[2 * m + 1] = __uint_as_float(pr & 0xFFFF0000u);
       }
-      uint32_t word = 0, ties = 0;
+      uint32_t word = 0;
+      bool any_tie = false;   // which elements tie is found again on the rare exact path
 #pragma unroll
       for (int l = 0; l < N; ++l) {
         bool tie;
         const int q = ASYM ? quant_code_nb(__fsub_rn(xs[l], zq[l]) * iv[l], 0, Q, tie)
                            : quant_code_nb(xs[l] * iv[l], -Q, Q, tie);
-        ties |= uint32_t(tie) << l;
+        any_tie |= tie;
         word |= (uint32_t(q) & MASK) << (BITS * word_field(l, N));
       }
-      if (__any_sync(0xffffffffu, ties != 0)) {
-        for (int l = 0; l < N; ++l)
-          if (ties & (1u << l)) {
+      if (__any_sync(0xffffffffu, any_tie)) {
+        for (int l = 0; l < N; ++l) {
+          bool tie;
+          (void)(ASYM ? quant_code_nb(__fsub_rn(xs[l], zq[l]) * iv[l], 0, Q, tie)
+                      : quant_code_nb(xs[l] * iv[l], -Q, Q, tie));
+          if (tie) {
             const int c = key_channel(kw * N + l);
             const int q = ASYM ? quant_asym_exact(xs[l], ksc[c], kzp[c], Q) : quant_sym_exact(xs[l], ksc[c], Q);
             const int sh = BITS * word_field(l, N);
             word = (word & ~(MASK << sh)) | ((uint32_t(q) & MASK) << sh);
           }
+        }
       }
       const int sub = rowi >> 4, rr = rowi & 15;
       *reinterpret_cast<uint32_t*>(chunk_of(sub >> lg_spp) + (sub & spp_mask) * g.sub_bytes +
@@ -679,7 +684,8 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
         const int gi = ((BITS == 2 ? 32 : BITS == 4 ? 16 : 8) * w) >> lg_gv;
         float xs[N];
         int tk[N / 2];
-        uint32_t word = 0, ties = 0;
+        uint32_t word = 0;
+        bool any_tie = false;   // which elements tie is found again on the rare exact path
 #pragma unroll
         for (int x = 0; x < N / 2; ++x) {
           int i, reg;
@@ -697,18 +703,22 @@ __global__ void __launch_bounds__(kFlushThreads) flush_group_kernel(const Geo g,
             bool tie;
             const int q = ASYM ? quant_code_nb(__fsub_rn(xs[l], vzp[m]) * vinv[m], 0, Q, tie)
                                : quant_code_nb(xs[l] * vinv[m], -Q, Q, tie);
-            ties |= uint32_t(tie) << l;
+            any_tie |= tie;
             word |= (uint32_t(q) & MASK) << (BITS * l);
           }
         }
-        if (__any_sync(0xffffffffu, ties != 0)) {
-          for (int l = 0; l < N; ++l)
-            if (ties & (1u << l)) {
-              const int t = tk[l % (N / 2)] + l / (N / 2);
-              const int m = t * g.nvg + gi;
+        if (__any_sync(0xffffffffu, any_tie)) {
+          for (int l = 0; l < N; ++l) {
+            const int t = tk[l % (N / 2)] + l / (N / 2);
+            const int m = t * g.nvg + gi;
+            bool tie;
+            (void)(ASYM ? quant_code_nb(__fsub_rn(xs[l], vzp[m]) * vinv[m], 0, Q, tie)
+                        : quant_code_nb(xs[l] * vinv[m], -Q, Q, tie));
+            if (tie) {
               const int q = ASYM ? quant_asym_exact(xs[l], vsc[m], vzp[m], Q) : quant_sym_exact(xs[l], vsc[m], Q);
               word = (word & ~(MASK << (BITS * l))) | ((uint32_t(q) & MASK) << (BITS * l));
             }
+          }
         }
         wd[j] = word;
       }
