@@ -959,4 +959,29 @@ cudaError_t launch_residual(const Geo& g, const DevState& d, const PlanView& p, 
   return cudaGetLastError();
 }
 
+// A step's inputs from page-locked host memory the device maps: every thread
+// loads 16-byte pieces over the bus, all in flight at once, and stores them
+// into the library's device staging (a copy engine pays its per-copy latency
+// instead).  Up to three segments per launch; sizes are multiples of 16 bytes.
+namespace {
+__global__ void __launch_bounds__(256) pull_kernel(const __grid_constant__ PullArgs a) {
+  for (int sgi = 0; sgi < a.n; ++sgi) {
+    const uint4* __restrict__ src = static_cast<const uint4*>(a.src[sgi]);
+    uint4* __restrict__ dst = static_cast<uint4*>(a.dst[sgi]);
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < a.n16[sgi];
+         i += int64_t(gridDim.x) * blockDim.x)
+      dst[i] = src[i];
+  }
+}
+}  // namespace
+
+cudaError_t launch_pull(const PullArgs& a, cudaStream_t s, int* launches) {
+  int64_t most = 0;
+  for (int i = 0; i < a.n; ++i) most = std::max(most, a.n16[i]);
+  if (most == 0) return cudaSuccess;
+  pull_kernel<<<unsigned(std::min<int64_t>((most + 255) / 256, 1184)), 256, 0, s>>>(a);
+  ++*launches;
+  return cudaGetLastError();
+}
+
 }  // namespace kvq

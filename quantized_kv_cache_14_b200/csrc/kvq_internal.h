@@ -164,6 +164,15 @@ size_t decode_partials_bytes(const Geo& g, int B, int grid);
 // Launches the attention kernel and the merge; `between` (optional) is
 // recorded between them.
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s, cudaEvent_t between, int* launches);
+// Up to three copies from mapped page-locked host memory (device addresses)
+// into device memory, run by one kernel; n16 in 16-byte units.
+struct PullArgs {
+  const void* src[3];
+  void* dst[3];
+  int64_t n16[3];
+  int n;
+};
+cudaError_t launch_pull(const PullArgs& a, cudaStream_t s, int* launches);
 constexpr int kMaxDecodeGrid = 1024;
 
 // HBM read-floor measurement kernels (kvq_floor.cu).  mode 0: bulk copies of

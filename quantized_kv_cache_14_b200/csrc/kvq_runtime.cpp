@@ -696,7 +696,39 @@ kvq_status kvq_step_host(kvq_handle h, const void* k_host, const void* v_host, c
   const uint8_t* hq = static_cast<const uint8_t*>(q_host);
   // a caller whose k, v and q are back to back in host memory gets one copy
   const bool packed = n > 0 && batch > 0 && hv == hk + kv_bytes && hq == hv + kv_bytes;
-  if (packed) {
+  // The device address of page-locked host memory the device maps, else null
+  // (an unregistered pointer is not an error here).
+  auto mapped = [](const void* ptr) -> const void* {
+    cudaPointerAttributes pa{};
+    if (ptr && cudaPointerGetAttributes(&pa, ptr) == cudaSuccess && pa.type == cudaMemoryTypeHost &&
+        pa.devicePointer != nullptr && aligned16(pa.devicePointer))
+      return pa.devicePointer;
+    (void)cudaGetLastError();
+    return nullptr;
+  };
+  const void* mk = n > 0 ? mapped(k_host) : nullptr;
+  const void* mv = n > 0 && !packed ? mapped(v_host) : nullptr;
+  const void* mq = batch > 0 && !packed ? mapped(q_host) : nullptr;
+  if (packed ? mk != nullptr : ((n == 0 || (mk && mv)) && (batch == 0 || mq))) {
+    // mapped inputs: one pull kernel reads them over the bus into the staging
+    kvq::PullArgs pa{};
+    auto seg = [&](const void* src, void* dst, size_t bytes) {
+      pa.src[pa.n] = src;
+      pa.dst[pa.n] = dst;
+      pa.n16[pa.n] = int64_t(bytes / 16);
+      ++pa.n;
+    };
+    if (packed) {
+      seg(mk, d_k, 2 * kv_bytes + q_bytes);
+    } else {
+      if (n > 0) {
+        seg(mk, d_k, kv_bytes);
+        seg(mv, d_v, kv_bytes);
+      }
+      if (batch > 0) seg(mq, d_q, q_bytes);
+    }
+    KVQ_CUDA(kvq::launch_pull(pa, stream, &h->launches));
+  } else if (packed) {
     KVQ_CUDA(cudaMemcpyAsync(d_k, hk, 2 * kv_bytes + q_bytes, cudaMemcpyHostToDevice, stream));
   } else {
     if (n > 0) {
@@ -712,16 +744,9 @@ kvq_status kvq_step_host(kvq_handle h, const void* k_host, const void* v_host, c
   if (batch == 0) return KVQ_OK;
   // page-locked output the device can write (mapped pinned memory) takes the
   // attention output straight from the decode kernel; else one D2H copy
-  cudaPointerAttributes pa{};
-  float* d_out = h->d_out;
-  bool direct = false;
-  if (cudaPointerGetAttributes(&pa, out_host) == cudaSuccess && pa.type == cudaMemoryTypeHost &&
-      pa.devicePointer != nullptr && aligned16(pa.devicePointer)) {
-    d_out = static_cast<float*>(pa.devicePointer);
-    direct = true;
-  } else {
-    (void)cudaGetLastError();   // an unregistered host pointer is not an error here
-  }
+  const void* mo = mapped(out_host);
+  float* d_out = mo ? static_cast<float*>(const_cast<void*>(mo)) : h->d_out;
+  const bool direct = mo != nullptr;
   st = launch_handle_decode(h, d_q, nullptr, 0, h->d_len, nullptr, batch, d_out, stream);
   if (st != KVQ_OK) return st;
   if (!direct) KVQ_CUDA(cudaMemcpyAsync(out_host, h->d_out, q_bytes * 2, cudaMemcpyDeviceToHost, stream));
