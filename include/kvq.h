@@ -223,15 +223,17 @@ kvq_status kvq_decode_attn(kvq_handle h, const void* q_bf16,
  *      attends over every stored token of sequence i (kvq_decode_attn with the
  *      library's own lengths, rows 0..batch-1 = sequences 0..batch-1);
  *   3. the output comes back to out_host (host fp32 [batch][h_q][d_h]).
- * out_host holds the result once the stream reaches that point.  Page-locked
- * host buffers let the copies run asynchronously; pageable ones work with the
- * copy semantics CUDA gives them.  When k_host, v_host and q_host lie back to
- * back in host memory (v right after the n K rows, q right after the n V rows)
- * the step issues one host-to-device copy instead of three; when out_host is
+ * out_host holds the result once the stream reaches that point.  Inputs in
  * page-locked memory the device can address (cudaPointerGetAttributes gives a
- * device pointer), the decode kernel writes the output there directly instead
- * of a device buffer plus a device-to-host copy.  n = 0 skips the append,
- * batch = 0 the decode.
+ * device pointer) come in through one library kernel that reads them over the
+ * bus with every load in flight at once (faster than copy-engine copies at
+ * these sizes); other inputs are copied (page-locked ones asynchronously,
+ * pageable ones with the copy semantics CUDA gives them).  When k_host, v_host
+ * and q_host lie back to back in host memory (v right after the n K rows, q
+ * right after the n V rows) that is one transfer instead of three.  When
+ * out_host is page-locked memory the device can address, the decode writes the
+ * output there directly instead of a device buffer plus a device-to-host copy.
+ * n = 0 skips the append, batch = 0 the decode.
  * The device buffers grow on demand (a device synchronize, then a reallocation)
  * and live until kvq_destroy; the host buffers stay the caller's and must
  * stay valid until the stream has reached the end of the step.
