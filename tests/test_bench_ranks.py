@@ -51,7 +51,7 @@ def test_algorithmic_bytes_of_the_int4_workload():
     # no window tokens, plus q (32 x 128 bf16) and out (fp32), plus 512 table entries
     b = bench.decode_bytes(w, [8192])
     assert b == 8192 * 8 * 136 + 32 * 128 * 6 + 512 * 4
-    # the first config's 16 x 8192 quantized tokens are the survey's 142,606,336 bytes
+    # 16 sequences of 8192 quantized tokens: 142,606,336 bytes of codes and scales
     assert 16 * 8192 * 8 * 136 == 142_606_336
     # 63 window tokens are bf16 rows of K and V
     assert bench.decode_bytes(w, [8192 + 63]) - b == 63 * 8 * 2 * 128 * 2
