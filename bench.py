@@ -21,8 +21,9 @@ output written into page-locked host memory) inside the timed region,
 synchronised every step.  With N > 1 every rank runs its own replica
 (sequences shard across GPUs; no collective is on the data path; the only
 collectives are the barrier and the max-over-ranks timing).  `--impl
-reference` times the CPU oracle (test infrastructure) on a bounded sample of
-the same workload.
+reference` times the CPU oracle (test infrastructure) on the same K steps
+after W warm-up steps, each decoding a sample of the sequences sized so that
+the run stays within a few minutes.
 
 Beside the headline (skipped with --no-workloads): `workloads` gives the same
 measurement for the other four workloads with min(K, 20) steps each.  On one
@@ -52,6 +53,7 @@ from quantized_kv_cache_14_b200.workloads import Draws, workload  # noqa: E402
 
 D = 128
 L2_FLUSH_BYTES = 256 << 20
+REF_BUDGET_S = 90.0   # oracle decode seconds of the reference arm's warm-up and timed steps
 
 
 # ---------------------------------------------------------------------------
@@ -833,13 +835,26 @@ def oracle_cache_for(w, dr, growth):
     return oc
 
 
-def run_oracle_sample(w, steps, warmup, rows, threads):
+def run_oracle_sample(w, steps, warmup, rows, threads, budget_s=None):
     """Oracle steps (append one token per sequence + decode of `rows`
-    sequences); returns (decode GB/s, seconds timed, bytes)."""
+    sequences); returns (decode GB/s, seconds timed, bytes, final lengths,
+    rows decoded per step).  With `budget_s`, one untimed decode of all `rows`
+    on the prefilled cache first measures the cost of a wave of (row, kv
+    head) items on `threads` threads, and the rows per step drop (to 1 at
+    least) until warmup + steps decodes fit the budget."""
     dr = Draws(w, steps=steps + warmup)
     oc = oracle_cache_for(w, dr, steps + warmup + 2)
     lens = list(dr.lengths)
     ids = np.arange(w.batch, dtype=np.int32)
+    if budget_s is not None:
+        sub = np.arange(rows, dtype=np.int32)
+        q0 = np.zeros((rows, w.h_q, D), np.uint16)   # the decode's cost does not depend on q
+        t0 = time.perf_counter()
+        oc.decode(q0, [lens[i] for i in sub], seq_ids=sub, nthreads=threads)
+        waves = -(-rows * w.h_kv // threads)
+        t_wave = (time.perf_counter() - t0) / waves
+        while rows > 1 and (steps + warmup) * t_wave * -(-rows * w.h_kv // threads) > budget_s:
+            rows -= 1
     t_dec, nbytes = 0.0, 0
     for s in range(warmup + steps):
         k, v, q = dr.step()
@@ -853,7 +868,7 @@ def run_oracle_sample(w, steps, warmup, rows, threads):
             t_dec += dt
             nbytes += decode_bytes(w, [lens[i] for i in sub])
     oc.close()
-    return nbytes / t_dec / 1e9, t_dec, nbytes, lens
+    return nbytes / t_dec / 1e9, t_dec, nbytes, lens, rows
 
 
 def workload_config(w, lens):
@@ -923,17 +938,20 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        steps = min(args.steps, 5)
-        gbs, secs, nbytes, lens = run_oracle_sample(w, steps, min(args.warmup, 1), rows, threads)
+        # the same K timed steps after W warm-up steps as the CUDA arm, each
+        # step a sample of the workload: rows per step sized so that the
+        # oracle's decodes take about REF_BUDGET_S in all
+        steps, warm = args.steps, args.warmup
+        gbs, secs, nbytes, lens, rows = run_oracle_sample(w, steps, warm, rows, threads, budget_s=REF_BUDGET_S)
         line = {
             "metric": "decode-attn KV GB/s", "value": gbs, "unit": "GB/s", "impl": "reference",
-            "n_gpus": 0, "steps": steps, "warmup": min(args.warmup, 1),
+            "n_gpus": 0, "steps": steps, "warmup": warm,
             "ms_per_step": secs / steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(w, lens),
             "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
-                             "sample": f"{steps} steps: append 1 token to each of {w.batch} sequences, "
-                                       f"decode {rows} of them, fp64 C++ oracle"},
+                             "sample": f"{steps} steps after {warm} warm-up: append 1 token to each of "
+                                       f"{w.batch} sequences, decode {rows} of them, fp64 C++ oracle"},
             "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         }
         print(json.dumps(line))
@@ -954,7 +972,7 @@ def main():
     cpu = None
     if ws == 1 and not args.no_cpu_baseline:
         n_cpu = 24   # about 10 s of oracle decode on the machine's host cores
-        gbs, secs, _, _ = run_oracle_sample(w, n_cpu, 0, rows, threads)
+        gbs, secs, _, _, _ = run_oracle_sample(w, n_cpu, 0, rows, threads)
         cpu = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
                "sample": f"{n_cpu} steps of {rows}/{w.batch} sequences (append + fp64 decode), "
                          f"{secs:.1f} s timed"}
