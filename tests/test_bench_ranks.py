@@ -1,6 +1,7 @@
-"""The N>1 path of bench.py on CPU: two gloo ranks, each a replica, combine their
-timings by max and their work by sum (the only collectives), and the
-algorithmic byte counts match the format arithmetic."""
+"""bench.py on CPU: the N>1 path (two gloo ranks, each a replica, combine
+their timings by max and their work by sum, the only collectives), the
+algorithmic byte counts against the format arithmetic, and the oracle arm's
+JSON line."""
 import os
 import socket
 
@@ -66,3 +67,22 @@ def test_bulk_append_bytes_of_the_int4_workload():
     # token-head), the 17 window tokens written as bf16 K and V rows
     row = 8 * 128 * 2
     assert bench.bulk_append_bytes(w, [8192 + 17]) == 2 * row * (8192 + 17) + 8192 * 8 * 136 + 2 * row * 17
+
+
+def test_reference_arm_runs_the_requested_steps():
+    """The oracle arm times the same K steps after W warm-up steps as the CUDA
+    arm (tiny workload, CPU only) and prints one JSON line of the contract."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "1", "--steps", "4",
+                        "--warmup", "3"], cwd=root, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["steps"] == 4 and d["warmup"] == 3
+    assert d["value"] > 0 and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert d["metric"] == "decode-attn KV GB/s" and d["higher_is_better"] is True
