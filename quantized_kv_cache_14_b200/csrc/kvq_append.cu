@@ -911,15 +911,11 @@ cudaError_t launch_flush(const Geo& g, const DevState& d, const PlanView& p, con
     const int extra = int(std::min<int64_t>((work + per_col - 1) / per_col, 256));
     return by_format(g, [&](auto B, auto A) {
       auto kern = flush_group_kernel<decltype(B)::value, decltype(A)::value>;
-      static thread_local size_t limit_set[32] = {};
       int dev = 0;
       cudaError_t e = cudaGetDevice(&dev);
       if (e != cudaSuccess) return e;
-      if (dev >= 32 || smem > limit_set[dev]) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        if (e != cudaSuccess) return e;
-        if (dev < 32) limit_set[dev] = smem;
-      }
+      e = raise_smem_limit(dev, reinterpret_cast<const void*>(kern), smem);
+      if (e != cudaSuccess) return e;
       kern<<<dim3(p.n_flush + extra, g.h_kv), kFlushThreads, smem, s>>>(g, d, p, k, v, fuse_rows ? 1 : 0);
       ++*launches;
       return cudaGetLastError();
@@ -932,16 +928,11 @@ cudaError_t launch_flush(const Geo& g, const DevState& d, const PlanView& p, con
   const int extra = int(std::min<int64_t>((work + per_col - 1) / per_col, 64));
   return by_format(g, [&](auto B, auto A) {
     auto kern = flush_kernel<decltype(B)::value, decltype(A)::value>;
-    // the shared-memory limit only grows: set it once per kernel, device and size
-    static thread_local size_t limit_set[32] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev >= 32 || smem > limit_set[dev]) {
-      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-      if (e != cudaSuccess) return e;
-      if (dev < 32) limit_set[dev] = smem;
-    }
+    e = raise_smem_limit(dev, reinterpret_cast<const void*>(kern), smem);
+    if (e != cudaSuccess) return e;
     kern<<<dim3(p.n_flush + extra, g.h_kv, g.R / 16), kFlushThreads, smem, s>>>(g, d, p, k, v,
                                                                               fuse_rows ? 1 : 0);
     ++*launches;

@@ -2227,10 +2227,11 @@ size_t decode_partials_bytes(const Geo& g, int B, int grid) {
 }
 
 // The dynamic shared-memory limit is an attribute of the kernel on a device,
-// shared by every handle and every allocation-free call.  Plans for different
-// batch sizes need different amounts, so the limit only ever rises: lowering
-// it for a small plan would make a live plan's larger launches fail.
-static cudaError_t raise_smem_limit(int dev, const void* kern, size_t smem) {
+// shared by every handle, thread and allocation-free call.  Plans for
+// different batch sizes or formats need different amounts, so the limit only
+// ever rises: lowering it for a small plan would make a live plan's larger
+// launches fail.  One record for every kernel of the library, under a mutex.
+cudaError_t raise_smem_limit(int dev, const void* kern, size_t smem) {
   struct Entry {
     int dev;
     const void* kern;

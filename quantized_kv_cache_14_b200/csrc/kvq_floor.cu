@@ -169,7 +169,10 @@ cudaError_t launch_floor(const void* base, const int64_t* offsets, int64_t n_chu
   a.stage_bytes = int((int64_t(per_unit) * chunk_bytes + 127) / 128 * 128);
   a.sink = sink;
   const size_t smem = floor_smem_bytes(chunk_bytes, per_unit, stages);
-  cudaError_t e = cudaFuncSetAttribute(floor_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = raise_smem_limit(dev, reinterpret_cast<const void*>(&floor_bulk_kernel), smem);
   if (e != cudaSuccess) return e;
   floor_bulk_kernel<<<ctas, kFloorWarps * 32, smem, s>>>(a);
   return cudaGetLastError();

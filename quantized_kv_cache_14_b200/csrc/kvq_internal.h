@@ -155,6 +155,10 @@ cudaError_t launch_quant_token(const Geo& g, const DevState& d, const PlanView& 
                                const uint16_t* k, const uint16_t* v, cudaStream_t s,
                                int* launches);
 
+// Raises kernel `kern`'s dynamic shared-memory limit on device `dev` to at
+// least `smem` bytes; never lowers it (kvq_decode.cu).
+cudaError_t raise_smem_limit(int dev, const void* kern, size_t smem);
+
 const void* decode_kernel_ptr(const Geo& g);
 // Sizes the pipeline for batches up to max_B on the current device, sets the
 // kernel's shared-memory limit and finds its residency.

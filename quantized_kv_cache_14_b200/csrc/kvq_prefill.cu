@@ -608,15 +608,11 @@ template <int BITS, int ASYM>
 cudaError_t launch_prefill_t(const PrefillArgs& a, int64_t n_rows, cudaStream_t s, int* launches) {
   const int smem = pf_smem(a.stage_bytes).total;
   auto kern = prefill_kernel<BITS, ASYM>;
-  static thread_local int limit_set[32] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 32 || smem > limit_set[dev]) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    if (dev < 32) limit_set[dev] = smem;
-  }
+  e = raise_smem_limit(dev, reinterpret_cast<const void*>(kern), size_t(smem));
+  if (e != cudaSuccess) return e;
   kern<<<a.n_tasks, kPfThreads, smem, s>>>(a);
   ++*launches;
   e = cudaGetLastError();
@@ -658,9 +654,11 @@ size_t prefill_smem_bytes(int stage_bytes) { return size_t(pf_smem(stage_bytes).
 
 int prefill_ctas_per_sm(const Geo& g, int stage_bytes) {
   const int smem = pf_smem(stage_bytes).total;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 1;
   auto occ = [&](auto kern) {
     int n = 0;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return 1;
+    if (raise_smem_limit(dev, reinterpret_cast<const void*>(kern), size_t(smem)) != cudaSuccess) return 1;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kPfThreads, smem) != cudaSuccess) return 1;
     return n > 0 ? n : 1;
   };

@@ -639,15 +639,11 @@ int prefill_tc_ctas_per_sm() {
 
 cudaError_t launch_prefill_tc(const PrefillArgs& a, int64_t n_rows, cudaStream_t s, int* launches) {
   const int smem = int(prefill_tc_smem_bytes());
-  static thread_local int limit_set[32] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 32 || smem > limit_set[dev]) {
-    e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    if (dev < 32) limit_set[dev] = smem;
-  }
+  e = raise_smem_limit(dev, reinterpret_cast<const void*>(&prefill_tc_kernel), size_t(smem));
+  if (e != cudaSuccess) return e;
   prefill_tc_kernel<<<a.n_tasks, kTcThreads, smem, s>>>(a);
   ++*launches;
   e = cudaGetLastError();

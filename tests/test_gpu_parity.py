@@ -331,6 +331,35 @@ def test_prefill_kernel_blocks(name, h_q, h_kv):
     p.close()
 
 
+def test_prefill_shared_memory_limit_only_rises():
+    """Two caches whose prefill runs one kernel instance (4-bit symmetric
+    keys per channel, the mma.sync kernel) with different stage sizes: the
+    smaller one's first call, which also sizes its residency, must not lower
+    the kernel's shared-memory limit under the larger one's next launch."""
+    rng = np.random.default_rng(71)
+    # 16-token key groups stage 4 pages of 2336 B, 64-token groups 4 of 2176 B
+    pairs = [Pair(FMTS["int4_chan16"], 8, 2, max_seqs=1, num_blocks=200, mbps=64, seed=7),
+             Pair(FMTS["int4_chan64"], 4, 2, max_seqs=1, num_blocks=200, mbps=64, seed=8)]
+    n_pre, n_chunk = 300, 24
+    for p in pairs:
+        ids = np.zeros(n_pre + n_chunk, np.int32)
+        p.append(outlier_keys(rng, ids.size, p.h_kv), random_bf16(rng, (ids.size, p.h_kv, D)), ids)
+    pos = np.arange(n_pre, n_pre + n_chunk, dtype=np.int32)
+    cids = np.zeros(n_chunk, np.int32)
+    for which in (0, 1, 0):
+        p = pairs[which]
+        q = random_bf16(rng, (n_chunk, p.h_q, D))
+        out = torch.full((n_chunk, p.h_q, D), float("nan"), dtype=torch.float32, device="cuda")
+        p.gpu.prefill_attn(bits_to_cuda_bf16(q), cids, pos, out)
+        torch.cuda.synchronize()
+        assert p.gpu.sync_status() == 0
+        want = p.orc.decode(q, (pos + 1).tolist(), seq_ids=cids)
+        err = float(np.max(np.abs(out.cpu().numpy().astype(np.float64) - want)))
+        assert err <= ATOL, f"cache {which}: max abs error {err}"
+    for p in pairs:
+        p.close()
+
+
 @pytest.mark.parametrize("name", ["int4_chan64", "int2_asym_chan32"])
 def test_prefill_repeated_split_calls(name):
     """Repeated split prefill calls on one cache give bit-identical outputs
