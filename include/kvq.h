@@ -399,8 +399,9 @@ kvq_status kvq_set_decode_event(kvq_handle h, void* event);
  * giving both sizes when batch * h_kv needs more scratch than the array holds;
  * KVQ_ERR_UNSUPPORTED for the FP8 format (its per-head scales live in a handle).
  * The partials take (batch * h_kv + grid) * 4 * G * 520 bytes, G = h_q / h_kv
- * and grid = resident decode CTAs (3 per SM, 444 on 148 SMs): with G = 4 that
- * allows about 1,500 (row, kv head) pairs. */
+ * and grid = the resident decode CTAs of the format's kernel (2 or 3 per SM:
+ * 296 or 444 on 148 SMs): with G = 4 that allows about 1,500 to 1,700
+ * (row, kv head) pairs. */
 kvq_status kvq_decode_attn_noalloc(const kvq_config* cfg, const void* pool, const void* k_window,
                                    const void* v_window, const int32_t* block_table,
                                    int32_t bt_stride, const int32_t* stored_lens,
