@@ -97,7 +97,11 @@ enum { KVQ_AXIS_TOKEN = 0, KVQ_AXIS_CHANNEL = 1 };
  *   page        P tokens per block: a power of two, at least 16.
  *   h_q, h_kv   query and key/value heads; h_q / h_kv must be 1, 2 or 4.
  *   d_h         head dimension: 128.
- *   max_seqs, num_blocks, max_blocks_per_seq   capacity.
+ *   max_seqs, num_blocks, max_blocks_per_seq   capacity.  The decode
+ *               kernels keep 16 bytes of work-list state per batch row in
+ *               shared memory beside their stages, so max_seqs is bounded by
+ *               the device's per-CTA shared memory: about 10,000 rows on a
+ *               B200 (kvq_create returns KVQ_ERR_UNSUPPORTED beyond it).
  *   seed        seeds the free list: a Fisher-Yates shuffle of
  *               [0, num_blocks) driven by splitmix64(seed); blocks are taken
  *               from its front and freed blocks return to its back.
@@ -171,7 +175,9 @@ typedef struct kvq_stats_t {
 /* Validates `cfg`, allocates the pool, residual windows, block table and
  * workspace on cfg->device, zero-fills them, and builds the free list.
  * Ownership: the handle owns every allocation until kvq_destroy().
- * Errors: KVQ_ERR_INVALID_ARG / KVQ_ERR_UNSUPPORTED (config), KVQ_ERR_CUDA. */
+ * Errors: KVQ_ERR_INVALID_ARG / KVQ_ERR_UNSUPPORTED (config, or a decode plan
+ * for max_seqs rows that does not fit the device's shared memory),
+ * KVQ_ERR_CUDA. */
 kvq_status kvq_create(const kvq_config* cfg, kvq_handle* out);
 
 /* Frees everything the handle owns (synchronizes the device first). */
