@@ -210,6 +210,27 @@ def test_step_host_equals_device_calls(name):
     a.close()
 
 
+@pytest.mark.parametrize("name", ["int4_chan64", "int8_tok_p16"])
+def test_large_batch(name):
+    """A thousand sequences of 0 to 140 tokens in one bulk append, then one
+    decode of every row and one of 700 shuffled rows with shorter prefixes.
+    At this batch the per-row work list no longer fits beside two
+    warp-specialised CTAs per SM, so the generic kernel runs, and its prefix
+    scan over the rows takes several rows per thread."""
+    rng = np.random.default_rng(97)
+    h_q, h_kv, S = 8, 2, 1000
+    p = Pair(FMTS[name], h_q, h_kv, max_seqs=S, num_blocks=S * 9, mbps=9, seed=11)
+    lens = [int(x) for x in rng.integers(0, 141, size=S)]
+    ids = rng.permutation(np.repeat(np.arange(S, dtype=np.int32), lens)).astype(np.int32)
+    p.append(outlier_keys(rng, ids.size, h_kv), random_bf16(rng, (ids.size, h_kv, D)), ids)
+    p.check_state()
+    p.check_decode(random_bf16(rng, (S, h_q, D)), lens)
+    rows = rng.permutation(S)[:700].astype(np.int32)
+    attend = [int(rng.integers(0, lens[r] + 1)) for r in rows]
+    p.check_decode(random_bf16(rng, (rows.size, h_q, D)), attend, seq_ids=rows)
+    p.close()
+
+
 @pytest.mark.parametrize("name", ["int4_chan64", "int8_tok_p16", "int2_asym_chan32", "bf16_control_p16", "fp8_p16"])
 def test_split_k_merge_is_invariant_to_grid(name):
     rng = np.random.default_rng(3)
