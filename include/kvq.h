@@ -101,7 +101,12 @@ enum { KVQ_AXIS_TOKEN = 0, KVQ_AXIS_CHANNEL = 1 };
  *               kernels keep 16 bytes of work-list state per batch row in
  *               shared memory beside their stages, so max_seqs is bounded by
  *               the device's per-CTA shared memory: about 10,000 rows on a
- *               B200 (kvq_create returns KVQ_ERR_UNSUPPORTED beyond it).
+ *               B200 (kvq_create returns KVQ_ERR_UNSUPPORTED beyond it).  The
+ *               warp-specialised decode kernels of the INT4 / INT2 KIVI-style
+ *               and INT8 per-token formats need two CTAs per SM, which holds
+ *               up to about 420 / 1,000 / 700 rows of max_seqs; a handle
+ *               planned for more rows decodes every batch with the generic
+ *               kernel (same results, about 15% slower on the INT4 format).
  *   seed        seeds the free list: a Fisher-Yates shuffle of
  *               [0, num_blocks) driven by splitmix64(seed); blocks are taken
  *               from its front and freed blocks return to its back.
