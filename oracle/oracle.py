@@ -35,9 +35,12 @@ class OracleConfig(ctypes.Structure):
 
 
 def lib():
+    """Loads liboracle.so (built on demand).  KVQ_ORACLE_LIB, when set, names
+    another build of the oracle's source to load instead: the pin suites run
+    against copies with a planted mistake this way (tests/test_oracle_mutants.py)."""
     global _LIB
     if _LIB is None:
-        path = _build.build()
+        path = os.environ.get("KVQ_ORACLE_LIB") or _build.build()
         L = ctypes.CDLL(path)
         P = ctypes.c_void_p
         L.orc_f32_to_f16.restype = ctypes.c_uint16

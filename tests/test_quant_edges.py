@@ -24,6 +24,8 @@ def test_edge_group_hits_its_branch(bits, asym, fp32, kind):
         s, z, q = O.quant_asym(x, bits, bool(fp32))
     else:
         s, q = O.quant_sym(x, bits, bool(fp32))
+    # every code lies in the quantizer's range: [-Q, Q], or [0, 2^b - 1] with a zero-point
+    assert q.min() >= (0 if asym else -Q) and q.max() <= (Qa if asym else Q)
     if kind == "zero":
         assert s == 0.0 and not q.any()
     elif kind == "constant":
@@ -43,6 +45,9 @@ def test_edge_group_hits_its_branch(bits, asym, fp32, kind):
             assert s == 65504.0
             lim = Qa if asym else Q
             assert np.any(q == lim) and np.max(np.abs(x - (z if asym else 0.0))) / s > lim   # the clip fired
+            if not asym:   # and at the negative end: elements below -(Q + 1/2) s take -Q exactly
+                below = x / s < -(Q + 0.5)
+                assert below.any() and np.all(q[below] == -Q)
     elif kind == "underflow":
         if not fp32:
             assert s == 0.0 and not q.any()
