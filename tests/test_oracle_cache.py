@@ -249,6 +249,33 @@ def test_freed_blocks_are_reused_after_the_untouched_ones():
     c.close()
 
 
+def test_reused_block_reads_zero_in_its_unused_slots():
+    """The layout contract zero-fills the pool, so a token slot that no append
+    has written reads as zero codes and zero scales.  A block freed with data
+    in all 16 slots and reused by a sequence that writes only 5 of them must
+    hold zeros in the other 11 (keys, values and metadata of those slots)."""
+    c = make("int8_tok_p16", num_blocks=1, seed=1, max_seqs=2)
+    rng = np.random.default_rng(8)
+    k = random_bf16(rng, (16, 2, D), 3.0); v = random_bf16(rng, (16, 2, D))
+    assert c.append(k, v, np.zeros(16, np.int32)) == 0     # the one block, every slot written
+    assert c.free_seq(0) == 0
+    assert c.append(k[:5], v[:5], np.ones(5, np.int32)) == 0   # the same block again, 5 slots
+    assert c.block_table(1).tolist() == [0]
+    pool, lay = c.pool(), c.layout
+    for h in range(2):
+        chunk = pool[h * lay["chunk_bytes"]:(h + 1) * lay["chunk_bytes"]]
+        for tok in range(5, 16):
+            for ch in range(D):
+                for sec, kind in ((0, "k"), (lay["off_V"], "v")):
+                    byte, _ = c.code_loc(kind, tok, ch)
+                    assert chunk[sec + byte] == 0, (h, kind, tok, ch)
+        # metadata of the unwritten slots: one key and one value scale per token (fp16)
+        for tok in range(5, 16):
+            assert not chunk[lay["off_Vm"] + 2 * tok:lay["off_Vm"] + 2 * tok + 2].any()
+            assert not chunk[lay["off_Km"] + 2 * tok:lay["off_Km"] + 2 * tok + 2].any()
+    c.close()
+
+
 @pytest.mark.parametrize("name", ["int8_tok_p16", "int4_chan64_p16"])
 def test_out_of_blocks_leaves_state_unchanged(name):
     c = make(name, num_blocks=5, max_seqs=2)
@@ -487,6 +514,24 @@ def test_shared_blocks_are_freed_by_their_last_holder():
             assert c.share_prefix(0, 1, 16) == 0                 # dst no longer empty
         assert c.share_prefix(*args) == code
     assert t0 != []
+    c.close()
+
+
+def test_windowed_cache_shares_whole_key_groups_only():
+    """With a BF16 window the pages hold whole key groups only (day-65 "Why
+    some systems keep a full-precision window": a group moves into the cache
+    when it fills); the newest tokens of a group still filling live in the
+    source's window, not in a block.  A prefix that is a whole number of pages
+    but not of groups is refused, with no state change; whole groups share."""
+    c = make("int4_chan64_p16", max_seqs=3, num_blocks=40)
+    k = random_bf16(np.random.default_rng(5), (150, 2, D))
+    assert c.append(k, k, np.zeros(150, np.int32)) == 0        # 2 groups in 8 blocks, 22 in the window
+    free0, t0 = c.free_count(), c.block_table(0).tolist()
+    for tokens in (16, 48, 80, 144):                           # pages, not whole groups
+        assert c.share_prefix(0, 1, tokens) == 4
+        assert c.seq_len(1) == 0 and c.block_table(1).tolist() == [] and c.free_count() == free0
+    assert c.share_prefix(0, 1, 128) == 0                      # two whole groups
+    assert c.block_table(1).tolist() == t0 and c.seq_len(1) == 128
     c.close()
 
 
