@@ -276,6 +276,25 @@ def test_reused_block_reads_zero_in_its_unused_slots():
     c.close()
 
 
+def test_admission_counts_only_the_blocks_a_call_adds():
+    """Blocks are allocated on demand (day-65 "How this connects to paging and
+    prefix caching"): an append needs only the blocks its new tokens open, so
+    a pool with exactly that many free blocks admits it, and one more token
+    than fits is refused with nothing changed.  Sequence ids run over
+    [0, max_seqs): max_seqs itself is refused."""
+    c = make("int8_tok_p16", num_blocks=3, max_seqs=2)
+    rng = np.random.default_rng(9)
+    k = random_bf16(rng, (49, 2, D)); v = random_bf16(rng, (49, 2, D))
+    assert c.append(k[:32], v[:32], np.zeros(32, np.int32)) == 0    # 2 blocks, 1 free
+    assert c.append(k[32:48], v[32:48], np.zeros(16, np.int32)) == 0  # fills the 3rd block exactly
+    assert c.free_count() == 0 and c.seq_len(0) == 48
+    pool = c.pool().copy()
+    assert c.append(k[48:], v[48:], np.zeros(1, np.int32)) == 2     # a 4th block: none left
+    assert c.append(k[48:], v[48:], np.full(1, 2, np.int32)) == 3   # id == max_seqs
+    assert c.seq_len(0) == 48 and c.seq_len(1) == 0 and np.array_equal(c.pool(), pool)
+    c.close()
+
+
 @pytest.mark.parametrize("name", ["int8_tok_p16", "int4_chan64_p16"])
 def test_out_of_blocks_leaves_state_unchanged(name):
     c = make(name, num_blocks=5, max_seqs=2)

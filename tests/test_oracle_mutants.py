@@ -97,6 +97,25 @@ MUTANTS = [
     ("value_lanes_transposed", "  int lane = 4 * g + t;", "  int lane = 4 * t + g;"),
     ("prefix_shared_by_page_under_a_window", "  const int32_t unit = c.residual ? c.residual : c.page;",
      "  const int32_t unit = c.page;"),
+    # admission and the remaining conversions and metadata
+    ("sequence_id_bound_off_by_one", "    if (seq_ids[i] < 0 || seq_ids[i] >= c.max_seqs) return 3;",
+     "    if (seq_ids[i] < 0 || seq_ids[i] > c.max_seqs) return 3;"),
+    ("e4m3_infinity_to_nan", "  if (exp == 0xFF) return man ? uint8_t(sign | 0x7Fu) : uint8_t(sign | 0x7Eu);",
+     "  if (exp == 0xFF) return uint8_t(sign | 0x7Fu);"),
+    ("e4m3_exponent_bias", "    return uint8_t(sign | (uint32_t(e + 7) << 3) | (uint32_t(r) & 7u));",
+     "    return uint8_t(sign | (uint32_t(e + 8) << 3) | (uint32_t(r) & 7u));"),
+    ("fp32_scales_rounded_to_fp16", "  if (scale_fp32) return s;", "  if (scale_fp32) return stored_value(s, 0);"),
+    ("value_zero_points_over_scales",
+     "    if (c.asym) put_meta(ch + L.off_Vm + (size_t(c.page) * L.nvg + idx) * L.es, z, c.scale_fp32);",
+     "    if (c.asym) put_meta(ch + L.off_Vm + idx * L.es, z, c.scale_fp32);"),
+    ("key_zero_points_over_scales",
+     "      if (c.asym) put_meta(km + (size_t(L.kslice) + off) * L.es, z, c.scale_fp32);",
+     "      if (c.asym) put_meta(km + size_t(off) * L.es, z, c.scale_fp32);"),
+    ("fail_alloc_after_off_by_one",
+     "  if (c.fail_alloc_after >= 0 && C.alloc_count + need > c.fail_alloc_after) return 2;",
+     "  if (c.fail_alloc_after >= 0 && C.alloc_count + need >= c.fail_alloc_after) return 2;"),
+    ("table_width_off_by_one", "    if (nb > c.max_blocks_per_seq) return 2;", "    if (nb >= c.max_blocks_per_seq) return 2;"),
+    ("blocks_needed_not_net", "    need += nb - blocks_for_len(c, C.len[size_t(s)]);", "    need += nb;"),
 ]
 
 
