@@ -10,7 +10,8 @@ oh-bug.com "KV Cache Quantization in Practice", KIVI paragraph).
 
 Functions with no independent pin: none -- every exported routine is pinned by
 tests/test_oracle_*.py against closed forms, the pages' worked numbers, numpy or
-brute force.
+brute force, and tests/test_oracle_mutants.py checks that those pins fail when a
+plausible mistake is planted in a copy of the oracle's source.
 """
 import ctypes
 import os
