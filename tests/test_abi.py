@@ -98,6 +98,29 @@ def test_planner_block_placement_matches_oracle(name):
     oc.close()
 
 
+def test_admission_counts_only_the_blocks_a_call_adds():
+    """The planner admits an append that needs exactly the free blocks left
+    (only the blocks its new tokens open count), refuses one more token with
+    KVQ_ERR_OOM and an id equal to max_seqs with KVQ_ERR_BAD_SEQ, both with
+    no state change, as the oracle does."""
+    cfg, d = cfg_of("int8_tok_p16", num_blocks=3, max_seqs=2)
+    h = kvq.kvq_create(cfg)
+    oc = O.OracleCache(**{k: v for k, v in d.items() if k not in ("host_only", "device")})
+    kb = np.zeros((32, 2, 128), np.uint16)
+    for n in (32, 16):
+        kvq.kvq_append(h, 0, 0, np.zeros(n, np.int32), n)
+        assert oc.append(kb[:n], kb[:n], np.zeros(n, np.int32)) == 0
+    assert kvq.kvq_stats(h)["blocks_free"] == oc.free_count() == 0
+    assert kvq.kvq_block_table_host(h, 0).tolist() == oc.block_table(0).tolist()
+    for ids, status in ((np.zeros(1, np.int32), kvq.KVQ_ERR_OOM), (np.full(1, 2, np.int32), kvq.KVQ_ERR_BAD_SEQ)):
+        with pytest.raises(kvq.KvqError) as e:
+            kvq.kvq_append(h, 0, 0, ids, 1)
+        assert e.value.status == status
+    assert kvq.kvq_seq_len(h, 0) == 48 and kvq.kvq_seq_len(h, 1) == 0
+    kvq.kvq_destroy(h)
+    oc.close()
+
+
 def test_errors_leave_state_unchanged():
     cfg, _ = cfg_of("int8_tok_p16", num_blocks=6, max_seqs=2)
     h = kvq.kvq_create(cfg)
@@ -142,6 +165,8 @@ def test_fail_alloc_after_and_table_width():
     ("page", 48, kvq.KVQ_ERR_INVALID_ARG),
     ("page", 128, kvq.KVQ_ERR_UNSUPPORTED),
     ("g_v", 48, kvq.KVQ_ERR_UNSUPPORTED),
+    ("g_v", 16, kvq.KVQ_ERR_UNSUPPORTED),      # value groups are 32, 64 or 128 channels
+    ("page", 8, kvq.KVQ_ERR_INVALID_ARG),      # a page holds at least one 16-token sub-tile
     ("num_blocks", 0, kvq.KVQ_ERR_INVALID_ARG),
     ("k_axis", 2, kvq.KVQ_ERR_INVALID_ARG),
     ("bits", 16, kvq.KVQ_ERR_INVALID_ARG),     # the BF16 control takes token-axis keys, no window
@@ -255,9 +280,14 @@ def test_share_prefix_planner_matches_oracle(name):
         assert kvq.kvq_stats(h)["blocks_free"] == oc.free_count()
     both_append(4 * unit, 3)     # blocks come back in the same order on both sides
     assert kvq.kvq_block_table_host(h, 3).tolist() == oc.block_table(3).tolist()
-    # format check and other errors, with no state change
-    for args, status in (((3, 0, unit + 1), kvq.KVQ_ERR_INVALID_ARG), ((3, 3, unit), kvq.KVQ_ERR_INVALID_ARG),
-                         ((3, 0, 99 * unit), kvq.KVQ_ERR_INVALID_ARG), ((3, 9, unit), kvq.KVQ_ERR_BAD_SEQ)):
+    # format check and other errors, with no state change; with a window only
+    # whole key groups share (a page-sized prefix is refused on both sides)
+    bad = [((3, 0, unit + 1), kvq.KVQ_ERR_INVALID_ARG), ((3, 3, unit), kvq.KVQ_ERR_INVALID_ARG),
+           ((3, 0, 99 * unit), kvq.KVQ_ERR_INVALID_ARG), ((3, 9, unit), kvq.KVQ_ERR_BAD_SEQ)]
+    if d["residual"]:
+        bad.append(((3, 0, d["page"]), kvq.KVQ_ERR_INVALID_ARG))
+        assert oc.share_prefix(0, 3, d["page"]) == 4
+    for args, status in bad:
         with pytest.raises(kvq.KvqError) as e:
             kvq.kvq_share_prefix(h, *args)
         assert e.value.status == status
