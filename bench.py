@@ -995,7 +995,10 @@ def main():
         "metric": "decode-attn KV GB/s", "value": res["kv_gbs"], "unit": "GB/s",
         "n_gpus": ws, "steps": res["K"], "warmup": args.warmup,
         "ms_per_step": res["ms_per_step"], "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        # the arithmetic: bf16 rows in, codes quantized in fp32, attention on
+        # fp16 tensor-core operands (hi + lo parts) accumulated in fp32, fp32
+        # softmax and output
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": workload_config(w, res["lens_final"]),
         "roofline": {"bound": "hbm", "achieved": res["attn_gbs"], "peak": peak, "unit": "GB/s",
                      "frac": res["attn_gbs"] / peak, "traffic": traffic,
