@@ -58,6 +58,35 @@ def test_algorithmic_bytes_of_the_int4_workload():
     assert bench.decode_bytes(w, [8192 + 63]) - b == 63 * 8 * 2 * 128 * 2
 
 
+def test_algorithmic_bytes_of_the_int8_and_int2_workloads():
+    import bench
+    from quantized_kv_cache_14_b200.workloads import workload
+    # INT8 keys and values per token, G = 128, fp16 scales: (128 + 128 codes +
+    # 2 + 2 scale bytes) per token and kv head, 16-token pages, no window
+    w = workload(2)
+    assert bench.decode_bytes(w, [4096]) == 4096 * 8 * 260 + 256 * 4 + 32 * 128 * 6
+    # INT2 with fp16 scale and zero-point per group of 32: 32 + 32 code bytes,
+    # keys 128 channels x 4 bytes per 32 tokens, values 4 groups x 4 bytes;
+    # 31 window tokens as bf16 K and V rows
+    w = workload(4)
+    assert bench.decode_bytes(w, [131072 + 31]) == (131072 * 8 * 96 + 31 * 8 * 2 * 128 * 2 + 8192 * 4
+                                                   + 32 * 128 * 6)
+
+
+def test_append_bytes_of_a_decode_step():
+    import bench
+    from quantized_kv_cache_14_b200.workloads import workload
+    w = workload(3)
+    row = 8 * 128 * 2   # one token's bf16 row over the 8 kv heads
+    # no group fills: the new K and V rows read, then written to the window
+    assert bench.append_bytes(w, [10]) == 2 * row + 2 * row
+    # the 64th token fills the key group: its rows read, the 63 earlier window
+    # rows of K and V read again, 64 tokens of codes + value scales written
+    # (8 heads x (128 code bytes + 4 scale bytes)) and the group's key scales
+    # (8 heads x 128 channels x 2 bytes)
+    assert bench.append_bytes(w, [63]) == 2 * row + 2 * row * 63 + 64 * 8 * 132 + 8 * 128 * 2
+
+
 def test_bulk_append_bytes_of_the_int4_workload():
     import bench
     from quantized_kv_cache_14_b200.workloads import workload
