@@ -35,7 +35,9 @@
  *  - Kernels check block ids, lengths and grid coverage themselves and record
  *    failures in a device error word instead of faulting; kvq_sync_status()
  *    reports and clears it.
- *  - A handle may be used from one host thread at a time.
+ *  - A handle may be used from one host thread at a time; different handles
+ *    may be used from different threads at once (each kernel's shared-memory
+ *    limit is one process-wide setting that calls only ever raise).
  */
 #ifndef KVQ_H_
 #define KVQ_H_
