@@ -116,6 +116,32 @@ def test_layout_hand_derived_locations_int2_int8():
     c.close()
 
 
+def test_layout_hand_derived_locations_fp8():
+    """FP8, one byte per element: key rows keep the key-list order with bytes
+    in natural order (list position = byte); a value lane record (4 g + t,
+    64 bytes) holds operand register x of channel tile i in bytes 2x, 2x + 1
+    of word 2 i + x / 2, low token first (a0 = channel g, tokens 2t | 2t+1;
+    a1 = channel + 8; a2 = tokens + 8; a3 = both)."""
+    c = O.OracleCache(bits=8, asym=0, k_axis=0, g_k=128, g_v=128, scale_fp32=0, residual=0, page=16, fp8=1,
+                      h_q=4, h_kv=2, d_h=D, max_seqs=1, num_blocks=4, max_blocks_per_seq=4, seed=0,
+                      fail_alloc_after=-1)
+    # keys: channels 0, 1, 8, 9, 16 are list positions 0, 1, 2, 3, 4; channel 2 is 32; rows of 128 bytes
+    for ch, byte in ((0, 0), (1, 1), (8, 2), (9, 3), (16, 4), (2, 32)):
+        assert c.code_loc("k", 0, ch) == (byte, 0)
+    assert c.code_loc("k", 3, 0) == (3 * 128, 0)
+    # values: (token, channel) -> byte of the sub-tile
+    for tok, ch, byte in ((0, 0, 0),      # a0 low token, word 0 byte 0
+                          (1, 0, 1),      # a0 high token, byte 1
+                          (0, 8, 2),      # a1 low, bytes 2-3 of word 0
+                          (8, 0, 4),      # a2 low, word 1
+                          (9, 8, 7),      # a3 high, word 1 byte 3
+                          (0, 16, 8),     # channel tile 1: word 2
+                          (2, 0, 64),     # t = 1: lane 1
+                          (0, 1, 256)):   # g = 1: lane 4
+        assert c.code_loc("v", tok, ch) == (byte, 0), (tok, ch)
+    c.close()
+
+
 # -------------------------------------------- grouping direction / round trip
 
 def _expected_dequant(name, k32, v32, R):

@@ -116,6 +116,26 @@ MUTANTS = [
      "  if (c.fail_alloc_after >= 0 && C.alloc_count + need >= c.fail_alloc_after) return 2;"),
     ("table_width_off_by_one", "    if (nb > c.max_blocks_per_seq) return 2;", "    if (nb >= c.max_blocks_per_seq) return 2;"),
     ("blocks_needed_not_net", "    need += nb - blocks_for_len(c, C.len[size_t(s)]);", "    need += nb;"),
+    # the FP8 and BF16 control layouts, the flush's value rows, the window read-back,
+    # the threaded decode, the e4m3 decode, token-axis key metadata
+    ("fp8_value_bytes_transposed", "size_t(4 * word) + size_t(2 * (reg & 1) + hi), 0};",
+     "size_t(4 * word) + size_t((reg & 1) + 2 * hi), 0};"),
+    ("bf16_control_keys_in_list_order",
+     "    return {size_t(tok / 16) * L.sub_bytes + size_t(tok % 16) * L.row_bytes + size_t(2 * ch), 0};\n  if (c.fp8)",
+     "    return {size_t(tok / 16) * L.sub_bytes + size_t(tok % 16) * L.row_bytes + size_t(2 * inv[ch]), 0};\n"
+     "  if (c.fp8)"),
+    ("flushed_value_rows_shifted",
+     "      write_value_row(C, C.table[s][size_t(pos / P)], int(pos % P), h, row.data());",
+     "      write_value_row(C, C.table[s][size_t(pos / P)], int((pos + 1) % P), h, row.data());"),
+    ("threaded_decode_skips_items",
+     "    th.emplace_back([&, w] { for (int64_t it = w; it < items; it += nt) work(it); });",
+     "    th.emplace_back([&, w] { for (int64_t it = w; it < items; it += nt + 1) work(it); });"),
+    ("e4m3_decode_exponent", "  else v = std::ldexp(float(8 + m), E - 10);", "  else v = std::ldexp(float(8 + m), E - 11);"),
+    ("window_keys_and_values_swapped",
+     "    for (int e = 0; e < D; ++e) { kout[e] = bf16_to_f32(kr[e]); vout[e] = bf16_to_f32(vr[e]); }",
+     "    for (int e = 0; e < D; ++e) { kout[e] = bf16_to_f32(vr[e]); vout[e] = bf16_to_f32(kr[e]); }"),
+    ("token_axis_key_scale_index", "      size_t idx = size_t(tok) * L.nkg + size_t(e / c.g_k);",
+     "      size_t idx = size_t(tok) + size_t(e / c.g_k);"),
 ]
 
 
