@@ -93,6 +93,8 @@ def outcomes(tmp_path_factory):
                         "-o", str(lib), "-lcudart"], check=True, capture_output=True)
         r = subprocess.run([sys.executable, "-c", _RUN, str(lib)], cwd=ROOT, capture_output=True, text=True,
                            timeout=600)
+        for built in (obj, lib):   # 8 MB each: not kept once the run is over
+            built.unlink()
         return name, (r.returncode, (r.stdout + r.stderr)[-3000:])
 
     with cf.ThreadPoolExecutor(max_workers=max(1, min(8, os.cpu_count() or 1))) as ex:
