@@ -5,7 +5,9 @@ sharing).  Each case plants one mistake in a copy of csrc/kvq_runtime.cpp,
 compiles it with the library's flags, links it with the library's kernel
 objects, and runs tests/test_abi.py against that build (host-only handles, no
 GPU): at least one test must fail.  The unaltered copy, built the same way,
-must pass them all.  The committed sources are never modified.  (Alignment
+must pass them all.  The committed sources are never modified, and the case
+runs only on a machine without a GPU, so no altered build ever meets one
+(host-only handles launch nothing in any case).  (Alignment
 changes to the chunk sections are not in the list: with pages of at least 16
 tokens every section is already a multiple of 32 bytes, so they change
 nothing.)"""
@@ -68,6 +70,9 @@ def outcomes(tmp_path_factory):
     """Builds the unaltered copy and every mutant of the runtime, links each
     with the library's kernel objects and runs the ABI tests on it (several
     at once); maps name -> (return code, output tail)."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("altered builds of the library run on machines without a GPU only")
     if shutil.which(kbuild.NVCC) is None and not os.path.exists(kbuild.NVCC):
         pytest.skip("nvcc is not available")
     kbuild.build()   # the kernel objects the copies link with
