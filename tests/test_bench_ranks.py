@@ -1,7 +1,7 @@
 """bench.py on CPU: the N>1 path (two gloo ranks, each a replica, combine
 their timings by max and their work by sum, the only collectives), the
-algorithmic byte counts against the format arithmetic, and the oracle arm's
-JSON line."""
+algorithmic byte counts against the format arithmetic, and the keys of both
+arms' JSON lines (the CUDA arm's assembled from a stand-in measurement)."""
 import os
 import socket
 
@@ -115,3 +115,40 @@ def test_reference_arm_runs_the_requested_steps():
     assert d["value"] > 0 and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert d["metric"] == "decode-attn KV GB/s" and d["higher_is_better"] is True
+
+
+def test_bench_line_carries_the_contract_keys(monkeypatch, capsys):
+    """The JSON line of the CUDA arm, assembled from a stand-in measurement
+    (no GPU here): every key of the line's contract is present, `value` is
+    the decode GB/s, the roofline divides the attention rate by the peak,
+    and e2e declares its copies."""
+    import json
+    import sys
+    import bench
+    from quantized_kv_cache_14_b200.workloads import workload
+    w = workload(3)
+    meas = {"w": w, "K": 20, "launches": 60, "clocks": {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []},
+            "kv_gbs": 3000.0, "attn_gbs": 3500.0, "attn_bytes_per_launch": 1.455e8, "attn_us": 41.6,
+            "decode_us": 48.5, "append_us": 9.4, "append_gbs": 22.0, "seq_tok_s": 2.3e9, "ms_per_step": 0.058,
+            "e2e_gbs": 2100.0, "kv_bytes_per_step": 1.455e8, "lens_final": [8192] * 16,
+            "h2d": 196608, "d2h": 262144, "bulk": None}
+    monkeypatch.setattr(bench, "run_gpu", lambda *a, **k: meas)
+    monkeypatch.setattr(bench, "run_oracle_sample", lambda *a, **k: (0.3, 10.0, 3.0e9, [8192] * 16, 16))
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--steps", "20", "--warmup", "5", "--no-workloads",
+                                      "--no-control"])
+    bench.main()
+    d = json.loads([ln for ln in capsys.readouterr().out.splitlines() if ln.startswith("{")][-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "cpu_baseline", "e2e",
+                "gpu_launches", "clocks"):
+        assert key in d, key
+    assert d["value"] == 3000.0 and d["unit"] == "GB/s" and d["n_gpus"] == 1 and d["steps"] == 20
+    assert d["warmup"] == 5 and d["higher_is_better"] is True and d["vs_baseline"] is None
+    assert "workload" in d["config"]
+    r = d["roofline"]
+    assert {"bound", "achieved", "peak", "unit", "frac", "traffic"} <= set(r)
+    assert r["achieved"] == 3500.0 and abs(r["frac"] - 3500.0 / r["peak"]) < 1e-12
+    assert set(d["cpu_baseline"]) >= {"value", "unit", "cores", "kind", "sample"}
+    assert d["e2e"] == {"value": 2100.0, "unit": "GB/s", "h2d_bytes_per_step": 196608,
+                        "d2h_bytes_per_step": 262144}
+    assert d["gpu_launches"] == 60 and set(d["clocks"]) >= {"sm_mhz", "sm_max_mhz", "reasons"}
